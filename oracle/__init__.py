@@ -1,0 +1,282 @@
+"""Reference oracle for Looped Latent Attention (LLA) decode and encode.
+
+TEST INFRASTRUCTURE. Only the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package. The CUDA library never
+calls it, and it never calls the CUDA library.
+
+Source: "Looped Latent Attention: Cross-Loop KV Compression for Looped
+Transformers" (O'Neill & Reid, arXiv 2607.15456).
+
+What is here, each in fp64:
+  * ``attend``: textbook softmax attention (the uncompressed per-loop path).
+  * ``decode_unit`` / ``decode_units`` / ``lla_decode`` / ``lla2d_decode``:
+    explicit reconstruction, k_t = W^K_up,t z^K + mu^K_t and the same for V
+    (§3 Eq. 3), then textbook attention. Per-head LLA reads one latent per
+    (token, head); LLA-2D (§3 "The LLA-2D variant") reads one latent per token
+    shared by every head, with decoders per (head, loop).
+  * ``decode_unit_absorbed``: the §7 bilinear identities, kept only so the
+    tests can compare the two forms by brute force.
+  * ``encode``: the latent write c = (x - mu) W_down (§3 Eq. 2) over a
+    loop-major stack (§3 Eq. 1).
+  * ``svd_init``: §3 "Initialization and conversion": centre by the
+    per-loop mean, take the top-r right singular vectors of the stacked-loop
+    matrix as W_down, and its loop slices as the initial W_up,t.
+  * ``compression_ratio``: §3 Eq. 4.
+
+The decode and encode arithmetic lives in ``lla_oracle.c`` (plain C, no
+BLAS). ``svd_init`` uses numpy's LAPACK SVD as a library step.
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, special cases and invariants the pages fix; none is
+left unpinned.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lla_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liblla_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``lla_oracle.c`` into ``liblla_oracle.so`` (gcc, OpenMP)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_attend.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          _dp, _dp, _dp, ctypes.c_double, _dp, _dp]
+            lib.oracle_attend.restype = ctypes.c_int
+            unit_args = [ctypes.c_int] * 4 + [_dp] * 7 + [ctypes.c_double, _dp, _dp]
+            lib.oracle_decode_unit.argtypes = unit_args
+            lib.oracle_decode_unit.restype = ctypes.c_int
+            lib.oracle_decode_unit_absorbed.argtypes = unit_args
+            lib.oracle_decode_unit_absorbed.restype = ctypes.c_int
+            lib.oracle_decode_units.argtypes = ([ctypes.c_int] * 5 + [_dp] * 7 +
+                                                [ctypes.c_double, _dp, _dp, ctypes.c_int])
+            lib.oracle_decode_units.restype = ctypes.c_int
+            lib.oracle_encode.argtypes = [ctypes.c_int] * 5 + [_dp] * 4
+            lib.oracle_encode.restype = None
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return ctypes.cast(None, _dp)
+    return a.ctypes.data_as(_dp)
+
+
+def max_threads() -> int:
+    """Threads an OpenMP region of the oracle uses by default."""
+    return int(_load().oracle_max_threads())
+
+
+# --------------------------------------------------------------------------
+# attention and decode
+# --------------------------------------------------------------------------
+
+def attend(q, K, V, scale):
+    """Textbook attention of one query over rows of K and V.
+
+    Returns (out [dv], lse) with lse = ln sum_j exp(scale q.K_j)."""
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    N, d = K.shape
+    dv = V.shape[1]
+    out = np.zeros(dv)
+    lse = np.zeros(1)
+    rc = _load().oracle_attend(d, dv, N, _ptr(q), _ptr(K), _ptr(V), float(scale),
+                               _ptr(out), _ptr(lse))
+    if rc:
+        raise ValueError("oracle_attend: empty context or out of memory")
+    return out, float(lse[0])
+
+
+def _unit(fn, q, zk, zv, dk, dv, mu_k, mu_v, scale):
+    q, zk, zv, dk, dv = map(_f64, (q, zk, zv, dk, dv))
+    mu_k = None if mu_k is None else _f64(mu_k)
+    mu_v = None if mu_v is None else _f64(mu_v)
+    N, r_k = zk.shape
+    r_v = zv.shape[1]
+    d = q.shape[0]
+    assert dk.shape == (d, r_k) and dv.shape == (d, r_v) and zv.shape[0] == N
+    out = np.zeros(d)
+    lse = np.zeros(1)
+    rc = fn(d, N, r_k, r_v, _ptr(q), _ptr(zk), _ptr(zv), _ptr(dk), _ptr(dv),
+            _ptr(mu_k), _ptr(mu_v), float(scale), _ptr(out), _ptr(lse))
+    if rc:
+        raise ValueError("oracle decode: empty context or out of memory")
+    return out, float(lse[0])
+
+
+def decode_unit(q, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None):
+    """One (batch row, head, layer, loop) unit, explicit reconstruction.
+
+    q [d]; zk [N, r_k]; zv [N, r_v]; dk = W^K_up,t [d, r_k];
+    dv = W^V_up,t [d, r_v]; mu_k, mu_v = mu_t slices [d] or None."""
+    if scale is None:
+        scale = 1.0 / np.sqrt(np.asarray(q).shape[0])
+    return _unit(_load().oracle_decode_unit, q, zk, zv, dk, dv, mu_k, mu_v, scale)
+
+
+def decode_unit_absorbed(q, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None):
+    """The same unit through the §7 absorbed identities (pins only)."""
+    if scale is None:
+        scale = 1.0 / np.sqrt(np.asarray(q).shape[0])
+    return _unit(_load().oracle_decode_unit_absorbed, q, zk, zv, dk, dv, mu_k,
+                 mu_v, scale)
+
+
+def decode_units(q, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None,
+                 nthreads: int = 0):
+    """Many independent units at once (OpenMP over units).
+
+    q [U, d]; zk [U, N, r_k]; zv [U, N, r_v]; dk [U, d, r_k];
+    dv [U, d, r_v]; mu_k, mu_v [U, d] or None. Returns out [U, d], lse [U]."""
+    q, zk, zv, dk, dv = map(_f64, (q, zk, zv, dk, dv))
+    mu_k = None if mu_k is None else _f64(mu_k)
+    mu_v = None if mu_v is None else _f64(mu_v)
+    U, d = q.shape
+    N, r_k = zk.shape[1], zk.shape[2]
+    r_v = zv.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.zeros((U, d))
+    lse = np.zeros(U)
+    bad = _load().oracle_decode_units(U, d, N, r_k, r_v, _ptr(q), _ptr(zk), _ptr(zv),
+                                      _ptr(dk), _ptr(dv), _ptr(mu_k), _ptr(mu_v),
+                                      float(scale), _ptr(out), _ptr(lse), int(nthreads))
+    if bad:
+        raise ValueError(f"oracle decode: {bad} units failed")
+    return out, lse
+
+
+def lla_decode(q, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None, N=None,
+               units=None, nthreads: int = 0):
+    """Per-head LLA decode for one (layer, loop) step.
+
+    q [B, H, d]; zk [B, H, n_cap, r_k]; zv [B, H, n_cap, r_v] (first N rows
+    used); dk [H, d, r_k]; dv [H, d, r_v]; mu_k, mu_v [H, d] or None.
+    ``units`` restricts the work to a list of (b, h) pairs; the result then
+    holds one row per listed unit. Returns out, lse."""
+    return _decode(q, zk, zv, dk, dv, mu_k, mu_v, scale, N, units, nthreads,
+                   shared_latent=False)
+
+
+def lla2d_decode(q, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None, N=None,
+                 units=None, nthreads: int = 0):
+    """LLA-2D decode for one (layer, loop) step: zk [B, n_cap, r_k] and
+    zv [B, n_cap, r_v] are shared by every head; dk [H, d, r_k] and
+    dv [H, d, r_v] are this loop's per-head decoders."""
+    return _decode(q, zk, zv, dk, dv, mu_k, mu_v, scale, N, units, nthreads,
+                   shared_latent=True)
+
+
+def _decode(q, zk, zv, dk, dv, mu_k, mu_v, scale, N, units, nthreads, shared_latent):
+    q = np.asarray(q)
+    B, H, d = q.shape
+    if N is None:
+        N = zk.shape[-2]
+    if units is None:
+        units = [(b, h) for b in range(B) for h in range(H)]
+    bs = np.array([u[0] for u in units], dtype=np.int64)
+    hs = np.array([u[1] for u in units], dtype=np.int64)
+    if shared_latent:
+        zk_u = np.asarray(zk)[bs, :N]
+        zv_u = np.asarray(zv)[bs, :N]
+    else:
+        zk_u = np.asarray(zk)[bs, hs, :N]
+        zv_u = np.asarray(zv)[bs, hs, :N]
+    out, lse = decode_units(
+        q[bs, hs], zk_u, zv_u, np.asarray(dk)[hs], np.asarray(dv)[hs],
+        None if mu_k is None else np.asarray(mu_k)[hs],
+        None if mu_v is None else np.asarray(mu_v)[hs], scale, nthreads)
+    if len(units) == B * H and list(units) == [(b, h) for b in range(B) for h in range(H)]:
+        return out.reshape(B, H, d), lse.reshape(B, H)
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# encode and codec initialisation
+# --------------------------------------------------------------------------
+
+def encode(x, w, mu=None):
+    """Latent write, Eq. 2: x [T, N, G, d_loop] loop-major; w [G, T*d_loop, r];
+    mu [G, T*d_loop] or None. Returns z [G, N, r]."""
+    x, w = _f64(x), _f64(w)
+    mu = None if mu is None else _f64(mu)
+    T, N, G, d_loop = x.shape
+    r = w.shape[2]
+    assert w.shape == (G, T * d_loop, r)
+    z = np.zeros((G, N, r))
+    _load().oracle_encode(T, N, G, d_loop, r, _ptr(x), _ptr(w), _ptr(mu), _ptr(z))
+    return z
+
+
+def svd_init(X, r, T):
+    """Codec initialisation of §3 "Initialization and conversion".
+
+    X [n_cal, T*d] holds one stacked-loop vector per row (Eq. 1). Returns
+    (w_down [T*d, r], w_up [T, d, r], mu [T*d]): mu is the column mean, which
+    is the per-loop mean of every loop stacked; w_down holds the top-r right
+    singular vectors of the centred matrix; w_up[t] is w_down's loop-t row
+    slice, so Eq. 3 gives xhat_t = c w_up[t]^T + mu_t."""
+    X = _f64(X)
+    n, K = X.shape
+    assert K % T == 0
+    d = K // T
+    mu = X.mean(axis=0)
+    _, _, vt = np.linalg.svd(X - mu, full_matrices=False)
+    w_down = np.ascontiguousarray(vt[:r].T)
+    w_up = np.ascontiguousarray(w_down.reshape(T, d, r))
+    return w_down, w_up, mu
+
+
+def reconstruct(z, w_up, mu=None):
+    """Eq. 3 for every loop: z [..., r], w_up [T, d, r], mu [T*d] or None.
+    Returns xhat [..., T, d]."""
+    z = _f64(z)
+    w_up = _f64(w_up)
+    T, d, r = w_up.shape
+    xhat = np.einsum("tdr,...r->...td", w_up, z)
+    if mu is not None:
+        xhat = xhat + _f64(mu).reshape(T, d)
+    return xhat
+
+
+def compression_ratio(T, d_head, r_k, r_v, H=1, two_d=False):
+    """Eq. 4: per-head rho = 2 T H d_head / ((r_k + r_v) H) = 2 T d_head /
+    (r_k + r_v). LLA-2D stores (r_k + r_v) scalars per token and layer for
+    all H heads, so its ratio is 2 T H d_head / (r_k + r_v)."""
+    if two_d:
+        return 2.0 * T * H * d_head / (r_k + r_v)
+    return (2.0 * T * H * d_head) / ((r_k + r_v) * H)
