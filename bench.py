@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the LLA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl lla|reference]
+
+One step is a full looped decode step of the chosen workload: for every loop
+t and layer d, one absorbed per-head decode call (query absorb, latent
+stream with online softmax, split merge with the V decoder) over every
+cached token of layer d, i.e. L*T calls. Prints one JSON line on rank 0.
+
+Metric: cached tokens attended per second per (layer, loop) step, i.e.
+B * N * L * T / step time. Inputs are resident in HBM when timing starts and
+each layer's latent store is larger than L2, so no flush is needed.
+
+Multi-GPU: every rank decodes its own batch of sequences (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (explicit reconstruction then
+textbook attention) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from decode_attention_encode_b200 import synth  # noqa: E402
+
+METRIC = "LLA decode: cached tokens attended/sec per loop step; HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+DEFAULT_CONFIG = "perhead_4x"
+KERNEL_SRC = os.path.join(ROOT, "decode_attention_encode_b200", "csrc", "decode.cu")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=int(os.environ.get("WORLD_SIZE", "1")))
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.DECODE_CONFIGS))
+    p.add_argument("--impl", default="lla", choices=["lla", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = sorted(r[0] for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2])
+                          if v.lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+
+class DecodeWorkload:
+    """All layers' latent stores, decoders and queries of one config on the
+    device. The 2-D config keeps one latent per token and layer."""
+
+    def __init__(self, cfg: synth.DecodeConfig, device: str, seed_offset: int = 0):
+        self.cfg = cfg
+        c = cfg
+        s = c.seed + seed_offset
+        zk_shape = (c.B, c.N, c.r_k) if c.two_d else (c.B, c.H, c.N, c.r_k)
+        zv_shape = (c.B, c.N, c.r_v) if c.two_d else (c.B, c.H, c.N, c.r_v)
+        self.zk = [synth.latents(zk_shape, s + 1000 * l + 1, device, decay=c.decay,
+                                 dtype=c.torch_dtype) for l in range(c.L)]
+        self.zv = [synth.latents(zv_shape, s + 1000 * l + 2, device, decay=c.decay,
+                                 dtype=c.torch_dtype) for l in range(c.L)]
+        self.dk = synth.orthonormal(c.L * c.T * c.H, c.d_h, c.r_k, s + 3, device).view(
+            c.L, c.T, c.H, c.d_h, c.r_k)
+        self.dv = synth.orthonormal(c.L * c.T * c.H, c.d_h, c.r_v, s + 4, device).view(
+            c.L, c.T, c.H, c.d_h, c.r_v)
+        self.q = synth.queries((c.L, c.T, c.B, c.H, c.d_h), c.d_h, s + 5, device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((c.L, c.T, c.B, c.H), device=device, dtype=torch.float32)
+        import decode_attention_encode_b200 as lla
+        self.lla = lla
+        wsfn = lla.lla2d_decode_attn_workspace if c.two_d else lla.lla_decode_attn_workspace
+        self.ws = torch.empty(max(16, wsfn(c.B, c.H, c.N, c.r_k, c.r_v)), dtype=torch.uint8,
+                              device=device)
+        self.fn = lla.lla2d_decode_attn if c.two_d else lla.lla_decode_attn
+        self.scale = 1.0 / math.sqrt(c.d_h)
+
+    def step(self, q=None, out=None, lse=None):
+        """One looped decode step: loops outer, layers inner (each loop's
+        query depends on the previous loop's output in a real model)."""
+        c = self.cfg
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
+        for t in range(c.T):
+            for l in range(c.L):
+                self.fn(q[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
+                        scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
+
+    def launches_per_step(self) -> int:
+        return 3 * self.cfg.L * self.cfg.T
+
+
+def kernel_hash() -> str:
+    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(config_name: str):
+    """DRAM bytes per launch of the stream kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(PROFILE_DIR, f"k_stream_{config_name}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not h or not t or h.group(1) != kernel_hash():
+        return None
+    return float(t.group(1))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(cfg: synth.DecodeConfig, budget_s: float = 15.0):
+    """Times the oracle, as it stands, on whole (b, h) units of one
+    (layer, loop) step of this workload. Returns (tokens/s, cores, sample)."""
+    import numpy as np
+
+    import oracle
+    c = cfg
+    threads = oracle.max_threads()
+    rng = np.random.default_rng(0)
+    # one unit's inputs on the host (fp64), drawn with the same recipes
+    zk_shape = (1, c.N, c.r_k)
+    done_units = 0
+    t_total = 0.0
+    batch = max(1, threads)
+    while t_total < budget_s and done_units < 4096:
+        seed = int(rng.integers(1 << 30))
+        zk = synth.latents((batch,) + zk_shape[1:], seed, "cpu", decay=c.decay,
+                           dtype=c.torch_dtype).double().numpy()
+        zv = synth.latents((batch, c.N, c.r_v), seed + 1, "cpu", decay=c.decay,
+                           dtype=c.torch_dtype).double().numpy()
+        dk = synth.orthonormal(batch, c.d_h, c.r_k, seed + 2).double().numpy()
+        dv = synth.orthonormal(batch, c.d_h, c.r_v, seed + 3).double().numpy()
+        q = synth.queries((batch, c.d_h), c.d_h, seed + 4).double().numpy()
+        t0 = time.perf_counter()
+        oracle.decode_units(q, zk, zv, dk, dv, scale=1.0 / math.sqrt(c.d_h))
+        t_total += time.perf_counter() - t0
+        done_units += batch
+    # a (layer, loop) step attends B*N cached tokens over H heads: one unit
+    # is N/H of those tokens' worth of work
+    tokens = done_units * c.N / c.H
+    sample = (f"{done_units} (b,h) units of one (layer, loop) step, {c.N} tokens each, "
+              f"explicit K/V reconstruction in fp64; tokens/s counts N/H tokens per unit")
+    return tokens / t_total, threads, sample
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    cfg = synth.DECODE_CONFIGS[args.config]
+    per_step = []
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, budget_s=2.0)
+    cores = 1
+    sample = ""
+    for _ in range(args.steps):
+        v, cores, sample = cpu_baseline(cfg, budget_s=10.0)
+        per_step.append(v)
+    value = sum(per_step) / len(per_step)
+    tokens_per_step = cfg.B * cfg.N * cfg.L * cfg.T
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tokens_per_step / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(cfg), "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def describe(cfg: synth.DecodeConfig) -> str:
+    kind = "LLA-2D" if cfg.two_d else "per-head LLA"
+    return (f"{cfg.name}: {kind} decode, L={cfg.L} T={cfg.T} H={cfg.H} d_h={cfg.d_h} "
+            f"r_k={cfg.r_k} r_v={cfg.r_v} B={cfg.B} N={cfg.N} {cfg.dtype} latents")
+
+
+def run_lla(args, world, rank, local):
+    cfg = synth.DECODE_CONFIGS[args.config]
+    dev = f"cuda:{local}"
+    wl = DecodeWorkload(cfg, dev, seed_offset=rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+
+    # device-timed region
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    call_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(cfg.L)]
+    ev[0].record(stream)
+    for k in range(args.steps):
+        if k == args.steps - 1:
+            # time each call of the last step's first loop on its own
+            c = cfg
+            for t in range(c.T):
+                for l in range(c.L):
+                    if t == 0:
+                        call_ev[l][0].record(stream)
+                    wl.fn(wl.q[l, t], wl.zk[l], wl.zv[l], wl.dk[l, t], wl.dv[l, t], N=c.N,
+                          scale=wl.scale, out=wl.out[l, t], lse=wl.lse[l, t], workspace=wl.ws)
+                    if t == 0:
+                        call_ev[l][1].record(stream)
+        else:
+            wl.step()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_ms = ev[0].elapsed_time(ev[1])
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    ms_per_step = elapsed_ms / args.steps
+    call_ms = sorted(a.elapsed_time(b) for a, b in call_ev)
+    call_ms_mean = sum(call_ms) / len(call_ms)
+
+    tokens_per_step = cfg.B * cfg.N * cfg.L * cfg.T
+    value = world * tokens_per_step / (ms_per_step * 1e-3)
+    step_bytes = cfg.step_bytes()
+    hbm_peak, peak_src = peaks()
+    achieved = step_bytes / (call_ms_mean * 1e-3) / 1e9
+
+    # end to end through the public API: queries from pinned host memory in,
+    # outputs back to pinned host memory, every step
+    e2e = None
+    if not args.no_e2e:
+        q_host = wl.q.to("cpu").pin_memory()
+        out_host = torch.empty(wl.out.shape, dtype=torch.float32).pin_memory()
+        lse_host = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
+        q_dev = torch.empty_like(wl.q)
+        for _ in range(2):
+            q_dev.copy_(q_host, non_blocking=True)
+            wl.step(q=q_dev)
+            out_host.copy_(wl.out, non_blocking=True)
+            lse_host.copy_(wl.lse, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            q_dev.copy_(q_host, non_blocking=True)
+            wl.step(q=q_dev)
+            out_host.copy_(wl.out, non_blocking=True)
+            lse_host.copy_(wl.lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        e2e = {"value": world * tokens_per_step / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": q_host.numel() * 4,
+               "d2h_bytes_per_step": (out_host.numel() + lse_host.numel()) * 4}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": describe(cfg),
+            "step": f"{cfg.L * cfg.T} decode calls (T loops x L layers), 3 kernels each",
+            "accumulation": "fp32",
+            "l2": "no flush: each layer's latent store "
+                  f"({step_bytes / 1e9:.2f} GB) is larger than L2 (126 MB)",
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+            "global_batch": cfg.B * world, "seq_len": cfg.N,
+        },
+        "hbm_gbs_per_call": achieved,
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": profiled_traffic(cfg.name),
+            "kernel": "k_stream (timed as the whole decode call incl. absorb and combine)",
+            "algorithmic_bytes_per_launch": step_bytes,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+            else "fallback 6.65 TB/s",
+        },
+        "call_ms": {"mean": call_ms_mean, "min": call_ms[0], "max": call_ms[-1]},
+        "gpu_launches": wl.launches_per_step() * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_baseline(cfg)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_lla(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+"""ctypes binding of liblla.so (the C ABI declared in include/lla.h).
+
+Argument marshalling only: every step of the decode and encode paths runs in
+the library's CUDA kernels. Torch supplies device memory and the current
+stream. If the library cannot be loaded the calls raise; there is no
+fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+LLA_OK = 0
+LLA_ERR_INVALID_ARG = 1
+LLA_ERR_UNSUPPORTED = 2
+LLA_ERR_WORKSPACE = 3
+LLA_ERR_CUDA = 4
+
+LLA_F32 = 0
+LLA_BF16 = 1
+
+LLA_DEVICE_WAIT_TIMEOUT = 0x1
+
+# Every symbol include/lla.h declares.
+EXPORTS = (
+    "lla_status_string", "lla_last_error", "lla_version", "lla_device_status",
+    "lla_decode_attn_workspace", "lla_decode_attn",
+    "lla2d_decode_attn_workspace", "lla2d_decode_attn",
+    "lla_encode",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class LLAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+_c_int, _c_size, _c_float, _c_ll, _vp = (ctypes.c_int, ctypes.c_size_t, ctypes.c_float,
+                                         ctypes.c_longlong, ctypes.c_void_p)
+
+_SIGS = {
+    "lla_status_string": ([_c_int], ctypes.c_char_p),
+    "lla_last_error": ([], ctypes.c_char_p),
+    "lla_version": ([], _c_int),
+    "lla_device_status": ([ctypes.POINTER(ctypes.c_uint), _c_int], _c_int),
+    "lla_decode_attn_workspace": ([_c_int] * 5, _c_size),
+    "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
+    "lla_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
+                        [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "lla2d_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
+                          [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "lla_encode": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp], _c_int),
+}
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib(build_if_missing: bool = True):
+    """Loads liblla.so (building it with nvcc if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build() if build_if_missing else _build.LIB
+            if not os.path.exists(path):
+                raise LLAError(LLA_ERR_CUDA, f"liblla.so not found at {path}")
+            h = ctypes.CDLL(path)
+            for name, (args, res) in _SIGS.items():
+                fn = getattr(h, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = h
+    return _lib
+
+
+def _check(status: int):
+    if status != LLA_OK:
+        h = lib()
+        raise LLAError(status, f"{h.lla_status_string(status).decode()}: "
+                               f"{h.lla_last_error().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return LLA_BF16
+    if t.dtype == torch.float32:
+        return LLA_F32
+    raise LLAError(LLA_ERR_INVALID_ARG, f"unsupported latent dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise LLAError(LLA_ERR_INVALID_ARG, "tensors must be contiguous CUDA tensors")
+
+
+def device_status(clear: bool = False) -> int:
+    v = ctypes.c_uint(0)
+    _check(lib().lla_device_status(ctypes.byref(v), int(clear)))
+    return v.value
+
+
+def lla_decode_attn_workspace(B, H, N, r_k, r_v) -> int:
+    return int(lib().lla_decode_attn_workspace(B, H, N, r_k, r_v))
+
+
+def lla2d_decode_attn_workspace(B, H, N, r_k, r_v) -> int:
+    return int(lib().lla2d_decode_attn_workspace(B, H, N, r_k, r_v))
+
+
+def _decode(fn_name, ws_name, q, zk, zv, dk_t, dv_t, N, mu_k_t, mu_v_t, scale, out, lse,
+            workspace, stream, want_lse, two_d):
+    _need_cuda(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
+    B, H, d_h = q.shape
+    if two_d:
+        n_cap, r_k = zk.shape[1], zk.shape[2]
+        r_v = zv.shape[2]
+    else:
+        n_cap, r_k = zk.shape[2], zk.shape[3]
+        r_v = zv.shape[3]
+    if N is None:
+        N = n_cap
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_h)
+    if out is None:
+        out = torch.empty((B, H, d_h), device=q.device, dtype=torch.float32)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    h = lib()
+    need = int(getattr(h, ws_name)(B, H, N, r_k, r_v))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    st = getattr(h, fn_name)(_ptr(q), _ptr(zk), _ptr(zv), _dtype_code(zk), B, H, d_h, N, n_cap,
+                             r_k, r_v, _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t),
+                             float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def lla_decode_attn(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, scale=None,
+                    out=None, lse=None, workspace=None, stream=None, want_lse=True):
+    """Per-head absorbed decode for one (layer, loop) step.
+
+    q [B,H,d_h] fp32; zk [B,H,n_cap,r_k], zv [B,H,n_cap,r_v] bf16 or fp32;
+    dk_t [H,d_h,r_k], dv_t [H,d_h,r_v] fp32; mu_k_t, mu_v_t [H,d_h] or None.
+    Returns (out [B,H,d_h], lse [B,H] or None)."""
+    return _decode("lla_decode_attn", "lla_decode_attn_workspace", q, zk, zv, dk_t, dv_t, N,
+                   mu_k_t, mu_v_t, scale, out, lse, workspace, stream, want_lse, two_d=False)
+
+
+def lla2d_decode_attn(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, scale=None,
+                      out=None, lse=None, workspace=None, stream=None, want_lse=True):
+    """LLA-2D absorbed decode for one (layer, loop) step: zk [B,n_cap,r_k],
+    zv [B,n_cap,r_v] bf16, shared by every head."""
+    return _decode("lla2d_decode_attn", "lla2d_decode_attn_workspace", q, zk, zv, dk_t, dv_t,
+                   N, mu_k_t, mu_v_t, scale, out, lse, workspace, stream, want_lse, two_d=True)
+
+
+def lla_encode(x, w_down, mu=None, z=None, z_row_stride=None, z_group_stride=None,
+               stream=None):
+    """Latent write: x [T,N,G,d_loop] bf16, w_down [G,T*d_loop,r] bf16,
+    mu [G,T*d_loop] fp32 or None. Writes z (default a new [G,N,r] bf16
+    tensor; pass z plus strides in elements to write into a larger store).
+    Returns z."""
+    _need_cuda(x, w_down, mu)
+    T, N, G, d_loop = x.shape
+    r = w_down.shape[2]
+    if z is None:
+        z = torch.empty((G, N, r), device=x.device, dtype=torch.bfloat16)
+        z_row_stride, z_group_stride = r, N * r
+    if z_row_stride is None or z_group_stride is None:
+        raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
+    st = lib().lla_encode(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down), _ptr(mu),
+                          _ptr(z), int(z_row_stride), int(z_group_stride), _stream(stream))
+    _check(st)
+    return z

@@ -1,0 +1,183 @@
+// C ABI entry points of liblla: argument checks, status reporting and the
+// per-device state (SM count, sticky status word).
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace lla {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Sticky device status word: kernels OR bits into it when a bounded wait
+// runs out. One instance per device (a module-scope __device__ variable).
+__device__ unsigned int g_status_word = 0u;
+
+thread_local char g_last_error[512] = "";
+
+std::mutex g_dev_mutex;
+bool g_dev_ready[kMaxDevices];
+DeviceInfo g_dev_info[kMaxDevices];
+unsigned int* g_status_ptr[kMaxDevices];
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return dev;
+}
+
+void init_device(int dev) {
+  // caller holds g_dev_mutex
+  if (dev < 0 || dev >= kMaxDevices || g_dev_ready[dev]) return;
+  DeviceInfo info{148, 227 * 1024};
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+    info.sms = v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
+      v > 0)
+    info.smem_optin = v;
+  cudaGetLastError();
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) {
+    cudaGetLastError();
+    p = nullptr;
+  }
+  g_dev_info[dev] = info;
+  g_status_ptr[dev] = static_cast<unsigned int*>(p);
+  g_dev_ready[dev] = true;
+}
+
+}  // namespace
+
+DeviceInfo device_info() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return DeviceInfo{148, 227 * 1024};
+  std::lock_guard<std::mutex> g(g_dev_mutex);
+  init_device(dev);
+  return g_dev_info[dev];
+}
+
+unsigned int* status_word() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> g(g_dev_mutex);
+  init_device(dev);
+  return g_status_ptr[dev];
+}
+
+lla_status fail(lla_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+lla_status check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return LLA_OK;
+  return fail(LLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace lla
+
+using namespace lla;
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+lla_status check_decode_args(const float* q, const void* zk, const void* zv, lla_dtype zdt,
+                             int B, int H, int d_h, int N, int n_cap, int r_k, int r_v,
+                             const float* dk, const float* dv, const float* mu_k,
+                             const float* mu_v, float* out, float* lse, void* ws, int* esz) {
+  if (zdt != LLA_BF16 && zdt != LLA_F32) return fail(LLA_ERR_INVALID_ARG, "zdt must be LLA_BF16 or LLA_F32");
+  *esz = (zdt == LLA_BF16) ? 2 : 4;
+  if (!q || !zk || !zv || !dk || !dv || !out)
+    return fail(LLA_ERR_INVALID_ARG, "q, zk, zv, dk_t, dv_t and out must be non-NULL");
+  if (B < 1 || H < 1) return fail(LLA_ERR_INVALID_ARG, "B and H must be >= 1");
+  if (d_h < 1 || d_h > 256) return fail(LLA_ERR_INVALID_ARG, "d_h must be in 1..256");
+  if (N < 1) return fail(LLA_ERR_INVALID_ARG, "N must be >= 1 (empty context is undefined)");
+  if (N > n_cap) return fail(LLA_ERR_INVALID_ARG, "N must be <= n_cap");
+  const int rmax = (*esz == 2) ? 256 : 128;
+  if (r_k < 8 || r_v < 8 || r_k % 8 || r_v % 8 || r_k > rmax || r_v > rmax)
+    return fail(LLA_ERR_INVALID_ARG, "r_k and r_v must be multiples of 8 in 8..%d", rmax);
+  if (!aligned(zk, 16) || !aligned(zv, 16))
+    return fail(LLA_ERR_INVALID_ARG, "zk and zv must be 16-byte aligned");
+  if (!aligned(q, 4) || !aligned(dk, 4) || !aligned(dv, 4) || !aligned(out, 4) ||
+      (mu_k && !aligned(mu_k, 4)) || (mu_v && !aligned(mu_v, 4)) || (lse && !aligned(lse, 4)))
+    return fail(LLA_ERR_INVALID_ARG, "fp32 arrays must be 4-byte aligned");
+  if (ws && !aligned(ws, 16)) return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  return LLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lla_status_string(lla_status s) {
+  switch (s) {
+    case LLA_OK: return "LLA_OK";
+    case LLA_ERR_INVALID_ARG: return "LLA_ERR_INVALID_ARG";
+    case LLA_ERR_UNSUPPORTED: return "LLA_ERR_UNSUPPORTED";
+    case LLA_ERR_WORKSPACE: return "LLA_ERR_WORKSPACE";
+    case LLA_ERR_CUDA: return "LLA_ERR_CUDA";
+  }
+  return "LLA_ERR_UNKNOWN";
+}
+
+const char* lla_last_error(void) { return g_last_error; }
+
+int lla_version(void) { return 100; }
+
+lla_status lla_device_status(unsigned int* status, int clear) {
+  if (!status) return fail(LLA_ERR_INVALID_ARG, "status must be non-NULL");
+  unsigned int* p = status_word();
+  if (!p) return fail(LLA_ERR_CUDA, "no device status word on the current device");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return check_cuda(e, "cudaDeviceSynchronize");
+  e = cudaMemcpy(status, p, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return check_cuda(e, "read status word");
+  if (clear) {
+    e = cudaMemset(p, 0, sizeof(unsigned int));
+    if (e != cudaSuccess) return check_cuda(e, "clear status word");
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return check_cuda(e, "cudaDeviceSynchronize");
+  }
+  return LLA_OK;
+}
+
+size_t lla_decode_attn_workspace(int B, int H, int N, int r_k, int r_v) {
+  if (B < 1 || H < 1 || N < 1 || r_k < 8 || r_v < 8 || r_k % 8 || r_v % 8) return 0;
+  // The bf16 plan needs at least as much workspace as the fp32 one.
+  DecodePlan p2, p4;
+  size_t need = 0;
+  if (plan_decode(B, H, N, r_k, r_v, 2, &p2) == LLA_OK) need = p2.ws_bytes;
+  if (r_k <= 128 && r_v <= 128 && plan_decode(B, H, N, r_k, r_v, 4, &p4) == LLA_OK)
+    need = need > p4.ws_bytes ? need : p4.ws_bytes;
+  return need;
+}
+
+lla_status lla_decode_attn(const float* q, const void* zk, const void* zv, lla_dtype zdt, int B,
+                           int H, int d_h, int N, int n_cap, int r_k, int r_v, const float* dk_t,
+                           const float* dv_t, const float* mu_k_t, const float* mu_v_t,
+                           float scale, float* out, float* lse, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  g_last_error[0] = '\0';
+  int esz = 0;
+  lla_status st = check_decode_args(q, zk, zv, zdt, B, H, d_h, N, n_cap, r_k, r_v, dk_t, dv_t,
+                                    mu_k_t, mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  return run_decode(q, zk, zv, esz, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t,
+                    mu_k_t, mu_v_t, scale, out, lse, workspace, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

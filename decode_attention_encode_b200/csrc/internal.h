@@ -1,0 +1,57 @@
+// Host-side internals of liblla shared between translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lla.h"
+
+namespace lla {
+
+// SM count and shared-memory limit of a device, queried once per device.
+// Without any visible device these describe a B200 (148 SMs, 227 KB), so
+// workspace queries still work on a host with no GPU.
+struct DeviceInfo {
+  int sms;
+  int smem_optin;
+};
+DeviceInfo device_info();
+
+// Device address of the sticky status word on the current device (one per
+// device, set up once with cudaGetSymbolAddress). NULL on failure.
+unsigned int* status_word();
+
+// Records a one-line reason for the calling thread and returns `s`.
+lla_status fail(lla_status s, const char* fmt, ...);
+
+// Maps a CUDA error to LLA_ERR_CUDA with its message, or LLA_OK.
+lla_status check_cuda(cudaError_t e, const char* what);
+
+// Launch plan of the per-head absorbed decode. See decode.cu.
+struct DecodePlan {
+  int esz;             // bytes per latent element (2 or 4)
+  int nseg_k, nseg_v;  // 16-byte segments per latent row
+  int lpt;             // lanes cooperating on one token
+  int sk, sv;          // segments each lane holds (registers)
+  bool exact;          // every lane's segments are all in range
+  int tile;            // tokens per pipeline stage
+  int nstage;          // pipeline depth per warp
+  int warps;           // warps per CTA of the stream kernel
+  int stage_bytes;     // bytes of one stage (K then V)
+  long long P;         // tokens each warp streams
+  int W;               // warps that stream
+  int grid;            // CTAs of the stream kernel
+  int pstride;         // floats per partial record
+  size_t off_qp, off_c0, off_part, ws_bytes;
+  size_t smem_bytes;   // dynamic shared memory of the stream kernel
+};
+
+lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePlan* plan);
+
+lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, int B, int H,
+                      int d_h, int N, long long n_cap, int r_k, int r_v, const float* dk,
+                      const float* dv, const float* mu_k, const float* mu_v, float scale,
+                      float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+}  // namespace lla

@@ -1,0 +1,177 @@
+/*
+ * lla.h - C ABI of liblla, the B200 (sm_100a) decode hot path of Looped
+ * Latent Attention (LLA).
+ *
+ * Source of the operations: "Looped Latent Attention: Cross-Loop KV
+ * Compression for Looped Transformers" (O'Neill & Reid, arXiv 2607.15456).
+ * A looped, weight-tied decoder runs T loops over D layers. For each
+ * (token, layer, head, axis) LLA keeps one latent c in R^r instead of the T
+ * per-loop vectors (§3 Eq. 2) and rebuilds loop t on read as
+ * xhat_t = W_up,t c + mu_t (§3 Eq. 3, written here in column form). The
+ * decode calls below never rebuild K or V: they use the absorbed form of §7
+ * ("Per-head LLA versus LLA-2D at inference"), moving W^K_up,t onto the
+ * query and applying W^V_up,t once to the latent-space value sum.
+ *
+ * Conventions shared by every call
+ *  - All array arguments are DEVICE pointers owned by the caller. The library
+ *    allocates nothing and keeps no per-call state.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream). The library never synchronises.
+ *  - Arrays are dense, row-major, in the layouts stated per call.
+ *  - A call returns LLA_OK once its kernels are queued; an argument problem
+ *    found on the host returns an error before anything is launched; a launch
+ *    failure returns LLA_ERR_CUDA. lla_last_error() gives a one-line reason
+ *    for the last failure on the calling thread.
+ *  - Device-side waits inside the kernels are bounded in time. A wait that
+ *    runs out sets a sticky device status word instead of hanging; read it
+ *    with lla_device_status() (which synchronises the device).
+ *  - Latent element types: LLA_BF16 or LLA_F32 where stated. Decoders,
+ *    queries, means and outputs are fp32.
+ */
+#ifndef LLA_H
+#define LLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLA_API __attribute__((visibility("default")))
+#else
+#define LLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LLA_OK = 0,
+    LLA_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer */
+    LLA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes */
+    LLA_ERR_WORKSPACE = 3,   /* workspace missing or too small */
+    LLA_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} lla_status;
+
+typedef enum { LLA_F32 = 0, LLA_BF16 = 1 } lla_dtype;
+
+/* Device status bits reported by lla_device_status(). */
+#define LLA_DEVICE_WAIT_TIMEOUT 0x1u /* a bounded device wait ran out */
+
+/* Human-readable name of a status code. Never NULL. */
+LLA_API const char *lla_status_string(lla_status s);
+
+/* One-line reason for the most recent non-OK return on this thread, or "". */
+LLA_API const char *lla_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+LLA_API int lla_version(void);
+
+/*
+ * Reads (and, if `clear` is nonzero, clears) the sticky device status word
+ * of the current device: 0 when no kernel has reported a problem, else a set
+ * of LLA_DEVICE_* bits. Synchronises the device. Returns LLA_ERR_CUDA if the
+ * runtime fails.
+ */
+LLA_API lla_status lla_device_status(unsigned int *status, int clear);
+
+/* --------------------------------------------------------------------------
+ * Per-head absorbed decode, one (layer d, loop t) step.
+ *
+ * Defines (§3 Eq. 3 and the §7 absorption identities), for each batch row b
+ * and head h, over the first N cached tokens j:
+ *   khat_j = dk_t[h] zk[b][h][j] + mu_k_t[h]
+ *   vhat_j = dv_t[h] zv[b][h][j] + mu_v_t[h]
+ *   s_j    = scale * q[b][h] . khat_j
+ *   out[b][h] = sum_j softmax(s)_j vhat_j,    lse[b][h] = ln sum_j exp(s_j)
+ * computed as q' = scale dk_t[h]^T q, s_j = q' . zk_j + scale q . mu_k,
+ * ubar = sum_j p_j zv_j, out = dv_t[h] ubar + mu_v_t[h].
+ *
+ * Arguments
+ *   q        [B][H][d_h] fp32: this loop's query of each sequence and head.
+ *   zk, zv   [B][H][n_cap][r_k] and [B][H][n_cap][r_v], element type zdt
+ *            (LLA_BF16 or LLA_F32): the per-head latent store of layer d.
+ *            Rows [N, n_cap) are never read. 16-byte aligned.
+ *   B, H     batch and heads, >= 1.
+ *   d_h      head width, 1..256.
+ *   N        cached tokens attended, 1 <= N <= n_cap.
+ *   r_k, r_v latent ranks, multiples of 8, at most 256 (bf16) or 128 (fp32).
+ *   dk_t     [H][d_h][r_k] fp32: W^K_up,t of layer d, loop t, per head.
+ *   dv_t     [H][d_h][r_v] fp32: W^V_up,t.
+ *   mu_k_t, mu_v_t  [H][d_h] fp32 loop-t slices of the codec means, or NULL
+ *            for zero.
+ *   scale    softmax scale (usually 1/sqrt(d_h)).
+ *   out      [B][H][d_h] fp32 output.
+ *   lse      [B][H] fp32 natural-log normaliser, or NULL.
+ *   workspace, ws_bytes  device scratch of at least
+ *            lla_decode_attn_workspace(B, H, N, r_k, r_v) bytes, 16-byte
+ *            aligned; its contents need no initialisation and are
+ *            overwritten. Calls that share a workspace must be ordered
+ *            (same stream, or synchronised).
+ * The workspace size depends on the current device's SM count: query it on
+ * the device that will run the call.
+ * -------------------------------------------------------------------------- */
+LLA_API size_t lla_decode_attn_workspace(int B, int H, int N, int r_k, int r_v);
+
+LLA_API lla_status lla_decode_attn(const float *q, const void *zk, const void *zv,
+                           lla_dtype zdt, int B, int H, int d_h, int N,
+                           int n_cap, int r_k, int r_v, const float *dk_t,
+                           const float *dv_t, const float *mu_k_t,
+                           const float *mu_v_t, float scale, float *out,
+                           float *lse, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/* --------------------------------------------------------------------------
+ * LLA-2D absorbed decode, one (layer d, loop t) step (§3 "The LLA-2D
+ * variant": one latent per token and layer, decoded into every head).
+ *
+ * Same definition as lla_decode_attn, except that every head reads the same
+ * latents: zk [B][n_cap][r_k], zv [B][n_cap][r_v] (bf16 only). dk_t
+ * [H][d_h][r_k] and dv_t [H][d_h][r_v] are the per-(head, loop) decoders.
+ * The score and value contractions run on the tensor cores with bf16
+ * operands (the absorbed query and the softmax weights are rounded to bf16)
+ * and fp32 accumulation.
+ * Limits: H <= 32 (H padded to a multiple of 16 inside), r_k and r_v
+ * multiples of 64 up to 256, d_h 1..256, N >= 1.
+ * -------------------------------------------------------------------------- */
+LLA_API size_t lla2d_decode_attn_workspace(int B, int H, int N, int r_k, int r_v);
+
+LLA_API lla_status lla2d_decode_attn(const float *q, const void *zk, const void *zv,
+                             lla_dtype zdt, int B, int H, int d_h, int N,
+                             int n_cap, int r_k, int r_v, const float *dk_t,
+                             const float *dv_t, const float *mu_k_t,
+                             const float *mu_v_t, float scale, float *out,
+                             float *lse, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/* --------------------------------------------------------------------------
+ * Latent write (§3 Eq. 2 over the loop-major stack of Eq. 1):
+ *   z[g][n][c] = bf16_rne( sum_k (xs[k] - mu[g][k]) * w_down[g][k][c] ),
+ *   xs[t*d_loop + i] = x[t][n][g][i].
+ *
+ * Arguments
+ *   x        [T][N][G][d_loop] bf16 (xdt must be LLA_BF16): the per-loop K
+ *            (or V) vectors of N finished tokens, as each loop emits them.
+ *            16-byte aligned.
+ *   T, N, G  loops (1..64), tokens (>= 1), groups (heads for per-head LLA,
+ *            1 for LLA-2D with d_loop = H*d_h).
+ *   d_loop   per-loop width, a multiple of 16; T*d_loop <= 16384.
+ *   r        latent rank, a multiple of 8, at most 256.
+ *   w_down   [G][T*d_loop][r] bf16 encoder. 16-byte aligned.
+ *   mu       [G][T*d_loop] fp32 calibration mean, or NULL for zero.
+ *   z        bf16 output; row n of group g starts at element
+ *            g*z_group_stride + n*z_row_stride. Strides are in elements,
+ *            multiples of 8, and rows must not overlap. This lets one call
+ *            write each sequence's newest token straight into its slot of a
+ *            [B][H][n_cap][r] store.
+ * The multiply runs on the tensor cores (bf16 operands, fp32 accumulation).
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla_encode(const void *x, lla_dtype xdt, int T, int N, int G,
+                      int d_loop, int r, const void *w_down, const float *mu,
+                      void *z, long long z_row_stride,
+                      long long z_group_stride, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLA_H */

@@ -1,0 +1,98 @@
+"""Shared builders for the GPU parity tests: seeded inputs on the device, the
+same values copied to the host for the oracle, and the tolerance checks."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from decode_attention_encode_b200 import synth
+
+# Tolerances (max over each checked output tensor):
+#   fp32 latents: max |o_gpu - o_ref| <= 1e-4
+#   bf16 latents: max |o_gpu - o_ref| / max |o_ref| <= 2e-2
+TOL_F32_ABS = 1e-4
+TOL_BF16_REL = 2e-2
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    """Exact widening of device values for the oracle."""
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def make_decode_inputs(B, H, d_h, N, r_k, r_v, dtype, *, n_cap=None, two_d=False, decay=False,
+                       mu=False, seed=0, q_scale=1.0, device="cuda"):
+    """Seeded inputs of one (layer, loop) decode step on `device`."""
+    n_cap = N if n_cap is None else n_cap
+    zshape_k = (B, n_cap, r_k) if two_d else (B, H, n_cap, r_k)
+    zshape_v = (B, n_cap, r_v) if two_d else (B, H, n_cap, r_v)
+    zk = synth.latents(zshape_k, seed + 1, device, decay=decay, dtype=dtype)
+    zv = synth.latents(zshape_v, seed + 2, device, decay=decay, dtype=dtype)
+    dk = synth.orthonormal(H, d_h, r_k, seed + 3, device)
+    dv = synth.orthonormal(H, d_h, r_v, seed + 4, device)
+    q = synth.queries((B, H, d_h), d_h, seed + 5, device)
+    if q_scale != 1.0:
+        q = q * q_scale
+    mu_k = synth.normal((H, d_h), seed + 6, device) if mu else None
+    mu_v = synth.normal((H, d_h), seed + 7, device) if mu else None
+    return dict(q=q, zk=zk, zv=zv, dk=dk, dv=dv, mu_k=mu_k, mu_v=mu_v, N=N)
+
+
+def sample_units(B, H, n_random=32, seed=0):
+    """32 seeded-random (b, h) units plus up to 16 corner units."""
+    corners_b = sorted({0, min(1, B - 1), B // 2, B - 1})
+    corners_h = sorted({0, min(1, H - 1), H // 2, H - 1})
+    units = [(b, h) for b in corners_b for h in corners_h]
+    r = np.random.default_rng(seed)
+    for _ in range(n_random):
+        units.append((int(r.integers(B)), int(r.integers(H))))
+    seen, out = set(), []
+    for u in units:
+        if u not in seen:
+            seen.add(u)
+            out.append(u)
+    return out
+
+
+def oracle_reference(inp, units, two_d=False, scale=None):
+    """Runs the oracle on the given units, reading only those units' data
+    back from the device."""
+    import oracle  # test infrastructure only
+
+    q = inp["q"]
+    d_h = q.shape[-1]
+    N = inp["N"]
+    scale = 1.0 / math.sqrt(d_h) if scale is None else scale
+    bs = torch.tensor([u[0] for u in units], device=q.device)
+    hs = torch.tensor([u[1] for u in units], device=q.device)
+    if two_d:
+        zk = to_f64(inp["zk"][bs, :N])
+        zv = to_f64(inp["zv"][bs, :N])
+    else:
+        zk = to_f64(inp["zk"][bs, hs, :N])
+        zv = to_f64(inp["zv"][bs, hs, :N])
+    out, lse = oracle.decode_units(
+        to_f64(q[bs, hs]), zk, zv, to_f64(inp["dk"][hs]), to_f64(inp["dv"][hs]),
+        None if inp["mu_k"] is None else to_f64(inp["mu_k"][hs]),
+        None if inp["mu_v"] is None else to_f64(inp["mu_v"][hs]), scale)
+    return out, lse
+
+
+def compare(out_gpu, lse_gpu, units, ref_out, ref_lse, dtype):
+    """Returns (err, lse_err) and asserts the stated tolerance."""
+    bs = [u[0] for u in units]
+    hs = [u[1] for u in units]
+    o = to_f64(out_gpu)[bs, hs]
+    diff = np.abs(o - ref_out).max()
+    if dtype == torch.float32:
+        err = diff
+        assert err <= TOL_F32_ABS, f"fp32 max-abs error {err:.3e} > {TOL_F32_ABS}"
+    else:
+        err = diff / np.abs(ref_out).max()
+        assert err <= TOL_BF16_REL, f"bf16 relative error {err:.3e} > {TOL_BF16_REL}"
+    lse_err = None
+    if lse_gpu is not None:
+        lse_err = np.abs(to_f64(lse_gpu)[bs, hs] - ref_lse).max()
+    return err, lse_err
