@@ -179,21 +179,21 @@ def lla2d_decode_attn(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, s
                    N, mu_k_t, mu_v_t, scale, out, lse, workspace, stream, want_lse, two_d=True)
 
 
-def lla_encode(x, w_down, mu=None, z=None, z_row_stride=None, z_group_stride=None,
+def lla_encode(x, w_down_t, mu=None, z=None, z_row_stride=None, z_group_stride=None,
                stream=None):
-    """Latent write: x [T,N,G,d_loop] bf16, w_down [G,T*d_loop,r] bf16,
+    """Latent write: x [T,N,G,d_loop] bf16, w_down_t [G,r,T*d_loop] bf16 (W_down transposed),
     mu [G,T*d_loop] fp32 or None. Writes z (default a new [G,N,r] bf16
     tensor; pass z plus strides in elements to write into a larger store).
     Returns z."""
-    _need_cuda(x, w_down, mu)
+    _need_cuda(x, w_down_t, mu)
     T, N, G, d_loop = x.shape
-    r = w_down.shape[2]
+    r = w_down_t.shape[1]
     if z is None:
         z = torch.empty((G, N, r), device=x.device, dtype=torch.bfloat16)
         z_row_stride, z_group_stride = r, N * r
     if z_row_stride is None or z_group_stride is None:
         raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
-    st = lib().lla_encode(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down), _ptr(mu),
+    st = lib().lla_encode(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t), _ptr(mu),
                           _ptr(z), int(z_row_stride), int(z_group_stride), _stream(stream))
     _check(st)
     return z

@@ -180,4 +180,30 @@ lla_status lla_decode_attn(const float* q, const void* zk, const void* zv, lla_d
                     static_cast<cudaStream_t>(stream));
 }
 
+lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,
+                      const void* w_down_t, const float* mu, void* z, long long z_row_stride,
+                      long long z_group_stride, void* stream) {
+  g_last_error[0] = '\0';
+  if (xdt != LLA_BF16) return fail(LLA_ERR_INVALID_ARG, "xdt must be LLA_BF16");
+  if (!x || !w_down_t || !z) return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be non-NULL");
+  if (!aligned(x, 16) || !aligned(w_down_t, 16) || !aligned(z, 16))
+    return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be 16-byte aligned");
+  if (mu && !aligned(mu, 4)) return fail(LLA_ERR_INVALID_ARG, "mu must be 4-byte aligned");
+  if (T < 1 || N < 1 || G < 1) return fail(LLA_ERR_INVALID_ARG, "T, N and G must be >= 1");
+  if (d_loop < 64 || d_loop % 64)
+    return fail(LLA_ERR_INVALID_ARG, "d_loop must be a positive multiple of 64");
+  if ((long long)T * d_loop > (1LL << 30)) return fail(LLA_ERR_INVALID_ARG, "T*d_loop too large");
+  if (r < 8 || r > 256 || r % 8) return fail(LLA_ERR_INVALID_ARG, "r must be a multiple of 8 in 8..256");
+  if (z_row_stride < r || z_group_stride < 0 || z_row_stride % 8 || z_group_stride % 8)
+    return fail(LLA_ERR_INVALID_ARG, "z strides must be multiples of 8 with z_row_stride >= r");
+  if (G > 1) {
+    const bool groups_outer = z_group_stride >= (long long)(N - 1) * z_row_stride + r;
+    const bool rows_outer = z_row_stride >= (long long)(G - 1) * z_group_stride + r && z_group_stride >= r;
+    if (!groups_outer && !rows_outer)
+      return fail(LLA_ERR_INVALID_ARG, "z strides make output rows overlap");
+  }
+  return run_encode(x, T, N, G, d_loop, r, w_down_t, mu, z, z_row_stride, z_group_stride,
+                    static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -1,0 +1,357 @@
+// Latent write (LLA encoder) on the sm_100a tensor cores.
+//
+// Source: "Looped Latent Attention: Cross-Loop KV Compression for Looped
+// Transformers" (arXiv 2607.15456), §3 "Teacher cache" Eq. 1 (loop-major
+// stacking of the T per-loop vectors) and §3 "Cross-loop codec" Eq. 2
+// (c = (x - mu) W_down).
+//
+// Per group g this is the GEMM Z_g[N x r] = X_g[N x T*d_loop] W_g - mu_g W_g.
+// X_g is never stacked in memory: the loop-major input x[T][N][G][d_loop] is
+// read through a 4-D TMA tensor map, and the contraction index k = t*d_loop+i
+// is walked as (t, 64-wide chunk) pairs, so each K chunk is one 128-token x
+// 64-channel box of one loop.
+//
+// Kernel layout (persistent, one CTA per SM, warp-specialised):
+//   warp 0      TMA producer: A box (128 tokens x 64 k, 128B swizzle) and
+//               the matching B box (r rows of W^T x 64 k) per pipeline stage.
+//   warp 1      allocates TMEM, issues tcgen05.mma (M=128, N=r padded to 16,
+//               K=16 per instruction) into one of two TMEM accumulators, and
+//               commits stage releases and accumulator hand-offs.
+//   warps 2-5   epilogue: tcgen05.ld of the 128 x r accumulator (one TMEM
+//               lane per token), subtract mu W, round to bf16 (RNE), store
+//               with the caller's row and group strides. Double-buffered
+//               accumulators let the epilogue of tile i overlap the MMAs of
+//               tile i+1.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "tc.cuh"
+
+namespace lla {
+namespace {
+
+constexpr int kTileM = 128;     // tokens per tile (TMEM lanes)
+constexpr int kChunkK = 64;     // K elements per stage (128 B rows)
+constexpr int kABytes = kTileM * kChunkK * 2;
+constexpr int kThreads = 192;   // 6 warps
+
+struct EncodeArgs {
+  int N, G, d_loop, r, r_pad, K, nk, mtiles, tiles, tiles_per_cta;
+  int nstage, b_bytes, stage_bytes;
+  uint32_t tmem_cols;
+  const float* mu;
+  const __nv_bfloat16* wt;
+  __nv_bfloat16* z;
+  long long zrs, zgs;
+  unsigned int* status;
+};
+
+struct SmemTail {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float muw[256];
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      report_status(status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_encode(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
+             EncodeArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the 128B-swizzle atoms
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemTail* tail = reinterpret_cast<SmemTail*>(smem + (size_t)a.nstage * a.stage_bytes);
+  volatile int* abort_flag = &tail->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_begin = blockIdx.x * a.tiles_per_cta;
+  const int t_end = min(t_begin + a.tiles_per_cta, a.tiles);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.nstage; ++s) {
+      mbar_init(smem_u32(&tail->full[s]), 1);
+      mbar_init(smem_u32(&tail->empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tail->tfull[i]), 1);
+      mbar_init(smem_u32(&tail->tempty[i]), 4);
+    }
+    mbar_init(smem_u32(&tail->drain), 1);
+    tail->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&tail->tmem_base), a.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tail->tmem_base;
+  const int cpl = a.d_loop / kChunkK;  // chunks per loop
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const uint64_t pol_x = l2_evict_first_policy();
+      const uint64_t pol_w = l2_evict_last_policy();
+      int it = 0;
+      bool ok = true;
+      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        const int g = tile / a.mtiles;
+        const int m0 = (tile - g * a.mtiles) * kTileM;
+        for (int kc = 0; kc < a.nk; ++kc, ++it) {
+          const int s = it % a.nstage;
+          const uint32_t ph = (uint32_t)(it / a.nstage) & 1u;
+          if (!wait_or_abort(smem_u32(&tail->empty[s]), ph ^ 1u, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = smem_u32(&tail->full[s]);
+          mbar_arrive_expect_tx(full, kABytes + a.b_bytes);
+          const uint32_t sa = smem_u32(smem + (size_t)s * a.stage_bytes);
+          const int t = kc / cpl, i0 = (kc - t * cpl) * kChunkK;
+          tma_load_4d(sa, &tx, i0, g, m0, t, full, pol_x);
+          tma_load_3d(sa + kABytes, &tw, kc * kChunkK, 0, g, full, pol_w);
+        }
+      }
+      if (!ok) {
+        // let copies already issued land before the CTA can exit
+        const int first = max(0, it - a.nstage);
+        for (int i = first; i < it; ++i)
+          (void)mbar_wait(smem_u32(&tail->full[i % a.nstage]), (uint32_t)(i / a.nstage) & 1u,
+                          kWaitTimeoutNs / 8);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileM, a.r_pad, false, false);
+      int it = 0;
+      bool ok = true;
+      for (int tile = t_begin, lt = 0; tile < t_end && ok; ++tile, ++lt) {
+        const int acc = lt & 1;
+        const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
+        if (!wait_or_abort(smem_u32(&tail->tempty[acc]), aph ^ 1u, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tbase + (uint32_t)(acc * a.r_pad);
+        for (int kc = 0; kc < a.nk; ++kc, ++it) {
+          const int s = it % a.nstage;
+          const uint32_t ph = (uint32_t)(it / a.nstage) & 1u;
+          if (!wait_or_abort(smem_u32(&tail->full[s]), ph, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * a.stage_bytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kChunkK / 16; ++kk)
+            umma_bf16(d, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idesc,
+                      (kc | kk) != 0);
+          umma_commit(smem_u32(&tail->empty[s]));
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&tail->tfull[acc]));
+      }
+      // all issued MMAs complete before TMEM can be released
+      umma_commit(smem_u32(&tail->drain));
+      (void)mbar_wait(smem_u32(&tail->drain), 0u, kWaitTimeoutNs / 8);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int ew = warp - 2;
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    int cur_g = -1;
+    for (int tile = t_begin, lt = 0; tile < t_end; ++tile, ++lt) {
+      const int g = tile / a.mtiles;
+      const int m0 = (tile - g * a.mtiles) * kTileM;
+      if (g != cur_g) {
+        named_bar(1, 128);  // previous tile's readers of muw are done
+        for (int c = ew; c < a.r; c += 4) {
+          float acc = 0.f;
+          if (a.mu) {
+            const float* mu = a.mu + (size_t)g * a.K;
+            const __nv_bfloat16* w = a.wt + ((size_t)g * a.r + c) * a.K;
+            for (int k = lane; k < a.K; k += 32) acc = fmaf(mu[k], __bfloat162float(w[k]), acc);
+            acc = warp_sum(acc);
+          }
+          if (lane == 0) tail->muw[c] = acc;
+        }
+        named_bar(1, 128);
+        cur_g = g;
+      }
+      const int acc = lt & 1;
+      const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
+      const bool ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&tail->tfull[acc]), aph,
+                                                            abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * a.r_pad);
+      const int n = m0 + row;
+      __nv_bfloat16* zrow = a.z + (size_t)g * a.zgs + (size_t)n * a.zrs;
+      for (int cc = 0; cc < a.r_pad; cc += 16) {
+        float v[16];
+        tmem_ld16(taddr + cc, v);
+        if (n < a.N) {
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const int c0 = cc + 8 * h8;
+            if (c0 < a.r) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(
+                    v[8 * h8 + 2 * e] - tail->muw[c0 + 2 * e],
+                    v[8 * h8 + 2 * e + 1] - tail->muw[c0 + 2 * e + 1]);
+                w[e] = *reinterpret_cast<const uint32_t*>(&p);
+              }
+              *reinterpret_cast<uint4*>(zrow + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tail->tempty[acc]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, a.tmem_cols);
+  }
+}
+
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeTiledFn get_encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) {
+    fail(LLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t gd[5];
+  cuuint64_t gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(LLA_ERR_INVALID_ARG, "tensor map rejected by the driver (CUresult %d)", (int)r);
+    return false;
+  }
+  return true;
+}
+
+lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
+                      const float* mu, void* z, long long zrs, long long zgs,
+                      cudaStream_t stream) {
+  const int K = T * d_loop;
+  const int r_pad = (r + 15) / 16 * 16;
+  EncodeArgs a{};
+  a.N = N;
+  a.G = G;
+  a.d_loop = d_loop;
+  a.r = r;
+  a.r_pad = r_pad;
+  a.K = K;
+  a.nk = K / kChunkK;
+  a.mtiles = (N + kTileM - 1) / kTileM;
+  a.tiles = a.mtiles * G;
+  a.b_bytes = r_pad * kChunkK * 2;
+  a.stage_bytes = kABytes + a.b_bytes;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * r_pad)) cols <<= 1;
+  a.tmem_cols = cols;
+  a.mu = mu;
+  a.wt = static_cast<const __nv_bfloat16*>(wt);
+  a.z = static_cast<__nv_bfloat16*>(z);
+  a.zrs = zrs;
+  a.zgs = zgs;
+  a.status = status_word();
+
+  const DeviceInfo di = device_info();
+  const size_t fixed = sizeof(SmemTail) + 1024;
+  int nst = (int)std::min<size_t>(8, ((size_t)di.smem_optin - fixed) / a.stage_bytes);
+  if (nst < 2) return fail(LLA_ERR_UNSUPPORTED, "encode stage does not fit in shared memory");
+  a.nstage = nst;
+  const size_t smem = (size_t)nst * a.stage_bytes + fixed;
+  const int grid0 = std::min(a.tiles, di.sms);
+  a.tiles_per_cta = (a.tiles + grid0 - 1) / grid0;
+  const int grid = (a.tiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+
+  CUtensorMap tx, tw;
+  {
+    const uint64_t dims[4] = {(uint64_t)d_loop, (uint64_t)G, (uint64_t)N, (uint64_t)T};
+    const uint64_t strides[3] = {(uint64_t)d_loop * 2, (uint64_t)G * d_loop * 2,
+                                 (uint64_t)N * G * d_loop * 2};
+    const uint32_t box[4] = {(uint32_t)kChunkK, 1, (uint32_t)kTileM, 1};
+    if (!make_tmap_bf16(&tx, x, 4, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)K, (uint64_t)r, (uint64_t)G};
+    const uint64_t strides[2] = {(uint64_t)K * 2, (uint64_t)r * K * 2};
+    const uint32_t box[3] = {(uint32_t)kChunkK, (uint32_t)r_pad, 1};
+    if (!make_tmap_bf16(&tw, wt, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  cudaError_t e = cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_encode)");
+  k_encode<<<grid, kThreads, smem, stream>>>(tx, tw, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return check_cuda(e, "launch k_encode");
+  return LLA_OK;
+}
+
+}  // namespace lla

@@ -54,4 +54,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
                       const float* dv, const float* mu_k, const float* mu_v, float scale,
                       float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
+                      const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream);
+
 }  // namespace lla

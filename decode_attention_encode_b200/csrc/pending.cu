@@ -14,9 +14,4 @@ lla_status lla2d_decode_attn(const float*, const void*, const void*, lla_dtype, 
   return fail(LLA_ERR_UNSUPPORTED, "lla2d_decode_attn is not built yet");
 }
 
-lla_status lla_encode(const void*, lla_dtype, int, int, int, int, int, const void*, const float*,
-                      void*, long long, long long, void*) {
-  return fail(LLA_ERR_UNSUPPORTED, "lla_encode is not built yet");
-}
-
 }  // extern "C"

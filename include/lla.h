@@ -145,30 +145,34 @@ LLA_API lla_status lla2d_decode_attn(const float *q, const void *zk, const void 
 
 /* --------------------------------------------------------------------------
  * Latent write (§3 Eq. 2 over the loop-major stack of Eq. 1):
- *   z[g][n][c] = bf16_rne( sum_k (xs[k] - mu[g][k]) * w_down[g][k][c] ),
+ *   z[g][n][c] = bf16_rne( sum_k (xs[k] - mu[g][k]) * W_down[g][k][c] ),
  *   xs[t*d_loop + i] = x[t][n][g][i].
  *
  * Arguments
  *   x        [T][N][G][d_loop] bf16 (xdt must be LLA_BF16): the per-loop K
  *            (or V) vectors of N finished tokens, as each loop emits them.
  *            16-byte aligned.
- *   T, N, G  loops (1..64), tokens (>= 1), groups (heads for per-head LLA,
+ *   T, N, G  loops (>= 1), tokens (>= 1), groups (heads for per-head LLA,
  *            1 for LLA-2D with d_loop = H*d_h).
- *   d_loop   per-loop width, a multiple of 16; T*d_loop <= 16384.
+ *   d_loop   per-loop width, a multiple of 64.
  *   r        latent rank, a multiple of 8, at most 256.
- *   w_down   [G][T*d_loop][r] bf16 encoder. 16-byte aligned.
+ *   w_down_t [G][r][T*d_loop] bf16: the encoder W_down of each group stored
+ *            transposed (row c holds column c of W_down), so both operands of
+ *            the tensor-core multiply are contiguous along the stacked index.
+ *            16-byte aligned.
  *   mu       [G][T*d_loop] fp32 calibration mean, or NULL for zero.
  *   z        bf16 output; row n of group g starts at element
  *            g*z_group_stride + n*z_row_stride. Strides are in elements,
  *            multiples of 8, and rows must not overlap. This lets one call
  *            write each sequence's newest token straight into its slot of a
- *            [B][H][n_cap][r] store.
- * The multiply runs on the tensor cores (bf16 operands, fp32 accumulation).
+ *            [B][H][n_cap][r] store. 16-byte aligned.
+ * The multiply runs on the tensor cores (bf16 operands, fp32 accumulation);
+ * the mean term mu W_down is formed in fp32 and subtracted before rounding.
  * -------------------------------------------------------------------------- */
 LLA_API lla_status lla_encode(const void *x, lla_dtype xdt, int T, int N, int G,
-                      int d_loop, int r, const void *w_down, const float *mu,
-                      void *z, long long z_row_stride,
-                      long long z_group_stride, void *stream);
+                              int d_loop, int r, const void *w_down_t,
+                              const float *mu, void *z, long long z_row_stride,
+                              long long z_group_stride, void *stream);
 
 #ifdef __cplusplus
 }
