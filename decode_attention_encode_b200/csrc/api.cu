@@ -109,9 +109,9 @@ lla_status check_decode_args(const float* q, const void* zk, const void* zv, lla
   const int rmax = (*esz == 2) ? 256 : 128;
   if (r_k < 8 || r_v < 8 || r_k % 8 || r_v % 8 || r_k > rmax || r_v > rmax)
     return fail(LLA_ERR_INVALID_ARG, "r_k and r_v must be multiples of 8 in 8..%d", rmax);
-  if (!aligned(zk, 16) || !aligned(zv, 16))
-    return fail(LLA_ERR_INVALID_ARG, "zk and zv must be 16-byte aligned");
-  if (!aligned(q, 4) || !aligned(dk, 4) || !aligned(dv, 4) || !aligned(out, 4) ||
+  if (!aligned(zk, 16) || !aligned(zv, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+    return fail(LLA_ERR_INVALID_ARG, "zk, zv, dk_t and dv_t must be 16-byte aligned");
+  if (!aligned(q, 4) || !aligned(out, 4) ||
       (mu_k && !aligned(mu_k, 4)) || (mu_v && !aligned(mu_v, 4)) || (lse && !aligned(lse, 4)))
     return fail(LLA_ERR_INVALID_ARG, "fp32 arrays must be 4-byte aligned");
   if (ws && !aligned(ws, 16)) return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
@@ -178,6 +178,32 @@ lla_status lla_decode_attn(const float* q, const void* zk, const void* zv, lla_d
   return run_decode(q, zk, zv, esz, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t,
                     mu_k_t, mu_v_t, scale, out, lse, workspace, ws_bytes,
                     static_cast<cudaStream_t>(stream));
+}
+
+size_t lla2d_decode_attn_workspace(int B, int H, int N, int r_k, int r_v) {
+  if (B < 1 || H < 1 || H > 32 || N < 1 || r_k < 64 || r_k > 256 || r_k % 64 || r_v < 128 ||
+      r_v > 256 || r_v % 128)
+    return 0;
+  return workspace_2d(B, H, N, r_k, r_v);
+}
+
+lla_status lla2d_decode_attn(const float* q, const void* zk, const void* zv, lla_dtype zdt, int B,
+                             int H, int d_h, int N, int n_cap, int r_k, int r_v,
+                             const float* dk_t, const float* dv_t, const float* mu_k_t,
+                             const float* mu_v_t, float scale, float* out, float* lse,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  int esz = 0;
+  lla_status st = check_decode_args(q, zk, zv, zdt, B, H, d_h, N, n_cap, r_k, r_v, dk_t, dv_t,
+                                    mu_k_t, mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
+  if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
+  if (r_k % 64 || r_v % 128)
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D needs r_k a multiple of 64 and r_v a multiple of 128");
+  return run_decode_2d(q, zk, zv, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t, mu_k_t,
+                       mu_v_t, scale, out, lse, workspace, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,

@@ -39,8 +39,9 @@ constexpr float kNegBig = -1.0e30f;
 // it by this much (log2 units), so p_j <= 2^8 and rescales are rare.
 constexpr float kRescaleSlack = 8.0f;
 
-constexpr int kAbsorbRows = 16;   // batch rows per k_absorb CTA
-constexpr int kCombineRows = 16;  // batch rows per k_combine CTA
+constexpr int kAbsorbRows = 8;    // batch rows per k_absorb CTA
+constexpr int kCombineRows = 8;   // batch rows (one per warp) per k_combine CTA
+constexpr int kSmemChunk = 8192;  // floats of a decoder chunk staged in shared memory
 
 // ---------------------------------------------------------------------------
 // k_absorb
@@ -56,8 +57,12 @@ struct AbsorbArgs {
   float* c0;  // [B*H], natural-log units
 };
 
+// One CTA per (head, block of kAbsorbRows batch rows). W^K_up,t of the head
+// is staged through shared memory in row chunks (coalesced float4 loads, all
+// issued before use); each thread owns fixed (b, c) outputs.
 __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
-  extern __shared__ float q_s[];  // [kAbsorbRows][d_h]
+  __shared__ float q_s[kAbsorbRows * 256];
+  __shared__ __align__(16) float d_s[kSmemChunk];
   pdl_launch_dependents();
   const int h = blockIdx.x;
   const int b0 = blockIdx.y * kAbsorbRows;
@@ -78,28 +83,48 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
     if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
   }
 
-  // q'[b][c] = qscale * sum_i D[i][c] q[b][i]; thread -> (column c, row group)
-  const int groups = max(1, (int)blockDim.x / a.r_k);
-  const int g = threadIdx.x / a.r_k;
-  const int c = threadIdx.x - g * a.r_k;
-  if (g >= groups) return;
-  float acc[kAbsorbRows];
+  // outputs (bb, c), bb < nb, c < r_k; at most kAbsorbRows*256/256 = 8 per thread
+  constexpr int kMaxOut = kAbsorbRows;
+  float acc[kMaxOut];
+  int ob[kMaxOut], oc[kMaxOut];
+  const int nout = nb * a.r_k;
 #pragma unroll
-  for (int k = 0; k < kAbsorbRows; ++k) acc[k] = 0.f;
-  const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c;
-  for (int i = 0; i < a.d_h; ++i) {
-    const float dval = __ldg(D + (size_t)i * a.r_k);
+  for (int k = 0; k < kMaxOut; ++k) {
+    const int o = threadIdx.x + k * blockDim.x;
+    acc[k] = 0.f;
+    ob[k] = o < nout ? o / a.r_k : 0;
+    oc[k] = o < nout ? o - ob[k] * a.r_k : 0;
+  }
+  const float* D = a.dk + (size_t)h * a.d_h * a.r_k;
+  const int rows_per_chunk = max(1, kSmemChunk / a.r_k);
+  for (int i0 = 0; i0 < a.d_h; i0 += rows_per_chunk) {
+    const int ni = min(rows_per_chunk, a.d_h - i0);
+    const int n4 = ni * a.r_k / 4;  // r_k is a multiple of 8
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < n4; idx += blockDim.x)
+      reinterpret_cast<float4*>(d_s)[idx] =
+          __ldg(reinterpret_cast<const float4*>(D + (size_t)i0 * a.r_k) + idx);
+    __syncthreads();
 #pragma unroll
-    for (int k = 0; k < kAbsorbRows; ++k) {
-      const int bb = g + k * groups;
-      if (bb < nb) acc[k] = fmaf(dval, q_s[bb * a.d_h + i], acc[k]);
+    for (int k = 0; k < kMaxOut; ++k) {
+      if (threadIdx.x + k * blockDim.x < nout) {
+        const float* qrow = q_s + ob[k] * a.d_h + i0;
+        const float* dcol = d_s + oc[k];
+        float s0 = 0.f, s1 = 0.f;
+        int i = 0;
+        for (; i + 1 < ni; i += 2) {
+          s0 = fmaf(dcol[i * a.r_k], qrow[i], s0);
+          s1 = fmaf(dcol[(i + 1) * a.r_k], qrow[i + 1], s1);
+        }
+        if (i < ni) s0 = fmaf(dcol[i * a.r_k], qrow[i], s0);
+        acc[k] += s0 + s1;
+      }
     }
   }
 #pragma unroll
-  for (int k = 0; k < kAbsorbRows; ++k) {
-    const int bb = g + k * groups;
-    if (bb < nb) a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c] = acc[k] * a.qscale;
-  }
+  for (int k = 0; k < kMaxOut; ++k)
+    if (threadIdx.x + k * blockDim.x < nout)
+      a.qp[((size_t)(b0 + ob[k]) * a.H + h) * a.r_k + oc[k]] = acc[k] * a.qscale;
 }
 
 // ---------------------------------------------------------------------------
@@ -136,6 +161,59 @@ __device__ __forceinline__ void unpack16<4>(const uint4& v, float* f) {
   f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
 }
 
+// Loads q' of unit u (this lane's segments) into registers.
+template <int E, int LPT, int SK, bool EXACT>
+__device__ __forceinline__ void load_qp(float (&qv)[SK][E], const float* qp, long long u, int r_k,
+                                        int nseg_k, int g) {
+#pragma unroll
+  for (int s = 0; s < SK; ++s) {
+    const int seg = s * LPT + g;
+    if (EXACT || seg < nseg_k) {
+      const float4* src = reinterpret_cast<const float4*>(qp + u * r_k + seg * E);
+#pragma unroll
+      for (int e4 = 0; e4 < E / 4; ++e4) {
+        const float4 t = src[e4];
+        qv[s][4 * e4 + 0] = t.x;
+        qv[s][4 * e4 + 1] = t.y;
+        qv[s][4 * e4 + 2] = t.z;
+        qv[s][4 * e4 + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[s][e] = 0.f;
+    }
+  }
+}
+
+// One token slot's online-softmax update with score sc (log2 units) and
+// value row v.
+template <int ESZ, int LPT, int SV, bool EXACT>
+__device__ __forceinline__ void slot_update(float sc, const unsigned char* vrow, float& m, float& l,
+                                            float (&acc)[SV][16 / ESZ], int nseg_v, int g) {
+  constexpr int E = 16 / ESZ;
+  if (sc > m + kRescaleSlack) {
+    const float alpha = exp2f(m - sc);
+    l *= alpha;
+#pragma unroll
+    for (int s = 0; s < SV; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[s][e] *= alpha;
+    m = sc;
+  }
+  const float p = exp2f(sc - m);
+  l += p;
+#pragma unroll
+  for (int s = 0; s < SV; ++s) {
+    const int seg = s * LPT + g;
+    if (EXACT || seg < nseg_v) {
+      float x[E];
+      unpack16<ESZ>(*reinterpret_cast<const uint4*>(vrow + seg * 16), x);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[s][e] = fmaf(p, x[e], acc[s][e]);
+    }
+  }
+}
+
 // ESZ: bytes per latent element. LPT: lanes per token. SK/SV: 16-byte
 // segments per lane for K/V. EXACT: nseg == LPT*S for both axes.
 template <int ESZ, int LPT, int SK, int SV, bool EXACT>
@@ -169,53 +247,46 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
   const uint64_t pol = l2_evict_first_policy();
 
   // Producer side (lane 0 issues): the tile sequence is the range [f0, f1)
-  // cut at unit boundaries and at `tile` tokens.
-  long long pf = f0;
-  int issued = 0;
+  // cut at unit boundaries and at `tile` tokens; (pu, pj) is the unit and
+  // token of the next tile to load, ps its stage.
+  long long pf = f0, pu = f0 / a.N, pj = f0 - pu * a.N;
+  int ps = 0, in_flight = 0;
   auto issue = [&]() {
-    const long long u = pf / a.N;
-    const long long j = pf - u * a.N;
-    const int len = (int)min((long long)a.tile, min(f1 - pf, a.N - j));
-    const int s = issued % a.nstage;
+    const int len = (int)min((long long)a.tile, min(f1 - pf, a.N - pj));
     if (lane == 0) {
       const uint32_t kb = (uint32_t)len * a.row_k, vb = (uint32_t)len * a.row_v;
-      const uint32_t bar = bar0 + 8 * s;
-      const long long row = u * a.n_cap + j;
+      const uint32_t bar = bar0 + 8 * ps;
+      const long long row = pu * a.n_cap + pj;
+      const uint32_t dst = buf0 + ps * a.stage_bytes;
       mbar_arrive_expect_tx(bar, kb + vb);
-      bulk_g2s(buf0 + s * a.stage_bytes, a.zk + row * a.row_k, kb, bar, pol);
-      bulk_g2s(buf0 + s * a.stage_bytes + v_off, a.zv + row * a.row_v, vb, bar, pol);
+      bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
+      bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
     }
     pf += len;
-    ++issued;
+    pj += len;
+    if (pj == a.N) {
+      pj = 0;
+      ++pu;
+    }
+    if (++ps == a.nstage) ps = 0;
+    ++in_flight;
   };
   for (int s = 0; s < a.nstage && pf < f1; ++s) issue();
 
   // q' is written by k_absorb.
   pdl_wait();
 
-  int consumed = 0;
+  int cs = 0;          // stage being consumed
+  uint32_t cpar = 0;   // its phase parity
   long long f = f0;
+  long long u = f0 / a.N;
+  const long long u_last = (f1 - 1) / a.N;
+  float qv[SK][E], qn[SK][E];
+  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g);
   while (f < f1) {
-    const long long u = f / a.N;
     const long long seg_end = min(f1, (u + 1) * a.N);
-
-    float qv[SK][E];
-#pragma unroll
-    for (int s = 0; s < SK; ++s) {
-      const int seg = s * LPT + g;
-      if (EXACT || seg < a.nseg_k) {
-        const float4* src = reinterpret_cast<const float4*>(a.qp + u * a.r_k + seg * E);
-#pragma unroll
-        for (int e4 = 0; e4 < E / 4; ++e4) {
-          const float4 t = src[e4];
-          qv[s][4 * e4 + 0] = t.x; qv[s][4 * e4 + 1] = t.y;
-          qv[s][4 * e4 + 2] = t.z; qv[s][4 * e4 + 3] = t.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) qv[s][e] = 0.f;
-      }
-    }
+    // the next unit's q' loads run under this unit's stream
+    if (u < u_last) load_qp<E, LPT, SK, EXACT>(qn, a.qp, u + 1, a.r_k, a.nseg_k, g);
     float m = kNegBig, l = 0.f;
     float acc[SV][E];
 #pragma unroll
@@ -225,23 +296,26 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
 
     while (f < seg_end) {
       const int len = (int)min((long long)a.tile, seg_end - f);
-      const int st = consumed % a.nstage;
-      const uint32_t par = (uint32_t)(consumed / a.nstage) & 1u;
-      const bool ok = __all_sync(FULL, mbar_wait(bar0 + 8 * st, par));
+      const bool ok = __all_sync(FULL, mbar_wait(bar0 + 8 * cs, cpar));
       if (!ok) {
         if (lane == 0) report_status(a.status, kStatusWaitTimeout);
-        for (int i = consumed; i < issued; ++i)
-          (void)mbar_wait(bar0 + 8 * (i % a.nstage), (uint32_t)(i / a.nstage) & 1u,
-                          kWaitTimeoutNs / 8);
+        int st = cs;
+        uint32_t par = cpar;
+        for (int i = 0; i < in_flight; ++i) {
+          (void)mbar_wait(bar0 + 8 * st, par, kWaitTimeoutNs / 8);
+          if (++st == a.nstage) {
+            st = 0;
+            par ^= 1u;
+          }
+        }
         return;
       }
-      const unsigned char* Ks = buf + st * a.stage_bytes;
+      const unsigned char* Ks = buf + cs * a.stage_bytes;
       const unsigned char* Vs = Ks + v_off;
 
       for (int t0 = 0; t0 < len; t0 += 2 * NS) {
         const int ta = t0 + slot, tb = t0 + NS + slot;
         const bool va = ta < len, vb = tb < len;
-        // scores of two token slots per lane
         float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
 #pragma unroll
         for (int s = 0; s < SK; ++s) {
@@ -272,56 +346,16 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
           sa += __shfl_xor_sync(FULL, sa, o);
           sb += __shfl_xor_sync(FULL, sb, o);
         }
-        if (va) {
-          if (sa > m + kRescaleSlack) {
-            const float alpha = exp2f(m - sa);
-            l *= alpha;
-#pragma unroll
-            for (int s = 0; s < SV; ++s)
-#pragma unroll
-              for (int e = 0; e < E; ++e) acc[s][e] *= alpha;
-            m = sa;
-          }
-          const float p = exp2f(sa - m);
-          l += p;
-#pragma unroll
-          for (int s = 0; s < SV; ++s) {
-            const int seg = s * LPT + g;
-            if (EXACT || seg < a.nseg_v) {
-              float x[E];
-              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Vs + ta * a.row_v + seg * 16), x);
-#pragma unroll
-              for (int e = 0; e < E; ++e) acc[s][e] = fmaf(p, x[e], acc[s][e]);
-            }
-          }
-        }
-        if (vb) {
-          if (sb > m + kRescaleSlack) {
-            const float alpha = exp2f(m - sb);
-            l *= alpha;
-#pragma unroll
-            for (int s = 0; s < SV; ++s)
-#pragma unroll
-              for (int e = 0; e < E; ++e) acc[s][e] *= alpha;
-            m = sb;
-          }
-          const float p = exp2f(sb - m);
-          l += p;
-#pragma unroll
-          for (int s = 0; s < SV; ++s) {
-            const int seg = s * LPT + g;
-            if (EXACT || seg < a.nseg_v) {
-              float x[E];
-              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Vs + tb * a.row_v + seg * 16), x);
-#pragma unroll
-              for (int e = 0; e < E; ++e) acc[s][e] = fmaf(p, x[e], acc[s][e]);
-            }
-          }
-        }
+        if (va) slot_update<ESZ, LPT, SV, EXACT>(sa, Vs + ta * a.row_v, m, l, acc, a.nseg_v, g);
+        if (vb) slot_update<ESZ, LPT, SV, EXACT>(sb, Vs + tb * a.row_v, m, l, acc, a.nseg_v, g);
       }
       __syncwarp();
-      ++consumed;
+      --in_flight;
       if (pf < f1) issue();  // refill the stage just read
+      if (++cs == a.nstage) {
+        cs = 0;
+        cpar ^= 1u;
+      }
       f += len;
     }
 
@@ -360,6 +394,11 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
         }
       }
     }
+    ++u;
+#pragma unroll
+    for (int s = 0; s < SK; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[s][e] = qn[s][e];
   }
 }
 
@@ -373,14 +412,19 @@ struct CombineArgs {
   const float* dv;
   const float* mu_v;
   int B, H, d_h, r_v;
-  long long N, P;
+  long long N, P;  // per-sequence and per-piece extents of the split
+  int shared;      // 1: one split per sequence shared by all heads (LLA-2D)
   float* out;
   float* lse;
 };
 
+// One CTA per (head, block of kCombineRows batch rows): warp w merges the
+// partial records of row w (lanes across the latent index), then W^V_up,t is
+// staged in shared memory in padded row chunks and applied to all rows.
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
-  extern __shared__ float ub[];  // [kCombineRows][r_v]
-  pdl_wait();                    // partials come from k_stream
+  __shared__ float ub[kCombineRows * 256];
+  __shared__ float d_s[kSmemChunk + 256];
+  pdl_wait();  // partials come from the streaming kernel
   const int h = blockIdx.x;
   const int b0 = blockIdx.y * kCombineRows;
   const int nb = min(kCombineRows, a.B - b0);
@@ -388,48 +432,60 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 
   for (int bb = warp; bb < nb; bb += nwarps) {
     const long long u = (long long)(b0 + bb) * a.H + h;
-    const long long wf = (u * a.N) / a.P;
-    const long long wl = ((u + 1) * a.N - 1) / a.P;
+    // The split runs over units (b, h) for per-head LLA and over sequences
+    // b for LLA-2D; piece w of split key k is partial record w + k.
+    const long long key = a.shared ? (long long)(b0 + bb) : u;
+    const long long wf = (key * a.N) / a.P;
+    const long long wl = ((key + 1) * a.N - 1) / a.P;
+    auto rec = [&](long long w) {
+      return a.shared ? a.part + ((w + key) * a.H + h) * a.pstride : a.part + (w + key) * a.pstride;
+    };
+    const int np = (int)(wl - wf + 1);
     float M = kNegBig;
-    for (long long w = wf; w <= wl; ++w) M = fmaxf(M, a.part[(w + u) * a.pstride]);
+    for (int k = lane; k < np; k += 32) M = fmaxf(M, rec(wf + k)[0]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (long long w = wf; w <= wl; ++w) {
-      const float* pp = a.part + (w + u) * a.pstride;
+    for (int k = lane; k < np; k += 32) {
+      const float* pp = rec(wf + k);
       L += pp[1] * exp2f(pp[0] - M);
     }
+    L = warp_sum(L);
     const float inv = 1.f / L;
     for (int c = lane; c < a.r_v; c += 32) {
       float acc = 0.f;
-      for (long long w = wf; w <= wl; ++w) {
-        const float* pp = a.part + (w + u) * a.pstride;
+      for (int k = 0; k < np; ++k) {
+        const float* pp = rec(wf + k);
         acc = fmaf(exp2f(pp[0] - M), pp[4 + c], acc);
       }
       ub[bb * a.r_v + c] = acc * inv;
     }
     if (lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
   }
-  __syncthreads();
 
-  // out[b][h][i] = sum_c W^V[i][c] ubar_b[c] + mu^V[i]: one warp per row i,
-  // lanes across c (coalesced reads of W^V from L2).
-  for (int i = warp; i < a.d_h; i += nwarps) {
-    const float* drow = a.dv + ((size_t)h * a.d_h + i) * a.r_v;
-    float acc[kCombineRows];
-#pragma unroll
-    for (int k = 0; k < kCombineRows; ++k) acc[k] = 0.f;
-    for (int c = lane; c < a.r_v; c += 32) {
-      const float dval = __ldg(drow + c);
-#pragma unroll
-      for (int k = 0; k < kCombineRows; ++k)
-        if (k < nb) acc[k] = fmaf(dval, ub[k * a.r_v + c], acc[k]);
+  // out[b][h][i] = sum_c W^V[i][c] ubar_b[c] + mu^V[i]
+  const float* D = a.dv + (size_t)h * a.d_h * a.r_v;
+  const int pitch = a.r_v + 1;  // padded rows: threads with consecutive i hit distinct banks
+  const int rows_per_chunk = max(1, kSmemChunk / pitch);
+  for (int i0 = 0; i0 < a.d_h; i0 += rows_per_chunk) {
+    const int ni = min(rows_per_chunk, a.d_h - i0);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < ni * a.r_v; idx += blockDim.x) {
+      const int i = idx / a.r_v, c = idx - i * a.r_v;
+      d_s[i * pitch + c] = __ldg(D + (size_t)(i0 + i) * a.r_v + c);
     }
-    const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i] : 0.f;
-#pragma unroll
-    for (int k = 0; k < kCombineRows; ++k) {
-      if (k < nb) {
-        const float v = warp_sum(acc[k]);
-        if (lane == 0) a.out[((size_t)(b0 + k) * a.H + h) * a.d_h + i] = v + mu;
+    __syncthreads();
+    for (int o = threadIdx.x; o < nb * ni; o += blockDim.x) {
+      const int bb = o / ni, i = o - bb * ni;
+      const float* drow = d_s + i * pitch;
+      const float* urow = ub + bb * a.r_v;
+      float s0 = 0.f, s1 = 0.f;
+      for (int c = 0; c < a.r_v; c += 2) {
+        s0 = fmaf(drow[c], urow[c], s0);
+        s1 = fmaf(drow[c + 1], urow[c + 1], s1);
       }
+      const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + i] : 0.f;
+      a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + i] = s0 + s1 + mu;
     }
   }
 }
@@ -473,6 +529,31 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
+                         int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream) {
+  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0};
+  dim3 grid(H, (B + kAbsorbRows - 1) / kAbsorbRows);
+  k_absorb<<<grid, 256, 0, stream>>>(a);
+  return check_cuda(cudaGetLastError(), "launch k_absorb");
+}
+
+lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
+                          const float* mu_v, int B, int H, int d_h, int r_v, long long N,
+                          long long P, int shared, float* out, float* lse, cudaStream_t stream) {
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse};
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(H, (B + kCombineRows - 1) / kCombineRows);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return check_cuda(cudaLaunchKernelEx(&cfg, k_combine, a), "launch k_combine");
+}
+
 lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePlan* p) {
   DecodePlan d{};
   d.esz = esz;
@@ -507,8 +588,8 @@ lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePla
   const int tok_bytes = (r_k + r_v) * esz;
   const DeviceInfo di = device_info();
   d.warps = std::max(1, std::min(8, env_int("LLA_DECODE_WARPS", 8)));
-  d.nstage = std::max(2, std::min(8, env_int("LLA_DECODE_STAGES", 4)));
-  const int target = std::max(1024, env_int("LLA_DECODE_STAGE_BYTES", 6144));
+  d.nstage = std::max(2, std::min(8, env_int("LLA_DECODE_STAGES", 2)));
+  const int target = std::max(1024, env_int("LLA_DECODE_STAGE_BYTES", 12288));
   const int pair = 2 * ns;
   d.tile = std::max(pair, (target / tok_bytes) / pair * pair);
   // fit the CTA's shared memory
@@ -563,14 +644,8 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_stream)");
 
   // 1. absorb
-  {
-    AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0};
-    dim3 grid(H, (B + kAbsorbRows - 1) / kAbsorbRows);
-    const size_t sm = (size_t)kAbsorbRows * d_h * sizeof(float);
-    k_absorb<<<grid, 256, sm, stream>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return check_cuda(e, "launch k_absorb");
-  }
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
+  if (st != LLA_OK) return st;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
@@ -607,18 +682,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
     if (e != cudaSuccess) return check_cuda(e, "launch k_stream");
   }
   // 3. combine
-  {
-    CombineArgs a{part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, (long long)N, d.P, out, lse};
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(H, (B + kCombineRows - 1) / kCombineRows);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = (size_t)kCombineRows * r_v * sizeof(float);
-    cfg.stream = stream;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k_combine, a);
-    if (e != cudaSuccess) return check_cuda(e, "launch k_combine");
-  }
+  return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, N, d.P, 0, out, lse, stream);
   return LLA_OK;
 }
 

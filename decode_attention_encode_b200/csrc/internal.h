@@ -54,6 +54,19 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
                       const float* dv, const float* mu_k, const float* mu_v, float scale,
                       float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+// Kernels shared by the per-head and LLA-2D decode paths (decode.cu).
+lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
+                         int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream);
+lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
+                          const float* mu_v, int B, int H, int d_h, int r_v, long long N,
+                          long long P, int shared, float* out, float* lse, cudaStream_t stream);
+
+size_t workspace_2d(int B, int H, int N, int r_k, int r_v);
+lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,
+                         int N, long long n_cap, int r_k, int r_v, const float* dk,
+                         const float* dv, const float* mu_k, const float* mu_v, float scale,
+                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream);
 

@@ -1,0 +1,624 @@
+// LLA-2D absorbed decode on the sm_100a tensor cores.
+//
+// Source: "Looped Latent Attention: Cross-Loop KV Compression for Looped
+// Transformers" (arXiv 2607.15456), §3 "The LLA-2D variant" (one latent per
+// token and layer, decoded into every head) and §7 "Per-head LLA versus
+// LLA-2D at inference" (absorbed attention reads latents directly).
+//
+// Every head of a sequence reads the same latents, so the H absorbed queries
+// against the shared latent store form real contractions:
+//   S  [128 tokens x H] = Z^K_tile [128 x r_k] . Q'^T [r_k x H]
+//   U  [r_v x H]       += Z^V_tile^T [r_v x 128] . P [128 x H]
+// Both run as tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in
+// TMEM). The softmax over tokens sits between them on CUDA cores: one thread
+// per token row reads its H scores from TMEM, keeps a per-head reference
+// maximum that is raised only when a score passes it by 2^8 (a CTA vote, then
+// a tile max and an in-TMEM rescale of U), and writes bf16 weights P into
+// shared memory in the layout the second MMA reads.
+//
+// Work split: the (sequence, 128-token tile) space is cut into equal runs of
+// whole tiles, one run per CTA of a one-wave grid. Each (CTA, sequence) piece
+// ends in one partial record per head (m, l, U); k_combine merges them and
+// applies W^V_up,t. k_absorb (shared with the per-head path) forms q'.
+//
+// CTA roles (6 warps):
+//   warp 0     TMA producer: 128 x 128-column latent groups (two 64-column
+//              128B-swizzled boxes, 32 KB) into a ring of stages; stages Q'
+//              (bf16, swizzled K-major) for each new sequence.
+//   warp 1     TMEM owner and MMA issuer. Issues the score MMA of tile i+1
+//              before the value MMA of tile i so the softmax of tile i
+//              overlaps the next score MMA.
+//   warps 2-5  softmax and epilogue (one thread per TMEM lane).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "internal.h"
+#include "tc.cuh"
+
+namespace lla {
+namespace {
+
+constexpr int kRows = 128;
+constexpr int kBoxBytes = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16
+constexpr int kStageBytes = 2 * kBoxBytes;
+constexpr int kThreads = 192;
+constexpr int kMaxStages = 8;
+constexpr float kNegBig = -1.0e30f;
+constexpr float kSlack = 8.0f;
+
+struct D2Args {
+  int B, H, N, tps, tiles, tpc;
+  int r_k, r_v, nkg, nvg, spt, nstage;
+  int off_q, off_p, off_tail, qbuf_bytes, pbuf_bytes;
+  uint32_t tmem_cols;
+  const float* qp;
+  float* part;
+  int pstride;
+  unsigned int* status;
+};
+
+struct Tail2 {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t s_full[2], s_empty[2], p_full[2], u_done[2], q_full[2], q_empty[2];
+  uint64_t epi;    // 4-warp rendezvous of the softmax warps
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int vote[2][4];
+  float red[2][4][32];
+  float lsum[4][32];
+};
+
+__device__ __forceinline__ bool wait_ab(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                        unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      report_status(status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// byte offset of element (row, col) in a K-major 128B-swizzled operand made
+// of 64-column chunks of `rows_per_chunk` rows
+__device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows_per_chunk) {
+  return (uint32_t)((col >> 6) * rows_per_chunk * 128 + row * 128) +
+         ((uint32_t)((col & 63) * 2) ^ (uint32_t)((row & 7) << 4));
+}
+
+template <int HP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_lla2d(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+            D2Args a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Tail2* tl = reinterpret_cast<Tail2*>(smem + a.off_tail);
+  volatile int* abort_flag = &tl->abort_flag;
+  const uint32_t s_stage0 = smem_u32(smem);
+  const uint32_t s_q0 = smem_u32(smem + a.off_q);
+  const uint32_t s_p0 = smem_u32(smem + a.off_p);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_begin = blockIdx.x * a.tpc;
+  const int t_end = min(t_begin + a.tpc, a.tiles);
+  const int ntile = t_end - t_begin;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.nstage; ++s) {
+      mbar_init(smem_u32(&tl->full[s]), 1);
+      mbar_init(smem_u32(&tl->empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tl->s_full[i]), 1);
+      mbar_init(smem_u32(&tl->s_empty[i]), 4);
+      mbar_init(smem_u32(&tl->p_full[i]), 4);
+      mbar_init(smem_u32(&tl->u_done[i]), 1);
+      mbar_init(smem_u32(&tl->q_full[i]), 1);
+      mbar_init(smem_u32(&tl->q_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&tl->epi), 4);
+    mbar_init(smem_u32(&tl->drain), 1);
+    tl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&tl->tmem_base), a.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tl->tmem_base;
+
+  auto seq_of = [&](int lt) { return (t_begin + lt) / a.tps; };
+  auto kboxes = [&](int kg) { return min(2, (a.r_k - kg * 128) / 64); };
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    const uint64_t pol = l2_evict_first_policy();
+    const int total = ntile * a.spt;
+    auto issue = [&](int it) -> bool {
+      const int s = it % a.nstage;
+      const uint32_t ph = (uint32_t)(it / a.nstage) & 1u;
+      const bool ok = __all_sync(0xffffffffu,
+                                 wait_ab(smem_u32(&tl->empty[s]), ph ^ 1u, abort_flag, a.status));
+      if (!ok) return false;
+      if (lane == 0) {
+        const int lt = it / a.spt, sub = it - lt * a.spt;
+        const int tile = t_begin + lt;
+        const int b = tile / a.tps, row0 = (tile - b * a.tps) * kRows;
+        const uint32_t full = smem_u32(&tl->full[s]);
+        const uint32_t dst = s_stage0 + (uint32_t)s * kStageBytes;
+        if (sub < a.nkg) {
+          const int nb = kboxes(sub);
+          mbar_arrive_expect_tx(full, nb * kBoxBytes);
+          for (int x = 0; x < nb; ++x)
+            tma_load_3d(dst + x * kBoxBytes, &tk, sub * 128 + x * 64, row0, b, full, pol);
+        } else {
+          const int vg = sub - a.nkg;
+          mbar_arrive_expect_tx(full, 2 * kBoxBytes);
+          for (int x = 0; x < 2; ++x)
+            tma_load_3d(dst + x * kBoxBytes, &tv, vg * 128 + x * 64, row0, b, full, pol);
+        }
+      }
+      return true;
+    };
+    auto stage_q = [&](int seg, int b) -> bool {
+      const int qb = seg & 1;
+      const bool ok = __all_sync(
+          0xffffffffu,
+          wait_ab(smem_u32(&tl->q_empty[qb]), (uint32_t)((seg >> 1) & 1) ^ 1u, abort_flag, a.status));
+      if (!ok) return false;
+      unsigned char* qs = smem + a.off_q + qb * a.qbuf_bytes;
+      for (int idx = lane; idx < HP * a.r_k; idx += 32) {
+        const int h = idx / a.r_k, c = idx - h * a.r_k;
+        const float v = h < a.H ? a.qp[((size_t)b * a.H + h) * a.r_k + c] : 0.f;
+        *reinterpret_cast<__nv_bfloat16*>(qs + sw128_off(h, c, HP)) = __float2bfloat16_rn(v);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tl->q_full[qb]));
+      return true;
+    };
+
+    bool ok = true;
+    int it = 0;
+    if (ntile > 0) {
+      const int b0 = seq_of(0);
+      // latent loads of the first sequence do not depend on k_absorb
+      while (ok && it < total && it < a.nstage && seq_of(it / a.spt) == b0) ok = issue(it++);
+      pdl_wait();
+      if (ok) ok = stage_q(0, b0);
+      int seg = 0, cur_b = b0;
+      for (; ok && it < total; ++it) {
+        const int lt = it / a.spt;
+        if (it - lt * a.spt == 0 && seq_of(lt) != cur_b) {
+          cur_b = seq_of(lt);
+          ok = stage_q(++seg, cur_b);
+          if (!ok) break;
+        }
+        ok = issue(it);
+      }
+    } else {
+      pdl_wait();
+    }
+    if (!ok && lane == 0) {
+      const int first = max(0, it - a.nstage);
+      for (int i = first; i < it; ++i)
+        (void)mbar_wait(smem_u32(&tl->full[i % a.nstage]), (uint32_t)(i / a.nstage) & 1u,
+                        kWaitTimeoutNs / 8);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0 && ntile > 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kRows, HP, false, false);
+      const uint32_t idesc_u = idesc_bf16_f32(kRows, HP, true, false);
+      bool ok = true;
+      auto mma_scores = [&](int lt, int seg) -> bool {
+        const int sb = lt & 1;
+        if (!wait_ab(smem_u32(&tl->s_empty[sb]), (uint32_t)((lt >> 1) & 1) ^ 1u, abort_flag,
+                     a.status))
+          return false;
+        tc_fence_after();
+        const uint32_t d = tbase + (uint32_t)(sb * HP);
+        const uint32_t qaddr = s_q0 + (uint32_t)((seg & 1) * a.qbuf_bytes);
+        for (int kg = 0; kg < a.nkg; ++kg) {
+          const int it = lt * a.spt + kg;
+          const int s = it % a.nstage;
+          if (!wait_ab(smem_u32(&tl->full[s]), (uint32_t)(it / a.nstage) & 1u, abort_flag,
+                       a.status))
+            return false;
+          tc_fence_after();
+          const int nb = kboxes(kg);
+          for (int x = 0; x < nb; ++x) {
+            const uint32_t abox = s_stage0 + (uint32_t)s * kStageBytes + x * kBoxBytes;
+            const uint32_t bchunk = qaddr + (uint32_t)((kg * 2 + x) * HP * 128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(d, desc_kmajor_sw128(abox + kk * 32), desc_kmajor_sw128(bchunk + kk * 32),
+                        idesc_s, (kg | x | kk) != 0);
+          }
+          umma_commit(smem_u32(&tl->empty[s]));
+        }
+        umma_commit(smem_u32(&tl->s_full[sb]));
+        return true;
+      };
+
+      int seg = 0;
+      ok = wait_ab(smem_u32(&tl->q_full[0]), 0u, abort_flag, a.status) && mma_scores(0, 0);
+      for (int lt = 0; ok && lt < ntile; ++lt) {
+        const bool first_of_seg = (lt == 0) || seq_of(lt) != seq_of(lt - 1);
+        if (lt + 1 < ntile) {
+          int seg_next = seg;
+          if (seq_of(lt + 1) != seq_of(lt)) {
+            umma_commit(smem_u32(&tl->q_empty[seg & 1]));  // after the last score MMA of seg
+            seg_next = seg + 1;
+            ok = wait_ab(smem_u32(&tl->q_full[seg_next & 1]), (uint32_t)((seg_next >> 1) & 1),
+                         abort_flag, a.status);
+            if (!ok) break;
+          }
+          ok = mma_scores(lt + 1, seg_next);
+          if (!ok) break;
+          // value MMA of tile lt belongs to `seg`; advance after it
+          const int pb = lt & 1;
+          ok = wait_ab(smem_u32(&tl->p_full[pb]), (uint32_t)((lt >> 1) & 1), abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          for (int vg = 0; vg < a.nvg && ok; ++vg) {
+            const int it = lt * a.spt + a.nkg + vg;
+            const int s = it % a.nstage;
+            ok = wait_ab(smem_u32(&tl->full[s]), (uint32_t)(it / a.nstage) & 1u, abort_flag,
+                         a.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d = tbase + (uint32_t)(2 * HP + vg * HP);
+            const uint32_t abase = s_stage0 + (uint32_t)s * kStageBytes;
+            const uint32_t pbase = s_p0 + (uint32_t)(pb * a.pbuf_bytes);
+#pragma unroll
+            for (int ks = 0; ks < kRows / 16; ++ks)
+              umma_bf16(d, desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
+                        desc_kmajor_sw128(pbase + (ks >> 2) * HP * 128 + (ks & 3) * 32), idesc_u,
+                        !(first_of_seg && ks == 0));
+            umma_commit(smem_u32(&tl->empty[s]));
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(&tl->u_done[pb]));
+          seg = seg_next;
+        } else {
+          const int pb = lt & 1;
+          ok = wait_ab(smem_u32(&tl->p_full[pb]), (uint32_t)((lt >> 1) & 1), abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          for (int vg = 0; vg < a.nvg && ok; ++vg) {
+            const int it = lt * a.spt + a.nkg + vg;
+            const int s = it % a.nstage;
+            ok = wait_ab(smem_u32(&tl->full[s]), (uint32_t)(it / a.nstage) & 1u, abort_flag,
+                         a.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d = tbase + (uint32_t)(2 * HP + vg * HP);
+            const uint32_t abase = s_stage0 + (uint32_t)s * kStageBytes;
+            const uint32_t pbase = s_p0 + (uint32_t)(pb * a.pbuf_bytes);
+#pragma unroll
+            for (int ks = 0; ks < kRows / 16; ++ks)
+              umma_bf16(d, desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
+                        desc_kmajor_sw128(pbase + (ks >> 2) * HP * 128 + (ks & 3) * 32), idesc_u,
+                        !(first_of_seg && ks == 0));
+            umma_commit(smem_u32(&tl->empty[s]));
+          }
+          if (!ok) break;
+          umma_commit(smem_u32(&tl->u_done[pb]));
+        }
+      }
+      umma_commit(smem_u32(&tl->drain));
+      (void)mbar_wait(smem_u32(&tl->drain), 0u, kWaitTimeoutNs / 8);
+    }
+  } else {
+    // --------------------------- softmax / epilogue ---------------------------
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tbase + ((uint32_t)(quarter * 32) << 16);
+    uint32_t epi_phase = 0;
+    auto epi_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tl->epi));
+      const bool ok = __all_sync(
+          0xffffffffu, wait_ab(smem_u32(&tl->epi), epi_phase & 1u, abort_flag, a.status));
+      ++epi_phase;
+      return ok;
+    };
+    float m[HP], l[HP];
+    for (int lt = 0; lt < ntile; ++lt) {
+      const int tile = t_begin + lt;
+      const int b = tile / a.tps;
+      const int row0 = (tile - b * a.tps) * kRows;
+      const bool first_of_seg = (lt == 0) || seq_of(lt) != b;
+      const bool last_of_seg = (lt == ntile - 1) || seq_of(lt + 1) != b;
+      if (first_of_seg) {
+#pragma unroll
+        for (int h = 0; h < HP; ++h) {
+          m[h] = kNegBig;
+          l[h] = 0.f;
+        }
+      }
+      const int sb = lt & 1;
+      bool ok = __all_sync(0xffffffffu, wait_ab(smem_u32(&tl->s_full[sb]), (uint32_t)((lt >> 1) & 1),
+                                                abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      float s[HP];
+#pragma unroll
+      for (int h0 = 0; h0 < HP; h0 += 16) tmem_ld16(lane_base + (uint32_t)(sb * HP + h0), s + h0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tl->s_empty[sb]));
+
+      const bool valid = row0 + row < a.N;
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < HP; ++h) need |= valid && h < a.H && s[h] > m[h] + kSlack;
+      const int vb = lt & 1;
+      const int any_need = __any_sync(0xffffffffu, need);
+      if (lane == 0) tl->vote[vb][ew] = any_need ? 1 : 0;
+      if (!epi_sync()) break;
+      const bool need_any = tl->vote[vb][0] | tl->vote[vb][1] | tl->vote[vb][2] | tl->vote[vb][3];
+      if (need_any) {
+#pragma unroll
+        for (int h = 0; h < HP; ++h) {
+          float v = valid ? s[h] : kNegBig;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (lane == 0) tl->red[vb][ew][h] = v;
+        }
+        if (!epi_sync()) break;
+        float alpha[HP];
+#pragma unroll
+        for (int h = 0; h < HP; ++h) {
+          const float mx = fmaxf(fmaxf(tl->red[vb][0][h], tl->red[vb][1][h]),
+                                 fmaxf(tl->red[vb][2][h], tl->red[vb][3][h]));
+          const float mn = fmaxf(m[h], mx);
+          alpha[h] = exp2f(m[h] - mn);
+          m[h] = mn;
+          l[h] *= alpha[h];
+        }
+        if (!first_of_seg) {
+          // U holds the value MMAs up to tile lt-1: wait for the last one
+          const int pb = (lt - 1) & 1;
+          ok = __all_sync(0xffffffffu,
+                          wait_ab(smem_u32(&tl->u_done[pb]), (uint32_t)(((lt - 1) >> 1) & 1),
+                                  abort_flag, a.status));
+          if (!ok) break;
+          tc_fence_after();
+          for (int vg = 0; vg < a.nvg; ++vg) {
+#pragma unroll
+            for (int h0 = 0; h0 < HP; h0 += 16) {
+              float u[16];
+              const uint32_t ta = lane_base + (uint32_t)(2 * HP + vg * HP + h0);
+              tmem_ld16(ta, u);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) u[e] *= alpha[h0 + e];
+              tmem_st16(ta, u);
+            }
+          }
+        }
+      }
+      float p[HP];
+#pragma unroll
+      for (int h = 0; h < HP; ++h) {
+        p[h] = (valid && h < a.H) ? exp2f(s[h] - m[h]) : 0.f;
+        l[h] += p[h];
+      }
+      // P buffer lt&1 was read by the value MMA of tile lt-2
+      if (lt >= 2) {
+        ok = __all_sync(0xffffffffu,
+                        wait_ab(smem_u32(&tl->u_done[lt & 1]), (uint32_t)(((lt - 2) >> 1) & 1),
+                                abort_flag, a.status));
+        if (!ok) break;
+      }
+      unsigned char* pbuf = smem + a.off_p + (lt & 1) * a.pbuf_bytes;
+#pragma unroll
+      for (int h = 0; h < HP; ++h)
+        *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_off(h, row, HP)) = __float2bfloat16_rn(p[h]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tl->p_full[lt & 1]));
+
+      if (last_of_seg) {
+        ok = __all_sync(0xffffffffu, wait_ab(smem_u32(&tl->u_done[lt & 1]), (uint32_t)((lt >> 1) & 1),
+                                             abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        const long long slot = (long long)blockIdx.x + b;
+        float* rec = a.part + slot * a.H * a.pstride;
+        for (int vg = 0; vg < a.nvg; ++vg) {
+#pragma unroll
+          for (int h0 = 0; h0 < HP; h0 += 16) {
+            float u[16];
+            tmem_ld16(lane_base + (uint32_t)(2 * HP + vg * HP + h0), u);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (h0 + e < a.H) rec[(size_t)(h0 + e) * a.pstride + 4 + vg * 128 + row] = u[e];
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < HP; ++h) {
+          const float v = warp_sum(l[h]);
+          if (lane == 0) tl->lsum[ew][h] = v;
+        }
+        if (!epi_sync()) break;
+        if (ew == 0 && lane < a.H) {
+          float mm = 0.f;
+#pragma unroll
+          for (int h = 0; h < HP; ++h)
+            if (h == lane) mm = m[h];
+          rec[(size_t)lane * a.pstride + 0] = mm;
+          rec[(size_t)lane * a.pstride + 1] =
+              tl->lsum[0][lane] + tl->lsum[1][lane] + tl->lsum[2][lane] + tl->lsum[3][lane];
+        }
+        tc_fence_before();
+        if (!epi_sync()) break;  // lsum is reused by the next sequence
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, a.tmem_cols);
+  }
+}
+
+struct D2Plan {
+  int hp, tps, tiles, tpc, grid, nkg, nvg, spt, nstage;
+  int off_q, off_p, off_tail, qbuf_bytes, pbuf_bytes;
+  size_t smem;
+  uint32_t tmem_cols;
+  int pstride;
+  size_t off_qp, off_c0, off_part, ws_bytes;
+};
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+lla_status plan_2d(int B, int H, int N, int r_k, int r_v, D2Plan* p) {
+  D2Plan d{};
+  d.hp = H <= 16 ? 16 : 32;
+  d.tps = (N + kRows - 1) / kRows;
+  d.tiles = B * d.tps;
+  const DeviceInfo di = device_info();
+  const int grid0 = std::max(1, std::min(d.tiles, di.sms));
+  d.tpc = (d.tiles + grid0 - 1) / grid0;
+  d.grid = (d.tiles + d.tpc - 1) / d.tpc;
+  d.nkg = (r_k + 127) / 128;
+  d.nvg = r_v / 128;
+  d.spt = d.nkg + d.nvg;
+  d.qbuf_bytes = (r_k / 64) * d.hp * 128;
+  d.pbuf_bytes = 2 * d.hp * 128;
+  const size_t fixed = 2 * (size_t)d.qbuf_bytes + 2 * (size_t)d.pbuf_bytes + sizeof(Tail2) + 1024;
+  int nst = (int)std::min<size_t>(kMaxStages, ((size_t)di.smem_optin - fixed) / kStageBytes);
+  nst = std::min(nst, 6);
+  if (nst < d.spt) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D stage ring does not fit in shared memory");
+  d.nstage = nst;
+  d.off_q = nst * kStageBytes;
+  d.off_p = d.off_q + 2 * d.qbuf_bytes;
+  d.off_tail = d.off_p + 2 * d.pbuf_bytes;
+  d.smem = (size_t)d.off_tail + sizeof(Tail2) + 1024;
+  const int cols = (2 + d.nvg) * d.hp;
+  uint32_t c = 32;
+  while (c < (uint32_t)cols) c <<= 1;
+  d.tmem_cols = c;
+  d.pstride = 4 + r_v;
+  const size_t units = (size_t)B * H;
+  d.off_qp = 0;
+  d.off_c0 = al256(units * r_k * sizeof(float));
+  d.off_part = al256(d.off_c0 + units * sizeof(float));
+  d.ws_bytes = al256(d.off_part + ((size_t)d.grid + B) * H * d.pstride * sizeof(float));
+  *p = d;
+  return LLA_OK;
+}
+
+}  // namespace
+
+size_t workspace_2d(int B, int H, int N, int r_k, int r_v) {
+  D2Plan d;
+  if (plan_2d(B, H, N, r_k, r_v, &d) != LLA_OK) return 0;
+  return d.ws_bytes;
+}
+
+lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,
+                         int N, long long n_cap, int r_k, int r_v, const float* dk,
+                         const float* dv, const float* mu_k, const float* mu_v, float scale,
+                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  D2Plan d;
+  lla_status st = plan_2d(B, H, N, r_k, r_v, &d);
+  if (st != LLA_OK) return st;
+  if (ws == nullptr || ws_bytes < d.ws_bytes)
+    return fail(LLA_ERR_WORKSPACE, "LLA-2D workspace needs %zu bytes, got %zu", d.ws_bytes, ws_bytes);
+  char* wsb = static_cast<char*>(ws);
+  float* qp = reinterpret_cast<float*>(wsb + d.off_qp);
+  float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
+  float* part = reinterpret_cast<float*>(wsb + d.off_part);
+
+  CUtensorMap tk, tv;
+  {
+    const uint64_t dims[3] = {(uint64_t)r_k, (uint64_t)N, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)r_k * 2, (uint64_t)n_cap * r_k * 2};
+    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    if (!make_tmap_bf16(&tk, zk, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)r_v, (uint64_t)N, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)r_v * 2, (uint64_t)n_cap * r_v * 2};
+    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
+  if (st != LLA_OK) return st;
+
+  D2Args a{};
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.tps = d.tps;
+  a.tiles = d.tiles;
+  a.tpc = d.tpc;
+  a.r_k = r_k;
+  a.r_v = r_v;
+  a.nkg = d.nkg;
+  a.nvg = d.nvg;
+  a.spt = d.spt;
+  a.nstage = d.nstage;
+  a.off_q = d.off_q;
+  a.off_p = d.off_p;
+  a.off_tail = d.off_tail;
+  a.qbuf_bytes = d.qbuf_bytes;
+  a.pbuf_bytes = d.pbuf_bytes;
+  a.tmem_cols = d.tmem_cols;
+  a.qp = qp;
+  a.part = part;
+  a.pstride = d.pstride;
+  a.status = status_word();
+
+  auto kern = d.hp == 16 ? k_lla2d<16> : k_lla2d<32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_lla2d)");
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(d.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = d.smem;
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a);
+  if (e != cudaSuccess) return check_cuda(e, "launch k_lla2d");
+
+  return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v,
+                        (long long)d.tps * kRows, (long long)d.tpc * kRows, 1, out, lse, stream);
+}
+
+}  // namespace lla

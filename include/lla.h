@@ -96,7 +96,8 @@ LLA_API lla_status lla_device_status(unsigned int *status, int clear);
  *   N        cached tokens attended, 1 <= N <= n_cap.
  *   r_k, r_v latent ranks, multiples of 8, at most 256 (bf16) or 128 (fp32).
  *   dk_t     [H][d_h][r_k] fp32: W^K_up,t of layer d, loop t, per head.
- *   dv_t     [H][d_h][r_v] fp32: W^V_up,t.
+ *            16-byte aligned.
+ *   dv_t     [H][d_h][r_v] fp32: W^V_up,t. 16-byte aligned.
  *   mu_k_t, mu_v_t  [H][d_h] fp32 loop-t slices of the codec means, or NULL
  *            for zero.
  *   scale    softmax scale (usually 1/sqrt(d_h)).
@@ -130,8 +131,10 @@ LLA_API lla_status lla_decode_attn(const float *q, const void *zk, const void *z
  * The score and value contractions run on the tensor cores with bf16
  * operands (the absorbed query and the softmax weights are rounded to bf16)
  * and fp32 accumulation.
- * Limits: H <= 32 (H padded to a multiple of 16 inside), r_k and r_v
- * multiples of 64 up to 256, d_h 1..256, N >= 1.
+ * Limits: H <= 32 (padded to 16 or 32 inside), r_k a multiple of 64 and
+ * r_v a multiple of 128, both at most 256, d_h 1..256, 1 <= N <= n_cap.
+ * Outside them the call returns LLA_ERR_UNSUPPORTED and the workspace query
+ * returns 0.
  * -------------------------------------------------------------------------- */
 LLA_API size_t lla2d_decode_attn_workspace(int B, int H, int N, int r_k, int r_v);
 

@@ -88,3 +88,44 @@ def test_workspace_sizes_are_consistent():
 
 def test_device_status_needs_a_pointer():
     assert lla.lib().lla_device_status(None, 0) == _lib.LLA_ERR_INVALID_ARG
+
+
+def test_lla2d_rejects_unsupported_shapes_on_the_host():
+    h = lla.lib()
+    fake = ctypes.c_void_p(0x100000)
+
+    def call(**over):
+        args = dict(q=fake, zk=fake, zv=fake, zdt=1, B=2, H=16, d_h=128, N=8, n_cap=8, r_k=256,
+                    r_v=256, dk=fake, dv=fake, mu_k=None, mu_v=None, scale=0.1, out=fake,
+                    lse=None, ws=fake, ws_bytes=0, stream=None)
+        args.update(over)
+        return h.lla2d_decode_attn(*args.values())
+
+    assert call(zdt=0, r_k=128, r_v=128) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(H=33) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(r_k=96) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(r_v=64) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
+    assert lla.lla2d_decode_attn_workspace(2, 33, 8, 256, 256) == 0
+    assert lla.lla2d_decode_attn_workspace(2, 16, 8, 256, 192) == 0
+    assert lla.lla2d_decode_attn_workspace(256, 16, 8192, 256, 256) > 256 * 16 * 256 * 4
+
+
+def test_encode_rejects_bad_arguments_on_the_host():
+    h = lla.lib()
+    fake = ctypes.c_void_p(0x100000)
+
+    def call(**over):
+        args = dict(x=fake, xdt=1, T=4, N=10, G=2, d_loop=128, r=16, w=fake, mu=None, z=fake,
+                    zrs=16, zgs=160, stream=None)
+        args.update(over)
+        return h.lla_encode(*args.values())
+
+    assert call(xdt=0) == _lib.LLA_ERR_INVALID_ARG
+    assert call(d_loop=96) == _lib.LLA_ERR_INVALID_ARG
+    assert call(r=12) == _lib.LLA_ERR_INVALID_ARG
+    assert call(r=264) == _lib.LLA_ERR_INVALID_ARG
+    assert call(zrs=8) == _lib.LLA_ERR_INVALID_ARG         # rows narrower than r
+    assert call(zgs=16) == _lib.LLA_ERR_INVALID_ARG        # groups overlap rows
+    assert call(x=ctypes.c_void_p(0x100008)) == _lib.LLA_ERR_INVALID_ARG
+    assert call(N=0) == _lib.LLA_ERR_INVALID_ARG

@@ -1,0 +1,105 @@
+"""GPU parity of the latent write (lla_encode, tcgen05 + TMA) against the fp64
+oracle's Eq. 2, through the C ABI.
+
+The kernel rounds its fp32 result to bf16 once (round to nearest even), so
+each element may differ from the exact value by half a bf16 ulp (2^-9
+relative) plus fp32 accumulation error. The stated gate is the bf16
+tolerance max|z_gpu - z_ref| / max|z_ref| <= 2e-2; the element-wise check
+below is the tighter bound that rounding allows."""
+
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_encode_b200 as lla
+import oracle
+from decode_attention_encode_b200 import synth
+from lla_cases import TOL_BF16_REL, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def check(z_gpu, z_ref):
+    zg = to_f64(z_gpu)
+    scale = np.abs(z_ref).max()
+    err = np.abs(zg - z_ref).max() / scale
+    assert err <= TOL_BF16_REL, f"relative error {err:.3e}"
+    # element-wise: half a bf16 ulp plus accumulation slack
+    bound = 2.0 ** -8 * np.abs(z_ref) + 1e-4 * scale
+    bad = np.abs(zg - z_ref) > bound
+    assert not bad.any(), f"{bad.sum()} elements outside rounding bound; max rel {err:.2e}"
+    return err
+
+
+def make(T, N, G, d_loop, r, mu, seed=0):
+    x = synth.normal((T, N, G, d_loop), seed + 1, "cuda", dtype=torch.bfloat16)
+    w = synth.orthonormal(G, T * d_loop, r, seed + 2, "cuda").to(torch.bfloat16)   # [G, K, r]
+    w_t = w.transpose(1, 2).contiguous()                                            # [G, r, K]
+    m = synth.normal((G, T * d_loop), seed + 3, "cuda", std=0.5) if mu else None
+    return x, w, w_t, m
+
+
+@pytest.mark.parametrize("r", [8, 16, 24, 64, 128, 256])
+@pytest.mark.parametrize("mu", [False, True])
+def test_encode_ranks_ragged_tokens(r, mu):
+    T, N, G, d = 4, 300, 3, 64
+    x, w, w_t, m = make(T, N, G, d, r, mu, seed=r)
+    z = lla.lla_encode(x, w_t, m)
+    torch.cuda.synchronize()
+    ref = oracle.encode(to_f64(x), to_f64(w), None if m is None else to_f64(m))
+    check(z, ref)
+    assert lla.device_status() == 0
+
+
+@pytest.mark.parametrize("N", [1, 127, 128, 129, 1000])
+def test_encode_token_counts(N):
+    x, w, w_t, m = make(4, N, 2, 128, 16, True, seed=N)
+    z = lla.lla_encode(x, w_t, m)
+    torch.cuda.synchronize()
+    check(z, oracle.encode(to_f64(x), to_f64(w), to_f64(m)))
+
+
+def test_encode_writes_newest_token_into_a_store():
+    # One finished token per sequence: x [T][B][H][d], written at slot n of a
+    # [B][H][n_cap][r] latent store; nothing else in the store changes.
+    T, B, H, d, r, n_cap, slot = 4, 5, 6, 128, 24, 40, 17
+    x, w, w_t, m = make(T, B, H, d, r, True, seed=3)
+    store = torch.full((B, H, n_cap, r), 7.0, device="cuda", dtype=torch.bfloat16)
+    lla.lla_encode(x, w_t, m, z=store[:, :, slot], z_row_stride=H * n_cap * r,
+                   z_group_stride=n_cap * r)
+    torch.cuda.synchronize()
+    ref = oracle.encode(to_f64(x), to_f64(w), to_f64(m))          # [H, B, r]
+    check(store[:, :, slot].permute(1, 0, 2), ref)
+    rest = torch.cat([store[:, :, :slot], store[:, :, slot + 1:]], dim=2)
+    assert torch.all(rest == 7.0)
+
+
+def test_encode_svd_codec_full_size_sampled():
+    # One (layer, axis) of the prefill workload: 32768 tokens x 16 heads,
+    # stacked width 4 x 128, r = 16 from an SVD of a seeded N(0,1)
+    # calibration set (2048 rows per head).
+    T, N, G, d, r = 4, 32768, 16, 128, 16
+    cal = synth.normal((G, 2048, T * d), 11, "cpu", dtype=torch.float64).numpy()
+    fits = [oracle.svd_init(cal[g], r, T) for g in range(G)]
+    w = np.stack([f[0] for f in fits])      # [G, K, r]
+    mu = np.stack([f[2] for f in fits])     # [G, K]
+    w_bf = torch.from_numpy(w).to(torch.bfloat16).cuda()
+    w_t = w_bf.transpose(1, 2).contiguous()
+    mu_t = torch.from_numpy(mu).float().cuda()
+    x = synth.normal((T, N, G, d), 12, "cuda", dtype=torch.bfloat16)
+    z = lla.lla_encode(x, w_t, mu_t)
+    torch.cuda.synchronize()
+    rows = torch.tensor(sorted({0, 1, 127, 128, N - 1} |
+                               set(np.random.default_rng(0).integers(0, N, 64).tolist())))
+    ref = oracle.encode(to_f64(x[:, rows.cuda()]), to_f64(w_bf), to_f64(mu_t))
+    check(z[:, rows.cuda()], ref)
+    assert lla.device_status() == 0
+
+
+def test_encode_wide_stack_for_lla2d_geometry():
+    # LLA-2D folds heads into the stack: G = 1, d_loop = H * d_h.
+    T, N, H, dh, r = 4, 200, 16, 128, 256
+    x, w, w_t, m = make(T, N, 1, H * dh, r, True, seed=5)
+    z = lla.lla_encode(x, w_t, m)
+    torch.cuda.synchronize()
+    check(z, oracle.encode(to_f64(x), to_f64(w), to_f64(m)))
