@@ -152,14 +152,21 @@ class ClockSampler:
 
 class DecodeWorkload:
     """All layers' latent stores, decoders and queries of one config on the
-    device. The 2-D config keeps one latent per token and layer."""
+    device. The 2-D config keeps one latent per token and layer.
+
+    Per-head configs also carry the latent write of each sequence's newest
+    token: after the T x L attention calls, the token's stacked per-loop K
+    and V of every layer are encoded into slot N of the store (the attended
+    range stays [0, N), so every step measures the same context)."""
 
     def __init__(self, cfg: synth.DecodeConfig, device: str, seed_offset: int = 0):
         self.cfg = cfg
         c = cfg
         s = c.seed + seed_offset
-        zk_shape = (c.B, c.N, c.r_k) if c.two_d else (c.B, c.H, c.N, c.r_k)
-        zv_shape = (c.B, c.N, c.r_v) if c.two_d else (c.B, c.H, c.N, c.r_v)
+        self.write_latents = (not c.two_d) and c.dtype == "bf16" and c.d_h % 64 == 0
+        n_cap = c.N + 1 if self.write_latents else c.N
+        zk_shape = (c.B, n_cap, c.r_k) if c.two_d else (c.B, c.H, n_cap, c.r_k)
+        zv_shape = (c.B, n_cap, c.r_v) if c.two_d else (c.B, c.H, n_cap, c.r_v)
         self.zk = [synth.latents(zk_shape, s + 1000 * l + 1, device, decay=c.decay,
                                  dtype=c.torch_dtype) for l in range(c.L)]
         self.zv = [synth.latents(zv_shape, s + 1000 * l + 2, device, decay=c.decay,
@@ -178,10 +185,24 @@ class DecodeWorkload:
                               device=device)
         self.fn = lla.lla2d_decode_attn if c.two_d else lla.lla_decode_attn
         self.scale = 1.0 / math.sqrt(c.d_h)
+        if self.write_latents:
+            K = c.T * c.d_h
+            # encoders W_down^T [H][r][T*d_h] per (layer, axis), means, and the
+            # newest token's stacked per-loop K and V [T][B][H][d_h]
+            self.wk = synth.orthonormal(c.L * c.H, K, c.r_k, s + 6, device).transpose(1, 2) \
+                .contiguous().to(torch.bfloat16).view(c.L, c.H, c.r_k, K)
+            self.wv = synth.orthonormal(c.L * c.H, K, c.r_v, s + 7, device).transpose(1, 2) \
+                .contiguous().to(torch.bfloat16).view(c.L, c.H, c.r_v, K)
+            self.muk = synth.normal((c.L, c.H, K), s + 8, device, std=0.1)
+            self.muv = synth.normal((c.L, c.H, K), s + 9, device, std=0.1)
+            self.xk = synth.normal((c.L, c.T, c.B, c.H, c.d_h), s + 10, device, dtype=torch.bfloat16)
+            self.xv = synth.normal((c.L, c.T, c.B, c.H, c.d_h), s + 11, device, dtype=torch.bfloat16)
+            self.n_cap = n_cap
 
-    def step(self, q=None, out=None, lse=None):
+    def step(self, q=None, out=None, lse=None, xk=None, xv=None):
         """One looped decode step: loops outer, layers inner (each loop's
-        query depends on the previous loop's output in a real model)."""
+        query depends on the previous loop's output in a real model), then
+        the newest token's latent write."""
         c = self.cfg
         q = self.q if q is None else q
         out = self.out if out is None else out
@@ -190,9 +211,23 @@ class DecodeWorkload:
             for l in range(c.L):
                 self.fn(q[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
                         scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
+        if self.write_latents:
+            self.write_newest(self.xk if xk is None else xk, self.xv if xv is None else xv)
+
+    def write_newest(self, xk, xv):
+        c = self.cfg
+        for l in range(c.L):
+            for x, w, mu, z, r in ((xk, self.wk, self.muk, self.zk, c.r_k),
+                                   (xv, self.wv, self.muv, self.zv, c.r_v)):
+                self.lla.lla_encode(x[l], w[l], mu[l], z=z[l][:, :, c.N],
+                                    z_row_stride=c.H * self.n_cap * r,
+                                    z_group_stride=self.n_cap * r)
 
     def launches_per_step(self) -> int:
-        return 3 * self.cfg.L * self.cfg.T
+        n = 3 * self.cfg.L * self.cfg.T
+        if self.write_latents:
+            n += 2 * self.cfg.L
+        return n
 
 
 def kernel_hash() -> str:
@@ -328,6 +363,8 @@ def run_lla(args, world, rank, local):
                           scale=wl.scale, out=wl.out[l, t], lse=wl.lse[l, t], workspace=wl.ws)
                     if t == 0:
                         call_ev[l][1].record(stream)
+            if wl.write_latents:
+                wl.write_newest(wl.xk, wl.xv)
         else:
             wl.step()
     ev[1].record(stream)
@@ -350,30 +387,36 @@ def run_lla(args, world, rank, local):
     # outputs back to pinned host memory, every step
     e2e = None
     if not args.no_e2e:
-        q_host = wl.q.to("cpu").pin_memory()
+        ins = [wl.q] + ([wl.xk, wl.xv] if wl.write_latents else [])
+        hosts = [t.to("cpu").pin_memory() for t in ins]
+        devs = [torch.empty_like(t) for t in ins]
         out_host = torch.empty(wl.out.shape, dtype=torch.float32).pin_memory()
         lse_host = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
-        q_dev = torch.empty_like(wl.q)
-        for _ in range(2):
-            q_dev.copy_(q_host, non_blocking=True)
-            wl.step(q=q_dev)
+
+        def e2e_step():
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            if wl.write_latents:
+                wl.step(q=devs[0], xk=devs[1], xv=devs[2])
+            else:
+                wl.step(q=devs[0])
             out_host.copy_(wl.out, non_blocking=True)
             lse_host.copy_(wl.lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
-            q_dev.copy_(q_host, non_blocking=True)
-            wl.step(q=q_dev)
-            out_host.copy_(wl.out, non_blocking=True)
-            lse_host.copy_(wl.lse, non_blocking=True)
+            e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
         e2e = {"value": world * tokens_per_step / (e2e_ms * 1e-3), "unit": UNIT,
-               "h2d_bytes_per_step": q_host.numel() * 4,
+               "h2d_bytes_per_step": sum(h_.numel() * h_.element_size() for h_ in hosts),
                "d2h_bytes_per_step": (out_host.numel() + lse_host.numel()) * 4}
 
     line = {
@@ -383,7 +426,8 @@ def run_lla(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": describe(cfg),
-            "step": f"{cfg.L * cfg.T} decode calls (T loops x L layers), 3 kernels each",
+            "step": f"{cfg.L * cfg.T} decode calls (T loops x L layers), 3 kernels each"
+                    + (f", then {2 * cfg.L} latent writes of the newest token" if wl.write_latents else ""),
             "accumulation": "fp32",
             "l2": "no flush: each layer's latent store "
                   f"({step_bytes / 1e9:.2f} GB) is larger than L2 (126 MB)",

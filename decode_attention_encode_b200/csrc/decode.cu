@@ -508,16 +508,15 @@ StreamFn pick_stream(int lpt, int s, bool exact) {
   }
 #define LLA_CASE(L, S) \
   if (lpt == L && s == S) return k_stream<ESZ, L, S, S, true>;
-  LLA_CASE(1, 1) LLA_CASE(1, 3) LLA_CASE(2, 1) LLA_CASE(2, 3) LLA_CASE(4, 1)
-  LLA_CASE(4, 3) LLA_CASE(8, 1) LLA_CASE(8, 2) LLA_CASE(8, 3) LLA_CASE(8, 4)
+  LLA_CASE(1, 1) LLA_CASE(1, 2) LLA_CASE(1, 3) LLA_CASE(1, 4)
+  LLA_CASE(2, 1) LLA_CASE(2, 2) LLA_CASE(2, 3) LLA_CASE(2, 4)
+  LLA_CASE(4, 1) LLA_CASE(4, 2) LLA_CASE(4, 3) LLA_CASE(4, 4)
+  LLA_CASE(8, 1) LLA_CASE(8, 2) LLA_CASE(8, 3) LLA_CASE(8, 4)
 #undef LLA_CASE
   return nullptr;
 }
 
-bool exact_variant(int lpt, int s) {
-  if (lpt == 8) return s >= 1 && s <= 4;
-  return s == 1 || s == 3;
-}
+bool exact_variant(int lpt, int s) { return lpt >= 1 && lpt <= 8 && s >= 1 && s <= 4; }
 
 int env_int(const char* name, int dflt) {
   const char* v = std::getenv(name);
@@ -573,6 +572,10 @@ lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePla
   // phase is one contiguous 128-byte row piece), so row reads are
   // conflict-free.
   int lpt = 1 << std::min(v2(d.nseg_k), v2(d.nseg_v));
+  // tuning override (power of two dividing both segment counts)
+  const int lpt_env = env_int("LLA_DECODE_LPT", 0);
+  if (lpt_env == 1 || lpt_env == 2 || lpt_env == 4 || lpt_env == 8)
+    if (d.nseg_k % lpt_env == 0 && d.nseg_v % lpt_env == 0) lpt = lpt_env;
   if (d.nseg_k == d.nseg_v && exact_variant(lpt, d.nseg_k / lpt)) {
     d.exact = true;
     d.sk = d.sv = d.nseg_k / lpt;
@@ -589,7 +592,7 @@ lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePla
   const DeviceInfo di = device_info();
   d.warps = std::max(1, std::min(8, env_int("LLA_DECODE_WARPS", 8)));
   d.nstage = std::max(2, std::min(8, env_int("LLA_DECODE_STAGES", 2)));
-  const int target = std::max(1024, env_int("LLA_DECODE_STAGE_BYTES", 12288));
+  const int target = std::max(1024, env_int("LLA_DECODE_STAGE_BYTES", 10240));
   const int pair = 2 * ns;
   d.tile = std::max(pair, (target / tok_bytes) / pair * pair);
   // fit the CTA's shared memory

@@ -56,6 +56,7 @@ struct SmemTail {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  uint64_t epi;  // 4-warp rendezvous of the epilogue warps
   uint32_t tmem_base;
   int abort_flag;
   float muw[256];
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&tail->tempty[i]), 4);
     }
     mbar_init(smem_u32(&tail->drain), 1);
+    mbar_init(smem_u32(&tail->epi), 4);
     tail->abort_flag = 0;
     fence_mbar_init();
   }
@@ -186,12 +188,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
+    uint32_t epi_phase = 0;
+    // bounded rendezvous of the 4 epilogue warps (an mbarrier, so a warp
+    // that aborts cannot leave the others waiting forever)
+    auto epi_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tail->epi));
+      const bool ok = __all_sync(
+          0xffffffffu, wait_or_abort(smem_u32(&tail->epi), epi_phase & 1u, abort_flag, a.status));
+      ++epi_phase;
+      return ok;
+    };
     int cur_g = -1;
     for (int tile = t_begin, lt = 0; tile < t_end; ++tile, ++lt) {
       const int g = tile / a.mtiles;
       const int m0 = (tile - g * a.mtiles) * kTileM;
       if (g != cur_g) {
-        named_bar(1, 128);  // previous tile's readers of muw are done
+        if (!epi_sync()) break;  // previous tile's readers of muw are done
         for (int c = ew; c < a.r; c += 4) {
           float acc = 0.f;
           if (a.mu) {
@@ -202,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (lane == 0) tail->muw[c] = acc;
         }
-        named_bar(1, 128);
+        if (!epi_sync()) break;
         cur_g = g;
       }
       const int acc = lt & 1;

@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile = t_begin + lt;
       const int b = tile / a.tps;
       const int row0 = (tile - b * a.tps) * kRows;
-      const bool first_of_seg = (lt == 0) || seq_of(lt) != b;
+      const bool first_of_seg = (lt == 0) || seq_of(lt - 1) != b;
       const bool last_of_seg = (lt == ntile - 1) || seq_of(lt + 1) != b;
       if (first_of_seg) {
 #pragma unroll

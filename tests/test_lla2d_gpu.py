@@ -49,7 +49,7 @@ def test_context_lengths(N):
     run(2, 16, 128, N, 256, 256, n_cap=N + 3, mu=True, seed=N)
 
 
-@pytest.mark.parametrize("B, N", [(37, 1000), (300, 200), (5, 40000)])
+@pytest.mark.parametrize("B, N", [(37, 1000), (300, 200), (5, 40000), (600, 100), (150, 700)])
 def test_sequences_split_across_ctas(B, N):
     run(B, 16, 128, N, 256, 256, units=sample_units(B, 16), decay=True, seed=B)
 
