@@ -31,7 +31,7 @@ LLA_DEVICE_WAIT_TIMEOUT = 0x1
 # Every symbol include/lla.h declares.
 EXPORTS = (
     "lla_status_string", "lla_last_error", "lla_version", "lla_device_status",
-    "lla_decode_attn_workspace", "lla_decode_attn",
+    "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn",
     "lla_encode",
 )
@@ -58,6 +58,8 @@ _SIGS = {
     "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
                         [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "lla_decode_attn_noalloc": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
+                                [_c_float, _vp, _vp, _vp], _c_int),
     "lla2d_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
                           [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla_encode": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp], _c_int),
@@ -169,6 +171,30 @@ def lla_decode_attn(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, sca
     Returns (out [B,H,d_h], lse [B,H] or None)."""
     return _decode("lla_decode_attn", "lla_decode_attn_workspace", q, zk, zv, dk_t, dv_t, N,
                    mu_k_t, mu_v_t, scale, out, lse, workspace, stream, want_lse, two_d=False)
+
+
+def lla_decode_attn_noalloc(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, scale=None,
+                            out=None, lse=None, stream=None, want_lse=True):
+    """Per-head decode like lla_decode_attn, for callers that cannot allocate
+    device memory: the library uses its own fixed scratch array instead of a
+    workspace (see include/lla.h for the size limit and the ordering rule).
+    Only `out` and `lse` are allocated here when not given."""
+    _need_cuda(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse)
+    B, H, d_h = q.shape
+    n_cap, r_k = zk.shape[2], zk.shape[3]
+    r_v = zv.shape[3]
+    N = n_cap if N is None else N
+    scale = 1.0 / math.sqrt(d_h) if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, d_h), device=q.device, dtype=torch.float32)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    st = lib().lla_decode_attn_noalloc(_ptr(q), _ptr(zk), _ptr(zv), _dtype_code(zk), B, H, d_h,
+                                       N, n_cap, r_k, r_v, _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t),
+                                       _ptr(mu_v_t), float(scale), _ptr(out), _ptr(lse),
+                                       _stream(stream))
+    _check(st)
+    return out, lse
 
 
 def lla2d_decode_attn(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, scale=None,

@@ -94,7 +94,9 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-lla_status check_decode_args(const float* q, const void* zk, const void* zv, lla_dtype zdt,
+}  // namespace
+
+lla_status lla::check_decode_args(const float* q, const void* zk, const void* zv, lla_dtype zdt,
                              int B, int H, int d_h, int N, int n_cap, int r_k, int r_v,
                              const float* dk, const float* dv, const float* mu_k,
                              const float* mu_v, float* out, float* lse, void* ws, int* esz) {
@@ -117,8 +119,6 @@ lla_status check_decode_args(const float* q, const void* zk, const void* zv, lla
   if (ws && !aligned(ws, 16)) return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   return LLA_OK;
 }
-
-}  // namespace
 
 extern "C" {
 

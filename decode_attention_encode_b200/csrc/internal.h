@@ -28,6 +28,13 @@ lla_status fail(lla_status s, const char* fmt, ...);
 // Maps a CUDA error to LLA_ERR_CUDA with its message, or LLA_OK.
 lla_status check_cuda(cudaError_t e, const char* what);
 
+// Host-side argument checks shared by the decode entry points; sets *esz to
+// the latent element size.
+lla_status check_decode_args(const float* q, const void* zk, const void* zv, lla_dtype zdt, int B,
+                             int H, int d_h, int N, int n_cap, int r_k, int r_v, const float* dk,
+                             const float* dv, const float* mu_k, const float* mu_v, float* out,
+                             float* lse, void* ws, int* esz);
+
 // Launch plan of the per-head absorbed decode. See decode.cu.
 struct DecodePlan {
   int esz;             // bytes per latent element (2 or 4)

@@ -122,6 +122,40 @@ LLA_API lla_status lla_decode_attn(const float *q, const void *zk, const void *z
                            void *stream);
 
 /* --------------------------------------------------------------------------
+ * Per-head absorbed decode without a caller workspace. The paper has no
+ * counterpart: this is a deployment convenience of this library.
+ *
+ * Some callers cannot allocate device memory: for example a plugin running
+ * inside a serving engine that has already reserved the whole device for its
+ * own pool, or code that must not call cudaMalloc after start-up because an
+ * allocation can synchronise the device at an unpredictable point. This call
+ * computes exactly what lla_decode_attn computes, with the same kernels and
+ * launch plan, and takes the same arguments minus the workspace. Its scratch
+ * is a fixed array of LLA_NOALLOC_SCRATCH_BYTES compiled into the library,
+ * which every GPU that loads liblla holds until the process exits.
+ *  - It allocates nothing and calls no allocating routine.
+ *  - Shapes whose workspace (lla_decode_attn_workspace) exceeds the scratch
+ *    return LLA_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device looks up the scratch's device address
+ *    (cudaGetSymbolAddress with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one scratch array, and it keeps the
+ *    last call's contents (nothing in it needs to start at zero). Calls
+ *    whose kernels overlap on the GPU (different streams without ordering)
+ *    race on it and give wrong results: order them.
+ * -------------------------------------------------------------------------- */
+#define LLA_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20) /* 4 MiB per device */
+
+LLA_API lla_status lla_decode_attn_noalloc(const float *q, const void *zk,
+                                           const void *zv, lla_dtype zdt, int B,
+                                           int H, int d_h, int N, int n_cap,
+                                           int r_k, int r_v, const float *dk_t,
+                                           const float *dv_t,
+                                           const float *mu_k_t,
+                                           const float *mu_v_t, float scale,
+                                           float *out, float *lse, void *stream);
+
+/* --------------------------------------------------------------------------
  * LLA-2D absorbed decode, one (layer d, loop t) step (§3 "The LLA-2D
  * variant": one latent per token and layer, decoded into every head).
  *
