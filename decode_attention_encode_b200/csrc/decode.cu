@@ -39,9 +39,9 @@ constexpr float kNegBig = -1.0e30f;
 // it by this much (log2 units), so p_j <= 2^8 and rescales are rare.
 constexpr float kRescaleSlack = 8.0f;
 
-constexpr int kAbsorbRows = 8;    // batch rows per k_absorb CTA
+constexpr int kAbsorbRows = 8;    // batch rows (one per warp) per k_absorb CTA
 constexpr int kCombineRows = 8;   // batch rows (one per warp) per k_combine CTA
-constexpr int kSmemChunk = 8192;  // floats of a decoder chunk staged in shared memory
+constexpr int kColChunk = 32;     // decoder columns (absorb) / rows (combine) per CTA
 
 // ---------------------------------------------------------------------------
 // k_absorb
@@ -57,74 +57,57 @@ struct AbsorbArgs {
   float* c0;  // [B*H], natural-log units
 };
 
-// One CTA per (head, block of kAbsorbRows batch rows). W^K_up,t of the head
-// is staged through shared memory in row chunks (coalesced float4 loads, all
-// issued before use); each thread owns fixed (b, c) outputs.
+// One CTA per (head, 8 batch rows, 32 latent columns): the CTA stages its
+// d_h x 32 slice of W^K_up,t and the 8 query rows in shared memory, and each
+// thread forms one q'[b][c] as a d_h-long dot product.
 __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
   __shared__ float q_s[kAbsorbRows * 256];
-  __shared__ __align__(16) float d_s[kSmemChunk];
+  __shared__ __align__(16) float d_s[256 * kColChunk];
   pdl_launch_dependents();
   const int h = blockIdx.x;
   const int b0 = blockIdx.y * kAbsorbRows;
+  const int c0 = blockIdx.z * kColChunk;
   const int nb = min(kAbsorbRows, a.B - b0);
+  const int nc = min(kColChunk, a.r_k - c0);
   for (int idx = threadIdx.x; idx < nb * a.d_h; idx += blockDim.x) {
     const int bb = idx / a.d_h, i = idx - bb * a.d_h;
     q_s[idx] = a.q[((size_t)(b0 + bb) * a.H + h) * a.d_h + i];
   }
+  // W^K rows i, columns [c0, c0 + nc): nc is a multiple of 8, so float4 loads
+  const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
+  const int n4 = nc / 4;
+  for (int idx = threadIdx.x; idx < a.d_h * n4; idx += blockDim.x) {
+    const int i = idx / n4, j = idx - i * n4;
+    reinterpret_cast<float4*>(d_s + i * kColChunk)[j] =
+        __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j);
+  }
   __syncthreads();
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int bb = warp; bb < nb; bb += nwarps) {
-    float acc = 0.f;
-    if (a.mu_k)
-      for (int i = lane; i < a.d_h; i += 32)
-        acc += q_s[bb * a.d_h + i] * a.mu_k[(size_t)h * a.d_h + i];
-    acc = warp_sum(acc);
-    if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
-  }
-
-  // outputs (bb, c), bb < nb, c < r_k; at most kAbsorbRows*256/256 = 8 per thread
-  constexpr int kMaxOut = kAbsorbRows;
-  float acc[kMaxOut];
-  int ob[kMaxOut], oc[kMaxOut];
-  const int nout = nb * a.r_k;
-#pragma unroll
-  for (int k = 0; k < kMaxOut; ++k) {
-    const int o = threadIdx.x + k * blockDim.x;
-    acc[k] = 0.f;
-    ob[k] = o < nout ? o / a.r_k : 0;
-    oc[k] = o < nout ? o - ob[k] * a.r_k : 0;
-  }
-  const float* D = a.dk + (size_t)h * a.d_h * a.r_k;
-  const int rows_per_chunk = max(1, kSmemChunk / a.r_k);
-  for (int i0 = 0; i0 < a.d_h; i0 += rows_per_chunk) {
-    const int ni = min(rows_per_chunk, a.d_h - i0);
-    const int n4 = ni * a.r_k / 4;  // r_k is a multiple of 8
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < n4; idx += blockDim.x)
-      reinterpret_cast<float4*>(d_s)[idx] =
-          __ldg(reinterpret_cast<const float4*>(D + (size_t)i0 * a.r_k) + idx);
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kMaxOut; ++k) {
-      if (threadIdx.x + k * blockDim.x < nout) {
-        const float* qrow = q_s + ob[k] * a.d_h + i0;
-        const float* dcol = d_s + oc[k];
-        float s0 = 0.f, s1 = 0.f;
-        int i = 0;
-        for (; i + 1 < ni; i += 2) {
-          s0 = fmaf(dcol[i * a.r_k], qrow[i], s0);
-          s1 = fmaf(dcol[(i + 1) * a.r_k], qrow[i + 1], s1);
-        }
-        if (i < ni) s0 = fmaf(dcol[i * a.r_k], qrow[i], s0);
-        acc[k] += s0 + s1;
-      }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.z == 0) {
+    // c0 = scale * q . mu_k (natural-log units), one warp per row
+    for (int bb = warp; bb < nb; bb += blockDim.x >> 5) {
+      float acc = 0.f;
+      if (a.mu_k)
+        for (int i = lane; i < a.d_h; i += 32)
+          acc += q_s[bb * a.d_h + i] * a.mu_k[(size_t)h * a.d_h + i];
+      acc = warp_sum(acc);
+      if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
     }
   }
-#pragma unroll
-  for (int k = 0; k < kMaxOut; ++k)
-    if (threadIdx.x + k * blockDim.x < nout)
-      a.qp[((size_t)(b0 + ob[k]) * a.H + h) * a.r_k + oc[k]] = acc[k] * a.qscale;
+  // thread -> (row bb = warp, column c0 + lane)
+  const int bb = warp;
+  if (bb < nb && lane < nc) {
+    const float* qrow = q_s + bb * a.d_h;
+    float s0 = 0.f, s1 = 0.f;
+    int i = 0;
+    for (; i + 1 < a.d_h; i += 2) {
+      s0 = fmaf(d_s[i * kColChunk + lane], qrow[i], s0);
+      s1 = fmaf(d_s[(i + 1) * kColChunk + lane], qrow[i + 1], s1);
+    }
+    if (i < a.d_h) s0 = fmaf(d_s[i * kColChunk + lane], qrow[i], s0);
+    a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = (s0 + s1) * a.qscale;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -418,19 +401,30 @@ struct CombineArgs {
   float* lse;
 };
 
-// One CTA per (head, block of kCombineRows batch rows): warp w merges the
-// partial records of row w (lanes across the latent index), then W^V_up,t is
-// staged in shared memory in padded row chunks and applied to all rows.
+// One CTA per (head, 8 batch rows, 32 output channels): warp w merges the
+// partial records of row w (lanes across the latent index) into ubar, the
+// CTA stages its 32 x r_v slice of W^V_up,t (rows padded by one float so
+// consecutive rows fall in distinct banks), and each thread forms one
+// out[b][h][i] as an r_v-long dot product.
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   __shared__ float ub[kCombineRows * 256];
-  __shared__ float d_s[kSmemChunk + 256];
-  pdl_wait();  // partials come from the streaming kernel
+  __shared__ float d_s[kColChunk * 257];
   const int h = blockIdx.x;
   const int b0 = blockIdx.y * kCombineRows;
+  const int i0 = blockIdx.z * kColChunk;
   const int nb = min(kCombineRows, a.B - b0);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-
-  for (int bb = warp; bb < nb; bb += nwarps) {
+  const int ni = min(kColChunk, a.d_h - i0);
+  const int pitch = a.r_v + 1;
+  // W^V does not depend on the streaming kernel: stage it before waiting
+  const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
+  for (int idx = threadIdx.x; idx < ni * a.r_v; idx += blockDim.x) {
+    const int i = idx / a.r_v, c = idx - i * a.r_v;
+    d_s[i * pitch + c] = __ldg(D + idx);
+  }
+  pdl_wait();  // partials come from the streaming kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bb = warp;
+  if (bb < nb) {
     const long long u = (long long)(b0 + bb) * a.H + h;
     // The split runs over units (b, h) for per-head LLA and over sequences
     // b for LLA-2D; piece w of split key k is partial record w + k.
@@ -460,33 +454,20 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
       }
       ub[bb * a.r_v + c] = acc * inv;
     }
-    if (lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
+    if (blockIdx.z == 0 && lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
   }
-
-  // out[b][h][i] = sum_c W^V[i][c] ubar_b[c] + mu^V[i]
-  const float* D = a.dv + (size_t)h * a.d_h * a.r_v;
-  const int pitch = a.r_v + 1;  // padded rows: threads with consecutive i hit distinct banks
-  const int rows_per_chunk = max(1, kSmemChunk / pitch);
-  for (int i0 = 0; i0 < a.d_h; i0 += rows_per_chunk) {
-    const int ni = min(rows_per_chunk, a.d_h - i0);
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < ni * a.r_v; idx += blockDim.x) {
-      const int i = idx / a.r_v, c = idx - i * a.r_v;
-      d_s[i * pitch + c] = __ldg(D + (size_t)(i0 + i) * a.r_v + c);
+  __syncthreads();
+  // thread -> (row bb = warp, output channel i0 + lane)
+  if (bb < nb && lane < ni) {
+    const float* drow = d_s + lane * pitch;
+    const float* urow = ub + bb * a.r_v;
+    float s0 = 0.f, s1 = 0.f;
+    for (int c = 0; c < a.r_v; c += 2) {
+      s0 = fmaf(drow[c], urow[c], s0);
+      s1 = fmaf(drow[c + 1], urow[c + 1], s1);
     }
-    __syncthreads();
-    for (int o = threadIdx.x; o < nb * ni; o += blockDim.x) {
-      const int bb = o / ni, i = o - bb * ni;
-      const float* drow = d_s + i * pitch;
-      const float* urow = ub + bb * a.r_v;
-      float s0 = 0.f, s1 = 0.f;
-      for (int c = 0; c < a.r_v; c += 2) {
-        s0 = fmaf(drow[c], urow[c], s0);
-        s1 = fmaf(drow[c + 1], urow[c + 1], s1);
-      }
-      const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + i] : 0.f;
-      a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + i] = s0 + s1 + mu;
-    }
+    const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + lane] : 0.f;
+    a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = s0 + s1 + mu;
   }
 }
 
@@ -531,7 +512,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream) {
   AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0};
-  dim3 grid(H, (B + kAbsorbRows - 1) / kAbsorbRows);
+  dim3 grid(H, (B + kAbsorbRows - 1) / kAbsorbRows, (r_k + kColChunk - 1) / kColChunk);
   k_absorb<<<grid, 256, 0, stream>>>(a);
   return check_cuda(cudaGetLastError(), "launch k_absorb");
 }
@@ -544,7 +525,7 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse};
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(H, (B + kCombineRows - 1) / kCombineRows);
+  cfg.gridDim = dim3(H, (B + kCombineRows - 1) / kCombineRows, (d_h + kColChunk - 1) / kColChunk);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
