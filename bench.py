@@ -41,8 +41,18 @@ from decode_attention_encode_b200 import synth  # noqa: E402
 METRIC = "LLA decode: cached tokens attended/sec per loop step; HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
 DEFAULT_CONFIG = "perhead_4x"
-KERNEL_SRC = os.path.join(ROOT, "decode_attention_encode_b200", "csrc", "decode.cu")
+CSRC = os.path.join(ROOT, "decode_attention_encode_b200", "csrc")
 PROFILE_DIR = os.path.join(ROOT, "profiles")
+ENCODE_CONFIGS = {synth.C5_ENCODE.name: synth.C5_ENCODE}
+
+
+def main_kernel(config_name: str):
+    """(kernel name, source file) of the kernel that dominates a workload."""
+    if config_name in ENCODE_CONFIGS:
+        return "k_encode", os.path.join(CSRC, "encode.cu")
+    if synth.DECODE_CONFIGS[config_name].two_d:
+        return "k_lla2d", os.path.join(CSRC, "lla2d.cu")
+    return "k_stream", os.path.join(CSRC, "stream.cu")
 
 
 def parse_args():
@@ -50,7 +60,8 @@ def parse_args():
     p.add_argument("--gpus", type=int, default=int(os.environ.get("WORLD_SIZE", "1")))
     p.add_argument("--steps", type=int, default=5)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.DECODE_CONFIGS))
+    p.add_argument("--config", default=DEFAULT_CONFIG,
+                   choices=sorted(synth.DECODE_CONFIGS) + sorted(ENCODE_CONFIGS))
     p.add_argument("--impl", default="lla", choices=["lla", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -230,20 +241,135 @@ class DecodeWorkload:
         return n
 
 
-def kernel_hash() -> str:
-    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+class EncodeWorkload:
+    """Prefill latent write of one sequence: for every layer and both axes,
+    the N tokens' stacked per-loop K (or V) vectors x [T][N][G][d_loop] are
+    encoded into the [G][N][r] latent store (48 calls at 24 layers). All
+    inputs are resident on the device; the encoders come from an SVD of a
+    seeded N(0, 1) calibration set per (layer, axis, head)."""
+
+    def __init__(self, cfg: synth.EncodeConfig, device: str, seed_offset: int = 0):
+        import decode_attention_encode_b200 as lla
+        self.lla = lla
+        c = self.cfg = cfg
+        s = c.seed + seed_offset
+        K = c.T * c.d_loop
+        self.x = [synth.normal((c.T, c.N, c.G, c.d_loop), s + 10 + i, device, dtype=torch.bfloat16)
+                  for i in range(2 * c.L)]
+        # codec fit: top-r right singular vectors of the centred calibration
+        # matrix, per (layer, axis, head); done once, outside the timed region
+        w_t, mu = [], []
+        for i in range(2 * c.L):
+            cal = synth.normal((c.G, c.n_cal, K), s + 1000 + i, device)
+            m = cal.mean(dim=1, keepdim=True)
+            _, _, vh = torch.linalg.svd(cal - m, full_matrices=False)
+            w_t.append(vh[:, :c.r, :].contiguous().to(torch.bfloat16))   # [G][r][K]
+            mu.append(m[:, 0, :].contiguous())                             # [G][K]
+        self.w_t, self.mu = w_t, mu
+        self.z = [torch.empty((c.G, c.N, c.r), device=device, dtype=torch.bfloat16)
+                  for _ in range(2 * c.L)]
+
+    def step(self, x=None):
+        x = self.x if x is None else x
+        for i in range(2 * self.cfg.L):
+            self.lla.lla_encode(x[i], self.w_t[i], self.mu[i], z=self.z[i],
+                                z_row_stride=self.cfg.r, z_group_stride=self.cfg.N * self.cfg.r)
+
+    def launches_per_step(self) -> int:
+        return 2 * self.cfg.L
+
+
+def run_encode_bench(args, world, rank, local):
+    cfg = ENCODE_CONFIGS[args.config]
+    dev = f"cuda:{local}"
+    wl = EncodeWorkload(cfg, dev, seed_offset=rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        wl.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_per_step = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    kern = []
+    for i in range(2 * cfg.L):
+        with wl.lla.kernel_timer() as kt:
+            wl.lla.lla_encode(wl.x[i], wl.w_t[i], wl.mu[i], z=wl.z[i], z_row_stride=cfg.r,
+                              z_group_stride=cfg.N * cfg.r)
+        kern.append(kt.ms)
+    kern_ms = sum(kern) / len(kern)
+    call_bytes = (cfg.T * cfg.N * cfg.G * cfg.d_loop + cfg.G * cfg.N * cfg.r) * 2
+    hbm_peak, peak_src = peaks()
+    achieved = call_bytes / (kern_ms * 1e-3) / 1e9
+    flops = 2 * cfg.N * cfg.G * cfg.T * cfg.d_loop * cfg.r
+    line = {
+        "metric": "LLA encode: prefill tokens encoded/sec (every layer, K and V)",
+        "value": world * cfg.N / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: lla_encode of N={cfg.N} tokens x G={cfg.G} heads x "
+                               f"{cfg.L} layers x 2 axes, stack {cfg.T}x{cfg.d_loop}, r={cfg.r}",
+                   "step": f"{2 * cfg.L} encode calls", "accumulation": "fp32",
+                   "l2": "no flush: each call reads 0.54 GB of fresh input",
+                   "parallelism": f"dp{world} (independent sequences per GPU)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": profiled_traffic(cfg.name),
+                     "kernel": "k_encode", "kernel_ms_mean": kern_ms,
+                     "algorithmic_bytes_per_launch": call_bytes,
+                     "tensor_tflops": flops / (kern_ms * 1e-3) / 1e12,
+                     "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs (copy, burst)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s"},
+        "gpu_launches": wl.launches_per_step() * args.steps,
+        "clocks": clk,
+        "e2e": None,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import numpy as np
+
+        import oracle
+        K = cfg.T * cfg.d_loop
+        n = 512
+        x = wl.x[0][:, :n].double().cpu().numpy()
+        w = wl.w_t[0].transpose(1, 2).double().cpu().numpy()
+        mu = wl.mu[0].double().cpu().numpy()
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < 10.0:
+            oracle.encode(x, w, mu)
+            reps += 1
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {
+            "value": reps * n / (2 * cfg.L) / dt, "unit": "tokens/s",
+            "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{reps} x {n} tokens of one (layer, axis) call in fp64; "
+                      f"tokens/s divides by the {2 * cfg.L} calls of a step"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def profiled_traffic(config_name: str):
-    """DRAM bytes per launch of the stream kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
-    path = os.path.join(PROFILE_DIR, f"k_stream_{config_name}.md")
+    """DRAM bytes per launch of the workload's main kernel from the committed
+    ncu summary, if that summary was taken on the current kernel source."""
+    kernel, src = main_kernel(config_name)
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{config_name}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not h or not t or h.group(1) != kernel_hash():
+    cur = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if not h or not t or h.group(1) != cur:
         return None
     return float(t.group(1))
 
@@ -302,6 +428,10 @@ def cpu_baseline(cfg: synth.DecodeConfig, budget_s: float = 15.0):
 def run_reference(args, world, rank):
     if rank != 0:
         return
+    if args.config in ENCODE_CONFIGS:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the reference arm times the decode workloads only"}), flush=True)
+        return
     cfg = synth.DECODE_CONFIGS[args.config]
     per_step = []
     for _ in range(args.warmup):
@@ -353,7 +483,7 @@ def run_lla(args, world, rank, local):
     ev[0].record(stream)
     for k in range(args.steps):
         if k == args.steps - 1:
-            # time each call of the last step's first loop on its own
+            # time each whole call of the last step's first loop on its own
             c = cfg
             for t in range(c.T):
                 for l in range(c.L):
@@ -377,11 +507,22 @@ def run_lla(args, world, rank, local):
     call_ms = sorted(a.elapsed_time(b) for a, b in call_ev)
     call_ms_mean = sum(call_ms) / len(call_ms)
 
+    # the main kernel alone, timed with CUDA events that the library records
+    # on the call's stream right around that kernel (one call per layer)
+    kern_ms = []
+    for l in range(cfg.L):
+        with wl.lla.kernel_timer() as kt:
+            wl.fn(wl.q[l, 0], wl.zk[l], wl.zv[l], wl.dk[l, 0], wl.dv[l, 0], N=cfg.N,
+                  scale=wl.scale, out=wl.out[l, 0], lse=wl.lse[l, 0], workspace=wl.ws)
+        kern_ms.append(kt.ms)
+    kern_ms_mean = sum(kern_ms) / len(kern_ms)
+
     tokens_per_step = cfg.B * cfg.N * cfg.L * cfg.T
     value = world * tokens_per_step / (ms_per_step * 1e-3)
     step_bytes = cfg.step_bytes()
     hbm_peak, peak_src = peaks()
-    achieved = step_bytes / (call_ms_mean * 1e-3) / 1e9
+    achieved = step_bytes / (kern_ms_mean * 1e-3) / 1e9
+    kname, _ = main_kernel(cfg.name)
 
     # end to end through the public API: queries from pinned host memory in,
     # outputs back to pinned host memory, every step
@@ -434,14 +575,14 @@ def run_lla(args, world, rank, local):
             "parallelism": f"dp{world} (independent sequences per GPU)",
             "global_batch": cfg.B * world, "seq_len": cfg.N,
         },
-        "hbm_gbs_per_call": achieved,
+        "hbm_gbs_per_call": step_bytes / (call_ms_mean * 1e-3) / 1e9,
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": profiled_traffic(cfg.name),
-            "kernel": "k_stream (timed as the whole decode call incl. absorb and combine)",
+            "kernel": kname, "kernel_ms_mean": kern_ms_mean,
             "algorithmic_bytes_per_launch": step_bytes,
-            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-            else "fallback 6.65 TB/s",
+            "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs (copy, burst)"
+            if peak_src == "measured" else "fallback 6.65 TB/s",
         },
         "call_ms": {"mean": call_ms_mean, "min": call_ms[0], "max": call_ms[-1]},
         "gpu_launches": wl.launches_per_step() * args.steps,
@@ -464,7 +605,10 @@ def main():
         return
     world, rank, local = dist_setup(args)
     try:
-        run_lla(args, world, rank, local)
+        if args.config in ENCODE_CONFIGS:
+            run_encode_bench(args, world, rank, local)
+        else:
+            run_lla(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

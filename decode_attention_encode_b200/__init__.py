@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     EXPORTS,
     LLAError,
     device_status,
+    kernel_timer,
     lib,
     library_path,
     lla2d_decode_attn,

@@ -31,6 +31,7 @@ LLA_DEVICE_WAIT_TIMEOUT = 0x1
 # Every symbol include/lla.h declares.
 EXPORTS = (
     "lla_status_string", "lla_last_error", "lla_version", "lla_device_status",
+    "lla_set_timing_events",
     "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn",
     "lla_encode",
@@ -54,6 +55,7 @@ _SIGS = {
     "lla_last_error": ([], ctypes.c_char_p),
     "lla_version": ([], _c_int),
     "lla_device_status": ([ctypes.POINTER(ctypes.c_uint), _c_int], _c_int),
+    "lla_set_timing_events": ([_vp, _vp], None),
     "lla_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
@@ -122,6 +124,28 @@ def device_status(clear: bool = False) -> int:
     v = ctypes.c_uint(0)
     _check(lib().lla_device_status(ctypes.byref(v), int(clear)))
     return v.value
+
+
+class kernel_timer:
+    """Context manager that times the main kernel of each library call made
+    inside it with CUDA events (lla_set_timing_events). After the block,
+    `ms` is the elapsed time of the last timed call's main kernel."""
+
+    def __init__(self):
+        self.begin = torch.cuda.Event(enable_timing=True)
+        self.end = torch.cuda.Event(enable_timing=True)
+        self.ms = None
+
+    def __enter__(self):
+        lib().lla_set_timing_events(ctypes.c_void_p(self.begin.cuda_event),
+                                    ctypes.c_void_p(self.end.cuda_event))
+        return self
+
+    def __exit__(self, *exc):
+        lib().lla_set_timing_events(None, None)
+        self.end.synchronize()
+        self.ms = self.begin.elapsed_time(self.end)
+        return False
 
 
 def lla_decode_attn_workspace(B, H, N, r_k, r_v) -> int:

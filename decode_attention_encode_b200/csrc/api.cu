@@ -19,6 +19,8 @@ constexpr int kMaxDevices = 64;
 __device__ unsigned int g_status_word = 0u;
 
 thread_local char g_last_error[512] = "";
+thread_local cudaEvent_t g_ev_begin = nullptr;
+thread_local cudaEvent_t g_ev_end = nullptr;
 
 std::mutex g_dev_mutex;
 bool g_dev_ready[kMaxDevices];
@@ -71,6 +73,16 @@ unsigned int* status_word() {
   std::lock_guard<std::mutex> g(g_dev_mutex);
   init_device(dev);
   return g_status_ptr[dev];
+}
+
+void timing_events(cudaEvent_t* begin, cudaEvent_t* end) {
+  *begin = g_ev_begin;
+  *end = g_ev_end;
+}
+
+cudaError_t record_timing(bool begin, cudaStream_t stream) {
+  if (!g_ev_begin || !g_ev_end) return cudaSuccess;
+  return cudaEventRecord(begin ? g_ev_begin : g_ev_end, stream);
 }
 
 lla_status fail(lla_status s, const char* fmt, ...) {
@@ -136,6 +148,11 @@ const char* lla_status_string(lla_status s) {
 const char* lla_last_error(void) { return g_last_error; }
 
 int lla_version(void) { return 100; }
+
+void lla_set_timing_events(void* ev_begin, void* ev_end) {
+  g_ev_begin = static_cast<cudaEvent_t>(ev_begin);
+  g_ev_end = static_cast<cudaEvent_t>(ev_end);
+}
 
 lla_status lla_device_status(unsigned int* status, int clear) {
   if (!status) return fail(LLA_ERR_INVALID_ARG, "status must be non-NULL");

@@ -28,19 +28,13 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "stream.cuh"
 
 namespace lla {
 namespace {
 
-constexpr float kLn2 = 0.69314718055994531f;
-constexpr float kLog2e = 1.44269504088896341f;
-constexpr float kNegBig = -1.0e30f;
-// Lazy rescaling: a slot keeps its reference maximum until a score exceeds
-// it by this much (log2 units), so p_j <= 2^8 and rescales are rare.
-constexpr float kRescaleSlack = 8.0f;
-
-constexpr int kAbsorbRows = 8;    // batch rows (one per warp) per k_absorb CTA
-constexpr int kCombineRows = 8;   // batch rows (one per warp) per k_combine CTA
+constexpr int kAbsorbRows = 64;   // batch rows per k_absorb CTA (8 per warp)
+constexpr int kCombineRows = 32;  // batch rows per k_combine CTA (4 per warp)
 constexpr int kColChunk = 32;     // decoder columns (absorb) / rows (combine) per CTA
 
 // ---------------------------------------------------------------------------
@@ -51,31 +45,35 @@ struct AbsorbArgs {
   const float* dk;
   const float* mu_k;
   int B, H, d_h, r_k;
+  int rows;  // batch rows per CTA: 8, 16, 32 or 64
   float qscale;  // scale * log2(e): scores leave k_stream in log2 units
   float scale;
   float* qp;  // [B*H][r_k]
   float* c0;  // [B*H], natural-log units
 };
 
-// One CTA per (head, 8 batch rows, 32 latent columns): the CTA stages its
-// d_h x 32 slice of W^K_up,t and the 8 query rows in shared memory, and each
-// thread forms one q'[b][c] as a d_h-long dot product.
+// One CTA per (head, `rows` batch rows, 32 latent columns). The CTA stages
+// the d_h x 32 slice of W^K_up,t once and its query rows in shared memory;
+// thread (warp w, lane l) forms q'[b][c0 + l] for the rows b = w + 8k, so
+// each decoder value read from shared memory feeds rows/8 FMAs. `rows` is
+// chosen on the host so the grid stays near 512-1024 CTAs.
 __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
-  __shared__ float q_s[kAbsorbRows * 256];
-  __shared__ __align__(16) float d_s[256 * kColChunk];
+  extern __shared__ __align__(16) float sm_absorb[];
+  float* q_s = sm_absorb;                        // [rows][d_h4]
+  const int d_h4 = (a.d_h + 3) & ~3;             // rows padded to float4
+  float* d_s = sm_absorb + a.rows * d_h4;        // [d_h][kColChunk]
   pdl_launch_dependents();
   const int h = blockIdx.x;
-  const int b0 = blockIdx.y * kAbsorbRows;
+  const int b0 = blockIdx.y * a.rows;
   const int c0 = blockIdx.z * kColChunk;
-  const int nb = min(kAbsorbRows, a.B - b0);
+  const int nb = min(a.rows, a.B - b0);
   const int nc = min(kColChunk, a.r_k - c0);
-  for (int idx = threadIdx.x; idx < nb * a.d_h; idx += blockDim.x) {
-    const int bb = idx / a.d_h, i = idx - bb * a.d_h;
-    q_s[idx] = a.q[((size_t)(b0 + bb) * a.H + h) * a.d_h + i];
+  for (int idx = threadIdx.x; idx < nb * d_h4; idx += blockDim.x) {
+    const int bb = idx / d_h4, i = idx - bb * d_h4;
+    q_s[idx] = i < a.d_h ? a.q[((size_t)(b0 + bb) * a.H + h) * a.d_h + i] : 0.f;
   }
-  // W^K rows i, columns [c0, c0 + nc): nc is a multiple of 8, so float4 loads
   const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
-  const int n4 = nc / 4;
+  const int n4 = nc / 4;  // nc is a multiple of 8
   for (int idx = threadIdx.x; idx < a.d_h * n4; idx += blockDim.x) {
     const int i = idx / n4, j = idx - i * n4;
     reinterpret_cast<float4*>(d_s + i * kColChunk)[j] =
@@ -86,302 +84,38 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.z == 0) {
     // c0 = scale * q . mu_k (natural-log units), one warp per row
-    for (int bb = warp; bb < nb; bb += blockDim.x >> 5) {
+    for (int bb = warp; bb < nb; bb += 8) {
       float acc = 0.f;
       if (a.mu_k)
         for (int i = lane; i < a.d_h; i += 32)
-          acc += q_s[bb * a.d_h + i] * a.mu_k[(size_t)h * a.d_h + i];
+          acc += q_s[bb * d_h4 + i] * a.mu_k[(size_t)h * a.d_h + i];
       acc = warp_sum(acc);
       if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
     }
   }
-  // thread -> (row bb = warp, column c0 + lane)
-  const int bb = warp;
-  if (bb < nb && lane < nc) {
-    const float* qrow = q_s + bb * a.d_h;
-    float s0 = 0.f, s1 = 0.f;
-    int i = 0;
-    for (; i + 1 < a.d_h; i += 2) {
-      s0 = fmaf(d_s[i * kColChunk + lane], qrow[i], s0);
-      s1 = fmaf(d_s[(i + 1) * kColChunk + lane], qrow[i + 1], s1);
-    }
-    if (i < a.d_h) s0 = fmaf(d_s[i * kColChunk + lane], qrow[i], s0);
-    a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = (s0 + s1) * a.qscale;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// k_stream
-// ---------------------------------------------------------------------------
-struct StreamArgs {
-  const char* zk;
-  const char* zv;
-  long long n_cap;
-  long long N;
-  long long total;  // units * N
-  long long P;      // tokens per warp
-  int W;            // streaming warps
-  int row_k, row_v;  // bytes per latent row
-  int nseg_k, nseg_v;
-  int r_k;  // elements (q' row stride)
-  int tile, nstage, stage_bytes;
-  const float* qp;
-  float* part;
-  int pstride;
-  unsigned int* status;
-};
-
-template <int ESZ>
-__device__ __forceinline__ void unpack16(const uint4& v, float* f);
-template <>
-__device__ __forceinline__ void unpack16<2>(const uint4& v, float* f) {
-  f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-  f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
-}
-template <>
-__device__ __forceinline__ void unpack16<4>(const uint4& v, float* f) {
-  f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
-  f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
-}
-
-// Loads q' of unit u (this lane's segments) into registers.
-template <int E, int LPT, int SK, bool EXACT>
-__device__ __forceinline__ void load_qp(float (&qv)[SK][E], const float* qp, long long u, int r_k,
-                                        int nseg_k, int g) {
+  constexpr int kPer = kAbsorbRows / 8;
+  float acc[kPer];
 #pragma unroll
-  for (int s = 0; s < SK; ++s) {
-    const int seg = s * LPT + g;
-    if (EXACT || seg < nseg_k) {
-      const float4* src = reinterpret_cast<const float4*>(qp + u * r_k + seg * E);
+  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+  if (lane < nc) {
+    for (int i = 0; i < a.d_h; i += 4) {
+      float dv[4];
 #pragma unroll
-      for (int e4 = 0; e4 < E / 4; ++e4) {
-        const float4 t = src[e4];
-        qv[s][4 * e4 + 0] = t.x;
-        qv[s][4 * e4 + 1] = t.y;
-        qv[s][4 * e4 + 2] = t.z;
-        qv[s][4 * e4 + 3] = t.w;
-      }
-    } else {
+      for (int e = 0; e < 4; ++e) dv[e] = (i + e < a.d_h) ? d_s[(i + e) * kColChunk + lane] : 0.f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) qv[s][e] = 0.f;
-    }
-  }
-}
-
-// One token slot's online-softmax update with score sc (log2 units) and
-// value row v.
-template <int ESZ, int LPT, int SV, bool EXACT>
-__device__ __forceinline__ void slot_update(float sc, const unsigned char* vrow, float& m, float& l,
-                                            float (&acc)[SV][16 / ESZ], int nseg_v, int g) {
-  constexpr int E = 16 / ESZ;
-  if (sc > m + kRescaleSlack) {
-    const float alpha = exp2f(m - sc);
-    l *= alpha;
-#pragma unroll
-    for (int s = 0; s < SV; ++s)
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[s][e] *= alpha;
-    m = sc;
-  }
-  const float p = exp2f(sc - m);
-  l += p;
-#pragma unroll
-  for (int s = 0; s < SV; ++s) {
-    const int seg = s * LPT + g;
-    if (EXACT || seg < nseg_v) {
-      float x[E];
-      unpack16<ESZ>(*reinterpret_cast<const uint4*>(vrow + seg * 16), x);
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[s][e] = fmaf(p, x[e], acc[s][e]);
-    }
-  }
-}
-
-// ESZ: bytes per latent element. LPT: lanes per token. SK/SV: 16-byte
-// segments per lane for K/V. EXACT: nseg == LPT*S for both axes.
-template <int ESZ, int LPT, int SK, int SV, bool EXACT>
-__global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
-  constexpr int E = 16 / ESZ;   // elements per 16-byte segment
-  constexpr int NS = 32 / LPT;  // token slots per warp
-  constexpr unsigned FULL = 0xffffffffu;
-  extern __shared__ __align__(128) unsigned char smem[];
-
-  pdl_launch_dependents();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  const long long w = (long long)blockIdx.x * nwarps + warp;
-  if (w >= a.W) return;
-  const int slot = lane / LPT, g = lane - slot * LPT;
-
-  const int bar_bytes = ((nwarps * a.nstage * 8) + 127) & ~127;
-  const uint32_t bar0 = smem_u32(smem) + warp * a.nstage * 8;
-  unsigned char* buf = smem + bar_bytes + (size_t)warp * a.nstage * a.stage_bytes;
-  const uint32_t buf0 = smem_u32(buf);
-  const int v_off = a.tile * a.row_k;  // V part of a stage follows K
-
-  if (lane == 0) {
-    for (int s = 0; s < a.nstage; ++s) mbar_init(bar0 + 8 * s, 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-
-  const long long f0 = w * a.P;
-  const long long f1 = min(f0 + a.P, a.total);
-  const uint64_t pol = l2_evict_first_policy();
-
-  // Producer side (lane 0 issues): the tile sequence is the range [f0, f1)
-  // cut at unit boundaries and at `tile` tokens; (pu, pj) is the unit and
-  // token of the next tile to load, ps its stage.
-  long long pf = f0, pu = f0 / a.N, pj = f0 - pu * a.N;
-  int ps = 0, in_flight = 0;
-  auto issue = [&]() {
-    const int len = (int)min((long long)a.tile, min(f1 - pf, a.N - pj));
-    if (lane == 0) {
-      const uint32_t kb = (uint32_t)len * a.row_k, vb = (uint32_t)len * a.row_v;
-      const uint32_t bar = bar0 + 8 * ps;
-      const long long row = pu * a.n_cap + pj;
-      const uint32_t dst = buf0 + ps * a.stage_bytes;
-      mbar_arrive_expect_tx(bar, kb + vb);
-      bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
-      bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
-    }
-    pf += len;
-    pj += len;
-    if (pj == a.N) {
-      pj = 0;
-      ++pu;
-    }
-    if (++ps == a.nstage) ps = 0;
-    ++in_flight;
-  };
-  for (int s = 0; s < a.nstage && pf < f1; ++s) issue();
-
-  // q' is written by k_absorb.
-  pdl_wait();
-
-  int cs = 0;          // stage being consumed
-  uint32_t cpar = 0;   // its phase parity
-  long long f = f0;
-  long long u = f0 / a.N;
-  const long long u_last = (f1 - 1) / a.N;
-  float qv[SK][E], qn[SK][E];
-  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g);
-  while (f < f1) {
-    const long long seg_end = min(f1, (u + 1) * a.N);
-    // the next unit's q' loads run under this unit's stream
-    if (u < u_last) load_qp<E, LPT, SK, EXACT>(qn, a.qp, u + 1, a.r_k, a.nseg_k, g);
-    float m = kNegBig, l = 0.f;
-    float acc[SV][E];
-#pragma unroll
-    for (int s = 0; s < SV; ++s)
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[s][e] = 0.f;
-
-    while (f < seg_end) {
-      const int len = (int)min((long long)a.tile, seg_end - f);
-      const bool ok = __all_sync(FULL, mbar_wait(bar0 + 8 * cs, cpar));
-      if (!ok) {
-        if (lane == 0) report_status(a.status, kStatusWaitTimeout);
-        int st = cs;
-        uint32_t par = cpar;
-        for (int i = 0; i < in_flight; ++i) {
-          (void)mbar_wait(bar0 + 8 * st, par, kWaitTimeoutNs / 8);
-          if (++st == a.nstage) {
-            st = 0;
-            par ^= 1u;
-          }
-        }
-        return;
-      }
-      const unsigned char* Ks = buf + cs * a.stage_bytes;
-      const unsigned char* Vs = Ks + v_off;
-
-      for (int t0 = 0; t0 < len; t0 += 2 * NS) {
-        const int ta = t0 + slot, tb = t0 + NS + slot;
-        const bool va = ta < len, vb = tb < len;
-        float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-#pragma unroll
-        for (int s = 0; s < SK; ++s) {
-          const int seg = s * LPT + g;
-          if (EXACT || seg < a.nseg_k) {
-            float x[E];
-            if (va) {
-              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + ta * a.row_k + seg * 16), x);
-#pragma unroll
-              for (int e = 0; e < E; e += 2) {
-                sa0 = fmaf(qv[s][e], x[e], sa0);
-                sa1 = fmaf(qv[s][e + 1], x[e + 1], sa1);
-              }
-            }
-            if (vb) {
-              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + tb * a.row_k + seg * 16), x);
-#pragma unroll
-              for (int e = 0; e < E; e += 2) {
-                sb0 = fmaf(qv[s][e], x[e], sb0);
-                sb1 = fmaf(qv[s][e + 1], x[e + 1], sb1);
-              }
-            }
-          }
-        }
-        float sa = sa0 + sa1, sb = sb0 + sb1;
-#pragma unroll
-        for (int o = LPT / 2; o > 0; o >>= 1) {
-          sa += __shfl_xor_sync(FULL, sa, o);
-          sb += __shfl_xor_sync(FULL, sb, o);
-        }
-        if (va) slot_update<ESZ, LPT, SV, EXACT>(sa, Vs + ta * a.row_v, m, l, acc, a.nseg_v, g);
-        if (vb) slot_update<ESZ, LPT, SV, EXACT>(sb, Vs + tb * a.row_v, m, l, acc, a.nseg_v, g);
-      }
-      __syncwarp();
-      --in_flight;
-      if (pf < f1) issue();  // refill the stage just read
-      if (++cs == a.nstage) {
-        cs = 0;
-        cpar ^= 1u;
-      }
-      f += len;
-    }
-
-    // Merge the NS token slots of this warp (log-sum-exp butterfly).
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) {
-      const float mo = __shfl_xor_sync(FULL, m, o);
-      const float lo = __shfl_xor_sync(FULL, l, o);
-      const float M = fmaxf(m, mo);
-      const float wa = exp2f(m - M), wb = exp2f(mo - M);
-      l = l * wa + lo * wb;
-#pragma unroll
-      for (int s = 0; s < SV; ++s)
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const float ao = __shfl_xor_sync(FULL, acc[s][e], o);
-          acc[s][e] = acc[s][e] * wa + ao * wb;
-        }
-      m = M;
-    }
-    if (slot == 0) {
-      float* pp = a.part + (size_t)(w + u) * a.pstride;
-      if (g == 0) {
-        pp[0] = m;
-        pp[1] = l;
-      }
-#pragma unroll
-      for (int s = 0; s < SV; ++s) {
-        const int seg = s * LPT + g;
-        if (EXACT || seg < a.nseg_v) {
-          float4* dst = reinterpret_cast<float4*>(pp + 4 + seg * E);
-#pragma unroll
-          for (int e4 = 0; e4 < E / 4; ++e4)
-            dst[e4] = make_float4(acc[s][4 * e4], acc[s][4 * e4 + 1], acc[s][4 * e4 + 2],
-                                  acc[s][4 * e4 + 3]);
+      for (int k = 0; k < kPer; ++k) {
+        const int bb = warp + 8 * k;
+        if (bb < nb) {
+          const float4 qv = *reinterpret_cast<const float4*>(q_s + bb * d_h4 + i);
+          acc[k] = fmaf(dv[0], qv.x, fmaf(dv[1], qv.y, fmaf(dv[2], qv.z, fmaf(dv[3], qv.w, acc[k]))));
         }
       }
     }
-    ++u;
 #pragma unroll
-    for (int s = 0; s < SK; ++s)
-#pragma unroll
-      for (int e = 0; e < E; ++e) qv[s][e] = qn[s][e];
+    for (int k = 0; k < kPer; ++k) {
+      const int bb = warp + 8 * k;
+      if (bb < nb) a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = acc[k] * a.qscale;
+    }
   }
 }
 
@@ -397,34 +131,37 @@ struct CombineArgs {
   int B, H, d_h, r_v;
   long long N, P;  // per-sequence and per-piece extents of the split
   int shared;      // 1: one split per sequence shared by all heads (LLA-2D)
+  int rows;        // batch rows per CTA: 8, 16 or 32
   float* out;
   float* lse;
 };
 
-// One CTA per (head, 8 batch rows, 32 output channels): warp w merges the
-// partial records of row w (lanes across the latent index) into ubar, the
-// CTA stages its 32 x r_v slice of W^V_up,t (rows padded by one float so
-// consecutive rows fall in distinct banks), and each thread forms one
-// out[b][h][i] as an r_v-long dot product.
+// One CTA per (head, `rows` batch rows, 32 output channels). Warp w merges
+// the partial records of rows w, w+8, ... into ubar (lanes across the latent
+// index); the CTA stages the 32 x r_v slice of W^V_up,t once (rows padded by
+// 4 floats, so float4 reads of 8 consecutive rows hit 8 distinct bank
+// groups); thread (warp w, lane l) forms out[b][h][i0 + l] for its rows.
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
-  __shared__ float ub[kCombineRows * 256];
-  __shared__ float d_s[kColChunk * 257];
+  extern __shared__ __align__(16) float sm_combine[];
+  const int pitch = a.r_v + 4;
+  float* ub = sm_combine;                         // [rows][r_v]
+  float* d_s = sm_combine + a.rows * a.r_v;       // [kColChunk][pitch]
   const int h = blockIdx.x;
-  const int b0 = blockIdx.y * kCombineRows;
+  const int b0 = blockIdx.y * a.rows;
   const int i0 = blockIdx.z * kColChunk;
-  const int nb = min(kCombineRows, a.B - b0);
+  const int nb = min(a.rows, a.B - b0);
   const int ni = min(kColChunk, a.d_h - i0);
-  const int pitch = a.r_v + 1;
   // W^V does not depend on the streaming kernel: stage it before waiting
   const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
-  for (int idx = threadIdx.x; idx < ni * a.r_v; idx += blockDim.x) {
-    const int i = idx / a.r_v, c = idx - i * a.r_v;
-    d_s[i * pitch + c] = __ldg(D + idx);
+  const int r4 = a.r_v / 4;
+  for (int idx = threadIdx.x; idx < ni * r4; idx += blockDim.x) {
+    const int i = idx / r4, j = idx - i * r4;
+    reinterpret_cast<float4*>(d_s + i * pitch)[j] =
+        __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j);
   }
   pdl_wait();  // partials come from the streaming kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bb = warp;
-  if (bb < nb) {
+  for (int bb = warp; bb < nb; bb += 8) {
     const long long u = (long long)(b0 + bb) * a.H + h;
     // The split runs over units (b, h) for per-head LLA and over sequences
     // b for LLA-2D; piece w of split key k is partial record w + k.
@@ -457,46 +194,35 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     if (blockIdx.z == 0 && lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
   }
   __syncthreads();
-  // thread -> (row bb = warp, output channel i0 + lane)
-  if (bb < nb && lane < ni) {
+  if (lane < ni) {
+    constexpr int kPer = kCombineRows / 8;
+    float acc[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
     const float* drow = d_s + lane * pitch;
-    const float* urow = ub + bb * a.r_v;
-    float s0 = 0.f, s1 = 0.f;
-    for (int c = 0; c < a.r_v; c += 2) {
-      s0 = fmaf(drow[c], urow[c], s0);
-      s1 = fmaf(drow[c + 1], urow[c + 1], s1);
+    for (int c = 0; c < a.r_v; c += 4) {
+      const float4 dv = *reinterpret_cast<const float4*>(drow + c);
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int bb = warp + 8 * k;
+        if (bb < nb) {
+          const float4 uv = *reinterpret_cast<const float4*>(ub + bb * a.r_v + c);
+          acc[k] = fmaf(dv.x, uv.x, fmaf(dv.y, uv.y, fmaf(dv.z, uv.z, fmaf(dv.w, uv.w, acc[k]))));
+        }
+      }
     }
     const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + lane] : 0.f;
-    a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = s0 + s1 + mu;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int bb = warp + 8 * k;
+      if (bb < nb) a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = acc[k] + mu;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-using StreamFn = void (*)(StreamArgs);
-
-template <int ESZ>
-StreamFn pick_stream(int lpt, int s, bool exact) {
-  if (!exact) {
-    switch (lpt) {
-      case 1: return k_stream<ESZ, 1, 4, 4, false>;
-      case 2: return k_stream<ESZ, 2, 4, 4, false>;
-      case 4: return k_stream<ESZ, 4, 4, 4, false>;
-      case 8: return k_stream<ESZ, 8, 4, 4, false>;
-    }
-    return nullptr;
-  }
-#define LLA_CASE(L, S) \
-  if (lpt == L && s == S) return k_stream<ESZ, L, S, S, true>;
-  LLA_CASE(1, 1) LLA_CASE(1, 2) LLA_CASE(1, 3) LLA_CASE(1, 4)
-  LLA_CASE(2, 1) LLA_CASE(2, 2) LLA_CASE(2, 3) LLA_CASE(2, 4)
-  LLA_CASE(4, 1) LLA_CASE(4, 2) LLA_CASE(4, 3) LLA_CASE(4, 4)
-  LLA_CASE(8, 1) LLA_CASE(8, 2) LLA_CASE(8, 3) LLA_CASE(8, 4)
-#undef LLA_CASE
-  return nullptr;
-}
-
 bool exact_variant(int lpt, int s) { return lpt >= 1 && lpt <= 8 && s >= 1 && s <= 4; }
 
 int env_int(const char* name, int dflt) {
@@ -511,9 +237,16 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream) {
-  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0};
-  dim3 grid(H, (B + kAbsorbRows - 1) / kAbsorbRows, (r_k + kColChunk - 1) / kColChunk);
-  k_absorb<<<grid, 256, 0, stream>>>(a);
+  const int zc = (r_k + kColChunk - 1) / kColChunk;
+  int rows = 8;
+  while (rows < kAbsorbRows && (long long)H * zc * ((B + rows - 1) / rows) > 1024) rows *= 2;
+  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, rows, scale * kLog2e, scale, qp, c0};
+  dim3 grid(H, (B + rows - 1) / rows, zc);
+  const size_t smem = ((size_t)rows * ((d_h + 3) & ~3) + (size_t)d_h * kColChunk) * 4;
+  cudaError_t e = cudaFuncSetAttribute(k_absorb, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_absorb)");
+  k_absorb<<<grid, 256, smem, stream>>>(a);
   return check_cuda(cudaGetLastError(), "launch k_absorb");
 }
 
@@ -523,11 +256,17 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse};
+  const int zc = (d_h + kColChunk - 1) / kColChunk;
+  int rows = 8;
+  while (rows < kCombineRows && (long long)H * zc * ((B + rows - 1) / rows) > 1024) rows *= 2;
+  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, rows, out, lse};
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(H, (B + kCombineRows - 1) / kCombineRows, (d_h + kColChunk - 1) / kColChunk);
+  cfg.gridDim = dim3(H, (B + rows - 1) / rows, zc);
   cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = ((size_t)rows * r_v + (size_t)kColChunk * (r_v + 4)) * 4;
+  cudaError_t e = cudaFuncSetAttribute(k_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)cfg.dynamicSmemBytes);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_combine)");
   cfg.stream = stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
@@ -620,7 +359,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
 
-  StreamFn fn = (esz == 2) ? pick_stream<2>(d.lpt, d.sk, d.exact) : pick_stream<4>(d.lpt, d.sk, d.exact);
+  StreamFn fn = pick_stream_kernel(esz, d.lpt, d.sk, d.exact);
   if (!fn) return fail(LLA_ERR_UNSUPPORTED, "no decode kernel for this latent shape");
 
   cudaError_t e;
@@ -662,8 +401,12 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
     cfg.stream = stream;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
+    e = record_timing(true, stream);
+    if (e != cudaSuccess) return check_cuda(e, "record timing event");
     e = cudaLaunchKernelEx(&cfg, fn, a);
     if (e != cudaSuccess) return check_cuda(e, "launch k_stream");
+    e = record_timing(false, stream);
+    if (e != cudaSuccess) return check_cuda(e, "record timing event");
   }
   // 3. combine
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, N, d.P, 0, out, lse, stream);

@@ -361,9 +361,13 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   cudaError_t e = cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_encode)");
+  e = record_timing(true, stream);
+  if (e != cudaSuccess) return check_cuda(e, "record timing event");
   k_encode<<<grid, kThreads, smem, stream>>>(tx, tw, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return check_cuda(e, "launch k_encode");
+  e = record_timing(false, stream);
+  if (e != cudaSuccess) return check_cuda(e, "record timing event");
   return LLA_OK;
 }
 

@@ -25,6 +25,11 @@ unsigned int* status_word();
 // Records a one-line reason for the calling thread and returns `s`.
 lla_status fail(lla_status s, const char* fmt, ...);
 
+// Timing hook events of the calling thread (lla_set_timing_events).
+void timing_events(cudaEvent_t* begin, cudaEvent_t* end);
+// Records the hook's begin (or end) event on `stream` if a hook is set.
+cudaError_t record_timing(bool begin, cudaStream_t stream);
+
 // Maps a CUDA error to LLA_ERR_CUDA with its message, or LLA_OK.
 lla_status check_cuda(cudaError_t e, const char* what);
 

@@ -21,14 +21,18 @@
 // ends in one partial record per head (m, l, U); k_combine merges them and
 // applies W^V_up,t. k_absorb (shared with the per-head path) forms q'.
 //
-// CTA roles (6 warps):
-//   warp 0     TMA producer: 128 x 128-column latent groups (two 64-column
-//              128B-swizzled boxes, 32 KB) into a ring of stages; stages Q'
-//              (bf16, swizzled K-major) for each new sequence.
+// CTA roles (7 warps):
+//   warp 0     K producer: 128 x 128-column Z^K groups (two 64-column
+//              128B-swizzled boxes, 32 KB) into the K ring; stages Q' (bf16,
+//              swizzled K-major) for each new sequence.
 //   warp 1     TMEM owner and MMA issuer. Issues the score MMA of tile i+1
 //              before the value MMA of tile i so the softmax of tile i
 //              overlaps the next score MMA.
 //   warps 2-5  softmax and epilogue (one thread per TMEM lane).
+//   warp 6     V producer: Z^V groups into the V ring.
+// K and V have separate rings, so a K slot is reused as soon as its score
+// MMA retires and the K stream runs up to two tiles ahead of the value
+// MMAs, which wait on the softmax.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -42,14 +46,20 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kBoxBytes = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int kStageBytes = 2 * kBoxBytes;
-constexpr int kThreads = 192;
-constexpr int kMaxStages = 8;
+constexpr int kThreads = 224;
+constexpr int kMaxStages = 4;  // per ring
 constexpr float kNegBig = -1.0e30f;
 constexpr float kSlack = 8.0f;
+// Each contraction is split over independent TMEM accumulators whose MMAs
+// are issued interleaved: with N = 16 a single accumulator serialises the
+// small MMAs on its own read-modify-write. The partial sums are added when
+// read back.
+constexpr int kSAcc = 4;  // score accumulators per S buffer
+constexpr int kUAcc = 2;  // value accumulators per r_v half
 
 struct D2Args {
   int B, H, N, tps, tiles, tpc;
-  int r_k, r_v, nkg, nvg, spt, nstage;
+  int r_k, r_v, nkg, nvg, nks, nvs;  // groups per tile; stages per ring
   int off_q, off_p, off_tail, qbuf_bytes, pbuf_bytes;
   uint32_t tmem_cols;
   const float* qp;
@@ -59,8 +69,8 @@ struct D2Args {
 };
 
 struct Tail2 {
-  uint64_t full[kMaxStages];
-  uint64_t empty[kMaxStages];
+  uint64_t kfull[kMaxStages], kempty[kMaxStages];
+  uint64_t vfull[kMaxStages], vempty[kMaxStages];
   uint64_t s_full[2], s_empty[2], p_full[2], u_done[2], q_full[2], q_empty[2];
   uint64_t epi;    // 4-warp rendezvous of the softmax warps
   uint64_t drain;
@@ -116,7 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Tail2* tl = reinterpret_cast<Tail2*>(smem + a.off_tail);
   volatile int* abort_flag = &tl->abort_flag;
-  const uint32_t s_stage0 = smem_u32(smem);
+  const uint32_t s_kring = smem_u32(smem);
+  const uint32_t s_vring = s_kring + (uint32_t)a.nks * kStageBytes;
   const uint32_t s_q0 = smem_u32(smem + a.off_q);
   const uint32_t s_p0 = smem_u32(smem + a.off_p);
 
@@ -126,9 +137,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntile = t_end - t_begin;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < a.nstage; ++s) {
-      mbar_init(smem_u32(&tl->full[s]), 1);
-      mbar_init(smem_u32(&tl->empty[s]), 1);
+    for (int s = 0; s < a.nks; ++s) {
+      mbar_init(smem_u32(&tl->kfull[s]), 1);
+      mbar_init(smem_u32(&tl->kempty[s]), 1);
+    }
+    for (int s = 0; s < a.nvs; ++s) {
+      mbar_init(smem_u32(&tl->vfull[s]), 1);
+      mbar_init(smem_u32(&tl->vempty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&tl->s_full[i]), 1);
@@ -152,33 +167,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto seq_of = [&](int lt) { return (t_begin + lt) / a.tps; };
   auto kboxes = [&](int kg) { return min(2, (a.r_k - kg * 128) / 64); };
 
-  if (warp == 0) {
-    // ------------------------------ producer ------------------------------
+  if (warp == 0 || warp == 6) {
+    // ------------------------------ producers ------------------------------
+    // warp 0 streams Z^K groups (and stages Q'), warp 6 streams Z^V groups.
+    const bool is_k = warp == 0;
     const uint64_t pol = l2_evict_first_policy();
-    const int total = ntile * a.spt;
+    const int ng = is_k ? a.nkg : a.nvg;
+    const int nring = is_k ? a.nks : a.nvs;
+    const uint32_t ring = is_k ? s_kring : s_vring;
+    uint64_t* fullb = is_k ? tl->kfull : tl->vfull;
+    uint64_t* emptyb = is_k ? tl->kempty : tl->vempty;
+    const CUtensorMap* map = is_k ? &tk : &tv;
+    const int total = ntile * ng;
     auto issue = [&](int it) -> bool {
-      const int s = it % a.nstage;
-      const uint32_t ph = (uint32_t)(it / a.nstage) & 1u;
+      const int s = it % nring;
+      const uint32_t ph = (uint32_t)(it / nring) & 1u;
       const bool ok = __all_sync(0xffffffffu,
-                                 wait_ab(smem_u32(&tl->empty[s]), ph ^ 1u, abort_flag, a.status));
+                                 wait_ab(smem_u32(&emptyb[s]), ph ^ 1u, abort_flag, a.status));
       if (!ok) return false;
       if (lane == 0) {
-        const int lt = it / a.spt, sub = it - lt * a.spt;
+        const int lt = it / ng, grp = it - lt * ng;
         const int tile = t_begin + lt;
         const int b = tile / a.tps, row0 = (tile - b * a.tps) * kRows;
-        const uint32_t full = smem_u32(&tl->full[s]);
-        const uint32_t dst = s_stage0 + (uint32_t)s * kStageBytes;
-        if (sub < a.nkg) {
-          const int nb = kboxes(sub);
-          mbar_arrive_expect_tx(full, nb * kBoxBytes);
-          for (int x = 0; x < nb; ++x)
-            tma_load_3d(dst + x * kBoxBytes, &tk, sub * 128 + x * 64, row0, b, full, pol);
-        } else {
-          const int vg = sub - a.nkg;
-          mbar_arrive_expect_tx(full, 2 * kBoxBytes);
-          for (int x = 0; x < 2; ++x)
-            tma_load_3d(dst + x * kBoxBytes, &tv, vg * 128 + x * 64, row0, b, full, pol);
-        }
+        const uint32_t full = smem_u32(&fullb[s]);
+        const uint32_t dst = ring + (uint32_t)s * kStageBytes;
+        const int nb = is_k ? kboxes(grp) : 2;
+        mbar_arrive_expect_tx(full, nb * kBoxBytes);
+        for (int x = 0; x < nb; ++x)
+          tma_load_3d(dst + x * kBoxBytes, map, grp * 128 + x * 64, row0, b, full, pol);
       }
       return true;
     };
@@ -202,16 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     bool ok = true;
     int it = 0;
-    if (ntile > 0) {
+    if (!is_k) {
+      for (; ok && it < total; ++it) ok = issue(it);
+    } else if (ntile > 0) {
       const int b0 = seq_of(0);
       // latent loads of the first sequence do not depend on k_absorb
-      while (ok && it < total && it < a.nstage && seq_of(it / a.spt) == b0) ok = issue(it++);
+      while (ok && it < total && it < nring && seq_of(it / ng) == b0) ok = issue(it++);
       pdl_wait();
       if (ok) ok = stage_q(0, b0);
       int seg = 0, cur_b = b0;
       for (; ok && it < total; ++it) {
-        const int lt = it / a.spt;
-        if (it - lt * a.spt == 0 && seq_of(lt) != cur_b) {
+        const int lt = it / ng;
+        if (it - lt * ng == 0 && seq_of(lt) != cur_b) {
           cur_b = seq_of(lt);
           ok = stage_q(++seg, cur_b);
           if (!ok) break;
@@ -222,9 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       pdl_wait();
     }
     if (!ok && lane == 0) {
-      const int first = max(0, it - a.nstage);
+      const int first = max(0, it - nring);
       for (int i = first; i < it; ++i)
-        (void)mbar_wait(smem_u32(&tl->full[i % a.nstage]), (uint32_t)(i / a.nstage) & 1u,
+        (void)mbar_wait(smem_u32(&fullb[i % nring]), (uint32_t)(i / nring) & 1u,
                         kWaitTimeoutNs / 8);
     }
   } else if (warp == 1) {
@@ -239,25 +257,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                      a.status))
           return false;
         tc_fence_after();
-        const uint32_t d = tbase + (uint32_t)(sb * HP);
+        const uint32_t d0 = tbase + (uint32_t)(sb * kSAcc * HP);
         const uint32_t qaddr = s_q0 + (uint32_t)((seg & 1) * a.qbuf_bytes);
         for (int kg = 0; kg < a.nkg; ++kg) {
-          const int it = lt * a.spt + kg;
-          const int s = it % a.nstage;
-          if (!wait_ab(smem_u32(&tl->full[s]), (uint32_t)(it / a.nstage) & 1u, abort_flag,
+          const int it = lt * a.nkg + kg;
+          const int s = it % a.nks;
+          if (!wait_ab(smem_u32(&tl->kfull[s]), (uint32_t)(it / a.nks) & 1u, abort_flag,
                        a.status))
             return false;
           tc_fence_after();
           const int nb = kboxes(kg);
           for (int x = 0; x < nb; ++x) {
-            const uint32_t abox = s_stage0 + (uint32_t)s * kStageBytes + x * kBoxBytes;
+            const uint32_t abox = s_kring + (uint32_t)s * kStageBytes + x * kBoxBytes;
             const uint32_t bchunk = qaddr + (uint32_t)((kg * 2 + x) * HP * 128);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(d, desc_kmajor_sw128(abox + kk * 32), desc_kmajor_sw128(bchunk + kk * 32),
-                        idesc_s, (kg | x | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              const int kidx = (kg * 2 + x) * 4 + kk;  // K step within the tile
+              umma_bf16(d0 + (uint32_t)((kidx % kSAcc) * HP), desc_kmajor_sw128(abox + kk * 32),
+                        desc_kmajor_sw128(bchunk + kk * 32), idesc_s, kidx >= kSAcc);
+            }
           }
-          umma_commit(smem_u32(&tl->empty[s]));
+          umma_commit(smem_u32(&tl->kempty[s]));
         }
         umma_commit(smem_u32(&tl->s_full[sb]));
         return true;
@@ -284,21 +304,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           for (int vg = 0; vg < a.nvg && ok; ++vg) {
-            const int it = lt * a.spt + a.nkg + vg;
-            const int s = it % a.nstage;
-            ok = wait_ab(smem_u32(&tl->full[s]), (uint32_t)(it / a.nstage) & 1u, abort_flag,
+            const int it = lt * a.nvg + vg;
+            const int s = it % a.nvs;
+            ok = wait_ab(smem_u32(&tl->vfull[s]), (uint32_t)(it / a.nvs) & 1u, abort_flag,
                          a.status);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t d = tbase + (uint32_t)(2 * HP + vg * HP);
-            const uint32_t abase = s_stage0 + (uint32_t)s * kStageBytes;
+            const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
+            const uint32_t abase = s_vring + (uint32_t)s * kStageBytes;
             const uint32_t pbase = s_p0 + (uint32_t)(pb * a.pbuf_bytes);
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks)
-              umma_bf16(d, desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
+              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP),
+                        desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
                         desc_kmajor_sw128(pbase + (ks >> 2) * HP * 128 + (ks & 3) * 32), idesc_u,
-                        !(first_of_seg && ks == 0));
-            umma_commit(smem_u32(&tl->empty[s]));
+                        !(first_of_seg && ks < kUAcc));
+            umma_commit(smem_u32(&tl->vempty[s]));
           }
           if (!ok) break;
           umma_commit(smem_u32(&tl->u_done[pb]));
@@ -309,21 +330,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           for (int vg = 0; vg < a.nvg && ok; ++vg) {
-            const int it = lt * a.spt + a.nkg + vg;
-            const int s = it % a.nstage;
-            ok = wait_ab(smem_u32(&tl->full[s]), (uint32_t)(it / a.nstage) & 1u, abort_flag,
+            const int it = lt * a.nvg + vg;
+            const int s = it % a.nvs;
+            ok = wait_ab(smem_u32(&tl->vfull[s]), (uint32_t)(it / a.nvs) & 1u, abort_flag,
                          a.status);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t d = tbase + (uint32_t)(2 * HP + vg * HP);
-            const uint32_t abase = s_stage0 + (uint32_t)s * kStageBytes;
+            const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
+            const uint32_t abase = s_vring + (uint32_t)s * kStageBytes;
             const uint32_t pbase = s_p0 + (uint32_t)(pb * a.pbuf_bytes);
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks)
-              umma_bf16(d, desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
+              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP),
+                        desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
                         desc_kmajor_sw128(pbase + (ks >> 2) * HP * 128 + (ks & 3) * 32), idesc_u,
-                        !(first_of_seg && ks == 0));
-            umma_commit(smem_u32(&tl->empty[s]));
+                        !(first_of_seg && ks < kUAcc));
+            umma_commit(smem_u32(&tl->vempty[s]));
           }
           if (!ok) break;
           umma_commit(smem_u32(&tl->u_done[pb]));
@@ -368,7 +390,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float s[HP];
 #pragma unroll
-      for (int h0 = 0; h0 < HP; h0 += 16) tmem_ld16(lane_base + (uint32_t)(sb * HP + h0), s + h0);
+      for (int h0 = 0; h0 < HP; h0 += 16) {
+        tmem_ld16(lane_base + (uint32_t)(sb * kSAcc * HP + h0), s + h0);
+#pragma unroll
+        for (int j = 1; j < kSAcc; ++j) {
+          float t[16];
+          tmem_ld16(lane_base + (uint32_t)(sb * kSAcc * HP + j * HP + h0), t);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) s[h0 + e] += t[e];
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tl->s_empty[sb]));
@@ -409,11 +440,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   abort_flag, a.status));
           if (!ok) break;
           tc_fence_after();
-          for (int vg = 0; vg < a.nvg; ++vg) {
+          for (int j = 0; j < a.nvg * kUAcc; ++j) {
 #pragma unroll
             for (int h0 = 0; h0 < HP; h0 += 16) {
               float u[16];
-              const uint32_t ta = lane_base + (uint32_t)(2 * HP + vg * HP + h0);
+              const uint32_t ta = lane_base + (uint32_t)(2 * kSAcc * HP + j * HP + h0);
               tmem_ld16(ta, u);
 #pragma unroll
               for (int e = 0; e < 16; ++e) u[e] *= alpha[h0 + e];
@@ -455,7 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h0 = 0; h0 < HP; h0 += 16) {
             float u[16];
-            tmem_ld16(lane_base + (uint32_t)(2 * HP + vg * HP + h0), u);
+            tmem_ld16(lane_base + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP + h0), u);
+#pragma unroll
+            for (int j = 1; j < kUAcc; ++j) {
+              float t[16];
+              tmem_ld16(lane_base + (uint32_t)(2 * kSAcc * HP + (vg * kUAcc + j) * HP + h0), t);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) u[e] += t[e];
+            }
 #pragma unroll
             for (int e = 0; e < 16; ++e)
               if (h0 + e < a.H) rec[(size_t)(h0 + e) * a.pstride + 4 + vg * 128 + row] = u[e];
@@ -491,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct D2Plan {
-  int hp, tps, tiles, tpc, grid, nkg, nvg, spt, nstage;
+  int hp, tps, tiles, tpc, grid, nkg, nvg, nks, nvs;
   int off_q, off_p, off_tail, qbuf_bytes, pbuf_bytes;
   size_t smem;
   uint32_t tmem_cols;
@@ -512,19 +550,23 @@ lla_status plan_2d(int B, int H, int N, int r_k, int r_v, D2Plan* p) {
   d.grid = (d.tiles + d.tpc - 1) / d.tpc;
   d.nkg = (r_k + 127) / 128;
   d.nvg = r_v / 128;
-  d.spt = d.nkg + d.nvg;
   d.qbuf_bytes = (r_k / 64) * d.hp * 128;
   d.pbuf_bytes = 2 * d.hp * 128;
   const size_t fixed = 2 * (size_t)d.qbuf_bytes + 2 * (size_t)d.pbuf_bytes + sizeof(Tail2) + 1024;
-  int nst = (int)std::min<size_t>(kMaxStages, ((size_t)di.smem_optin - fixed) / kStageBytes);
-  nst = std::min(nst, 6);
-  if (nst < d.spt) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D stage ring does not fit in shared memory");
-  d.nstage = nst;
-  d.off_q = nst * kStageBytes;
+  // Split the stages between the rings: each ring needs at least one
+  // tile's groups (its slots are reused only by later tiles) and gets at
+  // most kMaxStages; K gets the odd one out.
+  const int nst = (int)std::min<size_t>(2 * kMaxStages,
+                                        ((size_t)di.smem_optin - fixed) / kStageBytes);
+  d.nvs = std::min(kMaxStages, std::max(d.nvg, nst / 2));
+  d.nks = std::min(kMaxStages, nst - d.nvs);
+  if (d.nks < d.nkg || d.nvs < d.nvg)
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D stage rings do not fit in shared memory");
+  d.off_q = (d.nks + d.nvs) * kStageBytes;
   d.off_p = d.off_q + 2 * d.qbuf_bytes;
   d.off_tail = d.off_p + 2 * d.pbuf_bytes;
   d.smem = (size_t)d.off_tail + sizeof(Tail2) + 1024;
-  const int cols = (2 + d.nvg) * d.hp;
+  const int cols = (2 * kSAcc + d.nvg * kUAcc) * d.hp;
   uint32_t c = 32;
   while (c < (uint32_t)cols) c <<= 1;
   d.tmem_cols = c;
@@ -588,8 +630,8 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
   a.r_v = r_v;
   a.nkg = d.nkg;
   a.nvg = d.nvg;
-  a.spt = d.spt;
-  a.nstage = d.nstage;
+  a.nks = d.nks;
+  a.nvs = d.nvs;
   a.off_q = d.off_q;
   a.off_p = d.off_p;
   a.off_tail = d.off_tail;
@@ -614,8 +656,12 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
   cfg.stream = stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
+  e = record_timing(true, stream);
+  if (e != cudaSuccess) return check_cuda(e, "record timing event");
   e = cudaLaunchKernelEx(&cfg, kern, tk, tv, a);
   if (e != cudaSuccess) return check_cuda(e, "launch k_lla2d");
+  e = record_timing(false, stream);
+  if (e != cudaSuccess) return check_cuda(e, "record timing event");
 
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v,
                         (long long)d.tps * kRows, (long long)d.tpc * kRows, 1, out, lse, stream);

@@ -1,0 +1,306 @@
+// Per-head absorbed LLA decode, streaming kernel (sm_100a).
+//
+// Source: "Looped Latent Attention: Cross-Loop KV Compression for Looped
+// Transformers" (arXiv 2607.15456), §7 "Per-head LLA versus LLA-2D at
+// inference": scores read latents directly through the absorbed query, and
+// the value side is summed in latent space.
+//
+// The flattened (unit, token) range of one (layer, loop) step is cut into
+// equal contiguous pieces, one per warp of a one-wave grid. Each warp runs
+// its own bulk-async-copy pipeline (cp.async.bulk into a ring of shared-
+// memory stages, completion counted on one mbarrier per stage), computes
+// scores q' . z^K_j, keeps an online softmax per token slot and accumulates
+// sum_j p_j z^V_j in latent space. Each (warp, unit) piece ends in one
+// partial record (m, l, u) that k_combine merges.
+#include "common.cuh"
+#include "stream.cuh"
+
+namespace lla {
+namespace {
+
+
+
+template <int ESZ>
+__device__ __forceinline__ void unpack16(const uint4& v, float* f);
+template <>
+__device__ __forceinline__ void unpack16<2>(const uint4& v, float* f) {
+  f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+  f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+template <>
+__device__ __forceinline__ void unpack16<4>(const uint4& v, float* f) {
+  f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+}
+
+// Loads q' of unit u (this lane's segments) into registers.
+template <int E, int LPT, int SK, bool EXACT>
+__device__ __forceinline__ void load_qp(float (&qv)[SK][E], const float* qp, long long u, int r_k,
+                                        int nseg_k, int g) {
+#pragma unroll
+  for (int s = 0; s < SK; ++s) {
+    const int seg = s * LPT + g;
+    if (EXACT || seg < nseg_k) {
+      const float4* src = reinterpret_cast<const float4*>(qp + u * r_k + seg * E);
+#pragma unroll
+      for (int e4 = 0; e4 < E / 4; ++e4) {
+        const float4 t = src[e4];
+        qv[s][4 * e4 + 0] = t.x;
+        qv[s][4 * e4 + 1] = t.y;
+        qv[s][4 * e4 + 2] = t.z;
+        qv[s][4 * e4 + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[s][e] = 0.f;
+    }
+  }
+}
+
+// One token slot's online-softmax update with score sc (log2 units) and
+// value row v.
+template <int ESZ, int LPT, int SV, bool EXACT>
+__device__ __forceinline__ void slot_update(float sc, const unsigned char* vrow, float& m, float& l,
+                                            float (&acc)[SV][16 / ESZ], int nseg_v, int g) {
+  constexpr int E = 16 / ESZ;
+  if (sc > m + kRescaleSlack) {
+    const float alpha = exp2f(m - sc);
+    l *= alpha;
+#pragma unroll
+    for (int s = 0; s < SV; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[s][e] *= alpha;
+    m = sc;
+  }
+  const float p = exp2f(sc - m);
+  l += p;
+#pragma unroll
+  for (int s = 0; s < SV; ++s) {
+    const int seg = s * LPT + g;
+    if (EXACT || seg < nseg_v) {
+      float x[E];
+      unpack16<ESZ>(*reinterpret_cast<const uint4*>(vrow + seg * 16), x);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[s][e] = fmaf(p, x[e], acc[s][e]);
+    }
+  }
+}
+
+// ESZ: bytes per latent element. LPT: lanes per token. SK/SV: 16-byte
+// segments per lane for K/V. EXACT: nseg == LPT*S for both axes.
+template <int ESZ, int LPT, int SK, int SV, bool EXACT>
+__global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
+  constexpr int E = 16 / ESZ;   // elements per 16-byte segment
+  constexpr int NS = 32 / LPT;  // token slots per warp
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const long long w = (long long)blockIdx.x * nwarps + warp;
+  if (w >= a.W) return;
+  const int slot = lane / LPT, g = lane - slot * LPT;
+
+  const int bar_bytes = ((nwarps * a.nstage * 8) + 127) & ~127;
+  const uint32_t bar0 = smem_u32(smem) + warp * a.nstage * 8;
+  unsigned char* buf = smem + bar_bytes + (size_t)warp * a.nstage * a.stage_bytes;
+  const uint32_t buf0 = smem_u32(buf);
+  const int v_off = a.tile * a.row_k;  // V part of a stage follows K
+
+  if (lane == 0) {
+    for (int s = 0; s < a.nstage; ++s) mbar_init(bar0 + 8 * s, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const long long f0 = w * a.P;
+  const long long f1 = min(f0 + a.P, a.total);
+  const uint64_t pol = l2_evict_first_policy();
+
+  // Producer side (lane 0 issues): the tile sequence is the range [f0, f1)
+  // cut at unit boundaries and at `tile` tokens; (pu, pj) is the unit and
+  // token of the next tile to load, ps its stage.
+  long long pf = f0, pu = f0 / a.N, pj = f0 - pu * a.N;
+  int ps = 0, in_flight = 0;
+  auto issue = [&]() {
+    const int len = (int)min((long long)a.tile, min(f1 - pf, a.N - pj));
+    if (lane == 0) {
+      const uint32_t kb = (uint32_t)len * a.row_k, vb = (uint32_t)len * a.row_v;
+      const uint32_t bar = bar0 + 8 * ps;
+      const long long row = pu * a.n_cap + pj;
+      const uint32_t dst = buf0 + ps * a.stage_bytes;
+      mbar_arrive_expect_tx(bar, kb + vb);
+      bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
+      bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
+    }
+    pf += len;
+    pj += len;
+    if (pj == a.N) {
+      pj = 0;
+      ++pu;
+    }
+    if (++ps == a.nstage) ps = 0;
+    ++in_flight;
+  };
+  for (int s = 0; s < a.nstage && pf < f1; ++s) issue();
+
+  // q' is written by k_absorb.
+  pdl_wait();
+
+  int cs = 0;          // stage being consumed
+  uint32_t cpar = 0;   // its phase parity
+  long long f = f0;
+  long long u = f0 / a.N;
+  const long long u_last = (f1 - 1) / a.N;
+  float qv[SK][E], qn[SK][E];
+  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g);
+  while (f < f1) {
+    const long long seg_end = min(f1, (u + 1) * a.N);
+    // the next unit's q' loads run under this unit's stream
+    if (u < u_last) load_qp<E, LPT, SK, EXACT>(qn, a.qp, u + 1, a.r_k, a.nseg_k, g);
+    float m = kNegBig, l = 0.f;
+    float acc[SV][E];
+#pragma unroll
+    for (int s = 0; s < SV; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[s][e] = 0.f;
+
+    while (f < seg_end) {
+      const int len = (int)min((long long)a.tile, seg_end - f);
+      const bool ok = __all_sync(FULL, mbar_wait(bar0 + 8 * cs, cpar));
+      if (!ok) {
+        if (lane == 0) report_status(a.status, kStatusWaitTimeout);
+        int st = cs;
+        uint32_t par = cpar;
+        for (int i = 0; i < in_flight; ++i) {
+          (void)mbar_wait(bar0 + 8 * st, par, kWaitTimeoutNs / 8);
+          if (++st == a.nstage) {
+            st = 0;
+            par ^= 1u;
+          }
+        }
+        return;
+      }
+      const unsigned char* Ks = buf + cs * a.stage_bytes;
+      const unsigned char* Vs = Ks + v_off;
+
+      for (int t0 = 0; t0 < len; t0 += 2 * NS) {
+        const int ta = t0 + slot, tb = t0 + NS + slot;
+        const bool va = ta < len, vb = tb < len;
+        float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+#pragma unroll
+        for (int s = 0; s < SK; ++s) {
+          const int seg = s * LPT + g;
+          if (EXACT || seg < a.nseg_k) {
+            float x[E];
+            if (va) {
+              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + ta * a.row_k + seg * 16), x);
+#pragma unroll
+              for (int e = 0; e < E; e += 2) {
+                sa0 = fmaf(qv[s][e], x[e], sa0);
+                sa1 = fmaf(qv[s][e + 1], x[e + 1], sa1);
+              }
+            }
+            if (vb) {
+              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + tb * a.row_k + seg * 16), x);
+#pragma unroll
+              for (int e = 0; e < E; e += 2) {
+                sb0 = fmaf(qv[s][e], x[e], sb0);
+                sb1 = fmaf(qv[s][e + 1], x[e + 1], sb1);
+              }
+            }
+          }
+        }
+        float sa = sa0 + sa1, sb = sb0 + sb1;
+#pragma unroll
+        for (int o = LPT / 2; o > 0; o >>= 1) {
+          sa += __shfl_xor_sync(FULL, sa, o);
+          sb += __shfl_xor_sync(FULL, sb, o);
+        }
+        if (va) slot_update<ESZ, LPT, SV, EXACT>(sa, Vs + ta * a.row_v, m, l, acc, a.nseg_v, g);
+        if (vb) slot_update<ESZ, LPT, SV, EXACT>(sb, Vs + tb * a.row_v, m, l, acc, a.nseg_v, g);
+      }
+      __syncwarp();
+      --in_flight;
+      if (pf < f1) issue();  // refill the stage just read
+      if (++cs == a.nstage) {
+        cs = 0;
+        cpar ^= 1u;
+      }
+      f += len;
+    }
+
+    // Merge the NS token slots of this warp (log-sum-exp butterfly).
+#pragma unroll
+    for (int o = LPT; o < 32; o <<= 1) {
+      const float mo = __shfl_xor_sync(FULL, m, o);
+      const float lo = __shfl_xor_sync(FULL, l, o);
+      const float M = fmaxf(m, mo);
+      const float wa = exp2f(m - M), wb = exp2f(mo - M);
+      l = l * wa + lo * wb;
+#pragma unroll
+      for (int s = 0; s < SV; ++s)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float ao = __shfl_xor_sync(FULL, acc[s][e], o);
+          acc[s][e] = acc[s][e] * wa + ao * wb;
+        }
+      m = M;
+    }
+    if (slot == 0) {
+      float* pp = a.part + (size_t)(w + u) * a.pstride;
+      if (g == 0) {
+        pp[0] = m;
+        pp[1] = l;
+      }
+#pragma unroll
+      for (int s = 0; s < SV; ++s) {
+        const int seg = s * LPT + g;
+        if (EXACT || seg < a.nseg_v) {
+          float4* dst = reinterpret_cast<float4*>(pp + 4 + seg * E);
+#pragma unroll
+          for (int e4 = 0; e4 < E / 4; ++e4)
+            dst[e4] = make_float4(acc[s][4 * e4], acc[s][4 * e4 + 1], acc[s][4 * e4 + 2],
+                                  acc[s][4 * e4 + 3]);
+        }
+      }
+    }
+    ++u;
+#pragma unroll
+    for (int s = 0; s < SK; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[s][e] = qn[s][e];
+  }
+}
+
+
+
+template <int ESZ>
+StreamFn pick_stream(int lpt, int s, bool exact) {
+  if (!exact) {
+    switch (lpt) {
+      case 1: return k_stream<ESZ, 1, 4, 4, false>;
+      case 2: return k_stream<ESZ, 2, 4, 4, false>;
+      case 4: return k_stream<ESZ, 4, 4, 4, false>;
+      case 8: return k_stream<ESZ, 8, 4, 4, false>;
+    }
+    return nullptr;
+  }
+#define LLA_CASE(L, S) \
+  if (lpt == L && s == S) return k_stream<ESZ, L, S, S, true>;
+  LLA_CASE(1, 1) LLA_CASE(1, 2) LLA_CASE(1, 3) LLA_CASE(1, 4)
+  LLA_CASE(2, 1) LLA_CASE(2, 2) LLA_CASE(2, 3) LLA_CASE(2, 4)
+  LLA_CASE(4, 1) LLA_CASE(4, 2) LLA_CASE(4, 3) LLA_CASE(4, 4)
+  LLA_CASE(8, 1) LLA_CASE(8, 2) LLA_CASE(8, 3) LLA_CASE(8, 4)
+#undef LLA_CASE
+  return nullptr;
+}
+
+}  // namespace
+
+StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact) {
+  return esz == 2 ? pick_stream<2>(lpt, s, exact) : pick_stream<4>(lpt, s, exact);
+}
+
+}  // namespace lla

@@ -74,6 +74,18 @@ LLA_API int lla_version(void);
  */
 LLA_API lla_status lla_device_status(unsigned int *status, int clear);
 
+/*
+ * Timing hook for benchmarks and profilers. When both arguments are non-NULL
+ * (cudaEvent_t handles passed as void*), every later lla_decode_attn,
+ * lla_decode_attn_noalloc, lla2d_decode_attn or lla_encode call made on the
+ * calling thread records ev_begin on its stream just before its main kernel
+ * (the latent stream, the LLA-2D tensor-core kernel, or the encoder) and
+ * ev_end just after it. The recordings separate that kernel from its
+ * neighbours, so launch overlap between them is lost while a hook is set.
+ * Pass NULL, NULL to clear.
+ */
+LLA_API void lla_set_timing_events(void *ev_begin, void *ev_end);
+
 /* --------------------------------------------------------------------------
  * Per-head absorbed decode, one (layer d, loop t) step.
  *
