@@ -72,7 +72,11 @@ def parse_args():
 # distributed plumbing
 # ---------------------------------------------------------------------------
 
-def dist_setup(args):
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU: reads RANK / LOCAL_RANK / WORLD_SIZE / MASTER_*
+    from the environment. Sequences are sharded by rank (each rank decodes
+    its own batch), so the data path has no collective; the process group
+    only carries the barrier and the max-over-ranks timing."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -80,9 +84,11 @@ def dist_setup(args):
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -95,12 +101,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's value (step times are taken as the max over ranks)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(units_per_rank: float, ms_per_step: float, world: int) -> float:
+    """Whole-job throughput: every rank processes `units_per_rank` units per
+    step (weak scaling) and the step takes the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -314,7 +328,7 @@ def run_encode_bench(args, world, rank, local):
     flops = 2 * cfg.N * cfg.G * cfg.T * cfg.d_loop * cfg.r
     line = {
         "metric": "LLA encode: prefill tokens encoded/sec (every layer, K and V)",
-        "value": world * cfg.N / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "value": aggregate_rate(cfg.N, ms_per_step, world), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -518,7 +532,7 @@ def run_lla(args, world, rank, local):
     kern_ms_mean = sum(kern_ms) / len(kern_ms)
 
     tokens_per_step = cfg.B * cfg.N * cfg.L * cfg.T
-    value = world * tokens_per_step / (ms_per_step * 1e-3)
+    value = aggregate_rate(tokens_per_step, ms_per_step, world)
     step_bytes = cfg.step_bytes()
     hbm_peak, peak_src = peaks()
     achieved = step_bytes / (kern_ms_mean * 1e-3) / 1e9
@@ -556,7 +570,7 @@ def run_lla(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
-        e2e = {"value": world * tokens_per_step / (e2e_ms * 1e-3), "unit": UNIT,
+        e2e = {"value": aggregate_rate(tokens_per_step, e2e_ms, world), "unit": UNIT,
                "h2d_bytes_per_step": sum(h_.numel() * h_.element_size() for h_ in hosts),
                "d2h_bytes_per_step": (out_host.numel() + lse_host.numel()) * 4}
 
@@ -603,7 +617,7 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist_setup("nccl")
     try:
         if args.config in ENCODE_CONFIGS:
             run_encode_bench(args, world, rank, local)

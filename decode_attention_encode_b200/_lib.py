@@ -134,6 +134,11 @@ class kernel_timer:
     def __init__(self):
         self.begin = torch.cuda.Event(enable_timing=True)
         self.end = torch.cuda.Event(enable_timing=True)
+        # torch creates the underlying CUDA events on first record
+        stream = torch.cuda.current_stream()
+        self.begin.record(stream)
+        self.end.record(stream)
+        self.end.synchronize()
         self.ms = None
 
     def __enter__(self):

@@ -169,10 +169,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + (size_t)s * a.stage_bytes);
-          const uint32_t sb = sa + kABytes;
+          // descriptors built once per stage, advanced 32 B (2 x 16 B) per K step
+          const uint64_t a_base = desc_kmajor_sw128(sa);
+          const uint64_t b_base = desc_kmajor_sw128(sa + kABytes);
 #pragma unroll
           for (int kk = 0; kk < kChunkK / 16; ++kk)
-            umma_bf16(d, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idesc,
+            umma_bf16(d, a_base + (uint64_t)(kk * 2), b_base + (uint64_t)(kk * 2), idesc,
                       (kc | kk) != 0);
           umma_commit(smem_u32(&tail->empty[s]));
         }

@@ -266,16 +266,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                        a.status))
             return false;
           tc_fence_after();
-          const int nb = kboxes(kg);
-          for (int x = 0; x < nb; ++x) {
-            const uint32_t abox = s_kring + (uint32_t)s * kStageBytes + x * kBoxBytes;
-            const uint32_t bchunk = qaddr + (uint32_t)((kg * 2 + x) * HP * 128);
+          // Descriptors are built once per stage and advanced by constant
+          // start-address offsets (in 16-byte units): 32 B per K step inside
+          // a 128B-swizzled row, one box (16 KB) per 64 columns.
+          const uint64_t a_base = desc_kmajor_sw128(s_kring + (uint32_t)s * kStageBytes);
+          const uint64_t b_base = desc_kmajor_sw128(qaddr + (uint32_t)(kg * 2 * HP * 128));
+          const bool first = kg == 0;
+          if (kboxes(kg) == 2) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int kidx = (kg * 2 + x) * 4 + kk;  // K step within the tile
-              umma_bf16(d0 + (uint32_t)((kidx % kSAcc) * HP), desc_kmajor_sw128(abox + kk * 32),
-                        desc_kmajor_sw128(bchunk + kk * 32), idesc_s, kidx >= kSAcc);
+            for (int st = 0; st < 8; ++st) {
+              const int x = st >> 2, kk = st & 3;
+              const uint64_t a_d = a_base + (uint64_t)(x * (kBoxBytes >> 4) + kk * 2);
+              const uint64_t b_d = b_base + (uint64_t)(x * (HP * 128 >> 4) + kk * 2);
+              umma_bf16(d0 + (uint32_t)((st % kSAcc) * HP), a_d, b_d, idesc_s,
+                        !(first && st < kSAcc));
             }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(d0 + (uint32_t)((kk % kSAcc) * HP), a_base + (uint64_t)(kk * 2),
+                        b_base + (uint64_t)(kk * 2), idesc_s, !(first && kk < kSAcc));
           }
           umma_commit(smem_u32(&tl->kempty[s]));
         }
@@ -311,13 +321,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
-            const uint32_t abase = s_vring + (uint32_t)s * kStageBytes;
-            const uint32_t pbase = s_p0 + (uint32_t)(pb * a.pbuf_bytes);
+            // A (MN-major latents): 16 token rows (2 KB) per K step;
+            // B (K-major P): 32 B per K step inside a 64-token chunk.
+            const uint64_t a_base =
+                desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes, kBoxBytes);
+            const uint64_t b_base = desc_kmajor_sw128(s_p0 + (uint32_t)(pb * a.pbuf_bytes));
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks)
-              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP),
-                        desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
-                        desc_kmajor_sw128(pbase + (ks >> 2) * HP * 128 + (ks & 3) * 32), idesc_u,
+              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP), a_base + (uint64_t)(ks * (2048 >> 4)),
+                        b_base + (uint64_t)((ks >> 2) * (HP * 128 >> 4) + (ks & 3) * 2), idesc_u,
                         !(first_of_seg && ks < kUAcc));
             umma_commit(smem_u32(&tl->vempty[s]));
           }
@@ -337,13 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
-            const uint32_t abase = s_vring + (uint32_t)s * kStageBytes;
-            const uint32_t pbase = s_p0 + (uint32_t)(pb * a.pbuf_bytes);
+            // A (MN-major latents): 16 token rows (2 KB) per K step;
+            // B (K-major P): 32 B per K step inside a 64-token chunk.
+            const uint64_t a_base =
+                desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes, kBoxBytes);
+            const uint64_t b_base = desc_kmajor_sw128(s_p0 + (uint32_t)(pb * a.pbuf_bytes));
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks)
-              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP),
-                        desc_mnmajor_sw128(abase + ks * 2048, kBoxBytes),
-                        desc_kmajor_sw128(pbase + (ks >> 2) * HP * 128 + (ks & 3) * 32), idesc_u,
+              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP), a_base + (uint64_t)(ks * (2048 >> 4)),
+                        b_base + (uint64_t)((ks >> 2) * (HP * 128 >> 4) + (ks & 3) * 2), idesc_u,
                         !(first_of_seg && ks < kUAcc));
             umma_commit(smem_u32(&tl->vempty[s]));
           }
