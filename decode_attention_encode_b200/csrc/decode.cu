@@ -33,9 +33,15 @@
 namespace lla {
 namespace {
 
-constexpr int kAbsorbRows = 64;   // batch rows per k_absorb CTA (8 per warp)
-constexpr int kCombineRows = 32;  // batch rows per k_combine CTA (4 per warp)
-constexpr int kColChunk = 32;     // decoder columns (absorb) / rows (combine) per CTA
+// Rows per thread of k_absorb / k_combine: the largest of 1, 2, 4, 8 that
+// still gives at least ~256 CTAs (more rows per thread reuse each decoder
+// value from shared memory more often).
+int rows_per_thread(int ctas_per_row_block_of_8, int B) {
+  int rows = 8;
+  while (rows > 1 && (long long)ctas_per_row_block_of_8 * ((B + 8 * rows - 1) / (8 * rows)) < 256)
+    rows >>= 1;
+  return rows;
+}
 
 // ---------------------------------------------------------------------------
 // k_absorb
@@ -45,44 +51,44 @@ struct AbsorbArgs {
   const float* dk;
   const float* mu_k;
   int B, H, d_h, r_k;
-  int rows;  // batch rows per CTA: 8, 16, 32 or 64
   float qscale;  // scale * log2(e): scores leave k_stream in log2 units
   float scale;
   float* qp;  // [B*H][r_k]
   float* c0;  // [B*H], natural-log units
 };
 
-// One CTA per (head, `rows` batch rows, 32 latent columns). The CTA stages
-// the d_h x 32 slice of W^K_up,t once and its query rows in shared memory;
-// thread (warp w, lane l) forms q'[b][c0 + l] for the rows b = w + 8k, so
-// each decoder value read from shared memory feeds rows/8 FMAs. `rows` is
-// chosen on the host so the grid stays near 512-1024 CTAs.
+// One CTA per (head, 32 latent columns, 8*ROWS batch rows). The CTA stages
+// its d_h x 32 slice of W^K_up,t (all float4 loads issued before the first
+// use) and its query rows in shared memory; thread (warp w, lane l) forms
+// q'[b][c0 + l] for the ROWS rows b = b0 + w*ROWS + k, so one decoder value
+// read from shared memory feeds ROWS FMAs and one float4 query read feeds 4.
+template <int ROWS>
 __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
   extern __shared__ __align__(16) float sm_absorb[];
-  float* q_s = sm_absorb;                        // [rows][d_h4]
-  const int d_h4 = (a.d_h + 3) & ~3;             // rows padded to float4
-  float* d_s = sm_absorb + a.rows * d_h4;        // [d_h][kColChunk]
+  const int d_h4 = (a.d_h + 3) & ~3;
+  float* d_s = sm_absorb;                   // [d_h4][32]
+  float* q_s = sm_absorb + d_h4 * 32;       // [8*ROWS][d_h4]
   pdl_launch_dependents();
   const int h = blockIdx.x;
-  const int b0 = blockIdx.y * a.rows;
-  const int c0 = blockIdx.z * kColChunk;
-  const int nb = min(a.rows, a.B - b0);
-  const int nc = min(kColChunk, a.r_k - c0);
-  for (int idx = threadIdx.x; idx < nb * d_h4; idx += blockDim.x) {
-    const int bb = idx / d_h4, i = idx - bb * d_h4;
-    q_s[idx] = i < a.d_h ? a.q[((size_t)(b0 + bb) * a.H + h) * a.d_h + i] : 0.f;
-  }
+  const int c0 = blockIdx.y * 32;
+  const int b0 = blockIdx.z * (8 * ROWS);
+  const int nb = min(8 * ROWS, a.B - b0);
+  const int nc = min(32, a.r_k - c0);  // a multiple of 8
+  const int n4 = nc / 4;
   const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
-  const int n4 = nc / 4;  // nc is a multiple of 8
-  for (int idx = threadIdx.x; idx < a.d_h * n4; idx += blockDim.x) {
-    const int i = idx / n4, j = idx - i * n4;
-    reinterpret_cast<float4*>(d_s + i * kColChunk)[j] =
-        __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j);
+  for (int idx = threadIdx.x; idx < d_h4 * 8; idx += 256) {
+    const int i = idx >> 3, j = idx & 7;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < a.d_h && j < n4) v = __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j);
+    reinterpret_cast<float4*>(d_s + i * 32)[j] = v;
+  }
+  for (int idx = threadIdx.x; idx < 8 * ROWS * d_h4; idx += 256) {
+    const int bb = idx / d_h4, i = idx - bb * d_h4;
+    q_s[idx] = (bb < nb && i < a.d_h) ? a.q[((size_t)(b0 + bb) * a.H + h) * a.d_h + i] : 0.f;
   }
   __syncthreads();
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (blockIdx.z == 0) {
+  if (blockIdx.y == 0) {
     // c0 = scale * q . mu_k (natural-log units), one warp per row
     for (int bb = warp; bb < nb; bb += 8) {
       float acc = 0.f;
@@ -93,27 +99,23 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
       if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
     }
   }
-  constexpr int kPer = kAbsorbRows / 8;
-  float acc[kPer];
+  float acc[ROWS];
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  if (lane < nc) {
-    for (int i = 0; i < a.d_h; i += 4) {
-      float dv[4];
+  for (int k = 0; k < ROWS; ++k) acc[k] = 0.f;
+  const float* qrow = q_s + warp * ROWS * d_h4;
+  for (int i = 0; i < d_h4; i += 4) {
+    const float d0 = d_s[(i + 0) * 32 + lane], d1 = d_s[(i + 1) * 32 + lane];
+    const float d2 = d_s[(i + 2) * 32 + lane], d3 = d_s[(i + 3) * 32 + lane];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) dv[e] = (i + e < a.d_h) ? d_s[(i + e) * kColChunk + lane] : 0.f;
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int bb = warp + 8 * k;
-        if (bb < nb) {
-          const float4 qv = *reinterpret_cast<const float4*>(q_s + bb * d_h4 + i);
-          acc[k] = fmaf(dv[0], qv.x, fmaf(dv[1], qv.y, fmaf(dv[2], qv.z, fmaf(dv[3], qv.w, acc[k]))));
-        }
-      }
+    for (int k = 0; k < ROWS; ++k) {
+      const float4 qv = *reinterpret_cast<const float4*>(qrow + k * d_h4 + i);
+      acc[k] = fmaf(d0, qv.x, fmaf(d1, qv.y, fmaf(d2, qv.z, fmaf(d3, qv.w, acc[k]))));
     }
+  }
+  if (lane < nc) {
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int bb = warp + 8 * k;
+    for (int k = 0; k < ROWS; ++k) {
+      const int bb = warp * ROWS + k;
       if (bb < nb) a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = acc[k] * a.qscale;
     }
   }
@@ -131,90 +133,95 @@ struct CombineArgs {
   int B, H, d_h, r_v;
   long long N, P;  // per-sequence and per-piece extents of the split
   int shared;      // 1: one split per sequence shared by all heads (LLA-2D)
-  int rows;        // batch rows per CTA: 8, 16 or 32
   float* out;
   float* lse;
 };
 
-// One CTA per (head, `rows` batch rows, 32 output channels). Warp w merges
-// the partial records of rows w, w+8, ... into ubar (lanes across the latent
-// index); the CTA stages the 32 x r_v slice of W^V_up,t once (rows padded by
-// 4 floats, so float4 reads of 8 consecutive rows hit 8 distinct bank
-// groups); thread (warp w, lane l) forms out[b][h][i0 + l] for its rows.
+// One CTA per (head, 32 output channels, 8*ROWS batch rows). Warp w merges
+// the partial records of its ROWS rows into ubar (lanes across the latent
+// index in float4 steps); the CTA stages its 32 x r_v slice of W^V_up,t
+// (rows padded by 4 floats, so float4 reads of 8 consecutive rows hit
+// distinct bank groups; staged before waiting on the streaming kernel);
+// thread (w, l) forms out[b][h][i0 + l] for its ROWS rows.
+template <int ROWS>
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   extern __shared__ __align__(16) float sm_combine[];
   const int pitch = a.r_v + 4;
-  float* ub = sm_combine;                         // [rows][r_v]
-  float* d_s = sm_combine + a.rows * a.r_v;       // [kColChunk][pitch]
+  float* d_s = sm_combine;                        // [32][pitch]
+  float* ub = sm_combine + 32 * pitch;            // [8*ROWS][r_v]
   const int h = blockIdx.x;
-  const int b0 = blockIdx.y * a.rows;
-  const int i0 = blockIdx.z * kColChunk;
-  const int nb = min(a.rows, a.B - b0);
-  const int ni = min(kColChunk, a.d_h - i0);
-  // W^V does not depend on the streaming kernel: stage it before waiting
+  const int i0 = blockIdx.y * 32;
+  const int b0 = blockIdx.z * (8 * ROWS);
+  const int nb = min(8 * ROWS, a.B - b0);
+  const int ni = min(32, a.d_h - i0);
   const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
   const int r4 = a.r_v / 4;
-  for (int idx = threadIdx.x; idx < ni * r4; idx += blockDim.x) {
+  for (int idx = threadIdx.x; idx < ni * r4; idx += 256) {
     const int i = idx / r4, j = idx - i * r4;
     reinterpret_cast<float4*>(d_s + i * pitch)[j] =
         __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j);
   }
   pdl_wait();  // partials come from the streaming kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int bb = warp; bb < nb; bb += 8) {
+#pragma unroll
+  for (int k = 0; k < ROWS; ++k) {
+    const int bb = warp * ROWS + k;
+    float4* urow = reinterpret_cast<float4*>(ub + bb * a.r_v);
+    if (bb >= nb) {
+      for (int c4 = lane; c4 < r4; c4 += 32) urow[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
     const long long u = (long long)(b0 + bb) * a.H + h;
     // The split runs over units (b, h) for per-head LLA and over sequences
     // b for LLA-2D; piece w of split key k is partial record w + k.
     const long long key = a.shared ? (long long)(b0 + bb) : u;
     const long long wf = (key * a.N) / a.P;
     const long long wl = ((key + 1) * a.N - 1) / a.P;
-    auto rec = [&](long long w) {
-      return a.shared ? a.part + ((w + key) * a.H + h) * a.pstride : a.part + (w + key) * a.pstride;
-    };
     const int np = (int)(wl - wf + 1);
+    const float* rec0 = a.shared ? a.part + ((wf + key) * a.H + h) * a.pstride
+                                 : a.part + (wf + key) * a.pstride;
+    const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
     float M = kNegBig;
-    for (int k = lane; k < np; k += 32) M = fmaxf(M, rec(wf + k)[0]);
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, rec0[p * rstride]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (int k = lane; k < np; k += 32) {
-      const float* pp = rec(wf + k);
-      L += pp[1] * exp2f(pp[0] - M);
-    }
+    for (int p = lane; p < np; p += 32) L += rec0[p * rstride + 1] * exp2f(rec0[p * rstride] - M);
     L = warp_sum(L);
     const float inv = 1.f / L;
-    for (int c = lane; c < a.r_v; c += 32) {
-      float acc = 0.f;
-      for (int k = 0; k < np; ++k) {
-        const float* pp = rec(wf + k);
-        acc = fmaf(exp2f(pp[0] - M), pp[4 + c], acc);
+    for (int c4 = lane; c4 < r4; c4 += 32) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int p = 0; p < np; ++p) {
+        const float wk = exp2f(rec0[p * rstride] - M);
+        const float4 uv = reinterpret_cast<const float4*>(rec0 + p * rstride + 4)[c4];
+        acc.x = fmaf(wk, uv.x, acc.x);
+        acc.y = fmaf(wk, uv.y, acc.y);
+        acc.z = fmaf(wk, uv.z, acc.z);
+        acc.w = fmaf(wk, uv.w, acc.w);
       }
-      ub[bb * a.r_v + c] = acc * inv;
+      urow[c4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
-    if (blockIdx.z == 0 && lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
+    if (blockIdx.y == 0 && lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
   }
   __syncthreads();
   if (lane < ni) {
-    constexpr int kPer = kCombineRows / 8;
-    float acc[kPer];
+    float acc[ROWS];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-    const float* drow = d_s + lane * pitch;
-    for (int c = 0; c < a.r_v; c += 4) {
-      const float4 dv = *reinterpret_cast<const float4*>(drow + c);
+    for (int k = 0; k < ROWS; ++k) acc[k] = 0.f;
+    const float4* drow = reinterpret_cast<const float4*>(d_s + lane * pitch);
+    const float4* ubase = reinterpret_cast<const float4*>(ub + warp * ROWS * a.r_v);
+    for (int c4 = 0; c4 < r4; ++c4) {
+      const float4 dv = drow[c4];
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int bb = warp + 8 * k;
-        if (bb < nb) {
-          const float4 uv = *reinterpret_cast<const float4*>(ub + bb * a.r_v + c);
-          acc[k] = fmaf(dv.x, uv.x, fmaf(dv.y, uv.y, fmaf(dv.z, uv.z, fmaf(dv.w, uv.w, acc[k]))));
-        }
+      for (int k = 0; k < ROWS; ++k) {
+        const float4 uv = ubase[k * r4 + c4];
+        acc[k] = fmaf(dv.x, uv.x, fmaf(dv.y, uv.y, fmaf(dv.z, uv.z, fmaf(dv.w, uv.w, acc[k]))));
       }
     }
     const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + lane] : 0.f;
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int bb = warp + 8 * k;
+    for (int k = 0; k < ROWS; ++k) {
+      const int bb = warp * ROWS + k;
       if (bb < nb) a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = acc[k] + mu;
     }
   }
@@ -237,16 +244,17 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream) {
-  const int zc = (r_k + kColChunk - 1) / kColChunk;
-  int rows = 8;
-  while (rows < kAbsorbRows && (long long)H * zc * ((B + rows - 1) / rows) > 1024) rows *= 2;
-  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, rows, scale * kLog2e, scale, qp, c0};
-  dim3 grid(H, (B + rows - 1) / rows, zc);
-  const size_t smem = ((size_t)rows * ((d_h + 3) & ~3) + (size_t)d_h * kColChunk) * 4;
-  cudaError_t e = cudaFuncSetAttribute(k_absorb, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0};
+  const int ncol = (r_k + 31) / 32;
+  const int rows = rows_per_thread(H * ncol, B);
+  dim3 grid(H, ncol, (B + 8 * rows - 1) / (8 * rows));
+  const int d_h4 = (d_h + 3) & ~3;
+  const size_t smem = ((size_t)d_h4 * 32 + (size_t)8 * rows * d_h4) * sizeof(float);
+  void (*fn)(AbsorbArgs) = rows == 8 ? k_absorb<8> : rows == 4 ? k_absorb<4>
+                         : rows == 2 ? k_absorb<2> : k_absorb<1>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_absorb)");
-  k_absorb<<<grid, 256, smem, stream>>>(a);
+  fn<<<grid, 256, smem, stream>>>(a);
   return check_cuda(cudaGetLastError(), "launch k_absorb");
 }
 
@@ -256,21 +264,22 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  const int zc = (d_h + kColChunk - 1) / kColChunk;
-  int rows = 8;
-  while (rows < kCombineRows && (long long)H * zc * ((B + rows - 1) / rows) > 1024) rows *= 2;
-  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, rows, out, lse};
+  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse};
+  const int nch = (d_h + 31) / 32;
+  const int rows = rows_per_thread(H * nch, B);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(H, (B + rows - 1) / rows, zc);
+  cfg.gridDim = dim3(H, nch, (B + 8 * rows - 1) / (8 * rows));
   cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = ((size_t)rows * r_v + (size_t)kColChunk * (r_v + 4)) * 4;
-  cudaError_t e = cudaFuncSetAttribute(k_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cfg.dynamicSmemBytes = ((size_t)32 * (r_v + 4) + (size_t)8 * rows * r_v) * sizeof(float);
+  void (*fn)(CombineArgs) = rows == 8 ? k_combine<8> : rows == 4 ? k_combine<4>
+                          : rows == 2 ? k_combine<2> : k_combine<1>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_combine)");
   cfg.stream = stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  return check_cuda(cudaLaunchKernelEx(&cfg, k_combine, a), "launch k_combine");
+  return check_cuda(cudaLaunchKernelEx(&cfg, fn, a), "launch k_combine");
 }
 
 lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePlan* p) {

@@ -128,7 +128,7 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
 }
 
 // ---------------------------------------------------------------------------
-// tiled TMA loads (no multicast)
+// tiled TMA loads into this CTA's own shared memory
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint32_t bar, uint64_t policy) {
