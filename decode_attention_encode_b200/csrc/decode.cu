@@ -232,15 +232,15 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 // ---------------------------------------------------------------------------
 bool exact_variant(int lpt, int s) { return lpt >= 1 && lpt <= 8 && s >= 1 && s <= 4; }
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
 int env_int(const char* name, int dflt) {
   const char* v = std::getenv(name);
   if (!v || !*v) return dflt;
   return std::atoi(v);
 }
-
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-}  // namespace
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream) {

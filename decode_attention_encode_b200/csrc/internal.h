@@ -33,6 +33,10 @@ cudaError_t record_timing(bool begin, cudaStream_t stream);
 // Maps a CUDA error to LLA_ERR_CUDA with its message, or LLA_OK.
 lla_status check_cuda(cudaError_t e, const char* what);
 
+// Integer tuning override from the environment (planner sweeps); `dflt`
+// when the variable is unset or empty.
+int env_int(const char* name, int dflt);
+
 // Host-side argument checks shared by the decode entry points; sets *esz to
 // the latent element size.
 lla_status check_decode_args(const float* q, const void* zk, const void* zv, lla_dtype zdt, int B,

@@ -21,18 +21,20 @@
 // ends in one partial record per head (m, l, U); k_combine merges them and
 // applies W^V_up,t. k_absorb (shared with the per-head path) forms q'.
 //
-// CTA roles (7 warps):
+// CTA roles (8 warps):
 //   warp 0     K producer: 128 x 128-column Z^K groups (two 64-column
 //              128B-swizzled boxes, 32 KB) into the K ring; stages Q' (bf16,
 //              swizzled K-major) for each new sequence.
-//   warp 1     TMEM owner and MMA issuer. Issues the score MMA of tile i+1
-//              before the value MMA of tile i so the softmax of tile i
-//              overlaps the next score MMA.
+//   warp 1     TMEM owner and score MMA issuer (up to one tile ahead of the
+//              softmax, two S buffers).
 //   warps 2-5  softmax and epilogue (one thread per TMEM lane).
 //   warp 6     V producer: Z^V groups into the V ring.
-// K and V have separate rings, so a K slot is reused as soon as its score
-// MMA retires and the K stream runs up to two tiles ahead of the value
-// MMAs, which wait on the softmax.
+//   warp 7     value MMA issuer.
+// The MMAs here are small (N = H), so their issue cost, not the tensor pipe,
+// sets their time: one thread issues one about every 60 cycles, two threads
+// together one about every 40. Two issuers also decouple the rings: a V slot
+// is released as soon as its tile's value MMA retires, whatever the K
+// stream is doing, and a K slot as soon as its score MMA retires.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -46,7 +48,7 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kBoxBytes = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int kStageBytes = 2 * kBoxBytes;
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
 constexpr int kMaxStages = 4;  // per ring
 constexpr float kNegBig = -1.0e30f;
 constexpr float kSlack = 8.0f;
@@ -73,7 +75,7 @@ struct Tail2 {
   uint64_t vfull[kMaxStages], vempty[kMaxStages];
   uint64_t s_full[2], s_empty[2], p_full[2], u_done[2], q_full[2], q_empty[2];
   uint64_t epi;    // 4-warp rendezvous of the softmax warps
-  uint64_t drain;
+  uint64_t drain[2];  // score issuer, value issuer
   uint32_t tmem_base;
   int abort_flag;
   int vote[2][4];
@@ -154,7 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&tl->q_empty[i]), 1);
     }
     mbar_init(smem_u32(&tl->epi), 4);
-    mbar_init(smem_u32(&tl->drain), 1);
+    mbar_init(smem_u32(&tl->drain[0]), 1);
+    mbar_init(smem_u32(&tl->drain[1]), 1);
     tl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -246,10 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         kWaitTimeoutNs / 8);
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
+    // --------------------------- score MMA issuer ---------------------------
+    // S[tokens x heads] = Z^K tile . Q'^T, one tile ahead of the softmax at
+    // most (two S buffers). Independent of the value issuer, so a late value
+    // group never holds up the next tile's scores.
     if (lane == 0 && ntile > 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kRows, HP, false, false);
-      const uint32_t idesc_u = idesc_bf16_f32(kRows, HP, true, false);
       bool ok = true;
       auto mma_scores = [&](int lt, int seg) -> bool {
         const int sb = lt & 1;
@@ -294,79 +299,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       int seg = 0;
-      ok = wait_ab(smem_u32(&tl->q_full[0]), 0u, abort_flag, a.status) && mma_scores(0, 0);
+      ok = wait_ab(smem_u32(&tl->q_full[0]), 0u, abort_flag, a.status);
+      for (int lt = 0; ok && lt < ntile; ++lt) {
+        if (lt > 0 && seq_of(lt) != seq_of(lt - 1)) {
+          umma_commit(smem_u32(&tl->q_empty[seg & 1]));  // after the last score MMA of seg
+          ++seg;
+          ok = wait_ab(smem_u32(&tl->q_full[seg & 1]), (uint32_t)((seg >> 1) & 1), abort_flag,
+                       a.status);
+          if (!ok) break;
+        }
+        ok = mma_scores(lt, seg);
+      }
+      umma_commit(smem_u32(&tl->drain[0]));
+      (void)mbar_wait(smem_u32(&tl->drain[0]), 0u, kWaitTimeoutNs / 8);
+    }
+  } else if (warp == 7) {
+    // --------------------------- value MMA issuer ---------------------------
+    // U[r_v x heads] += Z^V tile^T . P, per 128-column group of r_v, as soon
+    // as the softmax has written P for the tile.
+    if (lane == 0 && ntile > 0) {
+      const uint32_t idesc_u = idesc_bf16_f32(kRows, HP, true, false);
+      bool ok = true;
       for (int lt = 0; ok && lt < ntile; ++lt) {
         const bool first_of_seg = (lt == 0) || seq_of(lt) != seq_of(lt - 1);
-        if (lt + 1 < ntile) {
-          int seg_next = seg;
-          if (seq_of(lt + 1) != seq_of(lt)) {
-            umma_commit(smem_u32(&tl->q_empty[seg & 1]));  // after the last score MMA of seg
-            seg_next = seg + 1;
-            ok = wait_ab(smem_u32(&tl->q_full[seg_next & 1]), (uint32_t)((seg_next >> 1) & 1),
-                         abort_flag, a.status);
-            if (!ok) break;
-          }
-          ok = mma_scores(lt + 1, seg_next);
-          if (!ok) break;
-          // value MMA of tile lt belongs to `seg`; advance after it
-          const int pb = lt & 1;
-          ok = wait_ab(smem_u32(&tl->p_full[pb]), (uint32_t)((lt >> 1) & 1), abort_flag, a.status);
+        const int pb = lt & 1;
+        ok = wait_ab(smem_u32(&tl->p_full[pb]), (uint32_t)((lt >> 1) & 1), abort_flag, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        for (int vg = 0; vg < a.nvg && ok; ++vg) {
+          const int it = lt * a.nvg + vg;
+          const int s = it % a.nvs;
+          ok = wait_ab(smem_u32(&tl->vfull[s]), (uint32_t)(it / a.nvs) & 1u, abort_flag,
+                       a.status);
           if (!ok) break;
           tc_fence_after();
-          for (int vg = 0; vg < a.nvg && ok; ++vg) {
-            const int it = lt * a.nvg + vg;
-            const int s = it % a.nvs;
-            ok = wait_ab(smem_u32(&tl->vfull[s]), (uint32_t)(it / a.nvs) & 1u, abort_flag,
-                         a.status);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
-            // A (MN-major latents): 16 token rows (2 KB) per K step;
-            // B (K-major P): 32 B per K step inside a 64-token chunk.
-            const uint64_t a_base =
-                desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes, kBoxBytes);
-            const uint64_t b_base = desc_kmajor_sw128(s_p0 + (uint32_t)(pb * a.pbuf_bytes));
+          const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
+          // A (MN-major latents): 16 token rows (2 KB) per K step;
+          // B (K-major P): 32 B per K step inside a 64-token chunk.
+          const uint64_t a_base =
+              desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes, kBoxBytes);
+          const uint64_t b_base = desc_kmajor_sw128(s_p0 + (uint32_t)(pb * a.pbuf_bytes));
 #pragma unroll
-            for (int ks = 0; ks < kRows / 16; ++ks)
-              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP), a_base + (uint64_t)(ks * (2048 >> 4)),
-                        b_base + (uint64_t)((ks >> 2) * (HP * 128 >> 4) + (ks & 3) * 2), idesc_u,
-                        !(first_of_seg && ks < kUAcc));
-            umma_commit(smem_u32(&tl->vempty[s]));
-          }
-          if (!ok) break;
-          umma_commit(smem_u32(&tl->u_done[pb]));
-          seg = seg_next;
-        } else {
-          const int pb = lt & 1;
-          ok = wait_ab(smem_u32(&tl->p_full[pb]), (uint32_t)((lt >> 1) & 1), abort_flag, a.status);
-          if (!ok) break;
-          tc_fence_after();
-          for (int vg = 0; vg < a.nvg && ok; ++vg) {
-            const int it = lt * a.nvg + vg;
-            const int s = it % a.nvs;
-            ok = wait_ab(smem_u32(&tl->vfull[s]), (uint32_t)(it / a.nvs) & 1u, abort_flag,
-                         a.status);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
-            // A (MN-major latents): 16 token rows (2 KB) per K step;
-            // B (K-major P): 32 B per K step inside a 64-token chunk.
-            const uint64_t a_base =
-                desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes, kBoxBytes);
-            const uint64_t b_base = desc_kmajor_sw128(s_p0 + (uint32_t)(pb * a.pbuf_bytes));
-#pragma unroll
-            for (int ks = 0; ks < kRows / 16; ++ks)
-              umma_bf16(d + (uint32_t)((ks % kUAcc) * HP), a_base + (uint64_t)(ks * (2048 >> 4)),
-                        b_base + (uint64_t)((ks >> 2) * (HP * 128 >> 4) + (ks & 3) * 2), idesc_u,
-                        !(first_of_seg && ks < kUAcc));
-            umma_commit(smem_u32(&tl->vempty[s]));
-          }
-          if (!ok) break;
-          umma_commit(smem_u32(&tl->u_done[pb]));
+          for (int ks = 0; ks < kRows / 16; ++ks)
+            umma_bf16(d + (uint32_t)((ks % kUAcc) * HP), a_base + (uint64_t)(ks * (2048 >> 4)),
+                      b_base + (uint64_t)((ks >> 2) * (HP * 128 >> 4) + (ks & 3) * 2), idesc_u,
+                      !(first_of_seg && ks < kUAcc));
+          umma_commit(smem_u32(&tl->vempty[s]));
         }
+        if (!ok) break;
+        umma_commit(smem_u32(&tl->u_done[pb]));
       }
-      umma_commit(smem_u32(&tl->drain));
-      (void)mbar_wait(smem_u32(&tl->drain), 0u, kWaitTimeoutNs / 8);
+      umma_commit(smem_u32(&tl->drain[1]));
+      (void)mbar_wait(smem_u32(&tl->drain[1]), 0u, kWaitTimeoutNs / 8);
     }
   } else {
     // --------------------------- softmax / epilogue ---------------------------

@@ -118,3 +118,37 @@ def test_full_size_sampled(name, B, H, N, r, decay):
                             seed=0)
     print(f"{name}: rel err {err:.2e}, lse err {lse_err:.2e}")
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dtype", [BF16, F32])
+def test_rows_beyond_N_are_never_read(dtype):
+    # Every cached row at or past N is NaN: one read of it would poison the
+    # softmax or the value sum.
+    B, H, d_h, N, n_cap, r = 3, 4, 64, 777, 900, 24
+    inp = make_decode_inputs(B, H, d_h, N, r, r, dtype, n_cap=n_cap, mu=True, seed=31)
+    inp["zk"][:, :, N:] = float("nan")
+    inp["zv"][:, :, N:] = float("nan")
+    out, lse = lla.lla_decode_attn(inp["q"], inp["zk"], inp["zv"], inp["dk"], inp["dv"], N=N,
+                                   mu_k_t=inp["mu_k"], mu_v_t=inp["mu_v"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    units = [(b, h) for b in range(B) for h in range(H)]
+    ref_out, ref_lse = oracle_reference(inp, units)
+    compare(out, lse, units, ref_out, ref_lse, dtype)
+
+
+def test_kernel_timer_brackets_the_streaming_kernel():
+    inp = make_decode_inputs(64, 16, 128, 2048, 128, 128, BF16, seed=5)
+    args = (inp["q"], inp["zk"], inp["zv"], inp["dk"], inp["dv"])
+    lla.lla_decode_attn(*args)
+    call0, call1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with lla.kernel_timer() as kt:
+        call0.record()
+        lla.lla_decode_attn(*args)
+        call1.record()
+    torch.cuda.synchronize()
+    call_ms = call0.elapsed_time(call1)
+    assert 0 < kt.ms <= call_ms
+    # after the block the hook is cleared: a plain call records nothing new
+    lla.lla_decode_attn(*args)
+    torch.cuda.synchronize()

@@ -77,3 +77,17 @@ def test_full_size_sampled():
     # LLA-2D workload: H=16, d_h=128, r_k=r_v=256, batch 256, context 8192
     err = run(256, 16, 128, 8192, 256, 256, units=sample_units(256, 16), decay=True, seed=0)
     print(f"lla2d full size: rel err {err:.2e}")
+
+
+def test_rows_beyond_N_are_never_read():
+    B, H, d_h, N, n_cap = 3, 16, 128, 300, 384
+    inp = make_decode_inputs(B, H, d_h, N, 256, 256, BF16, two_d=True, n_cap=n_cap, mu=True, seed=13)
+    inp["zk"][:, N:] = float("nan")
+    inp["zv"][:, N:] = float("nan")
+    out, lse = lla.lla2d_decode_attn(inp["q"], inp["zk"], inp["zv"], inp["dk"], inp["dv"], N=N,
+                                     mu_k_t=inp["mu_k"], mu_v_t=inp["mu_v"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    units = [(b, h) for b in range(B) for h in range(H)]
+    ref_out, ref_lse = oracle_reference(inp, units, two_d=True)
+    compare(out, lse, units, ref_out, ref_lse, BF16)
