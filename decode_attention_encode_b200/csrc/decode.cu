@@ -22,6 +22,8 @@
 //              mass and applies W^V_up,t once: out = W^V (u / l) + mu^V.
 // k_stream and k_combine are launched with programmatic dependent launch, so
 // the latent copies of k_stream start while k_absorb is still running.
+#include <cuda_bf16.h>
+
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
@@ -29,6 +31,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "stream.cuh"
+#include "tc.cuh"
 
 namespace lla {
 namespace {
@@ -53,8 +56,10 @@ struct AbsorbArgs {
   int B, H, d_h, r_k;
   float qscale;  // scale * log2(e): scores leave k_stream in log2 units
   float scale;
-  float* qp;  // [B*H][r_k]
+  float* qp;  // [B*H][r_k], or null
   float* c0;  // [B*H], natural-log units
+  unsigned char* qsw;  // LLA-2D MMA operand copy of q' (bf16, swizzled), or null
+  int hp;              // its rows (heads padded to the MMA N)
 };
 
 // One CTA per (head, 32 latent columns, 8*ROWS batch rows). The CTA stages
@@ -116,7 +121,19 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
 #pragma unroll
     for (int k = 0; k < ROWS; ++k) {
       const int bb = warp * ROWS + k;
-      if (bb < nb) a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = acc[k] * a.qscale;
+      if (bb >= nb) continue;
+      const float v = acc[k] * a.qscale;
+      if (a.qp) a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = v;
+      if (a.qsw) {
+        unsigned char* base = a.qsw + (size_t)(b0 + bb) * (a.r_k / 64) * a.hp * 128;
+        *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c0 + lane, a.hp)) =
+            __float2bfloat16_rn(v);
+        // the last head's CTAs also clear the padding rows h >= H
+        if (h == a.H - 1)
+          for (int hz = a.H; hz < a.hp; ++hz)
+            *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c0 + lane, a.hp)) =
+                __float2bfloat16_rn(0.f);
+      }
     }
   }
 }
@@ -243,8 +260,9 @@ int env_int(const char* name, int dflt) {
 }
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
-                         int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream) {
-  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0};
+                         int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
+                         unsigned char* qsw, int hp) {
+  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp};
   const int ncol = (r_k + 31) / 32;
   const int rows = rows_per_thread(H * ncol, B);
   dim3 grid(H, ncol, (B + 8 * rows - 1) / (8 * rows));

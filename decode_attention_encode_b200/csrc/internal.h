@@ -71,8 +71,13 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
                       float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // Kernels shared by the per-head and LLA-2D decode paths (decode.cu).
+// k_absorb writes q' (fp32, [B*H][r_k]) to qp when qp is non-null, and when
+// qsw is non-null also the bf16 copy LLA-2D stages per sequence: for each b,
+// an hp x r_k K-major 128B-swizzled operand (rows >= H zero), r_k a
+// multiple of 64, at qsw + b * (r_k / 64) * hp * 128.
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
-                         int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream);
+                         int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
+                         unsigned char* qsw = nullptr, int hp = 0);
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
                           long long P, int shared, float* out, float* lse, cudaStream_t stream);

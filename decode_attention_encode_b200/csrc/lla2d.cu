@@ -64,7 +64,7 @@ struct D2Args {
   int r_k, r_v, nkg, nvg, nks, nvs;  // groups per tile; stages per ring
   int off_q, off_p, off_tail, qbuf_bytes, pbuf_bytes;
   uint32_t tmem_cols;
-  const float* qp;
+  const unsigned char* qsw;  // per sequence: Q' as bf16 in the MMA operand layout
   float* part;
   int pstride;
   unsigned int* status;
@@ -110,13 +110,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[15]))
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// byte offset of element (row, col) in a K-major 128B-swizzled operand made
-// of 64-column chunks of `rows_per_chunk` rows
-__device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows_per_chunk) {
-  return (uint32_t)((col >> 6) * rows_per_chunk * 128 + row * 128) +
-         ((uint32_t)((col & 63) * 2) ^ (uint32_t)((row & 7) << 4));
 }
 
 template <int HP>
@@ -201,21 +194,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
+    // Q' of sequence b arrives by one bulk copy: k_absorb already wrote it
+    // as bf16 in the swizzled K-major layout the score MMA reads.
+    int q_issued = -1;  // last sequence segment whose Q' copy was issued
     auto stage_q = [&](int seg, int b) -> bool {
       const int qb = seg & 1;
       const bool ok = __all_sync(
           0xffffffffu,
           wait_ab(smem_u32(&tl->q_empty[qb]), (uint32_t)((seg >> 1) & 1) ^ 1u, abort_flag, a.status));
       if (!ok) return false;
-      unsigned char* qs = smem + a.off_q + qb * a.qbuf_bytes;
-      for (int idx = lane; idx < HP * a.r_k; idx += 32) {
-        const int h = idx / a.r_k, c = idx - h * a.r_k;
-        const float v = h < a.H ? a.qp[((size_t)b * a.H + h) * a.r_k + c] : 0.f;
-        *reinterpret_cast<__nv_bfloat16*>(qs + sw128_off(h, c, HP)) = __float2bfloat16_rn(v);
+      if (lane == 0) {
+        const uint32_t qfull = smem_u32(&tl->q_full[qb]);
+        mbar_arrive_expect_tx(qfull, (uint32_t)a.qbuf_bytes);
+        bulk_g2s(s_q0 + (uint32_t)(qb * a.qbuf_bytes), a.qsw + (size_t)b * a.qbuf_bytes,
+                 (uint32_t)a.qbuf_bytes, qfull, l2_evict_first_policy());
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tl->q_full[qb]));
+      q_issued = seg;
       return true;
     };
 
@@ -246,6 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int first = max(0, it - nring);
       for (int i = first; i < it; ++i)
         (void)mbar_wait(smem_u32(&fullb[i % nring]), (uint32_t)(i / nring) & 1u,
+                        kWaitTimeoutNs / 8);
+      if (is_k && q_issued >= 0)  // the last Q' copy may still be landing
+        (void)mbar_wait(smem_u32(&tl->q_full[q_issued & 1]), (uint32_t)((q_issued >> 1) & 1),
                         kWaitTimeoutNs / 8);
     }
   } else if (warp == 1) {
@@ -532,7 +529,7 @@ struct D2Plan {
   size_t smem;
   uint32_t tmem_cols;
   int pstride;
-  size_t off_qp, off_c0, off_part, ws_bytes;
+  size_t off_qsw, off_c0, off_part, ws_bytes;
 };
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -570,8 +567,8 @@ lla_status plan_2d(int B, int H, int N, int r_k, int r_v, D2Plan* p) {
   d.tmem_cols = c;
   d.pstride = 4 + r_v;
   const size_t units = (size_t)B * H;
-  d.off_qp = 0;
-  d.off_c0 = al256(units * r_k * sizeof(float));
+  d.off_qsw = 0;
+  d.off_c0 = al256((size_t)B * d.qbuf_bytes);
   d.off_part = al256(d.off_c0 + units * sizeof(float));
   d.ws_bytes = al256(d.off_part + ((size_t)d.grid + B) * H * d.pstride * sizeof(float));
   *p = d;
@@ -596,7 +593,7 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
   if (ws == nullptr || ws_bytes < d.ws_bytes)
     return fail(LLA_ERR_WORKSPACE, "LLA-2D workspace needs %zu bytes, got %zu", d.ws_bytes, ws_bytes);
   char* wsb = static_cast<char*>(ws);
-  float* qp = reinterpret_cast<float*>(wsb + d.off_qp);
+  unsigned char* qsw = reinterpret_cast<unsigned char*>(wsb + d.off_qsw);
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
 
@@ -614,7 +611,7 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
 
-  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, nullptr, c0, stream, qsw, d.hp);
   if (st != LLA_OK) return st;
 
   D2Args a{};
@@ -636,7 +633,7 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
   a.qbuf_bytes = d.qbuf_bytes;
   a.pbuf_bytes = d.pbuf_bytes;
   a.tmem_cols = d.tmem_cols;
-  a.qp = qp;
+  a.qsw = qsw;
   a.part = part;
   a.pstride = d.pstride;
   a.status = status_word();

@@ -116,6 +116,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Byte offset of element (row, col) of a bf16 K-major operand with 128-byte
+// swizzle, stored as 64-column chunks of `rows_per_chunk` rows each (the
+// layout a tiled TMA load with SWIZZLE_128B writes, and the one
+// desc_kmajor_sw128 describes).
+__host__ __device__ __forceinline__ uint32_t sw128_off(int row, int col, int rows_per_chunk) {
+  return (uint32_t)((col >> 6) * rows_per_chunk * 128 + row * 128) +
+         ((uint32_t)((col & 63) * 2) ^ (uint32_t)((row & 7) << 4));
+}
+
 // Makes generic-proxy writes to shared memory visible to the async proxy
 // (tensor cores, TMA) before they read it.
 __device__ __forceinline__ void fence_proxy_async_smem() {
