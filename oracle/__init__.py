@@ -22,6 +22,10 @@ What is here, each in fp64:
     per-loop mean, take the top-r right singular vectors of the stacked-loop
     matrix as W_down, and its loop slices as the initial W_up,t.
   * ``compression_ratio``: §3 Eq. 4.
+  * ``kept_positions`` / ``paged_decode``: the per-head decode over a paged
+    store with per-sequence lengths (a gather of each unit's rows, then the
+    explicit-reconstruction unit), with the attention-sink + window eviction
+    the pages compose with LLA (§7 "Memory", App. C).
 
 The decode and encode arithmetic lives in ``lla_oracle.c`` (plain C, no
 BLAS). ``svd_init`` uses numpy's LAPACK SVD as a library step.
@@ -222,6 +226,60 @@ def _decode(q, zk, zv, dk, dv, mu_k, mu_v, scale, N, units, nthreads, shared_lat
         None if mu_v is None else np.asarray(mu_v)[hs], scale, nthreads)
     if len(units) == B * H and list(units) == [(b, h) for b in range(B) for h in range(H)]:
         return out.reshape(B, H, d), lse.reshape(B, H)
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# ragged and paged latent stores, sequence-axis eviction
+# --------------------------------------------------------------------------
+
+def kept_positions(N, sink=0, window=0):
+    """Cached-token positions a sequence of N tokens attends.
+
+    With window > 0 this is the attention-sink + recent-window index set that
+    the pages stack on LLA (§7 "Memory"; App. C Table 9: a 260-token budget
+    of 4 sink tokens plus a 256-token window): the first ``sink`` tokens and
+    the last ``window`` tokens, or all N when N <= sink + window. With
+    window <= 0 nothing is evicted and all N positions are kept."""
+    N, sink, window = int(N), max(0, int(sink)), int(window)
+    if window <= 0 or N <= sink + window:
+        return np.arange(N, dtype=np.int64)
+    return np.concatenate([np.arange(sink, dtype=np.int64),
+                           np.arange(N - window, N, dtype=np.int64)])
+
+
+def paged_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=None,
+                 mu_v=None, scale=None, sink=0, window=0, nthreads: int = 0):
+    """Per-head LLA decode over a paged latent store with per-sequence lengths.
+
+    q [B, H, d]; zk_pages [P, H, page_size, r_k]; zv_pages [P, H, page_size,
+    r_v]; block_table [B, max_blocks] page indices; seq_lens [B]. Token j of
+    sequence b, head h is row j % page_size of head h in page
+    block_table[b, j // page_size]. Sequence b attends the positions
+    ``kept_positions(seq_lens[b], sink, window)``: each (b, h) unit gathers
+    those rows and goes through the explicit-reconstruction unit (§3 Eq. 3,
+    then textbook attention). The pages leave attention over an empty set
+    undefined; this oracle reads it as no attention mass: out = 0 and
+    lse = -inf, the neutral element of a log-sum-exp merge.
+    Returns out [B, H, d], lse [B, H]."""
+    q = np.asarray(q)
+    B, H, d = q.shape
+    zk_pages, zv_pages = np.asarray(zk_pages), np.asarray(zv_pages)
+    block_table, seq_lens = np.asarray(block_table), np.asarray(seq_lens)
+    ps = zk_pages.shape[2]
+    out = np.zeros((B, H, d))
+    lse = np.full((B, H), -np.inf)
+    for b in range(B):
+        pos = kept_positions(int(seq_lens[b]), sink, window)
+        if pos.size == 0:
+            continue
+        pages = block_table[b, pos // ps]
+        rows = pos % ps
+        # gathered [n, H, r] -> per-head [H, n, r]
+        zk_u = np.transpose(zk_pages[pages, :, rows], (1, 0, 2))
+        zv_u = np.transpose(zv_pages[pages, :, rows], (1, 0, 2))
+        o, l = decode_units(q[b], zk_u, zv_u, dk, dv, mu_k, mu_v, scale, nthreads)
+        out[b], lse[b] = o, l
     return out, lse
 
 

@@ -364,3 +364,144 @@ def test_capacity_ratios_follow_the_scalar_reduction():
     # bytes of the build's 21.3x workload store (24 layers, batch 768, 4k)
     store = 24 * 768 * 4096 * 16 * 48 * 2
     assert store / 1e9 == pytest.approx(115.96, abs=0.01)
+
+
+# ---------------------------------------------------------------------------
+# paged / ragged store and sink + window eviction
+# ---------------------------------------------------------------------------
+
+def test_kept_positions_match_the_printed_eviction_budget():
+    g = json.load(open(GOLDEN))["eviction_budget_gsm8k"]
+    N = g["prompt_tokens_approx"]
+    pos = oracle.kept_positions(N, g["sink"], g["window"])
+    assert pos.size == g["budget"] == g["sink"] + g["window"]
+    assert list(pos[:g["sink"]]) == list(range(g["sink"]))
+    assert list(pos[g["sink"]:]) == list(range(N - g["window"], N))
+    assert abs(1 - pos.size / N - g["evicted_fraction_approx"]) < 0.01
+    # the budget caps the set; shorter sequences keep everything
+    assert list(oracle.kept_positions(200, 4, 256)) == list(range(200))
+    assert list(oracle.kept_positions(260, 4, 256)) == list(range(260))
+    assert list(oracle.kept_positions(50, 0, 0)) == list(range(50))
+    assert oracle.kept_positions(0, 4, 256).size == 0
+
+
+def _paged_store(r, B, H, d, ps, lens, r_k=16, r_v=24, mu=True, spare=3):
+    """Dense per-sequence stores scattered into a shuffled page pool."""
+    maxb = max(1, max((n + ps - 1) // ps for n in lens))
+    npages = B * maxb + spare
+    order = r.permutation(npages)
+    bt = np.full((B, maxb), -1, dtype=np.int64)
+    zkp = r.standard_normal((npages, H, ps, r_k))
+    zvp = r.standard_normal((npages, H, ps, r_v))
+    dense_k = r.standard_normal((B, H, maxb * ps, r_k))
+    dense_v = r.standard_normal((B, H, maxb * ps, r_v))
+    k = 0
+    for b in range(B):
+        for blk in range((lens[b] + ps - 1) // ps):
+            pg = order[k]; k += 1
+            bt[b, blk] = pg
+            zkp[pg] = dense_k[b, :, blk * ps:(blk + 1) * ps]
+            zvp[pg] = dense_v[b, :, blk * ps:(blk + 1) * ps]
+    q = r.standard_normal((B, H, d)) / np.sqrt(d)
+    dk = r.standard_normal((H, d, r_k)) / np.sqrt(r_k)
+    dv = r.standard_normal((H, d, r_v)) / np.sqrt(r_v)
+    mk = r.standard_normal((H, d)) if mu else None
+    mv = r.standard_normal((H, d)) if mu else None
+    return dict(q=q, zkp=zkp, zvp=zvp, bt=bt, dense_k=dense_k, dense_v=dense_v, dk=dk, dv=dv,
+                mk=mk, mv=mv)
+
+
+def test_paged_equals_dense_decode_per_sequence_length():
+    r = rng(41)
+    lens = [1, 7, 8, 9, 23, 0, 16]
+    B, H, d, ps = len(lens), 3, 8, 8
+    s = _paged_store(r, B, H, d, ps, lens)
+    out, lse = oracle.paged_decode(s["q"], s["zkp"], s["zvp"], s["bt"], lens, s["dk"], s["dv"],
+                                   s["mk"], s["mv"])
+    for b, n in enumerate(lens):
+        if n == 0:
+            continue
+        ob, lb = oracle.lla_decode(s["q"][b:b + 1], s["dense_k"][b:b + 1], s["dense_v"][b:b + 1],
+                                   s["dk"], s["dv"], s["mk"], s["mv"], N=n)
+        np.testing.assert_allclose(out[b], ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=1e-12)
+
+
+def test_paged_single_token_is_the_reconstruction_from_its_page():
+    # one cached token: out is that token's reconstructed value, read from
+    # head h of the page the block table names (§3 Eq. 3)
+    r = rng(42)
+    B, H, d, ps = 3, 4, 6, 5
+    s = _paged_store(r, B, H, d, ps, [1, 1, 1])
+    out, lse = oracle.paged_decode(s["q"], s["zkp"], s["zvp"], s["bt"], [1, 1, 1], s["dk"],
+                                   s["dv"], s["mk"], s["mv"])
+    for b in range(B):
+        pg = s["bt"][b, 0]
+        for h in range(H):
+            vhat = s["dv"][h] @ s["zvp"][pg, h, 0] + s["mv"][h]
+            khat = s["dk"][h] @ s["zkp"][pg, h, 0] + s["mk"][h]
+            np.testing.assert_allclose(out[b, h], vhat, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[b, h], s["q"][b, h] @ khat / np.sqrt(d), atol=1e-12)
+
+
+def test_paged_page_relabelling_and_unused_pages_do_not_matter():
+    r = rng(43)
+    lens = [13, 4, 30]
+    B, H, d, ps = 3, 2, 8, 4
+    s = _paged_store(r, B, H, d, ps, lens)
+    out, lse = oracle.paged_decode(s["q"], s["zkp"], s["zvp"], s["bt"], lens, s["dk"], s["dv"])
+    perm = r.permutation(s["zkp"].shape[0])
+    inv = np.argsort(perm)
+    bt2 = np.where(s["bt"] >= 0, inv[np.maximum(s["bt"], 0)], -1)
+    zk2, zv2 = s["zkp"][perm].copy(), s["zvp"][perm].copy()
+    used = set(bt2[bt2 >= 0].tolist())
+    for pg in range(zk2.shape[0]):
+        if pg not in used:
+            zk2[pg] = np.nan
+            zv2[pg] = np.nan
+    # rows past each sequence's length inside its last page are never read
+    for b, n in enumerate(lens):
+        if n % ps:
+            zk2[bt2[b, n // ps], :, n % ps:] = np.nan
+            zv2[bt2[b, n // ps], :, n % ps:] = np.nan
+    out2, lse2 = oracle.paged_decode(s["q"], zk2, zv2, bt2, lens, s["dk"], s["dv"])
+    np.testing.assert_allclose(out2, out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse, rtol=0, atol=1e-12)
+
+
+def test_paged_eviction_attends_exactly_the_kept_positions():
+    r = rng(44)
+    lens = [40, 9, 26]
+    sink, window = 3, 6
+    B, H, d, ps = 3, 2, 8, 4
+    s = _paged_store(r, B, H, d, ps, lens, mu=True)
+    out, lse = oracle.paged_decode(s["q"], s["zkp"], s["zvp"], s["bt"], lens, s["dk"], s["dv"],
+                                   s["mk"], s["mv"], sink=sink, window=window)
+    for b, n in enumerate(lens):
+        pos = oracle.kept_positions(n, sink, window)
+        assert pos.size == min(n, sink + window)
+        ob, lb = oracle.lla_decode(s["q"][b:b + 1], s["dense_k"][b:b + 1, :, pos],
+                                   s["dense_v"][b:b + 1, :, pos], s["dk"], s["dv"], s["mk"],
+                                   s["mv"])
+        np.testing.assert_allclose(out[b], ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=1e-12)
+    # evicted tokens may hold anything
+    zk2, zv2 = s["zkp"].copy(), s["zvp"].copy()
+    for b, n in enumerate(lens):
+        kept = set(oracle.kept_positions(n, sink, window).tolist())
+        for j in range(n):
+            if j not in kept:
+                zk2[s["bt"][b, j // ps], :, j % ps] = 1e3
+                zv2[s["bt"][b, j // ps], :, j % ps] = -1e3
+    out2, lse2 = oracle.paged_decode(s["q"], zk2, zv2, s["bt"], lens, s["dk"], s["dv"], s["mk"],
+                                     s["mv"], sink=sink, window=window)
+    np.testing.assert_allclose(out2, out, rtol=0, atol=1e-12)
+
+
+def test_paged_empty_sequence_has_no_attention_mass():
+    r = rng(45)
+    s = _paged_store(r, 2, 2, 4, 4, [0, 5])
+    out, lse = oracle.paged_decode(s["q"], s["zkp"], s["zvp"], s["bt"], [0, 5], s["dk"], s["dv"],
+                                   s["mk"], s["mv"])
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(np.isfinite(out[1])) and np.all(np.isfinite(lse[1]))
