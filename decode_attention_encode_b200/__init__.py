@@ -20,6 +20,8 @@ from ._lib import (  # noqa: F401
     lla2d_decode_attn_workspace,
     lla_decode_attn,
     lla_decode_attn_noalloc,
+    lla_decode_attn_paged,
+    lla_decode_attn_paged_workspace,
     lla_decode_attn_workspace,
     lla_encode,
 )

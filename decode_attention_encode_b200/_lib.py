@@ -27,12 +27,14 @@ LLA_F32 = 0
 LLA_BF16 = 1
 
 LLA_DEVICE_WAIT_TIMEOUT = 0x1
+LLA_DEVICE_BAD_PAGED_INPUT = 0x2
 
 # Every symbol include/lla.h declares.
 EXPORTS = (
     "lla_status_string", "lla_last_error", "lla_version", "lla_device_status",
     "lla_set_timing_events",
     "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
+    "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn",
     "lla_encode",
 )
@@ -57,6 +59,10 @@ _SIGS = {
     "lla_device_status": ([ctypes.POINTER(ctypes.c_uint), _c_int], _c_int),
     "lla_set_timing_events": ([_vp, _vp], None),
     "lla_decode_attn_workspace": ([_c_int] * 5, _c_size),
+    "lla_decode_attn_paged_workspace": ([_c_int] * 4, _c_size),
+    "lla_decode_attn_paged": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp, _c_int, _vp] +
+                              [_c_int] * 2 + [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp],
+                              _c_int),
     "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
                         [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
@@ -222,6 +228,48 @@ def lla_decode_attn_noalloc(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=N
                                        N, n_cap, r_k, r_v, _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t),
                                        _ptr(mu_v_t), float(scale), _ptr(out), _ptr(lse),
                                        _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def lla_decode_attn_paged_workspace(B, H, r_k, r_v):
+    return int(lib().lla_decode_attn_paged_workspace(B, H, r_k, r_v))
+
+
+def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t=None,
+                          mu_v_t=None, scale=None, sink=0, window=0, out=None, lse=None,
+                          workspace=None, stream=None, want_lse=True):
+    """Per-head absorbed decode over a paged store with per-sequence lengths.
+
+    q [B,H,d_h] fp32; zk_pages [P,H,page_size,r_k], zv_pages [P,H,page_size,r_v]
+    bf16 or fp32; block_table [B,max_blocks] int32 and seq_lens [B] int32 on
+    the device; sink, window: the eviction set (window 0 keeps every token).
+    Returns (out [B,H,d_h], lse [B,H] or None)."""
+    _need_cuda(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, out,
+               lse, workspace)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise LLAError(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be int32")
+    if not (block_table.is_contiguous() and seq_lens.is_contiguous()):
+        raise LLAError(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be contiguous")
+    B, H, d_h = q.shape
+    num_pages, page_size, r_k = zk_pages.shape[0], zk_pages.shape[2], zk_pages.shape[3]
+    r_v = zv_pages.shape[3]
+    max_blocks = block_table.shape[1]
+    scale = 1.0 / math.sqrt(d_h) if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, d_h), device=q.device, dtype=torch.float32)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    h = lib()
+    need = int(h.lla_decode_attn_paged_workspace(B, H, r_k, r_v))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    st = h.lla_decode_attn_paged(_ptr(q), _ptr(zk_pages), _ptr(zv_pages), _dtype_code(zk_pages),
+                                 B, H, d_h, r_k, r_v, page_size, num_pages, _ptr(block_table),
+                                 max_blocks, _ptr(seq_lens), int(sink), int(window), _ptr(dk_t),
+                                 _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t), float(scale), _ptr(out),
+                                 _ptr(lse), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st)
     return out, lse
 

@@ -13,6 +13,7 @@ namespace lla {
 // return instead of hanging the GPU.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 constexpr unsigned int kStatusWaitTimeout = 0x1u;
+constexpr unsigned int kStatusBadPagedInput = 0x2u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

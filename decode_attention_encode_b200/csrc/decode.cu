@@ -152,6 +152,7 @@ struct CombineArgs {
   int shared;      // 1: one split per sequence shared by all heads (LLA-2D)
   float* out;
   float* lse;
+  RaggedMap ragged;  // seqinfo non-null: the paged plan's piece map
 };
 
 // One CTA per (head, 32 output channels, 8*ROWS batch rows). Warp w merges
@@ -163,6 +164,7 @@ struct CombineArgs {
 template <int ROWS>
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   extern __shared__ __align__(16) float sm_combine[];
+  __shared__ float s_keep[64];  // 0 for a row with no attended token
   const int pitch = a.r_v + 4;
   float* d_s = sm_combine;                        // [32][pitch]
   float* ub = sm_combine + 32 * pitch;            // [8*ROWS][r_v]
@@ -190,10 +192,27 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     }
     const long long u = (long long)(b0 + bb) * a.H + h;
     // The split runs over units (b, h) for per-head LLA and over sequences
-    // b for LLA-2D; piece w of split key k is partial record w + k.
+    // b for LLA-2D; piece w of split key k is partial record w + k. A
+    // ragged plan places unit (b, h) at cum[b] + h * n_b in the range.
     const long long key = a.shared ? (long long)(b0 + bb) : u;
-    const long long wf = (key * a.N) / a.P;
-    const long long wl = ((key + 1) * a.N - 1) / a.P;
+    long long wf, wl;
+    if (a.ragged.seqinfo) {
+      const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
+      if (n == 0) {  // nothing attended: out = 0, lse = -inf
+        for (int c4 = lane; c4 < r4; c4 += 32) urow[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0) s_keep[bb] = 0.f;
+        if (blockIdx.y == 0 && lane == 0 && a.lse) a.lse[u] = -INFINITY;
+        continue;
+      }
+      const long long P = a.ragged.plan[1];
+      const long long first = a.ragged.cum[b0 + bb] + (long long)h * n;
+      wf = first / P;
+      wl = (first + n - 1) / P;
+    } else {
+      wf = (key * a.N) / a.P;
+      wl = ((key + 1) * a.N - 1) / a.P;
+    }
+    if (lane == 0) s_keep[bb] = 1.f;
     const int np = (int)(wl - wf + 1);
     const float* rec0 = a.shared ? a.part + ((wf + key) * a.H + h) * a.pstride
                                  : a.part + (wf + key) * a.pstride;
@@ -239,7 +258,7 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 #pragma unroll
     for (int k = 0; k < ROWS; ++k) {
       const int bb = warp * ROWS + k;
-      if (bb < nb) a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = acc[k] + mu;
+      if (bb < nb) a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = acc[k] + mu * s_keep[bb];
     }
   }
 }
@@ -278,11 +297,14 @@ lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int
 
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
-                          long long P, int shared, float* out, float* lse, cudaStream_t stream) {
+                          long long P, int shared, float* out, float* lse, cudaStream_t stream,
+                          const RaggedMap* ragged) {
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse};
+  CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse,
+                RaggedMap{nullptr, nullptr, nullptr}};
+  if (ragged) a.ragged = *ragged;
   const int nch = (d_h + 31) / 32;
   const int rows = rows_per_thread(H * nch, B);
   cudaLaunchConfig_t cfg{};

@@ -70,6 +70,25 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
                       const float* dv, const float* mu_k, const float* mu_v, float scale,
                       float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Piece map of a ragged (paged) plan, all device arrays written by
+// k_plan_paged: per-sequence records {kept tokens n, sink part, gap, 0},
+// the flattened range's prefix sums [B+1] and {total, tokens per warp}.
+struct RaggedMap {
+  const int4* seqinfo;
+  const long long* cum;
+  const long long* plan;
+};
+
+size_t workspace_paged(int B, int H, int r_k, int r_v, int esz);
+lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int esz, int B, int H,
+                            int d_h, int r_k, int r_v, int page_size, int num_pages,
+                            const int* block_table, int max_blocks, const int* seq_lens, int sink,
+                            int window, const float* dk, const float* dv, const float* mu_k,
+                            const float* mu_v, float scale, float* out, float* lse, void* ws,
+                            size_t ws_bytes, cudaStream_t stream);
+
 // Kernels shared by the per-head and LLA-2D decode paths (decode.cu).
 // k_absorb writes q' (fp32, [B*H][r_k]) to qp when qp is non-null, and when
 // qsw is non-null also the bf16 copy LLA-2D stages per sequence: for each b,
@@ -80,7 +99,8 @@ lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int
                          unsigned char* qsw = nullptr, int hp = 0);
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
-                          long long P, int shared, float* out, float* lse, cudaStream_t stream);
+                          long long P, int shared, float* out, float* lse, cudaStream_t stream,
+                          const RaggedMap* ragged = nullptr);
 
 size_t workspace_2d(int B, int H, int N, int r_k, int r_v);
 lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,

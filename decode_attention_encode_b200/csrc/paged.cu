@@ -1,0 +1,280 @@
+// Per-head absorbed LLA decode over a paged latent store with per-sequence
+// lengths (sm_100a).
+//
+// Source: "Looped Latent Attention: Cross-Loop KV Compression for Looped
+// Transformers" (arXiv 2607.15456), §7 "Per-head LLA versus LLA-2D at
+// inference" (the absorbed form) and §7 "Memory" / App. C Table 9 (LLA
+// stacks with attention-sink + window eviction: the sequence keeps its first
+// `sink` tokens and its last `window`). The pages measure capacity with a
+// latent store; keeping it in fixed-size pages shared by sequences of
+// different lengths is how a serving engine holds such a store.
+//
+// One call runs four kernels on the caller's stream:
+//   k_plan_paged  one CTA: reads the lengths, checks every used block-table
+//                 entry, forms each sequence's kept-token record, the
+//                 flattened range's prefix sums, each streaming warp's share
+//                 and its starting (sequence, head, token). Nothing goes back
+//                 to the host.
+//   k_absorb      as in the dense path.
+//   k_stream_paged  the dense streaming kernel's pipeline over the page pool.
+//   k_combine     as in the dense path, with the ragged piece map.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "stream.cuh"
+
+namespace lla {
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+struct PlanArgs {
+  const int* seq_lens;
+  const int* block_table;
+  int B, H, page_size, num_pages, max_blocks, sink, window;
+  int W;     // streaming warps
+  int pmin;  // smallest share per warp
+  int4* seqinfo;
+  long long* cum;
+  long long* plan;
+  int4* wstart;
+  unsigned int* status;
+};
+
+// Every page index the kept positions [lo, hi) of sequence b touch lies in
+// the pool.
+__device__ bool pages_ok(const PlanArgs& p, int b, int lo, int hi) {
+  if (lo >= hi) return true;
+  const int* row = p.block_table + (size_t)b * p.max_blocks;
+  for (int blk = lo / p.page_size; blk <= (hi - 1) / p.page_size; ++blk) {
+    const int pg = row[blk];
+    if (pg < 0 || pg >= p.num_pages) return false;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
+  __shared__ long long scan[kPlanThreads];
+  __shared__ long long s_total, s_P;
+  const int t = threadIdx.x;
+  const int chunk = (p.B + kPlanThreads - 1) / kPlanThreads;
+  const int b0 = min(p.B, t * chunk), b1 = min(p.B, b0 + chunk);
+  const long long cap = (long long)p.max_blocks * p.page_size;
+
+  // 1. per-sequence records; a sequence with a bad length or page is empty
+  long long sum = 0;
+  bool bad = false;
+  for (int b = b0; b < b1; ++b) {
+    const int N = p.seq_lens[b];
+    int n = 0, s = 0, gap = 0;
+    if (N >= 0 && N <= cap) {
+      n = N;
+      s = N;
+      if (p.window > 0 && N > p.sink + p.window) {
+        n = p.sink + p.window;
+        s = p.sink;
+        gap = N - n;
+      }
+      if (!pages_ok(p, b, 0, s) || !pages_ok(p, b, s + gap, N)) n = s = gap = -1;
+    } else {
+      n = s = gap = -1;
+    }
+    if (n < 0) {
+      bad = true;
+      n = s = gap = 0;
+    }
+    p.seqinfo[b] = make_int4(n, s, gap, 0);
+    sum += (long long)n * p.H;
+  }
+  if (bad) report_status(p.status, kStatusBadPagedInput);
+
+  // 2. prefix sums of the flattened (sequence, head, token) range
+  scan[t] = sum;
+  __syncthreads();
+  for (int off = 1; off < kPlanThreads; off <<= 1) {
+    const long long v = t >= off ? scan[t - off] : 0;
+    __syncthreads();
+    scan[t] += v;
+    __syncthreads();
+  }
+  long long run = scan[t] - sum;
+  for (int b = b0; b < b1; ++b) {
+    p.cum[b] = run;
+    run += (long long)p.seqinfo[b].x * p.H;
+  }
+  if (t == kPlanThreads - 1) {
+    const long long total = scan[t];
+    const long long P = max((long long)p.pmin, (total + p.W - 1) / p.W);
+    p.cum[p.B] = total;
+    p.plan[0] = total;
+    p.plan[1] = P;
+    s_total = total;
+    s_P = P;
+  }
+  __syncthreads();
+
+  // 3. each warp's first (sequence, head, kept index)
+  const long long total = s_total, P = s_P;
+  for (int w = t; w < p.W; w += kPlanThreads) {
+    const long long f0 = (long long)w * P;
+    int4 c = make_int4(0, 0, 0, 0);
+    if (f0 < total) {
+      int lo = 0, hi = p.B - 1;  // the last b with cum[b] <= f0 (never empty)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cum[mid] <= f0) lo = mid;
+        else hi = mid - 1;
+      }
+      const long long off = f0 - p.cum[lo];
+      const int n = p.seqinfo[lo].x;
+      const int h = (int)(off / n);
+      c = make_int4(lo, h, (int)(off - (long long)h * n), 0);
+    }
+    p.wstart[w] = c;
+  }
+}
+
+struct PagedPlan {
+  DecodePlan d;
+  size_t off_seqinfo, off_cum, off_plan, off_wstart, ws_bytes;
+};
+
+lla_status plan_paged(int B, int H, int r_k, int r_v, int esz, PagedPlan* pp) {
+  PagedPlan p{};
+  // kernel shape (lanes per token, tile, stages) does not depend on N
+  lla_status st = plan_decode(B, H, 1, r_k, r_v, esz, &p.d);
+  if (st != LLA_OK) return st;
+  const DeviceInfo di = device_info();
+  p.d.grid = di.sms;
+  p.d.W = di.sms * p.d.warps;
+  p.d.P = 0;  // set on the device
+  const long long units = (long long)B * H;
+  p.d.off_qp = 0;
+  p.d.off_c0 = align_up((size_t)units * r_k * sizeof(float), 256);
+  p.d.off_part = align_up(p.d.off_c0 + (size_t)units * sizeof(float), 256);
+  p.off_seqinfo =
+      align_up(p.d.off_part + (size_t)(p.d.W + units) * p.d.pstride * sizeof(float), 256);
+  p.off_cum = align_up(p.off_seqinfo + (size_t)B * sizeof(int4), 256);
+  p.off_plan = align_up(p.off_cum + (size_t)(B + 1) * sizeof(long long), 256);
+  p.off_wstart = align_up(p.off_plan + 2 * sizeof(long long), 256);
+  p.ws_bytes = align_up(p.off_wstart + (size_t)p.d.W * sizeof(int4), 256);
+  p.d.ws_bytes = p.ws_bytes;
+  *pp = p;
+  return LLA_OK;
+}
+
+}  // namespace
+
+size_t workspace_paged(int B, int H, int r_k, int r_v, int esz) {
+  PagedPlan p;
+  if (plan_paged(B, H, r_k, r_v, esz, &p) != LLA_OK) return 0;
+  return p.ws_bytes;
+}
+
+lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int esz, int B, int H,
+                            int d_h, int r_k, int r_v, int page_size, int num_pages,
+                            const int* block_table, int max_blocks, const int* seq_lens, int sink,
+                            int window, const float* dk, const float* dv, const float* mu_k,
+                            const float* mu_v, float scale, float* out, float* lse, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
+  PagedPlan pp;
+  lla_status st = plan_paged(B, H, r_k, r_v, esz, &pp);
+  if (st != LLA_OK) return st;
+  const DecodePlan& d = pp.d;
+  if (ws == nullptr || ws_bytes < pp.ws_bytes)
+    return fail(LLA_ERR_WORKSPACE, "paged decode workspace needs %zu bytes, got %zu", pp.ws_bytes,
+                ws_bytes);
+  char* wsb = static_cast<char*>(ws);
+  float* qp = reinterpret_cast<float*>(wsb + d.off_qp);
+  float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
+  float* part = reinterpret_cast<float*>(wsb + d.off_part);
+  int4* seqinfo = reinterpret_cast<int4*>(wsb + pp.off_seqinfo);
+  long long* cum = reinterpret_cast<long long*>(wsb + pp.off_cum);
+  long long* plan = reinterpret_cast<long long*>(wsb + pp.off_plan);
+  int4* wstart = reinterpret_cast<int4*>(wsb + pp.off_wstart);
+
+  StreamFn fn = pick_stream_kernel(esz, d.lpt, d.sk, d.exact, true);
+  if (!fn) return fail(LLA_ERR_UNSUPPORTED, "no decode kernel for this latent shape");
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)d.smem_bytes);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_stream_paged)");
+
+  // 1. plan (a plain launch: it completes before k_absorb starts, so the
+  //    streaming kernel may read its results before griddepcontrol.wait)
+  {
+    PlanArgs p{};
+    p.seq_lens = seq_lens;
+    p.block_table = block_table;
+    p.B = B;
+    p.H = H;
+    p.page_size = page_size;
+    p.num_pages = num_pages;
+    p.max_blocks = max_blocks;
+    p.sink = sink;
+    p.window = window;
+    p.W = d.W;
+    p.pmin = 2 * d.tile;
+    p.seqinfo = seqinfo;
+    p.cum = cum;
+    p.plan = plan;
+    p.wstart = wstart;
+    p.status = status_word();
+    k_plan_paged<<<1, kPlanThreads, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return check_cuda(e, "launch k_plan_paged");
+  }
+  // 2. absorb (plain launch)
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
+  if (st != LLA_OK) return st;
+  // 3. stream
+  {
+    StreamArgs a{};
+    a.zk = static_cast<const char*>(zk);
+    a.zv = static_cast<const char*>(zv);
+    a.W = d.W;
+    a.row_k = r_k * esz;
+    a.row_v = r_v * esz;
+    a.nseg_k = d.nseg_k;
+    a.nseg_v = d.nseg_v;
+    a.r_k = r_k;
+    a.tile = d.tile;
+    a.nstage = d.nstage;
+    a.stage_bytes = d.stage_bytes;
+    a.qp = qp;
+    a.part = part;
+    a.pstride = d.pstride;
+    a.status = status_word();
+    a.seqinfo = seqinfo;
+    a.cum = cum;
+    a.plan = plan;
+    a.wstart = wstart;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks;
+    a.page_size = page_size;
+    a.H = H;
+    a.B = B;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(d.grid);
+    cfg.blockDim = dim3(32 * d.warps);
+    cfg.dynamicSmemBytes = d.smem_bytes;
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = record_timing(true, stream);
+    if (e != cudaSuccess) return check_cuda(e, "record timing event");
+    e = cudaLaunchKernelEx(&cfg, fn, a);
+    if (e != cudaSuccess) return check_cuda(e, "launch k_stream_paged");
+    e = record_timing(false, stream);
+    if (e != cudaSuccess) return check_cuda(e, "record timing event");
+  }
+  // 4. combine over the ragged piece map
+  RaggedMap rm{seqinfo, cum, plan};
+  return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 0, out, lse, stream,
+                        &rm);
+}
+
+}  // namespace lla

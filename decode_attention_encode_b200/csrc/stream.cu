@@ -86,12 +86,102 @@ __device__ __forceinline__ void slot_update(float sc, const unsigned char* vrow,
   }
 }
 
+// Scores and online-softmax updates for the `len` tokens of one stage: token
+// slot `slot` takes tokens slot, slot + NS, ... two at a time.
+template <int ESZ, int LPT, int SK, int SV, bool EXACT>
+__device__ __forceinline__ void stream_tile(const unsigned char* Ks, const unsigned char* Vs,
+                                            int len, const float (&qv)[SK][16 / ESZ], float& m,
+                                            float& l, float (&acc)[SV][16 / ESZ],
+                                            const StreamArgs& a, int slot, int g) {
+  constexpr int E = 16 / ESZ;
+  constexpr int NS = 32 / LPT;
+  constexpr unsigned FULL = 0xffffffffu;
+  for (int t0 = 0; t0 < len; t0 += 2 * NS) {
+    const int ta = t0 + slot, tb = t0 + NS + slot;
+    const bool va = ta < len, vb = tb < len;
+    float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+#pragma unroll
+    for (int s = 0; s < SK; ++s) {
+      const int seg = s * LPT + g;
+      if (EXACT || seg < a.nseg_k) {
+        float x[E];
+        if (va) {
+          unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + ta * a.row_k + seg * 16), x);
+#pragma unroll
+          for (int e = 0; e < E; e += 2) {
+            sa0 = fmaf(qv[s][e], x[e], sa0);
+            sa1 = fmaf(qv[s][e + 1], x[e + 1], sa1);
+          }
+        }
+        if (vb) {
+          unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + tb * a.row_k + seg * 16), x);
+#pragma unroll
+          for (int e = 0; e < E; e += 2) {
+            sb0 = fmaf(qv[s][e], x[e], sb0);
+            sb1 = fmaf(qv[s][e + 1], x[e + 1], sb1);
+          }
+        }
+      }
+    }
+    float sa = sa0 + sa1, sb = sb0 + sb1;
+#pragma unroll
+    for (int o = LPT / 2; o > 0; o >>= 1) {
+      sa += __shfl_xor_sync(FULL, sa, o);
+      sb += __shfl_xor_sync(FULL, sb, o);
+    }
+    if (va) slot_update<ESZ, LPT, SV, EXACT>(sa, Vs + ta * a.row_v, m, l, acc, a.nseg_v, g);
+    if (vb) slot_update<ESZ, LPT, SV, EXACT>(sb, Vs + tb * a.row_v, m, l, acc, a.nseg_v, g);
+  }
+}
+
+// Merges the NS token slots of a warp (log-sum-exp butterfly) and writes the
+// piece's partial record (m, l, u) at pp.
+template <int ESZ, int LPT, int SV, bool EXACT>
+__device__ __forceinline__ void stream_merge_write(float m, float l, float (&acc)[SV][16 / ESZ],
+                                                   float* pp, const StreamArgs& a, int slot,
+                                                   int g) {
+  constexpr int E = 16 / ESZ;
+  constexpr unsigned FULL = 0xffffffffu;
+#pragma unroll
+  for (int o = LPT; o < 32; o <<= 1) {
+    const float mo = __shfl_xor_sync(FULL, m, o);
+    const float lo = __shfl_xor_sync(FULL, l, o);
+    const float M = fmaxf(m, mo);
+    const float wa = exp2f(m - M), wb = exp2f(mo - M);
+    l = l * wa + lo * wb;
+#pragma unroll
+    for (int s = 0; s < SV; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float ao = __shfl_xor_sync(FULL, acc[s][e], o);
+        acc[s][e] = acc[s][e] * wa + ao * wb;
+      }
+    m = M;
+  }
+  if (slot == 0) {
+    if (g == 0) {
+      pp[0] = m;
+      pp[1] = l;
+    }
+#pragma unroll
+    for (int s = 0; s < SV; ++s) {
+      const int seg = s * LPT + g;
+      if (EXACT || seg < a.nseg_v) {
+        float4* dst = reinterpret_cast<float4*>(pp + 4 + seg * E);
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4)
+          dst[e4] = make_float4(acc[s][4 * e4], acc[s][4 * e4 + 1], acc[s][4 * e4 + 2],
+                                acc[s][4 * e4 + 3]);
+      }
+    }
+  }
+}
+
 // ESZ: bytes per latent element. LPT: lanes per token. SK/SV: 16-byte
 // segments per lane for K/V. EXACT: nseg == LPT*S for both axes.
 template <int ESZ, int LPT, int SK, int SV, bool EXACT>
 __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
-  constexpr int E = 16 / ESZ;   // elements per 16-byte segment
-  constexpr int NS = 32 / LPT;  // token slots per warp
+  constexpr int E = 16 / ESZ;  // elements per 16-byte segment
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ __align__(128) unsigned char smem[];
 
@@ -185,42 +275,7 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
       const unsigned char* Ks = buf + cs * a.stage_bytes;
       const unsigned char* Vs = Ks + v_off;
 
-      for (int t0 = 0; t0 < len; t0 += 2 * NS) {
-        const int ta = t0 + slot, tb = t0 + NS + slot;
-        const bool va = ta < len, vb = tb < len;
-        float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-#pragma unroll
-        for (int s = 0; s < SK; ++s) {
-          const int seg = s * LPT + g;
-          if (EXACT || seg < a.nseg_k) {
-            float x[E];
-            if (va) {
-              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + ta * a.row_k + seg * 16), x);
-#pragma unroll
-              for (int e = 0; e < E; e += 2) {
-                sa0 = fmaf(qv[s][e], x[e], sa0);
-                sa1 = fmaf(qv[s][e + 1], x[e + 1], sa1);
-              }
-            }
-            if (vb) {
-              unpack16<ESZ>(*reinterpret_cast<const uint4*>(Ks + tb * a.row_k + seg * 16), x);
-#pragma unroll
-              for (int e = 0; e < E; e += 2) {
-                sb0 = fmaf(qv[s][e], x[e], sb0);
-                sb1 = fmaf(qv[s][e + 1], x[e + 1], sb1);
-              }
-            }
-          }
-        }
-        float sa = sa0 + sa1, sb = sb0 + sb1;
-#pragma unroll
-        for (int o = LPT / 2; o > 0; o >>= 1) {
-          sa += __shfl_xor_sync(FULL, sa, o);
-          sb += __shfl_xor_sync(FULL, sb, o);
-        }
-        if (va) slot_update<ESZ, LPT, SV, EXACT>(sa, Vs + ta * a.row_v, m, l, acc, a.nseg_v, g);
-        if (vb) slot_update<ESZ, LPT, SV, EXACT>(sb, Vs + tb * a.row_v, m, l, acc, a.nseg_v, g);
-      }
+      stream_tile<ESZ, LPT, SK, SV, EXACT>(Ks, Vs, len, qv, m, l, acc, a, slot, g);
       __syncwarp();
       --in_flight;
       if (pf < f1) issue();  // refill the stage just read
@@ -231,41 +286,8 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
       f += len;
     }
 
-    // Merge the NS token slots of this warp (log-sum-exp butterfly).
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) {
-      const float mo = __shfl_xor_sync(FULL, m, o);
-      const float lo = __shfl_xor_sync(FULL, l, o);
-      const float M = fmaxf(m, mo);
-      const float wa = exp2f(m - M), wb = exp2f(mo - M);
-      l = l * wa + lo * wb;
-#pragma unroll
-      for (int s = 0; s < SV; ++s)
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const float ao = __shfl_xor_sync(FULL, acc[s][e], o);
-          acc[s][e] = acc[s][e] * wa + ao * wb;
-        }
-      m = M;
-    }
-    if (slot == 0) {
-      float* pp = a.part + (size_t)(w + u) * a.pstride;
-      if (g == 0) {
-        pp[0] = m;
-        pp[1] = l;
-      }
-#pragma unroll
-      for (int s = 0; s < SV; ++s) {
-        const int seg = s * LPT + g;
-        if (EXACT || seg < a.nseg_v) {
-          float4* dst = reinterpret_cast<float4*>(pp + 4 + seg * E);
-#pragma unroll
-          for (int e4 = 0; e4 < E / 4; ++e4)
-            dst[e4] = make_float4(acc[s][4 * e4], acc[s][4 * e4 + 1], acc[s][4 * e4 + 2],
-                                  acc[s][4 * e4 + 3]);
-        }
-      }
-    }
+    stream_merge_write<ESZ, LPT, SV, EXACT>(m, l, acc, a.part + (size_t)(w + u) * a.pstride, a,
+                                            slot, g);
     ++u;
 #pragma unroll
     for (int s = 0; s < SK; ++s)
@@ -275,32 +297,225 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
 }
 
 
+// ---------------------------------------------------------------------------
+// paged / ragged store
+// ---------------------------------------------------------------------------
 
-template <int ESZ>
+// Position in the flattened range of a paged plan: sequence b, head h, kept
+// index i, and sequence b's record (kept tokens n, sink part s, gap).
+struct PCursor {
+  int b, h, i;
+  int n, s, gap;
+};
+
+__device__ __forceinline__ void pc_load_seq(PCursor& c, const StreamArgs& a) {
+  const int4 v = __ldg(a.seqinfo + c.b);
+  c.n = v.x;
+  c.s = v.y;
+  c.gap = v.z;
+}
+
+// Tokens of the next tile: at most `tile`, and ending no later than the
+// warp's range, the unit, the sink part and the page.
+__device__ __forceinline__ int pc_len(const PCursor& c, long long f, long long f1, int tile,
+                                      int page_size) {
+  int lim = (int)min((long long)tile, f1 - f);
+  lim = min(lim, (c.i < c.s ? c.s : c.n) - c.i);
+  const int pos = c.i < c.s ? c.i : c.i + c.gap;
+  return min(lim, page_size - pos % page_size);
+}
+
+// Moves the cursor `len` tokens on; len never crosses a unit end, and at one
+// the cursor moves to the next head, or the next non-empty sequence.
+__device__ __forceinline__ void pc_advance(PCursor& c, int len, const StreamArgs& a) {
+  c.i += len;
+  if (c.i == c.n) {
+    c.i = 0;
+    if (++c.h == a.H) {
+      c.h = 0;
+      do {
+        ++c.b;
+      } while (c.b < a.B && __ldg(&a.seqinfo[c.b].x) == 0);
+      if (c.b < a.B) pc_load_seq(c, a);
+    }
+  }
+}
+
+// The streaming kernel over a paged store [pages][H][page_size][r] with
+// per-sequence lengths and the optional sink + window eviction set. The
+// flattened range, each warp's share P and each warp's starting cursor come
+// from k_plan_paged, which finished before k_absorb started, so they are
+// read before griddepcontrol.wait. Tiles are cut at page ends and at the
+// end of the sink part, so each is one contiguous run of rows.
+template <int ESZ, int LPT, int SK, int SV, bool EXACT>
+__global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
+  constexpr int E = 16 / ESZ;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const long long w = (long long)blockIdx.x * nwarps + warp;
+  if (w >= a.W) return;
+  const long long total = a.plan[0], P = a.plan[1];
+  const long long f0 = w * P;
+  if (f0 >= total) return;
+  const long long f1 = min(f0 + P, total);
+  const int slot = lane / LPT, g = lane - slot * LPT;
+
+  const int bar_bytes = ((nwarps * a.nstage * 8) + 127) & ~127;
+  const uint32_t bar0 = smem_u32(smem) + warp * a.nstage * 8;
+  unsigned char* buf = smem + bar_bytes + (size_t)warp * a.nstage * a.stage_bytes;
+  const uint32_t buf0 = smem_u32(buf);
+  const int v_off = a.tile * a.row_k;
+
+  if (lane == 0) {
+    for (int s = 0; s < a.nstage; ++s) mbar_init(bar0 + 8 * s, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t pol = l2_evict_first_policy();
+
+  const int4 st0 = a.wstart[w];
+  PCursor pc{st0.x, st0.y, st0.z, 0, 0, 0};
+  pc_load_seq(pc, a);
+  PCursor cc = pc;
+
+  // Producer (lane 0 issues). Block-table entries are cached, and the next
+  // entry of the same sequence is loaded ahead so a page change seldom
+  // waits on a global load. Entries past a sequence's used blocks are read
+  // only as that look-ahead and never used.
+  int cb = -1, cblk = -1, cpage = 0, nblk = -1, npage = 0;
+  auto page_of = [&](int b, int blk) -> int {
+    if (b != cb || blk != cblk) {
+      cpage = (b == cb && blk == nblk)
+                  ? npage
+                  : __ldg(a.block_table + (size_t)b * a.max_blocks + blk);
+      cb = b;
+      cblk = blk;
+      nblk = blk + 1 < a.max_blocks ? blk + 1 : -1;
+      if (nblk >= 0) npage = __ldg(a.block_table + (size_t)b * a.max_blocks + nblk);
+    }
+    return cpage;
+  };
+  long long pf = f0;
+  int ps = 0, in_flight = 0;
+  auto issue = [&]() {
+    const int len = pc_len(pc, pf, f1, a.tile, a.page_size);
+    if (lane == 0) {
+      const int pos = pc.i < pc.s ? pc.i : pc.i + pc.gap;
+      const int page = page_of(pc.b, pos / a.page_size);
+      const long long row =
+          ((long long)page * a.H + pc.h) * a.page_size + pos % a.page_size;
+      const uint32_t kb = (uint32_t)len * a.row_k, vb = (uint32_t)len * a.row_v;
+      const uint32_t bar = bar0 + 8 * ps;
+      const uint32_t dst = buf0 + ps * a.stage_bytes;
+      mbar_arrive_expect_tx(bar, kb + vb);
+      bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
+      bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
+    }
+    pf += len;
+    pc_advance(pc, len, a);
+    if (++ps == a.nstage) ps = 0;
+    ++in_flight;
+  };
+  for (int s = 0; s < a.nstage && pf < f1; ++s) issue();
+
+  // q' is written by k_absorb.
+  pdl_wait();
+
+  int cs = 0;
+  uint32_t cpar = 0;
+  long long f = f0;
+  long long u = (long long)cc.b * a.H + cc.h;
+  float qv[SK][E], qn[SK][E];
+  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g);
+  while (f < f1) {
+    const long long seg_end = min(f1, f + (cc.n - cc.i));
+    long long un = -1;
+    if (seg_end < f1) {  // the next unit's q' loads run under this unit's stream
+      PCursor nx = cc;
+      nx.i = nx.n - 1;
+      pc_advance(nx, 1, a);
+      un = (long long)nx.b * a.H + nx.h;
+      load_qp<E, LPT, SK, EXACT>(qn, a.qp, un, a.r_k, a.nseg_k, g);
+    }
+    float m = kNegBig, l = 0.f;
+    float acc[SV][E];
+#pragma unroll
+    for (int s = 0; s < SV; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[s][e] = 0.f;
+
+    while (f < seg_end) {
+      const int len = pc_len(cc, f, f1, a.tile, a.page_size);
+      const bool ok = __all_sync(FULL, mbar_wait(bar0 + 8 * cs, cpar));
+      if (!ok) {
+        if (lane == 0) report_status(a.status, kStatusWaitTimeout);
+        int st = cs;
+        uint32_t par = cpar;
+        for (int i = 0; i < in_flight; ++i) {
+          (void)mbar_wait(bar0 + 8 * st, par, kWaitTimeoutNs / 8);
+          if (++st == a.nstage) {
+            st = 0;
+            par ^= 1u;
+          }
+        }
+        return;
+      }
+      const unsigned char* Ks = buf + cs * a.stage_bytes;
+      stream_tile<ESZ, LPT, SK, SV, EXACT>(Ks, Ks + v_off, len, qv, m, l, acc, a, slot, g);
+      __syncwarp();
+      --in_flight;
+      if (pf < f1) issue();
+      if (++cs == a.nstage) {
+        cs = 0;
+        cpar ^= 1u;
+      }
+      f += len;
+      pc_advance(cc, len, a);
+    }
+
+    stream_merge_write<ESZ, LPT, SV, EXACT>(m, l, acc, a.part + (size_t)(w + u) * a.pstride, a,
+                                            slot, g);
+    u = un;
+#pragma unroll
+    for (int s = 0; s < SK; ++s)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[s][e] = qn[s][e];
+  }
+}
+
+template <int ESZ, bool PAGED>
 StreamFn pick_stream(int lpt, int s, bool exact) {
+#define LLA_KERNEL(L, SK_, SV_, EX) \
+  (PAGED ? k_stream_paged<ESZ, L, SK_, SV_, EX> : k_stream<ESZ, L, SK_, SV_, EX>)
   if (!exact) {
     switch (lpt) {
-      case 1: return k_stream<ESZ, 1, 4, 4, false>;
-      case 2: return k_stream<ESZ, 2, 4, 4, false>;
-      case 4: return k_stream<ESZ, 4, 4, 4, false>;
-      case 8: return k_stream<ESZ, 8, 4, 4, false>;
+      case 1: return LLA_KERNEL(1, 4, 4, false);
+      case 2: return LLA_KERNEL(2, 4, 4, false);
+      case 4: return LLA_KERNEL(4, 4, 4, false);
+      case 8: return LLA_KERNEL(8, 4, 4, false);
     }
     return nullptr;
   }
 #define LLA_CASE(L, S) \
-  if (lpt == L && s == S) return k_stream<ESZ, L, S, S, true>;
+  if (lpt == L && s == S) return LLA_KERNEL(L, S, S, true);
   LLA_CASE(1, 1) LLA_CASE(1, 2) LLA_CASE(1, 3) LLA_CASE(1, 4)
   LLA_CASE(2, 1) LLA_CASE(2, 2) LLA_CASE(2, 3) LLA_CASE(2, 4)
   LLA_CASE(4, 1) LLA_CASE(4, 2) LLA_CASE(4, 3) LLA_CASE(4, 4)
   LLA_CASE(8, 1) LLA_CASE(8, 2) LLA_CASE(8, 3) LLA_CASE(8, 4)
 #undef LLA_CASE
+#undef LLA_KERNEL
   return nullptr;
 }
 
 }  // namespace
 
-StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact) {
-  return esz == 2 ? pick_stream<2>(lpt, s, exact) : pick_stream<4>(lpt, s, exact);
+StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact, bool paged) {
+  if (paged) return esz == 2 ? pick_stream<2, true>(lpt, s, exact) : pick_stream<4, true>(lpt, s, exact);
+  return esz == 2 ? pick_stream<2, false>(lpt, s, exact) : pick_stream<4, false>(lpt, s, exact);
 }
 
 }  // namespace lla

@@ -33,13 +33,28 @@ struct StreamArgs {
   float* part;
   int pstride;
   unsigned int* status;
+  // Paged / ragged store (paged kernels only; written by k_plan_paged):
+  const int4* seqinfo;     // [B] {kept tokens n, sink part s, position gap, 0}
+  const long long* cum;    // [B+1] start of sequence b in the flattened range
+  const long long* plan;   // {total tokens, tokens per warp}
+  const int4* wstart;      // [W] first (b, h, i) of each warp's range
+  const int* block_table;  // [B][max_blocks]
+  int max_blocks, page_size, H, B;
+};
+
+// Per-sequence record of the paged plan: sequence b attends n tokens; kept
+// index i < s is position i, index i >= s is position i + gap (the sink +
+// window eviction set; s = n and gap = 0 when nothing is evicted).
+struct SeqInfo {
+  int n, s, gap, pad;
 };
 
 using StreamFn = void (*)(StreamArgs);
 
 // The k_stream instantiation for a latent element size (2 or 4 bytes),
 // lanes per token and segments per lane; exact means every lane's segments
-// are in range. nullptr if there is none.
-StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact);
+// are in range; paged selects the paged / ragged store. nullptr if there is
+// none.
+StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact, bool paged = false);
 
 }  // namespace lla

@@ -23,6 +23,7 @@ from __future__ import annotations
 
 from dataclasses import dataclass, field
 
+import numpy as np
 import torch
 
 
@@ -75,6 +76,33 @@ def orthonormal(n: int, rows: int, cols: int, seed: int, device="cpu",
 def queries(shape, d_h: int, seed: int, device="cpu") -> torch.Tensor:
     """q ~ N(0, 1/d_h), fp32."""
     return normal(shape, seed, device, std=d_h ** -0.5)
+
+
+def ragged_lengths(B: int, n_mean: int, seed: int, spread: float = 0.5) -> np.ndarray:
+    """Seeded per-sequence lengths, uniform in [(1 - spread) n, (1 + spread) n]
+    (a serving batch's length mix), at least 1. int32."""
+    r = np.random.default_rng(seed)
+    lo = max(1, int(round((1.0 - spread) * n_mean)))
+    hi = max(lo, int(round((1.0 + spread) * n_mean)))
+    return r.integers(lo, hi + 1, size=B).astype(np.int32)
+
+
+def page_table(lens, page_size: int, seed: int, spare: int = 0, max_blocks: int = 0):
+    """A shuffled page assignment for sequences of the given lengths: every
+    sequence gets ceil(n / page_size) distinct pages drawn from one pool in a
+    seeded random order. Unused table entries are -1. Returns (block_table
+    [B, max_blocks] int32, num_pages) with num_pages = pages used + spare."""
+    lens = np.asarray(lens, dtype=np.int64)
+    need = (lens + page_size - 1) // page_size
+    max_blocks = max(int(need.max(initial=0)), max_blocks, 1)
+    num_pages = int(need.sum()) + spare
+    order = np.random.default_rng(seed).permutation(max(num_pages, 1))
+    bt = np.full((len(lens), max_blocks), -1, dtype=np.int32)
+    k = 0
+    for b, nb in enumerate(need):
+        bt[b, :nb] = order[k:k + nb]
+        k += nb
+    return bt, max(num_pages, 1)
 
 
 # --------------------------------------------------------------------------

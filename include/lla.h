@@ -55,7 +55,10 @@ typedef enum {
 typedef enum { LLA_F32 = 0, LLA_BF16 = 1 } lla_dtype;
 
 /* Device status bits reported by lla_device_status(). */
-#define LLA_DEVICE_WAIT_TIMEOUT 0x1u /* a bounded device wait ran out */
+#define LLA_DEVICE_WAIT_TIMEOUT 0x1u     /* a bounded device wait ran out */
+#define LLA_DEVICE_BAD_PAGED_INPUT 0x2u  /* lla_decode_attn_paged: a length or
+                                            page index out of range (that
+                                            sequence was treated as empty) */
 
 /* Human-readable name of a status code. Never NULL. */
 LLA_API const char *lla_status_string(lla_status s);
@@ -166,6 +169,60 @@ LLA_API lla_status lla_decode_attn_noalloc(const float *q, const void *zk,
                                            const float *mu_k_t,
                                            const float *mu_v_t, float scale,
                                            float *out, float *lse, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Per-head absorbed decode over a paged latent store with per-sequence
+ * lengths and optional attention-sink + window eviction, one (layer d,
+ * loop t) step.
+ *
+ * Same definition as lla_decode_attn, except that sequence b attends its own
+ * set of cached tokens. The pages measure capacity with a latent store whose
+ * size bounds the batch (§7 "Memory", Table 7), and stack LLA with
+ * StreamingLLM-style eviction (§7, App. C Table 9: 4 sink tokens plus a
+ * 256-token window). Keeping the store in fixed-size pages shared by
+ * sequences of different lengths is this library's layout, not the
+ * paper's. The set is
+ *   window == 0:                         tokens [0, N_b),
+ *   window > 0 and N_b <= sink + window: tokens [0, N_b),
+ *   otherwise:                           [0, sink) and [N_b - window, N_b),
+ * with N_b = seq_lens[b]. A sequence with an empty set gets out = 0 and
+ * lse = -inf (no attention mass; the neutral element of a log-sum-exp
+ * merge). The pages leave that case undefined; this is the library's reading.
+ *
+ * Arguments beyond (or replacing) lla_decode_attn's:
+ *   zk_pages  [num_pages][H][page_size][r_k], zv_pages
+ *             [num_pages][H][page_size][r_v], element type zdt: the page
+ *             pool. Token j of sequence b, head h, is row j % page_size of
+ *             head h in page block_table[b][j / page_size]. 16-byte aligned.
+ *   page_size tokens per page, >= 1; num_pages >= 1.
+ *   block_table  [B][max_blocks] int32 device array of page indices;
+ *             max_blocks >= 1 and page_size * max_blocks < 2^31. Entries of
+ *             blocks holding no attended token are not read (except as a
+ *             look-ahead whose value is never used) and may hold anything.
+ *   seq_lens  [B] int32 device array, 0 <= N_b <= max_blocks * page_size.
+ *   sink, window  eviction set as above, both >= 0.
+ *   workspace, ws_bytes  at least lla_decode_attn_paged_workspace(B, H, r_k,
+ *             r_v) bytes, 16-byte aligned, no initialisation needed.
+ * Lengths and page indices are read only on the device: nothing is copied
+ * back to the host. Before any latent is read, a device kernel checks each
+ * length and every page index among the blocks of the attended set; a
+ * failure sets LLA_DEVICE_BAD_PAGED_INPUT in the device status word and
+ * that sequence is treated as empty. Host-side errors are as for
+ * lla_decode_attn.
+ * -------------------------------------------------------------------------- */
+LLA_API size_t lla_decode_attn_paged_workspace(int B, int H, int r_k, int r_v);
+
+LLA_API lla_status lla_decode_attn_paged(const float *q, const void *zk_pages,
+                                         const void *zv_pages, lla_dtype zdt, int B,
+                                         int H, int d_h, int r_k, int r_v,
+                                         int page_size, int num_pages,
+                                         const int *block_table, int max_blocks,
+                                         const int *seq_lens, int sink, int window,
+                                         const float *dk_t, const float *dv_t,
+                                         const float *mu_k_t, const float *mu_v_t,
+                                         float scale, float *out, float *lse,
+                                         void *workspace, size_t ws_bytes,
+                                         void *stream);
 
 /* --------------------------------------------------------------------------
  * LLA-2D absorbed decode, one (layer d, loop t) step (§3 "The LLA-2D

@@ -96,3 +96,58 @@ def compare(out_gpu, lse_gpu, units, ref_out, ref_lse, dtype):
     if lse_gpu is not None:
         lse_err = np.abs(to_f64(lse_gpu)[bs, hs] - ref_lse).max()
     return err, lse_err
+
+
+def make_paged_inputs(lens, H, d_h, r_k, r_v, dtype, page_size, *, spare=2, mu=False, seed=0,
+                      max_blocks=0, device="cuda"):
+    """Seeded paged store: a shuffled page pool [P, H, page_size, r] holding
+    sequences of the given lengths, with its block table and lengths as
+    int32 device arrays."""
+    bt, num_pages = synth.page_table(lens, page_size, seed + 11, spare=spare,
+                                     max_blocks=max_blocks)
+    B = len(lens)
+    zk = synth.latents((num_pages, H, page_size, r_k), seed + 1, device, dtype=dtype)
+    zv = synth.latents((num_pages, H, page_size, r_v), seed + 2, device, dtype=dtype)
+    dk = synth.orthonormal(H, d_h, r_k, seed + 3, device)
+    dv = synth.orthonormal(H, d_h, r_v, seed + 4, device)
+    q = synth.queries((B, H, d_h), d_h, seed + 5, device)
+    mu_k = synth.normal((H, d_h), seed + 6, device) if mu else None
+    mu_v = synth.normal((H, d_h), seed + 7, device) if mu else None
+    return dict(q=q, zk=zk, zv=zv, dk=dk, dv=dv, mu_k=mu_k, mu_v=mu_v,
+                block_table=torch.from_numpy(bt).to(device),
+                seq_lens=torch.from_numpy(np.asarray(lens, dtype=np.int32)).to(device))
+
+
+def oracle_paged_reference(inp, sink=0, window=0, scale=None):
+    """The oracle's paged decode on the exact device values."""
+    import oracle  # test infrastructure only
+
+    d_h = inp["q"].shape[-1]
+    scale = 1.0 / math.sqrt(d_h) if scale is None else scale
+    opt = lambda t: None if t is None else to_f64(t)
+    bt = inp["block_table"].cpu().numpy().astype(np.int64)
+    return oracle.paged_decode(to_f64(inp["q"]), to_f64(inp["zk"]), to_f64(inp["zv"]), bt,
+                               inp["seq_lens"].cpu().numpy(), to_f64(inp["dk"]), to_f64(inp["dv"]),
+                               opt(inp["mu_k"]), opt(inp["mu_v"]), scale, sink, window)
+
+
+def compare_paged(out, lse, ref_out, ref_lse, lens, dtype):
+    """Element-wise check of every (b, h): empty sequences exactly 0 / -inf,
+    the others within the stated tolerance. Returns (err, lse_err)."""
+    o = to_f64(out)
+    l = to_f64(lse)
+    lens = np.asarray(lens)
+    empty = lens == 0
+    assert np.all(o[empty] == 0.0) and np.all(np.isneginf(l[empty]))
+    full = ~empty
+    if not full.any():
+        return 0.0, 0.0
+    diff = np.abs(o[full] - ref_out[full]).max()
+    if dtype == torch.float32:
+        err = diff
+        assert err <= TOL_F32_ABS, f"fp32 max-abs error {err:.3e} > {TOL_F32_ABS}"
+    else:
+        err = diff / np.abs(ref_out[full]).max()
+        assert err <= TOL_BF16_REL, f"bf16 relative error {err:.3e} > {TOL_BF16_REL}"
+    lse_err = np.abs(l[full] - ref_lse[full]).max()
+    return err, lse_err
