@@ -52,6 +52,8 @@ def main_kernel(config_name: str):
         return "k_encode", os.path.join(CSRC, "encode.cu")
     if synth.DECODE_CONFIGS[config_name].two_d:
         return "k_lla2d", os.path.join(CSRC, "lla2d.cu")
+    if synth.DECODE_CONFIGS[config_name].page_size:
+        return "k_stream_paged", os.path.join(CSRC, "stream.cu")
     return "k_stream", os.path.join(CSRC, "stream.cu")
 
 
@@ -182,16 +184,30 @@ class DecodeWorkload:
     Per-head configs also carry the latent write of each sequence's newest
     token: after the T x L attention calls, the token's stacked per-loop K
     and V of every layer are encoded into slot N of the store (the attended
-    range stays [0, N), so every step measures the same context)."""
+    range stays [0, N), so every step measures the same context).
+
+    A paged config keeps each layer's store as a pool of pages with one
+    shared block table and seeded ragged lengths; its step is the T x L
+    attention calls alone (a newest-token write there is a scatter into
+    each sequence's last page, which this workload does not time)."""
 
     def __init__(self, cfg: synth.DecodeConfig, device: str, seed_offset: int = 0):
         self.cfg = cfg
         c = cfg
         s = c.seed + seed_offset
-        self.write_latents = (not c.two_d) and c.dtype == "bf16" and c.d_h % 64 == 0
+        self.paged = c.page_size > 0
+        self.write_latents = (not c.two_d and not self.paged and c.dtype == "bf16"
+                              and c.d_h % 64 == 0)
         n_cap = c.N + 1 if self.write_latents else c.N
         zk_shape = (c.B, n_cap, c.r_k) if c.two_d else (c.B, c.H, n_cap, c.r_k)
         zv_shape = (c.B, n_cap, c.r_v) if c.two_d else (c.B, c.H, n_cap, c.r_v)
+        if self.paged:
+            lens = c.lengths()
+            bt, num_pages = synth.page_table(lens, c.page_size, s + 12)
+            self.block_table = torch.from_numpy(bt).to(device)
+            self.seq_lens = torch.from_numpy(lens).to(device)
+            zk_shape = (num_pages, c.H, c.page_size, c.r_k)
+            zv_shape = (num_pages, c.H, c.page_size, c.r_v)
         self.zk = [synth.latents(zk_shape, s + 1000 * l + 1, device, decay=c.decay,
                                  dtype=c.torch_dtype) for l in range(c.L)]
         self.zv = [synth.latents(zv_shape, s + 1000 * l + 2, device, decay=c.decay,
@@ -205,9 +221,12 @@ class DecodeWorkload:
         self.lse = torch.empty((c.L, c.T, c.B, c.H), device=device, dtype=torch.float32)
         import decode_attention_encode_b200 as lla
         self.lla = lla
-        wsfn = lla.lla2d_decode_attn_workspace if c.two_d else lla.lla_decode_attn_workspace
-        self.ws = torch.empty(max(16, wsfn(c.B, c.H, c.N, c.r_k, c.r_v)), dtype=torch.uint8,
-                              device=device)
+        if self.paged:
+            need = lla.lla_decode_attn_paged_workspace(c.B, c.H, c.r_k, c.r_v)
+        else:
+            wsfn = lla.lla2d_decode_attn_workspace if c.two_d else lla.lla_decode_attn_workspace
+            need = wsfn(c.B, c.H, c.N, c.r_k, c.r_v)
+        self.ws = torch.empty(max(16, need), dtype=torch.uint8, device=device)
         self.fn = lla.lla2d_decode_attn if c.two_d else lla.lla_decode_attn
         self.scale = 1.0 / math.sqrt(c.d_h)
         if self.write_latents:
@@ -234,10 +253,24 @@ class DecodeWorkload:
         lse = self.lse if lse is None else lse
         for t in range(c.T):
             for l in range(c.L):
-                self.fn(q[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
-                        scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
+                self.call(l, t, q, out, lse)
         if self.write_latents:
             self.write_newest(self.xk if xk is None else xk, self.xv if xv is None else xv)
+
+    def call(self, l, t, q=None, out=None, lse=None):
+        """The (layer l, loop t) decode call through the public API."""
+        c = self.cfg
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
+        if self.paged:
+            self.lla.lla_decode_attn_paged(q[l, t], self.zk[l], self.zv[l], self.block_table,
+                                           self.seq_lens, self.dk[l, t], self.dv[l, t],
+                                           scale=self.scale, out=out[l, t], lse=lse[l, t],
+                                           workspace=self.ws)
+        else:
+            self.fn(q[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
+                    scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
 
     def write_newest(self, xk, xv):
         c = self.cfg
@@ -249,7 +282,7 @@ class DecodeWorkload:
                                     z_group_stride=self.n_cap * r)
 
     def launches_per_step(self) -> int:
-        n = 3 * self.cfg.L * self.cfg.T
+        n = (4 if self.paged else 3) * self.cfg.L * self.cfg.T
         if self.write_latents:
             n += 2 * self.cfg.L
         return n
@@ -472,8 +505,10 @@ def run_reference(args, world, rank):
 
 def describe(cfg: synth.DecodeConfig) -> str:
     kind = "LLA-2D" if cfg.two_d else "per-head LLA"
+    n = (f"N={cfg.N} mean (ragged +-{int(cfg.spread * 100)}%, {cfg.tokens()} tokens), "
+         f"{cfg.page_size}-token pages" if cfg.page_size else f"N={cfg.N}")
     return (f"{cfg.name}: {kind} decode, L={cfg.L} T={cfg.T} H={cfg.H} d_h={cfg.d_h} "
-            f"r_k={cfg.r_k} r_v={cfg.r_v} B={cfg.B} N={cfg.N} {cfg.dtype} latents")
+            f"r_k={cfg.r_k} r_v={cfg.r_v} B={cfg.B} {n} {cfg.dtype} latents")
 
 
 def run_lla(args, world, rank, local):
@@ -503,8 +538,7 @@ def run_lla(args, world, rank, local):
                 for l in range(c.L):
                     if t == 0:
                         call_ev[l][0].record(stream)
-                    wl.fn(wl.q[l, t], wl.zk[l], wl.zv[l], wl.dk[l, t], wl.dv[l, t], N=c.N,
-                          scale=wl.scale, out=wl.out[l, t], lse=wl.lse[l, t], workspace=wl.ws)
+                    wl.call(l, t)
                     if t == 0:
                         call_ev[l][1].record(stream)
             if wl.write_latents:
@@ -526,12 +560,11 @@ def run_lla(args, world, rank, local):
     kern_ms = []
     for l in range(cfg.L):
         with wl.lla.kernel_timer() as kt:
-            wl.fn(wl.q[l, 0], wl.zk[l], wl.zv[l], wl.dk[l, 0], wl.dv[l, 0], N=cfg.N,
-                  scale=wl.scale, out=wl.out[l, 0], lse=wl.lse[l, 0], workspace=wl.ws)
+            wl.call(l, 0)
         kern_ms.append(kt.ms)
     kern_ms_mean = sum(kern_ms) / len(kern_ms)
 
-    tokens_per_step = cfg.B * cfg.N * cfg.L * cfg.T
+    tokens_per_step = cfg.tokens() * cfg.L * cfg.T
     value = aggregate_rate(tokens_per_step, ms_per_step, world)
     step_bytes = cfg.step_bytes()
     hbm_peak, peak_src = peaks()
@@ -573,8 +606,7 @@ def run_lla(args, world, rank, local):
             for t in range(c.T):
                 for l in range(c.L):
                     stream.wait_event(in_ev[t][l])
-                    wl.fn(q_dev[l, t], wl.zk[l], wl.zv[l], wl.dk[l, t], wl.dv[l, t], N=c.N,
-                          scale=wl.scale, out=wl.out[l, t], lse=wl.lse[l, t], workspace=wl.ws)
+                    wl.call(l, t, q=q_dev)
                     done_ev[t][l].record(stream)
                     with torch.cuda.stream(d2h):
                         d2h.wait_event(done_ev[t][l])
@@ -609,7 +641,8 @@ def run_lla(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": describe(cfg),
-            "step": f"{cfg.L * cfg.T} decode calls (T loops x L layers), 3 kernels each"
+            "step": f"{cfg.L * cfg.T} decode calls (T loops x L layers), "
+                    f"{4 if wl.paged else 3} kernels each"
                     + (f", then {2 * cfg.L} latent writes of the newest token" if wl.write_latents else ""),
             "accumulation": "fp32",
             "l2": "no flush: each layer's latent store "

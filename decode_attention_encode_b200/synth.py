@@ -112,7 +112,9 @@ def page_table(lens, page_size: int, seed: int, spare: int = 0, max_blocks: int 
 @dataclass(frozen=True)
 class DecodeConfig:
     """One decode workload. ``two_d`` selects LLA-2D (one latent per token
-    and layer shared by all heads)."""
+    and layer shared by all heads). ``page_size`` > 0 selects a paged store
+    whose sequences have seeded ragged lengths with mean ``N`` (uniform
+    within +-``spread`` N)."""
     name: str
     L: int           # layers (D in the paper)
     T: int           # loops
@@ -127,6 +129,8 @@ class DecodeConfig:
     two_d: bool = False
     seed: int = 0
     note: str = field(default="", compare=False)
+    page_size: int = 0
+    spread: float = 0.0
 
     @property
     def esz(self) -> int:
@@ -136,9 +140,19 @@ class DecodeConfig:
     def torch_dtype(self):
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
+    def lengths(self) -> np.ndarray:
+        """Cached tokens of each sequence (int32)."""
+        if self.page_size:
+            return ragged_lengths(self.B, self.N, self.seed + 77, self.spread)
+        return np.full(self.B, self.N, dtype=np.int32)
+
+    def tokens(self) -> int:
+        """Cached tokens attended per (layer, loop) step, all sequences."""
+        return int(self.lengths().sum())
+
     def store_bytes_per_layer(self) -> int:
         per_tok = (self.r_k + self.r_v) * self.esz * (1 if self.two_d else self.H)
-        return self.B * self.N * per_tok
+        return self.tokens() * per_tok
 
     def step_bytes(self) -> int:
         """Algorithmic bytes of one (layer, loop) step: every cached latent
@@ -156,6 +170,10 @@ C4 = DecodeConfig("lla2d_32x", L=24, T=4, H=16, d_h=128, r_k=256, r_v=256, B=256
                   N=8192, dtype="bf16", decay=True, two_d=True)
 C5_DECODE = DecodeConfig("perhead_32x_long", L=24, T=4, H=16, d_h=128, r_k=16, r_v=16,
                          B=32, N=32768, dtype="bf16", decay=False)
+# the 4x geometry as a serving batch: 64 sequences of 2048..6144 tokens in a
+# pool of 64-token pages
+C2_PAGED = DecodeConfig("perhead_4x_paged", L=24, T=4, H=16, d_h=128, r_k=128, r_v=128, B=64,
+                        N=4096, dtype="bf16", decay=True, page_size=64, spread=0.5)
 
 
 @dataclass(frozen=True)
@@ -185,4 +203,4 @@ class EncodeConfig:
 C5_ENCODE = EncodeConfig("encode_32x", L=24, T=4, G=16, d_loop=128, r=16, N=32768,
                          n_cal=2048)
 
-DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE)}
+DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED)}
