@@ -22,6 +22,9 @@ What is here, each in fp64:
     per-loop mean, take the top-r right singular vectors of the stacked-loop
     matrix as W_down, and its loop slices as the initial W_up,t.
   * ``compression_ratio``: §3 Eq. 4.
+  * ``rope_rotate`` / ``decode_unit_rope`` / ``lla_decode_rope``: the
+    decoupled-RoPE split of §7 (NoPE latent content path plus an explicit
+    rotary branch), as attention over concatenated content and rotary keys.
   * ``kept_positions`` / ``paged_decode``: the per-head decode over a paged
     store with per-sequence lengths (a gather of each unit's rows, then the
     explicit-reconstruction unit), with the attention-sink + window eviction
@@ -225,6 +228,73 @@ def _decode(q, zk, zv, dk, dv, mu_k, mu_v, scale, N, units, nthreads, shared_lat
         None if mu_k is None else np.asarray(mu_k)[hs],
         None if mu_v is None else np.asarray(mu_v)[hs], scale, nthreads)
     if len(units) == B * H and list(units) == [(b, h) for b in range(B) for h in range(H)]:
+        return out.reshape(B, H, d), lse.reshape(B, H)
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# decoupled RoPE: a NoPE latent content path plus an explicit rotary branch
+# --------------------------------------------------------------------------
+
+def rope_rotate(x, pos, theta=10000.0):
+    """Rotary position embedding (Su et al., 2021, the work §3 "RoPE and
+    reconstruction" cites) of the last axis of x (even length d) at integer
+    positions ``pos`` (broadcast against x[..., 0]): the pair (x_2i, x_2i+1)
+    turns by the angle pos * theta^(-2i/d)."""
+    x = _f64(x)
+    d = x.shape[-1]
+    assert d % 2 == 0
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta ** (-np.arange(0, d, 2) / d)
+    c, s_ = np.cos(ang), np.sin(ang)
+    out = np.empty_like(x)
+    out[..., 0::2] = x[..., 0::2] * c - x[..., 1::2] * s_
+    out[..., 1::2] = x[..., 0::2] * s_ + x[..., 1::2] * c
+    return out
+
+
+def decode_unit_rope(q, q_rope, zk, k_rope, zv, dk, dv, mu_k=None, mu_v=None, scale=None):
+    """One unit with the decoupled-RoPE split of §7 ("Per-head LLA versus
+    LLA-2D at inference": RoPE blocks exact absorption of the positional
+    part, so the latent carries the NoPE content and a small explicit rotary
+    branch, shared across loops for a token, carries position).
+
+    q [d] content query; q_rope [d_r] this loop's rotated rotary query;
+    zk [N, r_k], zv [N, r_v] latents; k_rope [N, d_r] the tokens' rotated
+    rotary keys. Scores are scale * (q . khat_j + q_rope . k_rope_j) with
+    khat_j = dk zk_j + mu_k (§3 Eq. 3): textbook attention over keys that
+    concatenate the reconstructed content key and the rotary key."""
+    q, q_rope, zk, k_rope, zv = map(_f64, (q, q_rope, zk, k_rope, zv))
+    if scale is None:
+        scale = 1.0 / np.sqrt(q.shape[0])
+    khat = zk @ _f64(dk).T + (0.0 if mu_k is None else _f64(mu_k))
+    vhat = zv @ _f64(dv).T + (0.0 if mu_v is None else _f64(mu_v))
+    return attend(np.concatenate([q, q_rope]), np.concatenate([khat, k_rope], axis=1), vhat,
+                  scale)
+
+
+def lla_decode_rope(q, q_rope, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None, N=None,
+                    units=None):
+    """Per-head decode with the decoupled rotary branch for one (layer,
+    loop) step. The store keeps each key row as [latent (r_k) | rotated
+    rotary key (d_r)]: zk [B, H, n_cap, r_k + d_r]; q_rope [B, H, d_r].
+    Returns out, lse for the listed (b, h) units (all by default)."""
+    q, q_rope = np.asarray(q), np.asarray(q_rope)
+    B, H, d = q.shape
+    d_r = q_rope.shape[-1]
+    zk, zv = np.asarray(zk), np.asarray(zv)
+    r_k = zk.shape[-1] - d_r
+    N = zk.shape[2] if N is None else N
+    full = units is None
+    units = [(b, h) for b in range(B) for h in range(H)] if full else units
+    out = np.zeros((len(units), d))
+    lse = np.zeros(len(units))
+    for i, (b, h) in enumerate(units):
+        out[i], lse[i] = decode_unit_rope(
+            q[b, h], q_rope[b, h], zk[b, h, :N, :r_k], zk[b, h, :N, r_k:], zv[b, h, :N],
+            np.asarray(dk)[h], np.asarray(dv)[h],
+            None if mu_k is None else np.asarray(mu_k)[h],
+            None if mu_v is None else np.asarray(mu_v)[h], scale)
+    if full:
         return out.reshape(B, H, d), lse.reshape(B, H)
     return out, lse
 

@@ -505,3 +505,69 @@ def test_paged_empty_sequence_has_no_attention_mass():
                                    s["mk"], s["mv"])
     assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
     assert np.all(np.isfinite(out[1])) and np.all(np.isfinite(lse[1]))
+
+
+# ---------------------------------------------------------------------------
+# decoupled RoPE
+# ---------------------------------------------------------------------------
+
+def test_rope_is_a_rotation_that_sees_only_relative_position():
+    r = rng(51)
+    d = 16
+    q, k = r.standard_normal(d), r.standard_normal(d)
+    # position 0 is the identity; norms are kept
+    np.testing.assert_allclose(oracle.rope_rotate(q, 0), q, atol=0)
+    np.testing.assert_allclose(np.linalg.norm(oracle.rope_rotate(q, 37)), np.linalg.norm(q),
+                               rtol=1e-13)
+    # the score depends on p - j only
+    s1 = oracle.rope_rotate(q, 100) @ oracle.rope_rotate(k, 40)
+    s2 = oracle.rope_rotate(q, 1060) @ oracle.rope_rotate(k, 1000)
+    s3 = oracle.rope_rotate(q, 60) @ k
+    assert abs(s1 - s2) < 1e-10 and abs(s1 - s3) < 1e-10
+    # pair 0 turns by exactly pos radians (theta^0 = 1); the last pair slowest
+    x = np.zeros(d); x[0] = 1.0
+    y = oracle.rope_rotate(x, 0.5)
+    np.testing.assert_allclose(y[:2], [np.cos(0.5), np.sin(0.5)], atol=1e-15)
+    x = np.zeros(d); x[d - 2] = 1.0
+    y = oracle.rope_rotate(x, 3.0)
+    a = 3.0 * 10000.0 ** (-(d - 2) / d)
+    np.testing.assert_allclose(y[d - 2:], [np.cos(a), np.sin(a)], atol=1e-15)
+
+
+def test_rope_unit_reduces_to_the_nope_unit_and_to_rotary_attention():
+    r = rng(52)
+    u = _unit(52)
+    q, zk, zv, dk, dv, mk, mv = (u[k] for k in ("q", "zk", "zv", "dk", "dv", "mu_k", "mu_v"))
+    N, d_r = zk.shape[0], 8
+    k_rope = r.standard_normal((N, d_r))
+    # zero rotary query: the NoPE latent unit
+    o0, l0 = oracle.decode_unit_rope(q, np.zeros(d_r), zk, k_rope, zv, dk, dv, mk, mv)
+    o1, l1 = oracle.decode_unit(q, zk, zv, dk, dv, mk, mv)
+    np.testing.assert_allclose(o0, o1, atol=1e-12)
+    assert abs(l0 - l1) < 1e-12
+    # zero content query and key mean: plain attention over the rotary keys
+    q_rope = r.standard_normal(d_r)
+    o2, l2 = oracle.decode_unit_rope(np.zeros_like(q), q_rope, zk, k_rope, zv, dk, dv, None, mv)
+    vhat = zv @ dv.T + mv
+    o3, l3 = oracle.attend(q_rope, k_rope, vhat, 1.0 / np.sqrt(q.shape[0]))
+    np.testing.assert_allclose(o2, o3, atol=1e-12)
+    assert abs(l2 - l3) < 1e-12
+
+
+def test_rope_unit_matches_absorbed_query_with_appended_rotary_part():
+    # the §7 absorption applies to the content part only: q' = dk^T q,
+    # scores q'.z_j + q.mu_k + q_rope.k_rope_j (brute force, tiny inputs)
+    r = rng(53)
+    u = _unit(53)
+    q, zk, zv, dk, dv, mk, mv = (u[k] for k in ("q", "zk", "zv", "dk", "dv", "mu_k", "mu_v"))
+    N, d_r = zk.shape[0], 6
+    k_rope = r.standard_normal((N, d_r))
+    q_rope = r.standard_normal(d_r)
+    sc = 1.0 / np.sqrt(q.shape[0])
+    o, l = oracle.decode_unit_rope(q, q_rope, zk, k_rope, zv, dk, dv, mk, mv)
+    qa = np.concatenate([dk.T @ q, q_rope])
+    s = sc * (np.concatenate([zk, k_rope], axis=1) @ qa + q @ mk)
+    p = np.exp(s - s.max())
+    ubar = (p / p.sum()) @ zv
+    np.testing.assert_allclose(o, dv @ ubar + mv, atol=1e-12)
+    assert abs(l - (s.max() + np.log(p.sum()))) < 1e-12
