@@ -46,6 +46,28 @@ int rows_per_thread(int ctas_per_row_block_of_8, int B) {
   return rows;
 }
 
+// Stages n float4 items into shared memory with the whole CTA (256 threads):
+// each thread issues up to 8 global loads before its first shared store, so
+// a staging pass costs about one memory round trip per 2048 items instead
+// of one per item.
+template <typename Load, typename Store>
+__device__ __forceinline__ void stage_batched(int n, Load load, Store store) {
+  constexpr int kBatch = 8;
+  for (int base = threadIdx.x; base < n; base += 256 * kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int idx = base + k * 256;
+      v[k] = idx < n ? load(idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int idx = base + k * 256;
+      if (idx < n) store(idx, v[k]);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // k_absorb
 // ---------------------------------------------------------------------------
@@ -81,15 +103,32 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
   const int nc = min(32, a.r_k - c0);  // a multiple of 8
   const int n4 = nc / 4;
   const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
-  for (int idx = threadIdx.x; idx < d_h4 * 8; idx += 256) {
+  stage_batched(d_h4 * 8, [&](int idx) {
     const int i = idx >> 3, j = idx & 7;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < a.d_h && j < n4) v = __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j);
-    reinterpret_cast<float4*>(d_s + i * 32)[j] = v;
-  }
-  for (int idx = threadIdx.x; idx < 8 * ROWS * d_h4; idx += 256) {
-    const int bb = idx / d_h4, i = idx - bb * d_h4;
-    q_s[idx] = (bb < nb && i < a.d_h) ? a.q[((size_t)(b0 + bb) * a.H + h) * a.d_h + i] : 0.f;
+    return (i < a.d_h && j < n4) ? __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }, [&](int idx, float4 v) { reinterpret_cast<float4*>(d_s + (idx >> 3) * 32)[idx & 7] = v; });
+  const int q4 = d_h4 / 4;  // float4 per staged query row
+  if ((a.d_h & 3) == 0 && (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {
+    stage_batched(8 * ROWS * q4, [&](int idx) {
+      const int bb = idx / q4, i4 = idx - bb * q4;
+      return bb < nb ? __ldg(reinterpret_cast<const float4*>(
+                           a.q + ((size_t)(b0 + bb) * a.H + h) * a.d_h) + i4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }, [&](int idx, float4 v) { reinterpret_cast<float4*>(q_s)[idx] = v; });
+  } else {
+    stage_batched(8 * ROWS * q4, [&](int idx) {
+      const int bb = idx / q4, i = 4 * (idx - bb * q4);
+      const float* row = a.q + ((size_t)(b0 + bb) * a.H + h) * a.d_h;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (bb < nb) {
+        if (i + 0 < a.d_h) v.x = __ldg(row + i + 0);
+        if (i + 1 < a.d_h) v.y = __ldg(row + i + 1);
+        if (i + 2 < a.d_h) v.z = __ldg(row + i + 2);
+        if (i + 3 < a.d_h) v.w = __ldg(row + i + 3);
+      }
+      return v;
+    }, [&](int idx, float4 v) { reinterpret_cast<float4*>(q_s)[idx] = v; });
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,16 +194,23 @@ struct CombineArgs {
   RaggedMap ragged;  // seqinfo non-null: the paged plan's piece map
 };
 
-// One CTA per (head, 32 output channels, 8*ROWS batch rows). Warp w merges
-// the partial records of its ROWS rows into ubar (lanes across the latent
-// index in float4 steps); the CTA stages its 32 x r_v slice of W^V_up,t
-// (rows padded by 4 floats, so float4 reads of 8 consecutive rows hit
-// distinct bank groups; staged before waiting on the streaming kernel);
-// thread (w, l) forms out[b][h][i0 + l] for its ROWS rows.
+// One CTA per (head, 32 output channels, 8*ROWS batch rows). The CTA stages
+// its 32 x r_v slice of W^V_up,t (rows padded by 4 floats, so float4 reads
+// of 8 consecutive rows hit distinct bank groups; staged before waiting on
+// the streaming kernel), then merges the partial records of its rows into
+// ubar: one thread per row forms the merged maximum and normaliser, then
+// all threads sweep the (row, 4-column) items with several records in
+// flight each, since this kernel is bound by memory round trips, not
+// bandwidth. Thread (w, l) finally forms out[b][h][i0 + l] for its ROWS
+// rows.
 template <int ROWS>
-__global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+__global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
   extern __shared__ __align__(16) float sm_combine[];
-  __shared__ float s_keep[64];  // 0 for a row with no attended token
+  // per row of the CTA: pieces, offset of the first record, merged max,
+  // 1 / normaliser, and 0 for a row with no attended token
+  __shared__ int s_np[64];
+  __shared__ long long s_off[64];
+  __shared__ float s_M[64], s_inv[64], s_keep[64];
   const int pitch = a.r_v + 4;
   float* d_s = sm_combine;                        // [32][pitch]
   float* ub = sm_combine + 32 * pitch;            // [8*ROWS][r_v]
@@ -175,69 +221,133 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   const int ni = min(32, a.d_h - i0);
   const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
   const int r4 = a.r_v / 4;
-  for (int idx = threadIdx.x; idx < ni * r4; idx += 256) {
+  stage_batched(ni * r4, [&](int idx) {
     const int i = idx / r4, j = idx - i * r4;
-    reinterpret_cast<float4*>(d_s + i * pitch)[j] =
-        __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j);
-  }
+    return __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j);
+  }, [&](int idx, float4 v) {
+    const int i = idx / r4, j = idx - i * r4;
+    reinterpret_cast<float4*>(d_s + i * pitch)[j] = v;
+  });
   pdl_wait();  // partials come from the streaming kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int k = 0; k < ROWS; ++k) {
-    const int bb = warp * ROWS + k;
-    float4* urow = reinterpret_cast<float4*>(ub + bb * a.r_v);
-    if (bb >= nb) {
-      for (int c4 = lane; c4 < r4; c4 += 32) urow[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-      continue;
-    }
-    const long long u = (long long)(b0 + bb) * a.H + h;
-    // The split runs over units (b, h) for per-head LLA and over sequences
-    // b for LLA-2D; piece w of split key k is partial record w + k. A
-    // ragged plan places unit (b, h) at cum[b] + h * n_b in the range.
-    const long long key = a.shared ? (long long)(b0 + bb) : u;
-    long long wf, wl;
-    if (a.ragged.seqinfo) {
-      const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
-      if (n == 0) {  // nothing attended: out = 0, lse = -inf
-        for (int c4 = lane; c4 < r4; c4 += 32) urow[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lane == 0) s_keep[bb] = 0.f;
-        if (blockIdx.y == 0 && lane == 0 && a.lse) a.lse[u] = -INFINITY;
-        continue;
+  const int nrows = 8 * ROWS;
+  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
+
+  // 1. Per row: the range of partial records and the merged maximum and
+  //    normaliser, one thread per row with four record loads in flight.
+  //    The split runs over units (b, h) for per-head LLA and over sequences
+  //    b for LLA-2D; piece w of split key k is partial record w + k. A
+  //    ragged plan places unit (b, h) at cum[b] + h * n_b in the range.
+  if (threadIdx.x < nrows) {
+    const int bb = threadIdx.x;
+    int np = 0;
+    long long off = 0;
+    float M = kNegBig, L = 0.f, keep = 0.f;
+    if (bb < nb) {
+      const long long u = (long long)(b0 + bb) * a.H + h;
+      const long long key = a.shared ? (long long)(b0 + bb) : u;
+      long long wf = 0, wl = -1;
+      if (a.ragged.seqinfo) {
+        const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
+        if (n > 0) {
+          const long long P = a.ragged.plan[1];
+          const long long first = a.ragged.cum[b0 + bb] + (long long)h * n;
+          wf = first / P;
+          wl = (first + n - 1) / P;
+        }
+      } else {
+        wf = (key * a.N) / a.P;
+        wl = ((key + 1) * a.N - 1) / a.P;
       }
-      const long long P = a.ragged.plan[1];
-      const long long first = a.ragged.cum[b0 + bb] + (long long)h * n;
-      wf = first / P;
-      wl = (first + n - 1) / P;
-    } else {
-      wf = (key * a.N) / a.P;
-      wl = ((key + 1) * a.N - 1) / a.P;
-    }
-    if (lane == 0) s_keep[bb] = 1.f;
-    const int np = (int)(wl - wf + 1);
-    const float* rec0 = a.shared ? a.part + ((wf + key) * a.H + h) * a.pstride
-                                 : a.part + (wf + key) * a.pstride;
-    const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
-    float M = kNegBig;
-    for (int p = lane; p < np; p += 32) M = fmaxf(M, rec0[p * rstride]);
+      np = (int)(wl - wf + 1);
+      off = a.shared ? ((wf + key) * a.H + h) * a.pstride : (wf + key) * a.pstride;
+      const float* rec0 = a.part + off;
+      for (int p0 = 0; p0 < np; p0 += 4) {
+        float2 v[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int p = lane; p < np; p += 32) L += rec0[p * rstride + 1] * exp2f(rec0[p * rstride] - M);
-    L = warp_sum(L);
-    const float inv = 1.f / L;
-    for (int c4 = lane; c4 < r4; c4 += 32) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int p = 0; p < np; ++p) {
-        const float wk = exp2f(rec0[p * rstride] - M);
-        const float4 uv = reinterpret_cast<const float4*>(rec0 + p * rstride + 4)[c4];
-        acc.x = fmaf(wk, uv.x, acc.x);
-        acc.y = fmaf(wk, uv.y, acc.y);
-        acc.z = fmaf(wk, uv.z, acc.z);
-        acc.w = fmaf(wk, uv.w, acc.w);
+        for (int k = 0; k < 4; ++k)
+          v[k] = p0 + k < np ? __ldg(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride))
+                             : make_float2(kNegBig, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float Mn = fmaxf(M, v[k].x);
+          L = L * exp2f(M - Mn) + v[k].y * exp2f(v[k].x - Mn);
+          M = Mn;
+        }
       }
-      urow[c4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      keep = np > 0 ? 1.f : 0.f;
+      if (blockIdx.y == 0 && a.lse)  // no attended token: lse = -inf
+        a.lse[u] = np > 0 ? (M + log2f(L)) * kLn2 + a.c0[u] : -INFINITY;
     }
-    if (blockIdx.y == 0 && lane == 0 && a.lse) a.lse[u] = (M + log2f(L)) * kLn2 + a.c0[u];
+    s_np[bb] = np;
+    s_off[bb] = off;
+    s_M[bb] = M;
+    s_inv[bb] = np > 0 ? 1.f / L : 0.f;
+    s_keep[bb] = keep;
+  }
+  __syncthreads();
+
+  // 2. ubar[row] = sum_p exp2(m_p - M) u_p / L over all (row, 4-column)
+  //    items of the CTA, eight items per thread at a time so their record
+  //    loads are in flight together. Rows with no piece come out 0.
+  {
+    constexpr int kI = 8;
+    const int nitems = nrows * r4;
+    for (int base = threadIdx.x; base < nitems; base += 256 * kI) {
+      float4 acc[kI];
+      const float* rb[kI];
+      int npk[kI], c4k[kI];
+      float Mk[kI];
+      int npmax = 0;
+#pragma unroll
+      for (int k = 0; k < kI; ++k) {
+        const int idx = base + k * 256;
+        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        npk[k] = 0;
+        rb[k] = a.part;
+        c4k[k] = 0;
+        Mk[k] = 0.f;
+        if (idx < nitems) {
+          const int bb = idx / r4;
+          c4k[k] = idx - bb * r4;
+          npk[k] = s_np[bb];
+          rb[k] = a.part + s_off[bb];
+          Mk[k] = s_M[bb];
+        }
+        npmax = max(npmax, npk[k]);
+      }
+      for (int p = 0; p < npmax; ++p) {
+        float mv[kI];
+        float4 uv[kI];
+#pragma unroll
+        for (int k = 0; k < kI; ++k) {
+          if (p < npk[k]) {
+            mv[k] = __ldg(rb[k] + p * rstride);
+            uv[k] = __ldg(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kI; ++k) {
+          if (p < npk[k]) {
+            const float wk = exp2f(mv[k] - Mk[k]);
+            acc[k].x = fmaf(wk, uv[k].x, acc[k].x);
+            acc[k].y = fmaf(wk, uv[k].y, acc[k].y);
+            acc[k].z = fmaf(wk, uv[k].z, acc[k].z);
+            acc[k].w = fmaf(wk, uv[k].w, acc[k].w);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kI; ++k) {
+        const int idx = base + k * 256;
+        if (idx < nitems) {
+          const int bb = idx / r4;
+          const float inv = s_inv[bb];
+          reinterpret_cast<float4*>(ub + bb * a.r_v)[c4k[k]] =
+              make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+        }
+      }
+    }
   }
   __syncthreads();
   if (lane < ni) {
@@ -365,8 +475,10 @@ lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePla
   const int pair = 2 * ns;
   d.tile = std::max(pair, (target / tok_bytes) / pair * pair);
   // fit the CTA's shared memory
+  // per warp and stage: an 8-byte mbarrier and a 4-byte tile length (the
+  // paged kernel's producer hands each tile's length to its consumer)
   auto smem_of = [&](int tile, int nst) {
-    return (size_t)((d.warps * nst * 8 + 127) & ~127) + (size_t)d.warps * nst * tile * tok_bytes;
+    return (size_t)((d.warps * nst * 12 + 127) & ~127) + (size_t)d.warps * nst * tile * tok_bytes;
   };
   while (smem_of(d.tile, d.nstage) > (size_t)di.smem_optin && d.tile > pair) d.tile -= pair;
   while (smem_of(d.tile, d.nstage) > (size_t)di.smem_optin && d.nstage > 2) --d.nstage;

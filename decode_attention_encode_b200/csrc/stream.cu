@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
   if (w >= a.W) return;
   const int slot = lane / LPT, g = lane - slot * LPT;
 
-  const int bar_bytes = ((nwarps * a.nstage * 8) + 127) & ~127;
+  const int bar_bytes = ((nwarps * a.nstage * 12) + 127) & ~127;
   const uint32_t bar0 = smem_u32(smem) + warp * a.nstage * 8;
   unsigned char* buf = smem + bar_bytes + (size_t)warp * a.nstage * a.stage_bytes;
   const uint32_t buf0 = smem_u32(buf);
@@ -302,10 +302,13 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
 // ---------------------------------------------------------------------------
 
 // Position in the flattened range of a paged plan: sequence b, head h, kept
-// index i, and sequence b's record (kept tokens n, sink part s, gap).
+// index i, sequence b's record (kept tokens n, sink part s, gap), and the
+// page position of kept index i: block blk, row pp (tracked incrementally,
+// so a tile costs no division).
 struct PCursor {
   int b, h, i;
   int n, s, gap;
+  int blk, pp;
 };
 
 __device__ __forceinline__ void pc_load_seq(PCursor& c, const StreamArgs& a) {
@@ -315,20 +318,32 @@ __device__ __forceinline__ void pc_load_seq(PCursor& c, const StreamArgs& a) {
   c.gap = v.z;
 }
 
+// Page position of kept index c.i (a division; only at range starts and
+// where the kept set jumps over evicted tokens).
+__device__ __forceinline__ void pc_place(PCursor& c, int page_size) {
+  const int pos = c.i < c.s ? c.i : c.i + c.gap;
+  c.blk = pos / page_size;
+  c.pp = pos - c.blk * page_size;
+}
+
 // Tokens of the next tile: at most `tile`, and ending no later than the
 // warp's range, the unit, the sink part and the page.
 __device__ __forceinline__ int pc_len(const PCursor& c, long long f, long long f1, int tile,
                                       int page_size) {
   int lim = (int)min((long long)tile, f1 - f);
   lim = min(lim, (c.i < c.s ? c.s : c.n) - c.i);
-  const int pos = c.i < c.s ? c.i : c.i + c.gap;
-  return min(lim, page_size - pos % page_size);
+  return min(lim, page_size - c.pp);
 }
 
 // Moves the cursor `len` tokens on; len never crosses a unit end, and at one
 // the cursor moves to the next head, or the next non-empty sequence.
 __device__ __forceinline__ void pc_advance(PCursor& c, int len, const StreamArgs& a) {
   c.i += len;
+  c.pp += len;
+  if (c.pp == a.page_size) {
+    c.pp = 0;
+    ++c.blk;
+  }
   if (c.i == c.n) {
     c.i = 0;
     if (++c.h == a.H) {
@@ -338,6 +353,25 @@ __device__ __forceinline__ void pc_advance(PCursor& c, int len, const StreamArgs
       } while (c.b < a.B && __ldg(&a.seqinfo[c.b].x) == 0);
       if (c.b < a.B) pc_load_seq(c, a);
     }
+    // kept index 0 is position 0, or the window start when the sink is empty
+    c.blk = 0;
+    c.pp = 0;
+    if (c.s == 0 && c.gap != 0) pc_place(c, a.page_size);
+  } else if (c.i == c.s && c.gap != 0) {
+    pc_place(c, a.page_size);  // jump to the window part
+  }
+}
+
+// Moves a cursor at any token of a unit to the start of the next unit
+// (next head, or next non-empty sequence). Page fields are not kept.
+__device__ __forceinline__ void pc_next_unit(PCursor& c, const StreamArgs& a) {
+  c.i = 0;
+  if (++c.h == a.H) {
+    c.h = 0;
+    do {
+      ++c.b;
+    } while (c.b < a.B && __ldg(&a.seqinfo[c.b].x) == 0);
+    if (c.b < a.B) pc_load_seq(c, a);
   }
 }
 
@@ -364,11 +398,14 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   const long long f1 = min(f0 + P, total);
   const int slot = lane / LPT, g = lane - slot * LPT;
 
-  const int bar_bytes = ((nwarps * a.nstage * 8) + 127) & ~127;
+  const int bar_bytes = ((nwarps * a.nstage * 12) + 127) & ~127;
   const uint32_t bar0 = smem_u32(smem) + warp * a.nstage * 8;
   unsigned char* buf = smem + bar_bytes + (size_t)warp * a.nstage * a.stage_bytes;
   const uint32_t buf0 = smem_u32(buf);
   const int v_off = a.tile * a.row_k;
+  // tile length of each stage, written by the producer before its copies
+  volatile int* slen = reinterpret_cast<volatile int*>(smem + nwarps * a.nstage * 8) +
+                       warp * a.nstage;
 
   if (lane == 0) {
     for (int s = 0; s < a.nstage; ++s) mbar_init(bar0 + 8 * s, 1);
@@ -378,8 +415,9 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   const uint64_t pol = l2_evict_first_policy();
 
   const int4 st0 = a.wstart[w];
-  PCursor pc{st0.x, st0.y, st0.z, 0, 0, 0};
+  PCursor pc{st0.x, st0.y, st0.z, 0, 0, 0, 0, 0};
   pc_load_seq(pc, a);
+  pc_place(pc, a.page_size);
   PCursor cc = pc;
 
   // Producer (lane 0 issues). Block-table entries are cached, and the next
@@ -404,13 +442,12 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   auto issue = [&]() {
     const int len = pc_len(pc, pf, f1, a.tile, a.page_size);
     if (lane == 0) {
-      const int pos = pc.i < pc.s ? pc.i : pc.i + pc.gap;
-      const int page = page_of(pc.b, pos / a.page_size);
-      const long long row =
-          ((long long)page * a.H + pc.h) * a.page_size + pos % a.page_size;
+      const int page = page_of(pc.b, pc.blk);
+      const long long row = ((long long)page * a.H + pc.h) * a.page_size + pc.pp;
       const uint32_t kb = (uint32_t)len * a.row_k, vb = (uint32_t)len * a.row_v;
       const uint32_t bar = bar0 + 8 * ps;
       const uint32_t dst = buf0 + ps * a.stage_bytes;
+      slen[ps] = len;  // ordered before the consumer's wait by the arrive
       mbar_arrive_expect_tx(bar, kb + vb);
       bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
       bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
@@ -434,10 +471,9 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   while (f < f1) {
     const long long seg_end = min(f1, f + (cc.n - cc.i));
     long long un = -1;
+    PCursor nx = cc;
     if (seg_end < f1) {  // the next unit's q' loads run under this unit's stream
-      PCursor nx = cc;
-      nx.i = nx.n - 1;
-      pc_advance(nx, 1, a);
+      pc_next_unit(nx, a);
       un = (long long)nx.b * a.H + nx.h;
       load_qp<E, LPT, SK, EXACT>(qn, a.qp, un, a.r_k, a.nseg_k, g);
     }
@@ -449,7 +485,6 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
       for (int e = 0; e < E; ++e) acc[s][e] = 0.f;
 
     while (f < seg_end) {
-      const int len = pc_len(cc, f, f1, a.tile, a.page_size);
       const bool ok = __all_sync(FULL, mbar_wait(bar0 + 8 * cs, cpar));
       if (!ok) {
         if (lane == 0) report_status(a.status, kStatusWaitTimeout);
@@ -464,6 +499,7 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
         }
         return;
       }
+      const int len = slen[cs];
       const unsigned char* Ks = buf + cs * a.stage_bytes;
       stream_tile<ESZ, LPT, SK, SV, EXACT>(Ks, Ks + v_off, len, qv, m, l, acc, a, slot, g);
       __syncwarp();
@@ -474,8 +510,8 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
         cpar ^= 1u;
       }
       f += len;
-      pc_advance(cc, len, a);
     }
+    cc = nx;
 
     stream_merge_write<ESZ, LPT, SV, EXACT>(m, l, acc, a.part + (size_t)(w + u) * a.pstride, a,
                                             slot, g);
