@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     lla_decode_attn_noalloc,
     lla_decode_attn_paged,
     lla_decode_attn_paged_workspace,
+    lla_decode_attn_rope,
     lla_decode_attn_workspace,
     lla_encode,
 )

@@ -197,6 +197,26 @@ lla_status lla_decode_attn(const float* q, const void* zk, const void* zv, lla_d
                     static_cast<cudaStream_t>(stream));
 }
 
+lla_status lla_decode_attn_rope(const float* q, const float* q_rope, const void* zk, const void* zv,
+                                lla_dtype zdt, int B, int H, int d_h, int d_r, int N, int n_cap,
+                                int r_k, int r_v, const float* dk_t, const float* dv_t,
+                                const float* mu_k_t, const float* mu_v_t, float scale, float* out,
+                                float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  if (!q_rope) return fail(LLA_ERR_INVALID_ARG, "q_rope must be non-NULL");
+  if (!aligned(q_rope, 4)) return fail(LLA_ERR_INVALID_ARG, "q_rope must be 4-byte aligned");
+  if (d_r < 8 || d_r % 8) return fail(LLA_ERR_INVALID_ARG, "d_r must be a positive multiple of 8");
+  if (r_k < 8 || r_k % 8) return fail(LLA_ERR_INVALID_ARG, "r_k must be a positive multiple of 8");
+  int esz = 0;
+  // the key row (latent and rotary key) is checked as one rank-(r_k + d_r) row
+  lla_status st = check_decode_args(q, zk, zv, zdt, B, H, d_h, N, n_cap, r_k + d_r, r_v, dk_t, dv_t,
+                                    mu_k_t, mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  return run_decode(q, zk, zv, esz, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t, mu_k_t,
+                    mu_v_t, scale, out, lse, workspace, ws_bytes, static_cast<cudaStream_t>(stream),
+                    q_rope, d_r);
+}
+
 size_t lla_decode_attn_paged_workspace(int B, int H, int r_k, int r_v) {
   if (B < 1 || H < 1 || r_k < 8 || r_v < 8 || r_k % 8 || r_v % 8) return 0;
   size_t need = workspace_paged(B, H, r_k, r_v, 2);

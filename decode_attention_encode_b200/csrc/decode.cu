@@ -78,10 +78,12 @@ struct AbsorbArgs {
   int B, H, d_h, r_k;
   float qscale;  // scale * log2(e): scores leave k_stream in log2 units
   float scale;
-  float* qp;  // [B*H][r_k], or null
+  float* qp;  // [B*H][r_k + d_r], or null
   float* c0;  // [B*H], natural-log units
   unsigned char* qsw;  // LLA-2D MMA operand copy of q' (bf16, swizzled), or null
   int hp;              // its rows (heads padded to the MMA N)
+  const float* q_rope;  // [B*H][d_r] rotated rotary query, or null (d_r = 0)
+  int d_r;
 };
 
 // One CTA per (head, 32 latent columns, 8*ROWS batch rows). The CTA stages
@@ -100,8 +102,9 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
   const int c0 = blockIdx.y * 32;
   const int b0 = blockIdx.z * (8 * ROWS);
   const int nb = min(8 * ROWS, a.B - b0);
-  const int nc = min(32, a.r_k - c0);  // a multiple of 8
-  const int n4 = nc / 4;
+  const int rq = a.r_k + a.d_r;        // q' row: latent part, then rotary part
+  const int nc = min(32, rq - c0);     // columns of this CTA, a multiple of 8
+  const int n4 = max(0, min(32, a.r_k - c0)) / 4;  // of them from W^K, in float4
   const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
   stage_batched(d_h4 * 8, [&](int idx) {
     const int i = idx >> 3, j = idx & 7;
@@ -157,20 +160,24 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
     }
   }
   if (lane < nc) {
+    const int c = c0 + lane;
 #pragma unroll
     for (int k = 0; k < ROWS; ++k) {
       const int bb = warp * ROWS + k;
       if (bb >= nb) continue;
-      const float v = acc[k] * a.qscale;
-      if (a.qp) a.qp[((size_t)(b0 + bb) * a.H + h) * a.r_k + c0 + lane] = v;
+      const size_t unit = (size_t)(b0 + bb) * a.H + h;
+      // the rotary part of the query is not absorbed: it meets the cached
+      // rotated keys as it is
+      const float v = (c < a.r_k ? acc[k] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
+                      a.qscale;
+      if (a.qp) a.qp[unit * rq + c] = v;
       if (a.qsw) {
-        unsigned char* base = a.qsw + (size_t)(b0 + bb) * (a.r_k / 64) * a.hp * 128;
-        *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c0 + lane, a.hp)) =
-            __float2bfloat16_rn(v);
+        unsigned char* base = a.qsw + (size_t)(b0 + bb) * (rq / 64) * a.hp * 128;
+        *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)) = __float2bfloat16_rn(v);
         // the last head's CTAs also clear the padding rows h >= H
         if (h == a.H - 1)
           for (int hz = a.H; hz < a.hp; ++hz)
-            *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c0 + lane, a.hp)) =
+            *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)) =
                 __float2bfloat16_rn(0.f);
       }
     }
@@ -376,7 +383,6 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-bool exact_variant(int lpt, int s) { return lpt >= 1 && lpt <= 8 && s >= 1 && s <= 4; }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -390,9 +396,10 @@ int env_int(const char* name, int dflt) {
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
-                         unsigned char* qsw, int hp) {
-  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp};
-  const int ncol = (r_k + 31) / 32;
+                         unsigned char* qsw, int hp, const float* q_rope, int d_r) {
+  AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp,
+               q_rope, q_rope ? d_r : 0};
+  const int ncol = (r_k + a.d_r + 31) / 32;
   const int rows = rows_per_thread(H * ncol, B);
   dim3 grid(H, ncol, (B + 8 * rows - 1) / (8 * rows));
   const int d_h4 = (d_h + 3) & ~3;
@@ -455,15 +462,22 @@ lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePla
   const int lpt_env = env_int("LLA_DECODE_LPT", 0);
   if (lpt_env == 1 || lpt_env == 2 || lpt_env == 4 || lpt_env == 8)
     if (d.nseg_k % lpt_env == 0 && d.nseg_v % lpt_env == 0) lpt = lpt_env;
-  if (d.nseg_k == d.nseg_v && exact_variant(lpt, d.nseg_k / lpt)) {
+  // An exact kernel (every lane's segments in range) when one exists for
+  // the two per-lane counts; else the fewest lanes whose masked counts fit
+  // in 4, with a masked kernel sized to them, or the generic 4 / 4 one.
+  if (d.nseg_k % lpt == 0 && d.nseg_v % lpt == 0 &&
+      pick_stream_kernel(esz, lpt, d.nseg_k / lpt, d.nseg_v / lpt, true)) {
     d.exact = true;
-    d.sk = d.sv = d.nseg_k / lpt;
+    d.sk = d.nseg_k / lpt;
+    d.sv = d.nseg_v / lpt;
   } else {
     auto fits = [&](int l) { return (d.nseg_k + l - 1) / l <= 4 && (d.nseg_v + l - 1) / l <= 4; };
     while (lpt < 8 && !fits(lpt)) lpt *= 2;
     if (!fits(lpt)) return fail(LLA_ERR_UNSUPPORTED, "latent rank too large for the decode kernel");
     d.exact = false;
-    d.sk = d.sv = 4;
+    d.sk = (d.nseg_k + lpt - 1) / lpt;
+    d.sv = (d.nseg_v + lpt - 1) / lpt;
+    if (!pick_stream_kernel(esz, lpt, d.sk, d.sv, false)) d.sk = d.sv = 4;
   }
   d.lpt = lpt;
   const int ns = 32 / lpt;
@@ -508,9 +522,12 @@ lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePla
 lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, int B, int H,
                       int d_h, int N, long long n_cap, int r_k, int r_v, const float* dk,
                       const float* dv, const float* mu_k, const float* mu_v, float scale,
-                      float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                      float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                      const float* q_rope, int d_r) {
+  if (!q_rope) d_r = 0;
+  const int rq = r_k + d_r;  // key row: latent, then the rotated rotary key
   DecodePlan d;
-  lla_status st = plan_decode(B, H, N, r_k, r_v, esz, &d);
+  lla_status st = plan_decode(B, H, N, rq, r_v, esz, &d);
   if (st != LLA_OK) return st;
   if (ws == nullptr || ws_bytes < d.ws_bytes)
     return fail(LLA_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", d.ws_bytes,
@@ -520,7 +537,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
 
-  StreamFn fn = pick_stream_kernel(esz, d.lpt, d.sk, d.exact);
+  StreamFn fn = pick_stream_kernel(esz, d.lpt, d.sk, d.sv, d.exact);
   if (!fn) return fail(LLA_ERR_UNSUPPORTED, "no decode kernel for this latent shape");
 
   cudaError_t e;
@@ -528,7 +545,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_stream)");
 
   // 1. absorb
-  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, q_rope, d_r);
   if (st != LLA_OK) return st;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -543,11 +560,11 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
     a.total = (long long)B * H * N;
     a.P = d.P;
     a.W = d.W;
-    a.row_k = r_k * esz;
+    a.row_k = rq * esz;
     a.row_v = r_v * esz;
     a.nseg_k = d.nseg_k;
     a.nseg_v = d.nseg_v;
-    a.r_k = r_k;
+    a.r_k = rq;
     a.tile = d.tile;
     a.nstage = d.nstage;
     a.stage_bytes = d.stage_bytes;

@@ -65,10 +65,13 @@ struct DecodePlan {
 
 lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePlan* plan);
 
+// q_rope [B*H][d_r] (or null): the decoupled rotary branch; the key rows of
+// zk then hold r_k latent values followed by d_r rotated rotary-key values.
 lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, int B, int H,
                       int d_h, int N, long long n_cap, int r_k, int r_v, const float* dk,
                       const float* dv, const float* mu_k, const float* mu_v, float scale,
-                      float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+                      float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                      const float* q_rope = nullptr, int d_r = 0);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -90,13 +93,16 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
                             size_t ws_bytes, cudaStream_t stream);
 
 // Kernels shared by the per-head and LLA-2D decode paths (decode.cu).
-// k_absorb writes q' (fp32, [B*H][r_k]) to qp when qp is non-null, and when
-// qsw is non-null also the bf16 copy LLA-2D stages per sequence: for each b,
-// an hp x r_k K-major 128B-swizzled operand (rows >= H zero), r_k a
-// multiple of 64, at qsw + b * (r_k / 64) * hp * 128.
+// k_absorb writes q' (fp32, [B*H][r_k + d_r]) to qp when qp is non-null, and
+// when qsw is non-null also the bf16 copy LLA-2D stages per sequence: for
+// each b, an hp x (r_k + d_r) K-major 128B-swizzled operand (rows >= H
+// zero), r_k + d_r a multiple of 64, at qsw + b * ((r_k + d_r) / 64) * hp *
+// 128. With q_rope non-null the last d_r columns of q' are the rotary query
+// [B*H][d_r] times scale * log2(e) (not absorbed).
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
-                         unsigned char* qsw = nullptr, int hp = 0);
+                         unsigned char* qsw = nullptr, int hp = 0, const float* q_rope = nullptr,
+                         int d_r = 0);
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
                           long long P, int shared, float* out, float* lse, cudaStream_t stream,

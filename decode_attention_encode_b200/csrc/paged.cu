@@ -194,7 +194,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
   long long* plan = reinterpret_cast<long long*>(wsb + pp.off_plan);
   int4* wstart = reinterpret_cast<int4*>(wsb + pp.off_wstart);
 
-  StreamFn fn = pick_stream_kernel(esz, d.lpt, d.sk, d.exact, true);
+  StreamFn fn = pick_stream_kernel(esz, d.lpt, d.sk, d.sv, d.exact, true);
   if (!fn) return fail(LLA_ERR_UNSUPPORTED, "no decode kernel for this latent shape");
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)d.smem_bytes);

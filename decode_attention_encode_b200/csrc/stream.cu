@@ -524,24 +524,37 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
 }
 
 template <int ESZ, bool PAGED>
-StreamFn pick_stream(int lpt, int s, bool exact) {
+StreamFn pick_stream(int lpt, int sk, int sv, bool exact) {
 #define LLA_KERNEL(L, SK_, SV_, EX) \
   (PAGED ? k_stream_paged<ESZ, L, SK_, SV_, EX> : k_stream<ESZ, L, SK_, SV_, EX>)
-  if (!exact) {
-    switch (lpt) {
-      case 1: return LLA_KERNEL(1, 4, 4, false);
-      case 2: return LLA_KERNEL(2, 4, 4, false);
-      case 4: return LLA_KERNEL(4, 4, 4, false);
-      case 8: return LLA_KERNEL(8, 4, 4, false);
-    }
-    return nullptr;
+#define LLA_CASE(L, SK_, SV_, EX) \
+  if (lpt == L && sk == SK_ && sv == SV_ && exact == EX) return LLA_KERNEL(L, SK_, SV_, EX);
+  // every lanes-per-token count: equal K/V segment counts, exact; and the
+  // generic masked kernel
+  LLA_CASE(1, 1, 1, true) LLA_CASE(1, 2, 2, true) LLA_CASE(1, 3, 3, true) LLA_CASE(1, 4, 4, true)
+  LLA_CASE(2, 1, 1, true) LLA_CASE(2, 2, 2, true) LLA_CASE(2, 3, 3, true) LLA_CASE(2, 4, 4, true)
+  LLA_CASE(4, 1, 1, true) LLA_CASE(4, 2, 2, true) LLA_CASE(4, 3, 3, true) LLA_CASE(4, 4, 4, true)
+  LLA_CASE(8, 1, 1, true) LLA_CASE(8, 2, 2, true) LLA_CASE(8, 3, 3, true) LLA_CASE(8, 4, 4, true)
+  LLA_CASE(1, 4, 4, false) LLA_CASE(2, 4, 4, false) LLA_CASE(4, 4, 4, false)
+  LLA_CASE(8, 4, 4, false)
+  if constexpr (ESZ == 2) {
+    // bf16 rows of different K and V widths (asymmetric ranks, a rotary
+    // branch on the key side) at 8 lanes per token: exact when both widths
+    // are multiples of 128 bytes, else masked with per-axis segment counts
+    LLA_CASE(8, 1, 2, true) LLA_CASE(8, 1, 3, true) LLA_CASE(8, 1, 4, true)
+    LLA_CASE(8, 2, 1, true) LLA_CASE(8, 2, 3, true) LLA_CASE(8, 2, 4, true)
+    LLA_CASE(8, 3, 1, true) LLA_CASE(8, 3, 2, true) LLA_CASE(8, 3, 4, true)
+    LLA_CASE(8, 4, 1, true) LLA_CASE(8, 4, 2, true) LLA_CASE(8, 4, 3, true)
+    LLA_CASE(8, 1, 1, false) LLA_CASE(8, 1, 2, false) LLA_CASE(8, 1, 3, false)
+    LLA_CASE(8, 1, 4, false) LLA_CASE(8, 2, 1, false) LLA_CASE(8, 2, 2, false)
+    LLA_CASE(8, 2, 3, false) LLA_CASE(8, 2, 4, false) LLA_CASE(8, 3, 1, false)
+    LLA_CASE(8, 3, 2, false) LLA_CASE(8, 3, 3, false) LLA_CASE(8, 3, 4, false)
+    LLA_CASE(8, 4, 1, false) LLA_CASE(8, 4, 2, false) LLA_CASE(8, 4, 3, false)
+    // rows of 160 bf16 (20 segments; r_v = 160 of the 96 / 160 split at 4x,
+    // r = 80 at 2 lanes) exactly, five segments per lane
+    LLA_CASE(4, 3, 5, true) LLA_CASE(4, 5, 3, true) LLA_CASE(4, 5, 5, true)
+    LLA_CASE(2, 5, 5, true)
   }
-#define LLA_CASE(L, S) \
-  if (lpt == L && s == S) return LLA_KERNEL(L, S, S, true);
-  LLA_CASE(1, 1) LLA_CASE(1, 2) LLA_CASE(1, 3) LLA_CASE(1, 4)
-  LLA_CASE(2, 1) LLA_CASE(2, 2) LLA_CASE(2, 3) LLA_CASE(2, 4)
-  LLA_CASE(4, 1) LLA_CASE(4, 2) LLA_CASE(4, 3) LLA_CASE(4, 4)
-  LLA_CASE(8, 1) LLA_CASE(8, 2) LLA_CASE(8, 3) LLA_CASE(8, 4)
 #undef LLA_CASE
 #undef LLA_KERNEL
   return nullptr;
@@ -549,9 +562,12 @@ StreamFn pick_stream(int lpt, int s, bool exact) {
 
 }  // namespace
 
-StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact, bool paged) {
-  if (paged) return esz == 2 ? pick_stream<2, true>(lpt, s, exact) : pick_stream<4, true>(lpt, s, exact);
-  return esz == 2 ? pick_stream<2, false>(lpt, s, exact) : pick_stream<4, false>(lpt, s, exact);
+StreamFn pick_stream_kernel(int esz, int lpt, int sk, int sv, bool exact, bool paged) {
+  if (paged)
+    return esz == 2 ? pick_stream<2, true>(lpt, sk, sv, exact)
+                    : pick_stream<4, true>(lpt, sk, sv, exact);
+  return esz == 2 ? pick_stream<2, false>(lpt, sk, sv, exact)
+                  : pick_stream<4, false>(lpt, sk, sv, exact);
 }
 
 }  // namespace lla

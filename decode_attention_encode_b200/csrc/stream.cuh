@@ -52,9 +52,9 @@ struct SeqInfo {
 using StreamFn = void (*)(StreamArgs);
 
 // The k_stream instantiation for a latent element size (2 or 4 bytes),
-// lanes per token and segments per lane; exact means every lane's segments
-// are in range; paged selects the paged / ragged store. nullptr if there is
-// none.
-StreamFn pick_stream_kernel(int esz, int lpt, int s, bool exact, bool paged = false);
+// lanes per token and K / V segments per lane; exact means every lane's
+// segments are in range; paged selects the paged / ragged store. nullptr if
+// there is none.
+StreamFn pick_stream_kernel(int esz, int lpt, int sk, int sv, bool exact, bool paged = false);
 
 }  // namespace lla

@@ -137,6 +137,40 @@ LLA_API lla_status lla_decode_attn(const float *q, const void *zk, const void *z
                            void *stream);
 
 /* --------------------------------------------------------------------------
+ * Per-head absorbed decode with a decoupled rotary branch, one (layer d,
+ * loop t) step.
+ *
+ * §7 ("Per-head LLA versus LLA-2D at inference") notes that RoPE blocks
+ * exact absorption of the positional part and splits attention, MLA-style,
+ * into a NoPE latent content path and a small explicit rotary branch that a
+ * looped model shares across the loops of a token. Scores become
+ *   s_j = scale * ( q[b][h] . khat_j + q_rope[b][h] . krope_j ),
+ * with khat_j = dk_t[h] z_j + mu_k_t[h] as in lla_decode_attn; out and lse
+ * are defined from s_j as there. The rotary keys are stored already rotated
+ * at their own positions (they do not change between loops), and q_rope is
+ * this loop's rotary query, already rotated at the current position.
+ *
+ * Arguments as lla_decode_attn, plus:
+ *   q_rope  [B][H][d_r] fp32, 4-byte aligned.
+ *   d_r     rotary width, a positive multiple of 8.
+ *   zk      [B][H][n_cap][r_k + d_r]: each key row holds the r_k latent
+ *           values followed by the d_r rotated rotary-key values, so one
+ *           row read serves both paths. r_k + d_r obeys the rank limits of
+ *           lla_decode_attn (at most 256 for bf16, 128 for fp32).
+ *   workspace  at least lla_decode_attn_workspace(B, H, N, r_k + d_r, r_v)
+ *           bytes.
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla_decode_attn_rope(const float *q, const float *q_rope,
+                                        const void *zk, const void *zv,
+                                        lla_dtype zdt, int B, int H, int d_h,
+                                        int d_r, int N, int n_cap, int r_k,
+                                        int r_v, const float *dk_t,
+                                        const float *dv_t, const float *mu_k_t,
+                                        const float *mu_v_t, float scale,
+                                        float *out, float *lse, void *workspace,
+                                        size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
  * Per-head absorbed decode without a caller workspace. The paper has no
  * counterpart: this is a deployment convenience of this library.
  *

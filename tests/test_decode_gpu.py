@@ -61,7 +61,8 @@ def test_fp32_ranks(r):
     run_case(2, 3, 32, 333, r, r, F32, mu=True, seed=r)
 
 
-@pytest.mark.parametrize("r_k, r_v", [(96, 160), (24, 40), (16, 24), (8, 256), (40, 40)])
+@pytest.mark.parametrize("r_k, r_v", [(96, 160), (160, 96), (160, 160), (80, 80), (24, 40),
+                                      (16, 24), (8, 256), (40, 40), (192, 128), (128, 64)])
 def test_asymmetric_and_odd_ranks(r_k, r_v):
     run_case(2, 4, 128, 517, r_k, r_v, BF16, mu=True, seed=r_k + r_v)
 
