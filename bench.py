@@ -189,17 +189,21 @@ class DecodeWorkload:
     A paged config keeps each layer's store as a pool of pages with one
     shared block table and seeded ragged lengths; its step is the T x L
     attention calls alone (a newest-token write there is a scatter into
-    each sequence's last page, which this workload does not time)."""
+    each sequence's last page, which this workload does not time). A rotary
+    config stores [latent | rotated rotary key] key rows and takes one
+    rotary query per (layer, loop) call; its step is the attention calls
+    alone as well."""
 
     def __init__(self, cfg: synth.DecodeConfig, device: str, seed_offset: int = 0):
         self.cfg = cfg
         c = cfg
         s = c.seed + seed_offset
         self.paged = c.page_size > 0
-        self.write_latents = (not c.two_d and not self.paged and c.dtype == "bf16"
-                              and c.d_h % 64 == 0)
+        self.rope = c.d_r > 0
+        self.write_latents = (not c.two_d and not self.paged and not self.rope
+                              and c.dtype == "bf16" and c.d_h % 64 == 0)
         n_cap = c.N + 1 if self.write_latents else c.N
-        zk_shape = (c.B, n_cap, c.r_k) if c.two_d else (c.B, c.H, n_cap, c.r_k)
+        zk_shape = (c.B, n_cap, c.r_k) if c.two_d else (c.B, c.H, n_cap, c.r_k + c.d_r)
         zv_shape = (c.B, n_cap, c.r_v) if c.two_d else (c.B, c.H, n_cap, c.r_v)
         if self.paged:
             lens = c.lengths()
@@ -217,12 +221,16 @@ class DecodeWorkload:
         self.dv = synth.orthonormal(c.L * c.T * c.H, c.d_h, c.r_v, s + 4, device).view(
             c.L, c.T, c.H, c.d_h, c.r_v)
         self.q = synth.queries((c.L, c.T, c.B, c.H, c.d_h), c.d_h, s + 5, device)
+        if self.rope:
+            self.q_rope = synth.queries((c.L, c.T, c.B, c.H, c.d_r), c.d_r, s + 13, device)
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty((c.L, c.T, c.B, c.H), device=device, dtype=torch.float32)
         import decode_attention_encode_b200 as lla
         self.lla = lla
         if self.paged:
             need = lla.lla_decode_attn_paged_workspace(c.B, c.H, c.r_k, c.r_v)
+        elif self.rope:
+            need = lla.lla_decode_attn_workspace(c.B, c.H, c.N, c.r_k + c.d_r, c.r_v)
         else:
             wsfn = lla.lla2d_decode_attn_workspace if c.two_d else lla.lla_decode_attn_workspace
             need = wsfn(c.B, c.H, c.N, c.r_k, c.r_v)
@@ -257,10 +265,11 @@ class DecodeWorkload:
         if self.write_latents:
             self.write_newest(self.xk if xk is None else xk, self.xv if xv is None else xv)
 
-    def call(self, l, t, q=None, out=None, lse=None):
+    def call(self, l, t, q=None, out=None, lse=None, q_rope=None):
         """The (layer l, loop t) decode call through the public API."""
         c = self.cfg
         q = self.q if q is None else q
+        q_rope = getattr(self, "q_rope", None) if q_rope is None else q_rope
         out = self.out if out is None else out
         lse = self.lse if lse is None else lse
         if self.paged:
@@ -268,6 +277,10 @@ class DecodeWorkload:
                                            self.seq_lens, self.dk[l, t], self.dv[l, t],
                                            scale=self.scale, out=out[l, t], lse=lse[l, t],
                                            workspace=self.ws)
+        elif self.rope:
+            self.lla.lla_decode_attn_rope(q[l, t], q_rope[l, t], self.zk[l], self.zv[l],
+                                          self.dk[l, t], self.dv[l, t], N=c.N, scale=self.scale,
+                                          out=out[l, t], lse=lse[l, t], workspace=self.ws)
         else:
             self.fn(q[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
                     scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
@@ -507,8 +520,9 @@ def describe(cfg: synth.DecodeConfig) -> str:
     kind = "LLA-2D" if cfg.two_d else "per-head LLA"
     n = (f"N={cfg.N} mean (ragged +-{int(cfg.spread * 100)}%, {cfg.tokens()} tokens), "
          f"{cfg.page_size}-token pages" if cfg.page_size else f"N={cfg.N}")
+    rope = f" d_r={cfg.d_r} (rotary branch)" if cfg.d_r else ""
     return (f"{cfg.name}: {kind} decode, L={cfg.L} T={cfg.T} H={cfg.H} d_h={cfg.d_h} "
-            f"r_k={cfg.r_k} r_v={cfg.r_v} B={cfg.B} {n} {cfg.dtype} latents")
+            f"r_k={cfg.r_k}{rope} r_v={cfg.r_v} B={cfg.B} {n} {cfg.dtype} latents")
 
 
 def run_lla(args, world, rank, local):
@@ -584,6 +598,8 @@ def run_lla(args, world, rank, local):
         d2h = torch.cuda.Stream()
         q_host = wl.q.to("cpu").pin_memory()
         q_dev = torch.empty_like(wl.q)
+        qr_host = wl.q_rope.to("cpu").pin_memory() if wl.rope else None
+        qr_dev = torch.empty_like(wl.q_rope) if wl.rope else None
         x_hosts = [wl.xk.to("cpu").pin_memory(), wl.xv.to("cpu").pin_memory()] \
             if wl.write_latents else []
         x_devs = [torch.empty_like(wl.xk), torch.empty_like(wl.xv)] if wl.write_latents else []
@@ -599,6 +615,8 @@ def run_lla(args, world, rank, local):
                 for t in range(c.T):
                     for l in range(c.L):
                         q_dev[l, t].copy_(q_host[l, t], non_blocking=True)
+                        if wl.rope:
+                            qr_dev[l, t].copy_(qr_host[l, t], non_blocking=True)
                         in_ev[t][l].record(h2d)
                 for d_, h_ in zip(x_devs, x_hosts):
                     d_.copy_(h_, non_blocking=True)
@@ -606,7 +624,7 @@ def run_lla(args, world, rank, local):
             for t in range(c.T):
                 for l in range(c.L):
                     stream.wait_event(in_ev[t][l])
-                    wl.call(l, t, q=q_dev)
+                    wl.call(l, t, q=q_dev, q_rope=qr_dev)
                     done_ev[t][l].record(stream)
                     with torch.cuda.stream(d2h):
                         d2h.wait_event(done_ev[t][l])
@@ -630,7 +648,8 @@ def run_lla(args, world, rank, local):
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
         e2e = {"value": aggregate_rate(tokens_per_step, e2e_ms, world), "unit": UNIT,
-               "h2d_bytes_per_step": q_host.numel() * 4 + sum(h_.numel() * 2 for h_ in x_hosts),
+               "h2d_bytes_per_step": (q_host.numel() + (qr_host.numel() if wl.rope else 0)) * 4
+                                     + sum(h_.numel() * 2 for h_ in x_hosts),
                "d2h_bytes_per_step": (out_host.numel() + lse_host.numel()) * 4,
                "copies": "pinned host memory, per-call chunks on separate copy streams"}
 

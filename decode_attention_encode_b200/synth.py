@@ -114,7 +114,8 @@ class DecodeConfig:
     """One decode workload. ``two_d`` selects LLA-2D (one latent per token
     and layer shared by all heads). ``page_size`` > 0 selects a paged store
     whose sequences have seeded ragged lengths with mean ``N`` (uniform
-    within +-``spread`` N)."""
+    within +-``spread`` N). ``d_r`` > 0 adds a decoupled rotary branch of
+    that width to every key row."""
     name: str
     L: int           # layers (D in the paper)
     T: int           # loops
@@ -131,6 +132,7 @@ class DecodeConfig:
     note: str = field(default="", compare=False)
     page_size: int = 0
     spread: float = 0.0
+    d_r: int = 0
 
     @property
     def esz(self) -> int:
@@ -151,7 +153,7 @@ class DecodeConfig:
         return int(self.lengths().sum())
 
     def store_bytes_per_layer(self) -> int:
-        per_tok = (self.r_k + self.r_v) * self.esz * (1 if self.two_d else self.H)
+        per_tok = (self.r_k + self.d_r + self.r_v) * self.esz * (1 if self.two_d else self.H)
         return self.tokens() * per_tok
 
     def step_bytes(self) -> int:
@@ -203,4 +205,7 @@ class EncodeConfig:
 C5_ENCODE = EncodeConfig("encode_32x", L=24, T=4, G=16, d_loop=128, r=16, N=32768,
                          n_cal=2048)
 
-DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED)}
+# the 4x geometry with a 64-wide decoupled rotary branch on the key side
+C2_ROPE = DecodeConfig("perhead_4x_rope", L=24, T=4, H=16, d_h=128, r_k=128, r_v=128, B=64,
+                       N=4096, dtype="bf16", decay=True, d_r=64)
+DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE)}
