@@ -25,4 +25,6 @@ from ._lib import (  # noqa: F401
     lla_decode_attn_rope,
     lla_decode_attn_workspace,
     lla_encode,
+    lla_encode_bias,
+    lla_encode_with_bias,
 )

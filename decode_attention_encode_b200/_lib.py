@@ -37,7 +37,7 @@ EXPORTS = (
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn",
-    "lla_encode",
+    "lla_encode", "lla_encode_bias", "lla_encode_with_bias",
 )
 
 _lock = threading.Lock()
@@ -74,6 +74,9 @@ _SIGS = {
     "lla2d_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
                           [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla_encode": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp], _c_int),
+    "lla_encode_bias": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
+    "lla_encode_with_bias": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp],
+                             _c_int),
 }
 
 
@@ -334,5 +337,35 @@ def lla_encode(x, w_down_t, mu=None, z=None, z_row_stride=None, z_group_stride=N
         raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
     st = lib().lla_encode(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t), _ptr(mu),
                           _ptr(z), int(z_row_stride), int(z_group_stride), _stream(stream))
+    _check(st)
+    return z
+
+
+def lla_encode_bias(w_down_t, mu, muw=None, stream=None):
+    """mu W_down of a codec, once: w_down_t [G,r,K] bf16, mu [G,K] fp32.
+    Returns muw [G,r] fp32."""
+    _need_cuda(w_down_t, mu, muw)
+    G, r, K = w_down_t.shape
+    if muw is None:
+        muw = torch.empty((G, r), device=w_down_t.device, dtype=torch.float32)
+    _check(lib().lla_encode_bias(_ptr(w_down_t), _ptr(mu), G, K, r, _ptr(muw), _stream(stream)))
+    return muw
+
+
+def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_group_stride=None,
+                         stream=None):
+    """lla_encode with the mean term precomputed by lla_encode_bias (muw
+    [G,r] fp32, or None for a zero mean). Returns z."""
+    _need_cuda(x, w_down_t, muw)
+    T, N, G, d_loop = x.shape
+    r = w_down_t.shape[1]
+    if z is None:
+        z = torch.empty((G, N, r), device=x.device, dtype=torch.bfloat16)
+        z_row_stride, z_group_stride = r, N * r
+    if z_row_stride is None or z_group_stride is None:
+        raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
+    st = lib().lla_encode_with_bias(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t),
+                                    _ptr(muw), _ptr(z), int(z_row_stride), int(z_group_stride),
+                                    _stream(stream))
     _check(st)
     return z

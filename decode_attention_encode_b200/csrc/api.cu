@@ -132,6 +132,35 @@ lla_status lla::check_decode_args(const float* q, const void* zk, const void* zv
   return LLA_OK;
 }
 
+namespace {
+
+// Argument checks shared by the encode entry points.
+lla_status check_encode_args(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,
+                             const void* w_down_t, const float* mu, void* z,
+                             long long z_row_stride, long long z_group_stride) {
+  if (xdt != LLA_BF16) return fail(LLA_ERR_INVALID_ARG, "xdt must be LLA_BF16");
+  if (!x || !w_down_t || !z) return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be non-NULL");
+  if (!aligned(x, 16) || !aligned(w_down_t, 16) || !aligned(z, 16))
+    return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be 16-byte aligned");
+  if (mu && !aligned(mu, 4)) return fail(LLA_ERR_INVALID_ARG, "mu must be 4-byte aligned");
+  if (T < 1 || N < 1 || G < 1) return fail(LLA_ERR_INVALID_ARG, "T, N and G must be >= 1");
+  if (d_loop < 64 || d_loop % 64)
+    return fail(LLA_ERR_INVALID_ARG, "d_loop must be a positive multiple of 64");
+  if ((long long)T * d_loop > (1LL << 30)) return fail(LLA_ERR_INVALID_ARG, "T*d_loop too large");
+  if (r < 8 || r > 256 || r % 8) return fail(LLA_ERR_INVALID_ARG, "r must be a multiple of 8 in 8..256");
+  if (z_row_stride < r || z_group_stride < 0 || z_row_stride % 8 || z_group_stride % 8)
+    return fail(LLA_ERR_INVALID_ARG, "z strides must be multiples of 8 with z_row_stride >= r");
+  if (G > 1) {
+    const bool groups_outer = z_group_stride >= (long long)(N - 1) * z_row_stride + r;
+    const bool rows_outer = z_row_stride >= (long long)(G - 1) * z_group_stride + r && z_group_stride >= r;
+    if (!groups_outer && !rows_outer)
+      return fail(LLA_ERR_INVALID_ARG, "z strides make output rows overlap");
+  }
+  return LLA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* lla_status_string(lla_status s) {
@@ -285,26 +314,34 @@ lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_l
                       const void* w_down_t, const float* mu, void* z, long long z_row_stride,
                       long long z_group_stride, void* stream) {
   g_last_error[0] = '\0';
-  if (xdt != LLA_BF16) return fail(LLA_ERR_INVALID_ARG, "xdt must be LLA_BF16");
-  if (!x || !w_down_t || !z) return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be non-NULL");
-  if (!aligned(x, 16) || !aligned(w_down_t, 16) || !aligned(z, 16))
-    return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be 16-byte aligned");
-  if (mu && !aligned(mu, 4)) return fail(LLA_ERR_INVALID_ARG, "mu must be 4-byte aligned");
-  if (T < 1 || N < 1 || G < 1) return fail(LLA_ERR_INVALID_ARG, "T, N and G must be >= 1");
-  if (d_loop < 64 || d_loop % 64)
-    return fail(LLA_ERR_INVALID_ARG, "d_loop must be a positive multiple of 64");
-  if ((long long)T * d_loop > (1LL << 30)) return fail(LLA_ERR_INVALID_ARG, "T*d_loop too large");
-  if (r < 8 || r > 256 || r % 8) return fail(LLA_ERR_INVALID_ARG, "r must be a multiple of 8 in 8..256");
-  if (z_row_stride < r || z_group_stride < 0 || z_row_stride % 8 || z_group_stride % 8)
-    return fail(LLA_ERR_INVALID_ARG, "z strides must be multiples of 8 with z_row_stride >= r");
-  if (G > 1) {
-    const bool groups_outer = z_group_stride >= (long long)(N - 1) * z_row_stride + r;
-    const bool rows_outer = z_row_stride >= (long long)(G - 1) * z_group_stride + r && z_group_stride >= r;
-    if (!groups_outer && !rows_outer)
-      return fail(LLA_ERR_INVALID_ARG, "z strides make output rows overlap");
-  }
+  lla_status st = check_encode_args(x, xdt, T, N, G, d_loop, r, w_down_t, mu, z, z_row_stride,
+                                    z_group_stride);
+  if (st != LLA_OK) return st;
   return run_encode(x, T, N, G, d_loop, r, w_down_t, mu, z, z_row_stride, z_group_stride,
                     static_cast<cudaStream_t>(stream));
+}
+
+lla_status lla_encode_bias(const void* w_down_t, const float* mu, int G, int K, int r, float* muw,
+                           void* stream) {
+  g_last_error[0] = '\0';
+  if (!w_down_t || !mu || !muw) return fail(LLA_ERR_INVALID_ARG, "w_down_t, mu and muw must be non-NULL");
+  if (!aligned(w_down_t, 16) || !aligned(mu, 16) || !aligned(muw, 4))
+    return fail(LLA_ERR_INVALID_ARG, "w_down_t and mu must be 16-byte aligned, muw 4-byte");
+  if (G < 1 || K < 8 || K % 8) return fail(LLA_ERR_INVALID_ARG, "G >= 1 and K a positive multiple of 8");
+  if (r < 1 || r > 65535 * 8) return fail(LLA_ERR_INVALID_ARG, "r out of range");
+  return run_encode_bias(w_down_t, mu, G, K, r, muw, static_cast<cudaStream_t>(stream));
+}
+
+lla_status lla_encode_with_bias(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop,
+                                int r, const void* w_down_t, const float* muw, void* z,
+                                long long z_row_stride, long long z_group_stride, void* stream) {
+  g_last_error[0] = '\0';
+  lla_status st = check_encode_args(x, xdt, T, N, G, d_loop, r, w_down_t, nullptr, z,
+                                    z_row_stride, z_group_stride);
+  if (st != LLA_OK) return st;
+  if (muw && !aligned(muw, 4)) return fail(LLA_ERR_INVALID_ARG, "muw must be 4-byte aligned");
+  return run_encode(x, T, N, G, d_loop, r, w_down_t, nullptr, z, z_row_stride, z_group_stride,
+                    static_cast<cudaStream_t>(stream), muw);
 }
 
 }  // extern "C"

@@ -44,6 +44,7 @@ struct EncodeArgs {
   int nstage, b_bytes, stage_bytes;
   uint32_t tmem_cols;
   const float* mu;
+  const float* muw;  // precomputed mu W [G][r] (then mu is unused), or null
   const __nv_bfloat16* wt;
   __nv_bfloat16* z;
   long long zrs, zgs;
@@ -209,7 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!epi_sync()) break;  // previous tile's readers of muw are done
         for (int c = ew; c < a.r; c += 4) {
           float acc = 0.f;
-          if (a.mu) {
+          if (a.muw) {
+            acc = a.muw[(size_t)g * a.r + c];
+          } else if (a.mu) {
             const float* mu = a.mu + (size_t)g * a.K;
             const __nv_bfloat16* w = a.wt + ((size_t)g * a.r + c) * a.K;
             for (int k = lane; k < a.K; k += 32) acc = fmaf(mu[k], __bfloat162float(w[k]), acc);
@@ -281,6 +284,48 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+// muw[g][c] = sum_k mu[g][k] W_down[g][k][c] (fp32): one warp per (g, c),
+// 16-byte loads of W^T, eight in flight per lane.
+__global__ void __launch_bounds__(256) k_encode_bias(const __nv_bfloat16* wt, const float* mu,
+                                                     int G, int K, int r, float* muw) {
+  const int g = blockIdx.x;
+  const int c = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= r) return;
+  const uint4* w = reinterpret_cast<const uint4*>(wt + ((size_t)g * r + c) * K);
+  const float4* m = reinterpret_cast<const float4*>(mu + (size_t)g * K);
+  const int n8 = K / 8;
+  float acc = 0.f;
+  for (int i0 = lane; i0 < n8; i0 += 32 * 8) {
+    uint4 wv[8];
+    float4 m0[8], m1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = i0 + 32 * k;
+      if (i < n8) {
+        wv[k] = __ldg(w + i);
+        m0[k] = __ldg(m + 2 * i);
+        m1[k] = __ldg(m + 2 * i + 1);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (i0 + 32 * k < n8) {
+        acc = fmaf(m0[k].x, bf16lo(wv[k].x), acc);
+        acc = fmaf(m0[k].y, bf16hi(wv[k].x), acc);
+        acc = fmaf(m0[k].z, bf16lo(wv[k].y), acc);
+        acc = fmaf(m0[k].w, bf16hi(wv[k].y), acc);
+        acc = fmaf(m1[k].x, bf16lo(wv[k].z), acc);
+        acc = fmaf(m1[k].y, bf16hi(wv[k].z), acc);
+        acc = fmaf(m1[k].z, bf16lo(wv[k].w), acc);
+        acc = fmaf(m1[k].w, bf16hi(wv[k].w), acc);
+      }
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) muw[(size_t)g * r + c] = acc;
+}
+
 }  // namespace
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
@@ -309,9 +354,16 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
   return true;
 }
 
+lla_status run_encode_bias(const void* wt, const float* mu, int G, int K, int r, float* muw,
+                           cudaStream_t stream) {
+  k_encode_bias<<<dim3(G, (r + 7) / 8), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(wt),
+                                                          mu, G, K, r, muw);
+  return check_cuda(cudaGetLastError(), "launch k_encode_bias");
+}
+
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const float* muw) {
   const int K = T * d_loop;
   const int r_pad = (r + 15) / 16 * 16;
   EncodeArgs a{};
@@ -330,6 +382,7 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   while (cols < (uint32_t)(2 * r_pad)) cols <<= 1;
   a.tmem_cols = cols;
   a.mu = mu;
+  a.muw = muw;
   a.wt = static_cast<const __nv_bfloat16*>(wt);
   a.z = static_cast<__nv_bfloat16*>(z);
   a.zrs = zrs;

@@ -115,6 +115,11 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
                          float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
-                      const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream);
+                      const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream,
+                      const float* muw = nullptr);
+
+// muw[g][c] = sum_k mu[g][k] W_down[g][k][c] over K = T * d_loop (fp32).
+lla_status run_encode_bias(const void* wt, const float* mu, int G, int K, int r, float* muw,
+                           cudaStream_t stream);
 
 }  // namespace lla

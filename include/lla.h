@@ -314,6 +314,34 @@ LLA_API lla_status lla_encode(const void *x, lla_dtype xdt, int T, int N, int G,
                               const float *mu, void *z, long long z_row_stride,
                               long long z_group_stride, void *stream);
 
+/* --------------------------------------------------------------------------
+ * The mean term of the latent write, computed once per codec.
+ *
+ * §3 Eq. 2 subtracts the codec mean before the down-projection; since
+ * (x - mu) W_down = x W_down - mu W_down and mu, W_down are fixed codec
+ * parameters, b = mu W_down is a constant of the codec:
+ *   muw[g][c] = sum_k mu[g][k] * W_down[g][k][c]     (fp32 accumulation)
+ * lla_encode forms it inside every call, which is cheap at the per-head
+ * shapes but not for a wide LLA-2D stack (K = T H d_head). Computing it once
+ * here and calling lla_encode_with_bias avoids that.
+ *   w_down_t  [G][r][K] bf16 (W_down transposed, as for lla_encode),
+ *             16-byte aligned; K = T * d_loop, a positive multiple of 8.
+ *   mu        [G][K] fp32, 16-byte aligned.
+ *   muw       [G][r] fp32 output.
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla_encode_bias(const void *w_down_t, const float *mu, int G,
+                                   int K, int r, float *muw, void *stream);
+
+/* lla_encode with the mean term given as muw = mu W_down (from
+ * lla_encode_bias), or NULL for a zero mean:
+ *   z[g][n][c] = bf16_rne( sum_k xs[k] * W_down[g][k][c] - muw[g][c] ).
+ * Arguments and limits otherwise as lla_encode. */
+LLA_API lla_status lla_encode_with_bias(const void *x, lla_dtype xdt, int T, int N,
+                                        int G, int d_loop, int r,
+                                        const void *w_down_t, const float *muw,
+                                        void *z, long long z_row_stride,
+                                        long long z_group_stride, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -103,3 +103,37 @@ def test_encode_wide_stack_for_lla2d_geometry():
     z = lla.lla_encode(x, w_t, m)
     torch.cuda.synchronize()
     check(z, oracle.encode(to_f64(x), to_f64(w), to_f64(m)))
+
+
+def test_encode_bias_is_the_mean_term():
+    # muw = mu W_down per group, against the oracle's encode of a zero input
+    # (Eq. 2 with x = 0 gives -mu W_down exactly)
+    T, G, d, r = 4, 3, 128, 40
+    _, w, w_t, m = make(T, 1, G, d, r, True, seed=21)
+    muw = lla.lla_encode_bias(w_t, m)
+    torch.cuda.synchronize()
+    zero = np.zeros((T, 1, G, d))
+    ref = -oracle.encode(zero, to_f64(w), to_f64(m))[:, 0, :]
+    got = to_f64(muw)
+    assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("T, N, G, d_loop, r", [(4, 300, 3, 64, 16), (4, 200, 1, 2048, 256),
+                                                (32, 150, 2, 128, 16), (4, 129, 2, 128, 128)])
+def test_encode_with_precomputed_bias(T, N, G, d_loop, r):
+    x, w, w_t, m = make(T, N, G, d_loop, r, True, seed=T + r)
+    muw = lla.lla_encode_bias(w_t, m)
+    z = lla.lla_encode_with_bias(x, w_t, muw)
+    z0 = lla.lla_encode_with_bias(x, w_t, None)
+    torch.cuda.synchronize()
+    check(z, oracle.encode(to_f64(x), to_f64(w), to_f64(m)))
+    check(z0, oracle.encode(to_f64(x), to_f64(w), None))
+    assert lla.device_status() == 0
+
+
+def test_encode_huginn_scale_loop_count():
+    # T = 32 loops of d_head = 128: a 4096-wide stack per head
+    x, w, w_t, m = make(32, 257, 4, 128, 16, True, seed=33)
+    z = lla.lla_encode(x, w_t, m)
+    torch.cuda.synchronize()
+    check(z, oracle.encode(to_f64(x), to_f64(w), to_f64(m)))
