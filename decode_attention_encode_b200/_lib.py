@@ -37,7 +37,7 @@ EXPORTS = (
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn",
-    "lla_encode", "lla_encode_bias", "lla_encode_with_bias",
+    "lla_encode", "lla_encode_bias", "lla_encode_with_bias_workspace", "lla_encode_with_bias",
 )
 
 _lock = threading.Lock()
@@ -75,8 +75,9 @@ _SIGS = {
                           [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla_encode": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp], _c_int),
     "lla_encode_bias": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
-    "lla_encode_with_bias": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp],
-                             _c_int),
+    "lla_encode_with_bias_workspace": ([_c_int] * 5, _c_size),
+    "lla_encode_with_bias": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp,
+                                                              _c_size, _vp], _c_int),
 }
 
 
@@ -353,19 +354,26 @@ def lla_encode_bias(w_down_t, mu, muw=None, stream=None):
 
 
 def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_group_stride=None,
-                         stream=None):
+                         workspace=None, stream=None, split=True):
     """lla_encode with the mean term precomputed by lla_encode_bias (muw
-    [G,r] fp32, or None for a zero mean). Returns z."""
-    _need_cuda(x, w_down_t, muw)
+    [G,r] fp32, or None for a zero mean). With split (default) a workspace
+    is allocated when the shape benefits from a split over K (or pass one).
+    Returns z."""
+    _need_cuda(x, w_down_t, muw, workspace)
     T, N, G, d_loop = x.shape
     r = w_down_t.shape[1]
+    if workspace is None and split:
+        need = int(lib().lla_encode_with_bias_workspace(T, N, G, d_loop, r))
+        if need:
+            workspace = torch.empty(need, device=x.device, dtype=torch.uint8)
     if z is None:
         z = torch.empty((G, N, r), device=x.device, dtype=torch.bfloat16)
         z_row_stride, z_group_stride = r, N * r
     if z_row_stride is None or z_group_stride is None:
         raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().lla_encode_with_bias(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t),
                                     _ptr(muw), _ptr(z), int(z_row_stride), int(z_group_stride),
-                                    _stream(stream))
+                                    _ptr(workspace), ws_bytes, _stream(stream))
     _check(st)
     return z

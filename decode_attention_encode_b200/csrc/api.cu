@@ -332,16 +332,24 @@ lla_status lla_encode_bias(const void* w_down_t, const float* mu, int G, int K, 
   return run_encode_bias(w_down_t, mu, G, K, r, muw, static_cast<cudaStream_t>(stream));
 }
 
+size_t lla_encode_with_bias_workspace(int T, int N, int G, int d_loop, int r) {
+  if (T < 1 || N < 1 || G < 1 || d_loop < 64 || d_loop % 64 || r < 8 || r > 256 || r % 8) return 0;
+  return encode_workspace(T, N, G, d_loop, r);
+}
+
 lla_status lla_encode_with_bias(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop,
                                 int r, const void* w_down_t, const float* muw, void* z,
-                                long long z_row_stride, long long z_group_stride, void* stream) {
+                                long long z_row_stride, long long z_group_stride, void* workspace,
+                                size_t ws_bytes, void* stream) {
   g_last_error[0] = '\0';
   lla_status st = check_encode_args(x, xdt, T, N, G, d_loop, r, w_down_t, nullptr, z,
                                     z_row_stride, z_group_stride);
   if (st != LLA_OK) return st;
-  if (muw && !aligned(muw, 4)) return fail(LLA_ERR_INVALID_ARG, "muw must be 4-byte aligned");
+  if (muw && !aligned(muw, 16)) return fail(LLA_ERR_INVALID_ARG, "muw must be 16-byte aligned");
+  if (workspace && !aligned(workspace, 16))
+    return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   return run_encode(x, T, N, G, d_loop, r, w_down_t, nullptr, z, z_row_stride, z_group_stride,
-                    static_cast<cudaStream_t>(stream), muw);
+                    static_cast<cudaStream_t>(stream), muw, workspace, ws_bytes);
 }
 
 }  // extern "C"

@@ -40,7 +40,10 @@ constexpr int kABytes = kTileM * kChunkK * 2;
 constexpr int kThreads = 192;   // 6 warps
 
 struct EncodeArgs {
+  // work items are (tile, K split) pairs: item = tile * ksplit + split
   int N, G, d_loop, r, r_pad, K, nk, mtiles, tiles, tiles_per_cta;
+  int ksplit, cpk;  // K splits per tile and chunks per split
+  float* part;      // ksplit > 1: fp32 partials [ksplit][G][N][r]
   int nstage, b_bytes, stage_bytes;
   uint32_t tmem_cols;
   const float* mu;
@@ -89,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &tail->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t_begin = blockIdx.x * a.tiles_per_cta;
-  const int t_end = min(t_begin + a.tiles_per_cta, a.tiles);
+  const int t_begin = blockIdx.x * a.tiles_per_cta;  // work items, see EncodeArgs
+  const int t_end = min(t_begin + a.tiles_per_cta, a.tiles * a.ksplit);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.nstage; ++s) {
@@ -120,10 +123,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_w = l2_evict_last_policy();
       int it = 0;
       bool ok = true;
-      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+      for (int item = t_begin; item < t_end && ok; ++item) {
+        const int tile = item / a.ksplit, split = item - tile * a.ksplit;
         const int g = tile / a.mtiles;
         const int m0 = (tile - g * a.mtiles) * kTileM;
-        for (int kc = 0; kc < a.nk; ++kc, ++it) {
+        const int kc0 = split * a.cpk, kc1 = min(a.nk, kc0 + a.cpk);
+        for (int kc = kc0; kc < kc1; ++kc, ++it) {
           const int s = it % a.nstage;
           const uint32_t ph = (uint32_t)(it / a.nstage) & 1u;
           if (!wait_or_abort(smem_u32(&tail->empty[s]), ph ^ 1u, abort_flag, a.status)) {
@@ -152,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kTileM, a.r_pad, false, false);
       int it = 0;
       bool ok = true;
-      for (int tile = t_begin, lt = 0; tile < t_end && ok; ++tile, ++lt) {
+      for (int item = t_begin, lt = 0; item < t_end && ok; ++item, ++lt) {
         const int acc = lt & 1;
         const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
         if (!wait_or_abort(smem_u32(&tail->tempty[acc]), aph ^ 1u, abort_flag, a.status)) {
@@ -161,7 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tbase + (uint32_t)(acc * a.r_pad);
-        for (int kc = 0; kc < a.nk; ++kc, ++it) {
+        const int split = item % a.ksplit;
+        const int kc0 = split * a.cpk, kc1 = min(a.nk, kc0 + a.cpk);
+        for (int kc = kc0; kc < kc1; ++kc, ++it) {
           const int s = it % a.nstage;
           const uint32_t ph = (uint32_t)(it / a.nstage) & 1u;
           if (!wait_or_abort(smem_u32(&tail->full[s]), ph, abort_flag, a.status)) {
@@ -176,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kChunkK / 16; ++kk)
             umma_bf16(d, a_base + (uint64_t)(kk * 2), b_base + (uint64_t)(kk * 2), idesc,
-                      (kc | kk) != 0);
+                      kc != kc0 || kk != 0);
           umma_commit(smem_u32(&tail->empty[s]));
         }
         if (!ok) break;
@@ -203,10 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       return ok;
     };
     int cur_g = -1;
-    for (int tile = t_begin, lt = 0; tile < t_end; ++tile, ++lt) {
+    for (int item = t_begin, lt = 0; item < t_end; ++item, ++lt) {
+      const int tile = item / a.ksplit, split = item - tile * a.ksplit;
       const int g = tile / a.mtiles;
       const int m0 = (tile - g * a.mtiles) * kTileM;
-      if (g != cur_g) {
+      if (g != cur_g && !a.part) {
         if (!epi_sync()) break;  // previous tile's readers of muw are done
         for (int c = ew; c < a.r; c += 4) {
           float acc = 0.f;
@@ -232,10 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * a.r_pad);
       const int n = m0 + row;
       __nv_bfloat16* zrow = a.z + (size_t)g * a.zgs + (size_t)n * a.zrs;
+      // split K: this item's fp32 partial sum; k_encode_reduce finishes it
+      float* prow = a.part ? a.part + (((size_t)split * a.G + g) * a.N + n) * a.r : nullptr;
       for (int cc = 0; cc < a.r_pad; cc += 16) {
         float v[16];
         tmem_ld16(taddr + cc, v);
-        if (n < a.N) {
+        if (n < a.N && prow) {
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const int c0 = cc + 8 * h8;
+            if (c0 < a.r) {
+              float4* dst = reinterpret_cast<float4*>(prow + c0);
+              dst[0] = make_float4(v[8 * h8 + 0], v[8 * h8 + 1], v[8 * h8 + 2], v[8 * h8 + 3]);
+              dst[1] = make_float4(v[8 * h8 + 4], v[8 * h8 + 5], v[8 * h8 + 6], v[8 * h8 + 7]);
+            }
+          }
+        } else if (n < a.N) {
 #pragma unroll
           for (int h8 = 0; h8 < 2; ++h8) {
             const int c0 = cc + 8 * h8;
@@ -326,6 +346,40 @@ __global__ void __launch_bounds__(256) k_encode_bias(const __nv_bfloat16* wt, co
   if (lane == 0) muw[(size_t)g * r + c] = acc;
 }
 
+// Finishes a split-K encode: z[g][n][c..c+8) = bf16_rne(sum over splits of
+// the fp32 partials - muw[g][c..c+8)), one thread per 8 outputs.
+__global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const float* muw,
+                                                       int ksplit, int G, int N, int r,
+                                                       __nv_bfloat16* z, long long zrs,
+                                                       long long zgs) {
+  const int r8 = r / 8;
+  const long long total = (long long)G * N * r8;
+  const size_t plane = (size_t)G * N * r;
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += (long long)gridDim.x * 256) {
+    const int c = (int)(i % r8) * 8;
+    const long long gn = i / r8;
+    const int n = (int)(gn % N), g = (int)(gn / N);
+    const float4* p = reinterpret_cast<const float4*>(part + (size_t)gn * r + c);
+    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+    for (int k = 0; k < ksplit; ++k) {
+      const float4 a0 = __ldg(p + k * (plane / 4)), a1 = __ldg(p + k * (plane / 4) + 1);
+      s0.x += a0.x; s0.y += a0.y; s0.z += a0.z; s0.w += a0.w;
+      s1.x += a1.x; s1.y += a1.y; s1.z += a1.z; s1.w += a1.w;
+    }
+    if (muw) {
+      const float4 m0 = __ldg(reinterpret_cast<const float4*>(muw + (size_t)g * r + c));
+      const float4 m1 = __ldg(reinterpret_cast<const float4*>(muw + (size_t)g * r + c) + 1);
+      s0.x -= m0.x; s0.y -= m0.y; s0.z -= m0.z; s0.w -= m0.w;
+      s1.x -= m1.x; s1.y -= m1.y; s1.z -= m1.z; s1.w -= m1.w;
+    }
+    const __nv_bfloat162 b0 = __floats2bfloat162_rn(s0.x, s0.y), b1 = __floats2bfloat162_rn(s0.z, s0.w);
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(s1.x, s1.y), b3 = __floats2bfloat162_rn(s1.z, s1.w);
+    *reinterpret_cast<uint4*>(z + (size_t)g * zgs + (size_t)n * zrs + c) =
+        make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
+                   *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
+  }
+}
+
 }  // namespace
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
@@ -361,9 +415,25 @@ lla_status run_encode_bias(const void* wt, const float* mu, int G, int K, int r,
   return check_cuda(cudaGetLastError(), "launch k_encode_bias");
 }
 
+int encode_ksplit(int T, int N, int G, int d_loop) {
+  const int tiles = (N + kTileM - 1) / kTileM * G;
+  const int nk = T * d_loop / kChunkK;
+  const int sms = device_info().sms;
+  if (2 * tiles > sms) return 1;
+  const int S = std::min(nk / 2, sms / tiles);
+  if (S < 2) return 1;
+  const int cpk = (nk + S - 1) / S;
+  return (nk + cpk - 1) / cpk;
+}
+
+size_t encode_workspace(int T, int N, int G, int d_loop, int r) {
+  const int S = encode_ksplit(T, N, G, d_loop);
+  return S > 1 ? (size_t)S * G * N * r * sizeof(float) : 0;
+}
+
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs,
-                      cudaStream_t stream, const float* muw) {
+                      cudaStream_t stream, const float* muw, void* ws, size_t ws_bytes) {
   const int K = T * d_loop;
   const int r_pad = (r + 15) / 16 * 16;
   EncodeArgs a{};
@@ -376,6 +446,20 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   a.nk = K / kChunkK;
   a.mtiles = (N + kTileM - 1) / kTileM;
   a.tiles = a.mtiles * G;
+  // Few tiles and a long K (a wide LLA-2D stack at decode time) leave most
+  // SMs idle: with a workspace, K is split so every SM gets work, and a
+  // second kernel sums the fp32 partials.
+  a.ksplit = 1;
+  a.cpk = a.nk;
+  a.part = nullptr;
+  if (ws && !mu) {
+    const int S = encode_ksplit(T, N, G, d_loop);
+    if (S > 1 && ws_bytes >= (size_t)S * G * N * r * sizeof(float)) {
+      a.ksplit = S;
+      a.cpk = (a.nk + S - 1) / S;
+      a.part = static_cast<float*>(ws);
+    }
+  }
   a.b_bytes = r_pad * kChunkK * 2;
   a.stage_bytes = kABytes + a.b_bytes;
   uint32_t cols = 32;
@@ -395,9 +479,10 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   if (nst < 2) return fail(LLA_ERR_UNSUPPORTED, "encode stage does not fit in shared memory");
   a.nstage = nst;
   const size_t smem = (size_t)nst * a.stage_bytes + fixed;
-  const int grid0 = std::min(a.tiles, di.sms);
-  a.tiles_per_cta = (a.tiles + grid0 - 1) / grid0;
-  const int grid = (a.tiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+  const int items = a.tiles * a.ksplit;
+  const int grid0 = std::min(items, di.sms);
+  a.tiles_per_cta = (items + grid0 - 1) / grid0;
+  const int grid = (items + a.tiles_per_cta - 1) / a.tiles_per_cta;
 
   CUtensorMap tx, tw;
   {
@@ -421,6 +506,13 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   k_encode<<<grid, kThreads, smem, stream>>>(tx, tw, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return check_cuda(e, "launch k_encode");
+  if (a.part) {
+    const long long outs = (long long)G * N * (r / 8);
+    const int rgrid = (int)std::min<long long>((outs + 255) / 256, 4LL * di.sms);
+    k_encode_reduce<<<rgrid, 256, 0, stream>>>(a.part, muw, a.ksplit, G, N, r, a.z, zrs, zgs);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return check_cuda(e, "launch k_encode_reduce");
+  }
   e = record_timing(false, stream);
   if (e != cudaSuccess) return check_cuda(e, "record timing event");
   return LLA_OK;

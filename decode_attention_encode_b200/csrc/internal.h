@@ -116,7 +116,11 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
 
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream,
-                      const float* muw = nullptr);
+                      const float* muw = nullptr, void* ws = nullptr, size_t ws_bytes = 0);
+
+// Bytes of the split-K workspace run_encode uses for this shape (0: the
+// shape has enough tiles and runs unsplit).
+size_t encode_workspace(int T, int N, int G, int d_loop, int r);
 
 // muw[g][c] = sum_k mu[g][k] W_down[g][k][c] over K = T * d_loop (fp32).
 lla_status run_encode_bias(const void* wt, const float* mu, int G, int K, int r, float* muw,

@@ -333,14 +333,24 @@ LLA_API lla_status lla_encode_bias(const void *w_down_t, const float *mu, int G,
                                    int K, int r, float *muw, void *stream);
 
 /* lla_encode with the mean term given as muw = mu W_down (from
- * lla_encode_bias), or NULL for a zero mean:
+ * lla_encode_bias, 16-byte aligned), or NULL for a zero mean:
  *   z[g][n][c] = bf16_rne( sum_k xs[k] * W_down[g][k][c] - muw[g][c] ).
- * Arguments and limits otherwise as lla_encode. */
+ * Arguments and limits otherwise as lla_encode, plus an optional workspace:
+ * when the shape has too few 128-token tiles to occupy the GPU (a wide
+ * LLA-2D stack written for one decode step's tokens), a workspace of
+ * lla_encode_with_bias_workspace(...) bytes (16-byte aligned, no
+ * initialisation) lets the call split the contraction over K and add the
+ * fp32 partials in a second kernel. With workspace NULL, or a query result
+ * of 0, the call runs unsplit. The result is the same up to fp32 summation
+ * order. */
+LLA_API size_t lla_encode_with_bias_workspace(int T, int N, int G, int d_loop, int r);
+
 LLA_API lla_status lla_encode_with_bias(const void *x, lla_dtype xdt, int T, int N,
                                         int G, int d_loop, int r,
                                         const void *w_down_t, const float *muw,
                                         void *z, long long z_row_stride,
-                                        long long z_group_stride, void *stream);
+                                        long long z_group_stride, void *workspace,
+                                        size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

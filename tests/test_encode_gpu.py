@@ -137,3 +137,24 @@ def test_encode_huginn_scale_loop_count():
     z = lla.lla_encode(x, w_t, m)
     torch.cuda.synchronize()
     check(z, oracle.encode(to_f64(x), to_f64(w), to_f64(m)))
+
+
+@pytest.mark.parametrize("T, N, G, d_loop, r", [(4, 256, 1, 2048, 256), (4, 64, 2, 128, 128),
+                                                (32, 1, 1, 128, 16), (4, 300, 1, 2048, 64)])
+def test_encode_split_over_k_matches_unsplit(T, N, G, d_loop, r):
+    # the decode-time LLA-2D write: few tokens, a wide stack
+    assert lla._lib.lib().lla_encode_with_bias_workspace(T, N, G, d_loop, r) > 0
+    x, w, w_t, m = make(T, N, G, d_loop, r, True, seed=N + r)
+    muw = lla.lla_encode_bias(w_t, m)
+    z_split = lla.lla_encode_with_bias(x, w_t, muw)
+    z_one = lla.lla_encode_with_bias(x, w_t, muw, split=False)
+    torch.cuda.synchronize()
+    ref = oracle.encode(to_f64(x), to_f64(w), to_f64(m))
+    check(z_split, ref)
+    check(z_one, ref)
+    # the same sums in another order: a bf16 rounding step apart at most,
+    # with the oracle check's absolute floor for values near zero
+    d = (z_split.float() - z_one.float()).abs()
+    floor = 1e-4 * z_one.float().abs().max()
+    assert (d <= 2.0 ** -7 * z_one.float().abs() + floor).all()
+    assert lla.device_status() == 0
