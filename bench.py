@@ -200,8 +200,8 @@ class DecodeWorkload:
         s = c.seed + seed_offset
         self.paged = c.page_size > 0
         self.rope = c.d_r > 0
-        self.write_latents = (not c.two_d and not self.paged and not self.rope
-                              and c.dtype == "bf16" and c.d_h % 64 == 0)
+        self.write_latents = (not self.paged and not self.rope and c.dtype == "bf16"
+                              and c.d_h % 64 == 0)
         n_cap = c.N + 1 if self.write_latents else c.N
         zk_shape = (c.B, n_cap, c.r_k) if c.two_d else (c.B, c.H, n_cap, c.r_k + c.d_r)
         zv_shape = (c.B, n_cap, c.r_v) if c.two_d else (c.B, c.H, n_cap, c.r_v)
@@ -238,18 +238,29 @@ class DecodeWorkload:
         self.fn = lla.lla2d_decode_attn if c.two_d else lla.lla_decode_attn
         self.scale = 1.0 / math.sqrt(c.d_h)
         if self.write_latents:
-            K = c.T * c.d_h
-            # encoders W_down^T [H][r][T*d_h] per (layer, axis), means, and the
-            # newest token's stacked per-loop K and V [T][B][H][d_h]
-            self.wk = synth.orthonormal(c.L * c.H, K, c.r_k, s + 6, device).transpose(1, 2) \
-                .contiguous().to(torch.bfloat16).view(c.L, c.H, c.r_k, K)
-            self.wv = synth.orthonormal(c.L * c.H, K, c.r_v, s + 7, device).transpose(1, 2) \
-                .contiguous().to(torch.bfloat16).view(c.L, c.H, c.r_v, K)
-            self.muk = synth.normal((c.L, c.H, K), s + 8, device, std=0.1)
-            self.muv = synth.normal((c.L, c.H, K), s + 9, device, std=0.1)
+            # Encoders W_down^T [G][r][K] per (layer, axis), means, and the
+            # newest token's stacked per-loop K and V [T][B][H][d_h]. Per-head
+            # LLA encodes each head (G = H, K = T d_h); LLA-2D encodes the
+            # whole stack of a token (G = 1, K = T H d_h). The mean term
+            # mu W_down is a codec constant, formed once here.
+            G, K = (1, c.T * c.H * c.d_h) if c.two_d else (c.H, c.T * c.d_h)
+            self.enc_g, self.enc_k = G, K
+            self.wk = synth.orthonormal(c.L * G, K, c.r_k, s + 6, device).transpose(1, 2) \
+                .contiguous().to(torch.bfloat16).view(c.L, G, c.r_k, K)
+            self.wv = synth.orthonormal(c.L * G, K, c.r_v, s + 7, device).transpose(1, 2) \
+                .contiguous().to(torch.bfloat16).view(c.L, G, c.r_v, K)
+            self.muk = synth.normal((c.L, G, K), s + 8, device, std=0.1)
+            self.muv = synth.normal((c.L, G, K), s + 9, device, std=0.1)
+            self.muwk = torch.stack([lla.lla_encode_bias(self.wk[l], self.muk[l]) for l in range(c.L)])
+            self.muwv = torch.stack([lla.lla_encode_bias(self.wv[l], self.muv[l]) for l in range(c.L)])
             self.xk = synth.normal((c.L, c.T, c.B, c.H, c.d_h), s + 10, device, dtype=torch.bfloat16)
             self.xv = synth.normal((c.L, c.T, c.B, c.H, c.d_h), s + 11, device, dtype=torch.bfloat16)
             self.n_cap = n_cap
+            d_loop = K // c.T
+            need = max(lla.lla_encode_with_bias_workspace_bytes(c.T, c.B, G, d_loop, r)
+                       for r in (c.r_k, c.r_v))
+            self.enc_split = need > 0
+            self.enc_ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
 
     def step(self, q=None, out=None, lse=None, xk=None, xv=None):
         """One looped decode step: loops outer, layers inner (each loop's
@@ -286,18 +297,24 @@ class DecodeWorkload:
                     scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
 
     def write_newest(self, xk, xv):
+        """Each sequence's newest token into slot N of every layer's store."""
         c = self.cfg
         for l in range(c.L):
-            for x, w, mu, z, r in ((xk, self.wk, self.muk, self.zk, c.r_k),
-                                   (xv, self.wv, self.muv, self.zv, c.r_v)):
-                self.lla.lla_encode(x[l], w[l], mu[l], z=z[l][:, :, c.N],
-                                    z_row_stride=c.H * self.n_cap * r,
-                                    z_group_stride=self.n_cap * r)
+            for x, w, muw, z, r in ((xk, self.wk, self.muwk, self.zk, c.r_k),
+                                    (xv, self.wv, self.muwv, self.zv, c.r_v)):
+                if c.two_d:  # x [T][B][H][d_h] read as [T][B][1][H d_h]
+                    self.lla.lla_encode_with_bias(
+                        x[l].view(c.T, c.B, 1, c.H * c.d_h), w[l], muw[l], z=z[l][:, c.N],
+                        z_row_stride=self.n_cap * r, z_group_stride=0, workspace=self.enc_ws)
+                else:
+                    self.lla.lla_encode_with_bias(
+                        x[l], w[l], muw[l], z=z[l][:, :, c.N], z_row_stride=c.H * self.n_cap * r,
+                        z_group_stride=self.n_cap * r, workspace=self.enc_ws)
 
     def launches_per_step(self) -> int:
         n = (4 if self.paged else 3) * self.cfg.L * self.cfg.T
         if self.write_latents:
-            n += 2 * self.cfg.L
+            n += (4 if self.enc_split else 2) * self.cfg.L
         return n
 
 
@@ -326,14 +343,17 @@ class EncodeWorkload:
             w_t.append(vh[:, :c.r, :].contiguous().to(torch.bfloat16))   # [G][r][K]
             mu.append(m[:, 0, :].contiguous())                             # [G][K]
         self.w_t, self.mu = w_t, mu
+        # the mean term mu W_down is a codec constant: formed once
+        self.muw = [lla.lla_encode_bias(w_t[i], mu[i]) for i in range(2 * c.L)]
         self.z = [torch.empty((c.G, c.N, c.r), device=device, dtype=torch.bfloat16)
                   for _ in range(2 * c.L)]
 
     def step(self, x=None):
         x = self.x if x is None else x
         for i in range(2 * self.cfg.L):
-            self.lla.lla_encode(x[i], self.w_t[i], self.mu[i], z=self.z[i],
-                                z_row_stride=self.cfg.r, z_group_stride=self.cfg.N * self.cfg.r)
+            self.lla.lla_encode_with_bias(x[i], self.w_t[i], self.muw[i], z=self.z[i],
+                                          z_row_stride=self.cfg.r,
+                                          z_group_stride=self.cfg.N * self.cfg.r, split=False)
 
     def launches_per_step(self) -> int:
         return 2 * self.cfg.L
@@ -364,8 +384,9 @@ def run_encode_bench(args, world, rank, local):
     kern = []
     for i in range(2 * cfg.L):
         with wl.lla.kernel_timer() as kt:
-            wl.lla.lla_encode(wl.x[i], wl.w_t[i], wl.mu[i], z=wl.z[i], z_row_stride=cfg.r,
-                              z_group_stride=cfg.N * cfg.r)
+            wl.lla.lla_encode_with_bias(wl.x[i], wl.w_t[i], wl.muw[i], z=wl.z[i],
+                                        z_row_stride=cfg.r, z_group_stride=cfg.N * cfg.r,
+                                        split=False)
         kern.append(kt.ms)
     kern_ms = sum(kern) / len(kern)
     call_bytes = (cfg.T * cfg.N * cfg.G * cfg.d_loop + cfg.G * cfg.N * cfg.r) * 2

@@ -353,6 +353,11 @@ def lla_encode_bias(w_down_t, mu, muw=None, stream=None):
     return muw
 
 
+def lla_encode_with_bias_workspace_bytes(T, N, G, d_loop, r):
+    """Workspace bytes lla_encode_with_bias can use to split over K (0: none)."""
+    return int(lib().lla_encode_with_bias_workspace(T, N, G, d_loop, r))
+
+
 def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_group_stride=None,
                          workspace=None, stream=None, split=True):
     """lla_encode with the mean term precomputed by lla_encode_bias (muw
