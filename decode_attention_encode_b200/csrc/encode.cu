@@ -346,37 +346,45 @@ __global__ void __launch_bounds__(256) k_encode_bias(const __nv_bfloat16* wt, co
   if (lane == 0) muw[(size_t)g * r + c] = acc;
 }
 
-// Finishes a split-K encode: z[g][n][c..c+8) = bf16_rne(sum over splits of
-// the fp32 partials - muw[g][c..c+8)), one thread per 8 outputs.
+// Finishes a split-K encode: z[g][n][c..c+4) = bf16_rne(sum over splits of
+// the fp32 partials - muw[g][c..c+4)), one thread per 4 outputs with eight
+// partial loads in flight.
 __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const float* muw,
                                                        int ksplit, int G, int N, int r,
                                                        __nv_bfloat16* z, long long zrs,
                                                        long long zgs) {
-  const int r8 = r / 8;
-  const long long total = (long long)G * N * r8;
-  const size_t plane = (size_t)G * N * r;
+  const int r4 = r / 4;
+  const long long total = (long long)G * N * r4;
+  const size_t plane4 = (size_t)G * N * r / 4;  // float4 per split
   for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += (long long)gridDim.x * 256) {
-    const int c = (int)(i % r8) * 8;
-    const long long gn = i / r8;
+    const int c = (int)(i % r4) * 4;
+    const long long gn = i / r4;
     const int n = (int)(gn % N), g = (int)(gn / N);
-    const float4* p = reinterpret_cast<const float4*>(part + (size_t)gn * r + c);
-    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
-    for (int k = 0; k < ksplit; ++k) {
-      const float4 a0 = __ldg(p + k * (plane / 4)), a1 = __ldg(p + k * (plane / 4) + 1);
-      s0.x += a0.x; s0.y += a0.y; s0.z += a0.z; s0.w += a0.w;
-      s1.x += a1.x; s1.y += a1.y; s1.z += a1.z; s1.w += a1.w;
+    const float4* p = reinterpret_cast<const float4*>(part) + (size_t)i;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < ksplit; k0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        v[k] = k0 + k < ksplit ? __ldg(p + (size_t)(k0 + k) * plane4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        s.x += v[k].x;
+        s.y += v[k].y;
+        s.z += v[k].z;
+        s.w += v[k].w;
+      }
     }
     if (muw) {
-      const float4 m0 = __ldg(reinterpret_cast<const float4*>(muw + (size_t)g * r + c));
-      const float4 m1 = __ldg(reinterpret_cast<const float4*>(muw + (size_t)g * r + c) + 1);
-      s0.x -= m0.x; s0.y -= m0.y; s0.z -= m0.z; s0.w -= m0.w;
-      s1.x -= m1.x; s1.y -= m1.y; s1.z -= m1.z; s1.w -= m1.w;
+      const float4 m = __ldg(reinterpret_cast<const float4*>(muw + (size_t)g * r + c));
+      s.x -= m.x;
+      s.y -= m.y;
+      s.z -= m.z;
+      s.w -= m.w;
     }
-    const __nv_bfloat162 b0 = __floats2bfloat162_rn(s0.x, s0.y), b1 = __floats2bfloat162_rn(s0.z, s0.w);
-    const __nv_bfloat162 b2 = __floats2bfloat162_rn(s1.x, s1.y), b3 = __floats2bfloat162_rn(s1.z, s1.w);
-    *reinterpret_cast<uint4*>(z + (size_t)g * zgs + (size_t)n * zrs + c) =
-        make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
-                   *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
+    const __nv_bfloat162 b0 = __floats2bfloat162_rn(s.x, s.y), b1 = __floats2bfloat162_rn(s.z, s.w);
+    *reinterpret_cast<uint2*>(z + (size_t)g * zgs + (size_t)n * zrs + c) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
   }
 }
 
@@ -420,7 +428,9 @@ int encode_ksplit(int T, int N, int G, int d_loop) {
   const int nk = T * d_loop / kChunkK;
   const int sms = device_info().sms;
   if (2 * tiles > sms) return 1;
-  const int S = std::min(nk / 2, sms / tiles);
+  // at most 16 splits: beyond that the partial traffic and the final sum
+  // cost more than the idle SMs they would fill
+  const int S = std::min(std::min(nk / 2, sms / tiles), 16);
   if (S < 2) return 1;
   const int cpk = (nk + S - 1) / S;
   return (nk + cpk - 1) / cpk;
@@ -507,7 +517,7 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   e = cudaGetLastError();
   if (e != cudaSuccess) return check_cuda(e, "launch k_encode");
   if (a.part) {
-    const long long outs = (long long)G * N * (r / 8);
+    const long long outs = (long long)G * N * (r / 4);
     const int rgrid = (int)std::min<long long>((outs + 255) / 256, 4LL * di.sms);
     k_encode_reduce<<<rgrid, 256, 0, stream>>>(a.part, muw, a.ksplit, G, N, r, a.z, zrs, zgs);
     e = cudaGetLastError();

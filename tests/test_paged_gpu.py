@@ -127,9 +127,9 @@ def test_dense_equivalent_layout_matches_the_dense_kernel():
 
 
 def test_full_size_ragged_batch_sampled():
-    # a serving batch at the 4x geometry: 64 sequences of 2k..6k tokens,
-    # 64-token pages; checked on sampled sequences
-    lens = synth.ragged_lengths(64, 4096, seed=0)
+    # the perhead_4x_paged workload: a serving batch at the 4x geometry, 64
+    # sequences of 2k..6k tokens, 64-token pages; checked on sampled sequences
+    lens = synth.C2_PAGED.lengths()
     inp = make_paged_inputs(lens, 16, 128, 128, 128, BF16, 64, seed=0)
     out, lse = lla.lla_decode_attn_paged(inp["q"], inp["zk"], inp["zv"], inp["block_table"],
                                          inp["seq_lens"], inp["dk"], inp["dv"])
