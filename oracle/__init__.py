@@ -25,6 +25,7 @@ What is here, each in fp64:
   * ``rope_rotate`` / ``decode_unit_rope`` / ``lla_decode_rope``: the
     decoupled-RoPE split of §7 (NoPE latent content path plus an explicit
     rotary branch), as attention over concatenated content and rotary keys.
+  * ``paged2d_decode``: the same gather for the LLA-2D store.
   * ``kept_positions`` / ``paged_decode``: the per-head decode over a paged
     store with per-sequence lengths (a gather of each unit's rows, then the
     explicit-reconstruction unit), with the attention-sink + window eviction
@@ -350,6 +351,36 @@ def paged_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=None
         zv_u = np.transpose(zv_pages[pages, :, rows], (1, 0, 2))
         o, l = decode_units(q[b], zk_u, zv_u, dk, dv, mu_k, mu_v, scale, nthreads)
         out[b], lse[b] = o, l
+    return out, lse
+
+
+def paged2d_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=None, mu_v=None,
+                   scale=None, nthreads: int = 0):
+    """LLA-2D decode over a paged store with per-sequence lengths.
+
+    zk_pages [P, page_size, r_k], zv_pages [P, page_size, r_v]: one latent
+    per token shared by every head (§3 "The LLA-2D variant"); token j of
+    sequence b is row j % page_size of page block_table[b, j // page_size].
+    Each sequence gathers its rows and goes through the LLA-2D explicit
+    reconstruction; an empty sequence gives out = 0, lse = -inf (the same
+    reading as ``paged_decode``). Returns out [B, H, d], lse [B, H]."""
+    q = np.asarray(q)
+    B, H, d = q.shape
+    zk_pages, zv_pages = np.asarray(zk_pages), np.asarray(zv_pages)
+    block_table, seq_lens = np.asarray(block_table), np.asarray(seq_lens)
+    ps = zk_pages.shape[1]
+    out = np.zeros((B, H, d))
+    lse = np.full((B, H), -np.inf)
+    for b in range(B):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        pos = np.arange(n)
+        pages = block_table[b, pos // ps]
+        zk = zk_pages[pages, pos % ps][None]
+        zv = zv_pages[pages, pos % ps][None]
+        o, l = lla2d_decode(q[b:b + 1], zk, zv, dk, dv, mu_k, mu_v, scale, nthreads=nthreads)
+        out[b], lse[b] = o[0], l[0]
     return out, lse
 
 

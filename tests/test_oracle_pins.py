@@ -571,3 +571,41 @@ def test_rope_unit_matches_absorbed_query_with_appended_rotary_part():
     ubar = (p / p.sum()) @ zv
     np.testing.assert_allclose(o, dv @ ubar + mv, atol=1e-12)
     assert abs(l - (s.max() + np.log(p.sum()))) < 1e-12
+
+
+def test_paged2d_equals_dense_2d_decode_per_sequence_length():
+    r = rng(61)
+    lens = [1, 5, 8, 0, 13, 16]
+    B, H, d, ps, rk, rv = len(lens), 3, 8, 4, 16, 24
+    maxb = 4
+    npages = B * maxb + 2
+    order = r.permutation(npages)
+    bt = np.full((B, maxb), -1)
+    zkp = r.standard_normal((npages, ps, rk))
+    zvp = r.standard_normal((npages, ps, rv))
+    dense_k = r.standard_normal((B, maxb * ps, rk))
+    dense_v = r.standard_normal((B, maxb * ps, rv))
+    k = 0
+    for b, n in enumerate(lens):
+        for blk in range((n + ps - 1) // ps):
+            pg = order[k]; k += 1
+            bt[b, blk] = pg
+            zkp[pg] = dense_k[b, blk * ps:(blk + 1) * ps]
+            zvp[pg] = dense_v[b, blk * ps:(blk + 1) * ps]
+    q = r.standard_normal((B, H, d))
+    dk, dv = r.standard_normal((H, d, rk)), r.standard_normal((H, d, rv))
+    mk, mv = r.standard_normal((H, d)), r.standard_normal((H, d))
+    out, lse = oracle.paged2d_decode(q, zkp, zvp, bt, lens, dk, dv, mk, mv)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        ob, lb = oracle.lla2d_decode(q[b:b + 1], dense_k[b:b + 1], dense_v[b:b + 1], dk, dv, mk,
+                                     mv, N=n)
+        np.testing.assert_allclose(out[b], ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], lb[0], rtol=0, atol=1e-12)
+    # one token: every head's output is that token's reconstruction
+    o1, _ = oracle.paged2d_decode(q[:1], zkp, zvp, bt[:1], [1], dk, dv, mk, mv)
+    pg = bt[0, 0]
+    for h in range(H):
+        np.testing.assert_allclose(o1[0, h], dv[h] @ zvp[pg, 0] + mv[h], atol=1e-12)
