@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     lib,
     library_path,
     lla2d_decode_attn,
+    lla2d_decode_attn_paged,
     lla2d_decode_attn_workspace,
     lla_decode_attn,
     lla_decode_attn_noalloc,

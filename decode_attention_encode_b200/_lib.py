@@ -37,6 +37,7 @@ EXPORTS = (
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn",
+    "lla2d_decode_attn_paged_workspace", "lla2d_decode_attn_paged",
     "lla_encode", "lla_encode_bias", "lla_encode_with_bias_workspace", "lla_encode_with_bias",
 )
 
@@ -67,6 +68,9 @@ _SIGS = {
                               [_c_int] * 2 + [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp],
                               _c_int),
     "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
+    "lla2d_decode_attn_paged_workspace": ([_c_int] * 4, _c_size),
+    "lla2d_decode_attn_paged": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp, _c_int, _vp] +
+                                [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
                         [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla_decode_attn_noalloc": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
@@ -310,6 +314,40 @@ def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv
                                  _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t), float(scale), _ptr(out),
                                  _ptr(lse), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t,
+                            mu_k_t=None, mu_v_t=None, scale=None, out=None, lse=None,
+                            workspace=None, stream=None, want_lse=True):
+    """LLA-2D absorbed decode over a paged store: zk_pages [P,page_size,r_k],
+    zv_pages [P,page_size,r_v] bf16 shared by every head, page_size a
+    multiple of 128; block_table [B,max_blocks] and seq_lens [B] int32 on
+    the device. Returns (out [B,H,d_h], lse [B,H] or None)."""
+    _need_cuda(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, out,
+               lse, workspace)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise LLAError(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be int32")
+    B, H, d_h = q.shape
+    num_pages, page_size, r_k = zk_pages.shape
+    r_v = zv_pages.shape[2]
+    max_blocks = block_table.shape[1]
+    scale = 1.0 / math.sqrt(d_h) if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, d_h), device=q.device, dtype=torch.float32)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    h = lib()
+    need = int(h.lla2d_decode_attn_paged_workspace(B, H, r_k, r_v))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    st = h.lla2d_decode_attn_paged(_ptr(q), _ptr(zk_pages), _ptr(zv_pages),
+                                   _dtype_code(zk_pages), B, H, d_h, r_k, r_v, page_size,
+                                   num_pages, _ptr(block_table), max_blocks, _ptr(seq_lens),
+                                   _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t),
+                                   float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st)
     return out, lse
 

@@ -310,6 +310,44 @@ lla_status lla2d_decode_attn(const float* q, const void* zk, const void* zv, lla
                        static_cast<cudaStream_t>(stream));
 }
 
+size_t lla2d_decode_attn_paged_workspace(int B, int H, int r_k, int r_v) {
+  if (B < 1 || H < 1 || H > 32 || r_k < 64 || r_k > 256 || r_k % 64 || r_v < 128 || r_v > 256 ||
+      r_v % 128)
+    return 0;
+  return workspace_2d_paged(B, H, r_k, r_v);
+}
+
+lla_status lla2d_decode_attn_paged(const float* q, const void* zk_pages, const void* zv_pages,
+                                   lla_dtype zdt, int B, int H, int d_h, int r_k, int r_v,
+                                   int page_size, int num_pages, const int* block_table,
+                                   int max_blocks, const int* seq_lens, const float* dk_t,
+                                   const float* dv_t, const float* mu_k_t, const float* mu_v_t,
+                                   float scale, float* out, float* lse, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  int esz = 0;
+  lla_status st = check_decode_args(q, zk_pages, zv_pages, zdt, B, H, d_h, 1, 1, r_k, r_v, dk_t,
+                                    dv_t, mu_k_t, mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
+  if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
+  if (r_k % 64 || r_v % 128)
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D needs r_k a multiple of 64 and r_v a multiple of 128");
+  if (!block_table || !seq_lens)
+    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be non-NULL");
+  if (!aligned(block_table, 4) || !aligned(seq_lens, 4))
+    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be 4-byte aligned");
+  if (page_size < 128 || page_size % 128)
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D pages hold a positive multiple of 128 tokens");
+  if (num_pages < 1 || max_blocks < 1)
+    return fail(LLA_ERR_INVALID_ARG, "num_pages and max_blocks must be >= 1");
+  if ((long long)page_size * max_blocks > 0x7fffffffLL)
+    return fail(LLA_ERR_INVALID_ARG, "page_size * max_blocks must fit in 31 bits");
+  return run_decode_2d_paged(q, zk_pages, zv_pages, B, H, d_h, r_k, r_v, page_size, num_pages,
+                             block_table, max_blocks, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, scale,
+                             out, lse, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
 lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,
                       const void* w_down_t, const float* mu, void* z, long long z_row_stride,
                       long long z_group_stride, void* stream) {

@@ -258,7 +258,8 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
         const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
         if (n > 0) {
           const long long P = a.ragged.plan[1];
-          const long long first = a.ragged.cum[b0 + bb] + (long long)h * n;
+          // per head for per-head LLA; LLA-2D splits a sequence once for all heads
+          const long long first = a.ragged.cum[b0 + bb] + (a.shared ? 0LL : (long long)h * n);
           wf = first / P;
           wl = (first + n - 1) / P;
         }

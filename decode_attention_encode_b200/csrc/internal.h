@@ -85,6 +85,23 @@ struct RaggedMap {
 };
 
 size_t workspace_paged(int B, int H, int r_k, int r_v, int esz);
+
+// k_plan_paged: per-sequence records, prefix sums of the flattened range,
+// {total, share} and each worker's start (paged.cu). tile_tokens > 0 plans
+// LLA-2D: units are tiles of that many tokens, records {tiles, tokens}, and
+// the workers are CTAs.
+lla_status launch_plan_paged(const int* seq_lens, const int* block_table, int B, int H,
+                             int page_size, int num_pages, int max_blocks, int sink, int window,
+                             int W, int pmin, int tile_tokens, int4* seqinfo, long long* cum,
+                             long long* plan, int4* wstart, cudaStream_t stream);
+
+size_t workspace_2d_paged(int B, int H, int r_k, int r_v);
+lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, int B, int H,
+                               int d_h, int r_k, int r_v, int page_size, int num_pages,
+                               const int* block_table, int max_blocks, const int* seq_lens,
+                               const float* dk, const float* dv, const float* mu_k,
+                               const float* mu_v, float scale, float* out, float* lse, void* ws,
+                               size_t ws_bytes, cudaStream_t stream);
 lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int esz, int B, int H,
                             int d_h, int r_k, int r_v, int page_size, int num_pages,
                             const int* block_table, int max_blocks, const int* seq_lens, int sink,

@@ -65,6 +65,12 @@ struct D2Args {
   int off_q, off_p, off_tail, qbuf_bytes, pbuf_bytes;
   uint32_t tmem_cols;
   const unsigned char* qsw;  // per sequence: Q' as bf16 in the MMA operand layout
+  // paged store (seqinfo non-null): written by k_plan_paged
+  const int4* seqinfo;      // [B] {tiles, tokens, 0, 0}
+  const long long* plan;    // {total tiles, tiles per CTA}
+  const int4* cstart;       // [grid] first (sequence, 0, tile) of each CTA
+  const int* block_table;   // [B][max_blocks]
+  int max_blocks, page_size;
   float* part;
   int pstride;
   unsigned int* status;
@@ -112,6 +118,50 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// The (sequence b, tile j) a role is at, with sequence b's tile count nt and
+// token count n. Every role walks its CTA's tiles in order with its own
+// cursor: uniformly sized sequences (tps tiles of N tokens each) or the
+// ragged sequences of a paged plan.
+struct TileCur {
+  int b, j, nt, n;
+};
+
+__device__ __forceinline__ void tcur_load(TileCur& c, const D2Args& a) {
+  if (a.seqinfo) {
+    const int4 v = __ldg(a.seqinfo + c.b);
+    c.nt = v.x;
+    c.n = v.y;
+  } else {
+    c.nt = a.tps;
+    c.n = a.N;
+  }
+}
+
+__device__ __forceinline__ TileCur tcur_start(const D2Args& a) {
+  TileCur c;
+  if (a.seqinfo) {
+    const int4 s = __ldg(a.cstart + blockIdx.x);
+    c.b = s.x;
+    c.j = s.z;
+  } else {
+    const int t = blockIdx.x * a.tpc;
+    c.b = t / a.tps;
+    c.j = t - c.b * a.tps;
+  }
+  tcur_load(c, a);
+  return c;
+}
+
+__device__ __forceinline__ void tcur_next(TileCur& c, const D2Args& a) {
+  if (++c.j == c.nt) {
+    c.j = 0;
+    do {
+      ++c.b;
+    } while (a.seqinfo && c.b < a.B && __ldg(&a.seqinfo[c.b].x) == 0);
+    if (c.b < a.B) tcur_load(c, a);
+  }
+}
+
 template <int HP>
 __global__ void __launch_bounds__(kThreads, 1)
     k_lla2d(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -127,9 +177,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t s_p0 = smem_u32(smem + a.off_p);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t_begin = blockIdx.x * a.tpc;
-  const int t_end = min(t_begin + a.tpc, a.tiles);
-  const int ntile = t_end - t_begin;
+  // a paged plan sizes the split on the device (k_plan_paged finished before
+  // k_absorb started, so this is safe before griddepcontrol.wait)
+  const long long tiles = a.seqinfo ? a.plan[0] : (long long)a.tiles;
+  const long long tpc = a.seqinfo ? a.plan[1] : (long long)a.tpc;
+  const long long t_begin = blockIdx.x * tpc;
+  const int ntile = (int)max(0LL, min(t_begin + tpc, tiles) - t_begin);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.nks; ++s) {
@@ -160,7 +213,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = tl->tmem_base;
 
-  auto seq_of = [&](int lt) { return (t_begin + lt) / a.tps; };
   auto kboxes = [&](int kg) { return min(2, (a.r_k - kg * 128) / 64); };
 
   if (warp == 0 || warp == 6) {
@@ -175,22 +227,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* emptyb = is_k ? tl->kempty : tl->vempty;
     const CUtensorMap* map = is_k ? &tk : &tv;
     const int total = ntile * ng;
+    // Cursor at the tile of the next group to load, and that tile's TMA
+    // row and third coordinate: (row, sequence) in the dense store, (row in
+    // page, page) in a paged pool, whose block-table entry for the next
+    // tile is loaded one tile ahead.
+    TileCur pc = tcur_start(a);
+    int pc_lt = 0, c_row = 0, c_z = 0, n_z = 0;
+    auto place = [&]() {
+      if (a.seqinfo) {
+        const int pos = pc.j * kRows;
+        c_row = pos % a.page_size;
+        c_z = n_z;
+        TileCur nx = pc;
+        tcur_next(nx, a);
+        if (pc_lt + 1 < ntile)
+          n_z = __ldg(a.block_table + (size_t)nx.b * a.max_blocks + nx.j * kRows / a.page_size);
+      } else {
+        c_row = pc.j * kRows;
+        c_z = pc.b;
+      }
+    };
+    if (a.seqinfo && ntile > 0)
+      n_z = __ldg(a.block_table + (size_t)pc.b * a.max_blocks + pc.j * kRows / a.page_size);
+    if (ntile > 0) place();
+    auto tile_of = [&](int lt) {
+      while (pc_lt < lt) {
+        tcur_next(pc, a);
+        ++pc_lt;
+        place();
+      }
+    };
     auto issue = [&](int it) -> bool {
       const int s = it % nring;
       const uint32_t ph = (uint32_t)(it / nring) & 1u;
       const bool ok = __all_sync(0xffffffffu,
                                  wait_ab(smem_u32(&emptyb[s]), ph ^ 1u, abort_flag, a.status));
       if (!ok) return false;
+      const int lt = it / ng, grp = it - lt * ng;
+      tile_of(lt);
       if (lane == 0) {
-        const int lt = it / ng, grp = it - lt * ng;
-        const int tile = t_begin + lt;
-        const int b = tile / a.tps, row0 = (tile - b * a.tps) * kRows;
         const uint32_t full = smem_u32(&fullb[s]);
         const uint32_t dst = ring + (uint32_t)s * kStageBytes;
         const int nb = is_k ? kboxes(grp) : 2;
         mbar_arrive_expect_tx(full, nb * kBoxBytes);
         for (int x = 0; x < nb; ++x)
-          tma_load_3d(dst + x * kBoxBytes, map, grp * 128 + x * 64, row0, b, full, pol);
+          tma_load_3d(dst + x * kBoxBytes, map, grp * 128 + x * 64, c_row, c_z, full, pol);
       }
       return true;
     };
@@ -218,16 +299,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!is_k) {
       for (; ok && it < total; ++it) ok = issue(it);
     } else if (ntile > 0) {
-      const int b0 = seq_of(0);
+      const int b0 = pc.b;
       // latent loads of the first sequence do not depend on k_absorb
-      while (ok && it < total && it < nring && seq_of(it / ng) == b0) ok = issue(it++);
+      while (ok && it < total && it < nring) {
+        tile_of(it / ng);
+        if (pc.b != b0) break;
+        ok = issue(it++);
+      }
       pdl_wait();
       if (ok) ok = stage_q(0, b0);
       int seg = 0, cur_b = b0;
       for (; ok && it < total; ++it) {
         const int lt = it / ng;
-        if (it - lt * ng == 0 && seq_of(lt) != cur_b) {
-          cur_b = seq_of(lt);
+        tile_of(lt);
+        if (it - lt * ng == 0 && pc.b != cur_b) {
+          cur_b = pc.b;
           ok = stage_q(++seg, cur_b);
           if (!ok) break;
         }
@@ -296,9 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       int seg = 0;
+      TileCur cur = tcur_start(a);
       ok = wait_ab(smem_u32(&tl->q_full[0]), 0u, abort_flag, a.status);
-      for (int lt = 0; ok && lt < ntile; ++lt) {
-        if (lt > 0 && seq_of(lt) != seq_of(lt - 1)) {
+      for (int lt = 0; ok && lt < ntile; ++lt, tcur_next(cur, a)) {
+        if (lt > 0 && cur.j == 0) {
           umma_commit(smem_u32(&tl->q_empty[seg & 1]));  // after the last score MMA of seg
           ++seg;
           ok = wait_ab(smem_u32(&tl->q_full[seg & 1]), (uint32_t)((seg >> 1) & 1), abort_flag,
@@ -317,8 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && ntile > 0) {
       const uint32_t idesc_u = idesc_bf16_f32(kRows, HP, true, false);
       bool ok = true;
-      for (int lt = 0; ok && lt < ntile; ++lt) {
-        const bool first_of_seg = (lt == 0) || seq_of(lt) != seq_of(lt - 1);
+      TileCur cur = tcur_start(a);
+      for (int lt = 0; ok && lt < ntile; ++lt, tcur_next(cur, a)) {
+        const bool first_of_seg = (lt == 0) || cur.j == 0;
         const int pb = lt & 1;
         ok = wait_ab(smem_u32(&tl->p_full[pb]), (uint32_t)((lt >> 1) & 1), abort_flag, a.status);
         if (!ok) break;
@@ -365,12 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       return ok;
     };
     float m[HP], l[HP];
-    for (int lt = 0; lt < ntile; ++lt) {
-      const int tile = t_begin + lt;
-      const int b = tile / a.tps;
-      const int row0 = (tile - b * a.tps) * kRows;
-      const bool first_of_seg = (lt == 0) || seq_of(lt - 1) != b;
-      const bool last_of_seg = (lt == ntile - 1) || seq_of(lt + 1) != b;
+    TileCur cur = tcur_start(a);
+    for (int lt = 0; lt < ntile; ++lt, tcur_next(cur, a)) {
+      const int b = cur.b;
+      const int row0 = cur.j * kRows;
+      const bool first_of_seg = (lt == 0) || cur.j == 0;
+      const bool last_of_seg = (lt == ntile - 1) || cur.j == cur.nt - 1;
       if (first_of_seg) {
 #pragma unroll
         for (int h = 0; h < HP; ++h) {
@@ -399,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tl->s_empty[sb]));
 
-      const bool valid = row0 + row < a.N;
+      const bool valid = row0 + row < cur.n;
       bool need = false;
 #pragma unroll
       for (int h = 0; h < HP; ++h) need |= valid && h < a.H && s[h] > m[h] + kSlack;
@@ -583,35 +671,28 @@ size_t workspace_2d(int B, int H, int N, int r_k, int r_v) {
   return d.ws_bytes;
 }
 
-lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,
-                         int N, long long n_cap, int r_k, int r_v, const float* dk,
-                         const float* dv, const float* mu_k, const float* mu_v, float scale,
-                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  D2Plan d;
-  lla_status st = plan_2d(B, H, N, r_k, r_v, &d);
-  if (st != LLA_OK) return st;
-  if (ws == nullptr || ws_bytes < d.ws_bytes)
-    return fail(LLA_ERR_WORKSPACE, "LLA-2D workspace needs %zu bytes, got %zu", d.ws_bytes, ws_bytes);
-  char* wsb = static_cast<char*>(ws);
+namespace {
+
+// Paged-store arrays of one LLA-2D call (device), or none.
+struct Paged2D {
+  const int4* seqinfo;
+  long long* cum;
+  long long* plan;
+  const int4* cstart;
+  const int* block_table;
+  int max_blocks, page_size;
+};
+
+// Absorb, the tensor-core kernel and the merge, shared by the dense and the
+// paged entry points.
+lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& tv, int B, int H,
+                     int d_h, int N, int r_k, int r_v, const float* dk, const float* dv,
+                     const float* mu_k, const float* mu_v, float scale, float* out, float* lse,
+                     const D2Plan& d, char* wsb, const Paged2D* pg, cudaStream_t stream) {
   unsigned char* qsw = reinterpret_cast<unsigned char*>(wsb + d.off_qsw);
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
-
-  CUtensorMap tk, tv;
-  {
-    const uint64_t dims[3] = {(uint64_t)r_k, (uint64_t)N, (uint64_t)B};
-    const uint64_t strides[2] = {(uint64_t)r_k * 2, (uint64_t)n_cap * r_k * 2};
-    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
-    if (!make_tmap_bf16(&tk, zk, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)r_v, (uint64_t)N, (uint64_t)B};
-    const uint64_t strides[2] = {(uint64_t)r_v * 2, (uint64_t)n_cap * r_v * 2};
-    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
-    if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
-  }
-
-  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, nullptr, c0, stream, qsw, d.hp);
+  lla_status st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, nullptr, c0, stream, qsw, d.hp);
   if (st != LLA_OK) return st;
 
   D2Args a{};
@@ -637,6 +718,14 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
   a.part = part;
   a.pstride = d.pstride;
   a.status = status_word();
+  if (pg) {
+    a.seqinfo = pg->seqinfo;
+    a.plan = pg->plan;
+    a.cstart = pg->cstart;
+    a.block_table = pg->block_table;
+    a.max_blocks = pg->max_blocks;
+    a.page_size = pg->page_size;
+  }
 
   auto kern = d.hp == 16 ? k_lla2d<16> : k_lla2d<32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem);
@@ -658,8 +747,115 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
   e = record_timing(false, stream);
   if (e != cudaSuccess) return check_cuda(e, "record timing event");
 
+  if (pg) {  // sequence b's pieces: the CTAs of its tiles, cum[b] .. cum[b] + tiles - 1
+    RaggedMap rm{pg->seqinfo, pg->cum, pg->plan};
+    return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 1, out, lse, stream,
+                          &rm);
+  }
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v,
                         (long long)d.tps * kRows, (long long)d.tpc * kRows, 1, out, lse, stream);
+}
+
+// The paged plan: the dense plan's kernel shape with a one-wave grid (the
+// tile count is known only on the device), plus the planner's arrays.
+struct D2PagedPlan {
+  D2Plan d;
+  size_t off_seqinfo, off_cum, off_plan, off_cstart, ws_bytes;
+};
+
+lla_status plan_2d_paged(int B, int H, int r_k, int r_v, D2PagedPlan* pp) {
+  D2PagedPlan p{};
+  lla_status st = plan_2d(B, H, kRows, r_k, r_v, &p.d);
+  if (st != LLA_OK) return st;
+  p.d.grid = device_info().sms;
+  p.d.tpc = 0;
+  p.d.off_part = al256(p.d.off_c0 + (size_t)B * H * sizeof(float));
+  p.off_seqinfo =
+      al256(p.d.off_part + ((size_t)p.d.grid + B) * H * p.d.pstride * sizeof(float));
+  p.off_cum = al256(p.off_seqinfo + (size_t)B * sizeof(int4));
+  p.off_plan = al256(p.off_cum + (size_t)(B + 1) * sizeof(long long));
+  p.off_cstart = al256(p.off_plan + 2 * sizeof(long long));
+  p.ws_bytes = al256(p.off_cstart + (size_t)p.d.grid * sizeof(int4));
+  *pp = p;
+  return LLA_OK;
+}
+
+}  // namespace
+
+lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,
+                         int N, long long n_cap, int r_k, int r_v, const float* dk,
+                         const float* dv, const float* mu_k, const float* mu_v, float scale,
+                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  D2Plan d;
+  lla_status st = plan_2d(B, H, N, r_k, r_v, &d);
+  if (st != LLA_OK) return st;
+  if (ws == nullptr || ws_bytes < d.ws_bytes)
+    return fail(LLA_ERR_WORKSPACE, "LLA-2D workspace needs %zu bytes, got %zu", d.ws_bytes, ws_bytes);
+  CUtensorMap tk, tv;
+  {
+    const uint64_t dims[3] = {(uint64_t)r_k, (uint64_t)N, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)r_k * 2, (uint64_t)n_cap * r_k * 2};
+    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    if (!make_tmap_bf16(&tk, zk, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)r_v, (uint64_t)N, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)r_v * 2, (uint64_t)n_cap * r_v * 2};
+    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  return launch_2d(q, tk, tv, B, H, d_h, N, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, d,
+                   static_cast<char*>(ws), nullptr, stream);
+}
+
+size_t workspace_2d_paged(int B, int H, int r_k, int r_v) {
+  D2PagedPlan p;
+  if (plan_2d_paged(B, H, r_k, r_v, &p) != LLA_OK) return 0;
+  return p.ws_bytes;
+}
+
+lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, int B, int H,
+                               int d_h, int r_k, int r_v, int page_size, int num_pages,
+                               const int* block_table, int max_blocks, const int* seq_lens,
+                               const float* dk, const float* dv, const float* mu_k,
+                               const float* mu_v, float scale, float* out, float* lse, void* ws,
+                               size_t ws_bytes, cudaStream_t stream) {
+  D2PagedPlan pp;
+  lla_status st = plan_2d_paged(B, H, r_k, r_v, &pp);
+  if (st != LLA_OK) return st;
+  if (ws == nullptr || ws_bytes < pp.ws_bytes)
+    return fail(LLA_ERR_WORKSPACE, "paged LLA-2D workspace needs %zu bytes, got %zu", pp.ws_bytes,
+                ws_bytes);
+  char* wsb = static_cast<char*>(ws);
+  Paged2D pg{};
+  pg.seqinfo = reinterpret_cast<const int4*>(wsb + pp.off_seqinfo);
+  pg.cum = reinterpret_cast<long long*>(wsb + pp.off_cum);
+  pg.plan = reinterpret_cast<long long*>(wsb + pp.off_plan);
+  pg.cstart = reinterpret_cast<const int4*>(wsb + pp.off_cstart);
+  pg.block_table = block_table;
+  pg.max_blocks = max_blocks;
+  pg.page_size = page_size;
+  // The pool read page by page: rows of a page, pages outermost.
+  CUtensorMap tk, tv;
+  {
+    const uint64_t dims[3] = {(uint64_t)r_k, (uint64_t)page_size, (uint64_t)num_pages};
+    const uint64_t strides[2] = {(uint64_t)r_k * 2, (uint64_t)page_size * r_k * 2};
+    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    if (!make_tmap_bf16(&tk, zk, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)r_v, (uint64_t)page_size, (uint64_t)num_pages};
+    const uint64_t strides[2] = {(uint64_t)r_v * 2, (uint64_t)page_size * r_v * 2};
+    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  }
+  // 1. plan: tiles of kRows tokens, one worker per CTA
+  st = launch_plan_paged(seq_lens, block_table, B, 1, page_size, num_pages, max_blocks, 0, 0,
+                         pp.d.grid, 1, kRows, const_cast<int4*>(pg.seqinfo), pg.cum, pg.plan,
+                         const_cast<int4*>(pg.cstart), stream);
+  if (st != LLA_OK) return st;
+  return launch_2d(q, tk, tv, B, H, d_h, 0, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, pp.d,
+                   wsb, &pg, stream);
 }
 
 }  // namespace lla

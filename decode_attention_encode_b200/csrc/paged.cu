@@ -33,8 +33,9 @@ struct PlanArgs {
   const int* seq_lens;
   const int* block_table;
   int B, H, page_size, num_pages, max_blocks, sink, window;
-  int W;     // streaming warps
+  int W;     // streaming warps (LLA-2D: CTAs)
   int pmin;  // smallest share per warp
+  int tile_tokens;  // LLA-2D: the range counts tiles of this many tokens
   int4* seqinfo;
   long long* cum;
   long long* plan;
@@ -68,7 +69,12 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
   for (int b = b0; b < b1; ++b) {
     const int N = p.seq_lens[b];
     int n = 0, s = 0, gap = 0;
-    if (N >= 0 && N <= cap) {
+    if (N >= 0 && N <= cap && p.tile_tokens > 0) {
+      // LLA-2D: {tiles, tokens}; every used page is checked
+      n = (N + p.tile_tokens - 1) / p.tile_tokens;
+      s = N;
+      if (!pages_ok(p, b, 0, N)) n = s = gap = -1;
+    } else if (N >= 0 && N <= cap) {
       n = N;
       s = N;
       if (p.window > 0 && N > p.sink + p.window) {
@@ -166,6 +172,32 @@ lla_status plan_paged(int B, int H, int r_k, int r_v, int esz, PagedPlan* pp) {
 
 }  // namespace
 
+lla_status launch_plan_paged(const int* seq_lens, const int* block_table, int B, int H,
+                             int page_size, int num_pages, int max_blocks, int sink, int window,
+                             int W, int pmin, int tile_tokens, int4* seqinfo, long long* cum,
+                             long long* plan, int4* wstart, cudaStream_t stream) {
+  PlanArgs p{};
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.B = B;
+  p.H = H;
+  p.page_size = page_size;
+  p.num_pages = num_pages;
+  p.max_blocks = max_blocks;
+  p.sink = sink;
+  p.window = window;
+  p.W = W;
+  p.pmin = pmin;
+  p.tile_tokens = tile_tokens;
+  p.seqinfo = seqinfo;
+  p.cum = cum;
+  p.plan = plan;
+  p.wstart = wstart;
+  p.status = status_word();
+  k_plan_paged<<<1, kPlanThreads, 0, stream>>>(p);
+  return check_cuda(cudaGetLastError(), "launch k_plan_paged");
+}
+
 size_t workspace_paged(int B, int H, int r_k, int r_v, int esz) {
   PagedPlan p;
   if (plan_paged(B, H, r_k, r_v, esz, &p) != LLA_OK) return 0;
@@ -202,28 +234,9 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
 
   // 1. plan (a plain launch: it completes before k_absorb starts, so the
   //    streaming kernel may read its results before griddepcontrol.wait)
-  {
-    PlanArgs p{};
-    p.seq_lens = seq_lens;
-    p.block_table = block_table;
-    p.B = B;
-    p.H = H;
-    p.page_size = page_size;
-    p.num_pages = num_pages;
-    p.max_blocks = max_blocks;
-    p.sink = sink;
-    p.window = window;
-    p.W = d.W;
-    p.pmin = 2 * d.tile;
-    p.seqinfo = seqinfo;
-    p.cum = cum;
-    p.plan = plan;
-    p.wstart = wstart;
-    p.status = status_word();
-    k_plan_paged<<<1, kPlanThreads, 0, stream>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return check_cuda(e, "launch k_plan_paged");
-  }
+  st = launch_plan_paged(seq_lens, block_table, B, H, page_size, num_pages, max_blocks, sink,
+                         window, d.W, 2 * d.tile, 0, seqinfo, cum, plan, wstart, stream);
+  if (st != LLA_OK) return st;
   // 2. absorb (plain launch)
   st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
   if (st != LLA_OK) return st;

@@ -284,6 +284,39 @@ LLA_API lla_status lla2d_decode_attn(const float *q, const void *zk, const void 
                              void *stream);
 
 /* --------------------------------------------------------------------------
+ * LLA-2D absorbed decode over a paged latent store with per-sequence
+ * lengths, one (layer d, loop t) step: lla2d_decode_attn's definition with
+ * sequence b attending its first seq_lens[b] tokens (the paged-store
+ * reading of lla_decode_attn_paged, for the one-latent-per-token store).
+ *   zk_pages [num_pages][page_size][r_k], zv_pages [num_pages][page_size][r_v]
+ *             bf16: token j of sequence b is row j % page_size of page
+ *             block_table[b][j / page_size]. 16-byte aligned.
+ *   page_size a positive multiple of 128 (a 128-token tile never spans two
+ *             pages); num_pages, max_blocks >= 1.
+ *   block_table [B][max_blocks], seq_lens [B]: int32 device arrays, checked
+ *             on the device as for lla_decode_attn_paged (a bad length or
+ *             page index sets LLA_DEVICE_BAD_PAGED_INPUT and that sequence
+ *             is treated as empty: out = 0, lse = -inf).
+ *   workspace lla2d_decode_attn_paged_workspace(B, H, r_k, r_v) bytes.
+ * Rows of a sequence's last page past its length are read (the tensor
+ * cores take whole 128-token tiles) and weighted by zero: they must hold
+ * finite values, as a zero-initialised pool does. Other limits as
+ * lla2d_decode_attn.
+ * -------------------------------------------------------------------------- */
+LLA_API size_t lla2d_decode_attn_paged_workspace(int B, int H, int r_k, int r_v);
+
+LLA_API lla_status lla2d_decode_attn_paged(const float *q, const void *zk_pages,
+                                           const void *zv_pages, lla_dtype zdt,
+                                           int B, int H, int d_h, int r_k, int r_v,
+                                           int page_size, int num_pages,
+                                           const int *block_table, int max_blocks,
+                                           const int *seq_lens, const float *dk_t,
+                                           const float *dv_t, const float *mu_k_t,
+                                           const float *mu_v_t, float scale,
+                                           float *out, float *lse, void *workspace,
+                                           size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
  * Latent write (§3 Eq. 2 over the loop-major stack of Eq. 1):
  *   z[g][n][c] = bf16_rne( sum_k (xs[k] - mu[g][k]) * W_down[g][k][c] ),
  *   xs[t*d_loop + i] = x[t][n][g][i].
