@@ -210,8 +210,10 @@ class DecodeWorkload:
             bt, num_pages = synth.page_table(lens, c.page_size, s + 12)
             self.block_table = torch.from_numpy(bt).to(device)
             self.seq_lens = torch.from_numpy(lens).to(device)
-            zk_shape = (num_pages, c.H, c.page_size, c.r_k)
-            zv_shape = (num_pages, c.H, c.page_size, c.r_v)
+            zk_shape = ((num_pages, c.page_size, c.r_k) if c.two_d
+                        else (num_pages, c.H, c.page_size, c.r_k))
+            zv_shape = ((num_pages, c.page_size, c.r_v) if c.two_d
+                        else (num_pages, c.H, c.page_size, c.r_v))
         self.zk = [synth.latents(zk_shape, s + 1000 * l + 1, device, decay=c.decay,
                                  dtype=c.torch_dtype) for l in range(c.L)]
         self.zv = [synth.latents(zv_shape, s + 1000 * l + 2, device, decay=c.decay,
@@ -228,7 +230,9 @@ class DecodeWorkload:
         import decode_attention_encode_b200 as lla
         self.lla = lla
         if self.paged:
-            need = lla.lla_decode_attn_paged_workspace(c.B, c.H, c.r_k, c.r_v)
+            wsfn = (lla.lla2d_decode_attn_paged_workspace if c.two_d
+                    else lla.lla_decode_attn_paged_workspace)
+            need = wsfn(c.B, c.H, c.r_k, c.r_v)
         elif self.rope:
             need = lla.lla_decode_attn_workspace(c.B, c.H, c.N, c.r_k + c.d_r, c.r_v)
         else:
@@ -284,10 +288,9 @@ class DecodeWorkload:
         out = self.out if out is None else out
         lse = self.lse if lse is None else lse
         if self.paged:
-            self.lla.lla_decode_attn_paged(q[l, t], self.zk[l], self.zv[l], self.block_table,
-                                           self.seq_lens, self.dk[l, t], self.dv[l, t],
-                                           scale=self.scale, out=out[l, t], lse=lse[l, t],
-                                           workspace=self.ws)
+            fn = self.lla.lla2d_decode_attn_paged if c.two_d else self.lla.lla_decode_attn_paged
+            fn(q[l, t], self.zk[l], self.zv[l], self.block_table, self.seq_lens, self.dk[l, t],
+               self.dv[l, t], scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
         elif self.rope:
             self.lla.lla_decode_attn_rope(q[l, t], q_rope[l, t], self.zk[l], self.zv[l],
                                           self.dk[l, t], self.dv[l, t], N=c.N, scale=self.scale,

@@ -18,6 +18,7 @@ from ._lib import (  # noqa: F401
     library_path,
     lla2d_decode_attn,
     lla2d_decode_attn_paged,
+    lla2d_decode_attn_paged_workspace,
     lla2d_decode_attn_workspace,
     lla_decode_attn,
     lla_decode_attn_noalloc,

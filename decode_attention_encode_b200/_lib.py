@@ -318,6 +318,10 @@ def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv
     return out, lse
 
 
+def lla2d_decode_attn_paged_workspace(B, H, r_k, r_v):
+    return int(lib().lla2d_decode_attn_paged_workspace(B, H, r_k, r_v))
+
+
 def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t,
                             mu_k_t=None, mu_v_t=None, scale=None, out=None, lse=None,
                             workspace=None, stream=None, want_lse=True):

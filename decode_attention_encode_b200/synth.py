@@ -208,4 +208,8 @@ C5_ENCODE = EncodeConfig("encode_32x", L=24, T=4, G=16, d_loop=128, r=16, N=3276
 # the 4x geometry with a 64-wide decoupled rotary branch on the key side
 C2_ROPE = DecodeConfig("perhead_4x_rope", L=24, T=4, H=16, d_h=128, r_k=128, r_v=128, B=64,
                        N=4096, dtype="bf16", decay=True, d_r=64)
-DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE)}
+# the 32x LLA-2D geometry as a serving batch: 256 sequences of 4096..12288
+# tokens in a pool of 256-token pages
+C4_PAGED = DecodeConfig("lla2d_32x_paged", L=24, T=4, H=16, d_h=128, r_k=256, r_v=256, B=256,
+                        N=8192, dtype="bf16", decay=True, two_d=True, page_size=256, spread=0.5)
+DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE, C4_PAGED)}
