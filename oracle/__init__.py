@@ -24,7 +24,8 @@ What is here, each in fp64:
   * ``compression_ratio``: §3 Eq. 4.
   * ``rope_rotate`` / ``decode_unit_rope`` / ``lla_decode_rope``: the
     decoupled-RoPE split of §7 (NoPE latent content path plus an explicit
-    rotary branch), as attention over concatenated content and rotary keys.
+    rotary branch), as attention over concatenated content and rotary keys;
+    ``lla2d_decode_rope`` with the key row shared by every head.
   * ``paged2d_decode``: the same gather for the LLA-2D store.
   * ``kept_positions`` / ``paged_decode``: the per-head decode over a paged
     store with per-sequence lengths (a gather of each unit's rows, then the
@@ -292,6 +293,34 @@ def lla_decode_rope(q, q_rope, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None,
     for i, (b, h) in enumerate(units):
         out[i], lse[i] = decode_unit_rope(
             q[b, h], q_rope[b, h], zk[b, h, :N, :r_k], zk[b, h, :N, r_k:], zv[b, h, :N],
+            np.asarray(dk)[h], np.asarray(dv)[h],
+            None if mu_k is None else np.asarray(mu_k)[h],
+            None if mu_v is None else np.asarray(mu_v)[h], scale)
+    if full:
+        return out.reshape(B, H, d), lse.reshape(B, H)
+    return out, lse
+
+
+def lla2d_decode_rope(q, q_rope, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=None, N=None,
+                      units=None):
+    """LLA-2D decode with the decoupled rotary branch: the key row of each
+    token [latent (r_k) | rotated rotary key (d_r)] is shared by every head,
+    as MLA shares its rotary key (zk [B, n_cap, r_k + d_r], zv [B, n_cap,
+    r_v]); q_rope [B, H, d_r] is each head's rotated rotary query. Per unit
+    this is ``decode_unit_rope`` on the shared rows."""
+    q, q_rope = np.asarray(q), np.asarray(q_rope)
+    B, H, d = q.shape
+    d_r = q_rope.shape[-1]
+    zk, zv = np.asarray(zk), np.asarray(zv)
+    r_k = zk.shape[-1] - d_r
+    N = zk.shape[1] if N is None else N
+    full = units is None
+    units = [(b, h) for b in range(B) for h in range(H)] if full else units
+    out = np.zeros((len(units), d))
+    lse = np.zeros(len(units))
+    for i, (b, h) in enumerate(units):
+        out[i], lse[i] = decode_unit_rope(
+            q[b, h], q_rope[b, h], zk[b, :N, :r_k], zk[b, :N, r_k:], zv[b, :N],
             np.asarray(dk)[h], np.asarray(dv)[h],
             None if mu_k is None else np.asarray(mu_k)[h],
             None if mu_v is None else np.asarray(mu_v)[h], scale)

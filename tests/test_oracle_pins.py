@@ -609,3 +609,24 @@ def test_paged2d_equals_dense_2d_decode_per_sequence_length():
     pg = bt[0, 0]
     for h in range(H):
         np.testing.assert_allclose(o1[0, h], dv[h] @ zvp[pg, 0] + mv[h], atol=1e-12)
+
+
+def test_lla2d_rope_is_per_head_rope_with_the_row_shared_by_every_head():
+    r = rng(71)
+    B, H, d, N, rk, dr, rv = 2, 3, 8, 9, 8, 4, 12
+    zk = r.standard_normal((B, N, rk + dr))
+    zv = r.standard_normal((B, N, rv))
+    q, qr = r.standard_normal((B, H, d)), r.standard_normal((B, H, dr))
+    dk, dv = r.standard_normal((H, d, rk)), r.standard_normal((H, d, rv))
+    mk, mv = r.standard_normal((H, d)), r.standard_normal((H, d))
+    o2, l2 = oracle.lla2d_decode_rope(q, qr, zk, zv, dk, dv, mk, mv)
+    zk_h = np.repeat(zk[:, None], H, axis=1)
+    zv_h = np.repeat(zv[:, None], H, axis=1)
+    o1, l1 = oracle.lla_decode_rope(q, qr, zk_h, zv_h, dk, dv, mk, mv)
+    np.testing.assert_allclose(o2, o1, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, atol=1e-12)
+    # and with a zero rotary query it is the plain LLA-2D decode
+    o3, l3 = oracle.lla2d_decode_rope(q, np.zeros_like(qr), zk, zv, dk, dv, mk, mv)
+    o4, l4 = oracle.lla2d_decode(q, zk[:, :, :rk], zv, dk, dv, mk, mv)
+    np.testing.assert_allclose(o3, o4, atol=1e-12)
+    np.testing.assert_allclose(l3, l4, atol=1e-12)
