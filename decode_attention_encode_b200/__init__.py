@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     lla2d_decode_attn,
     lla2d_decode_attn_paged,
     lla2d_decode_attn_paged_workspace,
+    lla2d_decode_attn_rope,
     lla2d_decode_attn_workspace,
     lla_decode_attn,
     lla_decode_attn_noalloc,

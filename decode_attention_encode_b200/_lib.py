@@ -36,7 +36,7 @@ EXPORTS = (
     "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
-    "lla2d_decode_attn_workspace", "lla2d_decode_attn",
+    "lla2d_decode_attn_workspace", "lla2d_decode_attn", "lla2d_decode_attn_rope",
     "lla2d_decode_attn_paged_workspace", "lla2d_decode_attn_paged",
     "lla_encode", "lla_encode_bias", "lla_encode_with_bias_workspace", "lla_encode_with_bias",
 )
@@ -68,6 +68,8 @@ _SIGS = {
                               [_c_int] * 2 + [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp],
                               _c_int),
     "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
+    "lla2d_decode_attn_rope": ([_vp, _vp, _vp, _vp, _c_int] + [_c_int] * 8 + [_vp] * 4 +
+                               [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla2d_decode_attn_paged_workspace": ([_c_int] * 4, _c_size),
     "lla2d_decode_attn_paged": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp, _c_int, _vp] +
                                 [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
@@ -314,6 +316,38 @@ def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv
                                  _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t), float(scale), _ptr(out),
                                  _ptr(lse), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def lla2d_decode_attn_rope(q, q_rope, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None,
+                           scale=None, out=None, lse=None, workspace=None, stream=None,
+                           want_lse=True):
+    """LLA-2D decode with the decoupled rotary branch: zk [B,n_cap,r_k+d_r]
+    holds each token's latent followed by its rotated rotary key (shared by
+    every head); q_rope [B,H,d_r]; dk_t [H,d_h,r_k]. Returns (out, lse)."""
+    _need_cuda(q, q_rope, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
+    B, H, d_h = q.shape
+    d_r = q_rope.shape[2]
+    n_cap, rq = zk.shape[1], zk.shape[2]
+    r_k, r_v = dk_t.shape[2], zv.shape[2]
+    if rq != r_k + d_r:
+        raise LLAError(LLA_ERR_INVALID_ARG, "zk rows must hold r_k + d_r values")
+    N = n_cap if N is None else N
+    scale = 1.0 / math.sqrt(d_h) if scale is None else scale
+    if out is None:
+        out = torch.empty((B, H, d_h), device=q.device, dtype=torch.float32)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
+    h = lib()
+    need = int(h.lla2d_decode_attn_workspace(B, H, N, rq, r_v))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    st = h.lla2d_decode_attn_rope(_ptr(q), _ptr(q_rope), _ptr(zk), _ptr(zv), _dtype_code(zk), B,
+                                  H, d_h, d_r, N, n_cap, r_k, r_v, _ptr(dk_t), _ptr(dv_t),
+                                  _ptr(mu_k_t), _ptr(mu_v_t), float(scale), _ptr(out), _ptr(lse),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
     _check(st)
     return out, lse
 

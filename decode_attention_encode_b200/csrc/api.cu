@@ -285,7 +285,8 @@ lla_status lla_decode_attn_paged(const float* q, const void* zk_pages, const voi
 }
 
 size_t lla2d_decode_attn_workspace(int B, int H, int N, int r_k, int r_v) {
-  if (B < 1 || H < 1 || H > 32 || N < 1 || r_k < 64 || r_k > 256 || r_k % 64 || r_v < 128 ||
+  // r_k is the key row width (r_k + d_r for lla2d_decode_attn_rope)
+  if (B < 1 || H < 1 || H > 32 || N < 1 || r_k < 64 || r_k > 384 || r_k % 64 || r_v < 128 ||
       r_v > 256 || r_v % 128)
     return 0;
   return workspace_2d(B, H, N, r_k, r_v);
@@ -308,6 +309,34 @@ lla_status lla2d_decode_attn(const float* q, const void* zk, const void* zv, lla
   return run_decode_2d(q, zk, zv, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t, mu_k_t,
                        mu_v_t, scale, out, lse, workspace, ws_bytes,
                        static_cast<cudaStream_t>(stream));
+}
+
+lla_status lla2d_decode_attn_rope(const float* q, const float* q_rope, const void* zk,
+                                  const void* zv, lla_dtype zdt, int B, int H, int d_h, int d_r,
+                                  int N, int n_cap, int r_k, int r_v, const float* dk_t,
+                                  const float* dv_t, const float* mu_k_t, const float* mu_v_t,
+                                  float scale, float* out, float* lse, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  if (!q_rope) return fail(LLA_ERR_INVALID_ARG, "q_rope must be non-NULL");
+  if (!aligned(q_rope, 4)) return fail(LLA_ERR_INVALID_ARG, "q_rope must be 4-byte aligned");
+  if (d_r < 8 || d_r % 8) return fail(LLA_ERR_INVALID_ARG, "d_r must be a positive multiple of 8");
+  if (r_k < 8 || r_k % 8) return fail(LLA_ERR_INVALID_ARG, "r_k must be a positive multiple of 8");
+  int esz = 0;
+  // shared checks on the latent part; the key-row limits follow
+  lla_status st = check_decode_args(q, zk, zv, zdt, B, H, d_h, N, n_cap, 8, r_v, dk_t, dv_t, mu_k_t,
+                                    mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
+  if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
+  const int rq = r_k + d_r;
+  if (rq % 64 || rq > 384 || r_v % 128)
+    return fail(LLA_ERR_UNSUPPORTED,
+                "LLA-2D with a rotary branch needs r_k + d_r a multiple of 64 up to 384 and r_v "
+                "a multiple of 128");
+  return run_decode_2d(q, zk, zv, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t, mu_k_t,
+                       mu_v_t, scale, out, lse, workspace, ws_bytes,
+                       static_cast<cudaStream_t>(stream), q_rope, d_r);
 }
 
 size_t lla2d_decode_attn_paged_workspace(int B, int H, int r_k, int r_v) {

@@ -129,7 +129,8 @@ size_t workspace_2d(int B, int H, int N, int r_k, int r_v);
 lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,
                          int N, long long n_cap, int r_k, int r_v, const float* dk,
                          const float* dv, const float* mu_k, const float* mu_v, float scale,
-                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                         const float* q_rope = nullptr, int d_r = 0);
 
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream,

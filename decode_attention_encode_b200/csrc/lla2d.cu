@@ -685,14 +685,18 @@ struct Paged2D {
 
 // Absorb, the tensor-core kernel and the merge, shared by the dense and the
 // paged entry points.
+// r_k is the width of a key row, the latent part plus d_r rotary values
+// when q_rope is given.
 lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& tv, int B, int H,
                      int d_h, int N, int r_k, int r_v, const float* dk, const float* dv,
                      const float* mu_k, const float* mu_v, float scale, float* out, float* lse,
-                     const D2Plan& d, char* wsb, const Paged2D* pg, cudaStream_t stream) {
+                     const D2Plan& d, char* wsb, const Paged2D* pg, cudaStream_t stream,
+                     const float* q_rope = nullptr, int d_r = 0) {
   unsigned char* qsw = reinterpret_cast<unsigned char*>(wsb + d.off_qsw);
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
-  lla_status st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, nullptr, c0, stream, qsw, d.hp);
+  lla_status st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k - d_r, scale, nullptr, c0, stream, qsw,
+                                d.hp, q_rope, d_r);
   if (st != LLA_OK) return st;
 
   D2Args a{};
@@ -785,7 +789,10 @@ lla_status plan_2d_paged(int B, int H, int r_k, int r_v, D2PagedPlan* pp) {
 lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,
                          int N, long long n_cap, int r_k, int r_v, const float* dk,
                          const float* dv, const float* mu_k, const float* mu_v, float scale,
-                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                         float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                         const float* q_rope, int d_r) {
+  if (!q_rope) d_r = 0;
+  r_k += d_r;  // the key row: latent, then the rotary key
   D2Plan d;
   lla_status st = plan_2d(B, H, N, r_k, r_v, &d);
   if (st != LLA_OK) return st;
@@ -805,7 +812,7 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
   return launch_2d(q, tk, tv, B, H, d_h, N, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, d,
-                   static_cast<char*>(ws), nullptr, stream);
+                   static_cast<char*>(ws), nullptr, stream, q_rope, d_r);
 }
 
 size_t workspace_2d_paged(int B, int H, int r_k, int r_v) {

@@ -284,6 +284,31 @@ LLA_API lla_status lla2d_decode_attn(const float *q, const void *zk, const void 
                              void *stream);
 
 /* --------------------------------------------------------------------------
+ * LLA-2D absorbed decode with a decoupled rotary branch, one (layer d,
+ * loop t) step: lla_decode_attn_rope's definition on the LLA-2D store.
+ * Each token's key row [latent r_k | rotated rotary key d_r] is shared by
+ * every head, as MLA shares its rotary key (the pages' MLA-style split of
+ * §7 "Per-head LLA versus LLA-2D at inference" applied to §3 "The LLA-2D
+ * variant"); q_rope [B][H][d_r] fp32 is each head's rotated rotary query.
+ *   zk  [B][n_cap][r_k + d_r] bf16; zv [B][n_cap][r_v] bf16.
+ *   r_k + d_r a multiple of 64, at most 384; d_r a positive multiple of 8;
+ *   r_v a multiple of 128, at most 256; H <= 32.
+ *   workspace  lla2d_decode_attn_workspace(B, H, N, r_k + d_r, r_v) bytes
+ *   (that query takes the key-row width, up to 384).
+ * The rotary query is rounded to bf16 with the absorbed query for the
+ * tensor cores.
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla2d_decode_attn_rope(const float *q, const float *q_rope,
+                                          const void *zk, const void *zv,
+                                          lla_dtype zdt, int B, int H, int d_h,
+                                          int d_r, int N, int n_cap, int r_k,
+                                          int r_v, const float *dk_t,
+                                          const float *dv_t, const float *mu_k_t,
+                                          const float *mu_v_t, float scale,
+                                          float *out, float *lse, void *workspace,
+                                          size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
  * LLA-2D absorbed decode over a paged latent store with per-sequence
  * lengths, one (layer d, loop t) step: lla2d_decode_attn's definition with
  * sequence b attending its first seq_lens[b] tokens (the paged-store
