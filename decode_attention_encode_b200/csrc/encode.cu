@@ -38,11 +38,16 @@ constexpr int kTileM = 128;     // tokens per tile (TMEM lanes)
 constexpr int kChunkK = 64;     // K elements per stage (128 B rows)
 constexpr int kABytes = kTileM * kChunkK * 2;
 constexpr int kThreads = 192;   // 6 warps
+constexpr int kMaxStages = 12;  // enough bytes in flight to cover HBM latency at r = 16
 
 struct EncodeArgs {
   // work items are (tile, K split) pairs: item = tile * ksplit + split
   int N, G, d_loop, r, r_pad, K, nk, mtiles, tiles, tiles_per_cta;
   int ksplit, cpk;  // K splits per tile and chunks per split
+  // tile order: token-major (all groups of a 128-token tile in a row, so a
+  // token's G * d_loop input row is read at once) or group-major (one
+  // group's tiles in a row, so the in-kernel mean term changes rarely)
+  int token_major;
   float* part;      // ksplit > 1: fp32 partials [ksplit][G][N][r]
   int nstage, b_bytes, stage_bytes;
   uint32_t tmem_cols;
@@ -55,8 +60,8 @@ struct EncodeArgs {
 };
 
 struct SmemTail {
-  uint64_t full[8];
-  uint64_t empty[8];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -125,8 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int item = t_begin; item < t_end && ok; ++item) {
         const int tile = item / a.ksplit, split = item - tile * a.ksplit;
-        const int g = tile / a.mtiles;
-        const int m0 = (tile - g * a.mtiles) * kTileM;
+        const int g = a.token_major ? tile % a.G : tile / a.mtiles;
+        const int m0 = (a.token_major ? tile / a.G : tile - g * a.mtiles) * kTileM;
         const int kc0 = split * a.cpk, kc1 = min(a.nk, kc0 + a.cpk);
         for (int kc = kc0; kc < kc1; ++kc, ++it) {
           const int s = it % a.nstage;
@@ -212,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int cur_g = -1;
     for (int item = t_begin, lt = 0; item < t_end; ++item, ++lt) {
       const int tile = item / a.ksplit, split = item - tile * a.ksplit;
-      const int g = tile / a.mtiles;
-      const int m0 = (tile - g * a.mtiles) * kTileM;
+      const int g = a.token_major ? tile % a.G : tile / a.mtiles;
+      const int m0 = (a.token_major ? tile / a.G : tile - g * a.mtiles) * kTileM;
       if (g != cur_g && !a.part) {
         if (!epi_sync()) break;  // previous tile's readers of muw are done
         for (int c = ew; c < a.r; c += 4) {
@@ -470,6 +475,7 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
       a.part = static_cast<float*>(ws);
     }
   }
+  a.token_major = env_int("LLA_ENCODE_TOKEN_MAJOR", 0);
   a.b_bytes = r_pad * kChunkK * 2;
   a.stage_bytes = kABytes + a.b_bytes;
   uint32_t cols = 32;
@@ -485,12 +491,29 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
 
   const DeviceInfo di = device_info();
   const size_t fixed = sizeof(SmemTail) + 1024;
-  int nst = (int)std::min<size_t>(8, ((size_t)di.smem_optin - fixed) / a.stage_bytes);
+  // CTAs per SM: several independent producer / MMA / epilogue pipelines
+  // per SM stream faster than one (measured at r = 16: 104 us with one,
+  // 91 us with three). Take the most, up to 3, that leave each CTA 4
+  // stages, fit the SM's 512 TMEM columns and still have a tile each.
+  const int items_all = a.tiles * a.ksplit;
+  int per_sm = 1;
+  for (int p = 3; p >= 2; --p) {
+    const size_t per_cta = (size_t)di.smem_optin / p - 1024;
+    if ((size_t)p * cols <= 512 && per_cta > fixed && (per_cta - fixed) / a.stage_bytes >= 4 &&
+        items_all >= p * di.sms) {
+      per_sm = p;
+      break;
+    }
+  }
+  per_sm = std::max(1, std::min(3, env_int("LLA_ENCODE_CTAS_PER_SM", per_sm)));
+  const size_t smem_cta = (size_t)di.smem_optin / per_sm - (per_sm > 1 ? 1024 : 0);
+  int nst = (int)std::min<size_t>(std::max(2, std::min(kMaxStages, env_int("LLA_ENCODE_STAGES", kMaxStages))),
+                                  (smem_cta - fixed) / a.stage_bytes);
   if (nst < 2) return fail(LLA_ERR_UNSUPPORTED, "encode stage does not fit in shared memory");
   a.nstage = nst;
   const size_t smem = (size_t)nst * a.stage_bytes + fixed;
   const int items = a.tiles * a.ksplit;
-  const int grid0 = std::min(items, di.sms);
+  const int grid0 = std::min(items, di.sms * per_sm);
   a.tiles_per_cta = (items + grid0 - 1) / grid0;
   const int grid = (items + a.tiles_per_cta - 1) / a.tiles_per_cta;
 
