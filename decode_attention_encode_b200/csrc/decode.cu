@@ -36,15 +36,32 @@
 namespace lla {
 namespace {
 
-// Rows per thread of k_absorb / k_combine: the largest of 1, 2, 4, 8 that
-// still gives at least ~256 CTAs (more rows per thread reuse each decoder
-// value from shared memory more often).
-int rows_per_thread(int ctas_per_row_block_of_8, int B) {
-  int rows = 8;
-  while (rows > 1 && (long long)ctas_per_row_block_of_8 * ((B + 8 * rows - 1) / (8 * rows)) < 256)
-    rows >>= 1;
-  return rows;
+// Register block of k_absorb / k_combine threads: ROWS batch rows (1, 2, 4,
+// 8) by COLS columns (1, 2, 4) per thread, the largest ROWS * COLS that
+// still gives at least ~256 CTAs for `nh` heads, `ncols` output columns and
+// B rows; ties go to more rows, or with prefer_cols to more columns (fewer
+// column blocks, which k_combine pays for by merging the same partials in
+// each). Larger blocks reuse each shared-memory read for more FMAs.
+void pick_block(int nh, int ncols, int B, int* rows_out, int* cols_out, bool prefer_cols = false,
+                int max_cols = 4) {
+  int best_r = 1, best_c = 1, best = 0;
+  for (int r : {8, 4, 2, 1})
+    for (int c : {4, 2, 1}) {
+      if (c > max_cols) continue;
+      if (c > 1 && ncols < 32 * c) continue;  // lanes would sit idle
+      const long long ctas = (long long)nh * ((ncols + 32 * c - 1) / (32 * c)) *
+                             ((B + 8 * r - 1) / (8 * r));
+      if (ctas < 256 && !(r == 1 && c == 1)) continue;
+      if (r * c > best || (prefer_cols && r * c == best && c > best_c)) {
+        best = r * c;
+        best_r = r;
+        best_c = c;
+      }
+    }
+  *rows_out = best_r;
+  *cols_out = best_c;
 }
+
 
 // Stages n float4 items into shared memory with the whole CTA (256 threads):
 // each thread issues up to 8 global loads before its first shared store, so
@@ -86,31 +103,48 @@ struct AbsorbArgs {
   int d_r;
 };
 
-// One CTA per (head, 32 latent columns, 8*ROWS batch rows). The CTA stages
-// its d_h x 32 slice of W^K_up,t (all float4 loads issued before the first
-// use) and its query rows in shared memory; thread (warp w, lane l) forms
-// q'[b][c0 + l] for the ROWS rows b = b0 + w*ROWS + k, so one decoder value
-// read from shared memory feeds ROWS FMAs and one float4 query read feeds 4.
-template <int ROWS>
+// One CTA per (head, 32*COLS latent columns, 8*ROWS batch rows). The CTA
+// stages its d_h x 32*COLS slice of W^K_up,t and its query rows in shared
+// memory; thread (warp w, lane l) forms q'[b][c0 + l*COLS + j] for the ROWS
+// rows b = b0 + w*ROWS + k and its COLS columns j, so one shared-memory read
+// of COLS decoder values feeds ROWS*COLS FMAs and one float4 query read
+// (the same address for the whole warp) feeds 4*COLS. The kernel is bound by
+// shared-memory instructions, so larger ROWS*COLS blocks run faster.
+template <int COLS>
+__device__ __forceinline__ void lds_cols(const float* p, float (&v)[COLS]) {
+  if constexpr (COLS == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else if constexpr (COLS == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+    v[0] = *p;
+  }
+}
+
+template <int ROWS, int COLS>
 __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
+  constexpr int CW = 32 * COLS;  // columns per CTA
   extern __shared__ __align__(16) float sm_absorb[];
   const int d_h4 = (a.d_h + 3) & ~3;
-  float* d_s = sm_absorb;                   // [d_h4][32]
-  float* q_s = sm_absorb + d_h4 * 32;       // [8*ROWS][d_h4]
+  float* d_s = sm_absorb;                   // [d_h4][CW]
+  float* q_s = sm_absorb + d_h4 * CW;       // [8*ROWS][d_h4]
   pdl_launch_dependents();
   const int h = blockIdx.x;
-  const int c0 = blockIdx.y * 32;
+  const int c0 = blockIdx.y * CW;
   const int b0 = blockIdx.z * (8 * ROWS);
   const int nb = min(8 * ROWS, a.B - b0);
   const int rq = a.r_k + a.d_r;        // q' row: latent part, then rotary part
-  const int nc = min(32, rq - c0);     // columns of this CTA, a multiple of 8
-  const int n4 = max(0, min(32, a.r_k - c0)) / 4;  // of them from W^K, in float4
+  const int nc = min(CW, rq - c0);     // columns of this CTA, a multiple of 8
+  const int n4 = max(0, min(CW, a.r_k - c0)) / 4;  // of them from W^K, in float4
   const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
-  stage_batched(d_h4 * 8, [&](int idx) {
-    const int i = idx >> 3, j = idx & 7;
+  constexpr int F4 = CW / 4;  // float4 per staged decoder row
+  stage_batched(d_h4 * F4, [&](int idx) {
+    const int i = idx / F4, j = idx - i * F4;
     return (i < a.d_h && j < n4) ? __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j)
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-  }, [&](int idx, float4 v) { reinterpret_cast<float4*>(d_s + (idx >> 3) * 32)[idx & 7] = v; });
+  }, [&](int idx, float4 v) { reinterpret_cast<float4*>(d_s)[idx] = v; });
   const int q4 = d_h4 / 4;  // float4 per staged query row
   if ((a.d_h & 3) == 0 && (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {
     stage_batched(8 * ROWS * q4, [&](int idx) {
@@ -146,21 +180,31 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
       if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
     }
   }
-  float acc[ROWS];
+  float acc[ROWS][COLS];
 #pragma unroll
-  for (int k = 0; k < ROWS; ++k) acc[k] = 0.f;
+  for (int k = 0; k < ROWS; ++k)
+#pragma unroll
+    for (int j = 0; j < COLS; ++j) acc[k][j] = 0.f;
   const float* qrow = q_s + warp * ROWS * d_h4;
+  const float* dcol = d_s + lane * COLS;
   for (int i = 0; i < d_h4; i += 4) {
-    const float d0 = d_s[(i + 0) * 32 + lane], d1 = d_s[(i + 1) * 32 + lane];
-    const float d2 = d_s[(i + 2) * 32 + lane], d3 = d_s[(i + 3) * 32 + lane];
+    float dv[4][COLS];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) lds_cols<COLS>(dcol + (i + e) * CW, dv[e]);
 #pragma unroll
     for (int k = 0; k < ROWS; ++k) {
       const float4 qv = *reinterpret_cast<const float4*>(qrow + k * d_h4 + i);
-      acc[k] = fmaf(d0, qv.x, fmaf(d1, qv.y, fmaf(d2, qv.z, fmaf(d3, qv.w, acc[k]))));
+#pragma unroll
+      for (int j = 0; j < COLS; ++j)
+        acc[k][j] = fmaf(dv[0][j], qv.x,
+                         fmaf(dv[1][j], qv.y, fmaf(dv[2][j], qv.z, fmaf(dv[3][j], qv.w, acc[k][j]))));
     }
   }
-  if (lane < nc) {
-    const int c = c0 + lane;
+#pragma unroll
+  for (int j = 0; j < COLS; ++j) {
+    const int cl = lane * COLS + j;  // column within the CTA
+    if (cl >= nc) continue;
+    const int c = c0 + cl;
 #pragma unroll
     for (int k = 0; k < ROWS; ++k) {
       const int bb = warp * ROWS + k;
@@ -168,7 +212,7 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
       const size_t unit = (size_t)(b0 + bb) * a.H + h;
       // the rotary part of the query is not absorbed: it meets the cached
       // rotated keys as it is
-      const float v = (c < a.r_k ? acc[k] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
+      const float v = (c < a.r_k ? acc[k][j] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
                       a.qscale;
       if (a.qp) a.qp[unit * rq + c] = v;
       if (a.qsw) {
@@ -210,8 +254,9 @@ struct CombineArgs {
 // flight each, since this kernel is bound by memory round trips, not
 // bandwidth. Thread (w, l) finally forms out[b][h][i0 + l] for its ROWS
 // rows.
-template <int ROWS>
+template <int ROWS, int COLS>
 __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
+  constexpr int CW = 32 * COLS;  // output channels per CTA
   extern __shared__ __align__(16) float sm_combine[];
   // per row of the CTA: pieces, offset of the first record, merged max,
   // 1 / normaliser, and 0 for a row with no attended token
@@ -219,13 +264,13 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
   __shared__ long long s_off[64];
   __shared__ float s_M[64], s_inv[64], s_keep[64];
   const int pitch = a.r_v + 4;
-  float* d_s = sm_combine;                        // [32][pitch]
-  float* ub = sm_combine + 32 * pitch;            // [8*ROWS][r_v]
+  float* d_s = sm_combine;                        // [CW][pitch]
+  float* ub = sm_combine + CW * pitch;            // [8*ROWS][r_v]
   const int h = blockIdx.x;
-  const int i0 = blockIdx.y * 32;
+  const int i0 = blockIdx.y * CW;
   const int b0 = blockIdx.z * (8 * ROWS);
   const int nb = min(8 * ROWS, a.B - b0);
-  const int ni = min(32, a.d_h - i0);
+  const int ni = min(CW, a.d_h - i0);
   const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
   const int r4 = a.r_v / 4;
   stage_batched(ni * r4, [&](int idx) {
@@ -358,25 +403,38 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
     }
   }
   __syncthreads();
-  if (lane < ni) {
-    float acc[ROWS];
+  // thread (w, l): channels i0 + l + 32 j (j < COLS; consecutive lanes read
+  // consecutive padded rows, so the float4 reads are conflict-free) for the
+  // ROWS rows of warp w
+  float acc[ROWS][COLS];
 #pragma unroll
-    for (int k = 0; k < ROWS; ++k) acc[k] = 0.f;
-    const float4* drow = reinterpret_cast<const float4*>(d_s + lane * pitch);
-    const float4* ubase = reinterpret_cast<const float4*>(ub + warp * ROWS * a.r_v);
-    for (int c4 = 0; c4 < r4; ++c4) {
-      const float4 dv = drow[c4];
+  for (int k = 0; k < ROWS; ++k)
 #pragma unroll
-      for (int k = 0; k < ROWS; ++k) {
-        const float4 uv = ubase[k * r4 + c4];
-        acc[k] = fmaf(dv.x, uv.x, fmaf(dv.y, uv.y, fmaf(dv.z, uv.z, fmaf(dv.w, uv.w, acc[k]))));
-      }
+    for (int j = 0; j < COLS; ++j) acc[k][j] = 0.f;
+  const float4* ubase = reinterpret_cast<const float4*>(ub + warp * ROWS * a.r_v);
+  for (int c4 = 0; c4 < r4; ++c4) {
+    float4 dv[COLS];
+#pragma unroll
+    for (int j = 0; j < COLS; ++j)
+      dv[j] = reinterpret_cast<const float4*>(d_s + (lane + 32 * j) * pitch)[c4];
+#pragma unroll
+    for (int k = 0; k < ROWS; ++k) {
+      const float4 uv = ubase[k * r4 + c4];
+#pragma unroll
+      for (int j = 0; j < COLS; ++j)
+        acc[k][j] = fmaf(dv[j].x, uv.x, fmaf(dv[j].y, uv.y, fmaf(dv[j].z, uv.z, fmaf(dv[j].w, uv.w, acc[k][j]))));
     }
-    const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + lane] : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < COLS; ++j) {
+    const int il = lane + 32 * j;
+    if (il >= ni) continue;
+    const float mu = a.mu_v ? a.mu_v[(size_t)h * a.d_h + i0 + il] : 0.f;
 #pragma unroll
     for (int k = 0; k < ROWS; ++k) {
       const int bb = warp * ROWS + k;
-      if (bb < nb) a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + lane] = acc[k] + mu * s_keep[bb];
+      if (bb < nb)
+        a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + il] = acc[k][j] + mu * s_keep[bb];
     }
   }
 }
@@ -400,13 +458,18 @@ lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int
                          unsigned char* qsw, int hp, const float* q_rope, int d_r) {
   AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp,
                q_rope, q_rope ? d_r : 0};
-  const int ncol = (r_k + a.d_r + 31) / 32;
-  const int rows = rows_per_thread(H * ncol, B);
-  dim3 grid(H, ncol, (B + 8 * rows - 1) / (8 * rows));
+  const int rq = r_k + a.d_r;
+  int rows, cols;
+  pick_block(H, rq, B, &rows, &cols, false, env_int("LLA_ABSORB_MAX_COLS", 2));
+  dim3 grid(H, (rq + 32 * cols - 1) / (32 * cols), (B + 8 * rows - 1) / (8 * rows));
   const int d_h4 = (d_h + 3) & ~3;
-  const size_t smem = ((size_t)d_h4 * 32 + (size_t)8 * rows * d_h4) * sizeof(float);
-  void (*fn)(AbsorbArgs) = rows == 8 ? k_absorb<8> : rows == 4 ? k_absorb<4>
-                         : rows == 2 ? k_absorb<2> : k_absorb<1>;
+  const size_t smem = ((size_t)d_h4 * 32 * cols + (size_t)8 * rows * d_h4) * sizeof(float);
+  using Fn = void (*)(AbsorbArgs);
+  const Fn fns[4][3] = {{k_absorb<1, 1>, k_absorb<1, 2>, k_absorb<1, 4>},
+                        {k_absorb<2, 1>, k_absorb<2, 2>, k_absorb<2, 4>},
+                        {k_absorb<4, 1>, k_absorb<4, 2>, k_absorb<4, 4>},
+                        {k_absorb<8, 1>, k_absorb<8, 2>, k_absorb<8, 4>}};
+  const Fn fn = fns[rows == 8 ? 3 : rows == 4 ? 2 : rows == 2 ? 1 : 0][cols == 4 ? 2 : cols == 2 ? 1 : 0];
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_absorb)");
   fn<<<grid, 256, smem, stream>>>(a);
@@ -423,14 +486,18 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse,
                 RaggedMap{nullptr, nullptr, nullptr}};
   if (ragged) a.ragged = *ragged;
-  const int nch = (d_h + 31) / 32;
-  const int rows = rows_per_thread(H * nch, B);
+  int rows, cols;
+  pick_block(H, d_h, B, &rows, &cols, true, env_int("LLA_COMBINE_MAX_COLS", 1));
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(H, nch, (B + 8 * rows - 1) / (8 * rows));
+  cfg.gridDim = dim3(H, (d_h + 32 * cols - 1) / (32 * cols), (B + 8 * rows - 1) / (8 * rows));
   cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = ((size_t)32 * (r_v + 4) + (size_t)8 * rows * r_v) * sizeof(float);
-  void (*fn)(CombineArgs) = rows == 8 ? k_combine<8> : rows == 4 ? k_combine<4>
-                          : rows == 2 ? k_combine<2> : k_combine<1>;
+  cfg.dynamicSmemBytes = ((size_t)32 * cols * (r_v + 4) + (size_t)8 * rows * r_v) * sizeof(float);
+  using Fn = void (*)(CombineArgs);
+  const Fn fns[4][3] = {{k_combine<1, 1>, k_combine<1, 2>, k_combine<1, 4>},
+                        {k_combine<2, 1>, k_combine<2, 2>, k_combine<2, 4>},
+                        {k_combine<4, 1>, k_combine<4, 2>, k_combine<4, 4>},
+                        {k_combine<8, 1>, k_combine<8, 2>, k_combine<8, 4>}};
+  const Fn fn = fns[rows == 8 ? 3 : rows == 4 ? 2 : rows == 2 ? 1 : 0][cols == 4 ? 2 : cols == 2 ? 1 : 0];
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_combine)");
