@@ -129,3 +129,100 @@ def test_encode_rejects_bad_arguments_on_the_host():
     assert call(zgs=16) == _lib.LLA_ERR_INVALID_ARG        # groups overlap rows
     assert call(x=ctypes.c_void_p(0x100008)) == _lib.LLA_ERR_INVALID_ARG
     assert call(N=0) == _lib.LLA_ERR_INVALID_ARG
+
+
+FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: every call below fails on the host
+
+
+def test_paged_decode_rejects_bad_arguments_on_the_host():
+    h = lla.lib()
+
+    def call(**over):
+        args = dict(q=FAKE, zk=FAKE, zv=FAKE, zdt=1, B=2, H=2, d_h=16, r_k=8, r_v=8, ps=16,
+                    npages=4, bt=FAKE, maxb=2, sl=FAKE, sink=0, window=0, dk=FAKE, dv=FAKE,
+                    mu_k=None, mu_v=None, scale=0.25, out=FAKE, lse=None, ws=FAKE, ws_bytes=0,
+                    stream=None)
+        args.update(over)
+        return h.lla_decode_attn_paged(*args.values())
+
+    assert call(bt=None) == _lib.LLA_ERR_INVALID_ARG
+    assert call(sl=ctypes.c_void_p(0x100002)) == _lib.LLA_ERR_INVALID_ARG
+    assert call(ps=0) == _lib.LLA_ERR_INVALID_ARG
+    assert call(npages=0) == _lib.LLA_ERR_INVALID_ARG
+    assert call(maxb=0) == _lib.LLA_ERR_INVALID_ARG
+    assert call(ps=1 << 20, maxb=1 << 12) == _lib.LLA_ERR_INVALID_ARG  # 2^32 tokens
+    assert call(sink=-1) == _lib.LLA_ERR_INVALID_ARG
+    assert call(window=-1) == _lib.LLA_ERR_INVALID_ARG
+    assert call(r_k=12) == _lib.LLA_ERR_INVALID_ARG
+    need = lla.lla_decode_attn_paged_workspace(2, 2, 8, 8)
+    assert need > 0
+    assert call(ws_bytes=need - 16) == _lib.LLA_ERR_WORKSPACE
+    assert lla.lla_decode_attn_paged_workspace(0, 2, 8, 8) == 0
+
+
+def test_rope_decode_rejects_bad_arguments_on_the_host():
+    h = lla.lib()
+
+    def call(fn, **over):
+        args = dict(q=FAKE, qr=FAKE, zk=FAKE, zv=FAKE, zdt=1, B=2, H=16, d_h=128, d_r=64, N=8,
+                    n_cap=8, r_k=192, r_v=256, dk=FAKE, dv=FAKE, mu_k=None, mu_v=None,
+                    scale=0.1, out=FAKE, lse=None, ws=FAKE, ws_bytes=0, stream=None)
+        args.update(over)
+        return getattr(h, fn)(*args.values())
+
+    for fn in ("lla_decode_attn_rope", "lla2d_decode_attn_rope"):
+        assert call(fn, qr=None) == _lib.LLA_ERR_INVALID_ARG
+        assert call(fn, d_r=12) == _lib.LLA_ERR_INVALID_ARG
+        assert call(fn, d_r=0) == _lib.LLA_ERR_INVALID_ARG
+        assert call(fn, ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
+    # per-head: latent + rotary rows at most 256 bf16 wide
+    assert call("lla_decode_attn_rope", r_k=224) == _lib.LLA_ERR_INVALID_ARG
+    # LLA-2D: rows a multiple of 64 up to 384
+    assert call("lla2d_decode_attn_rope", r_k=200) == _lib.LLA_ERR_UNSUPPORTED
+    assert call("lla2d_decode_attn_rope", r_k=384) == _lib.LLA_ERR_UNSUPPORTED
+    assert call("lla2d_decode_attn_rope", r_k=320, ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
+    assert lla.lla2d_decode_attn_workspace(2, 16, 8, 384, 256) > 0
+    assert lla.lla2d_decode_attn_workspace(2, 16, 8, 448, 256) == 0
+
+
+def test_paged_lla2d_rejects_bad_arguments_on_the_host():
+    h = lla.lib()
+
+    def call(**over):
+        args = dict(q=FAKE, zk=FAKE, zv=FAKE, zdt=1, B=2, H=16, d_h=128, r_k=256, r_v=256,
+                    ps=256, npages=4, bt=FAKE, maxb=2, sl=FAKE, dk=FAKE, dv=FAKE, mu_k=None,
+                    mu_v=None, scale=0.1, out=FAKE, lse=None, ws=FAKE, ws_bytes=0, stream=None)
+        args.update(over)
+        return h.lla2d_decode_attn_paged(*args.values())
+
+    assert call(ps=64) == _lib.LLA_ERR_UNSUPPORTED       # pages hold whole 128-token tiles
+    assert call(ps=200) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(H=40) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(zdt=0, r_k=128, r_v=128) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(bt=None) == _lib.LLA_ERR_INVALID_ARG
+    assert call(npages=0) == _lib.LLA_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
+    assert lla.lla2d_decode_attn_paged_workspace(2, 16, 256, 256) > 0
+    assert lla.lla2d_decode_attn_paged_workspace(2, 16, 96, 256) == 0
+
+
+def test_encode_bias_entry_points_reject_bad_arguments_on_the_host():
+    h = lla.lib()
+    assert h.lla_encode_bias(None, FAKE, 2, 512, 16, FAKE, None) == _lib.LLA_ERR_INVALID_ARG
+    assert h.lla_encode_bias(FAKE, ctypes.c_void_p(0x100004), 2, 512, 16, FAKE, None) == \
+        _lib.LLA_ERR_INVALID_ARG                                     # mu not 16-byte aligned
+    assert h.lla_encode_bias(FAKE, FAKE, 2, 12, 16, FAKE, None) == _lib.LLA_ERR_INVALID_ARG
+
+    def call(**over):
+        args = dict(x=FAKE, xdt=1, T=4, N=10, G=2, d_loop=128, r=16, w=FAKE, muw=None, z=FAKE,
+                    zrs=16, zgs=160, ws=None, ws_bytes=0, stream=None)
+        args.update(over)
+        return h.lla_encode_with_bias(*args.values())
+
+    assert call(muw=ctypes.c_void_p(0x100004)) == _lib.LLA_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(0x100008)) == _lib.LLA_ERR_INVALID_ARG
+    assert call(d_loop=96) == _lib.LLA_ERR_INVALID_ARG
+    assert call(zgs=16) == _lib.LLA_ERR_INVALID_ARG
+    # split over K only where few tiles meet a long contraction
+    assert h.lla_encode_with_bias_workspace(4, 256, 1, 2048, 256) > 0
+    assert h.lla_encode_with_bias_workspace(4, 32768, 16, 128, 16) == 0
