@@ -32,7 +32,7 @@ LLA_DEVICE_BAD_PAGED_INPUT = 0x2
 # Every symbol include/lla.h declares.
 EXPORTS = (
     "lla_status_string", "lla_last_error", "lla_version", "lla_device_status",
-    "lla_set_timing_events",
+    "lla_selftest_wait_timeout", "lla_set_timing_events",
     "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
@@ -60,6 +60,7 @@ _SIGS = {
     "lla_version": ([], _c_int),
     "lla_device_status": ([ctypes.POINTER(ctypes.c_uint), _c_int], _c_int),
     "lla_set_timing_events": ([_vp, _vp], None),
+    "lla_selftest_wait_timeout": ([ctypes.c_uint, _vp], _c_int),
     "lla_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla_decode_attn_rope": ([_vp, _vp, _vp, _vp, _c_int] + [_c_int] * 8 + [_vp] * 4 +
                              [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),

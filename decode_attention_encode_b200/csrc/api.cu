@@ -200,6 +200,13 @@ lla_status lla_device_status(unsigned int* status, int clear) {
   return LLA_OK;
 }
 
+lla_status lla_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
+  g_last_error[0] = '\0';
+  if (timeout_us < 1 || timeout_us > 1000000)
+    return fail(LLA_ERR_INVALID_ARG, "timeout_us must be in 1..1000000");
+  return run_selftest_wait(timeout_us, static_cast<cudaStream_t>(stream));
+}
+
 size_t lla_decode_attn_workspace(int B, int H, int N, int r_k, int r_v) {
   if (B < 1 || H < 1 || N < 1 || r_k < 8 || r_v < 8 || r_k % 8 || r_v % 8) return 0;
   // The bf16 plan needs at least as much workspace as the fp32 one.

@@ -86,6 +86,9 @@ struct RaggedMap {
 
 size_t workspace_paged(int B, int H, int r_k, int r_v, int esz);
 
+// Launches the bounded-wait self-test (selftest.cu).
+lla_status run_selftest_wait(unsigned int timeout_us, cudaStream_t stream);
+
 // k_plan_paged: per-sequence records, prefix sums of the flattened range,
 // {total, share} and each worker's start (paged.cu). tile_tokens > 0 plans
 // LLA-2D: units are tiles of that many tokens, records {tiles, tokens}, and

@@ -78,6 +78,17 @@ LLA_API int lla_version(void);
 LLA_API lla_status lla_device_status(unsigned int *status, int clear);
 
 /*
+ * Self-test of the failure path of the bounded device waits. The paper has
+ * no counterpart; this exists so that tests can exercise the path without a
+ * fault. A one-thread kernel waits on a barrier that nothing arrives at,
+ * with the same bounded wait the decode and encode kernels use, gives up
+ * after timeout_us (1..1000000) microseconds and sets
+ * LLA_DEVICE_WAIT_TIMEOUT in the device status word. Read and clear it with
+ * lla_device_status.
+ */
+LLA_API lla_status lla_selftest_wait_timeout(unsigned int timeout_us, void *stream);
+
+/*
  * Timing hook for benchmarks and profilers. When both arguments are non-NULL
  * (cudaEvent_t handles passed as void*), every later lla_decode_attn,
  * lla_decode_attn_noalloc, lla2d_decode_attn or lla_encode call made on the

@@ -226,3 +226,9 @@ def test_encode_bias_entry_points_reject_bad_arguments_on_the_host():
     # split over K only where few tiles meet a long contraction
     assert h.lla_encode_with_bias_workspace(4, 256, 1, 2048, 256) > 0
     assert h.lla_encode_with_bias_workspace(4, 32768, 16, 128, 16) == 0
+
+
+def test_selftest_rejects_bad_timeouts_on_the_host():
+    h = lla.lib()
+    assert h.lla_selftest_wait_timeout(0, None) == _lib.LLA_ERR_INVALID_ARG
+    assert h.lla_selftest_wait_timeout(2000000, None) == _lib.LLA_ERR_INVALID_ARG
