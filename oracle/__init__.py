@@ -27,6 +27,8 @@ What is here, each in fp64:
     rotary branch), as attention over concatenated content and rotary keys;
     ``lla2d_decode_rope`` with the key row shared by every head.
   * ``paged2d_decode``: the same gather for the LLA-2D store.
+  * ``merge_attn``: the log-sum-exp merge of attention over disjoint parts
+    of a context (how a context split over GPUs recombines).
   * ``kept_positions`` / ``paged_decode``: the per-head decode over a paged
     store with per-sequence lengths (a gather of each unit's rows, then the
     explicit-reconstruction unit), with the attention-sink + window eviction
@@ -326,6 +328,25 @@ def lla2d_decode_rope(q, q_rope, zk, zv, dk, dv, mu_k=None, mu_v=None, scale=Non
             None if mu_v is None else np.asarray(mu_v)[h], scale)
     if full:
         return out.reshape(B, H, d), lse.reshape(B, H)
+    return out, lse
+
+
+def merge_attn(outs, lses):
+    """Merges attention results over disjoint parts of one context: with
+    L = ln sum_r exp(lse_r), out = sum_r exp(lse_r - L) out_r and lse = L.
+    Each part's out_r is its softmax-weighted value sum and lse_r its log
+    normaliser (the decode calls' outputs), so the merge is exact; a part
+    with lse_r = -inf (no token) has weight 0, and if every part is empty
+    the result is out = 0, lse = -inf. outs [R, ..., d], lses [R, ...]."""
+    outs, lses = _f64(outs), _f64(lses)
+    L = np.max(lses, axis=0)
+    finite = np.isfinite(L)
+    Ls = np.where(finite, L, 0.0)
+    w = np.where(np.isfinite(lses), np.exp(lses - Ls), 0.0)
+    tot = w.sum(axis=0)
+    lse = np.where(finite, Ls + np.log(np.where(finite, tot, 1.0)), -np.inf)
+    out = np.where(finite[..., None], (w[..., None] * outs).sum(axis=0) /
+                   np.where(finite, tot, 1.0)[..., None], 0.0)
     return out, lse
 
 

@@ -630,3 +630,28 @@ def test_lla2d_rope_is_per_head_rope_with_the_row_shared_by_every_head():
     o4, l4 = oracle.lla2d_decode(q, zk[:, :, :rk], zv, dk, dv, mk, mv)
     np.testing.assert_allclose(o3, o4, atol=1e-12)
     np.testing.assert_allclose(l3, l4, atol=1e-12)
+
+
+def test_merge_of_context_parts_equals_attention_over_the_whole():
+    # split the cached tokens into disjoint parts, attend each, merge
+    r = rng(81)
+    u = _unit(81, N=37)
+    q, zk, zv, dk, dv, mk, mv = (u[k] for k in ("q", "zk", "zv", "dk", "dv", "mu_k", "mu_v"))
+    full_o, full_l = oracle.decode_unit(q, zk, zv, dk, dv, mk, mv)
+    cuts = [0, 5, 6, 20, 37]
+    outs, lses = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, l = oracle.decode_unit(q, zk[a:b], zv[a:b], dk, dv, mk, mv)
+        outs.append(o)
+        lses.append(l)
+    # an empty part contributes nothing
+    outs.append(np.full_like(full_o, 123.0))
+    lses.append(-np.inf)
+    o, l = oracle.merge_attn(np.stack(outs), np.array(lses))
+    np.testing.assert_allclose(o, full_o, atol=1e-12)
+    assert abs(l - full_l) < 1e-12
+    # order of the parts does not matter; all-empty gives 0 / -inf
+    o2, l2 = oracle.merge_attn(np.stack(outs[::-1]), np.array(lses[::-1]))
+    np.testing.assert_allclose(o2, o, atol=1e-12)
+    oe, le = oracle.merge_attn(np.zeros((3, 4)), np.full(3, -np.inf))
+    assert np.all(oe == 0) and np.isneginf(le)
