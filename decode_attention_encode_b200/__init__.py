@@ -31,4 +31,5 @@ from ._lib import (  # noqa: F401
     lla_encode_bias,
     lla_encode_with_bias,
     lla_encode_with_bias_workspace_bytes,
+    lla_merge_attn,
 )

@@ -32,7 +32,7 @@ LLA_DEVICE_BAD_PAGED_INPUT = 0x2
 # Every symbol include/lla.h declares.
 EXPORTS = (
     "lla_status_string", "lla_last_error", "lla_version", "lla_device_status",
-    "lla_selftest_wait_timeout", "lla_set_timing_events",
+    "lla_selftest_wait_timeout", "lla_set_timing_events", "lla_merge_attn",
     "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
@@ -61,6 +61,7 @@ _SIGS = {
     "lla_device_status": ([ctypes.POINTER(ctypes.c_uint), _c_int], _c_int),
     "lla_set_timing_events": ([_vp, _vp], None),
     "lla_selftest_wait_timeout": ([ctypes.c_uint, _vp], _c_int),
+    "lla_merge_attn": ([_vp, _vp, _c_int, _c_ll, _c_int, _vp, _vp, _vp], _c_int),
     "lla_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla_decode_attn_rope": ([_vp, _vp, _vp, _vp, _c_int] + [_c_int] * 8 + [_vp] * 4 +
                              [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
@@ -459,3 +460,21 @@ def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_gro
                                     _ptr(workspace), ws_bytes, _stream(stream))
     _check(st)
     return z
+
+
+def lla_merge_attn(out_parts, lse_parts, out=None, lse=None, stream=None):
+    """Log-sum-exp merge of attention over disjoint context parts:
+    out_parts [R, ..., d], lse_parts [R, ...] fp32 on the device (each part
+    a decode call's (out, lse)). Returns (out [..., d], lse [...])."""
+    _need_cuda(out_parts, lse_parts, out, lse)
+    R, d = out_parts.shape[0], out_parts.shape[-1]
+    U = lse_parts[0].numel()
+    if out_parts[0].numel() != U * d:
+        raise LLAError(LLA_ERR_INVALID_ARG, "out_parts and lse_parts disagree on the units")
+    if out is None:
+        out = torch.empty(out_parts.shape[1:], device=out_parts.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty(lse_parts.shape[1:], device=out_parts.device, dtype=torch.float32)
+    _check(lib().lla_merge_attn(_ptr(out_parts), _ptr(lse_parts), R, U, d, _ptr(out), _ptr(lse),
+                                _stream(stream)))
+    return out, lse

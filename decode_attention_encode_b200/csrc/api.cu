@@ -200,6 +200,19 @@ lla_status lla_device_status(unsigned int* status, int clear) {
   return LLA_OK;
 }
 
+lla_status lla_merge_attn(const float* out_parts, const float* lse_parts, int R, long long U,
+                          int d, float* out, float* lse, void* stream) {
+  g_last_error[0] = '\0';
+  if (!out_parts || !lse_parts || !out)
+    return fail(LLA_ERR_INVALID_ARG, "out_parts, lse_parts and out must be non-NULL");
+  if (R < 1 || U < 1 || d < 1) return fail(LLA_ERR_INVALID_ARG, "R, U and d must be >= 1");
+  if ((U + 7) / 8 > 0x7fffffffLL) return fail(LLA_ERR_INVALID_ARG, "U too large");
+  if (!aligned(out_parts, 4) || !aligned(lse_parts, 4) || !aligned(out, 4) ||
+      (lse && !aligned(lse, 4)))
+    return fail(LLA_ERR_INVALID_ARG, "arrays must be 4-byte aligned");
+  return run_merge_attn(out_parts, lse_parts, R, U, d, out, lse, static_cast<cudaStream_t>(stream));
+}
+
 lla_status lla_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
   g_last_error[0] = '\0';
   if (timeout_us < 1 || timeout_us > 1000000)

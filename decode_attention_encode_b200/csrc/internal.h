@@ -86,6 +86,10 @@ struct RaggedMap {
 
 size_t workspace_paged(int B, int H, int r_k, int r_v, int esz);
 
+// Log-sum-exp merge of (out, lse) over R disjoint context parts (merge.cu).
+lla_status run_merge_attn(const float* outs, const float* lses, int R, long long U, int d,
+                          float* out, float* lse, cudaStream_t stream);
+
 // Launches the bounded-wait self-test (selftest.cu).
 lla_status run_selftest_wait(unsigned int timeout_us, cudaStream_t stream);
 

@@ -78,6 +78,24 @@ LLA_API int lla_version(void);
 LLA_API lla_status lla_device_status(unsigned int *status, int clear);
 
 /*
+ * Merge of attention results over disjoint parts of one context, for a
+ * context split across GPUs (each GPU decodes its part of a long sequence's
+ * latent store with any decode call above, the (out, lse) pairs are
+ * gathered, and this call combines them):
+ *   L = ln sum_r exp(lse_parts[r][u]),
+ *   out[u] = sum_r exp(lse_parts[r][u] - L) out_parts[r][u],  lse[u] = L.
+ * This is exact: each part's out is a convex combination of reconstructed
+ * values, and the weights renormalise the parts' softmax masses (§7's
+ * absorbed decode is a softmax over the union of the parts). A part with
+ * lse = -inf (no token) has weight 0; if all are, out = 0 and lse = -inf.
+ *   out_parts [R][U][d] fp32, lse_parts [R][U] fp32 (device); out [U][d];
+ *   lse [U] or NULL. R, U, d >= 1.
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla_merge_attn(const float *out_parts, const float *lse_parts,
+                                  int R, long long U, int d, float *out,
+                                  float *lse, void *stream);
+
+/*
  * Self-test of the failure path of the bounded device waits. The paper has
  * no counterpart; this exists so that tests can exercise the path without a
  * fault. A one-thread kernel waits on a barrier that nothing arrives at,
