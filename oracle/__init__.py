@@ -405,15 +405,16 @@ def paged_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=None
 
 
 def paged2d_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=None, mu_v=None,
-                   scale=None, nthreads: int = 0):
+                   scale=None, nthreads: int = 0, sink=0, window=0):
     """LLA-2D decode over a paged store with per-sequence lengths.
 
     zk_pages [P, page_size, r_k], zv_pages [P, page_size, r_v]: one latent
     per token shared by every head (§3 "The LLA-2D variant"); token j of
     sequence b is row j % page_size of page block_table[b, j // page_size].
-    Each sequence gathers its rows and goes through the LLA-2D explicit
-    reconstruction; an empty sequence gives out = 0, lse = -inf (the same
-    reading as ``paged_decode``). Returns out [B, H, d], lse [B, H]."""
+    Sequence b attends ``kept_positions(seq_lens[b], sink, window)`` (all
+    its tokens when window is 0): it gathers those rows and goes through the
+    LLA-2D explicit reconstruction; an empty set gives out = 0, lse = -inf
+    (the same reading as ``paged_decode``). Returns out [B, H, d], lse [B, H]."""
     q = np.asarray(q)
     B, H, d = q.shape
     zk_pages, zv_pages = np.asarray(zk_pages), np.asarray(zv_pages)
@@ -422,10 +423,9 @@ def paged2d_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=No
     out = np.zeros((B, H, d))
     lse = np.full((B, H), -np.inf)
     for b in range(B):
-        n = int(seq_lens[b])
-        if n == 0:
+        pos = kept_positions(int(seq_lens[b]), sink, window)
+        if pos.size == 0:
             continue
-        pos = np.arange(n)
         pages = block_table[b, pos // ps]
         zk = zk_pages[pages, pos % ps][None]
         zv = zv_pages[pages, pos % ps][None]

@@ -655,3 +655,32 @@ def test_merge_of_context_parts_equals_attention_over_the_whole():
     np.testing.assert_allclose(o2, o, atol=1e-12)
     oe, le = oracle.merge_attn(np.zeros((3, 4)), np.full(3, -np.inf))
     assert np.all(oe == 0) and np.isneginf(le)
+
+
+def test_paged2d_eviction_attends_exactly_the_kept_positions():
+    r = rng(91)
+    lens = [40, 9, 26, 0]
+    sink, window = 3, 6
+    B, H, d, ps, rk, rv = len(lens), 2, 8, 4, 8, 12
+    maxb = 10
+    npages = B * maxb
+    bt = np.arange(npages).reshape(B, maxb)
+    zkp = r.standard_normal((npages, ps, rk))
+    zvp = r.standard_normal((npages, ps, rv))
+    q = r.standard_normal((B, H, d))
+    dk, dv = r.standard_normal((H, d, rk)), r.standard_normal((H, d, rv))
+    out, lse = oracle.paged2d_decode(q, zkp, zvp, bt, lens, dk, dv, sink=sink, window=window)
+    for b, n in enumerate(lens):
+        pos = oracle.kept_positions(n, sink, window)
+        if pos.size == 0:
+            assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        zk = zkp[bt[b, pos // ps], pos % ps][None]
+        zv = zvp[bt[b, pos // ps], pos % ps][None]
+        ob, lb = oracle.lla2d_decode(q[b:b + 1], zk, zv, dk, dv)
+        np.testing.assert_allclose(out[b], ob[0], atol=1e-12)
+        np.testing.assert_allclose(lse[b], lb[0], atol=1e-12)
+    # no eviction when window is 0
+    o0, _ = oracle.paged2d_decode(q, zkp, zvp, bt, lens, dk, dv)
+    o1, _ = oracle.paged2d_decode(q, zkp, zvp, bt, lens, dk, dv, sink=5, window=0)
+    np.testing.assert_allclose(o0, o1, atol=0)
