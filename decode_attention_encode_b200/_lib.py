@@ -74,7 +74,8 @@ _SIGS = {
                                [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla2d_decode_attn_paged_workspace": ([_c_int] * 4, _c_size),
     "lla2d_decode_attn_paged": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp, _c_int, _vp] +
-                                [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
+                                [_c_int] * 2 + [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp],
+                                _c_int),
     "lla_decode_attn": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
                         [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla_decode_attn_noalloc": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp] * 4 +
@@ -359,8 +360,8 @@ def lla2d_decode_attn_paged_workspace(B, H, r_k, r_v):
 
 
 def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t,
-                            mu_k_t=None, mu_v_t=None, scale=None, out=None, lse=None,
-                            workspace=None, stream=None, want_lse=True):
+                            mu_k_t=None, mu_v_t=None, scale=None, sink=0, window=0, out=None,
+                            lse=None, workspace=None, stream=None, want_lse=True):
     """LLA-2D absorbed decode over a paged store: zk_pages [P,page_size,r_k],
     zv_pages [P,page_size,r_v] bf16 shared by every head, page_size a
     multiple of 128; block_table [B,max_blocks] and seq_lens [B] int32 on
@@ -385,7 +386,8 @@ def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, 
     st = h.lla2d_decode_attn_paged(_ptr(q), _ptr(zk_pages), _ptr(zv_pages),
                                    _dtype_code(zk_pages), B, H, d_h, r_k, r_v, page_size,
                                    num_pages, _ptr(block_table), max_blocks, _ptr(seq_lens),
-                                   _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t),
+                                   int(sink), int(window), _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t),
+                                   _ptr(mu_v_t),
                                    float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st)

@@ -369,10 +369,10 @@ size_t lla2d_decode_attn_paged_workspace(int B, int H, int r_k, int r_v) {
 lla_status lla2d_decode_attn_paged(const float* q, const void* zk_pages, const void* zv_pages,
                                    lla_dtype zdt, int B, int H, int d_h, int r_k, int r_v,
                                    int page_size, int num_pages, const int* block_table,
-                                   int max_blocks, const int* seq_lens, const float* dk_t,
-                                   const float* dv_t, const float* mu_k_t, const float* mu_v_t,
-                                   float scale, float* out, float* lse, void* workspace,
-                                   size_t ws_bytes, void* stream) {
+                                   int max_blocks, const int* seq_lens, int sink, int window,
+                                   const float* dk_t, const float* dv_t, const float* mu_k_t,
+                                   const float* mu_v_t, float scale, float* out, float* lse,
+                                   void* workspace, size_t ws_bytes, void* stream) {
   g_last_error[0] = '\0';
   int esz = 0;
   lla_status st = check_decode_args(q, zk_pages, zv_pages, zdt, B, H, d_h, 1, 1, r_k, r_v, dk_t,
@@ -392,9 +392,11 @@ lla_status lla2d_decode_attn_paged(const float* q, const void* zk_pages, const v
     return fail(LLA_ERR_INVALID_ARG, "num_pages and max_blocks must be >= 1");
   if ((long long)page_size * max_blocks > 0x7fffffffLL)
     return fail(LLA_ERR_INVALID_ARG, "page_size * max_blocks must fit in 31 bits");
+  if (sink < 0 || window < 0) return fail(LLA_ERR_INVALID_ARG, "sink and window must be >= 0");
   return run_decode_2d_paged(q, zk_pages, zv_pages, B, H, d_h, r_k, r_v, page_size, num_pages,
-                             block_table, max_blocks, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, scale,
-                             out, lse, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+                             block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t,
+                             mu_v_t, scale, out, lse, workspace, ws_bytes,
+                             static_cast<cudaStream_t>(stream));
 }
 
 lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,

@@ -106,9 +106,9 @@ size_t workspace_2d_paged(int B, int H, int r_k, int r_v);
 lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, int B, int H,
                                int d_h, int r_k, int r_v, int page_size, int num_pages,
                                const int* block_table, int max_blocks, const int* seq_lens,
-                               const float* dk, const float* dv, const float* mu_k,
-                               const float* mu_v, float scale, float* out, float* lse, void* ws,
-                               size_t ws_bytes, cudaStream_t stream);
+                               int sink, int window, const float* dk, const float* dv,
+                               const float* mu_k, const float* mu_v, float scale, float* out,
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
 lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int esz, int B, int H,
                             int d_h, int r_k, int r_v, int page_size, int num_pages,
                             const int* block_table, int max_blocks, const int* seq_lens, int sink,

@@ -66,11 +66,12 @@ struct D2Args {
   uint32_t tmem_cols;
   const unsigned char* qsw;  // per sequence: Q' as bf16 in the MMA operand layout
   // paged store (seqinfo non-null): written by k_plan_paged
-  const int4* seqinfo;      // [B] {tiles, tokens, 0, 0}
+  const int4* seqinfo;      // [B] {kept tiles, tokens, sink tiles, first window tile}
   const long long* plan;    // {total tiles, tiles per CTA}
   const int4* cstart;       // [grid] first (sequence, 0, tile) of each CTA
   const int* block_table;   // [B][max_blocks]
   int max_blocks, page_size;
+  int sink, window;         // eviction set (window 0: every token)
   float* part;
   int pstride;
   unsigned int* status;
@@ -118,12 +119,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// The (sequence b, tile j) a role is at, with sequence b's tile count nt and
-// token count n. Every role walks its CTA's tiles in order with its own
-// cursor: uniformly sized sequences (tps tiles of N tokens each) or the
-// ragged sequences of a paged plan.
+// The (sequence b, kept tile j) a role is at, with sequence b's kept tile
+// count nt, token count n, sink tiles st and first window tile fw (kept tile
+// j is tile j below st, tile fw + j - st from there), and its kept positions
+// [0, sk) and [ws, n). Every role walks its CTA's tiles in order with its
+// own cursor: uniformly sized sequences (tps tiles of N tokens each) or the
+// ragged, possibly evicted sequences of a paged plan.
 struct TileCur {
-  int b, j, nt, n;
+  int b, j, nt, n, st, fw, sk, ws;
 };
 
 __device__ __forceinline__ void tcur_load(TileCur& c, const D2Args& a) {
@@ -131,10 +134,28 @@ __device__ __forceinline__ void tcur_load(TileCur& c, const D2Args& a) {
     const int4 v = __ldg(a.seqinfo + c.b);
     c.nt = v.x;
     c.n = v.y;
+    c.st = v.z;
+    c.fw = v.w;
   } else {
-    c.nt = a.tps;
+    c.nt = c.st = c.fw = a.tps;
     c.n = a.N;
   }
+  if (a.window > 0 && c.n > a.sink + a.window) {
+    c.sk = a.sink;
+    c.ws = c.n - a.window;
+  } else {
+    c.sk = c.ws = c.n;
+  }
+}
+
+// first token position of the cursor's tile
+__device__ __forceinline__ int tcur_pos(const TileCur& c) {
+  return (c.j < c.st ? c.j : c.fw + c.j - c.st) * kRows;
+}
+
+// whether the token at `pos` of the cursor's sequence is attended
+__device__ __forceinline__ bool tcur_kept(const TileCur& c, int pos) {
+  return pos < c.n && (pos < c.sk || pos >= c.ws);
 }
 
 __device__ __forceinline__ TileCur tcur_start(const D2Args& a) {
@@ -235,20 +256,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pc_lt = 0, c_row = 0, c_z = 0, n_z = 0;
     auto place = [&]() {
       if (a.seqinfo) {
-        const int pos = pc.j * kRows;
+        const int pos = tcur_pos(pc);
         c_row = pos % a.page_size;
         c_z = n_z;
         TileCur nx = pc;
         tcur_next(nx, a);
         if (pc_lt + 1 < ntile)
-          n_z = __ldg(a.block_table + (size_t)nx.b * a.max_blocks + nx.j * kRows / a.page_size);
+          n_z = __ldg(a.block_table + (size_t)nx.b * a.max_blocks + tcur_pos(nx) / a.page_size);
       } else {
-        c_row = pc.j * kRows;
+        c_row = tcur_pos(pc);
         c_z = pc.b;
       }
     };
     if (a.seqinfo && ntile > 0)
-      n_z = __ldg(a.block_table + (size_t)pc.b * a.max_blocks + pc.j * kRows / a.page_size);
+      n_z = __ldg(a.block_table + (size_t)pc.b * a.max_blocks + tcur_pos(pc) / a.page_size);
     if (ntile > 0) place();
     auto tile_of = [&](int lt) {
       while (pc_lt < lt) {
@@ -456,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileCur cur = tcur_start(a);
     for (int lt = 0; lt < ntile; ++lt, tcur_next(cur, a)) {
       const int b = cur.b;
-      const int row0 = cur.j * kRows;
+      const int row0 = tcur_pos(cur);
       const bool first_of_seg = (lt == 0) || cur.j == 0;
       const bool last_of_seg = (lt == ntile - 1) || cur.j == cur.nt - 1;
       if (first_of_seg) {
@@ -487,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tl->s_empty[sb]));
 
-      const bool valid = row0 + row < cur.n;
+      const bool valid = tcur_kept(cur, row0 + row);
       bool need = false;
 #pragma unroll
       for (int h = 0; h < HP; ++h) need |= valid && h < a.H && s[h] > m[h] + kSlack;
@@ -680,7 +701,7 @@ struct Paged2D {
   long long* plan;
   const int4* cstart;
   const int* block_table;
-  int max_blocks, page_size;
+  int max_blocks, page_size, sink, window;
 };
 
 // Absorb, the tensor-core kernel and the merge, shared by the dense and the
@@ -729,6 +750,8 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
     a.block_table = pg->block_table;
     a.max_blocks = pg->max_blocks;
     a.page_size = pg->page_size;
+    a.sink = pg->sink;
+    a.window = pg->window;
   }
 
   auto kern = d.hp == 16 ? k_lla2d<16> : k_lla2d<32>;
@@ -824,9 +847,9 @@ size_t workspace_2d_paged(int B, int H, int r_k, int r_v) {
 lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, int B, int H,
                                int d_h, int r_k, int r_v, int page_size, int num_pages,
                                const int* block_table, int max_blocks, const int* seq_lens,
-                               const float* dk, const float* dv, const float* mu_k,
-                               const float* mu_v, float scale, float* out, float* lse, void* ws,
-                               size_t ws_bytes, cudaStream_t stream) {
+                               int sink, int window, const float* dk, const float* dv,
+                               const float* mu_k, const float* mu_v, float scale, float* out,
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
   D2PagedPlan pp;
   lla_status st = plan_2d_paged(B, H, r_k, r_v, &pp);
   if (st != LLA_OK) return st;
@@ -842,6 +865,8 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
   pg.block_table = block_table;
   pg.max_blocks = max_blocks;
   pg.page_size = page_size;
+  pg.sink = sink;
+  pg.window = window;
   // The pool read page by page: rows of a page, pages outermost.
   CUtensorMap tk, tv;
   {
@@ -857,9 +882,9 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
   // 1. plan: tiles of kRows tokens, one worker per CTA
-  st = launch_plan_paged(seq_lens, block_table, B, 1, page_size, num_pages, max_blocks, 0, 0,
-                         pp.d.grid, 1, kRows, const_cast<int4*>(pg.seqinfo), pg.cum, pg.plan,
-                         const_cast<int4*>(pg.cstart), stream);
+  st = launch_plan_paged(seq_lens, block_table, B, 1, page_size, num_pages, max_blocks, sink,
+                         window, pp.d.grid, 1, kRows, const_cast<int4*>(pg.seqinfo), pg.cum,
+                         pg.plan, const_cast<int4*>(pg.cstart), stream);
   if (st != LLA_OK) return st;
   return launch_2d(q, tk, tv, B, H, d_h, 0, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, pp.d,
                    wsb, &pg, stream);

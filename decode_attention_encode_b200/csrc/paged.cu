@@ -68,30 +68,40 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
   bool bad = false;
   for (int b = b0; b < b1; ++b) {
     const int N = p.seq_lens[b];
-    int n = 0, s = 0, gap = 0;
-    if (N >= 0 && N <= cap && p.tile_tokens > 0) {
-      // LLA-2D: {tiles, tokens}; every used page is checked
-      n = (N + p.tile_tokens - 1) / p.tile_tokens;
-      s = N;
-      if (!pages_ok(p, b, 0, N)) n = s = gap = -1;
-    } else if (N >= 0 && N <= cap) {
-      n = N;
-      s = N;
+    // per-head: {kept tokens n, sink part s, gap}; LLA-2D: {kept tiles n,
+    // tokens, sink tiles, first window tile}
+    int4 rec = make_int4(0, 0, 0, 0);
+    bool ok = N >= 0 && N <= cap;
+    if (ok && p.tile_tokens > 0) {
+      // The kept positions are [0, sk) and [ws, N); a tile is kept when it
+      // holds one, so the kept tiles are the sink tiles [0, st) and the
+      // window tiles [fw, ceil(N / T)).
+      const int T = p.tile_tokens;
+      int sk = N, ws = N;
+      if (p.window > 0 && N > p.sink + p.window) {
+        sk = p.sink;
+        ws = N - p.window;
+      }
+      const int st = (sk + T - 1) / T;
+      const int fw = max(ws / T, st);
+      rec = make_int4(st + max(0, (N + T - 1) / T - fw), N, st, fw);
+      ok = pages_ok(p, b, 0, sk) && pages_ok(p, b, ws, N);
+    } else if (ok) {
+      int n = N, s = N, gap = 0;
       if (p.window > 0 && N > p.sink + p.window) {
         n = p.sink + p.window;
         s = p.sink;
         gap = N - n;
       }
-      if (!pages_ok(p, b, 0, s) || !pages_ok(p, b, s + gap, N)) n = s = gap = -1;
-    } else {
-      n = s = gap = -1;
+      rec = make_int4(n, s, gap, 0);
+      ok = pages_ok(p, b, 0, s) && pages_ok(p, b, s + gap, N);
     }
-    if (n < 0) {
+    if (!ok) {
       bad = true;
-      n = s = gap = 0;
+      rec = make_int4(0, 0, 0, 0);
     }
-    p.seqinfo[b] = make_int4(n, s, gap, 0);
-    sum += (long long)n * p.H;
+    p.seqinfo[b] = rec;
+    sum += (long long)rec.x * p.H;
   }
   if (bad) report_status(p.status, kStatusBadPagedInput);
 

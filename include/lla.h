@@ -351,6 +351,10 @@ LLA_API lla_status lla2d_decode_attn_rope(const float *q, const float *q_rope,
  *             on the device as for lla_decode_attn_paged (a bad length or
  *             page index sets LLA_DEVICE_BAD_PAGED_INPUT and that sequence
  *             is treated as empty: out = 0, lse = -inf).
+ *   sink, window  the eviction set of lla_decode_attn_paged (window 0: every
+ *             token). The tensor cores read the 128-token tiles that hold a
+ *             kept token and weight the others' rows by zero; only the pages
+ *             of kept tokens are read or checked.
  *   workspace lla2d_decode_attn_paged_workspace(B, H, r_k, r_v) bytes.
  * Rows of a sequence's last page past its length are read (the tensor
  * cores take whole 128-token tiles) and weighted by zero: they must hold
@@ -364,11 +368,12 @@ LLA_API lla_status lla2d_decode_attn_paged(const float *q, const void *zk_pages,
                                            int B, int H, int d_h, int r_k, int r_v,
                                            int page_size, int num_pages,
                                            const int *block_table, int max_blocks,
-                                           const int *seq_lens, const float *dk_t,
-                                           const float *dv_t, const float *mu_k_t,
-                                           const float *mu_v_t, float scale,
-                                           float *out, float *lse, void *workspace,
-                                           size_t ws_bytes, void *stream);
+                                           const int *seq_lens, int sink, int window,
+                                           const float *dk_t, const float *dv_t,
+                                           const float *mu_k_t, const float *mu_v_t,
+                                           float scale, float *out, float *lse,
+                                           void *workspace, size_t ws_bytes,
+                                           void *stream);
 
 /* --------------------------------------------------------------------------
  * Latent write (§3 Eq. 2 over the loop-major stack of Eq. 1):

@@ -190,8 +190,9 @@ def test_paged_lla2d_rejects_bad_arguments_on_the_host():
 
     def call(**over):
         args = dict(q=FAKE, zk=FAKE, zv=FAKE, zdt=1, B=2, H=16, d_h=128, r_k=256, r_v=256,
-                    ps=256, npages=4, bt=FAKE, maxb=2, sl=FAKE, dk=FAKE, dv=FAKE, mu_k=None,
-                    mu_v=None, scale=0.1, out=FAKE, lse=None, ws=FAKE, ws_bytes=0, stream=None)
+                    ps=256, npages=4, bt=FAKE, maxb=2, sl=FAKE, sink=0, window=0, dk=FAKE,
+                    dv=FAKE, mu_k=None, mu_v=None, scale=0.1, out=FAKE, lse=None, ws=FAKE,
+                    ws_bytes=0, stream=None)
         args.update(over)
         return h.lla2d_decode_attn_paged(*args.values())
 
@@ -201,6 +202,7 @@ def test_paged_lla2d_rejects_bad_arguments_on_the_host():
     assert call(zdt=0, r_k=128, r_v=128) == _lib.LLA_ERR_UNSUPPORTED
     assert call(bt=None) == _lib.LLA_ERR_INVALID_ARG
     assert call(npages=0) == _lib.LLA_ERR_INVALID_ARG
+    assert call(window=-1) == _lib.LLA_ERR_INVALID_ARG
     assert call(ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
     assert lla.lla2d_decode_attn_paged_workspace(2, 16, 256, 256) > 0
     assert lla.lla2d_decode_attn_paged_workspace(2, 16, 96, 256) == 0

@@ -34,20 +34,21 @@ def make(lens, H, d_h, r_k, r_v, page_size, mu=False, seed=0, spare=2):
                 seq_lens=torch.tensor(np.asarray(lens, dtype=np.int32), device="cuda"))
 
 
-def run(inp):
+def run(inp, sink=0, window=0):
     return lla.lla2d_decode_attn_paged(inp["q"], inp["zk"], inp["zv"], inp["block_table"],
                                        inp["seq_lens"], inp["dk"], inp["dv"], inp["mu_k"],
-                                       inp["mu_v"])
+                                       inp["mu_v"], sink=sink, window=window)
 
 
-def reference(inp, pick=None):
+def reference(inp, pick=None, sink=0, window=0):
     import oracle  # test infrastructure only
     opt = lambda t: None if t is None else to_f64(t)
     sel = slice(None) if pick is None else pick
     return oracle.paged2d_decode(to_f64(inp["q"][sel]), to_f64(inp["zk"]), to_f64(inp["zv"]),
                                  inp["block_table"][sel].cpu().numpy().astype(np.int64),
                                  inp["seq_lens"][sel].cpu().numpy(), to_f64(inp["dk"]),
-                                 to_f64(inp["dv"]), opt(inp["mu_k"]), opt(inp["mu_v"]))
+                                 to_f64(inp["dv"]), opt(inp["mu_k"]), opt(inp["mu_v"]),
+                                 sink=sink, window=window)
 
 
 def compare(out, lse, ref_out, ref_lse, lens):
@@ -136,3 +137,26 @@ def test_full_size_ragged_32x_batch_sampled():
     pick = [0, 1, 127, 255]
     ref_out, ref_lse = reference(inp, pick)
     compare(out[pick], lse[pick], ref_out, ref_lse, lens[pick])
+
+
+@pytest.mark.parametrize("sink, window, page_size", [(4, 256, 256), (0, 300, 128), (130, 1, 128),
+                                                     (4, 5000, 256)])
+def test_sink_window_eviction(sink, window, page_size):
+    import oracle  # test infrastructure only
+    lens = [3000, 260, 261, 1, 0, 9000, 257, 700]
+    inp = make(lens, 16, 128, 256, 256, page_size, mu=True, seed=sink + window)
+    # pages holding no kept token: invalid table entries and NaN latents
+    bt = inp["block_table"].cpu().numpy()
+    for b, n in enumerate(lens):
+        kept_blocks = set((oracle.kept_positions(n, sink, window) // page_size).tolist())
+        for blk in range((n + page_size - 1) // page_size):
+            if blk not in kept_blocks:
+                inp["zk"][int(bt[b, blk])] = float("nan")
+                inp["zv"][int(bt[b, blk])] = float("nan")
+                bt[b, blk] = -7
+    inp["block_table"] = torch.from_numpy(bt).cuda()
+    out, lse = run(inp, sink, window)
+    torch.cuda.synchronize()
+    assert lla.device_status() == 0
+    assert torch.isfinite(out).all()
+    compare(out, lse, *reference(inp, sink=sink, window=window), lens)
