@@ -624,6 +624,11 @@ def run_lla(args, world, rank, local):
         q_dev = torch.empty_like(wl.q)
         qr_host = wl.q_rope.to("cpu").pin_memory() if wl.rope else None
         qr_dev = torch.empty_like(wl.q_rope) if wl.rope else None
+        # a paged store's per-step inputs: lengths and block table (a serving
+        # loop grows them every step); the decode calls read the device copies
+        pg_hosts = [wl.seq_lens.to("cpu").pin_memory(), wl.block_table.to("cpu").pin_memory()] \
+            if wl.paged else []
+        pg_devs = [wl.seq_lens, wl.block_table] if wl.paged else []
         x_hosts = [wl.xk.to("cpu").pin_memory(), wl.xv.to("cpu").pin_memory()] \
             if wl.write_latents else []
         x_devs = [torch.empty_like(wl.xk), torch.empty_like(wl.xv)] if wl.write_latents else []
@@ -636,6 +641,8 @@ def run_lla(args, world, rank, local):
         def e2e_step():
             with torch.cuda.stream(h2d):
                 h2d.wait_stream(stream)  # buffers of the previous step are free
+                for d_, h_ in zip(pg_devs, pg_hosts):
+                    d_.copy_(h_, non_blocking=True)
                 for t in range(c.T):
                     for l in range(c.L):
                         q_dev[l, t].copy_(q_host[l, t], non_blocking=True)
@@ -673,7 +680,8 @@ def run_lla(args, world, rank, local):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
         e2e = {"value": aggregate_rate(tokens_per_step, e2e_ms, world), "unit": UNIT,
                "h2d_bytes_per_step": (q_host.numel() + (qr_host.numel() if wl.rope else 0)) * 4
-                                     + sum(h_.numel() * 2 for h_ in x_hosts),
+                                     + sum(h_.numel() * 2 for h_ in x_hosts)
+                                     + sum(h_.numel() * 4 for h_ in pg_hosts),
                "d2h_bytes_per_step": (out_host.numel() + lse_host.numel()) * 4,
                "copies": "pinned host memory, per-call chunks on separate copy streams"}
 
