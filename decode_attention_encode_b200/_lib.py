@@ -364,7 +364,7 @@ def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, 
                             lse=None, workspace=None, stream=None, want_lse=True):
     """LLA-2D absorbed decode over a paged store: zk_pages [P,page_size,r_k],
     zv_pages [P,page_size,r_v] bf16 shared by every head, page_size a
-    multiple of 128; block_table [B,max_blocks] and seq_lens [B] int32 on
+    multiple of 64; block_table [B,max_blocks] and seq_lens [B] int32 on
     the device. Returns (out [B,H,d_h], lse [B,H] or None)."""
     _need_cuda(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, out,
                lse, workspace)

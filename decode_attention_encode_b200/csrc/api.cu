@@ -386,8 +386,8 @@ lla_status lla2d_decode_attn_paged(const float* q, const void* zk_pages, const v
     return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be non-NULL");
   if (!aligned(block_table, 4) || !aligned(seq_lens, 4))
     return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be 4-byte aligned");
-  if (page_size < 128 || page_size % 128)
-    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D pages hold a positive multiple of 128 tokens");
+  if (page_size < 64 || page_size % 64)
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D pages hold a positive multiple of 64 tokens");
   if (num_pages < 1 || max_blocks < 1)
     return fail(LLA_ERR_INVALID_ARG, "num_pages and max_blocks must be >= 1");
   if ((long long)page_size * max_blocks > 0x7fffffffLL)

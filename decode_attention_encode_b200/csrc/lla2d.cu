@@ -183,7 +183,7 @@ __device__ __forceinline__ void tcur_next(TileCur& c, const D2Args& a) {
   }
 }
 
-template <int HP>
+template <int HP, int NSUB>
 __global__ void __launch_bounds__(kThreads, 1)
     k_lla2d(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
             D2Args a) {
@@ -249,27 +249,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     const CUtensorMap* map = is_k ? &tk : &tv;
     const int total = ntile * ng;
     // Cursor at the tile of the next group to load, and that tile's TMA
-    // row and third coordinate: (row, sequence) in the dense store, (row in
-    // page, page) in a paged pool, whose block-table entry for the next
-    // tile is loaded one tile ahead.
+    // rows and third coordinates: (row, sequence) in the dense store, (row
+    // in page, page) in a paged pool. Pages of a multiple of 128 tokens hold
+    // whole tiles; pages of an odd multiple of 64 give each 64-row half of a
+    // tile its own page, and a half that holds no kept token is zero-filled
+    // in shared memory instead of read (its page may be unallocated or
+    // evicted). The block-table entries of the next tile are loaded one tile
+    // ahead.
     TileCur pc = tcur_start(a);
-    int pc_lt = 0, c_row = 0, c_z = 0, n_z = 0;
+    constexpr int kSubRows = kRows / NSUB, kSubBytes = kBoxBytes / NSUB;
+    int pc_lt = 0;
+    int c_row[NSUB], c_z[NSUB], n_z[NSUB];
+#pragma unroll
+    for (int sb = 0; sb < NSUB; ++sb) c_row[sb] = c_z[sb] = n_z[sb] = 0;
+    // page of rows [pos, pos + kSubRows) of the cursor's tile; whole-tile
+    // boxes always hold a kept token, halves may not (-1: not read)
+    auto lookup = [&](const TileCur& c, int sb) -> int {
+      const int p0 = tcur_pos(c) + sb * kSubRows;
+      const int* row = a.block_table + (size_t)c.b * a.max_blocks;
+      if (NSUB == 1) return __ldg(row + p0 / a.page_size);
+      const bool kept = p0 < c.sk || (p0 < c.n && p0 + kSubRows > c.ws);
+      return kept ? __ldg(row + p0 / a.page_size) : -1;
+    };
     auto place = [&]() {
       if (a.seqinfo) {
         const int pos = tcur_pos(pc);
-        c_row = pos % a.page_size;
-        c_z = n_z;
+#pragma unroll
+        for (int sb = 0; sb < NSUB; ++sb) {
+          c_row[sb] = (pos + sb * kSubRows) % a.page_size;
+          c_z[sb] = n_z[sb];
+        }
         TileCur nx = pc;
         tcur_next(nx, a);
-        if (pc_lt + 1 < ntile)
-          n_z = __ldg(a.block_table + (size_t)nx.b * a.max_blocks + tcur_pos(nx) / a.page_size);
+        if (pc_lt + 1 < ntile) {
+#pragma unroll
+          for (int sb = 0; sb < NSUB; ++sb) n_z[sb] = lookup(nx, sb);
+        }
       } else {
-        c_row = tcur_pos(pc);
-        c_z = pc.b;
+        c_row[0] = tcur_pos(pc);
+        c_z[0] = pc.b;
       }
     };
-    if (a.seqinfo && ntile > 0)
-      n_z = __ldg(a.block_table + (size_t)pc.b * a.max_blocks + tcur_pos(pc) / a.page_size);
+    if (a.seqinfo && ntile > 0) {
+#pragma unroll
+      for (int sb = 0; sb < NSUB; ++sb) n_z[sb] = lookup(pc, sb);
+    }
     if (ntile > 0) place();
     auto tile_of = [&](int lt) {
       while (pc_lt < lt) {
@@ -286,13 +310,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) return false;
       const int lt = it / ng, grp = it - lt * ng;
       tile_of(lt);
+      const uint32_t dst = ring + (uint32_t)s * kStageBytes;
+      const int nb = is_k ? kboxes(grp) : 2;
+      int loaded = NSUB;
+      if (NSUB > 1) {
+        // a half with no kept token: zeros (generic stores, made visible to
+        // the tensor cores before the stage is announced full)
+        bool zeroed = false;
+#pragma unroll
+        for (int sb = 0; sb < NSUB; ++sb) {
+          if (c_z[sb] >= 0) continue;
+          --loaded;
+          zeroed = true;
+          for (int x = 0; x < nb; ++x) {
+            uint4* z = reinterpret_cast<uint4*>(smem + (dst - s_kring) + x * kBoxBytes +
+                                                sb * kSubBytes);
+            for (int k = lane; k < kSubBytes / 16; k += 32) z[k] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        if (zeroed) fence_proxy_async_smem();
+        __syncwarp();
+      }
       if (lane == 0) {
         const uint32_t full = smem_u32(&fullb[s]);
-        const uint32_t dst = ring + (uint32_t)s * kStageBytes;
-        const int nb = is_k ? kboxes(grp) : 2;
-        mbar_arrive_expect_tx(full, nb * kBoxBytes);
-        for (int x = 0; x < nb; ++x)
-          tma_load_3d(dst + x * kBoxBytes, map, grp * 128 + x * 64, c_row, c_z, full, pol);
+        mbar_arrive_expect_tx(full, (uint32_t)(nb * loaded * kSubBytes));
+        for (int x = 0; x < nb; ++x) {
+#pragma unroll
+          for (int sb = 0; sb < NSUB; ++sb)
+            if (NSUB == 1 || c_z[sb] >= 0)
+              tma_load_3d(dst + x * kBoxBytes + sb * kSubBytes, map, grp * 128 + x * 64,
+                          c_row[sb], c_z[sb], full, pol);
+        }
       }
       return true;
     };
@@ -754,7 +802,10 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
     a.window = pg->window;
   }
 
-  auto kern = d.hp == 16 ? k_lla2d<16> : k_lla2d<32>;
+  // pages of an odd multiple of 64 tokens: each tile half from its own page
+  const bool split = pg && pg->page_size % kRows;
+  auto kern = d.hp == 16 ? (split ? k_lla2d<16, 2> : k_lla2d<16, 1>)
+                         : (split ? k_lla2d<32, 2> : k_lla2d<32, 1>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_lla2d)");
   cudaLaunchAttribute pdl[1];
@@ -867,18 +918,20 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
   pg.page_size = page_size;
   pg.sink = sink;
   pg.window = window;
-  // The pool read page by page: rows of a page, pages outermost.
+  // The pool read page by page: rows of a page, pages outermost; boxes of
+  // 64 rows when pages hold an odd multiple of 64 tokens.
+  const uint32_t box_rows = page_size % kRows ? kRows / 2 : kRows;
   CUtensorMap tk, tv;
   {
     const uint64_t dims[3] = {(uint64_t)r_k, (uint64_t)page_size, (uint64_t)num_pages};
     const uint64_t strides[2] = {(uint64_t)r_k * 2, (uint64_t)page_size * r_k * 2};
-    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    const uint32_t box[3] = {64, box_rows, 1};
     if (!make_tmap_bf16(&tk, zk, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
   {
     const uint64_t dims[3] = {(uint64_t)r_v, (uint64_t)page_size, (uint64_t)num_pages};
     const uint64_t strides[2] = {(uint64_t)r_v * 2, (uint64_t)page_size * r_v * 2};
-    const uint32_t box[3] = {64, (uint32_t)kRows, 1};
+    const uint32_t box[3] = {64, box_rows, 1};
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
   // 1. plan: tiles of kRows tokens, one worker per CTA

@@ -212,4 +212,8 @@ C2_ROPE = DecodeConfig("perhead_4x_rope", L=24, T=4, H=16, d_h=128, r_k=128, r_v
 # tokens in a pool of 256-token pages
 C4_PAGED = DecodeConfig("lla2d_32x_paged", L=24, T=4, H=16, d_h=128, r_k=256, r_v=256, B=256,
                         N=8192, dtype="bf16", decay=True, two_d=True, page_size=256, spread=0.5)
-DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE, C4_PAGED)}
+# the same batch in 64-token pages: every 128-token tile spans two pages
+C4_PAGED64 = DecodeConfig("lla2d_32x_paged64", L=24, T=4, H=16, d_h=128, r_k=256, r_v=256, B=256,
+                          N=8192, dtype="bf16", decay=True, two_d=True, page_size=64, spread=0.5)
+DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE, C4_PAGED,
+                                      C4_PAGED64)}

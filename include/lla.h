@@ -345,20 +345,23 @@ LLA_API lla_status lla2d_decode_attn_rope(const float *q, const float *q_rope,
  *   zk_pages [num_pages][page_size][r_k], zv_pages [num_pages][page_size][r_v]
  *             bf16: token j of sequence b is row j % page_size of page
  *             block_table[b][j / page_size]. 16-byte aligned.
- *   page_size a positive multiple of 128 (a 128-token tile never spans two
- *             pages); num_pages, max_blocks >= 1.
+ *   page_size a positive multiple of 64; num_pages, max_blocks >= 1. With
+ *             a multiple of 128 a 128-token tile lies in one page; otherwise
+ *             each 64-token half of a tile is read from its own page.
  *   block_table [B][max_blocks], seq_lens [B]: int32 device arrays, checked
  *             on the device as for lla_decode_attn_paged (a bad length or
  *             page index sets LLA_DEVICE_BAD_PAGED_INPUT and that sequence
  *             is treated as empty: out = 0, lse = -inf).
  *   sink, window  the eviction set of lla_decode_attn_paged (window 0: every
- *             token). The tensor cores read the 128-token tiles that hold a
+ *             token). The tensor cores take the 128-token tiles that hold a
  *             kept token and weight the others' rows by zero; only the pages
- *             of kept tokens are read or checked.
+ *             of kept tokens are read or checked (with 64-token pages a tile
+ *             half that holds no kept token is zero-filled, not read).
  *   workspace lla2d_decode_attn_paged_workspace(B, H, r_k, r_v) bytes.
- * Rows of a sequence's last page past its length are read (the tensor
- * cores take whole 128-token tiles) and weighted by zero: they must hold
- * finite values, as a zero-initialised pool does. Other limits as
+ * Rows of a page that holds a kept token but are themselves past the
+ * length or evicted may be read (the tensor cores take whole 64- or
+ * 128-token boxes) and are weighted by zero: they must hold finite values,
+ * as a zero-initialised pool does. Other limits as
  * lla2d_decode_attn.
  * -------------------------------------------------------------------------- */
 LLA_API size_t lla2d_decode_attn_paged_workspace(int B, int H, int r_k, int r_v);

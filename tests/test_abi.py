@@ -196,7 +196,7 @@ def test_paged_lla2d_rejects_bad_arguments_on_the_host():
         args.update(over)
         return h.lla2d_decode_attn_paged(*args.values())
 
-    assert call(ps=64) == _lib.LLA_ERR_UNSUPPORTED       # pages hold whole 128-token tiles
+    assert call(ps=32) == _lib.LLA_ERR_UNSUPPORTED       # pages hold whole 64-token boxes
     assert call(ps=200) == _lib.LLA_ERR_UNSUPPORTED
     assert call(H=40) == _lib.LLA_ERR_UNSUPPORTED
     assert call(zdt=0, r_k=128, r_v=128) == _lib.LLA_ERR_UNSUPPORTED

@@ -2,7 +2,8 @@
 against the fp64 oracle, through the C ABI.
 
 Cases: ragged length mixes around the 128-token tile (0, 1, 127, 128, 129,
-page boundaries), page sizes 128 and 256, shuffled pools, more sequences
+page boundaries), page sizes 64, 128, 192 and 256 (64-token pages split
+a tile over two pages), shuffled pools, more sequences
 than CTAs and sequences spread over many CTAs, device-side rejection of bad
 lengths and page indices, agreement with the dense kernel on a
 dense-equivalent layout, and the 32x geometry as a ragged serving batch."""
@@ -63,7 +64,7 @@ def compare(out, lse, ref_out, ref_lse, lens):
     return err
 
 
-@pytest.mark.parametrize("page_size", [128, 256])
+@pytest.mark.parametrize("page_size", [64, 128, 192, 256])
 def test_ragged_lengths_around_the_tile(page_size):
     lens = [1, 127, 128, 129, 0, 255, 256, 257, 1000, 3]
     inp = make(lens, 16, 128, 256, 256, page_size, mu=True, seed=page_size)
@@ -140,7 +141,8 @@ def test_full_size_ragged_32x_batch_sampled():
 
 
 @pytest.mark.parametrize("sink, window, page_size", [(4, 256, 256), (0, 300, 128), (130, 1, 128),
-                                                     (4, 5000, 256)])
+                                                     (4, 5000, 256), (4, 256, 64), (4, 230, 64),
+                                                     (70, 100, 192), (0, 300, 192), (130, 1, 64)])
 def test_sink_window_eviction(sink, window, page_size):
     import oracle  # test infrastructure only
     lens = [3000, 260, 261, 1, 0, 9000, 257, 700]
@@ -160,3 +162,34 @@ def test_sink_window_eviction(sink, window, page_size):
     assert lla.device_status() == 0
     assert torch.isfinite(out).all()
     compare(out, lse, *reference(inp, sink=sink, window=window), lens)
+
+
+@pytest.mark.parametrize("H, r_k, r_v", [(32, 192, 128), (8, 64, 256)])
+def test_64_token_pages_heads_and_ranks(H, r_k, r_v):
+    # every tile half from its own shuffled page; key rows of one and three boxes
+    lens = [64, 65, 128, 1, 191, 640, 333]
+    inp = make(lens, H, 64, r_k, r_v, 64, mu=True, seed=H + r_v)
+    out, lse = run(inp)
+    torch.cuda.synchronize()
+    assert lla.device_status() == 0
+    compare(out, lse, *reference(inp), lens)
+
+
+def test_64_token_pages_never_read_past_the_length():
+    # a tile half wholly past a sequence's length is zero-filled, not read:
+    # its table entry names a NaN-filled spare page
+    lens = [64, 192, 320]
+    inp = make(lens, 16, 128, 256, 256, 64, mu=True, seed=21, spare=1)
+    bt = inp["block_table"].cpu().numpy()
+    used = set(bt[bt >= 0].tolist())
+    poison = next(p for p in range(inp["zk"].shape[0]) if p not in used)
+    inp["zk"][poison] = float("nan")
+    inp["zv"][poison] = float("nan")
+    bt[bt < 0] = poison
+    assert (bt == poison).sum() == 6
+    inp["block_table"] = torch.from_numpy(bt).cuda()
+    out, lse = run(inp)
+    torch.cuda.synchronize()
+    assert lla.device_status() == 0
+    assert torch.isfinite(out).all()
+    compare(out, lse, *reference(inp), lens)
