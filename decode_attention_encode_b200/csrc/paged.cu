@@ -44,29 +44,29 @@ struct PlanArgs {
 };
 
 // Every page index the kept positions [lo, hi) of sequence b touch lies in
-// the pool.
-__device__ bool pages_ok(const PlanArgs& p, int b, int lo, int hi) {
+// the pool. The warp's lanes check the pages together, so a long sequence in
+// small pages (hundreds of table entries) costs a few round trips.
+__device__ bool pages_ok(const PlanArgs& p, int b, int lo, int hi, int lane) {
   if (lo >= hi) return true;
   const int* row = p.block_table + (size_t)b * p.max_blocks;
-  for (int blk = lo / p.page_size; blk <= (hi - 1) / p.page_size; ++blk) {
-    const int pg = row[blk];
-    if (pg < 0 || pg >= p.num_pages) return false;
+  bool bad = false;
+  for (int blk = lo / p.page_size + lane; blk <= (hi - 1) / p.page_size; blk += 32) {
+    const int pg = __ldg(row + blk);
+    bad |= pg < 0 || pg >= p.num_pages;
   }
-  return true;
+  return !__any_sync(0xffffffffu, bad);
 }
 
 __global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
   __shared__ long long scan[kPlanThreads];
   __shared__ long long s_total, s_P;
-  const int t = threadIdx.x;
-  const int chunk = (p.B + kPlanThreads - 1) / kPlanThreads;
-  const int b0 = min(p.B, t * chunk), b1 = min(p.B, b0 + chunk);
+  const int t = threadIdx.x, lane = t & 31;
   const long long cap = (long long)p.max_blocks * p.page_size;
 
-  // 1. per-sequence records; a sequence with a bad length or page is empty
-  long long sum = 0;
+  // 1. per-sequence records, one warp per sequence; a sequence with a bad
+  //    length or page is empty
   bool bad = false;
-  for (int b = b0; b < b1; ++b) {
+  for (int b = t >> 5; b < p.B; b += kPlanThreads / 32) {
     const int N = p.seq_lens[b];
     // per-head: {kept tokens n, sink part s, gap}; LLA-2D: {kept tiles n,
     // tokens, sink tiles, first window tile}
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
       const int st = (sk + T - 1) / T;
       const int fw = max(ws / T, st);
       rec = make_int4(st + max(0, (N + T - 1) / T - fw), N, st, fw);
-      ok = pages_ok(p, b, 0, sk) && pages_ok(p, b, ws, N);
+      ok = pages_ok(p, b, 0, sk, lane) && pages_ok(p, b, ws, N, lane);
     } else if (ok) {
       int n = N, s = N, gap = 0;
       if (p.window > 0 && N > p.sink + p.window) {
@@ -94,16 +94,21 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
         gap = N - n;
       }
       rec = make_int4(n, s, gap, 0);
-      ok = pages_ok(p, b, 0, s) && pages_ok(p, b, s + gap, N);
+      ok = pages_ok(p, b, 0, s, lane) && pages_ok(p, b, s + gap, N, lane);
     }
     if (!ok) {
       bad = true;
       rec = make_int4(0, 0, 0, 0);
     }
-    p.seqinfo[b] = rec;
-    sum += (long long)rec.x * p.H;
+    if (lane == 0) p.seqinfo[b] = rec;
   }
-  if (bad) report_status(p.status, kStatusBadPagedInput);
+  if (bad && lane == 0) report_status(p.status, kStatusBadPagedInput);
+  __syncthreads();
+
+  const int chunk = (p.B + kPlanThreads - 1) / kPlanThreads;
+  const int b0 = min(p.B, t * chunk), b1 = min(p.B, b0 + chunk);
+  long long sum = 0;
+  for (int b = b0; b < b1; ++b) sum += (long long)p.seqinfo[b].x * p.H;
 
   // 2. prefix sums of the flattened (sequence, head, token) range
   scan[t] = sum;
