@@ -439,6 +439,418 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Tensor-core forms of k_absorb and k_combine (bf16 latents)
+// ---------------------------------------------------------------------------
+// Both kernels are small GEMMs per head (q' = q W^K, out = W^V ubar) that the
+// CUDA-core forms above spend most of their time on as FFMA chains. Here the
+// contraction runs on warp-level bf16 tensor-core MMAs (m16n8k16, fp32
+// accumulate). Each fp32 operand x is split as hi = bf16(x), lo = bf16(x - hi)
+// (x - hi is exact in fp32) and the product is hi.hi + hi.lo + lo.hi; the
+// dropped lo.lo term and the split's residue are below 2^-16 of each product,
+// far under the bf16 rounding the latents and the LLA-2D query already carry.
+// Accumulators stay in registers: no tensor memory is allocated, so these
+// kernels never contend with the programmatically overlapped k_lla2d for it.
+//
+// Operands are staged row by row as [row][k] bf16 with a pitch of kp + 8
+// elements (kp = k padded to 16). A pitch of kp/2 + 4 words makes the eight
+// rows of a fragment load start 4*(odd) banks apart, so the 32 lanes of every
+// fragment load hit 32 distinct banks.
+
+// hi and lo bf16 parts of four consecutive fp32 values, as 8-byte stores
+__device__ __forceinline__ void store_split4(__nv_bfloat16* hi, __nv_bfloat16* lo, float4 v) {
+  const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 h23 = __floats2bfloat162_rn(v.z, v.w);
+  const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+  const __nv_bfloat162 l01 = __floats2bfloat162_rn(v.x - f01.x, v.y - f01.y);
+  const __nv_bfloat162 l23 = __floats2bfloat162_rn(v.z - f23.x, v.w - f23.y);
+  uint2 uh, ul;
+  uh.x = *reinterpret_cast<const uint32_t*>(&h01);
+  uh.y = *reinterpret_cast<const uint32_t*>(&h23);
+  ul.x = *reinterpret_cast<const uint32_t*>(&l01);
+  ul.y = *reinterpret_cast<const uint32_t*>(&l23);
+  *reinterpret_cast<uint2*>(hi) = uh;
+  *reinterpret_cast<uint2*>(lo) = ul;
+}
+
+// fragment of a 16 x 16 A tile (rows m0.., k0..) of a [row][k] bf16 array
+__device__ __forceinline__ void frag_a(uint32_t (&f)[4], const __nv_bfloat16* s, int pitch, int m0,
+                                       int k0, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const __nv_bfloat16* p = s + (m0 + g) * pitch + k0 + 2 * t;
+  f[0] = *reinterpret_cast<const uint32_t*>(p);
+  f[1] = *reinterpret_cast<const uint32_t*>(p + 8 * pitch);
+  f[2] = *reinterpret_cast<const uint32_t*>(p + 8);
+  f[3] = *reinterpret_cast<const uint32_t*>(p + 8 * pitch + 8);
+}
+
+// fragment of a 16 x 8 B tile (k0.., columns n0..) stored as [column][k]
+__device__ __forceinline__ void frag_b(uint32_t (&f)[2], const __nv_bfloat16* s, int pitch, int n0,
+                                       int k0, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const __nv_bfloat16* p = s + (n0 + g) * pitch + k0 + 2 * t;
+  f[0] = *reinterpret_cast<const uint32_t*>(p);
+  f[1] = *reinterpret_cast<const uint32_t*>(p + 8);
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// d += a.b with both operands split: hi.hi + hi.lo + lo.hi
+__device__ __forceinline__ void mma_split(float (&d)[4], const uint32_t (&ah)[4],
+                                          const uint32_t (&al)[4], const uint32_t (&bh)[2],
+                                          const uint32_t (&bl)[2]) {
+  mma_bf16(d, al, bh);
+  mma_bf16(d, ah, bl);
+  mma_bf16(d, ah, bh);
+}
+
+constexpr int kTcRows = 64;  // batch rows per CTA in both kernels
+constexpr int kTcCols = 64;  // q' columns per k_absorb_tc CTA
+constexpr int kTcCh = 32;    // output channels per k_combine_tc CTA
+
+size_t absorb_tc_smem(int d_h) {
+  const int pitch = ((d_h + 15) & ~15) + 8;
+  return (size_t)2 * (kTcRows + kTcCols) * pitch * sizeof(__nv_bfloat16);
+}
+
+size_t combine_tc_smem(int r_v) {
+  const int pitch = ((r_v + 15) & ~15) + 8;
+  return (size_t)2 * (kTcCh + kTcRows) * pitch * sizeof(__nv_bfloat16);
+}
+
+// One CTA per (head h, 64 q' columns, 64 batch rows): M = batch rows, N =
+// q' columns, K = d_h. Warp w computes rows 16*(w%4).. and columns
+// 32*(w/4).. of the tile. d_h is a multiple of 16 and q 16-byte aligned
+// (the launcher checks); columns past r_k (the rotary part) take q_rope.
+__global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
+  extern __shared__ __align__(16) unsigned char sm_abs_tc[];
+  const int pitch = a.d_h + 8;
+  __nv_bfloat16* q_hi = reinterpret_cast<__nv_bfloat16*>(sm_abs_tc);  // [64 rows][pitch]
+  __nv_bfloat16* q_lo = q_hi + kTcRows * pitch;
+  __nv_bfloat16* w_hi = q_lo + kTcRows * pitch;                        // [64 columns][pitch]
+  __nv_bfloat16* w_lo = w_hi + kTcCols * pitch;
+  pdl_launch_dependents();
+  const int h = blockIdx.x;
+  const int c0 = blockIdx.y * kTcCols;
+  const int b0 = blockIdx.z * kTcRows;
+  const int nb = min(kTcRows, a.B - b0);
+  const int rq = a.r_k + a.d_r;
+  const int nc = min(kTcCols, rq - c0);
+  const int ncw = max(0, min(kTcCols, a.r_k - c0));  // columns from W^K, a multiple of 8
+  // Stage the query rows and W^K_h's columns c0.. together: both are
+  // 64 * d_h values, 16 * d_h float4 items, and every thread issues its
+  // loads of both before its first shared store (one memory round trip per
+  // 2048 items of each). W^K_h rows i hold the columns contiguously; they
+  // are staged as [column][i], and consecutive threads take consecutive i
+  // so a warp's 2-byte transposed stores fall in 16 consecutive words (the
+  // loads of four columns each reach L1 by rows).
+  const int d4 = a.d_h / 4;
+  const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
+  const int n_items = kTcRows * d4;  // = d_h * kTcCols / 4
+  constexpr int kBatch = 8;
+  for (int base = threadIdx.x; base < n_items; base += 256 * kBatch) {
+    float4 vq[kBatch], vw[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int idx = base + k * 256;
+      vq[k] = vw[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (idx < n_items) {
+        const int bb = idx / d4, i4 = idx - bb * d4;
+        if (bb < nb)
+          vq[k] = __ldg(reinterpret_cast<const float4*>(
+                            a.q + ((size_t)(b0 + bb) * a.H + h) * a.d_h) + i4);
+        const int j = idx / a.d_h, i = idx - j * a.d_h;
+        if (4 * j < ncw) vw[k] = __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int idx = base + k * 256;
+      if (idx >= n_items) continue;
+      const int bb = idx / d4, i4 = idx - bb * d4;
+      store_split4(q_hi + bb * pitch + 4 * i4, q_lo + bb * pitch + 4 * i4, vq[k]);
+      const int j = idx / a.d_h, i = idx - j * a.d_h;
+      const float e[4] = {vw[k].x, vw[k].y, vw[k].z, vw[k].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(e[c]);
+        w_hi[(4 * j + c) * pitch + i] = hi;
+        w_lo[(4 * j + c) * pitch + i] = __float2bfloat16_rn(e[c] - __bfloat162float(hi));
+      }
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.y == 0) {
+    // c0 = scale * q . mu_k (natural-log units) in fp32 from the query rows
+    // in global memory (L2), warp w taking rows w, w + 8, ..: all of a
+    // lane's loads are issued before the first sum
+    float part[kTcRows / 8];
+#pragma unroll
+    for (int k = 0; k < kTcRows / 8; ++k) part[k] = 0.f;
+    if (a.mu_k) {
+      float mu[8];  // d_h <= 256: at most 8 values per lane
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int i = lane + 32 * m;
+        mu[m] = i < a.d_h ? __ldg(a.mu_k + (size_t)h * a.d_h + i) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < kTcRows / 8; ++k) {
+        const int bb = warp + 8 * k;
+        const float* qr = a.q + ((size_t)(b0 + bb) * a.H + h) * a.d_h;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int i = lane + 32 * m;
+          if (bb < nb && i < a.d_h) part[k] = fmaf(__ldg(qr + i), mu[m], part[k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kTcRows / 8; ++k) {
+      const int bb = warp + 8 * k;
+      const float acc = warp_sum(part[k]);
+      if (lane == 0 && bb < nb) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
+    }
+  }
+  const int m0 = (warp & 3) * 16, n0 = (warp >> 2) * 32;
+  float acc[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  if (n0 < ncw) {
+    for (int k0 = 0; k0 < a.d_h; k0 += 16) {
+      uint32_t ah[4], al[4];
+      frag_a(ah, q_hi, pitch, m0, k0, lane);
+      frag_a(al, q_lo, pitch, m0, k0, lane);
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        uint32_t bh[2], bl[2];
+        frag_b(bh, w_hi, pitch, n0 + 8 * nt, k0, lane);
+        frag_b(bl, w_lo, pitch, n0 + 8 * nt, k0, lane);
+        mma_split(acc[nt], ah, al, bh, bl);
+      }
+    }
+  }
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int bb = m0 + g + (e >> 1) * 8;
+      const int cl = n0 + 8 * nt + 2 * t + (e & 1);
+      if (bb >= nb || cl >= nc) continue;
+      const int c = c0 + cl;
+      const size_t unit = (size_t)(b0 + bb) * a.H + h;
+      // the rotary part of the query is not absorbed: it meets the cached
+      // rotated keys as it is
+      const float v = (c < a.r_k ? acc[nt][e] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
+                      a.qscale;
+      if (a.qp) a.qp[unit * rq + c] = v;
+      if (a.qsw) {
+        unsigned char* base = a.qsw + (size_t)(b0 + bb) * (rq / 64) * a.hp * 128;
+        *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)) = __float2bfloat16_rn(v);
+        if (h == a.H - 1)
+          for (int hz = a.H; hz < a.hp; ++hz)
+            *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)) =
+                __float2bfloat16_rn(0.f);
+      }
+    }
+}
+
+// One CTA per (head h, 32 output channels, 64 batch rows): the merge of
+// k_combine (same record map, same order of operations), with ubar written
+// split into shared memory, then out = W^V ubar with M = channels, N = batch
+// rows, K = r_v. Warp w computes channels 16*(w%2).. for rows 16*(w/2)...
+__global__ void __launch_bounds__(256, 2) k_combine_tc(CombineArgs a) {
+  extern __shared__ __align__(16) unsigned char sm_cmb_tc[];
+  __shared__ int s_np[kTcRows];
+  __shared__ long long s_off[kTcRows];
+  __shared__ float s_M[kTcRows], s_inv[kTcRows], s_keep[kTcRows], s_mu[kTcCh];
+  const int kp = (a.r_v + 15) & ~15;
+  const int pitch = kp + 8;
+  __nv_bfloat16* d_hi = reinterpret_cast<__nv_bfloat16*>(sm_cmb_tc);  // [32 channels][pitch]
+  __nv_bfloat16* d_lo = d_hi + kTcCh * pitch;
+  __nv_bfloat16* u_hi = d_lo + kTcCh * pitch;                          // [64 rows][pitch]
+  __nv_bfloat16* u_lo = u_hi + kTcRows * pitch;
+  const int h = blockIdx.x;
+  const int i0 = blockIdx.y * kTcCh;
+  const int b0 = blockIdx.z * kTcRows;
+  const int nb = min(kTcRows, a.B - b0);
+  const int ni = min(kTcCh, a.d_h - i0);
+  const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
+  const int r4 = a.r_v / 4, k4 = kp / 4;
+  // decoder slice; channels past d_h and columns past r_v are zero
+  stage_batched(kTcCh * k4, [&](int idx) {
+    const int i = idx / k4, j = idx - i * k4;
+    return (i < ni && j < r4) ? __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+  }, [&](int idx, float4 v) {
+    const int i = idx / k4, j = idx - i * k4;
+    store_split4(d_hi + i * pitch + 4 * j, d_lo + i * pitch + 4 * j, v);
+  });
+  if (threadIdx.x < kTcCh)
+    s_mu[threadIdx.x] = (a.mu_v && (int)threadIdx.x < ni) ? __ldg(a.mu_v + (size_t)h * a.d_h + i0 + threadIdx.x) : 0.f;
+  pdl_wait();  // partials come from the streaming kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
+
+  // 1. per row: its records, merged maximum and normaliser (as k_combine)
+  if (threadIdx.x < kTcRows) {
+    const int bb = threadIdx.x;
+    int np = 0;
+    long long off = 0;
+    float M = kNegBig, L = 0.f, keep = 0.f;
+    if (bb < nb) {
+      const long long u = (long long)(b0 + bb) * a.H + h;
+      const float c0u = (blockIdx.y == 0 && a.lse) ? a.c0[u] : 0.f;  // in flight with the records
+      const long long key = a.shared ? (long long)(b0 + bb) : u;
+      long long wf = 0, wl = -1;
+      if (a.ragged.seqinfo) {
+        const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
+        if (n > 0) {
+          const long long P = a.ragged.plan[1];
+          const long long first = a.ragged.cum[b0 + bb] + (a.shared ? 0LL : (long long)h * n);
+          wf = first / P;
+          wl = (first + n - 1) / P;
+        }
+      } else {
+        wf = (key * a.N) / a.P;
+        wl = ((key + 1) * a.N - 1) / a.P;
+      }
+      np = (int)(wl - wf + 1);
+      off = a.shared ? ((wf + key) * a.H + h) * a.pstride : (wf + key) * a.pstride;
+      const float* rec0 = a.part + off;
+      for (int p0 = 0; p0 < np; p0 += 4) {
+        float2 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          v[k] = p0 + k < np ? __ldg(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride))
+                             : make_float2(kNegBig, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float Mn = fmaxf(M, v[k].x);
+          L = L * exp2f(M - Mn) + v[k].y * exp2f(v[k].x - Mn);
+          M = Mn;
+        }
+      }
+      keep = np > 0 ? 1.f : 0.f;
+      if (blockIdx.y == 0 && a.lse)  // no attended token: lse = -inf
+        a.lse[u] = np > 0 ? (M + log2f(L)) * kLn2 + c0u : -INFINITY;
+    }
+    s_np[bb] = np;
+    s_off[bb] = off;
+    s_M[bb] = M;
+    s_inv[bb] = np > 0 ? 1.f / L : 0.f;
+    s_keep[bb] = keep;
+  }
+  __syncthreads();
+
+  // 2. ubar rows, split into shared memory; rows with no piece and the
+  //    padding columns come out 0
+  {
+    constexpr int kI = 8;
+    const int nitems = kTcRows * k4;
+    for (int base = threadIdx.x; base < nitems; base += 256 * kI) {
+      float4 acc[kI];
+      const float* rb[kI];
+      int npk[kI], c4k[kI];
+      float Mk[kI];
+      int npmax = 0;
+#pragma unroll
+      for (int k = 0; k < kI; ++k) {
+        const int idx = base + k * 256;
+        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        npk[k] = 0;
+        rb[k] = a.part;
+        c4k[k] = 0;
+        Mk[k] = 0.f;
+        if (idx < nitems) {
+          const int bb = idx / k4;
+          c4k[k] = idx - bb * k4;
+          npk[k] = c4k[k] < r4 ? s_np[bb] : 0;
+          rb[k] = a.part + s_off[bb];
+          Mk[k] = s_M[bb];
+        }
+        npmax = max(npmax, npk[k]);
+      }
+      for (int p = 0; p < npmax; ++p) {
+        float mv[kI];
+        float4 uv[kI];
+#pragma unroll
+        for (int k = 0; k < kI; ++k) {
+          if (p < npk[k]) {
+            mv[k] = __ldg(rb[k] + p * rstride);
+            uv[k] = __ldg(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kI; ++k) {
+          if (p < npk[k]) {
+            const float wk = exp2f(mv[k] - Mk[k]);
+            acc[k].x = fmaf(wk, uv[k].x, acc[k].x);
+            acc[k].y = fmaf(wk, uv[k].y, acc[k].y);
+            acc[k].z = fmaf(wk, uv[k].z, acc[k].z);
+            acc[k].w = fmaf(wk, uv[k].w, acc[k].w);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kI; ++k) {
+        const int idx = base + k * 256;
+        if (idx < nitems) {
+          const int bb = idx / k4;
+          const float inv = s_inv[bb];
+          store_split4(u_hi + bb * pitch + 4 * c4k[k], u_lo + bb * pitch + 4 * c4k[k],
+                       make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv));
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. out tile = W^V slice (32 x kp) . ubar^T (kp x 64)
+  const int m0 = (warp & 1) * 16, n0 = (warp >> 1) * 16;
+  float acc[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  if (m0 < ni && n0 < nb) {
+    for (int k0 = 0; k0 < kp; k0 += 16) {
+      uint32_t ah[4], al[4];
+      frag_a(ah, d_hi, pitch, m0, k0, lane);
+      frag_a(al, d_lo, pitch, m0, k0, lane);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bh[2], bl[2];
+        frag_b(bh, u_hi, pitch, n0 + 8 * nt, k0, lane);
+        frag_b(bl, u_lo, pitch, n0 + 8 * nt, k0, lane);
+        mma_split(acc[nt], ah, al, bh, bl);
+      }
+    }
+  }
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int il = m0 + g + (e >> 1) * 8;
+      const int bb = n0 + 8 * nt + 2 * t + (e & 1);
+      if (il >= ni || bb >= nb) continue;
+      a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + il] = acc[nt][e] + s_mu[il] * s_keep[bb];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -455,10 +867,19 @@ int env_int(const char* name, int dflt) {
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
-                         unsigned char* qsw, int hp, const float* q_rope, int d_r) {
+                         unsigned char* qsw, int hp, const float* q_rope, int d_r, bool tc) {
   AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp,
                q_rope, q_rope ? d_r : 0};
   const int rq = r_k + a.d_r;
+  if (tc && d_h % 16 == 0 && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
+    const size_t smem = absorb_tc_smem(d_h);
+    cudaError_t e = cudaFuncSetAttribute(k_absorb_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_absorb_tc)");
+    dim3 grid(H, (rq + kTcCols - 1) / kTcCols, (B + kTcRows - 1) / kTcRows);
+    k_absorb_tc<<<grid, 256, smem, stream>>>(a);
+    return check_cuda(cudaGetLastError(), "launch k_absorb_tc");
+  }
   int rows, cols;
   pick_block(H, rq, B, &rows, &cols, false, env_int("LLA_ABSORB_MAX_COLS", 2));
   dim3 grid(H, (rq + 32 * cols - 1) / (32 * cols), (B + 8 * rows - 1) / (8 * rows));
@@ -479,13 +900,26 @@ lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
                           long long P, int shared, float* out, float* lse, cudaStream_t stream,
-                          const RaggedMap* ragged) {
+                          const RaggedMap* ragged, bool tc) {
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse,
                 RaggedMap{nullptr, nullptr, nullptr}};
   if (ragged) a.ragged = *ragged;
+  if (tc) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(H, (d_h + kTcCh - 1) / kTcCh, (B + kTcRows - 1) / kTcRows);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = combine_tc_smem(r_v);
+    cudaError_t e = cudaFuncSetAttribute(k_combine_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)cfg.dynamicSmemBytes);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_combine_tc)");
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    return check_cuda(cudaLaunchKernelEx(&cfg, k_combine_tc, a), "launch k_combine_tc");
+  }
   int rows, cols;
   pick_block(H, d_h, B, &rows, &cols, true, env_int("LLA_COMBINE_MAX_COLS", 1));
   cudaLaunchConfig_t cfg{};
@@ -505,6 +939,17 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   return check_cuda(cudaLaunchKernelEx(&cfg, fn, a), "launch k_combine");
+}
+
+// Per-head decode takes the tensor-core absorb and combine for bf16
+// latents, large batches and wide ranks only. Both forms are bound by memory
+// round trips at these sizes, and the FFMA work the tensor cores remove
+// grows with B * r. Measured on B200 (whole decode call): B = 64, r = 128
+// and B = 768, r = 24 ran as fast or faster on the CUDA-core forms (327 vs
+// 327 us, 746 vs 751 us), while the LLA-2D shape (B = 256, r = 256) gained
+// 15 us per call on the tensor-core forms.
+bool small_gemm_tc(int esz, int B, int r_k, int r_v) {
+  return esz == 2 && B >= 256 && std::max(r_k, r_v) >= 192;
 }
 
 lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePlan* p) {
@@ -617,7 +1062,8 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_stream)");
 
   // 1. absorb
-  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, q_rope, d_r);
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, q_rope, d_r,
+                     small_gemm_tc(esz, B, r_k, r_v));
   if (st != LLA_OK) return st;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -659,7 +1105,8 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
     if (e != cudaSuccess) return check_cuda(e, "record timing event");
   }
   // 3. combine
-  return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, N, d.P, 0, out, lse, stream);
+  return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, N, d.P, 0, out, lse, stream,
+                        nullptr, small_gemm_tc(esz, B, r_k, r_v));
   return LLA_OK;
 }
 

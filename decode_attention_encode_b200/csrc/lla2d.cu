@@ -765,7 +765,7 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
   lla_status st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k - d_r, scale, nullptr, c0, stream, qsw,
-                                d.hp, q_rope, d_r);
+                                d.hp, q_rope, d_r, true);
   if (st != LLA_OK) return st;
 
   D2Args a{};
@@ -828,10 +828,11 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
   if (pg) {  // sequence b's pieces: the CTAs of its tiles, cum[b] .. cum[b] + tiles - 1
     RaggedMap rm{pg->seqinfo, pg->cum, pg->plan};
     return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 1, out, lse, stream,
-                          &rm);
+                          &rm, true);
   }
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v,
-                        (long long)d.tps * kRows, (long long)d.tpc * kRows, 1, out, lse, stream);
+                        (long long)d.tps * kRows, (long long)d.tpc * kRows, 1, out, lse, stream,
+                        nullptr, true);
 }
 
 // The paged plan: the dense plan's kernel shape with a one-wave grid (the

@@ -253,7 +253,8 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
                          window, d.W, 2 * d.tile, 0, seqinfo, cum, plan, wstart, stream);
   if (st != LLA_OK) return st;
   // 2. absorb (plain launch)
-  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream);
+  st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, nullptr, 0,
+                     small_gemm_tc(esz, B, r_k, r_v));
   if (st != LLA_OK) return st;
   // 3. stream
   {
@@ -302,7 +303,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
   // 4. combine over the ragged piece map
   RaggedMap rm{seqinfo, cum, plan};
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 0, out, lse, stream,
-                        &rm);
+                        &rm, small_gemm_tc(esz, B, r_k, r_v));
 }
 
 }  // namespace lla
