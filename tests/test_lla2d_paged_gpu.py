@@ -129,9 +129,11 @@ def test_dense_equivalent_layout_matches_the_dense_kernel():
     assert (l1 - l2).abs().max().item() <= 1e-4
 
 
-def test_full_size_ragged_32x_batch_sampled():
+@pytest.mark.parametrize("page_size", [256, 64])
+def test_full_size_ragged_32x_batch_sampled(page_size):
+    # the lla2d_32x_paged and lla2d_32x_paged64 workloads
     lens = synth.ragged_lengths(256, 8192, seed=0)
-    inp = make(lens, 16, 128, 256, 256, 256, seed=0)
+    inp = make(lens, 16, 128, 256, 256, page_size, seed=0)
     out, lse = run(inp)
     torch.cuda.synchronize()
     assert lla.device_status() == 0
