@@ -129,6 +129,10 @@ LLA_API void lla_set_timing_events(void *ev_begin, void *ev_end);
  *   out[b][h] = sum_j softmax(s)_j vhat_j,    lse[b][h] = ln sum_j exp(s_j)
  * computed as q' = scale dk_t[h]^T q, s_j = q' . zk_j + scale q . mu_k,
  * ubar = sum_j p_j zv_j, out = dv_t[h] ubar + mu_v_t[h].
+ * Arithmetic is fp32. For bf16 latents with B >= 256 and a rank of 192 or
+ * more, the two small products q' and dv_t ubar run on the tensor cores
+ * with each fp32 operand split into two bf16 parts (hi + lo) and fp32
+ * accumulation; their error stays below 2^-16 of each product term.
  *
  * Arguments
  *   q        [B][H][d_h] fp32: this loop's query of each sequence and head.
@@ -296,7 +300,9 @@ LLA_API lla_status lla_decode_attn_paged(const float *q, const void *zk_pages,
  * [H][d_h][r_k] and dv_t [H][d_h][r_v] are the per-(head, loop) decoders.
  * The score and value contractions run on the tensor cores with bf16
  * operands (the absorbed query and the softmax weights are rounded to bf16)
- * and fp32 accumulation.
+ * and fp32 accumulation. The absorbed query and dv_t ubar are formed on the
+ * tensor cores from split (hi + lo) bf16 operands with fp32 accumulation,
+ * within 2^-16 of each product term.
  * Limits: H <= 32 (padded to 16 or 32 inside), r_k a multiple of 64 and
  * r_v a multiple of 128, both at most 256, d_h 1..256, 1 <= N <= n_cap.
  * Outside them the call returns LLA_ERR_UNSUPPORTED and the workspace query
