@@ -447,9 +447,11 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
 // CUDA-core forms above spend most of their time on as FFMA chains. Here the
 // contraction runs on warp-level bf16 tensor-core MMAs (m16n8k16, fp32
 // accumulate). Each fp32 operand x is split as hi = bf16(x), lo = bf16(x - hi)
-// (x - hi is exact in fp32) and the product is hi.hi + hi.lo + lo.hi; the
-// dropped lo.lo term and the split's residue are below 2^-16 of each product,
-// far under the bf16 rounding the latents and the LLA-2D query already carry.
+// (x - hi is exact in fp32) and the product is hi.hi + hi.lo + lo.hi. With
+// bf16's 8-bit significand |lo| <= 2^-8 |x| and |x - hi - lo| <= 2^-16 |x|,
+// so the dropped lo.lo term and the two residues together stay within
+// 3 * 2^-16 of each product |x y|: far under the bf16 rounding the latents
+// and the LLA-2D query already carry.
 // Accumulators stay in registers: no tensor memory is allocated, so these
 // kernels never contend with the programmatically overlapped k_lla2d for it.
 //

@@ -132,7 +132,7 @@ LLA_API void lla_set_timing_events(void *ev_begin, void *ev_end);
  * Arithmetic is fp32. For bf16 latents with B >= 256 and a rank of 192 or
  * more, the two small products q' and dv_t ubar run on the tensor cores
  * with each fp32 operand split into two bf16 parts (hi + lo) and fp32
- * accumulation; their error stays below 2^-16 of each product term.
+ * accumulation; their error stays within 3 * 2^-16 of each product term.
  *
  * Arguments
  *   q        [B][H][d_h] fp32: this loop's query of each sequence and head.
@@ -302,7 +302,7 @@ LLA_API lla_status lla_decode_attn_paged(const float *q, const void *zk_pages,
  * operands (the absorbed query and the softmax weights are rounded to bf16)
  * and fp32 accumulation. The absorbed query and dv_t ubar are formed on the
  * tensor cores from split (hi + lo) bf16 operands with fp32 accumulation,
- * within 2^-16 of each product term.
+ * within 3 * 2^-16 of each product term.
  * Limits: H <= 32 (padded to 16 or 32 inside), r_k a multiple of 64 and
  * r_v a multiple of 128, both at most 256, d_h 1..256, 1 <= N <= n_cap.
  * Outside them the call returns LLA_ERR_UNSUPPORTED and the workspace query
