@@ -702,6 +702,8 @@ def run_lla(args, world, rank, local):
             "global_batch": cfg.B * world, "seq_len": cfg.N,
         },
         "hbm_gbs_per_call": step_bytes / (call_ms_mean * 1e-3) / 1e9,
+        # per-head decode reads each cached token once per head
+        "token_head_reads_per_s": None if cfg.two_d else value * cfg.H,
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": profiled_traffic(cfg.name),
