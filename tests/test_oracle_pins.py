@@ -632,6 +632,95 @@ def test_lla2d_rope_is_per_head_rope_with_the_row_shared_by_every_head():
     np.testing.assert_allclose(l3, l4, atol=1e-12)
 
 
+def _rope_batch(seed, B=3, H=4, d=8, n_cap=11, rk=8, dr=6, rv=12):
+    """Per-head store with a DIFFERENT latent and rotary key for every
+    (b, h): zk [B, H, n_cap, rk + dr], zv [B, H, n_cap, rv]."""
+    r = rng(seed)
+    return dict(q=r.normal(size=(B, H, d)), qr=r.normal(size=(B, H, dr)),
+                zk=r.normal(size=(B, H, n_cap, rk + dr)), zv=r.normal(size=(B, H, n_cap, rv)),
+                dk=r.normal(size=(H, d, rk)), dv=r.normal(size=(H, d, rv)),
+                mk=r.normal(size=(H, d)), mv=r.normal(size=(H, d)), rk=rk, dr=dr)
+
+
+def test_per_head_rope_reads_each_heads_own_row_and_units_pick_their_unit():
+    # §7 "Per-head LLA versus LLA-2D at inference": each (b, h) unit is the
+    # decoupled-RoPE unit on ITS OWN latent rows. Distinct rows per head, so
+    # reading another head's (or batch row's) latents fails here.
+    u = _rope_batch(301)
+    q, qr, zk, zv, dk, dv, mk, mv = (u[k] for k in ("q", "qr", "zk", "zv", "dk", "dv", "mk", "mv"))
+    rk = u["rk"]
+    B, H = q.shape[:2]
+    N = 9  # rows [N, n_cap) must be ignored
+    out, lse = oracle.lla_decode_rope(q, qr, zk, zv, dk, dv, mk, mv, scale=0.3, N=N)
+    for b in range(B):
+        for h in range(H):
+            o1, l1 = oracle.decode_unit_rope(q[b, h], qr[b, h], zk[b, h, :N, :rk],
+                                             zk[b, h, :N, rk:], zv[b, h, :N], dk[h], dv[h],
+                                             mk[h], mv[h], 0.3)
+            np.testing.assert_allclose(out[b, h], o1, rtol=0, atol=1e-12)
+            assert abs(lse[b, h] - l1) < 1e-12
+    # a shuffled subset of units, with a repeat, returns one row per listed unit
+    units = [(2, 3), (0, 1), (1, 0), (2, 0), (0, 1), (1, 3)]
+    sub_o, sub_l = oracle.lla_decode_rope(q, qr, zk, zv, dk, dv, mk, mv, scale=0.3, N=N,
+                                          units=units)
+    assert sub_o.shape == (len(units), q.shape[2])
+    for i, (b, h) in enumerate(units):
+        np.testing.assert_allclose(sub_o[i], out[b, h], rtol=0, atol=1e-12)
+        assert abs(sub_l[i] - lse[b, h]) < 1e-12
+
+
+def test_per_head_rope_is_nope_decode_on_a_block_embedded_codec():
+    # An independent route through the NoPE decode: append the rotary part to
+    # the query, the identity on the rotary coordinates to W^K_up, zeros to
+    # W^V_up and to the means. Then q'.(W' z' + mu') = q.(W z + mu) + q_rope.k_rope,
+    # so lla_decode on the block-embedded codec gives the rotary scores, and
+    # its output is [out | 0]. Distinct per-head rows, on a shuffled subset.
+    u = _rope_batch(302, B=2, H=3, d=8, n_cap=10, rk=8, dr=4, rv=16)
+    q, qr, zk, zv, dk, dv, mk, mv = (u[k] for k in ("q", "qr", "zk", "zv", "dk", "dv", "mk", "mv"))
+    rk, dr = u["rk"], u["dr"]
+    H, d = q.shape[1], q.shape[2]
+    rv = zv.shape[-1]
+    q_e = np.concatenate([q, qr], axis=-1)
+    dk_e = np.zeros((H, d + dr, rk + dr))
+    dk_e[:, :d, :rk] = dk
+    dk_e[:, d:, rk:] = np.eye(dr)
+    dv_e = np.zeros((H, d + dr, rv))
+    dv_e[:, :d] = dv
+    mk_e = np.concatenate([mk, np.zeros((H, dr))], axis=-1)
+    mv_e = np.concatenate([mv, np.zeros((H, dr))], axis=-1)
+    units = [(1, 2), (0, 0), (1, 0), (0, 2)]
+    sc = 0.25
+    o_r, l_r = oracle.lla_decode_rope(q, qr, zk, zv, dk, dv, mk, mv, scale=sc, N=7, units=units)
+    o_e, l_e = oracle.lla_decode(q_e, zk, zv, dk_e, dv_e, mk_e, mv_e, sc, N=7, units=units)
+    np.testing.assert_allclose(o_r, o_e[:, :d], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o_e[:, d:], 0.0, atol=0)
+    np.testing.assert_allclose(l_r, l_e, rtol=0, atol=1e-12)
+
+
+def test_lla2d_rope_units_pick_their_unit_from_the_shared_row():
+    r = rng(303)
+    B, H, d, n_cap, rk, dr, rv = 3, 4, 8, 10, 8, 4, 12
+    zk = r.normal(size=(B, n_cap, rk + dr))
+    zv = r.normal(size=(B, n_cap, rv))
+    q, qr = r.normal(size=(B, H, d)), r.normal(size=(B, H, dr))
+    dk, dv = r.normal(size=(H, d, rk)), r.normal(size=(H, d, rv))
+    mk, mv = r.normal(size=(H, d)), r.normal(size=(H, d))
+    N = 8
+    out, lse = oracle.lla2d_decode_rope(q, qr, zk, zv, dk, dv, mk, mv, scale=0.3, N=N)
+    for b in range(B):
+        for h in range(H):
+            o1, l1 = oracle.decode_unit_rope(q[b, h], qr[b, h], zk[b, :N, :rk], zk[b, :N, rk:],
+                                             zv[b, :N], dk[h], dv[h], mk[h], mv[h], 0.3)
+            np.testing.assert_allclose(out[b, h], o1, rtol=0, atol=1e-12)
+            assert abs(lse[b, h] - l1) < 1e-12
+    units = [(2, 1), (0, 3), (2, 1), (1, 0)]
+    sub_o, sub_l = oracle.lla2d_decode_rope(q, qr, zk, zv, dk, dv, mk, mv, scale=0.3, N=N,
+                                            units=units)
+    for i, (b, h) in enumerate(units):
+        np.testing.assert_allclose(sub_o[i], out[b, h], rtol=0, atol=1e-12)
+        assert abs(sub_l[i] - lse[b, h]) < 1e-12
+
+
 def test_merge_of_context_parts_equals_attention_over_the_whole():
     # split the cached tokens into disjoint parts, attend each, merge
     r = rng(81)
