@@ -137,9 +137,107 @@ def _dtype_code(t):
 
 
 def _need_cuda(*ts):
+    """Every given tensor is a contiguous CUDA tensor on one device, and that
+    device is the current one (the call's stream and kernels run there)."""
+    dev = None
     for t in ts:
-        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
             raise LLAError(LLA_ERR_INVALID_ARG, "tensors must be contiguous CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise LLAError(LLA_ERR_INVALID_ARG, f"tensors on {dev} and {t.device}: use one device")
+    if dev is not None and dev.index != torch.cuda.current_device():
+        raise LLAError(LLA_ERR_INVALID_ARG, f"tensors are on {dev} but the current device is "
+                                            f"cuda:{torch.cuda.current_device()}")
+
+
+def _expect(cond, msg):
+    if not cond:
+        raise LLAError(LLA_ERR_INVALID_ARG, msg)
+
+
+def _shape(name, t, shape):
+    """t has exactly this shape (None: t is optional and absent)."""
+    if t is None:
+        return
+    _expect(tuple(t.shape) == tuple(shape),
+            f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _f32(name, t, shape=None):
+    if t is None:
+        return
+    _expect(t.dtype == torch.float32, f"{name} must be float32, got {t.dtype}")
+    if shape is not None:
+        _shape(name, t, shape)
+
+
+def _same_latent_type(zk, zv):
+    _dtype_code(zk)
+    _expect(zv.dtype == zk.dtype, f"zv must have zk's dtype {zk.dtype}, got {zv.dtype}")
+
+
+def _check_query_side(q, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, r_k, r_v, q_rope=None):
+    """fp32 operands of a decode call against q [B,H,d_h]: decoders
+    [H,d_h,r_k] and [H,d_h,r_v], means [H,d_h], out [B,H,d_h], lse [B,H],
+    and the rotary query [B,H,d_r] when there is one."""
+    _f32("q", q)
+    _expect(q.dim() == 3, f"q must be [B, H, d_h], got {tuple(q.shape)}")
+    B, H, d_h = q.shape
+    if q_rope is not None:
+        _f32("q_rope", q_rope)
+        _expect(q_rope.dim() == 3 and tuple(q_rope.shape[:2]) == (B, H),
+                f"q_rope must be [B, H, d_r], got {tuple(q_rope.shape)}")
+    _f32("dk_t", dk_t, (H, d_h, r_k))
+    _f32("dv_t", dv_t, (H, d_h, r_v))
+    _f32("mu_k_t", mu_k_t, (H, d_h))
+    _f32("mu_v_t", mu_v_t, (H, d_h))
+    _f32("out", out, (B, H, d_h))
+    _f32("lse", lse, (B, H))
+
+
+def _check_decode(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, *, two_d, r_k=None,
+                  q_rope=None):
+    """Shapes and element types of a dense decode call's operands, checked
+    before anything reaches the library (whose kernels trust them): latents
+    [B,(H,)n_cap,r] of one type matching q [B,H,d_h], plus the fp32 operands
+    of _check_query_side. r_k, when given, is the latent part of a key row
+    that also holds a rotary key."""
+    _expect(q.dim() == 3, f"q must be [B, H, d_h], got {tuple(q.shape)}")
+    B, H = q.shape[0], q.shape[1]
+    _same_latent_type(zk, zv)
+    lead = 2 if two_d else 3
+    _expect(zk.dim() == lead + 1 and zv.dim() == lead + 1,
+            "latents must be [B, n_cap, r]" if two_d else "latents must be [B, H, n_cap, r]")
+    want = (B, zk.shape[-2]) if two_d else (B, H, zk.shape[-2])
+    _expect(tuple(zk.shape[:lead]) == want and tuple(zv.shape[:lead]) == want,
+            f"zk {tuple(zk.shape)} and zv {tuple(zv.shape)} do not match q {tuple(q.shape)}")
+    _check_query_side(q, dk_t, dv_t, mu_k_t, mu_v_t, out, lse,
+                      zk.shape[-1] if r_k is None else r_k, zv.shape[-1], q_rope)
+
+
+def _check_paged(q, zk_pages, zv_pages, block_table, seq_lens, *, two_d):
+    """Page pools [P,(H,)page_size,r] of one latent type, an int32
+    [B,max_blocks] block table and int32 [B] lengths."""
+    _expect(q.dim() == 3, f"q must be [B, H, d_h], got {tuple(q.shape)}")
+    B = q.shape[0]
+    _same_latent_type(zk_pages, zv_pages)
+    lead = 2 if two_d else 3
+    _expect(zk_pages.dim() == lead + 1 and zv_pages.dim() == lead + 1,
+            "page pools must be [P, page_size, r]" if two_d
+            else "page pools must be [P, H, page_size, r]")
+    _expect(tuple(zk_pages.shape[:lead]) == tuple(zv_pages.shape[:lead]),
+            f"zk_pages {tuple(zk_pages.shape)} and zv_pages {tuple(zv_pages.shape)} disagree")
+    if not two_d:
+        _expect(zk_pages.shape[1] == q.shape[1], "page pools must hold q's H heads")
+    _expect(block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32,
+            "block_table and seq_lens must be int32")
+    _expect(block_table.dim() == 2 and block_table.shape[0] == B,
+            f"block_table must be [B, max_blocks] with B = {B}, got {tuple(block_table.shape)}")
+    _shape("seq_lens", seq_lens, (B,))
 
 
 def device_status(clear: bool = False) -> int:
@@ -185,6 +283,7 @@ def lla2d_decode_attn_workspace(B, H, N, r_k, r_v) -> int:
 
 def _decode(fn_name, ws_name, q, zk, zv, dk_t, dv_t, N, mu_k_t, mu_v_t, scale, out, lse,
             workspace, stream, want_lse, two_d):
+    _check_decode(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, two_d=two_d)
     _need_cuda(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
     B, H, d_h = q.shape
     if two_d:
@@ -230,6 +329,7 @@ def lla_decode_attn_noalloc(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=N
     device memory: the library uses its own fixed scratch array instead of a
     workspace (see include/lla.h for the size limit and the ordering rule).
     Only `out` and `lse` are allocated here when not given."""
+    _check_decode(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, two_d=False)
     _need_cuda(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse)
     B, H, d_h = q.shape
     n_cap, r_k = zk.shape[2], zk.shape[3]
@@ -255,13 +355,16 @@ def lla_decode_attn_rope(q, q_rope, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_
     holds each token's latent followed by its rotated rotary key; q_rope
     [B,H,d_r] fp32 is this loop's rotated rotary query; dk_t [H,d_h,r_k].
     Returns (out [B,H,d_h], lse [B,H] or None)."""
-    _need_cuda(q, q_rope, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
+    _expect(q.dim() == 3 and q_rope.dim() == 3, "q and q_rope must be [B, H, d_h] and [B, H, d_r]")
     B, H, d_h = q.shape
     d_r = q_rope.shape[2]
     n_cap, rq = zk.shape[2], zk.shape[3]
     r_k, r_v = dk_t.shape[2], zv.shape[3]
     if rq != r_k + d_r:
         raise LLAError(LLA_ERR_INVALID_ARG, "zk rows must hold r_k + d_r values")
+    _check_decode(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, two_d=False, r_k=r_k,
+                  q_rope=q_rope)
+    _need_cuda(q, q_rope, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
     N = n_cap if N is None else N
     scale = 1.0 / math.sqrt(d_h) if scale is None else scale
     if out is None:
@@ -294,12 +397,11 @@ def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv
     bf16 or fp32; block_table [B,max_blocks] int32 and seq_lens [B] int32 on
     the device; sink, window: the eviction set (window 0 keeps every token).
     Returns (out [B,H,d_h], lse [B,H] or None)."""
+    _check_paged(q, zk_pages, zv_pages, block_table, seq_lens, two_d=False)
+    _check_query_side(q, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, zk_pages.shape[-1],
+                      zv_pages.shape[-1])
     _need_cuda(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, out,
                lse, workspace)
-    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
-        raise LLAError(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be int32")
-    if not (block_table.is_contiguous() and seq_lens.is_contiguous()):
-        raise LLAError(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be contiguous")
     B, H, d_h = q.shape
     num_pages, page_size, r_k = zk_pages.shape[0], zk_pages.shape[2], zk_pages.shape[3]
     r_v = zv_pages.shape[3]
@@ -329,13 +431,16 @@ def lla2d_decode_attn_rope(q, q_rope, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, m
     """LLA-2D decode with the decoupled rotary branch: zk [B,n_cap,r_k+d_r]
     holds each token's latent followed by its rotated rotary key (shared by
     every head); q_rope [B,H,d_r]; dk_t [H,d_h,r_k]. Returns (out, lse)."""
-    _need_cuda(q, q_rope, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
+    _expect(q.dim() == 3 and q_rope.dim() == 3, "q and q_rope must be [B, H, d_h] and [B, H, d_r]")
     B, H, d_h = q.shape
     d_r = q_rope.shape[2]
     n_cap, rq = zk.shape[1], zk.shape[2]
     r_k, r_v = dk_t.shape[2], zv.shape[2]
     if rq != r_k + d_r:
         raise LLAError(LLA_ERR_INVALID_ARG, "zk rows must hold r_k + d_r values")
+    _check_decode(q, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, two_d=True, r_k=r_k,
+                  q_rope=q_rope)
+    _need_cuda(q, q_rope, zk, zv, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, workspace)
     N = n_cap if N is None else N
     scale = 1.0 / math.sqrt(d_h) if scale is None else scale
     if out is None:
@@ -366,10 +471,11 @@ def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, 
     zv_pages [P,page_size,r_v] bf16 shared by every head, page_size a
     multiple of 64; block_table [B,max_blocks] and seq_lens [B] int32 on
     the device. Returns (out [B,H,d_h], lse [B,H] or None)."""
+    _check_paged(q, zk_pages, zv_pages, block_table, seq_lens, two_d=True)
+    _check_query_side(q, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, zk_pages.shape[-1],
+                      zv_pages.shape[-1])
     _need_cuda(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t, mu_v_t, out,
                lse, workspace)
-    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
-        raise LLAError(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be int32")
     B, H, d_h = q.shape
     num_pages, page_size, r_k = zk_pages.shape
     r_v = zv_pages.shape[2]
@@ -402,12 +508,40 @@ def lla2d_decode_attn(q, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None, s
                    N, mu_k_t, mu_v_t, scale, out, lse, workspace, stream, want_lse, two_d=True)
 
 
+def _check_encode(x, w_down_t, mu=None, muw=None):
+    """x [T,N,G,d_loop] bf16, w_down_t [G,r,T*d_loop] bf16, mu [G,T*d_loop]
+    fp32, muw [G,r] fp32."""
+    _expect(x.dtype == torch.bfloat16, f"x must be bfloat16, got {x.dtype}")
+    _expect(x.dim() == 4, f"x must be [T, N, G, d_loop], got {tuple(x.shape)}")
+    T, N, G, d_loop = x.shape
+    _expect(w_down_t.dtype == torch.bfloat16, f"w_down_t must be bfloat16, got {w_down_t.dtype}")
+    _expect(w_down_t.dim() == 3 and w_down_t.shape[0] == G and w_down_t.shape[2] == T * d_loop,
+            f"w_down_t must be [G, r, T*d_loop] = [{G}, r, {T * d_loop}], "
+            f"got {tuple(w_down_t.shape)}")
+    r = w_down_t.shape[1]
+    _f32("mu", mu, (G, T * d_loop))
+    _f32("muw", muw, (G, r))
+
+
+def _check_z(z, x, G, N, r, z_row_stride, z_group_stride):
+    """z is a bfloat16 CUDA tensor on x's device whose storage holds every
+    row the strides address (z may be a strided view into a larger store;
+    the library writes through its data pointer)."""
+    _expect(z.dtype == torch.bfloat16, f"z must be bfloat16, got {z.dtype}")
+    _expect(z.is_cuda and z.device == x.device, f"z must be on {x.device}")
+    last = (G - 1) * int(z_group_stride) + (N - 1) * int(z_row_stride) + r
+    have = z.untyped_storage().nbytes() // 2 - z.storage_offset()
+    _expect(last <= have, f"z strides address {last} elements past z's start; its storage "
+                          f"holds {have}")
+
+
 def lla_encode(x, w_down_t, mu=None, z=None, z_row_stride=None, z_group_stride=None,
                stream=None):
     """Latent write: x [T,N,G,d_loop] bf16, w_down_t [G,r,T*d_loop] bf16 (W_down transposed),
     mu [G,T*d_loop] fp32 or None. Writes z (default a new [G,N,r] bf16
     tensor; pass z plus strides in elements to write into a larger store).
     Returns z."""
+    _check_encode(x, w_down_t, mu=mu)
     _need_cuda(x, w_down_t, mu)
     T, N, G, d_loop = x.shape
     r = w_down_t.shape[1]
@@ -416,6 +550,7 @@ def lla_encode(x, w_down_t, mu=None, z=None, z_row_stride=None, z_group_stride=N
         z_row_stride, z_group_stride = r, N * r
     if z_row_stride is None or z_group_stride is None:
         raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
+    _check_z(z, x, G, N, r, z_row_stride, z_group_stride)
     st = lib().lla_encode(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t), _ptr(mu),
                           _ptr(z), int(z_row_stride), int(z_group_stride), _stream(stream))
     _check(st)
@@ -425,8 +560,12 @@ def lla_encode(x, w_down_t, mu=None, z=None, z_row_stride=None, z_group_stride=N
 def lla_encode_bias(w_down_t, mu, muw=None, stream=None):
     """mu W_down of a codec, once: w_down_t [G,r,K] bf16, mu [G,K] fp32.
     Returns muw [G,r] fp32."""
-    _need_cuda(w_down_t, mu, muw)
+    _expect(w_down_t.dtype == torch.bfloat16 and w_down_t.dim() == 3,
+            "w_down_t must be a bfloat16 [G, r, K] tensor")
     G, r, K = w_down_t.shape
+    _f32("mu", mu, (G, K))
+    _f32("muw", muw, (G, r))
+    _need_cuda(w_down_t, mu, muw)
     if muw is None:
         muw = torch.empty((G, r), device=w_down_t.device, dtype=torch.float32)
     _check(lib().lla_encode_bias(_ptr(w_down_t), _ptr(mu), G, K, r, _ptr(muw), _stream(stream)))
@@ -444,6 +583,7 @@ def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_gro
     [G,r] fp32, or None for a zero mean). With split (default) a workspace
     is allocated when the shape benefits from a split over K (or pass one).
     Returns z."""
+    _check_encode(x, w_down_t, muw=muw)
     _need_cuda(x, w_down_t, muw, workspace)
     T, N, G, d_loop = x.shape
     r = w_down_t.shape[1]
@@ -456,6 +596,7 @@ def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_gro
         z_row_stride, z_group_stride = r, N * r
     if z_row_stride is None or z_group_stride is None:
         raise LLAError(LLA_ERR_INVALID_ARG, "pass z_row_stride and z_group_stride with z")
+    _check_z(z, x, G, N, r, z_row_stride, z_group_stride)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().lla_encode_with_bias(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t),
                                     _ptr(muw), _ptr(z), int(z_row_stride), int(z_group_stride),
@@ -468,11 +609,16 @@ def lla_merge_attn(out_parts, lse_parts, out=None, lse=None, stream=None):
     """Log-sum-exp merge of attention over disjoint context parts:
     out_parts [R, ..., d], lse_parts [R, ...] fp32 on the device (each part
     a decode call's (out, lse)). Returns (out [..., d], lse [...])."""
+    _f32("out_parts", out_parts)
+    _f32("lse_parts", lse_parts)
+    _expect(out_parts.dim() >= 2 and tuple(lse_parts.shape) == tuple(out_parts.shape[:-1]),
+            f"lse_parts {tuple(lse_parts.shape)} must be out_parts {tuple(out_parts.shape)} "
+            "without its last axis")
+    _f32("out", out, out_parts.shape[1:])
+    _f32("lse", lse, lse_parts.shape[1:])
     _need_cuda(out_parts, lse_parts, out, lse)
     R, d = out_parts.shape[0], out_parts.shape[-1]
     U = lse_parts[0].numel()
-    if out_parts[0].numel() != U * d:
-        raise LLAError(LLA_ERR_INVALID_ARG, "out_parts and lse_parts disagree on the units")
     if out is None:
         out = torch.empty(out_parts.shape[1:], device=out_parts.device, dtype=torch.float32)
     if lse is None:

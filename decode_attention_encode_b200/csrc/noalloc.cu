@@ -9,6 +9,13 @@
 // runs the same kernels with the same launch plan, but its scratch is a
 // fixed array compiled into the library: every GPU that loads liblla holds
 // LLA_NOALLOC_SCRATCH_BYTES of it until the process exits.
+//
+// Under CUDA's default lazy module loading the array is placed on a device
+// when this file's module loads there, which happens at the first call's
+// address lookup; a caller that reserves the rest of the device up front
+// should make one call before that reservation (or load modules eagerly).
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "internal.h"
@@ -26,9 +33,40 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];
 
-// Device address of the scratch on the current device, looked up once per
-// device (the first call on each device does this).
+// Identifier of the calling thread's current CUDA context, or 0 when there
+// is none yet or the driver cannot say. cudaDeviceReset destroys a device's
+// primary context and the next runtime call creates a new one, with a new
+// identifier and a new copy of the scratch, so an address looked up in one
+// context is reused only within that context.
+unsigned long long current_context_id() {
+  static std::once_flag once;
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch on the current device. It is looked up once
+// per device and context: the first call on a device (and the first after a
+// cudaDeviceReset) does this set-up.
 lla_status scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -36,11 +74,14 @@ lla_status scratch_address(void** out) {
   if (dev < 0 || dev >= kMaxDevices)
     return fail(LLA_ERR_UNSUPPORTED, "device index %d out of range", dev);
   std::lock_guard<std::mutex> g(g_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress(noalloc scratch)");
     g_scratch_ptr[dev] = p;
+    // the lookup made the device's context current if it was not yet
+    g_scratch_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return LLA_OK;

@@ -220,7 +220,12 @@ LLA_API lla_status lla_decode_attn_rope(const float *q, const float *q_rope,
  *    return LLA_ERR_WORKSPACE before anything is launched.
  *  - The first call on each device looks up the scratch's device address
  *    (cudaGetSymbolAddress with that device current); make that first call
- *    before any stream capture.
+ *    before any stream capture. The lookup is repeated once after a
+ *    cudaDeviceReset (a new context holds a new copy of the scratch).
+ *  - Under CUDA's default lazy module loading the scratch is placed on a
+ *    device when that first lookup loads it. A caller that reserves the
+ *    rest of the device for its own pool should make one call at start-up,
+ *    before that reservation, or set CUDA_MODULE_LOADING=EAGER.
  *  - All calls on a device share the one scratch array, and it keeps the
  *    last call's contents (nothing in it needs to start at zero). Calls
  *    whose kernels overlap on the GPU (different streams without ordering)

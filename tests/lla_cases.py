@@ -151,3 +151,35 @@ def compare_paged(out, lse, ref_out, ref_lse, lens, dtype):
         assert err <= TOL_BF16_REL, f"bf16 relative error {err:.3e} > {TOL_BF16_REL}"
     lse_err = np.abs(l[full] - ref_lse[full]).max()
     return err, lse_err
+
+
+def add_undeclared_pages(inp, extra=2):
+    """Moves the page pool into an allocation with `extra` NaN-filled pages
+    after the declared ones. The calls see only the declared pool (the
+    binding takes num_pages from zk.shape[0]), so a table entry naming one of
+    the extra pages is out of range for the library, yet still lands in
+    allocated memory: if a device check regressed, the test would see NaN
+    output or a wrong status, never an out-of-bounds access. Returns the
+    extra pages' indices."""
+    P = inp["zk"].shape[0]
+    for key in ("zk", "zv"):
+        z = inp[key]
+        full = torch.full((P + extra,) + tuple(z.shape[1:]), float("nan"), dtype=z.dtype,
+                          device=z.device)
+        full[:P] = z
+        inp[key + "_alloc"] = full
+        inp[key] = full[:P]
+    return list(range(P, P + extra))
+
+
+def pad_block_table(inp, bt, fill_page=0):
+    """Installs the [B, max_blocks] table `bt` as the first B rows of a
+    [B + 1, max_blocks] allocation whose last row names `fill_page` (a
+    declared page). A read one block past the end of any row, even the last,
+    then stays inside the allocation and names a real page."""
+    B, mb = bt.shape
+    full = np.full((B + 1, mb), fill_page, dtype=np.int32)
+    full[:B] = bt
+    t = torch.from_numpy(full).to(inp["q"].device)
+    inp["block_table_alloc"] = t
+    inp["block_table"] = t[:B]

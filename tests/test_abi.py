@@ -234,3 +234,34 @@ def test_selftest_rejects_bad_timeouts_on_the_host():
     h = lla.lib()
     assert h.lla_selftest_wait_timeout(0, None) == _lib.LLA_ERR_INVALID_ARG
     assert h.lla_selftest_wait_timeout(2000000, None) == _lib.LLA_ERR_INVALID_ARG
+
+
+_NOALLOC_REJECT = r"""
+import ctypes, sys
+sys.path.insert(0, sys.argv[1])
+import decode_attention_encode_b200 as lla
+from decode_attention_encode_b200 import _lib
+# 512 sequences x 16 heads with r = 128 need over 4 MiB for the absorbed
+# queries alone
+need = lla.lla_decode_attn_workspace(512, 16, 1, 128, 128)
+assert need > 4 << 20, need
+fake = ctypes.c_void_p(0x100000)
+st = lla.lib().lla_decode_attn_noalloc(fake, fake, fake, 1, 512, 16, 128, 1, 1, 128, 128,
+                                       fake, fake, None, None, 0.1, fake, None, None)
+assert st == _lib.LLA_ERR_WORKSPACE, st
+assert b"scratch" in lla.lib().lla_last_error()
+print("rejected")
+"""
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch_before_launching():
+    # Runs in a child process with no visible CUDA device, so the fake
+    # pointers can never reach a kernel whatever the machine: the call must
+    # return LLA_ERR_WORKSPACE from its host-side size check.
+    import subprocess
+    import sys
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    res = subprocess.run([sys.executable, "-c", _NOALLOC_REJECT, ROOT], env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stdout + res.stderr
+    assert "rejected" in res.stdout

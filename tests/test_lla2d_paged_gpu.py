@@ -14,7 +14,7 @@ import torch
 
 import decode_attention_encode_b200 as lla
 from decode_attention_encode_b200 import synth
-from lla_cases import TOL_BF16_REL, to_f64
+from lla_cases import TOL_BF16_REL, add_undeclared_pages, pad_block_table, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -96,11 +96,16 @@ def test_many_short_and_one_long_sequence():
 
 
 def test_bad_lengths_and_pages_are_rejected_on_the_device():
+    # Planted errors stay inside allocated memory: sequence 1 names a page
+    # past the declared pool that is allocated (add_undeclared_pages), and
+    # sequence 2, the table's last row, is one token longer than its table
+    # row, whose next entry lies in the padding row (pad_block_table).
     lens = [300, 400, 500]
     inp = make(lens, 16, 64, 128, 128, 128, seed=4)
+    extra = add_undeclared_pages(inp)
     bt = inp["block_table"].cpu().numpy()
-    bt[1, 1] = inp["zk"].shape[0] + 5
-    inp["block_table"] = torch.from_numpy(bt).cuda()
+    bt[1, 1] = extra[1]
+    pad_block_table(inp, bt)
     inp["seq_lens"] = torch.tensor([300, 400, bt.shape[1] * 128 + 1], dtype=torch.int32,
                                    device="cuda")
     lla.device_status(clear=True)
@@ -149,7 +154,11 @@ def test_sink_window_eviction(sink, window, page_size):
     import oracle  # test infrastructure only
     lens = [3000, 260, 261, 1, 0, 9000, 257, 700]
     inp = make(lens, 16, 128, 256, 256, page_size, mu=True, seed=sink + window)
-    # pages holding no kept token: invalid table entries and NaN latents
+    # Pages holding no kept token: NaN latents, and table entries that name a
+    # page past the declared pool (allocated and NaN-filled by
+    # add_undeclared_pages), so reading or checking them fails the test
+    # without leaving the allocation.
+    extra = add_undeclared_pages(inp)
     bt = inp["block_table"].cpu().numpy()
     for b, n in enumerate(lens):
         kept_blocks = set((oracle.kept_positions(n, sink, window) // page_size).tolist())
@@ -157,7 +166,7 @@ def test_sink_window_eviction(sink, window, page_size):
             if blk not in kept_blocks:
                 inp["zk"][int(bt[b, blk])] = float("nan")
                 inp["zv"][int(bt[b, blk])] = float("nan")
-                bt[b, blk] = -7
+                bt[b, blk] = extra[blk % len(extra)]
     inp["block_table"] = torch.from_numpy(bt).cuda()
     out, lse = run(inp, sink, window)
     torch.cuda.synchronize()

@@ -4,7 +4,8 @@ against the fp64 oracle, through the C ABI.
 Cases: ragged length mixes (1 token, page-boundary lengths, empty
 sequences), page sizes that do and do not divide the stage tile, both latent
 types and several ranks, the attention-sink + window eviction set (with the
-table entries of evicted blocks invalid and their pages NaN), device-side
+table entries of evicted blocks out of the declared pool and their pages
+NaN), device-side
 rejection of bad lengths and page indices, agreement with the dense kernel
 on a dense-equivalent layout, and a full-size ragged batch."""
 
@@ -14,7 +15,8 @@ import torch
 
 import decode_attention_encode_b200 as lla
 from decode_attention_encode_b200 import synth
-from lla_cases import compare_paged, make_paged_inputs, oracle_paged_reference, to_f64
+from lla_cases import (add_undeclared_pages, compare_paged, make_paged_inputs,
+                       oracle_paged_reference, pad_block_table, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -70,8 +72,12 @@ def test_sink_window_eviction(sink, window):
     lens = [1000, 260, 261, 3, 0, 4000, 257]
     ps = 32
     inp = make_paged_inputs(lens, 3, 64, 24, 24, BF16, ps, mu=True, seed=sink + window)
-    # blocks that hold no kept token: invalid table entries and NaN pages
+    # Blocks that hold no kept token: their pages become NaN and their table
+    # entries name a page past the declared pool (out of range for the call,
+    # but allocated and NaN-filled by add_undeclared_pages), so reading or
+    # checking an evicted block fails the test without leaving the allocation.
     import oracle
+    extra = add_undeclared_pages(inp)
     bt = inp["block_table"].cpu().numpy()
     for b, n in enumerate(lens):
         kept = set((oracle.kept_positions(n, sink, window) // ps).tolist())
@@ -79,21 +85,29 @@ def test_sink_window_eviction(sink, window):
             if blk not in kept:
                 inp["zk"][int(bt[b, blk])] = float("nan")
                 inp["zv"][int(bt[b, blk])] = float("nan")
-                bt[b, blk] = -7
+                bt[b, blk] = extra[blk % len(extra)]
     inp["block_table"] = torch.from_numpy(bt).cuda()
     out, lse = run_paged(inp, BF16, sink=sink, window=window)
     assert torch.isfinite(out).all()
 
 
 def test_bad_lengths_and_pages_are_rejected_on_the_device():
+    # Every planted error stays inside allocated memory, so a regressed check
+    # gives a wrong number or status, not an illegal access:
+    # - sequence 1 names a page one past the declared pool, which is an
+    #   allocated NaN page (add_undeclared_pages);
+    # - sequence 3, the table's last row, is one token longer than the table;
+    #   its extra block lies in the padding row of the table's allocation,
+    #   which names declared page 0 (pad_block_table).
+    # A negative length has no in-bounds place to land, so none is planted.
     lens = [40, 50, 60, 70]
     inp = make_paged_inputs(lens, 2, 32, 16, 16, BF16, 16, seed=9)
+    extra = add_undeclared_pages(inp)
     bt = inp["block_table"].cpu().numpy()
-    num_pages = inp["zk"].shape[0]
-    bt[1, 2] = num_pages          # a used block past the pool
-    inp["block_table"] = torch.from_numpy(bt).cuda()
-    sl = torch.tensor([40, 50, bt.shape[1] * 16 + 1, -5], dtype=torch.int32, device="cuda")
-    inp["seq_lens"] = sl
+    bt[1, 2] = extra[0]           # a used block past the declared pool
+    pad_block_table(inp, bt)
+    inp["seq_lens"] = torch.tensor([40, 50, 60, bt.shape[1] * 16 + 1], dtype=torch.int32,
+                                   device="cuda")
     lla.device_status(clear=True)
     out, lse = lla.lla_decode_attn_paged(inp["q"], inp["zk"], inp["zv"], inp["block_table"],
                                          inp["seq_lens"], inp["dk"], inp["dv"])
@@ -101,12 +115,15 @@ def test_bad_lengths_and_pages_are_rejected_on_the_device():
     st = lla.device_status(clear=True)
     assert st & lla._lib.LLA_DEVICE_BAD_PAGED_INPUT
     assert lla.device_status() == 0
-    # sequences 1..3 are treated as empty; sequence 0 is intact
+    # sequences 1 and 3 are treated as empty; sequences 0 and 2 are intact
     o, l = out.cpu(), lse.cpu()
-    assert torch.all(o[1:] == 0) and torch.all(torch.isneginf(l[1:]))
-    inp["seq_lens"] = torch.tensor([40, 0, 0, 0], dtype=torch.int32, device="cuda")
+    for b in (1, 3):
+        assert torch.all(o[b] == 0) and torch.all(torch.isneginf(l[b]))
+    inp["seq_lens"] = torch.tensor([40, 0, 60, 0], dtype=torch.int32, device="cuda")
     ref_out, ref_lse = oracle_paged_reference(inp)
-    np.testing.assert_allclose(to_f64(out)[0], ref_out[0], atol=2e-2 * np.abs(ref_out[0]).max())
+    for b in (0, 2):
+        np.testing.assert_allclose(to_f64(out)[b], ref_out[b],
+                                   atol=2e-2 * np.abs(ref_out[b]).max())
 
 
 def test_dense_equivalent_layout_matches_the_dense_kernel():
