@@ -40,7 +40,7 @@ from decode_attention_encode_b200 import synth  # noqa: E402
 
 METRIC = "LLA decode: cached tokens attended/sec per loop step; HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
-DEFAULT_CONFIG = "perhead_4x"
+DEFAULT_CONFIG = "perhead_21x"
 CSRC = os.path.join(ROOT, "decode_attention_encode_b200", "csrc")
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 ENCODE_CONFIGS = {synth.C5_ENCODE.name: synth.C5_ENCODE}
@@ -419,25 +419,29 @@ def run_encode_bench(args, world, rank, local):
         "e2e": None,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import numpy as np
-
         import oracle
-        K = cfg.T * cfg.d_loop
         n = 512
         x = wl.x[0][:, :n].double().cpu().numpy()
         w = wl.w_t[0].transpose(1, 2).double().cpu().numpy()
         mu = wl.mu[0].double().cpu().numpy()
-        t0 = time.perf_counter()
-        reps = 0
-        while time.perf_counter() - t0 < 10.0:
-            oracle.encode(x, w, mu)
-            reps += 1
-        dt = time.perf_counter() - t0
+        threads = max(1, oracle.max_threads())
+        rates = {}
+        for nt, budget in ((1, 6.0), (threads, 6.0)):
+            t0, reps = time.perf_counter(), 0
+            while True:
+                oracle.encode(x, w, mu, nthreads=nt)
+                reps += 1
+                if time.perf_counter() - t0 >= budget:
+                    break
+            rates[nt] = reps * n / (2 * cfg.L) / (time.perf_counter() - t0)
         line["cpu_baseline"] = {
-            "value": reps * n / (2 * cfg.L) / dt, "unit": "tokens/s",
-            "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"{reps} x {n} tokens of one (layer, axis) call in fp64; "
-                      f"tokens/s divides by the {2 * cfg.L} calls of a step"}
+            "value": rates[threads], "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} tokens of one (layer, axis) call in fp64, repeated; tokens/s "
+                      f"divides by the {2 * cfg.L} calls of a step",
+            "single_thread": {"value": rates[1], "threads": 1},
+            "all_cores": {"value": rates[threads], "threads": threads,
+                          "parallel": "OpenMP over (group, token)"},
+            **host_cores()}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -467,42 +471,170 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
-# CPU baseline: the fp64 oracle on a bounded sample
+# CPU baseline: the fp64 oracle on a fixed sample of decode units
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(cfg: synth.DecodeConfig, budget_s: float = 15.0):
-    """Times the oracle, as it stands, on whole (b, h) units of one
-    (layer, loop) step of this workload. Returns (tokens/s, cores, sample)."""
+def host_cores():
+    """os.cpu_count(), the CPUs this process may run on, and nproc's answer."""
+    try:
+        nproc = int(subprocess.run(["nproc"], capture_output=True, text=True,
+                                   timeout=10).stdout.strip())
+    except Exception:
+        nproc = None
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except Exception:
+        usable = None
+    return {"os_cpu_count": os.cpu_count(), "usable": usable, "nproc": nproc}
+
+
+def unit_tokens(cfg: synth.DecodeConfig, units) -> float:
+    """Cached tokens a sample of (b, layer, loop, h) units stands for: a
+    (layer, loop) step attends each sequence's tokens once over all H heads,
+    so a unit is N_b / H of them."""
+    lens = cfg.lengths()
+    return float(sum(int(lens[b]) for b, _, _, _ in units)) / cfg.H
+
+
+def draw_unit_inputs(cfg: synth.DecodeConfig, units, seed: int = 0):
+    """Host fp64 inputs of each sampled unit drawn with the workload's
+    recipes (the reference arm has no device store to read from)."""
+    lens = cfg.lengths()
+    out = []
+    for i, (b, l, t, h) in enumerate(units):
+        n, s = int(lens[b]), seed + 10 * i
+        f = lambda x: x.double().numpy()
+        u = dict(q=f(synth.queries((cfg.d_h,), cfg.d_h, s)),
+                 zk=f(synth.latents((n, cfg.r_k), s + 1, decay=cfg.decay, dtype=cfg.torch_dtype)),
+                 zv=f(synth.latents((n, cfg.r_v), s + 2, decay=cfg.decay, dtype=cfg.torch_dtype)),
+                 dk=f(synth.orthonormal(1, cfg.d_h, cfg.r_k, s + 3)[0]),
+                 dv=f(synth.orthonormal(1, cfg.d_h, cfg.r_v, s + 4)[0]))
+        if cfg.d_r:
+            u["q_rope"] = f(synth.queries((cfg.d_r,), cfg.d_r, s + 5))
+            u["k_rope"] = f(synth.latents((n, cfg.d_r), s + 6, dtype=cfg.torch_dtype))
+        out.append(u)
+    return out
+
+
+def gather_unit_inputs(wl, units):
+    """Host fp64 copies of each sampled unit's device inputs (its query, its
+    own latent rows, this loop's decoders), read from the benchmark's store."""
+    c = wl.cfg
+    lens = c.lengths()
+    f = lambda x: x.double().cpu().numpy()
+    out = []
+    for b, l, t, h in units:
+        n = int(lens[b])
+        if wl.paged:
+            pos = torch.arange(n, device=wl.block_table.device)
+            pages = wl.block_table[b, pos // c.page_size].long()
+            rows = pos % c.page_size
+            zk = wl.zk[l][pages, rows] if c.two_d else wl.zk[l][pages, h, rows]
+            zv = wl.zv[l][pages, rows] if c.two_d else wl.zv[l][pages, h, rows]
+        elif c.two_d:
+            zk, zv = wl.zk[l][b, :n], wl.zv[l][b, :n]
+        else:
+            zk, zv = wl.zk[l][b, h, :n], wl.zv[l][b, h, :n]
+        u = dict(q=f(wl.q[l, t, b, h]), zk=f(zk[:, :c.r_k]), zv=f(zv), dk=f(wl.dk[l, t, h]),
+                 dv=f(wl.dv[l, t, h]))
+        if c.d_r:
+            u["q_rope"] = f(wl.q_rope[l, t, b, h])
+            u["k_rope"] = f(zk[:, c.r_k:])
+        out.append(u)
+    return out
+
+
+def run_oracle_units(cfg: synth.DecodeConfig, inputs, threads: int):
+    """The oracle, as it stands, on every unit of the sample with `threads`
+    host threads. Units of one length go through the oracle's batched call
+    (OpenMP over units); ragged or rotary samples take one oracle call per
+    unit, spread over a pool of `threads` Python threads (ctypes releases the
+    interpreter lock inside the C code). Returns (out [U, d_h], lse [U])."""
     import numpy as np
 
     import oracle
-    c = cfg
-    threads = oracle.max_threads()
-    rng = np.random.default_rng(0)
-    # one unit's inputs on the host (fp64), drawn with the same recipes
-    zk_shape = (1, c.N, c.r_k)
-    done_units = 0
-    t_total = 0.0
-    batch = max(1, threads)
-    while t_total < budget_s and done_units < 4096:
-        seed = int(rng.integers(1 << 30))
-        zk = synth.latents((batch,) + zk_shape[1:], seed, "cpu", decay=c.decay,
-                           dtype=c.torch_dtype).double().numpy()
-        zv = synth.latents((batch, c.N, c.r_v), seed + 1, "cpu", decay=c.decay,
-                           dtype=c.torch_dtype).double().numpy()
-        dk = synth.orthonormal(batch, c.d_h, c.r_k, seed + 2).double().numpy()
-        dv = synth.orthonormal(batch, c.d_h, c.r_v, seed + 3).double().numpy()
-        q = synth.queries((batch, c.d_h), c.d_h, seed + 4).double().numpy()
+    scale = 1.0 / math.sqrt(cfg.d_h)
+    uniform = not cfg.page_size and not cfg.d_r
+    if uniform:
+        st = lambda k: np.stack([u[k] for u in inputs])
+        return oracle.decode_units(st("q"), st("zk"), st("zv"), st("dk"), st("dv"), scale=scale,
+                                   nthreads=threads)
+
+    def one(u):
+        if cfg.d_r:
+            return oracle.decode_unit_rope(u["q"], u["q_rope"], u["zk"], u["k_rope"], u["zv"],
+                                           u["dk"], u["dv"], scale=scale)
+        o, l = oracle.decode_units(u["q"][None], u["zk"][None], u["zv"][None], u["dk"][None],
+                                   u["dv"][None], scale=scale, nthreads=1)
+        return o[0], float(l[0])
+
+    if threads <= 1:
+        res = [one(u) for u in inputs]
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            res = list(ex.map(one, inputs))
+    return np.stack([r[0] for r in res]), np.array([r[1] for r in res])
+
+
+def oracle_rates(cfg: synth.DecodeConfig, units, inputs, single_budget_s: float = 8.0,
+                 all_budget_s: float = 5.0):
+    """Times the oracle on the fixed sample: single-threaded on the longest
+    prefix of the sample that fits the budget (at least one unit), and on all
+    host threads over the whole sample, repeated for about `all_budget_s`.
+    Returns (all-core rate, record, all-core outputs)."""
+    import oracle
+    threads = max(1, oracle.max_threads())  # read before any call changes it
+    t0 = time.perf_counter()
+    run_oracle_units(cfg, inputs[:1], 1)
+    t1 = time.perf_counter() - t0
+    k = max(1, min(len(units), int(single_budget_s / max(t1, 1e-6))))
+    if k > 1:
         t0 = time.perf_counter()
-        oracle.decode_units(q, zk, zv, dk, dv, scale=1.0 / math.sqrt(c.d_h))
-        t_total += time.perf_counter() - t0
-        done_units += batch
-    # a (layer, loop) step attends B*N cached tokens over H heads: one unit
-    # is N/H of those tokens' worth of work
-    tokens = done_units * c.N / c.H
-    sample = (f"{done_units} (b,h) units of one (layer, loop) step, {c.N} tokens each, "
-              f"explicit K/V reconstruction in fp64; tokens/s counts N/H tokens per unit")
-    return tokens / t_total, threads, sample
+        run_oracle_units(cfg, inputs[:k], 1)
+        t1 = time.perf_counter() - t0
+    single = unit_tokens(cfg, units[:k]) / t1
+    # whole passes over the sample until about `all_budget_s` have passed
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        res = run_oracle_units(cfg, inputs, threads)
+        passes += 1
+        if time.perf_counter() - t0 >= all_budget_s:
+            break
+    tall = (time.perf_counter() - t0) / passes
+    rate = unit_tokens(cfg, units) / tall
+    cores = host_cores()
+    rec = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "sample": f"{len(units)} (b, layer, loop, h) units of this workload (32 seeded-random "
+                     f"units plus the 16 corners, repeats removed), "
+                     f"{'ragged lengths, ' if cfg.page_size else ''}"
+                     f"explicit K/V reconstruction then textbook softmax in fp64; tokens/s "
+                     f"counts N_b/H cached tokens per unit",
+           "all_cores": {"value": rate, "threads": threads, "units_timed": len(units),
+                         "seconds_per_pass": tall, "passes": passes,
+                         "parallel": "OpenMP over units" if not cfg.page_size and not cfg.d_r
+                         else "one oracle call per unit on a thread pool"},
+           "single_thread": {"value": single, "threads": 1, "units_timed": k, "seconds": t1},
+           **cores}
+    return rate, rec, res
+
+
+def cpu_baseline(wl):
+    """The oracle timed on the fixed sample of the benchmark's own store, and
+    that sample's GPU outputs checked against it."""
+    import numpy as np
+    c = wl.cfg
+    units = synth.sample_units(c.B, c.L, c.T, c.H)
+    inputs = gather_unit_inputs(wl, units)
+    rate, rec, (ref_o, ref_l) = oracle_rates(c, units, inputs)
+    idx = [list(x) for x in zip(*[(l, t, b, h) for b, l, t, h in units])]
+    got = wl.out[idx[0], idx[1], idx[2], idx[3]].double().cpu().numpy()
+    got_l = wl.lse[idx[0], idx[1], idx[2], idx[3]].double().cpu().numpy()
+    err = float(np.abs(got - ref_o).max() / np.abs(ref_o).max())
+    rec["parity"] = {"units": len(units), "max_rel_err": err,
+                     "lse_max_abs_err": float(np.abs(got_l - ref_l).max()),
+                     "tolerance": "max|o_gpu - o_ref| / max|o_ref| <= 2e-2"}
+    return rate, rec
 
 
 # ---------------------------------------------------------------------------
@@ -510,31 +642,41 @@ def cpu_baseline(cfg: synth.DecodeConfig, budget_s: float = 15.0):
 # ---------------------------------------------------------------------------
 
 def run_reference(args, world, rank):
+    """The oracle arm: each step is one all-core pass of the oracle over the
+    fixed 48-unit sample of the workload (inputs drawn on the host with the
+    workload's recipes); ms_per_step is that pass's measured wall time."""
     if rank != 0:
         return
     if args.config in ENCODE_CONFIGS:
         print(json.dumps({"impl": "reference", "unavailable":
                           "the reference arm times the decode workloads only"}), flush=True)
         return
+    import oracle
     cfg = synth.DECODE_CONFIGS[args.config]
-    per_step = []
+    units = synth.sample_units(cfg.B, cfg.L, cfg.T, cfg.H)
+    inputs = draw_unit_inputs(cfg, units)
+    threads = max(1, oracle.max_threads())
+    _, rec, _ = oracle_rates(cfg, units, inputs)
     for _ in range(args.warmup):
-        cpu_baseline(cfg, budget_s=2.0)
-    cores = 1
-    sample = ""
+        run_oracle_units(cfg, inputs, threads)
+    step_s = []
     for _ in range(args.steps):
-        v, cores, sample = cpu_baseline(cfg, budget_s=10.0)
-        per_step.append(v)
-    value = sum(per_step) / len(per_step)
-    tokens_per_step = cfg.B * cfg.N * cfg.L * cfg.T
+        t0 = time.perf_counter()
+        run_oracle_units(cfg, inputs, threads)
+        step_s.append(time.perf_counter() - t0)
+    mean_s = sum(step_s) / len(step_s)
+    value = unit_tokens(cfg, units) / mean_s
+    rec.update({"value": value, "all_cores": dict(rec["all_cores"], value=value,
+                                                  seconds_per_pass=mean_s, passes=args.steps)})
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * tokens_per_step / value, "higher_is_better": True,
+        "ms_per_step": 1e3 * mean_s, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": describe(cfg), "parallelism": "cpu"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "config": {"workload": describe(cfg), "parallelism": f"cpu ({threads} threads)",
+                   "step": f"one all-core oracle pass over the fixed sample of {len(units)} "
+                           "(b, layer, loop, h) units (a bounded sample of the decode step)"},
+        "cpu_baseline": rec,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -718,9 +860,7 @@ def run_lla(args, world, rank, local):
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = cpu_baseline(cfg)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        _, line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
 

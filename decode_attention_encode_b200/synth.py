@@ -217,3 +217,23 @@ C4_PAGED64 = DecodeConfig("lla2d_32x_paged64", L=24, T=4, H=16, d_h=128, r_k=256
                           N=8192, dtype="bf16", decay=True, two_d=True, page_size=64, spread=0.5)
 DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE, C4_PAGED,
                                       C4_PAGED64)}
+
+
+def sample_units(B: int, L: int, T: int, H: int, n_random: int = 32, seed: int = 0):
+    """The fixed sample of (b, layer, loop, h) decode units on which the
+    CPU baseline times the oracle: ``n_random`` seeded-random units, then the
+    16 corners (each index at its first or last value), without repeats."""
+    r = np.random.default_rng(seed)
+    units = [(int(r.integers(B)), int(r.integers(L)), int(r.integers(T)), int(r.integers(H)))
+             for _ in range(n_random)]
+    for b in (0, B - 1):
+        for l in (0, L - 1):
+            for t in (0, T - 1):
+                for h in (0, H - 1):
+                    units.append((b, l, t, h))
+    seen, out = set(), []
+    for u in units:
+        if u not in seen:
+            seen.add(u)
+            out.append(u)
+    return out

@@ -89,7 +89,7 @@ def _load():
             lib.oracle_decode_units.argtypes = ([ctypes.c_int] * 5 + [_dp] * 7 +
                                                 [ctypes.c_double, _dp, _dp, ctypes.c_int])
             lib.oracle_decode_units.restype = ctypes.c_int
-            lib.oracle_encode.argtypes = [ctypes.c_int] * 5 + [_dp] * 4
+            lib.oracle_encode.argtypes = [ctypes.c_int] * 5 + [_dp] * 4 + [ctypes.c_int]
             lib.oracle_encode.restype = None
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = ctypes.c_int
@@ -438,16 +438,18 @@ def paged2d_decode(q, zk_pages, zv_pages, block_table, seq_lens, dk, dv, mu_k=No
 # encode and codec initialisation
 # --------------------------------------------------------------------------
 
-def encode(x, w, mu=None):
+def encode(x, w, mu=None, nthreads: int = 0):
     """Latent write, Eq. 2: x [T, N, G, d_loop] loop-major; w [G, T*d_loop, r];
-    mu [G, T*d_loop] or None. Returns z [G, N, r]."""
+    mu [G, T*d_loop] or None. Returns z [G, N, r]. ``nthreads`` > 0 sets the
+    OpenMP thread count (as for ``decode_units``)."""
     x, w = _f64(x), _f64(w)
     mu = None if mu is None else _f64(mu)
     T, N, G, d_loop = x.shape
     r = w.shape[2]
     assert w.shape == (G, T * d_loop, r)
     z = np.zeros((G, N, r))
-    _load().oracle_encode(T, N, G, d_loop, r, _ptr(x), _ptr(w), _ptr(mu), _ptr(z))
+    _load().oracle_encode(T, N, G, d_loop, r, _ptr(x), _ptr(w), _ptr(mu), _ptr(z),
+                          int(nthreads))
     return z
 
 

@@ -195,12 +195,14 @@ int oracle_max_threads(void)
  *   mu   [G][T*d_loop] or NULL
  *   z    [G][N][r]
  * z[g][n][c] = sum_k (x_stack[k] - mu[g][k]) * w[g][k][c], where
- * x_stack[t*d_loop + i] = x[t][n][g][i] (Eq. 1). */
+ * x_stack[t*d_loop + i] = x[t][n][g][i] (Eq. 1). nthreads > 0 sets the
+ * OpenMP thread count; otherwise the runtime default is kept. */
 void oracle_encode(int T, int N, int G, int d_loop, int r, const double *x,
-                   const double *w, const double *mu, double *z)
+                   const double *w, const double *mu, double *z, int nthreads)
 {
     const size_t K = (size_t)T * d_loop;
 #ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
 #pragma omp parallel for collapse(2) schedule(static)
 #endif
     for (int g = 0; g < G; ++g) {
