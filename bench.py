@@ -43,7 +43,7 @@ UNIT = "tokens/s"
 DEFAULT_CONFIG = "perhead_21x"
 CSRC = os.path.join(ROOT, "decode_attention_encode_b200", "csrc")
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-ENCODE_CONFIGS = {synth.C5_ENCODE.name: synth.C5_ENCODE}
+ENCODE_CONFIGS = synth.ENCODE_CONFIGS
 
 
 def main_kernel(config_name: str):
@@ -57,6 +57,12 @@ def main_kernel(config_name: str):
     return "k_stream", os.path.join(CSRC, "stream.cu")
 
 
+def with_layers(cfg, layers: int):
+    """The workload with `layers` layers (0: its own count)."""
+    import dataclasses
+    return dataclasses.replace(cfg, L=layers) if layers > 0 else cfg
+
+
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=int(os.environ.get("WORLD_SIZE", "1")))
@@ -65,6 +71,9 @@ def parse_args():
     p.add_argument("--config", default=DEFAULT_CONFIG,
                    choices=sorted(synth.DECODE_CONFIGS) + sorted(ENCODE_CONFIGS))
     p.add_argument("--impl", default="lla", choices=["lla", "reference"])
+    p.add_argument("--layers", type=int, default=0,
+                   help="run the workload with this many layers instead of its own (a smaller "
+                        "case for profiler captures; the JSON line names the layer count)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -181,18 +190,17 @@ class DecodeWorkload:
     """All layers' latent stores, decoders and queries of one config on the
     device. The 2-D config keeps one latent per token and layer.
 
-    Per-head configs also carry the latent write of each sequence's newest
+    The step also carries the latent write of each sequence's newest
     token: after the T x L attention calls, the token's stacked per-loop K
-    and V of every layer are encoded into slot N of the store (the attended
-    range stays [0, N), so every step measures the same context).
+    and V of every layer are encoded into the slot after the attended range
+    (position N_b), so every step measures the same context.
 
     A paged config keeps each layer's store as a pool of pages with one
-    shared block table and seeded ragged lengths; its step is the T x L
-    attention calls alone (a newest-token write there is a scatter into
-    each sequence's last page, which this workload does not time). A rotary
-    config stores [latent | rotated rotary key] key rows and takes one
-    rotary query per (layer, loop) call; its step is the attention calls
-    alone as well."""
+    shared block table and seeded ragged lengths; the table covers position
+    N_b too, and the newest token goes there through lla_encode_paged (its
+    page looked up on the device). A rotary config stores [latent | rotated
+    rotary key] key rows and takes one rotary query per (layer, loop) call;
+    its step is the attention calls alone."""
 
     def __init__(self, cfg: synth.DecodeConfig, device: str, seed_offset: int = 0):
         self.cfg = cfg
@@ -200,14 +208,15 @@ class DecodeWorkload:
         s = c.seed + seed_offset
         self.paged = c.page_size > 0
         self.rope = c.d_r > 0
-        self.write_latents = (not self.paged and not self.rope and c.dtype == "bf16"
-                              and c.d_h % 64 == 0)
+        self.write_latents = not self.rope and c.dtype == "bf16" and c.d_h % 64 == 0
         n_cap = c.N + 1 if self.write_latents else c.N
-        zk_shape = (c.B, n_cap, c.r_k) if c.two_d else (c.B, c.H, n_cap, c.r_k + c.d_r)
+        zk_shape = (c.B, n_cap, c.r_k + c.d_r) if c.two_d else (c.B, c.H, n_cap, c.r_k + c.d_r)
         zv_shape = (c.B, n_cap, c.r_v) if c.two_d else (c.B, c.H, n_cap, c.r_v)
         if self.paged:
             lens = c.lengths()
-            bt, num_pages = synth.page_table(lens, c.page_size, s + 12)
+            # the table also covers position N_b, where the newest token goes
+            bt, num_pages = synth.page_table(lens + 1 if self.write_latents else lens,
+                                             c.page_size, s + 12)
             self.block_table = torch.from_numpy(bt).to(device)
             self.seq_lens = torch.from_numpy(lens).to(device)
             zk_shape = ((num_pages, c.page_size, c.r_k) if c.two_d
@@ -234,7 +243,8 @@ class DecodeWorkload:
                     else lla.lla_decode_attn_paged_workspace)
             need = wsfn(c.B, c.H, c.r_k, c.r_v)
         elif self.rope:
-            need = lla.lla_decode_attn_workspace(c.B, c.H, c.N, c.r_k + c.d_r, c.r_v)
+            wsfn = lla.lla2d_decode_attn_workspace if c.two_d else lla.lla_decode_attn_workspace
+            need = wsfn(c.B, c.H, c.N, c.r_k + c.d_r, c.r_v)
         else:
             wsfn = lla.lla2d_decode_attn_workspace if c.two_d else lla.lla_decode_attn_workspace
             need = wsfn(c.B, c.H, c.N, c.r_k, c.r_v)
@@ -274,11 +284,25 @@ class DecodeWorkload:
         q = self.q if q is None else q
         out = self.out if out is None else out
         lse = self.lse if lse is None else lse
+        self.plan()
         for t in range(c.T):
             for l in range(c.L):
                 self.call(l, t, q, out, lse)
         if self.write_latents:
             self.write_newest(self.xk if xk is None else xk, self.xv if xv is None else xv)
+
+    def plan(self):
+        """A paged store's step plan, made once: every (layer, loop) call of
+        the step attends the same lengths through the same table."""
+        if not self.paged:
+            return
+        c = self.cfg
+        if c.two_d:
+            self.lla.lla2d_decode_attn_paged_plan(self.zk[0], self.zv[0], self.block_table,
+                                                  self.seq_lens, c.H, self.ws)
+        else:
+            self.lla.lla_decode_attn_paged_plan(self.zk[0], self.zv[0], self.block_table,
+                                                self.seq_lens, self.ws)
 
     def call(self, l, t, q=None, out=None, lse=None, q_rope=None):
         """The (layer l, loop t) decode call through the public API."""
@@ -287,25 +311,32 @@ class DecodeWorkload:
         q_rope = getattr(self, "q_rope", None) if q_rope is None else q_rope
         out = self.out if out is None else out
         lse = self.lse if lse is None else lse
-        if self.paged:
+        if self.paged:  # on the step's plan (plan())
             fn = self.lla.lla2d_decode_attn_paged if c.two_d else self.lla.lla_decode_attn_paged
             fn(q[l, t], self.zk[l], self.zv[l], self.block_table, self.seq_lens, self.dk[l, t],
-               self.dv[l, t], scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
+               self.dv[l, t], scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws,
+               planned=True)
         elif self.rope:
-            self.lla.lla_decode_attn_rope(q[l, t], q_rope[l, t], self.zk[l], self.zv[l],
-                                          self.dk[l, t], self.dv[l, t], N=c.N, scale=self.scale,
-                                          out=out[l, t], lse=lse[l, t], workspace=self.ws)
+            fn = self.lla.lla2d_decode_attn_rope if c.two_d else self.lla.lla_decode_attn_rope
+            fn(q[l, t], q_rope[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
+               scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
         else:
             self.fn(q[l, t], self.zk[l], self.zv[l], self.dk[l, t], self.dv[l, t], N=c.N,
                     scale=self.scale, out=out[l, t], lse=lse[l, t], workspace=self.ws)
 
     def write_newest(self, xk, xv):
-        """Each sequence's newest token into slot N of every layer's store."""
+        """Each sequence's newest token into position N_b of every layer's
+        store (slot N of a dense store; through the block table of a paged
+        one)."""
         c = self.cfg
         for l in range(c.L):
             for x, w, muw, z, r in ((xk, self.wk, self.muwk, self.zk, c.r_k),
                                     (xv, self.wv, self.muwv, self.zv, c.r_v)):
-                if c.two_d:  # x [T][B][H][d_h] read as [T][B][1][H d_h]
+                xs = x[l].view(c.T, c.B, 1, c.H * c.d_h) if c.two_d else x[l]
+                if self.paged:
+                    self.lla.lla_encode_paged(xs, w[l], muw[l], z[l], self.block_table,
+                                              self.seq_lens, workspace=self.enc_ws)
+                elif c.two_d:  # x [T][B][H][d_h] read as [T][B][1][H d_h]
                     self.lla.lla_encode_with_bias(
                         x[l].view(c.T, c.B, 1, c.H * c.d_h), w[l], muw[l], z=z[l][:, c.N],
                         z_row_stride=self.n_cap * r, z_group_stride=0, workspace=self.enc_ws)
@@ -315,7 +346,7 @@ class DecodeWorkload:
                         z_group_stride=self.n_cap * r, workspace=self.enc_ws)
 
     def launches_per_step(self) -> int:
-        n = (4 if self.paged else 3) * self.cfg.L * self.cfg.T
+        n = 3 * self.cfg.L * self.cfg.T + (1 if self.paged else 0)
         if self.write_latents:
             n += (4 if self.enc_split else 2) * self.cfg.L
         return n
@@ -363,7 +394,7 @@ class EncodeWorkload:
 
 
 def run_encode_bench(args, world, rank, local):
-    cfg = ENCODE_CONFIGS[args.config]
+    cfg = with_layers(ENCODE_CONFIGS[args.config], args.layers)
     dev = f"cuda:{local}"
     wl = EncodeWorkload(cfg, dev, seed_offset=rank)
     stream = torch.cuda.current_stream()
@@ -394,8 +425,12 @@ def run_encode_bench(args, world, rank, local):
     kern_ms = sum(kern) / len(kern)
     call_bytes = (cfg.T * cfg.N * cfg.G * cfg.d_loop + cfg.G * cfg.N * cfg.r) * 2
     hbm_peak, peak_src = peaks()
+    tc_peak, tc_src = tensor_peak()
     achieved = call_bytes / (kern_ms * 1e-3) / 1e9
     flops = 2 * cfg.N * cfg.G * cfg.T * cfg.d_loop * cfg.r
+    tflops = flops / (kern_ms * 1e-3) / 1e12
+    # which roof binds: the arithmetic intensity against the ridge point
+    tensor_bound = flops / call_bytes > tc_peak * 1e12 / (hbm_peak * 1e9)
     line = {
         "metric": "LLA encode: prefill tokens encoded/sec (every layer, K and V)",
         "value": aggregate_rate(cfg.N, ms_per_step, world), "unit": "tokens/s", "n_gpus": world,
@@ -407,17 +442,22 @@ def run_encode_bench(args, world, rank, local):
                    "step": f"{2 * cfg.L} encode calls", "accumulation": "fp32",
                    "l2": "no flush: each call reads 0.54 GB of fresh input",
                    "parallelism": f"dp{world} (independent sequences per GPU)"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": profiled_traffic(cfg.name),
-                     "kernel": "k_encode", "kernel_ms_mean": kern_ms,
-                     "algorithmic_bytes_per_launch": call_bytes,
-                     "tensor_tflops": flops / (kern_ms * 1e-3) / 1e12,
-                     "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs (copy, burst)"
-                     if peak_src == "measured" else "fallback 6.65 TB/s"},
+        "roofline": ({"bound": "tensor", "achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                      "frac": tflops / tc_peak, "hbm_gbs": achieved, "hbm_frac": achieved / hbm_peak,
+                      "peak_source": tc_src}
+                     if tensor_bound else
+                     {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                      "frac": achieved / hbm_peak, "tensor_tflops": tflops,
+                      "tensor_frac": tflops / tc_peak,
+                      "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs (copy, burst)"
+                      if peak_src == "measured" else "fallback 6.65 TB/s"}),
         "gpu_launches": wl.launches_per_step() * args.steps,
         "clocks": clk,
         "e2e": None,
     }
+    line["roofline"].update({"traffic": profiled_traffic(cfg.name), "kernel": "k_encode",
+                             "kernel_ms_mean": kern_ms, "algorithmic_bytes_per_launch": call_bytes,
+                             "algorithmic_flops_per_launch": flops})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         n = 512
@@ -460,6 +500,17 @@ def profiled_traffic(config_name: str):
     if not h or not t or h.group(1) != cur:
         return None
     return float(t.group(1))
+
+
+def tensor_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s): the measured burst figure,
+    since one encode launch is timed alone."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured: MEASURED_PEAKS.json bf16_tflops (burst)"
+    return 1590.0, "fallback 1.59 PFLOP/s (burst)"
 
 
 def peaks():
@@ -652,7 +703,7 @@ def run_reference(args, world, rank):
                           "the reference arm times the decode workloads only"}), flush=True)
         return
     import oracle
-    cfg = synth.DECODE_CONFIGS[args.config]
+    cfg = with_layers(synth.DECODE_CONFIGS[args.config], args.layers)
     units = synth.sample_units(cfg.B, cfg.L, cfg.T, cfg.H)
     inputs = draw_unit_inputs(cfg, units)
     threads = max(1, oracle.max_threads())
@@ -692,7 +743,7 @@ def describe(cfg: synth.DecodeConfig) -> str:
 
 
 def run_lla(args, world, rank, local):
-    cfg = synth.DECODE_CONFIGS[args.config]
+    cfg = with_layers(synth.DECODE_CONFIGS[args.config], args.layers)
     dev = f"cuda:{local}"
     wl = DecodeWorkload(cfg, dev, seed_offset=rank)
     stream = torch.cuda.current_stream()
@@ -714,6 +765,7 @@ def run_lla(args, world, rank, local):
         if k == args.steps - 1:
             # time each whole call of the last step's first loop on its own
             c = cfg
+            wl.plan()
             for t in range(c.T):
                 for l in range(c.L):
                     if t == 0:
@@ -794,6 +846,9 @@ def run_lla(args, world, rank, local):
                 for d_, h_ in zip(x_devs, x_hosts):
                     d_.copy_(h_, non_blocking=True)
                 x_ev.record(h2d)
+            if wl.paged:  # the step's plan reads the lengths and table just copied
+                stream.wait_event(in_ev[0][0])
+                wl.plan()
             for t in range(c.T):
                 for l in range(c.L):
                     stream.wait_event(in_ev[t][l])
@@ -834,8 +889,8 @@ def run_lla(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": describe(cfg),
-            "step": f"{cfg.L * cfg.T} decode calls (T loops x L layers), "
-                    f"{4 if wl.paged else 3} kernels each"
+            "step": (f"one plan kernel, then " if wl.paged else "")
+                    + f"{cfg.L * cfg.T} decode calls (T loops x L layers), 3 kernels each"
                     + (f", then {2 * cfg.L} latent writes of the newest token" if wl.write_latents else ""),
             "accumulation": "fp32",
             "l2": "no flush: each layer's latent store "

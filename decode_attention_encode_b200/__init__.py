@@ -18,17 +18,22 @@ from ._lib import (  # noqa: F401
     library_path,
     lla2d_decode_attn,
     lla2d_decode_attn_paged,
+    lla2d_decode_attn_paged_plan,
+    lla2d_decode_attn_paged_planned,
     lla2d_decode_attn_paged_workspace,
     lla2d_decode_attn_rope,
     lla2d_decode_attn_workspace,
     lla_decode_attn,
     lla_decode_attn_noalloc,
     lla_decode_attn_paged,
+    lla_decode_attn_paged_plan,
+    lla_decode_attn_paged_planned,
     lla_decode_attn_paged_workspace,
     lla_decode_attn_rope,
     lla_decode_attn_workspace,
     lla_encode,
     lla_encode_bias,
+    lla_encode_paged,
     lla_encode_with_bias,
     lla_encode_with_bias_workspace_bytes,
     lla_merge_attn,

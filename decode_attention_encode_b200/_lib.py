@@ -28,6 +28,7 @@ LLA_BF16 = 1
 
 LLA_DEVICE_WAIT_TIMEOUT = 0x1
 LLA_DEVICE_BAD_PAGED_INPUT = 0x2
+LLA_DEVICE_PAGED_PLAN_MISMATCH = 0x4
 
 # Every symbol include/lla.h declares.
 EXPORTS = (
@@ -36,9 +37,12 @@ EXPORTS = (
     "lla_decode_attn_workspace", "lla_decode_attn", "lla_decode_attn_noalloc",
     "lla_decode_attn_rope",
     "lla_decode_attn_paged_workspace", "lla_decode_attn_paged",
+    "lla_decode_attn_paged_plan", "lla_decode_attn_paged_planned",
     "lla2d_decode_attn_workspace", "lla2d_decode_attn", "lla2d_decode_attn_rope",
     "lla2d_decode_attn_paged_workspace", "lla2d_decode_attn_paged",
+    "lla2d_decode_attn_paged_plan", "lla2d_decode_attn_paged_planned",
     "lla_encode", "lla_encode_bias", "lla_encode_with_bias_workspace", "lla_encode_with_bias",
+    "lla_encode_paged",
 )
 
 _lock = threading.Lock()
@@ -69,10 +73,20 @@ _SIGS = {
     "lla_decode_attn_paged": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp, _c_int, _vp] +
                               [_c_int] * 2 + [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp],
                               _c_int),
+    "lla_decode_attn_paged_plan": ([_c_int] * 7 + [_vp, _c_int, _vp, _c_int, _c_int, _vp,
+                                                    _c_size, _vp], _c_int),
+    "lla2d_decode_attn_paged_plan": ([_c_int] * 6 + [_vp, _c_int, _vp, _c_int, _c_int, _vp,
+                                                      _c_size, _vp], _c_int),
     "lla2d_decode_attn_workspace": ([_c_int] * 5, _c_size),
     "lla2d_decode_attn_rope": ([_vp, _vp, _vp, _vp, _c_int] + [_c_int] * 8 + [_vp] * 4 +
                                [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla2d_decode_attn_paged_workspace": ([_c_int] * 4, _c_size),
+    "lla_decode_attn_paged_planned": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 +
+                                      [_vp, _c_int, _vp] + [_c_int] * 2 + [_vp] * 4 +
+                                      [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
+    "lla2d_decode_attn_paged_planned": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 +
+                                        [_vp, _c_int, _vp] + [_c_int] * 2 + [_vp] * 4 +
+                                        [_c_float, _vp, _vp, _vp, _c_size, _vp], _c_int),
     "lla2d_decode_attn_paged": ([_vp, _vp, _vp, _c_int] + [_c_int] * 7 + [_vp, _c_int, _vp] +
                                 [_c_int] * 2 + [_vp] * 4 + [_c_float, _vp, _vp, _vp, _c_size, _vp],
                                 _c_int),
@@ -87,6 +101,9 @@ _SIGS = {
     "lla_encode_with_bias_workspace": ([_c_int] * 5, _c_size),
     "lla_encode_with_bias": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _vp,
                                                               _c_size, _vp], _c_int),
+    "lla_encode_paged": ([_vp, _c_int] + [_c_int] * 5 + [_vp, _vp, _vp, _c_ll, _c_ll, _c_ll,
+                                                          _c_int, _c_int, _vp, _c_int, _c_int,
+                                                          _vp, _vp, _vp, _c_size, _vp], _c_int),
 }
 
 
@@ -390,12 +407,14 @@ def lla_decode_attn_paged_workspace(B, H, r_k, r_v):
 
 def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t, mu_k_t=None,
                           mu_v_t=None, scale=None, sink=0, window=0, out=None, lse=None,
-                          workspace=None, stream=None, want_lse=True):
+                          workspace=None, stream=None, want_lse=True, planned=False):
     """Per-head absorbed decode over a paged store with per-sequence lengths.
 
     q [B,H,d_h] fp32; zk_pages [P,H,page_size,r_k], zv_pages [P,H,page_size,r_v]
     bf16 or fp32; block_table [B,max_blocks] int32 and seq_lens [B] int32 on
     the device; sink, window: the eviction set (window 0 keeps every token).
+    With planned=True this is lla_decode_attn_paged_planned: it reuses the
+    plan that lla_decode_attn_paged_plan left in `workspace` (required).
     Returns (out [B,H,d_h], lse [B,H] or None)."""
     _check_paged(q, zk_pages, zv_pages, block_table, seq_lens, two_d=False)
     _check_query_side(q, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, zk_pages.shape[-1],
@@ -413,9 +432,11 @@ def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv
         lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
     h = lib()
     need = int(h.lla_decode_attn_paged_workspace(B, H, r_k, r_v))
+    _expect(workspace is not None or not planned, "a planned call needs the plan's workspace")
     if workspace is None:
         workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
-    st = h.lla_decode_attn_paged(_ptr(q), _ptr(zk_pages), _ptr(zv_pages), _dtype_code(zk_pages),
+    fn = h.lla_decode_attn_paged_planned if planned else h.lla_decode_attn_paged
+    st = fn(_ptr(q), _ptr(zk_pages), _ptr(zv_pages), _dtype_code(zk_pages),
                                  B, H, d_h, r_k, r_v, page_size, num_pages, _ptr(block_table),
                                  max_blocks, _ptr(seq_lens), int(sink), int(window), _ptr(dk_t),
                                  _ptr(dv_t), _ptr(mu_k_t), _ptr(mu_v_t), float(scale), _ptr(out),
@@ -423,6 +444,66 @@ def lla_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st)
     return out, lse
+
+
+def _paged_plan(two_d, zk_pages, zv_pages, block_table, seq_lens, H, workspace, sink, window,
+                stream):
+    _same_latent_type(zk_pages, zv_pages)
+    lead = 2 if two_d else 3
+    _expect(zk_pages.dim() == lead + 1 and zv_pages.dim() == lead + 1 and
+            tuple(zk_pages.shape[:lead]) == tuple(zv_pages.shape[:lead]),
+            "page pools must be [P, page_size, r]" if two_d else "page pools must be [P, H, page_size, r]")
+    _expect(block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32,
+            "block_table and seq_lens must be int32")
+    _expect(block_table.dim() == 2, "block_table must be [B, max_blocks]")
+    B = block_table.shape[0]
+    _shape("seq_lens", seq_lens, (B,))
+    _expect(workspace is not None, "the plan is written into `workspace`; pass the one the "
+                                   "planned calls will use")
+    _need_cuda(zk_pages, zv_pages, block_table, seq_lens, workspace)
+    P, ps = zk_pages.shape[0], zk_pages.shape[-2]
+    r_k, r_v = zk_pages.shape[-1], zv_pages.shape[-1]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    h = lib()
+    if two_d:
+        st = h.lla2d_decode_attn_paged_plan(B, H, r_k, r_v, ps, P, _ptr(block_table),
+                                            block_table.shape[1], _ptr(seq_lens), int(sink),
+                                            int(window), _ptr(workspace), ws_bytes,
+                                            _stream(stream))
+    else:
+        st = h.lla_decode_attn_paged_plan(_dtype_code(zk_pages), B, zk_pages.shape[1], r_k, r_v,
+                                          ps, P, _ptr(block_table), block_table.shape[1],
+                                          _ptr(seq_lens), int(sink), int(window), _ptr(workspace),
+                                          ws_bytes, _stream(stream))
+    _check(st)
+    return workspace
+
+
+def lla_decode_attn_paged_plan(zk_pages, zv_pages, block_table, seq_lens, workspace, sink=0,
+                               window=0, stream=None):
+    """Plans a per-head paged decode step once: writes the plan of the
+    lengths and table into `workspace` (sized by
+    lla_decode_attn_paged_workspace) for later
+    lla_decode_attn_paged(..., planned=True) calls. Returns workspace."""
+    return _paged_plan(False, zk_pages, zv_pages, block_table, seq_lens, None, workspace, sink,
+                       window, stream)
+
+
+def lla_decode_attn_paged_planned(*args, **kw):
+    """lla_decode_attn_paged on the plan already in `workspace`."""
+    return lla_decode_attn_paged(*args, planned=True, **kw)
+
+
+def lla2d_decode_attn_paged_plan(zk_pages, zv_pages, block_table, seq_lens, H, workspace, sink=0,
+                                 window=0, stream=None):
+    """The LLA-2D counterpart of lla_decode_attn_paged_plan (H heads)."""
+    return _paged_plan(True, zk_pages, zv_pages, block_table, seq_lens, H, workspace, sink,
+                       window, stream)
+
+
+def lla2d_decode_attn_paged_planned(*args, **kw):
+    """lla2d_decode_attn_paged on the plan already in `workspace`."""
+    return lla2d_decode_attn_paged(*args, planned=True, **kw)
 
 
 def lla2d_decode_attn_rope(q, q_rope, zk, zv, dk_t, dv_t, N=None, mu_k_t=None, mu_v_t=None,
@@ -466,11 +547,12 @@ def lla2d_decode_attn_paged_workspace(B, H, r_k, r_v):
 
 def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, dv_t,
                             mu_k_t=None, mu_v_t=None, scale=None, sink=0, window=0, out=None,
-                            lse=None, workspace=None, stream=None, want_lse=True):
+                            lse=None, workspace=None, stream=None, want_lse=True, planned=False):
     """LLA-2D absorbed decode over a paged store: zk_pages [P,page_size,r_k],
     zv_pages [P,page_size,r_v] bf16 shared by every head, page_size a
     multiple of 64; block_table [B,max_blocks] and seq_lens [B] int32 on
-    the device. Returns (out [B,H,d_h], lse [B,H] or None)."""
+    the device. planned=True: lla2d_decode_attn_paged_planned on the plan in
+    `workspace`. Returns (out [B,H,d_h], lse [B,H] or None)."""
     _check_paged(q, zk_pages, zv_pages, block_table, seq_lens, two_d=True)
     _check_query_side(q, dk_t, dv_t, mu_k_t, mu_v_t, out, lse, zk_pages.shape[-1],
                       zv_pages.shape[-1])
@@ -487,9 +569,11 @@ def lla2d_decode_attn_paged(q, zk_pages, zv_pages, block_table, seq_lens, dk_t, 
         lse = torch.empty((B, H), device=q.device, dtype=torch.float32)
     h = lib()
     need = int(h.lla2d_decode_attn_paged_workspace(B, H, r_k, r_v))
+    _expect(workspace is not None or not planned, "a planned call needs the plan's workspace")
     if workspace is None:
         workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
-    st = h.lla2d_decode_attn_paged(_ptr(q), _ptr(zk_pages), _ptr(zv_pages),
+    fn = h.lla2d_decode_attn_paged_planned if planned else h.lla2d_decode_attn_paged
+    st = fn(_ptr(q), _ptr(zk_pages), _ptr(zv_pages),
                                    _dtype_code(zk_pages), B, H, d_h, r_k, r_v, page_size,
                                    num_pages, _ptr(block_table), max_blocks, _ptr(seq_lens),
                                    int(sink), int(window), _ptr(dk_t), _ptr(dv_t), _ptr(mu_k_t),
@@ -603,6 +687,50 @@ def lla_encode_with_bias(x, w_down_t, muw=None, z=None, z_row_stride=None, z_gro
                                     _ptr(workspace), ws_bytes, _stream(stream))
     _check(st)
     return z
+
+
+def lla_encode_paged(x, w_down_t, muw, z_pages, block_table, positions, seq_idx=None,
+                     workspace=None, stream=None, split=True):
+    """Latent write into a paged store: token n's latent (lla_encode_with_bias
+    of x [T,N,G,d_loop] bf16 with w_down_t [G,r,T*d_loop] and muw [G,r] or
+    None) goes to position positions[n] of sequence seq_idx[n] (n when
+    seq_idx is None) through block_table [n_seq,max_blocks] int32.
+    z_pages is the pool, contiguous bf16: [P,G,page_size,r_row] per head, or
+    [P,page_size,r_row] for LLA-2D (G = 1); each row's first r values are
+    written (r_row > r keeps a rotary tail). Returns z_pages."""
+    _check_encode(x, w_down_t, muw=muw)
+    T, N, G, d_loop = x.shape
+    r = w_down_t.shape[1]
+    _expect(z_pages.dtype == torch.bfloat16, f"z_pages must be bfloat16, got {z_pages.dtype}")
+    if z_pages.dim() == 3:
+        _expect(G == 1, "an LLA-2D pool [P, page_size, r] takes G = 1")
+        P, ps, rr = z_pages.shape
+        strides = (ps * rr, 0, rr)
+    else:
+        _expect(z_pages.dim() == 4 and z_pages.shape[1] == G,
+                f"z_pages must be [P, G={G}, page_size, r] or [P, page_size, r], "
+                f"got {tuple(z_pages.shape)}")
+        P, _, ps, rr = z_pages.shape
+        strides = (G * ps * rr, ps * rr, rr)
+    _expect(rr >= r, f"pool rows hold {rr} values, fewer than r = {r}")
+    _expect(block_table.dtype == torch.int32 and positions.dtype == torch.int32 and
+            (seq_idx is None or seq_idx.dtype == torch.int32),
+            "block_table, positions and seq_idx must be int32")
+    _expect(block_table.dim() == 2, "block_table must be [n_seq, max_blocks]")
+    _shape("positions", positions, (N,))
+    _shape("seq_idx", seq_idx, (N,))
+    _need_cuda(x, w_down_t, muw, z_pages, block_table, positions, seq_idx, workspace)
+    if workspace is None and split:
+        need = int(lib().lla_encode_with_bias_workspace(T, N, G, d_loop, r))
+        if need:
+            workspace = torch.empty(need, device=x.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().lla_encode_paged(_ptr(x), _dtype_code(x), T, N, G, d_loop, r, _ptr(w_down_t),
+                                _ptr(muw), _ptr(z_pages), *strides, ps, P, _ptr(block_table),
+                                block_table.shape[0], block_table.shape[1], _ptr(seq_idx),
+                                _ptr(positions), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st)
+    return z_pages
 
 
 def lla_merge_attn(out_parts, lse_parts, out=None, lse=None, stream=None):

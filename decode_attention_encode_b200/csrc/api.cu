@@ -134,10 +134,12 @@ lla_status lla::check_decode_args(const float* q, const void* zk, const void* zv
 
 namespace {
 
-// Argument checks shared by the encode entry points.
+// Argument checks shared by the encode entry points. `rows` is the number
+// of rows of one group that the strides lay out (N for a dense write,
+// page_size inside a page of a paged store).
 lla_status check_encode_args(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,
                              const void* w_down_t, const float* mu, void* z,
-                             long long z_row_stride, long long z_group_stride) {
+                             long long z_row_stride, long long z_group_stride, int rows) {
   if (xdt != LLA_BF16) return fail(LLA_ERR_INVALID_ARG, "xdt must be LLA_BF16");
   if (!x || !w_down_t || !z) return fail(LLA_ERR_INVALID_ARG, "x, w_down_t and z must be non-NULL");
   if (!aligned(x, 16) || !aligned(w_down_t, 16) || !aligned(z, 16))
@@ -151,12 +153,109 @@ lla_status check_encode_args(const void* x, lla_dtype xdt, int T, int N, int G, 
   if (z_row_stride < r || z_group_stride < 0 || z_row_stride % 8 || z_group_stride % 8)
     return fail(LLA_ERR_INVALID_ARG, "z strides must be multiples of 8 with z_row_stride >= r");
   if (G > 1) {
-    const bool groups_outer = z_group_stride >= (long long)(N - 1) * z_row_stride + r;
+    const bool groups_outer = z_group_stride >= (long long)(rows - 1) * z_row_stride + r;
     const bool rows_outer = z_row_stride >= (long long)(G - 1) * z_group_stride + r && z_group_stride >= r;
     if (!groups_outer && !rows_outer)
       return fail(LLA_ERR_INVALID_ARG, "z strides make output rows overlap");
   }
   return LLA_OK;
+}
+
+// Checks shared by the paged calls: the pool's geometry, the block table
+// and lengths (device arrays, read only on the device) and the eviction set.
+lla_status check_paged_table(int page_size, int num_pages, const int* block_table,
+                             int max_blocks, const int* seq_lens, int sink, int window,
+                             bool two_d) {
+  if (!block_table || !seq_lens)
+    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be non-NULL");
+  if (!aligned(block_table, 4) || !aligned(seq_lens, 4))
+    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be 4-byte aligned");
+  if (two_d && (page_size < 64 || page_size % 64))
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D pages hold a positive multiple of 64 tokens");
+  if (page_size < 1 || num_pages < 1 || max_blocks < 1)
+    return fail(LLA_ERR_INVALID_ARG, "page_size, num_pages and max_blocks must be >= 1");
+  if ((long long)page_size * max_blocks > 0x7fffffffLL)
+    return fail(LLA_ERR_INVALID_ARG, "page_size * max_blocks must fit in 31 bits");
+  if (sink < 0 || window < 0) return fail(LLA_ERR_INVALID_ARG, "sink and window must be >= 0");
+  return LLA_OK;
+}
+
+// The per-head paged call in each mode (plan and decode, or decode on a plan
+// already in the workspace).
+lla_status paged_call(const float* q, const void* zk_pages, const void* zv_pages, lla_dtype zdt,
+                      int B, int H, int d_h, int r_k, int r_v, int page_size, int num_pages,
+                      const int* block_table, int max_blocks, const int* seq_lens, int sink,
+                      int window, const float* dk_t, const float* dv_t, const float* mu_k_t,
+                      const float* mu_v_t, float scale, float* out, float* lse, void* workspace,
+                      size_t ws_bytes, void* stream, PagedMode mode) {
+  g_last_error[0] = '\0';
+  int esz = 0;
+  // the shared checks; lengths live on the device and are checked there
+  lla_status st = check_decode_args(q, zk_pages, zv_pages, zdt, B, H, d_h, 1, 1, r_k, r_v, dk_t,
+                                    dv_t, mu_k_t, mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  st = check_paged_table(page_size, num_pages, block_table, max_blocks, seq_lens, sink, window,
+                         false);
+  if (st != LLA_OK) return st;
+  return run_decode_paged(q, zk_pages, zv_pages, esz, B, H, d_h, r_k, r_v, page_size, num_pages,
+                          block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t,
+                          mu_v_t, scale, out, lse, workspace, ws_bytes,
+                          static_cast<cudaStream_t>(stream), mode);
+}
+
+lla_status paged2d_call(const float* q, const void* zk_pages, const void* zv_pages, lla_dtype zdt,
+                        int B, int H, int d_h, int r_k, int r_v, int page_size, int num_pages,
+                        const int* block_table, int max_blocks, const int* seq_lens, int sink,
+                        int window, const float* dk_t, const float* dv_t, const float* mu_k_t,
+                        const float* mu_v_t, float scale, float* out, float* lse,
+                        void* workspace, size_t ws_bytes, void* stream, PagedMode mode) {
+  g_last_error[0] = '\0';
+  int esz = 0;
+  lla_status st = check_decode_args(q, zk_pages, zv_pages, zdt, B, H, d_h, 1, 1, r_k, r_v, dk_t,
+                                    dv_t, mu_k_t, mu_v_t, out, lse, workspace, &esz);
+  if (st != LLA_OK) return st;
+  if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
+  if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
+  st = check_paged_table(page_size, num_pages, block_table, max_blocks, seq_lens, sink, window,
+                         true);
+  if (st != LLA_OK) return st;
+  return run_decode_2d_paged(q, zk_pages, zv_pages, B, H, d_h, r_k, r_v, page_size, num_pages,
+                             block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t,
+                             mu_v_t, scale, out, lse, workspace, ws_bytes,
+                             static_cast<cudaStream_t>(stream), mode);
+}
+
+// The plan-only calls: the ranks and table checks of the decode calls,
+// without the query-side arrays.
+lla_status paged_plan_call(lla_dtype zdt, int B, int H, int r_k, int r_v, int page_size,
+                           int num_pages, const int* block_table, int max_blocks,
+                           const int* seq_lens, int sink, int window, void* workspace,
+                           size_t ws_bytes, void* stream, bool two_d) {
+  g_last_error[0] = '\0';
+  if (zdt != LLA_BF16 && zdt != LLA_F32)
+    return fail(LLA_ERR_INVALID_ARG, "zdt must be LLA_BF16 or LLA_F32");
+  if (B < 1 || H < 1) return fail(LLA_ERR_INVALID_ARG, "B and H must be >= 1");
+  const int esz = zdt == LLA_BF16 ? 2 : 4;
+  const int rmax = esz == 2 ? 256 : 128;
+  if (r_k < 8 || r_v < 8 || r_k % 8 || r_v % 8 || r_k > rmax || r_v > rmax)
+    return fail(LLA_ERR_INVALID_ARG, "r_k and r_v must be multiples of 8 in 8..%d", rmax);
+  if (two_d && zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
+  if (two_d && H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
+  if (workspace && !aligned(workspace, 16))
+    return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  lla_status st = check_paged_table(page_size, num_pages, block_table, max_blocks, seq_lens,
+                                    sink, window, two_d);
+  if (st != LLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (two_d)
+    return run_decode_2d_paged(nullptr, nullptr, nullptr, B, H, 1, r_k, r_v, page_size, num_pages,
+                               block_table, max_blocks, seq_lens, sink, window, nullptr, nullptr,
+                               nullptr, nullptr, 0.f, nullptr, nullptr, workspace, ws_bytes, s,
+                               kPlanOnly);
+  return run_decode_paged(nullptr, nullptr, nullptr, esz, B, H, 1, r_k, r_v, page_size, num_pages,
+                          block_table, max_blocks, seq_lens, sink, window, nullptr, nullptr,
+                          nullptr, nullptr, 0.f, nullptr, nullptr, workspace, ws_bytes, s,
+                          kPlanOnly);
 }
 
 }  // namespace
@@ -283,31 +382,37 @@ lla_status lla_decode_attn_paged(const float* q, const void* zk_pages, const voi
                                  const float* dk_t, const float* dv_t, const float* mu_k_t,
                                  const float* mu_v_t, float scale, float* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream) {
-  g_last_error[0] = '\0';
-  int esz = 0;
-  // the shared checks; lengths live on the device and are checked there
-  lla_status st = check_decode_args(q, zk_pages, zv_pages, zdt, B, H, d_h, 1, 1, r_k, r_v, dk_t,
-                                    dv_t, mu_k_t, mu_v_t, out, lse, workspace, &esz);
-  if (st != LLA_OK) return st;
-  if (!block_table || !seq_lens)
-    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be non-NULL");
-  if (!aligned(block_table, 4) || !aligned(seq_lens, 4))
-    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be 4-byte aligned");
-  if (page_size < 1 || num_pages < 1 || max_blocks < 1)
-    return fail(LLA_ERR_INVALID_ARG, "page_size, num_pages and max_blocks must be >= 1");
-  if ((long long)page_size * max_blocks > 0x7fffffffLL)
-    return fail(LLA_ERR_INVALID_ARG, "page_size * max_blocks must fit in 31 bits");
-  if (sink < 0 || window < 0) return fail(LLA_ERR_INVALID_ARG, "sink and window must be >= 0");
-  return run_decode_paged(q, zk_pages, zv_pages, esz, B, H, d_h, r_k, r_v, page_size, num_pages,
-                          block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t,
-                          mu_v_t, scale, out, lse, workspace, ws_bytes,
-                          static_cast<cudaStream_t>(stream));
+  return paged_call(q, zk_pages, zv_pages, zdt, B, H, d_h, r_k, r_v, page_size, num_pages,
+                    block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t, mu_v_t,
+                    scale, out, lse, workspace, ws_bytes, stream, kPlanAndDecode);
+}
+
+lla_status lla_decode_attn_paged_plan(lla_dtype zdt, int B, int H, int r_k, int r_v,
+                                      int page_size, int num_pages, const int* block_table,
+                                      int max_blocks, const int* seq_lens, int sink, int window,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  return paged_plan_call(zdt, B, H, r_k, r_v, page_size, num_pages, block_table, max_blocks,
+                         seq_lens, sink, window, workspace, ws_bytes, stream, false);
+}
+
+lla_status lla_decode_attn_paged_planned(const float* q, const void* zk_pages,
+                                         const void* zv_pages, lla_dtype zdt, int B, int H,
+                                         int d_h, int r_k, int r_v, int page_size, int num_pages,
+                                         const int* block_table, int max_blocks,
+                                         const int* seq_lens, int sink, int window,
+                                         const float* dk_t, const float* dv_t,
+                                         const float* mu_k_t, const float* mu_v_t, float scale,
+                                         float* out, float* lse, void* workspace,
+                                         size_t ws_bytes, void* stream) {
+  return paged_call(q, zk_pages, zv_pages, zdt, B, H, d_h, r_k, r_v, page_size, num_pages,
+                    block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t, mu_v_t,
+                    scale, out, lse, workspace, ws_bytes, stream, kDecodePlanned);
 }
 
 size_t lla2d_decode_attn_workspace(int B, int H, int N, int r_k, int r_v) {
   // r_k is the key row width (r_k + d_r for lla2d_decode_attn_rope)
-  if (B < 1 || H < 1 || H > 32 || N < 1 || r_k < 64 || r_k > 384 || r_k % 64 || r_v < 128 ||
-      r_v > 256 || r_v % 128)
+  if (B < 1 || H < 1 || H > 32 || N < 1 || r_k < 8 || r_k > 384 || r_k % 8 || r_v < 8 ||
+      r_v > 256 || r_v % 8)
     return 0;
   return workspace_2d(B, H, N, r_k, r_v);
 }
@@ -324,8 +429,6 @@ lla_status lla2d_decode_attn(const float* q, const void* zk, const void* zv, lla
   if (st != LLA_OK) return st;
   if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
   if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
-  if (r_k % 64 || r_v % 128)
-    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D needs r_k a multiple of 64 and r_v a multiple of 128");
   return run_decode_2d(q, zk, zv, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t, mu_k_t,
                        mu_v_t, scale, out, lse, workspace, ws_bytes,
                        static_cast<cudaStream_t>(stream));
@@ -350,18 +453,16 @@ lla_status lla2d_decode_attn_rope(const float* q, const float* q_rope, const voi
   if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
   if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
   const int rq = r_k + d_r;
-  if (rq % 64 || rq > 384 || r_v % 128)
-    return fail(LLA_ERR_UNSUPPORTED,
-                "LLA-2D with a rotary branch needs r_k + d_r a multiple of 64 up to 384 and r_v "
-                "a multiple of 128");
+  if (rq > 384)
+    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D with a rotary branch needs r_k + d_r <= 384");
   return run_decode_2d(q, zk, zv, B, H, d_h, N, (long long)n_cap, r_k, r_v, dk_t, dv_t, mu_k_t,
                        mu_v_t, scale, out, lse, workspace, ws_bytes,
                        static_cast<cudaStream_t>(stream), q_rope, d_r);
 }
 
 size_t lla2d_decode_attn_paged_workspace(int B, int H, int r_k, int r_v) {
-  if (B < 1 || H < 1 || H > 32 || r_k < 64 || r_k > 256 || r_k % 64 || r_v < 128 || r_v > 256 ||
-      r_v % 128)
+  if (B < 1 || H < 1 || H > 32 || r_k < 8 || r_k > 256 || r_k % 8 || r_v < 8 || r_v > 256 ||
+      r_v % 8)
     return 0;
   return workspace_2d_paged(B, H, r_k, r_v);
 }
@@ -373,30 +474,31 @@ lla_status lla2d_decode_attn_paged(const float* q, const void* zk_pages, const v
                                    const float* dk_t, const float* dv_t, const float* mu_k_t,
                                    const float* mu_v_t, float scale, float* out, float* lse,
                                    void* workspace, size_t ws_bytes, void* stream) {
-  g_last_error[0] = '\0';
-  int esz = 0;
-  lla_status st = check_decode_args(q, zk_pages, zv_pages, zdt, B, H, d_h, 1, 1, r_k, r_v, dk_t,
-                                    dv_t, mu_k_t, mu_v_t, out, lse, workspace, &esz);
-  if (st != LLA_OK) return st;
-  if (zdt != LLA_BF16) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D latents must be LLA_BF16");
-  if (H > 32) return fail(LLA_ERR_UNSUPPORTED, "LLA-2D supports H <= 32");
-  if (r_k % 64 || r_v % 128)
-    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D needs r_k a multiple of 64 and r_v a multiple of 128");
-  if (!block_table || !seq_lens)
-    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be non-NULL");
-  if (!aligned(block_table, 4) || !aligned(seq_lens, 4))
-    return fail(LLA_ERR_INVALID_ARG, "block_table and seq_lens must be 4-byte aligned");
-  if (page_size < 64 || page_size % 64)
-    return fail(LLA_ERR_UNSUPPORTED, "LLA-2D pages hold a positive multiple of 64 tokens");
-  if (num_pages < 1 || max_blocks < 1)
-    return fail(LLA_ERR_INVALID_ARG, "num_pages and max_blocks must be >= 1");
-  if ((long long)page_size * max_blocks > 0x7fffffffLL)
-    return fail(LLA_ERR_INVALID_ARG, "page_size * max_blocks must fit in 31 bits");
-  if (sink < 0 || window < 0) return fail(LLA_ERR_INVALID_ARG, "sink and window must be >= 0");
-  return run_decode_2d_paged(q, zk_pages, zv_pages, B, H, d_h, r_k, r_v, page_size, num_pages,
-                             block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t,
-                             mu_v_t, scale, out, lse, workspace, ws_bytes,
-                             static_cast<cudaStream_t>(stream));
+  return paged2d_call(q, zk_pages, zv_pages, zdt, B, H, d_h, r_k, r_v, page_size, num_pages,
+                      block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t, mu_v_t,
+                      scale, out, lse, workspace, ws_bytes, stream, kPlanAndDecode);
+}
+
+lla_status lla2d_decode_attn_paged_plan(int B, int H, int r_k, int r_v, int page_size,
+                                        int num_pages, const int* block_table, int max_blocks,
+                                        const int* seq_lens, int sink, int window,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  return paged_plan_call(LLA_BF16, B, H, r_k, r_v, page_size, num_pages, block_table, max_blocks,
+                         seq_lens, sink, window, workspace, ws_bytes, stream, true);
+}
+
+lla_status lla2d_decode_attn_paged_planned(const float* q, const void* zk_pages,
+                                           const void* zv_pages, lla_dtype zdt, int B, int H,
+                                           int d_h, int r_k, int r_v, int page_size,
+                                           int num_pages, const int* block_table, int max_blocks,
+                                           const int* seq_lens, int sink, int window,
+                                           const float* dk_t, const float* dv_t,
+                                           const float* mu_k_t, const float* mu_v_t, float scale,
+                                           float* out, float* lse, void* workspace,
+                                           size_t ws_bytes, void* stream) {
+  return paged2d_call(q, zk_pages, zv_pages, zdt, B, H, d_h, r_k, r_v, page_size, num_pages,
+                      block_table, max_blocks, seq_lens, sink, window, dk_t, dv_t, mu_k_t, mu_v_t,
+                      scale, out, lse, workspace, ws_bytes, stream, kDecodePlanned);
 }
 
 lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,
@@ -404,7 +506,7 @@ lla_status lla_encode(const void* x, lla_dtype xdt, int T, int N, int G, int d_l
                       long long z_group_stride, void* stream) {
   g_last_error[0] = '\0';
   lla_status st = check_encode_args(x, xdt, T, N, G, d_loop, r, w_down_t, mu, z, z_row_stride,
-                                    z_group_stride);
+                                    z_group_stride, N);
   if (st != LLA_OK) return st;
   return run_encode(x, T, N, G, d_loop, r, w_down_t, mu, z, z_row_stride, z_group_stride,
                     static_cast<cudaStream_t>(stream));
@@ -432,13 +534,48 @@ lla_status lla_encode_with_bias(const void* x, lla_dtype xdt, int T, int N, int 
                                 size_t ws_bytes, void* stream) {
   g_last_error[0] = '\0';
   lla_status st = check_encode_args(x, xdt, T, N, G, d_loop, r, w_down_t, nullptr, z,
-                                    z_row_stride, z_group_stride);
+                                    z_row_stride, z_group_stride, N);
   if (st != LLA_OK) return st;
   if (muw && !aligned(muw, 16)) return fail(LLA_ERR_INVALID_ARG, "muw must be 16-byte aligned");
   if (workspace && !aligned(workspace, 16))
     return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   return run_encode(x, T, N, G, d_loop, r, w_down_t, nullptr, z, z_row_stride, z_group_stride,
                     static_cast<cudaStream_t>(stream), muw, workspace, ws_bytes);
+}
+
+lla_status lla_encode_paged(const void* x, lla_dtype xdt, int T, int N, int G, int d_loop, int r,
+                            const void* w_down_t, const float* muw, void* z_pages,
+                            long long z_page_stride, long long z_group_stride,
+                            long long z_row_stride, int page_size, int num_pages,
+                            const int* block_table, int n_seq, int max_blocks, const int* seq_idx,
+                            const int* positions, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  g_last_error[0] = '\0';
+  if (page_size < 1 || num_pages < 1 || n_seq < 1 || max_blocks < 1)
+    return fail(LLA_ERR_INVALID_ARG, "page_size, num_pages, n_seq and max_blocks must be >= 1");
+  if ((long long)page_size * max_blocks > 0x7fffffffLL)
+    return fail(LLA_ERR_INVALID_ARG, "page_size * max_blocks must fit in 31 bits");
+  // the rows of one page are laid out like a dense write of page_size tokens
+  lla_status st = check_encode_args(x, xdt, T, N, G, d_loop, r, w_down_t, nullptr, z_pages,
+                                    z_row_stride, z_group_stride, page_size);
+  if (st != LLA_OK) return st;
+  const long long page_extent =
+      (long long)(G - 1) * z_group_stride + (long long)(page_size - 1) * z_row_stride + r;
+  if (z_page_stride % 8 || z_page_stride < page_extent)
+    return fail(LLA_ERR_INVALID_ARG,
+                "z_page_stride must be a multiple of 8 covering a page (>= %lld)", page_extent);
+  if (!block_table || !positions)
+    return fail(LLA_ERR_INVALID_ARG, "block_table and positions must be non-NULL");
+  if (!aligned(block_table, 4) || !aligned(positions, 4) || (seq_idx && !aligned(seq_idx, 4)))
+    return fail(LLA_ERR_INVALID_ARG, "block_table, seq_idx and positions must be 4-byte aligned");
+  if (muw && !aligned(muw, 16)) return fail(LLA_ERR_INVALID_ARG, "muw must be 16-byte aligned");
+  if (workspace && !aligned(workspace, 16))
+    return fail(LLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  PagedOut pd{block_table, seq_idx, positions, n_seq, max_blocks, page_size, num_pages,
+              z_page_stride};
+  return run_encode(x, T, N, G, d_loop, r, w_down_t, nullptr, z_pages, z_row_stride,
+                    z_group_stride, static_cast<cudaStream_t>(stream), muw, workspace, ws_bytes,
+                    &pd);
 }
 
 }  // extern "C"

@@ -14,6 +14,7 @@ namespace lla {
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 constexpr unsigned int kStatusWaitTimeout = 0x1u;
 constexpr unsigned int kStatusBadPagedInput = 0x2u;
+constexpr unsigned int kStatusPlanMismatch = 0x4u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

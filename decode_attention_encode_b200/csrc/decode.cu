@@ -123,6 +123,29 @@ __device__ __forceinline__ void lds_cols(const float* p, float (&v)[COLS]) {
   }
 }
 
+// Byte offset of sequence b's Q' block in the LLA-2D operand: rq columns
+// rounded up to whole 64-column (128-byte) swizzle chunks of hp rows.
+__device__ __forceinline__ size_t qsw_block(const AbsorbArgs& a, int rq, int b) {
+  return (size_t)b * ((rq + 63) / 64) * a.hp * 128;
+}
+
+// The LLA-2D operand's columns from rq up to the next multiple of 64 are
+// zero for batch rows b0 .. b0+nb-1 of head h (and of the padding heads when
+// h is the last head): the tensor map fills the latent tile's matching
+// columns with zeros, and those products must stay finite. Called by the
+// CTA that holds the last columns.
+__device__ __forceinline__ void zero_qsw_tail(const AbsorbArgs& a, int rq, int h, int b0, int nb) {
+  const int npad = ((rq + 63) & ~63) - rq;
+  const int nh = h == a.H - 1 ? 1 + a.hp - a.H : 1;
+  for (int idx = threadIdx.x; idx < nb * npad * nh; idx += blockDim.x) {
+    const int bb = idx / (npad * nh), rest = idx - bb * npad * nh;
+    const int k = rest / npad, c = rq + rest - k * npad;
+    const int hh = k == 0 ? h : a.H + k - 1;
+    *reinterpret_cast<__nv_bfloat16*>(a.qsw + qsw_block(a, rq, b0 + bb) + sw128_off(hh, c, a.hp)) =
+        __float2bfloat16_rn(0.f);
+  }
+}
+
 template <int ROWS, int COLS>
 __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
   constexpr int CW = 32 * COLS;  // columns per CTA
@@ -216,7 +239,7 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
                       a.qscale;
       if (a.qp) a.qp[unit * rq + c] = v;
       if (a.qsw) {
-        unsigned char* base = a.qsw + (size_t)(b0 + bb) * (rq / 64) * a.hp * 128;
+        unsigned char* base = a.qsw + qsw_block(a, rq, b0 + bb);
         *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)) = __float2bfloat16_rn(v);
         // the last head's CTAs also clear the padding rows h >= H
         if (h == a.H - 1)
@@ -226,6 +249,7 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
       }
     }
   }
+  if (a.qsw && c0 + nc == rq) zero_qsw_tail(a, rq, h, b0, nb);
 }
 
 // ---------------------------------------------------------------------------
@@ -243,7 +267,146 @@ struct CombineArgs {
   float* out;
   float* lse;
   RaggedMap ragged;  // seqinfo non-null: the paged plan's piece map
+  unsigned int* status;
 };
+
+// The merge pass shared by k_combine and k_combine_tc.
+//
+// merge_rows: per row bb < nrows of a combine CTA (batch rows b0 .. b0+nb-1
+// of head h), one thread per row: the row's first partial record and piece
+// count, and the merged maximum and normaliser over its pieces, with four
+// record loads in flight; it also writes lse. The split runs over units
+// (b, h) for per-head LLA and over sequences b for LLA-2D; piece w of split
+// key k is partial record w + k. A ragged plan places unit (b, h) at
+// cum[b] + h * n_b in the range. A row with no attended token gets no piece,
+// keep = 0 and lse = -inf.
+__device__ __forceinline__ void merge_rows(const CombineArgs& a, int h, int b0, int nb, int nrows,
+                                           int* s_np, long long* s_off, float* s_M, float* s_inv,
+                                           float* s_keep) {
+  if ((int)threadIdx.x >= nrows) return;
+  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
+  const int bb = threadIdx.x;
+  // a ragged map whose plan is not this call's (its stamp differs): every
+  // row is empty, and the mismatch is reported
+  const bool plan_ok = !a.ragged.seqinfo || (unsigned long long)a.ragged.plan[2] == a.ragged.stamp;
+  if (!plan_ok && bb == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    report_status(a.status, kStatusPlanMismatch);
+  int np = 0;
+  long long off = 0;
+  float M = kNegBig, L = 0.f, keep = 0.f;
+  if (bb < nb) {
+    const long long u = (long long)(b0 + bb) * a.H + h;
+    const float c0u = (blockIdx.y == 0 && a.lse) ? a.c0[u] : 0.f;  // in flight with the records
+    const long long key = a.shared ? (long long)(b0 + bb) : u;
+    long long wf = 0, wl = -1;
+    if (a.ragged.seqinfo) {
+      const int n = plan_ok ? __ldg(&a.ragged.seqinfo[b0 + bb].x) : 0;
+      if (n > 0) {
+        const long long P = a.ragged.plan[1];
+        // per head for per-head LLA; LLA-2D splits a sequence once for all heads
+        const long long first = a.ragged.cum[b0 + bb] + (a.shared ? 0LL : (long long)h * n);
+        wf = first / P;
+        wl = (first + n - 1) / P;
+      }
+    } else {
+      wf = (key * a.N) / a.P;
+      wl = ((key + 1) * a.N - 1) / a.P;
+    }
+    np = (int)(wl - wf + 1);
+    off = a.shared ? ((wf + key) * a.H + h) * a.pstride : (wf + key) * a.pstride;
+    const float* rec0 = a.part + off;
+    for (int p0 = 0; p0 < np; p0 += 4) {
+      float2 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[k] = p0 + k < np ? __ldg(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride))
+                           : make_float2(kNegBig, 0.f);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float Mn = fmaxf(M, v[k].x);
+        L = L * exp2f(M - Mn) + v[k].y * exp2f(v[k].x - Mn);
+        M = Mn;
+      }
+    }
+    keep = np > 0 ? 1.f : 0.f;
+    if (blockIdx.y == 0 && a.lse)  // no attended token: lse = -inf
+      a.lse[u] = np > 0 ? (M + log2f(L)) * kLn2 + c0u : -INFINITY;
+  }
+  s_np[bb] = np;
+  s_off[bb] = off;
+  s_M[bb] = M;
+  s_inv[bb] = np > 0 ? 1.f / L : 0.f;
+  s_keep[bb] = keep;
+}
+
+// merge_sweep: ubar[row] = sum_p exp2(m_p - M) u_p / L over the CTA's
+// (row, 4-column) items, k4 items per row of which the first r4 hold values
+// (the rest are padding and come out 0), eight items per thread at a time
+// so their record loads are in flight together. Rows with no piece come out
+// 0. store(bb, c4, v) places each normalised float4.
+template <class Store>
+__device__ __forceinline__ void merge_sweep(const CombineArgs& a, int nrows, int k4, int r4,
+                                            const int* s_np, const long long* s_off,
+                                            const float* s_M, const float* s_inv, Store store) {
+  constexpr int kI = 8;
+  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
+  const int nitems = nrows * k4;
+  for (int base = threadIdx.x; base < nitems; base += 256 * kI) {
+    float4 acc[kI];
+    const float* rb[kI];
+    int npk[kI], c4k[kI];
+    float Mk[kI];
+    int npmax = 0;
+#pragma unroll
+    for (int k = 0; k < kI; ++k) {
+      const int idx = base + k * 256;
+      acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      npk[k] = 0;
+      rb[k] = a.part;
+      c4k[k] = 0;
+      Mk[k] = 0.f;
+      if (idx < nitems) {
+        const int bb = idx / k4;
+        c4k[k] = idx - bb * k4;
+        npk[k] = c4k[k] < r4 ? s_np[bb] : 0;
+        rb[k] = a.part + s_off[bb];
+        Mk[k] = s_M[bb];
+      }
+      npmax = max(npmax, npk[k]);
+    }
+    for (int p = 0; p < npmax; ++p) {
+      float mv[kI];
+      float4 uv[kI];
+#pragma unroll
+      for (int k = 0; k < kI; ++k) {
+        if (p < npk[k]) {
+          mv[k] = __ldg(rb[k] + p * rstride);
+          uv[k] = __ldg(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kI; ++k) {
+        if (p < npk[k]) {
+          const float wk = exp2f(mv[k] - Mk[k]);
+          acc[k].x = fmaf(wk, uv[k].x, acc[k].x);
+          acc[k].y = fmaf(wk, uv[k].y, acc[k].y);
+          acc[k].z = fmaf(wk, uv[k].z, acc[k].z);
+          acc[k].w = fmaf(wk, uv[k].w, acc[k].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kI; ++k) {
+      const int idx = base + k * 256;
+      if (idx < nitems) {
+        const int bb = idx / k4;
+        const float inv = s_inv[bb];
+        store(bb, c4k[k],
+              make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv));
+      }
+    }
+  }
+}
 
 // One CTA per (head, 32 output channels, 8*ROWS batch rows). The CTA stages
 // its 32 x r_v slice of W^V_up,t (rows padded by 4 floats, so float4 reads
@@ -283,125 +446,13 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
   pdl_wait();  // partials come from the streaming kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nrows = 8 * ROWS;
-  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
-
-  // 1. Per row: the range of partial records and the merged maximum and
-  //    normaliser, one thread per row with four record loads in flight.
-  //    The split runs over units (b, h) for per-head LLA and over sequences
-  //    b for LLA-2D; piece w of split key k is partial record w + k. A
-  //    ragged plan places unit (b, h) at cum[b] + h * n_b in the range.
-  if (threadIdx.x < nrows) {
-    const int bb = threadIdx.x;
-    int np = 0;
-    long long off = 0;
-    float M = kNegBig, L = 0.f, keep = 0.f;
-    if (bb < nb) {
-      const long long u = (long long)(b0 + bb) * a.H + h;
-      const long long key = a.shared ? (long long)(b0 + bb) : u;
-      long long wf = 0, wl = -1;
-      if (a.ragged.seqinfo) {
-        const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
-        if (n > 0) {
-          const long long P = a.ragged.plan[1];
-          // per head for per-head LLA; LLA-2D splits a sequence once for all heads
-          const long long first = a.ragged.cum[b0 + bb] + (a.shared ? 0LL : (long long)h * n);
-          wf = first / P;
-          wl = (first + n - 1) / P;
-        }
-      } else {
-        wf = (key * a.N) / a.P;
-        wl = ((key + 1) * a.N - 1) / a.P;
-      }
-      np = (int)(wl - wf + 1);
-      off = a.shared ? ((wf + key) * a.H + h) * a.pstride : (wf + key) * a.pstride;
-      const float* rec0 = a.part + off;
-      for (int p0 = 0; p0 < np; p0 += 4) {
-        float2 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          v[k] = p0 + k < np ? __ldg(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride))
-                             : make_float2(kNegBig, 0.f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float Mn = fmaxf(M, v[k].x);
-          L = L * exp2f(M - Mn) + v[k].y * exp2f(v[k].x - Mn);
-          M = Mn;
-        }
-      }
-      keep = np > 0 ? 1.f : 0.f;
-      if (blockIdx.y == 0 && a.lse)  // no attended token: lse = -inf
-        a.lse[u] = np > 0 ? (M + log2f(L)) * kLn2 + a.c0[u] : -INFINITY;
-    }
-    s_np[bb] = np;
-    s_off[bb] = off;
-    s_M[bb] = M;
-    s_inv[bb] = np > 0 ? 1.f / L : 0.f;
-    s_keep[bb] = keep;
-  }
+  // 1. per row: its records, merged maximum and normaliser
+  merge_rows(a, h, b0, nb, nrows, s_np, s_off, s_M, s_inv, s_keep);
   __syncthreads();
-
-  // 2. ubar[row] = sum_p exp2(m_p - M) u_p / L over all (row, 4-column)
-  //    items of the CTA, eight items per thread at a time so their record
-  //    loads are in flight together. Rows with no piece come out 0.
-  {
-    constexpr int kI = 8;
-    const int nitems = nrows * r4;
-    for (int base = threadIdx.x; base < nitems; base += 256 * kI) {
-      float4 acc[kI];
-      const float* rb[kI];
-      int npk[kI], c4k[kI];
-      float Mk[kI];
-      int npmax = 0;
-#pragma unroll
-      for (int k = 0; k < kI; ++k) {
-        const int idx = base + k * 256;
-        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        npk[k] = 0;
-        rb[k] = a.part;
-        c4k[k] = 0;
-        Mk[k] = 0.f;
-        if (idx < nitems) {
-          const int bb = idx / r4;
-          c4k[k] = idx - bb * r4;
-          npk[k] = s_np[bb];
-          rb[k] = a.part + s_off[bb];
-          Mk[k] = s_M[bb];
-        }
-        npmax = max(npmax, npk[k]);
-      }
-      for (int p = 0; p < npmax; ++p) {
-        float mv[kI];
-        float4 uv[kI];
-#pragma unroll
-        for (int k = 0; k < kI; ++k) {
-          if (p < npk[k]) {
-            mv[k] = __ldg(rb[k] + p * rstride);
-            uv[k] = __ldg(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k]);
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < kI; ++k) {
-          if (p < npk[k]) {
-            const float wk = exp2f(mv[k] - Mk[k]);
-            acc[k].x = fmaf(wk, uv[k].x, acc[k].x);
-            acc[k].y = fmaf(wk, uv[k].y, acc[k].y);
-            acc[k].z = fmaf(wk, uv[k].z, acc[k].z);
-            acc[k].w = fmaf(wk, uv[k].w, acc[k].w);
-          }
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kI; ++k) {
-        const int idx = base + k * 256;
-        if (idx < nitems) {
-          const int bb = idx / r4;
-          const float inv = s_inv[bb];
-          reinterpret_cast<float4*>(ub + bb * a.r_v)[c4k[k]] =
-              make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
-        }
-      }
-    }
-  }
+  // 2. ubar rows into shared memory
+  merge_sweep(a, nrows, r4, r4, s_np, s_off, s_M, s_inv, [&](int bb, int c4, float4 v) {
+    reinterpret_cast<float4*>(ub + bb * a.r_v)[c4] = v;
+  });
   __syncthreads();
   // thread (w, l): channels i0 + l + 32 j (j < COLS; consecutive lanes read
   // consecutive padded rows, so the float4 reads are conflict-free) for the
@@ -659,7 +710,7 @@ __global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
                       a.qscale;
       if (a.qp) a.qp[unit * rq + c] = v;
       if (a.qsw) {
-        unsigned char* base = a.qsw + (size_t)(b0 + bb) * (rq / 64) * a.hp * 128;
+        unsigned char* base = a.qsw + qsw_block(a, rq, b0 + bb);
         *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)) = __float2bfloat16_rn(v);
         if (h == a.H - 1)
           for (int hz = a.H; hz < a.hp; ++hz)
@@ -667,6 +718,7 @@ __global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
                 __float2bfloat16_rn(0.f);
       }
     }
+  if (a.qsw && c0 + nc == rq) zero_qsw_tail(a, rq, h, b0, nb);
 }
 
 // One CTA per (head h, 32 output channels, 64 batch rows): the merge of
@@ -704,120 +756,16 @@ __global__ void __launch_bounds__(256, 2) k_combine_tc(CombineArgs a) {
     s_mu[threadIdx.x] = (a.mu_v && (int)threadIdx.x < ni) ? __ldg(a.mu_v + (size_t)h * a.d_h + i0 + threadIdx.x) : 0.f;
   pdl_wait();  // partials come from the streaming kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
 
-  // 1. per row: its records, merged maximum and normaliser (as k_combine)
-  if (threadIdx.x < kTcRows) {
-    const int bb = threadIdx.x;
-    int np = 0;
-    long long off = 0;
-    float M = kNegBig, L = 0.f, keep = 0.f;
-    if (bb < nb) {
-      const long long u = (long long)(b0 + bb) * a.H + h;
-      const float c0u = (blockIdx.y == 0 && a.lse) ? a.c0[u] : 0.f;  // in flight with the records
-      const long long key = a.shared ? (long long)(b0 + bb) : u;
-      long long wf = 0, wl = -1;
-      if (a.ragged.seqinfo) {
-        const int n = __ldg(&a.ragged.seqinfo[b0 + bb].x);
-        if (n > 0) {
-          const long long P = a.ragged.plan[1];
-          const long long first = a.ragged.cum[b0 + bb] + (a.shared ? 0LL : (long long)h * n);
-          wf = first / P;
-          wl = (first + n - 1) / P;
-        }
-      } else {
-        wf = (key * a.N) / a.P;
-        wl = ((key + 1) * a.N - 1) / a.P;
-      }
-      np = (int)(wl - wf + 1);
-      off = a.shared ? ((wf + key) * a.H + h) * a.pstride : (wf + key) * a.pstride;
-      const float* rec0 = a.part + off;
-      for (int p0 = 0; p0 < np; p0 += 4) {
-        float2 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          v[k] = p0 + k < np ? __ldg(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride))
-                             : make_float2(kNegBig, 0.f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float Mn = fmaxf(M, v[k].x);
-          L = L * exp2f(M - Mn) + v[k].y * exp2f(v[k].x - Mn);
-          M = Mn;
-        }
-      }
-      keep = np > 0 ? 1.f : 0.f;
-      if (blockIdx.y == 0 && a.lse)  // no attended token: lse = -inf
-        a.lse[u] = np > 0 ? (M + log2f(L)) * kLn2 + c0u : -INFINITY;
-    }
-    s_np[bb] = np;
-    s_off[bb] = off;
-    s_M[bb] = M;
-    s_inv[bb] = np > 0 ? 1.f / L : 0.f;
-    s_keep[bb] = keep;
-  }
+  // 1. per row: its records, merged maximum and normaliser
+  merge_rows(a, h, b0, nb, kTcRows, s_np, s_off, s_M, s_inv, s_keep);
   __syncthreads();
 
   // 2. ubar rows, split into shared memory; rows with no piece and the
   //    padding columns come out 0
-  {
-    constexpr int kI = 8;
-    const int nitems = kTcRows * k4;
-    for (int base = threadIdx.x; base < nitems; base += 256 * kI) {
-      float4 acc[kI];
-      const float* rb[kI];
-      int npk[kI], c4k[kI];
-      float Mk[kI];
-      int npmax = 0;
-#pragma unroll
-      for (int k = 0; k < kI; ++k) {
-        const int idx = base + k * 256;
-        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        npk[k] = 0;
-        rb[k] = a.part;
-        c4k[k] = 0;
-        Mk[k] = 0.f;
-        if (idx < nitems) {
-          const int bb = idx / k4;
-          c4k[k] = idx - bb * k4;
-          npk[k] = c4k[k] < r4 ? s_np[bb] : 0;
-          rb[k] = a.part + s_off[bb];
-          Mk[k] = s_M[bb];
-        }
-        npmax = max(npmax, npk[k]);
-      }
-      for (int p = 0; p < npmax; ++p) {
-        float mv[kI];
-        float4 uv[kI];
-#pragma unroll
-        for (int k = 0; k < kI; ++k) {
-          if (p < npk[k]) {
-            mv[k] = __ldg(rb[k] + p * rstride);
-            uv[k] = __ldg(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k]);
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < kI; ++k) {
-          if (p < npk[k]) {
-            const float wk = exp2f(mv[k] - Mk[k]);
-            acc[k].x = fmaf(wk, uv[k].x, acc[k].x);
-            acc[k].y = fmaf(wk, uv[k].y, acc[k].y);
-            acc[k].z = fmaf(wk, uv[k].z, acc[k].z);
-            acc[k].w = fmaf(wk, uv[k].w, acc[k].w);
-          }
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kI; ++k) {
-        const int idx = base + k * 256;
-        if (idx < nitems) {
-          const int bb = idx / k4;
-          const float inv = s_inv[bb];
-          store_split4(u_hi + bb * pitch + 4 * c4k[k], u_lo + bb * pitch + 4 * c4k[k],
-                       make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv));
-        }
-      }
-    }
-  }
+  merge_sweep(a, kTcRows, k4, r4, s_np, s_off, s_M, s_inv, [&](int bb, int c4, float4 v) {
+    store_split4(u_hi + bb * pitch + 4 * c4, u_lo + bb * pitch + 4 * c4, v);
+  });
   __syncthreads();
 
   // 3. out tile = W^V slice (32 x kp) . ubar^T (kp x 64)
@@ -907,7 +855,7 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse,
-                RaggedMap{nullptr, nullptr, nullptr}};
+                RaggedMap{nullptr, nullptr, nullptr, 0ull}, status_word()};
   if (ragged) a.ragged = *ragged;
   if (tc) {
     cudaLaunchConfig_t cfg{};

@@ -19,7 +19,9 @@
 //               commits stage releases and accumulator hand-offs.
 //   warps 2-5   epilogue: tcgen05.ld of the 128 x r accumulator (one TMEM
 //               lane per token), subtract mu W, round to bf16 (RNE), store
-//               with the caller's row and group strides. Double-buffered
+//               with the caller's row and group strides, or at each token's
+//               slot of a paged store (its page from the block table).
+//               Double-buffered
 //               accumulators let the epilogue of tile i overlap the MMAs of
 //               tile i+1.
 #include <cuda_bf16.h>
@@ -40,9 +42,38 @@ constexpr int kABytes = kTileM * kChunkK * 2;
 constexpr int kThreads = 192;   // 6 warps
 constexpr int kMaxStages = 12;  // enough bytes in flight to cover HBM latency at r = 16
 
+// Where each token's output row goes. Dense: row n of group g starts at
+// element g * zgs + n * zrs. Paged: token n belongs to sequence seq[n] (n
+// when seq is null) at position pos[n], and its row is row pos % page_size
+// of page block_table[s][pos / page_size], starting at element
+// page * page_stride + g * zgs + (pos % page_size) * zrs.
+struct OutMap {
+  __nv_bfloat16* z;
+  long long zrs, zgs;
+  int paged;
+  PagedOut pd;
+};
+
+// Element offset of token n's row (group 0), or -1 when a paged destination
+// is out of range: its sequence index, position or page lies outside the
+// table or the pool. Such a row is not written.
+__device__ __forceinline__ long long out_row(const OutMap& o, int n) {
+  if (!o.paged) return (long long)n * o.zrs;
+  const int s = o.pd.seq ? __ldg(o.pd.seq + n) : n;
+  const int p = __ldg(o.pd.pos + n);
+  // page_size * max_blocks < 2^31 is checked on the host
+  if (s < 0 || s >= o.pd.n_seq || p < 0 || p >= o.pd.max_blocks * o.pd.page_size) return -1;
+  const int page = __ldg(o.pd.block_table + (size_t)s * o.pd.max_blocks + p / o.pd.page_size);
+  if (page < 0 || page >= o.pd.num_pages) return -1;
+  return (long long)page * o.pd.page_stride + (long long)(p % o.pd.page_size) * o.zrs;
+}
+
 struct EncodeArgs {
   // work items are (tile, K split) pairs: item = tile * ksplit + split
   int N, G, d_loop, r, r_pad, K, nk, mtiles, tiles, tiles_per_cta;
+  // a tile is msub sub-tiles of 128 tokens that share each stage's W^T box
+  // (one accumulator each); nacc tiles' accumulators fit in TMEM at once
+  int msub, nacc;
   int ksplit, cpk;  // K splits per tile and chunks per split
   // tile order: token-major (all groups of a 128-token tile in a row, so a
   // token's G * d_loop input row is read at once) or group-major (one
@@ -54,8 +85,7 @@ struct EncodeArgs {
   const float* mu;
   const float* muw;  // precomputed mu W [G][r] (then mu is unused), or null
   const __nv_bfloat16* wt;
-  __nv_bfloat16* z;
-  long long zrs, zgs;
+  OutMap out;
   unsigned int* status;
 };
 
@@ -131,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = t_begin; item < t_end && ok; ++item) {
         const int tile = item / a.ksplit, split = item - tile * a.ksplit;
         const int g = a.token_major ? tile % a.G : tile / a.mtiles;
-        const int m0 = (a.token_major ? tile / a.G : tile - g * a.mtiles) * kTileM;
+        const int m0 = (a.token_major ? tile / a.G : tile - g * a.mtiles) * kTileM * a.msub;
         const int kc0 = split * a.cpk, kc1 = min(a.nk, kc0 + a.cpk);
         for (int kc = kc0; kc < kc1; ++kc, ++it) {
           const int s = it % a.nstage;
@@ -141,11 +171,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t full = smem_u32(&tail->full[s]);
-          mbar_arrive_expect_tx(full, kABytes + a.b_bytes);
+          mbar_arrive_expect_tx(full, a.msub * kABytes + a.b_bytes);
           const uint32_t sa = smem_u32(smem + (size_t)s * a.stage_bytes);
           const int t = kc / cpl, i0 = (kc - t * cpl) * kChunkK;
-          tma_load_4d(sa, &tx, i0, g, m0, t, full, pol_x);
-          tma_load_3d(sa + kABytes, &tw, kc * kChunkK, 0, g, full, pol_w);
+          // rows past N (a sub-tile beyond the last token) read as zeros
+          for (int sub = 0; sub < a.msub; ++sub)
+            tma_load_4d(sa + sub * kABytes, &tx, i0, g, m0 + sub * kTileM, t, full, pol_x);
+          tma_load_3d(sa + a.msub * kABytes, &tw, kc * kChunkK, 0, g, full, pol_w);
         }
       }
       if (!ok) {
@@ -163,14 +195,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int item = t_begin, lt = 0; item < t_end && ok; ++item, ++lt) {
-        const int acc = lt & 1;
-        const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
+        const int acc = lt % a.nacc;
+        const uint32_t aph = (uint32_t)(lt / a.nacc) & 1u;
         if (!wait_or_abort(smem_u32(&tail->tempty[acc]), aph ^ 1u, abort_flag, a.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d = tbase + (uint32_t)(acc * a.r_pad);
+        const uint32_t d = tbase + (uint32_t)(acc * a.msub * a.r_pad);
         const int split = item % a.ksplit;
         const int kc0 = split * a.cpk, kc1 = min(a.nk, kc0 + a.cpk);
         for (int kc = kc0; kc < kc1; ++kc, ++it) {
@@ -182,13 +214,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + (size_t)s * a.stage_bytes);
-          // descriptors built once per stage, advanced 32 B (2 x 16 B) per K step
-          const uint64_t a_base = desc_kmajor_sw128(sa);
-          const uint64_t b_base = desc_kmajor_sw128(sa + kABytes);
+          // descriptors built once per stage, advanced 32 B (2 x 16 B) per K
+          // step; every sub-tile multiplies the stage's one W^T box
+          const uint64_t b_base = desc_kmajor_sw128(sa + a.msub * kABytes);
+          for (int sub = 0; sub < a.msub; ++sub) {
+            const uint64_t a_base = desc_kmajor_sw128(sa + sub * kABytes);
 #pragma unroll
-          for (int kk = 0; kk < kChunkK / 16; ++kk)
-            umma_bf16(d, a_base + (uint64_t)(kk * 2), b_base + (uint64_t)(kk * 2), idesc,
-                      kc != kc0 || kk != 0);
+            for (int kk = 0; kk < kChunkK / 16; ++kk)
+              umma_bf16(d + (uint32_t)(sub * a.r_pad), a_base + (uint64_t)(kk * 2),
+                        b_base + (uint64_t)(kk * 2), idesc, kc != kc0 || kk != 0);
+          }
           umma_commit(smem_u32(&tail->empty[s]));
         }
         if (!ok) break;
@@ -218,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int item = t_begin, lt = 0; item < t_end; ++item, ++lt) {
       const int tile = item / a.ksplit, split = item - tile * a.ksplit;
       const int g = a.token_major ? tile % a.G : tile / a.mtiles;
-      const int m0 = (a.token_major ? tile / a.G : tile - g * a.mtiles) * kTileM;
+      const int m0 = (a.token_major ? tile / a.G : tile - g * a.mtiles) * kTileM * a.msub;
       if (g != cur_g && !a.part) {
         if (!epi_sync()) break;  // previous tile's readers of muw are done
         for (int c = ew; c < a.r; c += 4) {
@@ -236,48 +271,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!epi_sync()) break;
         cur_g = g;
       }
-      const int acc = lt & 1;
-      const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
+      const int acc = lt % a.nacc;
+      const uint32_t aph = (uint32_t)(lt / a.nacc) & 1u;
       const bool ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&tail->tfull[acc]), aph,
                                                             abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * a.r_pad);
-      const int n = m0 + row;
-      __nv_bfloat16* zrow = a.z + (size_t)g * a.zgs + (size_t)n * a.zrs;
-      // split K: this item's fp32 partial sum; k_encode_reduce finishes it
-      float* prow = a.part ? a.part + (((size_t)split * a.G + g) * a.N + n) * a.r : nullptr;
-      for (int cc = 0; cc < a.r_pad; cc += 16) {
-        float v[16];
-        tmem_ld16(taddr + cc, v);
-        if (n < a.N && prow) {
-#pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            const int c0 = cc + 8 * h8;
-            if (c0 < a.r) {
-              float4* dst = reinterpret_cast<float4*>(prow + c0);
-              dst[0] = make_float4(v[8 * h8 + 0], v[8 * h8 + 1], v[8 * h8 + 2], v[8 * h8 + 3]);
-              dst[1] = make_float4(v[8 * h8 + 4], v[8 * h8 + 5], v[8 * h8 + 6], v[8 * h8 + 7]);
-            }
+      for (int sub = 0; sub < a.msub; ++sub) {
+        const uint32_t taddr = tbase + ((uint32_t)(quarter * 32) << 16) +
+                               (uint32_t)((acc * a.msub + sub) * a.r_pad);
+        const int n = m0 + sub * kTileM + row;
+        long long roff = 0;
+        bool write = n < a.N;
+        if (write && !a.part) {
+          roff = out_row(a.out, n);
+          if (roff < 0) {
+            write = false;
+            if (g == 0) report_status(a.status, kStatusBadPagedInput);
           }
-        } else if (n < a.N) {
+        }
+        __nv_bfloat16* zrow = a.out.z + (size_t)g * a.out.zgs + roff;
+        // split K: this item's fp32 partial sum; k_encode_reduce finishes it
+        float* prow = a.part ? a.part + (((size_t)split * a.G + g) * a.N + n) * a.r : nullptr;
+        for (int cc = 0; cc < a.r_pad; cc += 16) {
+          float v[16];
+          tmem_ld16(taddr + cc, v);
+          if (n < a.N && prow) {
 #pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            const int c0 = cc + 8 * h8;
-            if (c0 < a.r) {
-              uint32_t w[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 p = __floats2bfloat162_rn(
-                    v[8 * h8 + 2 * e] - tail->muw[c0 + 2 * e],
-                    v[8 * h8 + 2 * e + 1] - tail->muw[c0 + 2 * e + 1]);
-                w[e] = *reinterpret_cast<const uint32_t*>(&p);
+            for (int h8 = 0; h8 < 2; ++h8) {
+              const int c0 = cc + 8 * h8;
+              if (c0 < a.r) {
+                float4* dst = reinterpret_cast<float4*>(prow + c0);
+                dst[0] = make_float4(v[8 * h8 + 0], v[8 * h8 + 1], v[8 * h8 + 2], v[8 * h8 + 3]);
+                dst[1] = make_float4(v[8 * h8 + 4], v[8 * h8 + 5], v[8 * h8 + 6], v[8 * h8 + 7]);
               }
-              *reinterpret_cast<uint4*>(zrow + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else if (write) {
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+              const int c0 = cc + 8 * h8;
+              if (c0 < a.r) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const __nv_bfloat162 p = __floats2bfloat162_rn(
+                      v[8 * h8 + 2 * e] - tail->muw[c0 + 2 * e],
+                      v[8 * h8 + 2 * e + 1] - tail->muw[c0 + 2 * e + 1]);
+                  w[e] = *reinterpret_cast<const uint32_t*>(&p);
+                }
+                *reinterpret_cast<uint4*>(zrow + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
             }
           }
         }
-      }
+      }  // sub-tiles
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tail->tempty[acc]));
@@ -356,8 +403,7 @@ __global__ void __launch_bounds__(256) k_encode_bias(const __nv_bfloat16* wt, co
 // partial loads in flight.
 __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const float* muw,
                                                        int ksplit, int G, int N, int r,
-                                                       __nv_bfloat16* z, long long zrs,
-                                                       long long zgs) {
+                                                       OutMap out, unsigned int* status) {
   const int r4 = r / 4;
   const long long total = (long long)G * N * r4;
   const size_t plane4 = (size_t)G * N * r / 4;  // float4 per split
@@ -365,6 +411,11 @@ __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const 
     const int c = (int)(i % r4) * 4;
     const long long gn = i / r4;
     const int n = (int)(gn % N), g = (int)(gn / N);
+    const long long roff = out_row(out, n);
+    if (roff < 0) {
+      if (g == 0 && c == 0) report_status(status, kStatusBadPagedInput);
+      continue;
+    }
     const float4* p = reinterpret_cast<const float4*>(part) + (size_t)i;
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int k0 = 0; k0 < ksplit; k0 += 8) {
@@ -388,7 +439,7 @@ __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const 
       s.w -= m.w;
     }
     const __nv_bfloat162 b0 = __floats2bfloat162_rn(s.x, s.y), b1 = __floats2bfloat162_rn(s.z, s.w);
-    *reinterpret_cast<uint2*>(z + (size_t)g * zgs + (size_t)n * zrs + c) =
+    *reinterpret_cast<uint2*>(out.z + (size_t)g * out.zgs + roff + c) =
         make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
   }
 }
@@ -448,7 +499,8 @@ size_t encode_workspace(int T, int N, int G, int d_loop, int r) {
 
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs,
-                      cudaStream_t stream, const float* muw, void* ws, size_t ws_bytes) {
+                      cudaStream_t stream, const float* muw, void* ws, size_t ws_bytes,
+                      const PagedOut* paged) {
   const int K = T * d_loop;
   const int r_pad = (r + 15) / 16 * 16;
   EncodeArgs a{};
@@ -459,6 +511,7 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   a.r_pad = r_pad;
   a.K = K;
   a.nk = K / kChunkK;
+  a.msub = 1;
   a.mtiles = (N + kTileM - 1) / kTileM;
   a.tiles = a.mtiles * G;
   // Few tiles and a long K (a wide LLA-2D stack at decode time) leave most
@@ -477,16 +530,29 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   }
   a.token_major = env_int("LLA_ENCODE_TOKEN_MAJOR", 0);
   a.b_bytes = r_pad * kChunkK * 2;
-  a.stage_bytes = kABytes + a.b_bytes;
+  // A wide W^T (r >= 128: its box is at least the 16 KB token box) is
+  // re-read from L2 for every tile. Tiles of two 128-token sub-tiles read
+  // each W^T box once for both, cutting the stage bytes per MMA by a third
+  // at r = 256. Unsplit writes only: split-K partials stay per 128 rows.
+  if (a.ksplit == 1 && r_pad >= 128 && N > kTileM)
+    a.msub = std::max(1, std::min(2, env_int("LLA_ENCODE_MSUB", 2)));
+  a.mtiles = (N + kTileM * a.msub - 1) / (kTileM * a.msub);
+  a.tiles = a.mtiles * G;
+  a.stage_bytes = a.msub * kABytes + a.b_bytes;
+  // two tiles' accumulators when they fit in the 512 TMEM columns, so the
+  // epilogue of one tile overlaps the next tile's MMAs
+  a.nacc = 2 * a.msub * r_pad <= 512 ? 2 : 1;
   uint32_t cols = 32;
-  while (cols < (uint32_t)(2 * r_pad)) cols <<= 1;
+  while (cols < (uint32_t)(a.nacc * a.msub * r_pad)) cols <<= 1;
   a.tmem_cols = cols;
   a.mu = mu;
   a.muw = muw;
   a.wt = static_cast<const __nv_bfloat16*>(wt);
-  a.z = static_cast<__nv_bfloat16*>(z);
-  a.zrs = zrs;
-  a.zgs = zgs;
+  a.out.z = static_cast<__nv_bfloat16*>(z);
+  a.out.zrs = zrs;
+  a.out.zgs = zgs;
+  a.out.paged = paged != nullptr;
+  if (paged) a.out.pd = *paged;
   a.status = status_word();
 
   const DeviceInfo di = device_info();
@@ -542,7 +608,7 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   if (a.part) {
     const long long outs = (long long)G * N * (r / 4);
     const int rgrid = (int)std::min<long long>((outs + 255) / 256, 4LL * di.sms);
-    k_encode_reduce<<<rgrid, 256, 0, stream>>>(a.part, muw, a.ksplit, G, N, r, a.z, zrs, zgs);
+    k_encode_reduce<<<rgrid, 256, 0, stream>>>(a.part, muw, a.ksplit, G, N, r, a.out, a.status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return check_cuda(e, "launch k_encode_reduce");
   }

@@ -81,8 +81,24 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct RaggedMap {
   const int4* seqinfo;
   const long long* cum;
-  const long long* plan;
+  const long long* plan;      // {total, share, stamp}
+  unsigned long long stamp;   // the stamp plan[2] must hold (else: no work)
 };
+
+// What a paged decode call runs: the plan kernel and the decode kernels
+// (kPlanAndDecode), the plan alone (kPlanOnly), or the decode kernels on a
+// plan an earlier kPlanOnly call left in the same workspace (kDecodePlanned).
+enum PagedMode { kPlanAndDecode = 0, kPlanOnly = 1, kDecodePlanned = 2 };
+
+// Identifies a paged plan: a 64-bit hash (FNV-1a) of everything the plan
+// depends on except the contents of the lengths and the table. k_plan_paged
+// stores it next to the plan; the kernels that read the plan compare it
+// first and do nothing (status LLA_DEVICE_PAGED_PLAN_MISMATCH) on a
+// mismatch, so a workspace that holds no plan for this call is never used.
+unsigned long long paged_plan_stamp(int family, int esz, int B, int H, int r_k, int r_v,
+                                    int page_size, int num_pages, const int* block_table,
+                                    int max_blocks, const int* seq_lens, int sink, int window,
+                                    int W, int pmin, int tile_tokens);
 
 size_t workspace_paged(int B, int H, int r_k, int r_v, int esz);
 
@@ -100,7 +116,8 @@ lla_status run_selftest_wait(unsigned int timeout_us, cudaStream_t stream);
 lla_status launch_plan_paged(const int* seq_lens, const int* block_table, int B, int H,
                              int page_size, int num_pages, int max_blocks, int sink, int window,
                              int W, int pmin, int tile_tokens, int4* seqinfo, long long* cum,
-                             long long* plan, int4* wstart, cudaStream_t stream);
+                             long long* plan, int4* wstart, unsigned long long stamp,
+                             cudaStream_t stream);
 
 size_t workspace_2d_paged(int B, int H, int r_k, int r_v);
 lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, int B, int H,
@@ -108,13 +125,15 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
                                const int* block_table, int max_blocks, const int* seq_lens,
                                int sink, int window, const float* dk, const float* dv,
                                const float* mu_k, const float* mu_v, float scale, float* out,
-                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                               PagedMode mode = kPlanAndDecode);
 lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int esz, int B, int H,
                             int d_h, int r_k, int r_v, int page_size, int num_pages,
                             const int* block_table, int max_blocks, const int* seq_lens, int sink,
                             int window, const float* dk, const float* dv, const float* mu_k,
                             const float* mu_v, float scale, float* out, float* lse, void* ws,
-                            size_t ws_bytes, cudaStream_t stream);
+                            size_t ws_bytes, cudaStream_t stream,
+                            PagedMode mode = kPlanAndDecode);
 
 // Kernels shared by the per-head and LLA-2D decode paths (decode.cu).
 // k_absorb writes q' (fp32, [B*H][r_k + d_r]) to qp when qp is non-null, and
@@ -144,9 +163,24 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
                          float* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
                          const float* q_rope = nullptr, int d_r = 0);
 
+// Destination of a latent write into a paged store (lla_encode_paged): token
+// n of sequence seq[n] (n when seq is null) at position pos[n] goes to row
+// pos % page_size of page block_table[s][pos / page_size]; page_stride is in
+// elements. Device arrays: block_table [n_seq][max_blocks], seq and pos [N].
+struct PagedOut {
+  const int* block_table;
+  const int* seq;
+  const int* pos;
+  int n_seq, max_blocks, page_size, num_pages;
+  long long page_stride;
+};
+
+// The latent write. With `paged` the output rows go to each token's slot of
+// a paged store (zrs, zgs are then the row and group strides inside a page).
 lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, const void* wt,
                       const float* mu, void* z, long long zrs, long long zgs, cudaStream_t stream,
-                      const float* muw = nullptr, void* ws = nullptr, size_t ws_bytes = 0);
+                      const float* muw = nullptr, void* ws = nullptr, size_t ws_bytes = 0,
+                      const PagedOut* paged = nullptr);
 
 // Bytes of the split-K workspace run_encode uses for this shape (0: the
 // shape has enough tiles and runs unsplit).

@@ -6,7 +6,9 @@
 // LLA-2D at inference" (absorbed attention reads latents directly).
 //
 // Every head of a sequence reads the same latents, so the H absorbed queries
-// against the shared latent store form real contractions:
+// against the shared latent store form real contractions (ranks that are
+// not whole 64-column boxes or 128-row tiles are zero-padded by the tensor
+// maps' out-of-range fill, which reads nothing from memory):
 //   S  [128 tokens x H] = Z^K_tile [128 x r_k] . Q'^T [r_k x H]
 //   U  [r_v x H]       += Z^V_tile^T [r_v x 128] . P [128 x H]
 // Both run as tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in
@@ -67,7 +69,8 @@ struct D2Args {
   const unsigned char* qsw;  // per sequence: Q' as bf16 in the MMA operand layout
   // paged store (seqinfo non-null): written by k_plan_paged
   const int4* seqinfo;      // [B] {kept tiles, tokens, sink tiles, first window tile}
-  const long long* plan;    // {total tiles, tiles per CTA}
+  const long long* plan;    // {total tiles, tiles per CTA, stamp}
+  unsigned long long stamp; // plan[2] must equal it, else no tile is taken
   const int4* cstart;       // [grid] first (sequence, 0, tile) of each CTA
   const int* block_table;   // [B][max_blocks]
   int max_blocks, page_size;
@@ -161,8 +164,10 @@ __device__ __forceinline__ bool tcur_kept(const TileCur& c, int pos) {
 __device__ __forceinline__ TileCur tcur_start(const D2Args& a) {
   TileCur c;
   if (a.seqinfo) {
+    // a CTA with no tiles (or a workspace that holds no plan for this call)
+    // still builds a cursor: its sequence index is kept inside [0, B)
     const int4 s = __ldg(a.cstart + blockIdx.x);
-    c.b = s.x;
+    c.b = min(max(s.x, 0), a.B - 1);
     c.j = s.z;
   } else {
     const int t = blockIdx.x * a.tpc;
@@ -200,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // a paged plan sizes the split on the device (k_plan_paged finished before
   // k_absorb started, so this is safe before griddepcontrol.wait)
-  const long long tiles = a.seqinfo ? a.plan[0] : (long long)a.tiles;
+  const bool plan_ok = !a.seqinfo || (unsigned long long)a.plan[2] == a.stamp;
+  const long long tiles = a.seqinfo ? (plan_ok ? a.plan[0] : 0LL) : (long long)a.tiles;
   const long long tpc = a.seqinfo ? a.plan[1] : (long long)a.tpc;
   const long long t_begin = blockIdx.x * tpc;
   const int ntile = (int)max(0LL, min(t_begin + tpc, tiles) - t_begin);
@@ -234,7 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = tl->tmem_base;
 
-  auto kboxes = [&](int kg) { return min(2, (a.r_k - kg * 128) / 64); };
+  // 64-column boxes of K group kg; the last one may run past r_k, where the
+  // tensor map fills zeros (and Q' holds zeros)
+  auto kboxes = [&](int kg) { return min(2, (a.r_k - kg * 128 + 63) / 64); };
 
   if (warp == 0 || warp == 6) {
     // ------------------------------ producers ------------------------------
@@ -646,9 +654,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 16; ++e) u[e] += t[e];
             }
+            // rows past r_v (zero-filled latent columns) are not stored
+            if (vg * 128 + row < a.r_v) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (h0 + e < a.H) rec[(size_t)(h0 + e) * a.pstride + 4 + vg * 128 + row] = u[e];
+              for (int e = 0; e < 16; ++e)
+                if (h0 + e < a.H) rec[(size_t)(h0 + e) * a.pstride + 4 + vg * 128 + row] = u[e];
+            }
           }
         }
 #pragma unroll
@@ -700,9 +711,11 @@ lla_status plan_2d(int B, int H, int N, int r_k, int r_v, D2Plan* p) {
   const int grid0 = std::max(1, std::min(d.tiles, di.sms));
   d.tpc = (d.tiles + grid0 - 1) / grid0;
   d.grid = (d.tiles + d.tpc - 1) / d.tpc;
+  // ranks that are not whole 64-column boxes (K) or 128-row MMA tiles (V)
+  // are padded up: the tensor maps fill the missing columns with zeros
   d.nkg = (r_k + 127) / 128;
-  d.nvg = r_v / 128;
-  d.qbuf_bytes = (r_k / 64) * d.hp * 128;
+  d.nvg = (r_v + 127) / 128;
+  d.qbuf_bytes = ((r_k + 63) / 64) * d.hp * 128;
   d.pbuf_bytes = 2 * d.hp * 128;
   const size_t fixed = 2 * (size_t)d.qbuf_bytes + 2 * (size_t)d.pbuf_bytes + sizeof(Tail2) + 1024;
   // Split the stages between the rings: each ring needs at least one
@@ -750,6 +763,7 @@ struct Paged2D {
   const int4* cstart;
   const int* block_table;
   int max_blocks, page_size, sink, window;
+  unsigned long long stamp;
 };
 
 // Absorb, the tensor-core kernel and the merge, shared by the dense and the
@@ -794,6 +808,7 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
   if (pg) {
     a.seqinfo = pg->seqinfo;
     a.plan = pg->plan;
+    a.stamp = pg->stamp;
     a.cstart = pg->cstart;
     a.block_table = pg->block_table;
     a.max_blocks = pg->max_blocks;
@@ -826,7 +841,7 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
   if (e != cudaSuccess) return check_cuda(e, "record timing event");
 
   if (pg) {  // sequence b's pieces: the CTAs of its tiles, cum[b] .. cum[b] + tiles - 1
-    RaggedMap rm{pg->seqinfo, pg->cum, pg->plan};
+    RaggedMap rm{pg->seqinfo, pg->cum, pg->plan, pg->stamp};
     return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 1, out, lse, stream,
                           &rm, true);
   }
@@ -853,7 +868,7 @@ lla_status plan_2d_paged(int B, int H, int r_k, int r_v, D2PagedPlan* pp) {
       al256(p.d.off_part + ((size_t)p.d.grid + B) * H * p.d.pstride * sizeof(float));
   p.off_cum = al256(p.off_seqinfo + (size_t)B * sizeof(int4));
   p.off_plan = al256(p.off_cum + (size_t)(B + 1) * sizeof(long long));
-  p.off_cstart = al256(p.off_plan + 2 * sizeof(long long));
+  p.off_cstart = al256(p.off_plan + 3 * sizeof(long long));
   p.ws_bytes = al256(p.off_cstart + (size_t)p.d.grid * sizeof(int4));
   *pp = p;
   return LLA_OK;
@@ -901,7 +916,8 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
                                const int* block_table, int max_blocks, const int* seq_lens,
                                int sink, int window, const float* dk, const float* dv,
                                const float* mu_k, const float* mu_v, float scale, float* out,
-                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream,
+                               PagedMode mode) {
   D2PagedPlan pp;
   lla_status st = plan_2d_paged(B, H, r_k, r_v, &pp);
   if (st != LLA_OK) return st;
@@ -919,6 +935,16 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
   pg.page_size = page_size;
   pg.sink = sink;
   pg.window = window;
+  pg.stamp = paged_plan_stamp(2, 2, B, 1, r_k, r_v, page_size, num_pages, block_table, max_blocks,
+                              seq_lens, sink, window, pp.d.grid, 1, kRows);
+  // 1. plan: tiles of kRows tokens, one worker per CTA (skipped when an
+  //    earlier plan-only call already left it in this workspace)
+  if (mode != kDecodePlanned) {
+    st = launch_plan_paged(seq_lens, block_table, B, 1, page_size, num_pages, max_blocks, sink,
+                           window, pp.d.grid, 1, kRows, const_cast<int4*>(pg.seqinfo), pg.cum,
+                           pg.plan, const_cast<int4*>(pg.cstart), pg.stamp, stream);
+    if (st != LLA_OK || mode == kPlanOnly) return st;
+  }
   // The pool read page by page: rows of a page, pages outermost; boxes of
   // 64 rows when pages hold an odd multiple of 64 tokens.
   const uint32_t box_rows = page_size % kRows ? kRows / 2 : kRows;
@@ -935,11 +961,6 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
     const uint32_t box[3] = {64, box_rows, 1};
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
-  // 1. plan: tiles of kRows tokens, one worker per CTA
-  st = launch_plan_paged(seq_lens, block_table, B, 1, page_size, num_pages, max_blocks, sink,
-                         window, pp.d.grid, 1, kRows, const_cast<int4*>(pg.seqinfo), pg.cum,
-                         pg.plan, const_cast<int4*>(pg.cstart), stream);
-  if (st != LLA_OK) return st;
   return launch_2d(q, tk, tv, B, H, d_h, 0, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, pp.d,
                    wsb, &pg, stream);
 }

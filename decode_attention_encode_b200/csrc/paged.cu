@@ -40,6 +40,7 @@ struct PlanArgs {
   long long* cum;
   long long* plan;
   int4* wstart;
+  unsigned long long stamp;
   unsigned int* status;
 };
 
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan_paged(PlanArgs p) {
     p.cum[p.B] = total;
     p.plan[0] = total;
     p.plan[1] = P;
+    p.plan[2] = (long long)p.stamp;  // this plan's identity, checked by its readers
     s_total = total;
     s_P = P;
   }
@@ -178,7 +180,7 @@ lla_status plan_paged(int B, int H, int r_k, int r_v, int esz, PagedPlan* pp) {
       align_up(p.d.off_part + (size_t)(p.d.W + units) * p.d.pstride * sizeof(float), 256);
   p.off_cum = align_up(p.off_seqinfo + (size_t)B * sizeof(int4), 256);
   p.off_plan = align_up(p.off_cum + (size_t)(B + 1) * sizeof(long long), 256);
-  p.off_wstart = align_up(p.off_plan + 2 * sizeof(long long), 256);
+  p.off_wstart = align_up(p.off_plan + 3 * sizeof(long long), 256);
   p.ws_bytes = align_up(p.off_wstart + (size_t)p.d.W * sizeof(int4), 256);
   p.d.ws_bytes = p.ws_bytes;
   *pp = p;
@@ -187,10 +189,34 @@ lla_status plan_paged(int B, int H, int r_k, int r_v, int esz, PagedPlan* pp) {
 
 }  // namespace
 
+unsigned long long paged_plan_stamp(int family, int esz, int B, int H, int r_k, int r_v,
+                                    int page_size, int num_pages, const int* block_table,
+                                    int max_blocks, const int* seq_lens, int sink, int window,
+                                    int W, int pmin, int tile_tokens) {
+  const unsigned long long v[] = {(unsigned long long)family, (unsigned long long)esz,
+                                  (unsigned long long)B, (unsigned long long)H,
+                                  (unsigned long long)r_k, (unsigned long long)r_v,
+                                  (unsigned long long)page_size, (unsigned long long)num_pages,
+                                  (unsigned long long)(uintptr_t)block_table,
+                                  (unsigned long long)max_blocks,
+                                  (unsigned long long)(uintptr_t)seq_lens,
+                                  (unsigned long long)sink, (unsigned long long)window,
+                                  (unsigned long long)W, (unsigned long long)pmin,
+                                  (unsigned long long)tile_tokens};
+  unsigned long long h = 1469598103934665603ull;  // FNV-1a, byte by byte
+  for (unsigned long long x : v)
+    for (int i = 0; i < 8; ++i) {
+      h ^= (x >> (8 * i)) & 0xffu;
+      h *= 1099511628211ull;
+    }
+  return h ? h : 1ull;
+}
+
 lla_status launch_plan_paged(const int* seq_lens, const int* block_table, int B, int H,
                              int page_size, int num_pages, int max_blocks, int sink, int window,
                              int W, int pmin, int tile_tokens, int4* seqinfo, long long* cum,
-                             long long* plan, int4* wstart, cudaStream_t stream) {
+                             long long* plan, int4* wstart, unsigned long long stamp,
+                             cudaStream_t stream) {
   PlanArgs p{};
   p.seq_lens = seq_lens;
   p.block_table = block_table;
@@ -208,6 +234,7 @@ lla_status launch_plan_paged(const int* seq_lens, const int* block_table, int B,
   p.cum = cum;
   p.plan = plan;
   p.wstart = wstart;
+  p.stamp = stamp;
   p.status = status_word();
   k_plan_paged<<<1, kPlanThreads, 0, stream>>>(p);
   return check_cuda(cudaGetLastError(), "launch k_plan_paged");
@@ -224,7 +251,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
                             const int* block_table, int max_blocks, const int* seq_lens, int sink,
                             int window, const float* dk, const float* dv, const float* mu_k,
                             const float* mu_v, float scale, float* out, float* lse, void* ws,
-                            size_t ws_bytes, cudaStream_t stream) {
+                            size_t ws_bytes, cudaStream_t stream, PagedMode mode) {
   PagedPlan pp;
   lla_status st = plan_paged(B, H, r_k, r_v, esz, &pp);
   if (st != LLA_OK) return st;
@@ -246,12 +273,18 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)d.smem_bytes);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_stream_paged)");
+  const unsigned long long stamp =
+      paged_plan_stamp(1, esz, B, H, r_k, r_v, page_size, num_pages, block_table, max_blocks,
+                       seq_lens, sink, window, d.W, 2 * d.tile, 0);
 
   // 1. plan (a plain launch: it completes before k_absorb starts, so the
-  //    streaming kernel may read its results before griddepcontrol.wait)
-  st = launch_plan_paged(seq_lens, block_table, B, H, page_size, num_pages, max_blocks, sink,
-                         window, d.W, 2 * d.tile, 0, seqinfo, cum, plan, wstart, stream);
-  if (st != LLA_OK) return st;
+  //    streaming kernel may read its results before griddepcontrol.wait; a
+  //    planned call relies on the plan call having been ordered before it)
+  if (mode != kDecodePlanned) {
+    st = launch_plan_paged(seq_lens, block_table, B, H, page_size, num_pages, max_blocks, sink,
+                           window, d.W, 2 * d.tile, 0, seqinfo, cum, plan, wstart, stamp, stream);
+    if (st != LLA_OK || mode == kPlanOnly) return st;
+  }
   // 2. absorb (plain launch)
   st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, nullptr, 0,
                      small_gemm_tc(esz, B, r_k, r_v));
@@ -277,10 +310,12 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
     a.seqinfo = seqinfo;
     a.cum = cum;
     a.plan = plan;
+    a.stamp = stamp;
     a.wstart = wstart;
     a.block_table = block_table;
     a.max_blocks = max_blocks;
     a.page_size = page_size;
+    a.num_pages = num_pages;
     a.H = H;
     a.B = B;
     cudaLaunchAttribute pdl[1];
@@ -301,7 +336,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
     if (e != cudaSuccess) return check_cuda(e, "record timing event");
   }
   // 4. combine over the ragged piece map
-  RaggedMap rm{seqinfo, cum, plan};
+  RaggedMap rm{seqinfo, cum, plan, stamp};
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 0, out, lse, stream,
                         &rm, small_gemm_tc(esz, B, r_k, r_v));
 }

@@ -392,6 +392,9 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   const int nwarps = blockDim.x >> 5;
   const long long w = (long long)blockIdx.x * nwarps + warp;
   if (w >= a.W) return;
+  // a workspace that does not hold this call's plan: no work (the merge
+  // reports it and writes empty results)
+  if ((unsigned long long)a.plan[2] != a.stamp) return;
   const long long total = a.plan[0], P = a.plan[1];
   const long long f0 = w * P;
   if (f0 >= total) return;
@@ -434,6 +437,13 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
       cblk = blk;
       nblk = blk + 1 < a.max_blocks ? blk + 1 : -1;
       if (nblk >= 0) npage = __ldg(a.block_table + (size_t)b * a.max_blocks + nblk);
+      // The plan checked every page it uses, but a table changed after the
+      // plan was made is read here: an index outside the pool is reported
+      // and replaced by page 0, so no copy leaves the pool.
+      if (cpage < 0 || cpage >= a.num_pages) {
+        report_status(a.status, kStatusBadPagedInput);
+        cpage = 0;
+      }
     }
     return cpage;
   };

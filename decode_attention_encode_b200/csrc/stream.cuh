@@ -36,10 +36,12 @@ struct StreamArgs {
   // Paged / ragged store (paged kernels only; written by k_plan_paged):
   const int4* seqinfo;     // [B] {kept tokens n, sink part s, position gap, 0}
   const long long* cum;    // [B+1] start of sequence b in the flattened range
-  const long long* plan;   // {total tokens, tokens per warp}
+  const long long* plan;   // {total tokens, tokens per warp, stamp}
+  unsigned long long stamp;  // plan[2] must equal it, else the kernel does nothing
   const int4* wstart;      // [W] first (b, h, i) of each warp's range
   const int* block_table;  // [B][max_blocks]
   int max_blocks, page_size, H, B;
+  int num_pages;           // page indices are checked against it as they are read
 };
 
 // Per-sequence record of the paged plan: sequence b attends n tokens; kept

@@ -204,6 +204,12 @@ class EncodeConfig:
 
 C5_ENCODE = EncodeConfig("encode_32x", L=24, T=4, G=16, d_loop=128, r=16, N=32768,
                          n_cal=2048)
+# the LLA-2D latent write of a 32768-token prefill: each token's whole stack
+# (T loops x 16 heads x 128 channels = 8192) to one r = 256 latent per
+# (layer, axis); a tensor-bound GEMM at about 250 flop/B
+C4_ENCODE = EncodeConfig("encode2d_32x", L=24, T=4, G=1, d_loop=2048, r=256, N=32768,
+                         n_cal=512)
+ENCODE_CONFIGS = {c.name: c for c in (C5_ENCODE, C4_ENCODE)}
 
 # the 4x geometry with a 64-wide decoupled rotary branch on the key side
 C2_ROPE = DecodeConfig("perhead_4x_rope", L=24, T=4, H=16, d_h=128, r_k=128, r_v=128, B=64,
@@ -215,8 +221,12 @@ C4_PAGED = DecodeConfig("lla2d_32x_paged", L=24, T=4, H=16, d_h=128, r_k=256, r_
 # the same batch in 64-token pages: every 128-token tile spans two pages
 C4_PAGED64 = DecodeConfig("lla2d_32x_paged64", L=24, T=4, H=16, d_h=128, r_k=256, r_v=256, B=256,
                           N=8192, dtype="bf16", decay=True, two_d=True, page_size=64, spread=0.5)
+# the 32x LLA-2D geometry with a 64-wide rotary key shared by every head:
+# key rows [256 latent | 64 rotary], 320 wide
+C4_ROPE = DecodeConfig("lla2d_32x_rope", L=24, T=4, H=16, d_h=128, r_k=256, r_v=256, B=256,
+                       N=8192, dtype="bf16", decay=True, two_d=True, d_r=64)
 DECODE_CONFIGS = {c.name: c for c in (C1, C2, C3, C4, C5_DECODE, C2_PAGED, C2_ROPE, C4_PAGED,
-                                      C4_PAGED64)}
+                                      C4_PAGED64, C4_ROPE)}
 
 
 def sample_units(B: int, L: int, T: int, H: int, n_random: int = 32, seed: int = 0):

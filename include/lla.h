@@ -56,9 +56,16 @@ typedef enum { LLA_F32 = 0, LLA_BF16 = 1 } lla_dtype;
 
 /* Device status bits reported by lla_device_status(). */
 #define LLA_DEVICE_WAIT_TIMEOUT 0x1u     /* a bounded device wait ran out */
-#define LLA_DEVICE_BAD_PAGED_INPUT 0x2u  /* lla_decode_attn_paged: a length or
+#define LLA_DEVICE_BAD_PAGED_INPUT 0x2u  /* a paged decode found a length or
                                             page index out of range (that
-                                            sequence was treated as empty) */
+                                            sequence was treated as empty),
+                                            or lla_encode_paged a token's
+                                            sequence, position or page (that
+                                            token was not written) */
+#define LLA_DEVICE_PAGED_PLAN_MISMATCH 0x4u /* a *_paged_planned call found no
+                                            plan for itself in its workspace
+                                            (nothing was decoded: out = 0,
+                                            lse = -inf) */
 
 /* Human-readable name of a status code. Never NULL. */
 LLA_API const char *lla_status_string(lla_status s);
@@ -297,6 +304,48 @@ LLA_API lla_status lla_decode_attn_paged(const float *q, const void *zk_pages,
                                          void *stream);
 
 /* --------------------------------------------------------------------------
+ * A paged decode step planned once. Every paged decode call first runs a
+ * small plan kernel: it checks the lengths and the block-table entries in
+ * use and splits the ragged token range over the streaming warps. A
+ * looped model makes T x L calls per decode step over the same lengths and
+ * table, so the plan can be made once per step:
+ *   lla_decode_attn_paged_plan  runs only that kernel, writing the plan into
+ *     the workspace (arguments as lla_decode_attn_paged; the query-side
+ *     arrays are not needed);
+ *   lla_decode_attn_paged_planned  is lla_decode_attn_paged without the
+ *     plan kernel: it reuses the plan in its workspace.
+ * The planned call must use the same workspace, zdt, B, H, r_k, r_v,
+ * page_size, num_pages, block_table and seq_lens pointers, max_blocks, sink
+ * and window as the plan call, be ordered after it (same stream, or
+ * synchronised), and come before the lengths or the table change. The plan
+ * carries a stamp of those arguments: a planned call whose workspace holds
+ * no matching plan decodes nothing (out = 0, lse = -inf) and sets
+ * LLA_DEVICE_PAGED_PLAN_MISMATCH. If the table's contents change after the
+ * plan, a page index outside the pool is still caught as it is read (page 0
+ * is read instead, and LLA_DEVICE_BAD_PAGED_INPUT is set), so no copy leaves
+ * the pool; the result is then undefined. Calls that share the workspace
+ * between the plan and its planned calls must not overwrite it (the plan
+ * region is written only by plan calls and unplanned paged calls).
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla_decode_attn_paged_plan(lla_dtype zdt, int B, int H, int r_k, int r_v,
+                                              int page_size, int num_pages,
+                                              const int *block_table, int max_blocks,
+                                              const int *seq_lens, int sink, int window,
+                                              void *workspace, size_t ws_bytes, void *stream);
+
+LLA_API lla_status lla_decode_attn_paged_planned(const float *q, const void *zk_pages,
+                                                 const void *zv_pages, lla_dtype zdt, int B,
+                                                 int H, int d_h, int r_k, int r_v,
+                                                 int page_size, int num_pages,
+                                                 const int *block_table, int max_blocks,
+                                                 const int *seq_lens, int sink, int window,
+                                                 const float *dk_t, const float *dv_t,
+                                                 const float *mu_k_t, const float *mu_v_t,
+                                                 float scale, float *out, float *lse,
+                                                 void *workspace, size_t ws_bytes,
+                                                 void *stream);
+
+/* --------------------------------------------------------------------------
  * LLA-2D absorbed decode, one (layer d, loop t) step (§3 "The LLA-2D
  * variant": one latent per token and layer, decoded into every head).
  *
@@ -308,10 +357,12 @@ LLA_API lla_status lla_decode_attn_paged(const float *q, const void *zk_pages,
  * and fp32 accumulation. The absorbed query and dv_t ubar are formed on the
  * tensor cores from split (hi + lo) bf16 operands with fp32 accumulation,
  * within 3 * 2^-16 of each product term.
- * Limits: H <= 32 (padded to 16 or 32 inside), r_k a multiple of 64 and
- * r_v a multiple of 128, both at most 256, d_h 1..256, 1 <= N <= n_cap.
- * Outside them the call returns LLA_ERR_UNSUPPORTED and the workspace query
- * returns 0.
+ * Limits: H <= 32 (padded to 16 or 32 inside), r_k and r_v multiples of 8,
+ * at most 256, d_h 1..256, 1 <= N <= n_cap. Inside, r_k is padded to whole
+ * 64-column boxes and r_v to whole 128-row tiles with zeros that the tensor
+ * maps supply without reading memory (the padding costs tensor-core work,
+ * not HBM traffic). Outside the limits the call returns LLA_ERR_UNSUPPORTED
+ * and the workspace query returns 0.
  * -------------------------------------------------------------------------- */
 LLA_API size_t lla2d_decode_attn_workspace(int B, int H, int N, int r_k, int r_v);
 
@@ -331,8 +382,8 @@ LLA_API lla_status lla2d_decode_attn(const float *q, const void *zk, const void 
  * §7 "Per-head LLA versus LLA-2D at inference" applied to §3 "The LLA-2D
  * variant"); q_rope [B][H][d_r] fp32 is each head's rotated rotary query.
  *   zk  [B][n_cap][r_k + d_r] bf16; zv [B][n_cap][r_v] bf16.
- *   r_k + d_r a multiple of 64, at most 384; d_r a positive multiple of 8;
- *   r_v a multiple of 128, at most 256; H <= 32.
+ *   r_k + d_r at most 384; r_k and d_r positive multiples of 8;
+ *   r_v a multiple of 8, at most 256; H <= 32.
  *   workspace  lla2d_decode_attn_workspace(B, H, N, r_k + d_r, r_v) bytes
  *   (that query takes the key-row width, up to 384).
  * The rotary query is rounded to bf16 with the absorbed query for the
@@ -388,6 +439,28 @@ LLA_API lla_status lla2d_decode_attn_paged(const float *q, const void *zk_pages,
                                            float scale, float *out, float *lse,
                                            void *workspace, size_t ws_bytes,
                                            void *stream);
+
+/* The LLA-2D paged step planned once: the same pair as
+ * lla_decode_attn_paged_plan / lla_decode_attn_paged_planned (and the same
+ * rules), for lla2d_decode_attn_paged. The plan call takes no element type
+ * (LLA-2D latents are bf16). */
+LLA_API lla_status lla2d_decode_attn_paged_plan(int B, int H, int r_k, int r_v, int page_size,
+                                                int num_pages, const int *block_table,
+                                                int max_blocks, const int *seq_lens, int sink,
+                                                int window, void *workspace, size_t ws_bytes,
+                                                void *stream);
+
+LLA_API lla_status lla2d_decode_attn_paged_planned(const float *q, const void *zk_pages,
+                                                   const void *zv_pages, lla_dtype zdt, int B,
+                                                   int H, int d_h, int r_k, int r_v,
+                                                   int page_size, int num_pages,
+                                                   const int *block_table, int max_blocks,
+                                                   const int *seq_lens, int sink, int window,
+                                                   const float *dk_t, const float *dv_t,
+                                                   const float *mu_k_t, const float *mu_v_t,
+                                                   float scale, float *out, float *lse,
+                                                   void *workspace, size_t ws_bytes,
+                                                   void *stream);
 
 /* --------------------------------------------------------------------------
  * Latent write (§3 Eq. 2 over the loop-major stack of Eq. 1):
@@ -457,6 +530,58 @@ LLA_API lla_status lla_encode_with_bias(const void *x, lla_dtype xdt, int T, int
                                         void *z, long long z_row_stride,
                                         long long z_group_stride, void *workspace,
                                         size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Latent write into a paged store: lla_encode_with_bias's latents (§3 Eq. 2
+ * over the loop-major stack of Eq. 1) written at each token's slot of the
+ * page pool that lla_decode_attn_paged and lla2d_decode_attn_paged read.
+ * A serving loop calls it once per (layer, axis) and decode step to append
+ * every sequence's newest token; a chunked prefill passes many tokens of
+ * one sequence. The pages measure capacity with a latent store whose size
+ * bounds the batch (§7 "Memory", Table 7); the paged layout is this
+ * library's, as for the paged decode calls.
+ *
+ * Token n belongs to sequence s = seq_idx[n] (s = n when seq_idx is NULL)
+ * at position p = positions[n]. Its row c = bf16_rne(xs_n W_down - muw) of
+ * group g is written to the r elements starting at
+ *   z_pages + page * z_page_stride + g * z_group_stride
+ *           + (p % page_size) * z_row_stride,
+ *   page = block_table[s][p / page_size].
+ * For a per-head pool [num_pages][H][page_size][r] (G = H) the strides are
+ * (H * page_size * r, page_size * r, r); for an LLA-2D pool
+ * [num_pages][page_size][r] (G = 1) they are (page_size * r, 0, r). A key
+ * row [latent r_k | rotary key d_r] takes z_row_stride = r_k + d_r and
+ * keeps its rotary part. Nothing else in the pool is written.
+ *
+ * Arguments beyond lla_encode_with_bias's (x, xdt, T, N, G, d_loop, r,
+ * w_down_t, muw, workspace, ws_bytes, stream: same meaning and limits; the
+ * workspace query is lla_encode_with_bias_workspace):
+ *   z_pages       bf16 page pool, 16-byte aligned.
+ *   z_page_stride, z_group_stride, z_row_stride  in elements, multiples of
+ *                 8, z_row_stride >= r. Rows of one page must not overlap
+ *                 (groups outer or rows outer), and z_page_stride must cover
+ *                 a whole page: >= (G-1) z_group_stride + (page_size-1)
+ *                 z_row_stride + r.
+ *   page_size     tokens per page, >= 1; num_pages >= 1.
+ *   block_table   [n_seq][max_blocks] int32 device array; n_seq,
+ *                 max_blocks >= 1 and page_size * max_blocks < 2^31.
+ *   seq_idx       [N] int32 device array, or NULL.
+ *   positions     [N] int32 device array.
+ * Sequence indices, positions and page indices are read only on the device.
+ * A token whose sequence index lies outside [0, n_seq), whose position
+ * lies outside [0, max_blocks * page_size), or whose page lies outside
+ * [0, num_pages), is not written, and LLA_DEVICE_BAD_PAGED_INPUT is set in
+ * the device status word. Two tokens of one call must not name the same
+ * slot (their writes would race). Host-side errors as for lla_encode.
+ * -------------------------------------------------------------------------- */
+LLA_API lla_status lla_encode_paged(const void *x, lla_dtype xdt, int T, int N, int G,
+                                    int d_loop, int r, const void *w_down_t,
+                                    const float *muw, void *z_pages,
+                                    long long z_page_stride, long long z_group_stride,
+                                    long long z_row_stride, int page_size, int num_pages,
+                                    const int *block_table, int n_seq, int max_blocks,
+                                    const int *seq_idx, const int *positions,
+                                    void *workspace, size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

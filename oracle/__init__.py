@@ -17,7 +17,8 @@ What is here, each in fp64:
   * ``decode_unit_absorbed``: the §7 bilinear identities, kept only so the
     tests can compare the two forms by brute force.
   * ``encode``: the latent write c = (x - mu) W_down (§3 Eq. 2) over a
-    loop-major stack (§3 Eq. 1).
+    loop-major stack (§3 Eq. 1); ``paged_write`` places its rows in a paged
+    store through a block table (the layout ``paged_decode`` reads).
   * ``svd_init``: §3 "Initialization and conversion": centre by the
     per-loop mean, take the top-r right singular vectors of the stacked-loop
     matrix as W_down, and its loop slices as the initial W_up,t.
@@ -451,6 +452,43 @@ def encode(x, w, mu=None, nthreads: int = 0):
     _load().oracle_encode(T, N, G, d_loop, r, _ptr(x), _ptr(w), _ptr(mu), _ptr(z),
                           int(nthreads))
     return z
+
+
+def paged_write(pool, z, block_table, positions, seq_idx=None):
+    """Places encoded latent rows in a paged store: the write side of the
+    paged layout ``paged_decode`` and ``paged2d_decode`` read.
+
+    Token n belongs to sequence s = seq_idx[n] (s = n when seq_idx is None)
+    at position p = positions[n]; its row lands in row p % page_size of page
+    block_table[s, p // page_size]. pool is [P, G, page_size, r_row] for a
+    per-head store (G heads) or [P, page_size, r_row] for LLA-2D (G = 1);
+    z is [G, N, r] as ``encode`` returns it, and only the first r values of
+    a row (the latent part of a [latent | rotary key] row) are written. A
+    token whose sequence index, position or page lies outside the table or
+    the pool is not written. Returns (new pool, list of skipped tokens)."""
+    pool = np.array(pool, dtype=np.float64, copy=True)
+    z = _f64(z)
+    block_table = np.asarray(block_table)
+    two_d = pool.ndim == 3
+    ps = pool.shape[1] if two_d else pool.shape[2]
+    G, N, r = z.shape
+    n_seq, max_blocks = block_table.shape
+    skipped = []
+    for n in range(N):
+        s = n if seq_idx is None else int(seq_idx[n])
+        p = int(positions[n])
+        if not (0 <= s < n_seq and 0 <= p < max_blocks * ps):
+            skipped.append(n)
+            continue
+        page = int(block_table[s, p // ps])
+        if not 0 <= page < pool.shape[0]:
+            skipped.append(n)
+            continue
+        if two_d:
+            pool[page, p % ps, :r] = z[0, n]
+        else:
+            pool[page, :, p % ps, :r] = z[:, n]
+    return pool, skipped
 
 
 def svd_init(X, r, T):

@@ -183,3 +183,20 @@ def pad_block_table(inp, bt, fill_page=0):
     t = torch.from_numpy(full).to(inp["q"].device)
     inp["block_table_alloc"] = t
     inp["block_table"] = t[:B]
+
+
+def check_encoded(z_gpu, z_ref):
+    """A latent write against the oracle's Eq. 2: the kernel rounds its fp32
+    result to bf16 once (round to nearest even), so each element may differ
+    from the exact value by half a bf16 ulp (2^-9 relative) plus fp32
+    accumulation error. Checks the stated gate max|z_gpu - z_ref| / max|z_ref|
+    <= 2e-2 and the tighter element-wise bound 2^-8 |z_ref| + 1e-4 max|z_ref|.
+    Returns the relative error."""
+    zg = to_f64(z_gpu) if isinstance(z_gpu, torch.Tensor) else np.asarray(z_gpu)
+    scale = np.abs(z_ref).max()
+    err = np.abs(zg - z_ref).max() / scale
+    assert err <= TOL_BF16_REL, f"relative error {err:.3e}"
+    bound = 2.0 ** -8 * np.abs(z_ref) + 1e-4 * scale
+    bad = np.abs(zg - z_ref) > bound
+    assert not bad.any(), f"{bad.sum()} elements outside rounding bound; max rel {err:.2e}"
+    return err

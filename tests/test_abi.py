@@ -1,17 +1,27 @@
 """Host-side checks of the C ABI: the library builds, loads, exports every
 symbol include/lla.h declares, and rejects bad arguments before touching a
-device. Nothing here launches a kernel."""
+device. Nothing here launches a kernel.
+
+Many calls below pass placeholder pointers that are never valid device
+addresses; each is meant to fail a host-side check first. So that a case
+which wrongly passed those checks could never reach a kernel, this file
+runs only where no CUDA device is visible (the CPU test pass)."""
 
 import ctypes
 import os
 import re
 
 import pytest
+import torch
 
 import decode_attention_encode_b200 as lla
 from decode_attention_encode_b200 import _lib
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+pytestmark = pytest.mark.skipif(
+    torch.cuda.is_available(),
+    reason="placeholder-pointer calls run only where no CUDA device is visible")
 
 
 def header_functions():
@@ -103,11 +113,16 @@ def test_lla2d_rejects_unsupported_shapes_on_the_host():
 
     assert call(zdt=0, r_k=128, r_v=128) == _lib.LLA_ERR_UNSUPPORTED
     assert call(H=33) == _lib.LLA_ERR_UNSUPPORTED
-    assert call(r_k=96) == _lib.LLA_ERR_UNSUPPORTED
-    assert call(r_v=64) == _lib.LLA_ERR_UNSUPPORTED
+    assert call(r_k=12) == _lib.LLA_ERR_INVALID_ARG          # ranks are multiples of 8
+    assert call(r_v=264) == _lib.LLA_ERR_INVALID_ARG
+    # ranks that are not whole boxes or tiles are accepted (zero-padded
+    # inside): these stop at the workspace check
+    assert call(r_k=96, r_v=160) == _lib.LLA_ERR_WORKSPACE
+    assert call(r_k=8, r_v=72) == _lib.LLA_ERR_WORKSPACE
     assert call(ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
     assert lla.lla2d_decode_attn_workspace(2, 33, 8, 256, 256) == 0
-    assert lla.lla2d_decode_attn_workspace(2, 16, 8, 256, 192) == 0
+    assert lla.lla2d_decode_attn_workspace(2, 16, 8, 256, 196) == 0
+    assert lla.lla2d_decode_attn_workspace(2, 16, 8, 96, 160) > 0
     assert lla.lla2d_decode_attn_workspace(256, 16, 8192, 256, 256) > 256 * 16 * 256 * 4
 
 
@@ -132,6 +147,75 @@ def test_encode_rejects_bad_arguments_on_the_host():
 
 
 FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: every call below fails on the host
+
+
+@pytest.mark.parametrize("fn", ["lla_decode_attn_paged_plan", "lla2d_decode_attn_paged_plan"])
+def test_paged_plan_rejects_bad_arguments_on_the_host(fn):
+    h = lla.lib()
+    two_d = fn.startswith("lla2d")
+
+    def call(**over):
+        args = dict(zdt=1, B=2, H=16, r_k=128, r_v=128, ps=64, P=9, bt=FAKE, mb=3, sl=FAKE,
+                    sink=0, window=0, ws=FAKE, ws_bytes=0, stream=None)
+        args.update(over)
+        if two_d:
+            del args["zdt"]
+        return getattr(h, fn)(*args.values())
+
+    cases = [
+        (dict(bt=None), _lib.LLA_ERR_INVALID_ARG, b"non-NULL"),
+        (dict(sl=ctypes.c_void_p(0x100002)), _lib.LLA_ERR_INVALID_ARG, b"4-byte"),
+        (dict(B=0), _lib.LLA_ERR_INVALID_ARG, b"B and H"),
+        (dict(r_k=12), _lib.LLA_ERR_INVALID_ARG, b"multiples of 8"),
+        (dict(P=0), _lib.LLA_ERR_INVALID_ARG, b"num_pages"),
+        (dict(mb=1 << 28), _lib.LLA_ERR_INVALID_ARG, b"31 bits"),
+        (dict(window=-1), _lib.LLA_ERR_INVALID_ARG, b"sink and window"),
+        (dict(ws=ctypes.c_void_p(0x100008)), _lib.LLA_ERR_INVALID_ARG, b"16-byte"),
+        (dict(ws_bytes=16), _lib.LLA_ERR_WORKSPACE, b"workspace"),
+    ]
+    if two_d:
+        cases += [(dict(H=33), _lib.LLA_ERR_UNSUPPORTED, b"H <= 32"),
+                  (dict(ps=96), _lib.LLA_ERR_UNSUPPORTED, b"multiple of 64")]
+    else:
+        cases += [(dict(zdt=3), _lib.LLA_ERR_INVALID_ARG, b"zdt"),
+                  (dict(zdt=0, r_k=136), _lib.LLA_ERR_INVALID_ARG, b"multiples of 8")]
+    for over, code, why in cases:
+        assert call(**over) == code, over
+        assert why in h.lla_last_error(), (over, h.lla_last_error())
+
+
+def test_paged_encode_rejects_bad_arguments_on_the_host():
+    h = lla.lib()
+
+    def call(**over):
+        # a per-head pool [P=9][G=2][page_size=4][r_row=24] written at r = 16:
+        # one page spans (G-1)*96 + (4-1)*24 + 16 = 184 elements
+        args = dict(x=FAKE, xdt=1, T=4, N=10, G=2, d_loop=128, r=16, w=FAKE, muw=None, z=FAKE,
+                    zps=2 * 4 * 24, zgs=4 * 24, zrs=24, ps=4, P=9, bt=FAKE, n_seq=10, mb=3,
+                    seq=None, pos=FAKE, ws=None, ws_bytes=0, stream=None)
+        args.update(over)
+        return h.lla_encode_paged(*args.values())
+
+    # every case must fail on the host for its own reason (the message says
+    # which), so no placeholder pointer can reach a launch
+    for over, why in [
+        (dict(ps=0), b"page_size, num_pages"),
+        (dict(n_seq=0), b"page_size, num_pages"),
+        (dict(mb=1 << 30), b"31 bits"),
+        (dict(zrs=8), b"z_row_stride >= r"),
+        (dict(zgs=24), b"overlap"),
+        (dict(zps=176), b"z_page_stride"),
+        (dict(zps=188), b"z_page_stride"),
+        (dict(bt=None), b"non-NULL"),
+        (dict(pos=None), b"non-NULL"),
+        (dict(pos=ctypes.c_void_p(0x100002)), b"4-byte aligned"),
+        (dict(seq=ctypes.c_void_p(0x100002)), b"4-byte aligned"),
+        (dict(z=ctypes.c_void_p(0x100008)), b"16-byte aligned"),
+        (dict(muw=ctypes.c_void_p(0x100004)), b"muw must be 16-byte"),
+        (dict(xdt=0), b"xdt"),
+    ]:
+        assert call(**over) == _lib.LLA_ERR_INVALID_ARG, over
+        assert why in h.lla_last_error(), (over, h.lla_last_error())
 
 
 def test_paged_decode_rejects_bad_arguments_on_the_host():
@@ -177,8 +261,9 @@ def test_rope_decode_rejects_bad_arguments_on_the_host():
         assert call(fn, ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
     # per-head: latent + rotary rows at most 256 bf16 wide
     assert call("lla_decode_attn_rope", r_k=224) == _lib.LLA_ERR_INVALID_ARG
-    # LLA-2D: rows a multiple of 64 up to 384
-    assert call("lla2d_decode_attn_rope", r_k=200) == _lib.LLA_ERR_UNSUPPORTED
+    # LLA-2D: rows up to 384 wide (200 + 64 is accepted and zero-padded;
+    # it stops at the workspace check)
+    assert call("lla2d_decode_attn_rope", r_k=200) == _lib.LLA_ERR_WORKSPACE
     assert call("lla2d_decode_attn_rope", r_k=384) == _lib.LLA_ERR_UNSUPPORTED
     assert call("lla2d_decode_attn_rope", r_k=320, ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
     assert lla.lla2d_decode_attn_workspace(2, 16, 8, 384, 256) > 0
@@ -205,7 +290,7 @@ def test_paged_lla2d_rejects_bad_arguments_on_the_host():
     assert call(window=-1) == _lib.LLA_ERR_INVALID_ARG
     assert call(ws_bytes=16) == _lib.LLA_ERR_WORKSPACE
     assert lla.lla2d_decode_attn_paged_workspace(2, 16, 256, 256) > 0
-    assert lla.lla2d_decode_attn_paged_workspace(2, 16, 96, 256) == 0
+    assert lla.lla2d_decode_attn_paged_workspace(2, 16, 100, 256) == 0
 
 
 def test_encode_bias_entry_points_reject_bad_arguments_on_the_host():

@@ -14,21 +14,13 @@ import torch
 import decode_attention_encode_b200 as lla
 import oracle
 from decode_attention_encode_b200 import synth
-from lla_cases import TOL_BF16_REL, to_f64
+from lla_cases import check_encoded, to_f64
 
 pytestmark = pytest.mark.gpu
 
 
 def check(z_gpu, z_ref):
-    zg = to_f64(z_gpu)
-    scale = np.abs(z_ref).max()
-    err = np.abs(zg - z_ref).max() / scale
-    assert err <= TOL_BF16_REL, f"relative error {err:.3e}"
-    # element-wise: half a bf16 ulp plus accumulation slack
-    bound = 2.0 ** -8 * np.abs(z_ref) + 1e-4 * scale
-    bad = np.abs(zg - z_ref) > bound
-    assert not bad.any(), f"{bad.sum()} elements outside rounding bound; max rel {err:.2e}"
-    return err
+    return check_encoded(z_gpu, z_ref)
 
 
 def make(T, N, G, d_loop, r, mu, seed=0):

@@ -44,6 +44,21 @@ def test_ranks(r_k, r_v):
     run(2, 16, 128, 333, r_k, r_v, seed=r_k + r_v)
 
 
+@pytest.mark.parametrize("r_k, r_v", [(96, 160), (192, 192), (8, 8), (24, 40), (136, 200),
+                                      (64, 64), (16, 256), (256, 72)])
+def test_ranks_padded_to_whole_boxes_and_tiles(r_k, r_v):
+    # ranks that are not whole 64-column boxes (K) or 128-row MMA tiles (V):
+    # the tensor maps fill the missing columns with zeros and the records
+    # keep only the r_v real rows; 96/160 is the paper's asymmetric split
+    run(3, 16, 128, 333, r_k, r_v, n_cap=340, mu=True, decay=True, seed=r_k * 7 + r_v)
+
+
+def test_full_size_asymmetric_96_160_sampled():
+    # the 32x geometry with the paper's 96/160 key/value split
+    err = run(256, 16, 128, 8192, 96, 160, units=sample_units(256, 16), decay=True, seed=2)
+    print(f"lla2d 96/160 full size: rel err {err:.2e}")
+
+
 @pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 1000])
 def test_context_lengths(N):
     run(2, 16, 128, N, 256, 256, n_cap=N + 3, mu=True, seed=N)

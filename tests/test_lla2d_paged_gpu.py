@@ -74,7 +74,8 @@ def test_ragged_lengths_around_the_tile(page_size):
     compare(out, lse, *reference(inp), lens)
 
 
-@pytest.mark.parametrize("H, r_k, r_v", [(8, 64, 128), (20, 128, 256), (32, 192, 128)])
+@pytest.mark.parametrize("H, r_k, r_v", [(8, 64, 128), (20, 128, 256), (32, 192, 128),
+                                         (16, 96, 160), (4, 200, 8)])
 def test_heads_and_ranks(H, r_k, r_v):
     lens = synth.ragged_lengths(7, 700, seed=H)
     inp = make(lens, H, 64, r_k, r_v, 128, seed=H + r_k)
@@ -175,7 +176,8 @@ def test_sink_window_eviction(sink, window, page_size):
     compare(out, lse, *reference(inp, sink=sink, window=window), lens)
 
 
-@pytest.mark.parametrize("H, r_k, r_v", [(32, 192, 128), (8, 64, 256)])
+@pytest.mark.parametrize("H, r_k, r_v", [(32, 192, 128), (8, 64, 256), (16, 96, 160),
+                                         (12, 40, 24)])
 def test_64_token_pages_heads_and_ranks(H, r_k, r_v):
     # every tile half from its own shuffled page; key rows of one and three boxes
     lens = [64, 65, 128, 1, 191, 640, 333]

@@ -773,3 +773,106 @@ def test_paged2d_eviction_attends_exactly_the_kept_positions():
     o0, _ = oracle.paged2d_decode(q, zkp, zvp, bt, lens, dk, dv)
     o1, _ = oracle.paged2d_decode(q, zkp, zvp, bt, lens, dk, dv, sink=5, window=0)
     np.testing.assert_allclose(o0, o1, atol=0)
+
+
+# --------------------------------------------------------------------------
+# the latent write into a paged store (the write side of the paged layout)
+# --------------------------------------------------------------------------
+
+def _shuffled_table(r, lens, ps, extra_pages=3):
+    need = [(n + ps - 1) // ps for n in lens]
+    P = sum(need) + extra_pages
+    order = r.permutation(P)
+    bt = np.full((len(lens), max(need)), -1)
+    k = 0
+    for b, nb in enumerate(need):
+        bt[b, :nb] = order[k:k + nb]
+        k += nb
+    return bt, P
+
+
+def test_paged_write_then_paged_decode_equals_a_dense_prefill():
+    # Appending each sequence's tokens one decode step at a time (a serving
+    # loop: position = current length) into a shuffled page pool, then
+    # decoding the pool, gives the same result as encoding every token at
+    # once into a dense [B, H, n, r] store and decoding that. This ties the
+    # write side's addresses to the read side's gather (itself pinned
+    # against the dense decode above).
+    r = rng(401)
+    lens = [5, 1, 9, 4]
+    B, T, H, d, rk, ps = len(lens), 2, 3, 4, 5, 3
+    n_max = max(lens)
+    bt, P = _shuffled_table(r, lens, ps)
+    w = r.normal(size=(H, T * d, rk))
+    mu = r.normal(size=(H, T * d))
+    x = r.normal(size=(n_max, T, B, H, d))            # token j of every sequence
+    pool = r.normal(size=(P, H, ps, rk))              # stale contents
+    for j in range(n_max):
+        live = [b for b in range(B) if j < lens[b]]
+        z = oracle.encode(x[j][:, live], w, mu)       # one step's newest tokens
+        pool, skipped = oracle.paged_write(pool, z, bt, positions=[j] * len(live),
+                                           seq_idx=live)
+        assert skipped == []
+    dense = np.zeros((B, H, n_max, rk))
+    for b in range(B):
+        xb = np.transpose(x[:lens[b], :, b], (1, 0, 2, 3))   # [T, n_b, H, d]
+        dense[b, :, :lens[b]] = oracle.encode(xb, w, mu)      # [H, n_b, rk]
+    q = r.normal(size=(B, H, 6))
+    dk, dv = r.normal(size=(H, 6, rk)), r.normal(size=(H, 6, rk))
+    out_p, lse_p = oracle.paged_decode(q, pool, pool, bt, lens, dk, dv, scale=0.4)
+    for b in range(B):
+        o, l = oracle.lla_decode(q[b:b + 1], dense[b:b + 1], dense[b:b + 1], dk, dv, scale=0.4,
+                                 N=lens[b])
+        np.testing.assert_allclose(out_p[b], o[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse_p[b], l[0], rtol=0, atol=1e-12)
+
+
+def test_paged_write_touches_exactly_the_addressed_rows():
+    r = rng(402)
+    G, N, rk, ps, r_row = 2, 6, 4, 4, 7                 # rows wider than the latent
+    bt = np.array([[3, 0, 5], [1, 4, 2]])
+    pool = r.normal(size=(7, G, ps, r_row))
+    z = r.normal(size=(G, N, rk))
+    seq = [0, 1, 1, 0, 1, 0]
+    pos = [0, 5, 11, 9, 12, 6]                          # 12 is past the table: skipped
+    new, skipped = oracle.paged_write(pool, z, bt, pos, seq_idx=seq)
+    assert skipped == [4]
+    expect = pool.copy()
+    for n in (0, 1, 2, 3, 5):
+        page, row = bt[seq[n], pos[n] // ps], pos[n] % ps
+        expect[page, :, row, :rk] = z[:, n]
+    np.testing.assert_array_equal(new, expect)          # the rotary tail is untouched too
+    # bad sequence index and a page outside the pool are skipped as well
+    bt2 = np.array([[3, 9]])
+    new2, sk2 = oracle.paged_write(pool, z[:, :3], bt2, [1, 5, 0], seq_idx=[0, 0, 2])
+    assert sk2 == [1, 2]
+    expect2 = pool.copy()
+    expect2[3, :, 1, :rk] = z[:, 0]
+    np.testing.assert_array_equal(new2, expect2)
+
+
+def test_paged_write_lla2d_rows_and_default_sequence_per_token():
+    r = rng(403)
+    N, rk, ps = 4, 6, 2
+    bt = np.array([[2, 0], [5, 1], [3, 4], [6, 7]])
+    pool = r.normal(size=(8, ps, rk))
+    z = r.normal(size=(1, N, rk))
+    pos = [3, 0, 2, 1]                                  # token n is sequence n's newest
+    new, skipped = oracle.paged_write(pool, z, bt, pos)
+    assert skipped == []
+    expect = pool.copy()
+    for n in range(N):
+        expect[bt[n, pos[n] // ps], pos[n] % ps] = z[0, n]
+    np.testing.assert_array_equal(new, expect)
+    # reading the rows back through the LLA-2D paged decode with one token
+    # gives each token's own reconstruction
+    H, d = 3, 5
+    dv = r.normal(size=(H, d, rk))
+    q = r.normal(size=(N, H, d))
+    bt1 = np.array([[bt[n, pos[n] // ps]] for n in range(N)])
+    rows = [pos[n] % ps for n in range(N)]
+    for n in range(N):
+        one = new[bt1[n, 0], rows[n]][None, None]        # a 1-row page holding that row
+        o, _ = oracle.paged2d_decode(q[n:n + 1], one, one, np.array([[0]]), [1],
+                                     r.normal(size=(H, d, rk)), dv)
+        np.testing.assert_allclose(o[0], (dv @ z[0, n]), atol=1e-12)

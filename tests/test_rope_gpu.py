@@ -129,7 +129,8 @@ def check_2d(inp, units=None):
 
 
 @pytest.mark.parametrize("r_k, d_r, r_v", [(192, 64, 256), (256, 64, 256), (128, 64, 128),
-                                           (320, 64, 128), (64, 64, 256)])
+                                           (320, 64, 128), (64, 64, 256), (96, 32, 160),
+                                           (200, 8, 96)])
 def test_lla2d_rotary_key_row_widths(r_k, d_r, r_v):
     check_2d(make_2d(3, 16, 128, 1000, r_k, d_r, r_v, n_cap=1030, mu=True, seed=r_k))
 
