@@ -29,6 +29,7 @@ LLA_BF16 = 1
 LLA_DEVICE_WAIT_TIMEOUT = 0x1
 LLA_DEVICE_BAD_PAGED_INPUT = 0x2
 LLA_DEVICE_PAGED_PLAN_MISMATCH = 0x4
+LLA_DEVICE_OUT_OF_BOUNDS = 0x8
 
 # Every symbol include/lla.h declares.
 EXPORTS = (
@@ -107,18 +108,26 @@ _SIGS = {
 }
 
 
+def library_variant() -> str:
+    """The build this process loads: "release" (liblla.so), or "check"
+    (liblla_check.so, the bounds-check build) when LLA_LIBRARY_VARIANT=check."""
+    return os.environ.get("LLA_LIBRARY_VARIANT", "release") or "release"
+
+
 def library_path() -> str:
-    return _build.LIB
+    return _build.lib_path(library_variant())
 
 
 def lib(build_if_missing: bool = True):
-    """Loads liblla.so (building it with nvcc if it is missing or stale)."""
+    """Loads the library (building it with nvcc if it is missing or stale)."""
     global _lib
     with _lock:
         if _lib is None:
-            path = _build.build() if build_if_missing else _build.LIB
+            variant = library_variant()
+            path = (_build.build(variant=variant) if build_if_missing
+                    else _build.lib_path(variant))
             if not os.path.exists(path):
-                raise LLAError(LLA_ERR_CUDA, f"liblla.so not found at {path}")
+                raise LLAError(LLA_ERR_CUDA, f"library not found at {path}")
             h = ctypes.CDLL(path)
             for name, (args, res) in _SIGS.items():
                 fn = getattr(h, name)

@@ -15,6 +15,7 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 constexpr unsigned int kStatusWaitTimeout = 0x1u;
 constexpr unsigned int kStatusBadPagedInput = 0x2u;
 constexpr unsigned int kStatusPlanMismatch = 0x4u;
+constexpr unsigned int kStatusOutOfBounds = 0x8u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -70,6 +71,49 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
 
 __device__ __forceinline__ void report_status(unsigned int* status, unsigned int bits) {
   if (status) atomicOr(status, bits);
+}
+
+// The extent of a device buffer, [p, p + n) in bytes. The default span has
+// no extent and admits every address.
+struct Span {
+  const char* p = nullptr;
+  unsigned long long n = ~0ull;
+};
+inline Span span_of(const void* p, unsigned long long bytes) {
+  return Span{static_cast<const char*>(p), bytes};
+}
+
+// Bounds-check build (compiled with LLA_BOUNDS_CHECK): the kernels test each
+// computed global access against the span of the buffer it belongs to. An
+// access outside its span sets the status bit kStatusOutOfBounds and is not
+// made (a store is skipped, a load or copy takes zeros or nothing). The
+// release build compiles every check to `true`.
+#ifdef LLA_BOUNDS_CHECK
+__device__ __forceinline__ bool in_span(const Span& s, const void* q, unsigned long long bytes,
+                                        unsigned int* status) {
+  const char* c = static_cast<const char*>(q);
+  const bool ok = s.p == nullptr || (c >= s.p && bytes <= s.n && c - s.p <= (long long)(s.n - bytes));
+  if (!ok) report_status(status, kStatusOutOfBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_span(const Span&, const void*, unsigned long long,
+                                                  unsigned int*) {
+  return true;
+}
+#endif
+
+// A store of v at p that the bounds-check build makes only inside span s.
+template <class T>
+__device__ __forceinline__ void st_chk(T* p, T v, const Span& s, unsigned int* status) {
+  if (in_span(s, p, sizeof(T), status)) *p = v;
+}
+
+// A read-only load from p, or `dflt` when the bounds-check build finds p
+// outside span s.
+template <class T>
+__device__ __forceinline__ T ld_chk(const T* p, const Span& s, unsigned int* status, T dflt) {
+  return in_span(s, p, sizeof(T), status) ? __ldg(p) : dflt;
 }
 
 // L2 policy for data read exactly once (the latent stream).

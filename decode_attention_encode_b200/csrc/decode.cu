@@ -101,6 +101,8 @@ struct AbsorbArgs {
   int hp;              // its rows (heads padded to the MMA N)
   const float* q_rope;  // [B*H][d_r] rotated rotary query, or null (d_r = 0)
   int d_r;
+  Span ws_span;         // the workspace holding qp, c0 and qsw (bounds-check build)
+  unsigned int* status;
 };
 
 // One CTA per (head, 32*COLS latent columns, 8*ROWS batch rows). The CTA
@@ -141,8 +143,8 @@ __device__ __forceinline__ void zero_qsw_tail(const AbsorbArgs& a, int rq, int h
     const int bb = idx / (npad * nh), rest = idx - bb * npad * nh;
     const int k = rest / npad, c = rq + rest - k * npad;
     const int hh = k == 0 ? h : a.H + k - 1;
-    *reinterpret_cast<__nv_bfloat16*>(a.qsw + qsw_block(a, rq, b0 + bb) + sw128_off(hh, c, a.hp)) =
-        __float2bfloat16_rn(0.f);
+    st_chk(reinterpret_cast<__nv_bfloat16*>(a.qsw + qsw_block(a, rq, b0 + bb) + sw128_off(hh, c, a.hp)),
+           __float2bfloat16_rn(0.f), a.ws_span, a.status);
   }
 }
 
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
         for (int i = lane; i < a.d_h; i += 32)
           acc += q_s[bb * d_h4 + i] * a.mu_k[(size_t)h * a.d_h + i];
       acc = warp_sum(acc);
-      if (lane == 0) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
+      if (lane == 0) st_chk(&a.c0[(size_t)(b0 + bb) * a.H + h], a.scale * acc, a.ws_span, a.status);
     }
   }
   float acc[ROWS][COLS];
@@ -237,15 +239,16 @@ __global__ void __launch_bounds__(256) k_absorb(AbsorbArgs a) {
       // rotated keys as it is
       const float v = (c < a.r_k ? acc[k][j] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
                       a.qscale;
-      if (a.qp) a.qp[unit * rq + c] = v;
+      if (a.qp) st_chk(&a.qp[unit * rq + c], v, a.ws_span, a.status);
       if (a.qsw) {
         unsigned char* base = a.qsw + qsw_block(a, rq, b0 + bb);
-        *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)) = __float2bfloat16_rn(v);
+        st_chk(reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)), __float2bfloat16_rn(v),
+               a.ws_span, a.status);
         // the last head's CTAs also clear the padding rows h >= H
         if (h == a.H - 1)
           for (int hz = a.H; hz < a.hp; ++hz)
-            *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)) =
-                __float2bfloat16_rn(0.f);
+            st_chk(reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)),
+                   __float2bfloat16_rn(0.f), a.ws_span, a.status);
       }
     }
   }
@@ -268,6 +271,7 @@ struct CombineArgs {
   float* lse;
   RaggedMap ragged;  // seqinfo non-null: the paged plan's piece map
   unsigned int* status;
+  Span ws_span, out_span, lse_span;  // extents (bounds-check build)
 };
 
 // The merge pass shared by k_combine and k_combine_tc.
@@ -296,7 +300,8 @@ __device__ __forceinline__ void merge_rows(const CombineArgs& a, int h, int b0, 
   float M = kNegBig, L = 0.f, keep = 0.f;
   if (bb < nb) {
     const long long u = (long long)(b0 + bb) * a.H + h;
-    const float c0u = (blockIdx.y == 0 && a.lse) ? a.c0[u] : 0.f;  // in flight with the records
+    const float c0u =  // in flight with the records
+        (blockIdx.y == 0 && a.lse) ? ld_chk(&a.c0[u], a.ws_span, a.status, 0.f) : 0.f;
     const long long key = a.shared ? (long long)(b0 + bb) : u;
     long long wf = 0, wl = -1;
     if (a.ragged.seqinfo) {
@@ -319,7 +324,8 @@ __device__ __forceinline__ void merge_rows(const CombineArgs& a, int h, int b0, 
       float2 v[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        v[k] = p0 + k < np ? __ldg(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride))
+        v[k] = p0 + k < np ? ld_chk(reinterpret_cast<const float2*>(rec0 + (p0 + k) * rstride),
+                                    a.ws_span, a.status, make_float2(kNegBig, 0.f))
                            : make_float2(kNegBig, 0.f);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -330,7 +336,7 @@ __device__ __forceinline__ void merge_rows(const CombineArgs& a, int h, int b0, 
     }
     keep = np > 0 ? 1.f : 0.f;
     if (blockIdx.y == 0 && a.lse)  // no attended token: lse = -inf
-      a.lse[u] = np > 0 ? (M + log2f(L)) * kLn2 + c0u : -INFINITY;
+      st_chk(&a.lse[u], np > 0 ? (M + log2f(L)) * kLn2 + c0u : -INFINITY, a.lse_span, a.status);
   }
   s_np[bb] = np;
   s_off[bb] = off;
@@ -380,8 +386,9 @@ __device__ __forceinline__ void merge_sweep(const CombineArgs& a, int nrows, int
 #pragma unroll
       for (int k = 0; k < kI; ++k) {
         if (p < npk[k]) {
-          mv[k] = __ldg(rb[k] + p * rstride);
-          uv[k] = __ldg(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k]);
+          mv[k] = ld_chk(rb[k] + p * rstride, a.ws_span, a.status, kNegBig);
+          uv[k] = ld_chk(reinterpret_cast<const float4*>(rb[k] + p * rstride + 4) + c4k[k],
+                         a.ws_span, a.status, make_float4(0.f, 0.f, 0.f, 0.f));
         }
       }
 #pragma unroll
@@ -485,7 +492,8 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
     for (int k = 0; k < ROWS; ++k) {
       const int bb = warp * ROWS + k;
       if (bb < nb)
-        a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + il] = acc[k][j] + mu * s_keep[bb];
+        st_chk(&a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + il],
+               acc[k][j] + mu * s_keep[bb], a.out_span, a.status);
     }
   }
 }
@@ -671,7 +679,8 @@ __global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
     for (int k = 0; k < kTcRows / 8; ++k) {
       const int bb = warp + 8 * k;
       const float acc = warp_sum(part[k]);
-      if (lane == 0 && bb < nb) a.c0[(size_t)(b0 + bb) * a.H + h] = a.scale * acc;
+      if (lane == 0 && bb < nb)
+        st_chk(&a.c0[(size_t)(b0 + bb) * a.H + h], a.scale * acc, a.ws_span, a.status);
     }
   }
   const int m0 = (warp & 3) * 16, n0 = (warp >> 2) * 32;
@@ -708,14 +717,15 @@ __global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
       // rotated keys as it is
       const float v = (c < a.r_k ? acc[nt][e] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
                       a.qscale;
-      if (a.qp) a.qp[unit * rq + c] = v;
+      if (a.qp) st_chk(&a.qp[unit * rq + c], v, a.ws_span, a.status);
       if (a.qsw) {
         unsigned char* base = a.qsw + qsw_block(a, rq, b0 + bb);
-        *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)) = __float2bfloat16_rn(v);
+        st_chk(reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)), __float2bfloat16_rn(v),
+               a.ws_span, a.status);
         if (h == a.H - 1)
           for (int hz = a.H; hz < a.hp; ++hz)
-            *reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)) =
-                __float2bfloat16_rn(0.f);
+            st_chk(reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)),
+                   __float2bfloat16_rn(0.f), a.ws_span, a.status);
       }
     }
   if (a.qsw && c0 + nc == rq) zero_qsw_tail(a, rq, h, b0, nb);
@@ -797,7 +807,8 @@ __global__ void __launch_bounds__(256, 2) k_combine_tc(CombineArgs a) {
       const int il = m0 + g + (e >> 1) * 8;
       const int bb = n0 + 8 * nt + 2 * t + (e & 1);
       if (il >= ni || bb >= nb) continue;
-      a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + il] = acc[nt][e] + s_mu[il] * s_keep[bb];
+      st_chk(&a.out[((size_t)(b0 + bb) * a.H + h) * a.d_h + i0 + il],
+             acc[nt][e] + s_mu[il] * s_keep[bb], a.out_span, a.status);
     }
 }
 
@@ -817,9 +828,10 @@ int env_int(const char* name, int dflt) {
 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
-                         unsigned char* qsw, int hp, const float* q_rope, int d_r, bool tc) {
+                         unsigned char* qsw, int hp, const float* q_rope, int d_r, bool tc,
+                         Span ws) {
   AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp,
-               q_rope, q_rope ? d_r : 0};
+               q_rope, q_rope ? d_r : 0, ws, status_word()};
   const int rq = r_k + a.d_r;
   if (tc && d_h % 16 == 0 && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
     const size_t smem = absorb_tc_smem(d_h);
@@ -850,12 +862,14 @@ lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
                           long long P, int shared, float* out, float* lse, cudaStream_t stream,
-                          const RaggedMap* ragged, bool tc) {
+                          const RaggedMap* ragged, bool tc, Span ws) {
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   CombineArgs a{part, pstride, c0, dv, mu_v, B, H, d_h, r_v, N, P, shared, out, lse,
-                RaggedMap{nullptr, nullptr, nullptr, 0ull}, status_word()};
+                RaggedMap{nullptr, nullptr, nullptr, 0ull}, status_word(), ws,
+                span_of(out, (unsigned long long)B * H * d_h * sizeof(float)),
+                lse ? span_of(lse, (unsigned long long)B * H * sizeof(float)) : Span{}};
   if (ragged) a.ragged = *ragged;
   if (tc) {
     cudaLaunchConfig_t cfg{};
@@ -1013,7 +1027,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
 
   // 1. absorb
   st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, q_rope, d_r,
-                     small_gemm_tc(esz, B, r_k, r_v));
+                     small_gemm_tc(esz, B, r_k, r_v), span_of(ws, ws_bytes));
   if (st != LLA_OK) return st;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1040,6 +1054,9 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
     a.part = part;
     a.pstride = d.pstride;
     a.status = status_word();
+    a.zk_span = span_of(zk, (unsigned long long)B * H * n_cap * a.row_k);
+    a.zv_span = span_of(zv, (unsigned long long)B * H * n_cap * a.row_v);
+    a.ws_span = span_of(ws, ws_bytes);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(d.grid);
     cfg.blockDim = dim3(32 * d.warps);
@@ -1056,7 +1073,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
   }
   // 3. combine
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, N, d.P, 0, out, lse, stream,
-                        nullptr, small_gemm_tc(esz, B, r_k, r_v));
+                        nullptr, small_gemm_tc(esz, B, r_k, r_v), span_of(ws, ws_bytes));
   return LLA_OK;
 }
 

@@ -52,6 +52,7 @@ struct OutMap {
   long long zrs, zgs;
   int paged;
   PagedOut pd;
+  Span z_span;  // every row the map can address (bounds-check build)
 };
 
 // Element offset of token n's row (group 0), or -1 when a paged destination
@@ -80,6 +81,7 @@ struct EncodeArgs {
   // group's tiles in a row, so the in-kernel mean term changes rarely)
   int token_major;
   float* part;      // ksplit > 1: fp32 partials [ksplit][G][N][r]
+  Span ws_span;     // the workspace holding them (bounds-check build)
   int nstage, b_bytes, stage_bytes;
   uint32_t tmem_cols;
   const float* mu;
@@ -302,8 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int c0 = cc + 8 * h8;
               if (c0 < a.r) {
                 float4* dst = reinterpret_cast<float4*>(prow + c0);
-                dst[0] = make_float4(v[8 * h8 + 0], v[8 * h8 + 1], v[8 * h8 + 2], v[8 * h8 + 3]);
-                dst[1] = make_float4(v[8 * h8 + 4], v[8 * h8 + 5], v[8 * h8 + 6], v[8 * h8 + 7]);
+                if (in_span(a.ws_span, dst, 32, a.status)) {
+                  dst[0] = make_float4(v[8 * h8 + 0], v[8 * h8 + 1], v[8 * h8 + 2], v[8 * h8 + 3]);
+                  dst[1] = make_float4(v[8 * h8 + 4], v[8 * h8 + 5], v[8 * h8 + 6], v[8 * h8 + 7]);
+                }
               }
             }
           } else if (write) {
@@ -319,7 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       v[8 * h8 + 2 * e + 1] - tail->muw[c0 + 2 * e + 1]);
                   w[e] = *reinterpret_cast<const uint32_t*>(&p);
                 }
-                *reinterpret_cast<uint4*>(zrow + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+                st_chk(reinterpret_cast<uint4*>(zrow + c0), make_uint4(w[0], w[1], w[2], w[3]),
+                       a.out.z_span, a.status);
               }
             }
           }
@@ -403,7 +408,8 @@ __global__ void __launch_bounds__(256) k_encode_bias(const __nv_bfloat16* wt, co
 // partial loads in flight.
 __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const float* muw,
                                                        int ksplit, int G, int N, int r,
-                                                       OutMap out, unsigned int* status) {
+                                                       OutMap out, unsigned int* status,
+                                                       Span ws_span) {
   const int r4 = r / 4;
   const long long total = (long long)G * N * r4;
   const size_t plane4 = (size_t)G * N * r / 4;  // float4 per split
@@ -422,7 +428,9 @@ __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const 
       float4 v[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        v[k] = k0 + k < ksplit ? __ldg(p + (size_t)(k0 + k) * plane4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k] = k0 + k < ksplit ? ld_chk(p + (size_t)(k0 + k) * plane4, ws_span, status,
+                                        make_float4(0.f, 0.f, 0.f, 0.f))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         s.x += v[k].x;
@@ -439,8 +447,9 @@ __global__ void __launch_bounds__(256) k_encode_reduce(const float* part, const 
       s.w -= m.w;
     }
     const __nv_bfloat162 b0 = __floats2bfloat162_rn(s.x, s.y), b1 = __floats2bfloat162_rn(s.z, s.w);
-    *reinterpret_cast<uint2*>(out.z + (size_t)g * out.zgs + roff + c) =
-        make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+    st_chk(reinterpret_cast<uint2*>(out.z + (size_t)g * out.zgs + roff + c),
+           make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1)),
+           out.z_span, status);
   }
 }
 
@@ -553,6 +562,13 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   a.out.zgs = zgs;
   a.out.paged = paged != nullptr;
   if (paged) a.out.pd = *paged;
+  // the last element any row can reach, in elements from z
+  const unsigned long long zlast =
+      paged ? (unsigned long long)(paged->num_pages - 1) * paged->page_stride +
+                  (unsigned long long)(G - 1) * zgs + (unsigned long long)(paged->page_size - 1) * zrs + r
+            : (unsigned long long)(G - 1) * zgs + (unsigned long long)(N - 1) * zrs + r;
+  a.out.z_span = span_of(z, zlast * 2);
+  a.ws_span = span_of(ws, ws_bytes);
   a.status = status_word();
 
   const DeviceInfo di = device_info();
@@ -608,7 +624,8 @@ lla_status run_encode(const void* x, int T, int N, int G, int d_loop, int r, con
   if (a.part) {
     const long long outs = (long long)G * N * (r / 4);
     const int rgrid = (int)std::min<long long>((outs + 255) / 256, 4LL * di.sms);
-    k_encode_reduce<<<rgrid, 256, 0, stream>>>(a.part, muw, a.ksplit, G, N, r, a.out, a.status);
+    k_encode_reduce<<<rgrid, 256, 0, stream>>>(a.part, muw, a.ksplit, G, N, r, a.out, a.status,
+                                               a.ws_span);
     e = cudaGetLastError();
     if (e != cudaSuccess) return check_cuda(e, "launch k_encode_reduce");
   }

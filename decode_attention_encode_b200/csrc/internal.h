@@ -5,6 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "lla.h"
 
 namespace lla {
@@ -148,13 +149,13 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
                          unsigned char* qsw = nullptr, int hp = 0, const float* q_rope = nullptr,
-                         int d_r = 0, bool tc = false);
+                         int d_r = 0, bool tc = false, Span ws = Span{});
 // whether per-head decode runs launch_absorb / launch_combine with tc
 bool small_gemm_tc(int esz, int B, int r_k, int r_v);
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
                           long long P, int shared, float* out, float* lse, cudaStream_t stream,
-                          const RaggedMap* ragged = nullptr, bool tc = false);
+                          const RaggedMap* ragged = nullptr, bool tc = false, Span ws = Span{});
 
 size_t workspace_2d(int B, int H, int N, int r_k, int r_v);
 lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, int H, int d_h,

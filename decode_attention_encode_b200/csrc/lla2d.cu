@@ -78,6 +78,7 @@ struct D2Args {
   float* part;
   int pstride;
   unsigned int* status;
+  Span ws_span;             // the workspace (bounds-check build)
 };
 
 struct Tail2 {
@@ -134,7 +135,7 @@ struct TileCur {
 
 __device__ __forceinline__ void tcur_load(TileCur& c, const D2Args& a) {
   if (a.seqinfo) {
-    const int4 v = __ldg(a.seqinfo + c.b);
+    const int4 v = ld_chk(a.seqinfo + c.b, a.ws_span, a.status, make_int4(0, 0, 0, 0));
     c.nt = v.x;
     c.n = v.y;
     c.st = v.z;
@@ -166,7 +167,7 @@ __device__ __forceinline__ TileCur tcur_start(const D2Args& a) {
   if (a.seqinfo) {
     // a CTA with no tiles (or a workspace that holds no plan for this call)
     // still builds a cursor: its sequence index is kept inside [0, B)
-    const int4 s = __ldg(a.cstart + blockIdx.x);
+    const int4 s = ld_chk(a.cstart + blockIdx.x, a.ws_span, a.status, make_int4(0, 0, 0, 0));
     c.b = min(max(s.x, 0), a.B - 1);
     c.j = s.z;
   } else {
@@ -363,9 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) return false;
       if (lane == 0) {
         const uint32_t qfull = smem_u32(&tl->q_full[qb]);
-        mbar_arrive_expect_tx(qfull, (uint32_t)a.qbuf_bytes);
-        bulk_g2s(s_q0 + (uint32_t)(qb * a.qbuf_bytes), a.qsw + (size_t)b * a.qbuf_bytes,
-                 (uint32_t)a.qbuf_bytes, qfull, l2_evict_first_policy());
+        const unsigned char* qsrc = a.qsw + (size_t)b * a.qbuf_bytes;
+        if (in_span(a.ws_span, qsrc, (unsigned long long)a.qbuf_bytes, a.status)) {
+          mbar_arrive_expect_tx(qfull, (uint32_t)a.qbuf_bytes);
+          bulk_g2s(s_q0 + (uint32_t)(qb * a.qbuf_bytes), qsrc, (uint32_t)a.qbuf_bytes, qfull,
+                   l2_evict_first_policy());
+        } else {
+          mbar_arrive(qfull);  // nothing copied
+        }
       }
       q_issued = seg;
       return true;
@@ -658,7 +664,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (vg * 128 + row < a.r_v) {
 #pragma unroll
               for (int e = 0; e < 16; ++e)
-                if (h0 + e < a.H) rec[(size_t)(h0 + e) * a.pstride + 4 + vg * 128 + row] = u[e];
+                if (h0 + e < a.H)
+                  st_chk(&rec[(size_t)(h0 + e) * a.pstride + 4 + vg * 128 + row], u[e], a.ws_span,
+                         a.status);
             }
           }
         }
@@ -673,9 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < HP; ++h)
             if (h == lane) mm = m[h];
-          rec[(size_t)lane * a.pstride + 0] = mm;
-          rec[(size_t)lane * a.pstride + 1] =
-              tl->lsum[0][lane] + tl->lsum[1][lane] + tl->lsum[2][lane] + tl->lsum[3][lane];
+          st_chk(&rec[(size_t)lane * a.pstride + 0], mm, a.ws_span, a.status);
+          st_chk(&rec[(size_t)lane * a.pstride + 1],
+                 tl->lsum[0][lane] + tl->lsum[1][lane] + tl->lsum[2][lane] + tl->lsum[3][lane],
+                 a.ws_span, a.status);
         }
         tc_fence_before();
         if (!epi_sync()) break;  // lsum is reused by the next sequence
@@ -773,13 +782,13 @@ struct Paged2D {
 lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& tv, int B, int H,
                      int d_h, int N, int r_k, int r_v, const float* dk, const float* dv,
                      const float* mu_k, const float* mu_v, float scale, float* out, float* lse,
-                     const D2Plan& d, char* wsb, const Paged2D* pg, cudaStream_t stream,
+                     const D2Plan& d, char* wsb, Span ws, const Paged2D* pg, cudaStream_t stream,
                      const float* q_rope = nullptr, int d_r = 0) {
   unsigned char* qsw = reinterpret_cast<unsigned char*>(wsb + d.off_qsw);
   float* c0 = reinterpret_cast<float*>(wsb + d.off_c0);
   float* part = reinterpret_cast<float*>(wsb + d.off_part);
   lla_status st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k - d_r, scale, nullptr, c0, stream, qsw,
-                                d.hp, q_rope, d_r, true);
+                                d.hp, q_rope, d_r, true, ws);
   if (st != LLA_OK) return st;
 
   D2Args a{};
@@ -805,6 +814,7 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
   a.part = part;
   a.pstride = d.pstride;
   a.status = status_word();
+  a.ws_span = ws;
   if (pg) {
     a.seqinfo = pg->seqinfo;
     a.plan = pg->plan;
@@ -843,11 +853,11 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
   if (pg) {  // sequence b's pieces: the CTAs of its tiles, cum[b] .. cum[b] + tiles - 1
     RaggedMap rm{pg->seqinfo, pg->cum, pg->plan, pg->stamp};
     return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 1, out, lse, stream,
-                          &rm, true);
+                          &rm, true, ws);
   }
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v,
                         (long long)d.tps * kRows, (long long)d.tpc * kRows, 1, out, lse, stream,
-                        nullptr, true);
+                        nullptr, true, ws);
 }
 
 // The paged plan: the dense plan's kernel shape with a one-wave grid (the
@@ -902,7 +912,7 @@ lla_status run_decode_2d(const float* q, const void* zk, const void* zv, int B, 
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
   return launch_2d(q, tk, tv, B, H, d_h, N, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, d,
-                   static_cast<char*>(ws), nullptr, stream, q_rope, d_r);
+                   static_cast<char*>(ws), span_of(ws, ws_bytes), nullptr, stream, q_rope, d_r);
 }
 
 size_t workspace_2d_paged(int B, int H, int r_k, int r_v) {
@@ -962,7 +972,7 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
     if (!make_tmap_bf16(&tv, zv, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
   return launch_2d(q, tk, tv, B, H, d_h, 0, r_k, r_v, dk, dv, mu_k, mu_v, scale, out, lse, pp.d,
-                   wsb, &pg, stream);
+                   wsb, span_of(ws, ws_bytes), &pg, stream);
 }
 
 }  // namespace lla

@@ -42,6 +42,7 @@ struct PlanArgs {
   int4* wstart;
   unsigned long long stamp;
   unsigned int* status;
+  Span bt_span;  // the block table (bounds-check build)
 };
 
 // Every page index the kept positions [lo, hi) of sequence b touch lies in
@@ -52,7 +53,7 @@ __device__ bool pages_ok(const PlanArgs& p, int b, int lo, int hi, int lane) {
   const int* row = p.block_table + (size_t)b * p.max_blocks;
   bool bad = false;
   for (int blk = lo / p.page_size + lane; blk <= (hi - 1) / p.page_size; blk += 32) {
-    const int pg = __ldg(row + blk);
+    const int pg = ld_chk(row + blk, p.bt_span, p.status, -1);
     bad |= pg < 0 || pg >= p.num_pages;
   }
   return !__any_sync(0xffffffffu, bad);
@@ -236,6 +237,7 @@ lla_status launch_plan_paged(const int* seq_lens, const int* block_table, int B,
   p.wstart = wstart;
   p.stamp = stamp;
   p.status = status_word();
+  p.bt_span = span_of(block_table, (unsigned long long)B * max_blocks * sizeof(int));
   k_plan_paged<<<1, kPlanThreads, 0, stream>>>(p);
   return check_cuda(cudaGetLastError(), "launch k_plan_paged");
 }
@@ -287,7 +289,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
   }
   // 2. absorb (plain launch)
   st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, nullptr, 0,
-                     small_gemm_tc(esz, B, r_k, r_v));
+                     small_gemm_tc(esz, B, r_k, r_v), span_of(ws, ws_bytes));
   if (st != LLA_OK) return st;
   // 3. stream
   {
@@ -307,6 +309,9 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
     a.part = part;
     a.pstride = d.pstride;
     a.status = status_word();
+    a.zk_span = span_of(zk, (unsigned long long)num_pages * H * page_size * a.row_k);
+    a.zv_span = span_of(zv, (unsigned long long)num_pages * H * page_size * a.row_v);
+    a.ws_span = span_of(ws, ws_bytes);
     a.seqinfo = seqinfo;
     a.cum = cum;
     a.plan = plan;
@@ -338,7 +343,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
   // 4. combine over the ragged piece map
   RaggedMap rm{seqinfo, cum, plan, stamp};
   return launch_combine(part, d.pstride, c0, dv, mu_v, B, H, d_h, r_v, 0, 0, 0, out, lse, stream,
-                        &rm, small_gemm_tc(esz, B, r_k, r_v));
+                        &rm, small_gemm_tc(esz, B, r_k, r_v), span_of(ws, ws_bytes));
 }
 
 }  // namespace lla

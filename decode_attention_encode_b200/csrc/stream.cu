@@ -36,11 +36,11 @@ __device__ __forceinline__ void unpack16<4>(const uint4& v, float* f) {
 // Loads q' of unit u (this lane's segments) into registers.
 template <int E, int LPT, int SK, bool EXACT>
 __device__ __forceinline__ void load_qp(float (&qv)[SK][E], const float* qp, long long u, int r_k,
-                                        int nseg_k, int g) {
+                                        int nseg_k, int g, const StreamArgs& a) {
 #pragma unroll
   for (int s = 0; s < SK; ++s) {
     const int seg = s * LPT + g;
-    if (EXACT || seg < nseg_k) {
+    if ((EXACT || seg < nseg_k) && in_span(a.ws_span, qp + u * r_k + seg * E, E * 4, a.status)) {
       const float4* src = reinterpret_cast<const float4*>(qp + u * r_k + seg * E);
 #pragma unroll
       for (int e4 = 0; e4 < E / 4; ++e4) {
@@ -158,7 +158,8 @@ __device__ __forceinline__ void stream_merge_write(float m, float l, float (&acc
       }
     m = M;
   }
-  if (slot == 0) {
+  // the whole record [m, l, pad, pad, u[nseg_v * E]] must lie in the workspace
+  if (slot == 0 && in_span(a.ws_span, pp, (4 + (size_t)a.nseg_v * E) * 4, a.status)) {
     if (g == 0) {
       pp[0] = m;
       pp[1] = l;
@@ -220,9 +221,15 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
       const uint32_t bar = bar0 + 8 * ps;
       const long long row = pu * a.n_cap + pj;
       const uint32_t dst = buf0 + ps * a.stage_bytes;
-      mbar_arrive_expect_tx(bar, kb + vb);
-      bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
-      bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
+      const char* ksrc = a.zk + row * a.row_k;
+      const char* vsrc = a.zv + row * a.row_v;
+      if (in_span(a.zk_span, ksrc, kb, a.status) && in_span(a.zv_span, vsrc, vb, a.status)) {
+        mbar_arrive_expect_tx(bar, kb + vb);
+        bulk_g2s(dst, ksrc, kb, bar, pol);
+        bulk_g2s(dst + v_off, vsrc, vb, bar, pol);
+      } else {
+        mbar_arrive(bar);  // nothing copied: the stage completes as it is
+      }
     }
     pf += len;
     pj += len;
@@ -244,11 +251,11 @@ __global__ void __launch_bounds__(256, 1) k_stream(StreamArgs a) {
   long long u = f0 / a.N;
   const long long u_last = (f1 - 1) / a.N;
   float qv[SK][E], qn[SK][E];
-  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g);
+  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g, a);
   while (f < f1) {
     const long long seg_end = min(f1, (u + 1) * a.N);
     // the next unit's q' loads run under this unit's stream
-    if (u < u_last) load_qp<E, LPT, SK, EXACT>(qn, a.qp, u + 1, a.r_k, a.nseg_k, g);
+    if (u < u_last) load_qp<E, LPT, SK, EXACT>(qn, a.qp, u + 1, a.r_k, a.nseg_k, g, a);
     float m = kNegBig, l = 0.f;
     float acc[SV][E];
 #pragma unroll
@@ -312,7 +319,9 @@ struct PCursor {
 };
 
 __device__ __forceinline__ void pc_load_seq(PCursor& c, const StreamArgs& a) {
-  const int4 v = __ldg(a.seqinfo + c.b);
+  const int4 v = in_span(a.ws_span, a.seqinfo + c.b, sizeof(int4), a.status)
+                     ? __ldg(a.seqinfo + c.b)
+                     : make_int4(0, 0, 0, 0);
   c.n = v.x;
   c.s = v.y;
   c.gap = v.z;
@@ -417,7 +426,9 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   __syncwarp();
   const uint64_t pol = l2_evict_first_policy();
 
-  const int4 st0 = a.wstart[w];
+  const int4 st0 = in_span(a.ws_span, a.wstart + w, sizeof(int4), a.status)
+                       ? a.wstart[w]
+                       : make_int4(0, 0, 0, 0);
   PCursor pc{st0.x, st0.y, st0.z, 0, 0, 0, 0, 0};
   pc_load_seq(pc, a);
   pc_place(pc, a.page_size);
@@ -458,9 +469,15 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
       const uint32_t bar = bar0 + 8 * ps;
       const uint32_t dst = buf0 + ps * a.stage_bytes;
       slen[ps] = len;  // ordered before the consumer's wait by the arrive
-      mbar_arrive_expect_tx(bar, kb + vb);
-      bulk_g2s(dst, a.zk + row * a.row_k, kb, bar, pol);
-      bulk_g2s(dst + v_off, a.zv + row * a.row_v, vb, bar, pol);
+      const char* ksrc = a.zk + row * a.row_k;
+      const char* vsrc = a.zv + row * a.row_v;
+      if (in_span(a.zk_span, ksrc, kb, a.status) && in_span(a.zv_span, vsrc, vb, a.status)) {
+        mbar_arrive_expect_tx(bar, kb + vb);
+        bulk_g2s(dst, ksrc, kb, bar, pol);
+        bulk_g2s(dst + v_off, vsrc, vb, bar, pol);
+      } else {
+        mbar_arrive(bar);  // nothing copied: the stage completes as it is
+      }
     }
     pf += len;
     pc_advance(pc, len, a);
@@ -477,7 +494,7 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
   long long f = f0;
   long long u = (long long)cc.b * a.H + cc.h;
   float qv[SK][E], qn[SK][E];
-  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g);
+  load_qp<E, LPT, SK, EXACT>(qv, a.qp, u, a.r_k, a.nseg_k, g, a);
   while (f < f1) {
     const long long seg_end = min(f1, f + (cc.n - cc.i));
     long long un = -1;
@@ -485,7 +502,7 @@ __global__ void __launch_bounds__(256, 1) k_stream_paged(StreamArgs a) {
     if (seg_end < f1) {  // the next unit's q' loads run under this unit's stream
       pc_next_unit(nx, a);
       un = (long long)nx.b * a.H + nx.h;
-      load_qp<E, LPT, SK, EXACT>(qn, a.qp, un, a.r_k, a.nseg_k, g);
+      load_qp<E, LPT, SK, EXACT>(qn, a.qp, un, a.r_k, a.nseg_k, g, a);
     }
     float m = kNegBig, l = 0.f;
     float acc[SV][E];

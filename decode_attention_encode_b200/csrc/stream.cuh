@@ -42,6 +42,8 @@ struct StreamArgs {
   const int* block_table;  // [B][max_blocks]
   int max_blocks, page_size, H, B;
   int num_pages;           // page indices are checked against it as they are read
+  // extents for the bounds-check build: the latent stores and the workspace
+  Span zk_span, zv_span, ws_span;
 };
 
 // Per-sequence record of the paged plan: sequence b attends n tokens; kept

@@ -66,6 +66,11 @@ typedef enum { LLA_F32 = 0, LLA_BF16 = 1 } lla_dtype;
                                             plan for itself in its workspace
                                             (nothing was decoded: out = 0,
                                             lse = -inf) */
+#define LLA_DEVICE_OUT_OF_BOUNDS 0x8u    /* bounds-check build only (compiled
+                                            with LLA_BOUNDS_CHECK): a kernel
+                                            computed a global address outside
+                                            the buffer it belongs to, and did
+                                            not make that access */
 
 /* Human-readable name of a status code. Never NULL. */
 LLA_API const char *lla_status_string(lla_status s);
