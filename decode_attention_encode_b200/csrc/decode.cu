@@ -885,7 +885,10 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
     return check_cuda(cudaLaunchKernelEx(&cfg, k_combine_tc, a), "launch k_combine_tc");
   }
   int rows, cols;
-  pick_block(H, d_h, B, &rows, &cols, true, env_int("LLA_COMBINE_MAX_COLS", 1));
+  // Up to four 32-channel column blocks per CTA: at large batches fewer CTAs
+  // merge each row's records once for more channels (768 -> 384 CTAs at
+  // B = 768); below that the CTA-count floor keeps one or two.
+  pick_block(H, d_h, B, &rows, &cols, true, env_int("LLA_COMBINE_MAX_COLS", 4));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(H, (d_h + 32 * cols - 1) / (32 * cols), (B + 8 * rows - 1) / (8 * rows));
   cfg.blockDim = dim3(256);
