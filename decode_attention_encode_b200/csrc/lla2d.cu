@@ -50,6 +50,7 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kBoxBytes = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 constexpr int kStageBytes = 2 * kBoxBytes;
+constexpr int kSubBytesV = kBoxBytes / 2;  // one 64-row half of a 64-column block
 constexpr int kThreads = 256;
 constexpr int kMaxStages = 4;  // per ring
 constexpr float kNegBig = -1.0e30f;
@@ -189,7 +190,7 @@ __device__ __forceinline__ void tcur_next(TileCur& c, const D2Args& a) {
   }
 }
 
-template <int HP, int NSUB>
+template <int HP, int NSUB, bool VPAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_lla2d(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
             D2Args a) {
@@ -321,6 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_of(lt);
       const uint32_t dst = ring + (uint32_t)s * kStageBytes;
       const int nb = is_k ? kboxes(grp) : 2;
+      // VPAIR (V ring, 64-token halves): one load brings both 64-column
+      // blocks of a half, laid out [half][block][64 rows]; otherwise a
+      // stage is [block][half][64 rows]
+      const bool pair = VPAIR && !is_k;
       int loaded = NSUB;
       if (NSUB > 1) {
         // a half with no kept token: zeros (generic stores, made visible to
@@ -332,8 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           --loaded;
           zeroed = true;
           for (int x = 0; x < nb; ++x) {
-            uint4* z = reinterpret_cast<uint4*>(smem + (dst - s_kring) + x * kBoxBytes +
-                                                sb * kSubBytes);
+            const int off = pair ? sb * kBoxBytes + x * kSubBytes : x * kBoxBytes + sb * kSubBytes;
+            uint4* z = reinterpret_cast<uint4*>(smem + (dst - s_kring) + off);
             for (int k = lane; k < kSubBytes / 16; k += 32) z[k] = make_uint4(0u, 0u, 0u, 0u);
           }
         }
@@ -343,12 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const uint32_t full = smem_u32(&fullb[s]);
         mbar_arrive_expect_tx(full, (uint32_t)(nb * loaded * kSubBytes));
-        for (int x = 0; x < nb; ++x) {
+        if (pair) {
 #pragma unroll
           for (int sb = 0; sb < NSUB; ++sb)
-            if (NSUB == 1 || c_z[sb] >= 0)
-              tma_load_3d(dst + x * kBoxBytes + sb * kSubBytes, map, grp * 128 + x * 64,
-                          c_row[sb], c_z[sb], full, pol);
+            if (c_z[sb] >= 0)
+              tma_load_4d(dst + sb * kBoxBytes, map, 0, c_row[sb], grp * 2, c_z[sb], full, pol);
+        } else {
+          for (int x = 0; x < nb; ++x) {
+#pragma unroll
+            for (int sb = 0; sb < NSUB; ++sb)
+              if (NSUB == 1 || c_z[sb] >= 0)
+                tma_load_3d(dst + x * kBoxBytes + sb * kSubBytes, map, grp * 128 + x * 64,
+                            c_row[sb], c_z[sb], full, pol);
+          }
         }
       }
       return true;
@@ -504,12 +516,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d = tbase + (uint32_t)(2 * kSAcc * HP + vg * kUAcc * HP);
           // A (MN-major latents): 16 token rows (2 KB) per K step;
           // B (K-major P): 32 B per K step inside a 64-token chunk.
-          const uint64_t a_base =
-              desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes, kBoxBytes);
+          // With VPAIR the two 64-column blocks of a half sit 8 KB apart and
+          // the second half's rows start 16 KB in.
+          const uint64_t a_base = desc_mnmajor_sw128(s_vring + (uint32_t)s * kStageBytes,
+                                                     VPAIR ? kSubBytesV : kBoxBytes);
           const uint64_t b_base = desc_kmajor_sw128(s_p0 + (uint32_t)(pb * a.pbuf_bytes));
 #pragma unroll
           for (int ks = 0; ks < kRows / 16; ++ks)
-            umma_bf16(d + (uint32_t)((ks % kUAcc) * HP), a_base + (uint64_t)(ks * (2048 >> 4)),
+            umma_bf16(d + (uint32_t)((ks % kUAcc) * HP),
+                      a_base + (uint64_t)((VPAIR ? (ks >> 2) * kBoxBytes + (ks & 3) * 2048
+                                                 : ks * 2048) >> 4),
                       b_base + (uint64_t)((ks >> 2) * (HP * 128 >> 4) + (ks & 3) * 2), idesc_u,
                       !(first_of_seg && ks < kUAcc));
           umma_commit(smem_u32(&tl->vempty[s]));
@@ -773,6 +789,7 @@ struct Paged2D {
   const int* block_table;
   int max_blocks, page_size, sink, window;
   unsigned long long stamp;
+  bool vpair;  // 64-token pages: the V map loads both blocks of a half at once
 };
 
 // Absorb, the tensor-core kernel and the merge, shared by the dense and the
@@ -829,8 +846,10 @@ lla_status launch_2d(const float* q, const CUtensorMap& tk, const CUtensorMap& t
 
   // pages of an odd multiple of 64 tokens: each tile half from its own page
   const bool split = pg && pg->page_size % kRows;
-  auto kern = d.hp == 16 ? (split ? k_lla2d<16, 2> : k_lla2d<16, 1>)
-                         : (split ? k_lla2d<32, 2> : k_lla2d<32, 1>);
+  const bool vpair = split && pg->vpair;
+  auto kern = d.hp == 16
+                  ? (vpair ? k_lla2d<16, 2, true> : split ? k_lla2d<16, 2> : k_lla2d<16, 1>)
+                  : (vpair ? k_lla2d<32, 2, true> : split ? k_lla2d<32, 2> : k_lla2d<32, 1>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_lla2d)");
   cudaLaunchAttribute pdl[1];
@@ -965,7 +984,16 @@ lla_status run_decode_2d_paged(const float* q, const void* zk, const void* zv, i
     const uint32_t box[3] = {64, box_rows, 1};
     if (!make_tmap_bf16(&tk, zk, 3, dims, strides, box)) return LLA_ERR_INVALID_ARG;
   }
-  {
+  // 64-token pages with r_v a multiple of 64: the V pool viewed as
+  // [pages][64-column blocks][rows][64 columns], so one box of two blocks x
+  // 64 rows loads a whole half of a value group
+  pg.vpair = page_size % kRows != 0 && r_v % 64 == 0;
+  if (pg.vpair) {
+    const uint64_t dims[4] = {64, (uint64_t)page_size, (uint64_t)(r_v / 64), (uint64_t)num_pages};
+    const uint64_t strides[3] = {(uint64_t)r_v * 2, 128, (uint64_t)page_size * r_v * 2};
+    const uint32_t box[4] = {64, box_rows, 2, 1};
+    if (!make_tmap_bf16(&tv, zv, 4, dims, strides, box)) return LLA_ERR_INVALID_ARG;
+  } else {
     const uint64_t dims[3] = {(uint64_t)r_v, (uint64_t)page_size, (uint64_t)num_pages};
     const uint64_t strides[2] = {(uint64_t)r_v * 2, (uint64_t)page_size * r_v * 2};
     const uint32_t box[3] = {64, box_rows, 1};
