@@ -514,10 +514,9 @@ __global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
 // Accumulators stay in registers: no tensor memory is allocated, so these
 // kernels never contend with the programmatically overlapped k_lla2d for it.
 //
-// Operands are staged row by row as [row][k] bf16 with a pitch of kp + 8
-// elements (kp = k padded to 16). A pitch of kp/2 + 4 words makes the eight
-// rows of a fragment load start 4*(odd) banks apart, so the 32 lanes of every
-// fragment load hit 32 distinct banks.
+// Operands are staged as bf16 rows whose pitch is their width (a multiple
+// of 16 elements) plus 8: the eight 16-byte rows of every ldmatrix then
+// start 4*(odd) banks apart and hit 32 distinct banks.
 
 // hi and lo bf16 parts of four consecutive fp32 values, as 8-byte stores
 __device__ __forceinline__ void store_split4(__nv_bfloat16* hi, __nv_bfloat16* lo, float4 v) {
@@ -533,26 +532,6 @@ __device__ __forceinline__ void store_split4(__nv_bfloat16* hi, __nv_bfloat16* l
   ul.y = *reinterpret_cast<const uint32_t*>(&l23);
   *reinterpret_cast<uint2*>(hi) = uh;
   *reinterpret_cast<uint2*>(lo) = ul;
-}
-
-// fragment of a 16 x 16 A tile (rows m0.., k0..) of a [row][k] bf16 array
-__device__ __forceinline__ void frag_a(uint32_t (&f)[4], const __nv_bfloat16* s, int pitch, int m0,
-                                       int k0, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const __nv_bfloat16* p = s + (m0 + g) * pitch + k0 + 2 * t;
-  f[0] = *reinterpret_cast<const uint32_t*>(p);
-  f[1] = *reinterpret_cast<const uint32_t*>(p + 8 * pitch);
-  f[2] = *reinterpret_cast<const uint32_t*>(p + 8);
-  f[3] = *reinterpret_cast<const uint32_t*>(p + 8 * pitch + 8);
-}
-
-// fragment of a 16 x 8 B tile (k0.., columns n0..) stored as [column][k]
-__device__ __forceinline__ void frag_b(uint32_t (&f)[2], const __nv_bfloat16* s, int pitch, int n0,
-                                       int k0, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const __nv_bfloat16* p = s + (n0 + g) * pitch + k0 + 2 * t;
-  f[0] = *reinterpret_cast<const uint32_t*>(p);
-  f[1] = *reinterpret_cast<const uint32_t*>(p + 8);
 }
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4],
@@ -578,8 +557,7 @@ constexpr int kTcCols = 64;  // q' columns per k_absorb_tc CTA
 constexpr int kTcCh = 32;    // output channels per k_combine_tc CTA
 
 size_t absorb_tc_smem(int d_h) {
-  const int pitch = ((d_h + 15) & ~15) + 8;
-  return (size_t)2 * (kTcRows + kTcCols) * pitch * sizeof(__nv_bfloat16);
+  return (size_t)2 * (kTcRows * (d_h + 8) + d_h * (kTcCols + 8)) * sizeof(__nv_bfloat16);
 }
 
 size_t combine_tc_smem(int r_v) {
@@ -587,17 +565,56 @@ size_t combine_tc_smem(int r_v) {
   return (size_t)2 * (kTcCh + kTcRows) * pitch * sizeof(__nv_bfloat16);
 }
 
+// Fragment loads with ldmatrix: four 8 x 8 bf16 matrices whose rows start
+// at the addresses lanes 0-7, 8-15, 16-23 and 24-31 give. The plain form
+// feeds an A fragment (or two B fragments of a [column][k] array), the
+// transposed form two B fragments of a [k][column] array.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&f)[4], const __nv_bfloat16* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(f[0]), "=r"(f[1]), "=r"(f[2]), "=r"(f[3])
+               : "r"(a));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&f)[4], const __nv_bfloat16* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(f[0]), "=r"(f[1]), "=r"(f[2]), "=r"(f[3])
+               : "r"(a));
+}
+
+__device__ __forceinline__ void mma_split2(float (&d0)[4], float (&d1)[4], const uint32_t (&ah)[4],
+                                           const uint32_t (&al)[4], const uint32_t (&bh)[4],
+                                           const uint32_t (&bl)[4]) {
+  const uint32_t bh0[2] = {bh[0], bh[1]}, bl0[2] = {bl[0], bl[1]};
+  const uint32_t bh1[2] = {bh[2], bh[3]}, bl1[2] = {bl[2], bl[3]};
+  mma_split(d0, ah, al, bh0, bl0);
+  mma_split(d1, ah, al, bh1, bl1);
+}
+
 // One CTA per (head h, 64 q' columns, 64 batch rows): M = batch rows, N =
-// q' columns, K = d_h. Warp w computes rows 16*(w%4).. and columns
-// 32*(w/4).. of the tile. d_h is a multiple of 16 and q 16-byte aligned
-// (the launcher checks); columns past r_k (the rotary part) take q_rope.
-__global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
+// q' columns, K = d_h = DH (64 or 128, a compile-time constant so that the
+// staging index arithmetic is shifts). Warp w computes rows 16*(w%4).. and
+// columns 32*(w/4).. of the tile; columns past r_k (the rotary part) take
+// q_rope. Every thread issues all its loads of both operands before its
+// first shared store: thread t holds float4 t % (DH/4) of query rows
+// t / (DH/4) + k * 1024/DH, and float4 t % 16 of W^K_h rows t / 16 + 16 k,
+// both staged as bf16 hi/lo rows with a pitch of 8 extra elements (the
+// eight rows of every ldmatrix hit distinct banks). W^K_h keeps its
+// [i][column] order; the transposed ldmatrix forms the B fragments. The
+// LLA-2D operand leaves through a shared tile: each batch row's 64 columns
+// are one 128-byte swizzled row of the operand, written as eight 16-byte
+// stores.
+template <int DH>
+__global__ void __launch_bounds__(256, 2) k_absorb_tc(AbsorbArgs a) {
+  static_assert(DH == 64 || DH == 128, "k_absorb_tc stages d_h of 64 or 128");
+  constexpr int QP = DH + 8, WP = kTcCols + 8;
+  constexpr int D4 = DH / 4, KB = DH / 16, QSTEP = 256 / D4;
   extern __shared__ __align__(16) unsigned char sm_abs_tc[];
-  const int pitch = a.d_h + 8;
-  __nv_bfloat16* q_hi = reinterpret_cast<__nv_bfloat16*>(sm_abs_tc);  // [64 rows][pitch]
-  __nv_bfloat16* q_lo = q_hi + kTcRows * pitch;
-  __nv_bfloat16* w_hi = q_lo + kTcRows * pitch;                        // [64 columns][pitch]
-  __nv_bfloat16* w_lo = w_hi + kTcCols * pitch;
+  __nv_bfloat16* q_hi = reinterpret_cast<__nv_bfloat16*>(sm_abs_tc);  // [64 rows][QP]
+  __nv_bfloat16* q_lo = q_hi + kTcRows * QP;
+  __nv_bfloat16* w_hi = q_lo + kTcRows * QP;  // [DH][WP]: W^K_h row i, columns c0..
+  __nv_bfloat16* w_lo = w_hi + DH * WP;
   pdl_launch_dependents();
   const int h = blockIdx.x;
   const int c0 = blockIdx.y * kTcCols;
@@ -606,135 +623,120 @@ __global__ void __launch_bounds__(256, 1) k_absorb_tc(AbsorbArgs a) {
   const int rq = a.r_k + a.d_r;
   const int nc = min(kTcCols, rq - c0);
   const int ncw = max(0, min(kTcCols, a.r_k - c0));  // columns from W^K, a multiple of 8
-  // Stage the query rows and W^K_h's columns c0.. together: both are
-  // 64 * d_h values, 16 * d_h float4 items, and every thread issues its
-  // loads of both before its first shared store (one memory round trip per
-  // 2048 items of each). W^K_h rows i hold the columns contiguously; they
-  // are staged as [column][i], and consecutive threads take consecutive i
-  // so a warp's 2-byte transposed stores fall in 16 consecutive words (the
-  // loads of four columns each reach L1 by rows).
-  const int d4 = a.d_h / 4;
-  const float* D = a.dk + (size_t)h * a.d_h * a.r_k + c0;
-  const int n_items = kTcRows * d4;  // = d_h * kTcCols / 4
-  constexpr int kBatch = 8;
-  for (int base = threadIdx.x; base < n_items; base += 256 * kBatch) {
-    float4 vq[kBatch], vw[kBatch];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qi4 = tid % D4, qrow0 = tid / D4;
+  const int wj4 = tid & 15, wrow0 = tid >> 4;
+  const float* qh = a.q + (size_t)h * DH + 4 * qi4;
+  const float* D = a.dk + (size_t)h * DH * a.r_k + c0 + 4 * wj4;
+  const bool wcol = 4 * wj4 < ncw;
+  float4 vq[KB], vw[KB];
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int idx = base + k * 256;
-      vq[k] = vw[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (idx < n_items) {
-        const int bb = idx / d4, i4 = idx - bb * d4;
-        if (bb < nb)
-          vq[k] = __ldg(reinterpret_cast<const float4*>(
-                            a.q + ((size_t)(b0 + bb) * a.H + h) * a.d_h) + i4);
-        const int j = idx / a.d_h, i = idx - j * a.d_h;
-        if (4 * j < ncw) vw[k] = __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_k) + j);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int idx = base + k * 256;
-      if (idx >= n_items) continue;
-      const int bb = idx / d4, i4 = idx - bb * d4;
-      store_split4(q_hi + bb * pitch + 4 * i4, q_lo + bb * pitch + 4 * i4, vq[k]);
-      const int j = idx / a.d_h, i = idx - j * a.d_h;
-      const float e[4] = {vw[k].x, vw[k].y, vw[k].z, vw[k].w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const __nv_bfloat16 hi = __float2bfloat16_rn(e[c]);
-        w_hi[(4 * j + c) * pitch + i] = hi;
-        w_lo[(4 * j + c) * pitch + i] = __float2bfloat16_rn(e[c] - __bfloat162float(hi));
-      }
-    }
+  for (int k = 0; k < KB; ++k) {
+    const int bb = qrow0 + k * QSTEP;
+    vq[k] = bb < nb ? __ldg(reinterpret_cast<const float4*>(qh + (size_t)(b0 + bb) * a.H * DH))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    vw[k] = wcol ? __ldg(reinterpret_cast<const float4*>(D + (size_t)(wrow0 + 16 * k) * a.r_k))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.y == 0) {
-    // c0 = scale * q . mu_k (natural-log units) in fp32 from the query rows
-    // in global memory (L2), warp w taking rows w, w + 8, ..: all of a
-    // lane's loads are issued before the first sum
-    float part[kTcRows / 8];
+    // c0 = scale * q . mu_k (natural-log units) in fp32 from the loaded
+    // query values: a row's D4 float4s sit in D4 consecutive lanes
+    float mu[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.mu_k)
 #pragma unroll
-    for (int k = 0; k < kTcRows / 8; ++k) part[k] = 0.f;
-    if (a.mu_k) {
-      float mu[8];  // d_h <= 256: at most 8 values per lane
+      for (int e = 0; e < 4; ++e) mu[e] = __ldg(a.mu_k + (size_t)h * DH + 4 * qi4 + e);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int i = lane + 32 * m;
-        mu[m] = i < a.d_h ? __ldg(a.mu_k + (size_t)h * a.d_h + i) : 0.f;
-      }
+    for (int k = 0; k < KB; ++k) {
+      float acc = fmaf(vq[k].x, mu[0], fmaf(vq[k].y, mu[1], fmaf(vq[k].z, mu[2], vq[k].w * mu[3])));
 #pragma unroll
-      for (int k = 0; k < kTcRows / 8; ++k) {
-        const int bb = warp + 8 * k;
-        const float* qr = a.q + ((size_t)(b0 + bb) * a.H + h) * a.d_h;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int i = lane + 32 * m;
-          if (bb < nb && i < a.d_h) part[k] = fmaf(__ldg(qr + i), mu[m], part[k]);
-        }
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kTcRows / 8; ++k) {
-      const int bb = warp + 8 * k;
-      const float acc = warp_sum(part[k]);
-      if (lane == 0 && bb < nb)
+      for (int o = D4 / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      const int bb = qrow0 + k * QSTEP;
+      if (qi4 == 0 && bb < nb)
         st_chk(&a.c0[(size_t)(b0 + bb) * a.H + h], a.scale * acc, a.ws_span, a.status);
     }
   }
+#pragma unroll
+  for (int k = 0; k < KB; ++k) {
+    const int bb = qrow0 + k * QSTEP, i = wrow0 + 16 * k;
+    store_split4(q_hi + bb * QP + 4 * qi4, q_lo + bb * QP + 4 * qi4, vq[k]);
+    store_split4(w_hi + i * WP + 4 * wj4, w_lo + i * WP + 4 * wj4, vw[k]);
+  }
+  __syncthreads();
   const int m0 = (warp & 3) * 16, n0 = (warp >> 2) * 32;
+  const int lr = lane & 15, lc = (lane >> 4) * 8;
   float acc[4][4];
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
   if (n0 < ncw) {
-    for (int k0 = 0; k0 < a.d_h; k0 += 16) {
-      uint32_t ah[4], al[4];
-      frag_a(ah, q_hi, pitch, m0, k0, lane);
-      frag_a(al, q_lo, pitch, m0, k0, lane);
+#pragma unroll 4
+    for (int k0 = 0; k0 < DH; k0 += 16) {
+      uint32_t ah[4], al[4], bh[4], bl[4];
+      ldsm_x4(ah, q_hi + (m0 + lr) * QP + k0 + lc);
+      ldsm_x4(al, q_lo + (m0 + lr) * QP + k0 + lc);
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        uint32_t bh[2], bl[2];
-        frag_b(bh, w_hi, pitch, n0 + 8 * nt, k0, lane);
-        frag_b(bl, w_lo, pitch, n0 + 8 * nt, k0, lane);
-        mma_split(acc[nt], ah, al, bh, bl);
+      for (int np = 0; np < 2; ++np) {
+        ldsm_x4_t(bh, w_hi + (k0 + lr) * WP + n0 + 16 * np + lc);
+        ldsm_x4_t(bl, w_lo + (k0 + lr) * WP + n0 + 16 * np + lc);
+        mma_split2(acc[2 * np], acc[2 * np + 1], ah, al, bh, bl);
       }
     }
   }
+  if (a.qsw) __syncthreads();  // the output tile reuses q_hi
+  __nv_bfloat16* tile = q_hi;  // [64 rows][WP] bf16 q' of this column block
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int bb = m0 + g + (e >> 1) * 8;
-      const int cl = n0 + 8 * nt + 2 * t + (e & 1);
-      if (bb >= nb || cl >= nc) continue;
-      const int c = c0 + cl;
+    for (int hr = 0; hr < 2; ++hr) {
+      const int bb = m0 + g + 8 * hr;
+      const int cl = n0 + 8 * nt + 2 * t;
       const size_t unit = (size_t)(b0 + bb) * a.H + h;
-      // the rotary part of the query is not absorbed: it meets the cached
-      // rotated keys as it is
-      const float v = (c < a.r_k ? acc[nt][e] : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) *
-                      a.qscale;
-      if (a.qp) st_chk(&a.qp[unit * rq + c], v, a.ws_span, a.status);
-      if (a.qsw) {
-        unsigned char* base = a.qsw + qsw_block(a, rq, b0 + bb);
-        st_chk(reinterpret_cast<__nv_bfloat16*>(base + sw128_off(h, c, a.hp)), __float2bfloat16_rn(v),
-               a.ws_span, a.status);
-        if (h == a.H - 1)
-          for (int hz = a.H; hz < a.hp; ++hz)
-            st_chk(reinterpret_cast<__nv_bfloat16*>(base + sw128_off(hz, c, a.hp)),
-                   __float2bfloat16_rn(0.f), a.ws_span, a.status);
+      float v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = c0 + cl + e;
+        // the rotary part of the query is not absorbed: it meets the cached
+        // rotated keys as it is; columns past rq are the operand's zero pad
+        v[e] = (bb >= nb || cl + e >= nc) ? 0.f
+               : (c < a.r_k ? acc[nt][2 * hr + e]
+                            : __ldg(a.q_rope + unit * a.d_r + (c - a.r_k))) * a.qscale;
+        if (a.qp && bb < nb && cl + e < nc) st_chk(&a.qp[unit * rq + c], v[e], a.ws_span, a.status);
       }
+      if (a.qsw)
+        *reinterpret_cast<__nv_bfloat162*>(tile + bb * WP + cl) = __floats2bfloat162_rn(v[0], v[1]);
     }
-  if (a.qsw && c0 + nc == rq) zero_qsw_tail(a, rq, h, b0, nb);
+  if (!a.qsw) return;
+  __syncthreads();
+  // 16-byte chunk j (columns 8j..8j+7) of a batch row lands at chunk
+  // j ^ (h & 7) of row h of the 128-byte swizzle row; the padding heads'
+  // rows (after the last head) are zero
+  const size_t cblock = (size_t)(c0 / 64) * a.hp * 128;
+  for (int idx = tid; idx < kTcRows * 8; idx += 256) {
+    const int bb = idx >> 3, j = idx & 7;
+    if (bb >= nb) continue;
+    unsigned char* rowp = a.qsw + qsw_block(a, rq, b0 + bb) + cblock;
+    st_chk(reinterpret_cast<uint4*>(rowp + h * 128 + ((j ^ (h & 7)) << 4)),
+           *reinterpret_cast<const uint4*>(tile + bb * WP + 8 * j), a.ws_span, a.status);
+    if (h == a.H - 1)
+      for (int hz = a.H; hz < a.hp; ++hz)
+        st_chk(reinterpret_cast<uint4*>(rowp + hz * 128 + (j << 4)), make_uint4(0u, 0u, 0u, 0u),
+               a.ws_span, a.status);
+  }
 }
 
 // One CTA per (head h, 32 output channels, 64 batch rows): the merge of
 // k_combine (same record map, same order of operations), with ubar written
 // split into shared memory, then out = W^V ubar with M = channels, N = batch
 // rows, K = r_v. Warp w computes channels 16*(w%2).. for rows 16*(w/2)...
+//
+// Shared-memory work is spread so that every index is a warp or lane
+// number, not a quotient: warp w stages W^V rows w, w+8, .. and merges
+// batch rows w, w+8, .. (a row's record offset, piece count, maximum and
+// normaliser are the same for the whole warp), lane l taking the float4
+// columns l, l+32, .. of each. Both tiles are [row][k] bf16 hi/lo arrays
+// read with ldmatrix.
 __global__ void __launch_bounds__(256, 2) k_combine_tc(CombineArgs a) {
   extern __shared__ __align__(16) unsigned char sm_cmb_tc[];
   __shared__ int s_np[kTcRows];
@@ -751,31 +753,98 @@ __global__ void __launch_bounds__(256, 2) k_combine_tc(CombineArgs a) {
   const int b0 = blockIdx.z * kTcRows;
   const int nb = min(kTcRows, a.B - b0);
   const int ni = min(kTcCh, a.d_h - i0);
-  const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r4 = a.r_v / 4, k4 = kp / 4;
-  // decoder slice; channels past d_h and columns past r_v are zero
-  stage_batched(kTcCh * k4, [&](int idx) {
-    const int i = idx / k4, j = idx - i * k4;
-    return (i < ni && j < r4) ? __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-  }, [&](int idx, float4 v) {
-    const int i = idx / k4, j = idx - i * k4;
-    store_split4(d_hi + i * pitch + 4 * j, d_lo + i * pitch + 4 * j, v);
-  });
+  // decoder slice, 64 float4 columns of 4 rows per warp in flight; channels
+  // past d_h and columns past r_v are zero
+  const float* D = a.dv + ((size_t)h * a.d_h + i0) * a.r_v;
+  for (int cb = 0; cb < k4; cb += 64) {
+    float4 v[4][2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int i = warp + 8 * k, j = cb + lane + 32 * cc;
+        v[k][cc] = (i < ni && j < r4)
+                       ? __ldg(reinterpret_cast<const float4*>(D + (size_t)i * a.r_v) + j)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int i = warp + 8 * k, j = cb + lane + 32 * cc;
+        if (j < k4) store_split4(d_hi + i * pitch + 4 * j, d_lo + i * pitch + 4 * j, v[k][cc]);
+      }
+  }
   if (threadIdx.x < kTcCh)
     s_mu[threadIdx.x] = (a.mu_v && (int)threadIdx.x < ni) ? __ldg(a.mu_v + (size_t)h * a.d_h + i0 + threadIdx.x) : 0.f;
   pdl_wait();  // partials come from the streaming kernel
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // 1. per row: its records, merged maximum and normaliser
   merge_rows(a, h, b0, nb, kTcRows, s_np, s_off, s_M, s_inv, s_keep);
   __syncthreads();
 
-  // 2. ubar rows, split into shared memory; rows with no piece and the
-  //    padding columns come out 0
-  merge_sweep(a, kTcRows, k4, r4, s_np, s_off, s_M, s_inv, [&](int bb, int c4, float4 v) {
-    store_split4(u_hi + bb * pitch + 4 * c4, u_lo + bb * pitch + 4 * c4, v);
-  });
+  // 2. ubar rows, split into shared memory: warp w takes rows w + 8k, four
+  //    at a time with all their piece loads in flight; rows with no piece
+  //    and the padding columns come out 0
+  const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
+  for (int cb = 0; cb < k4; cb += 64)
+    for (int k0 = 0; k0 < kTcRows / 8; k0 += 4) {
+      float4 acc[4][2];
+      int np[4];
+      int npmax = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        np[k] = s_np[warp + 8 * (k0 + k)];
+        npmax = max(npmax, np[k]);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) acc[k][cc] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int p = 0; p < npmax; ++p) {
+        float mv[4];
+        float4 uv[4][2];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int bb = warp + 8 * (k0 + k);
+          const float* rec = a.part + s_off[bb] + p * rstride;
+          mv[k] = p < np[k] ? ld_chk(rec, a.ws_span, a.status, kNegBig) : kNegBig;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int j = cb + lane + 32 * cc;
+            uv[k][cc] = (p < np[k] && j < r4)
+                            ? ld_chk(reinterpret_cast<const float4*>(rec + 4) + j, a.ws_span,
+                                     a.status, make_float4(0.f, 0.f, 0.f, 0.f))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (p < np[k]) {
+            const float wk = exp2f(mv[k] - s_M[warp + 8 * (k0 + k)]);
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              acc[k][cc].x = fmaf(wk, uv[k][cc].x, acc[k][cc].x);
+              acc[k][cc].y = fmaf(wk, uv[k][cc].y, acc[k][cc].y);
+              acc[k][cc].z = fmaf(wk, uv[k][cc].z, acc[k][cc].z);
+              acc[k][cc].w = fmaf(wk, uv[k][cc].w, acc[k][cc].w);
+            }
+          }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int bb = warp + 8 * (k0 + k);
+        const float inv = s_inv[bb];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int j = cb + lane + 32 * cc;
+          if (j < k4)
+            store_split4(u_hi + bb * pitch + 4 * j, u_lo + bb * pitch + 4 * j,
+                         make_float4(acc[k][cc].x * inv, acc[k][cc].y * inv, acc[k][cc].z * inv,
+                                     acc[k][cc].w * inv));
+        }
+      }
+    }
   __syncthreads();
 
   // 3. out tile = W^V slice (32 x kp) . ubar^T (kp x 64)
@@ -786,17 +855,17 @@ __global__ void __launch_bounds__(256, 2) k_combine_tc(CombineArgs a) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
   if (m0 < ni && n0 < nb) {
+    const __nv_bfloat16* pa = d_hi + (m0 + (lane & 15)) * pitch + (lane >> 4) * 8;
+    const __nv_bfloat16* pb =
+        u_hi + (n0 + (lane & 7) + ((lane >> 4) << 3)) * pitch + ((lane >> 3) & 1) * 8;
+    const int lo_a = kTcCh * pitch, lo_b = kTcRows * pitch;
     for (int k0 = 0; k0 < kp; k0 += 16) {
-      uint32_t ah[4], al[4];
-      frag_a(ah, d_hi, pitch, m0, k0, lane);
-      frag_a(al, d_lo, pitch, m0, k0, lane);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        uint32_t bh[2], bl[2];
-        frag_b(bh, u_hi, pitch, n0 + 8 * nt, k0, lane);
-        frag_b(bl, u_lo, pitch, n0 + 8 * nt, k0, lane);
-        mma_split(acc[nt], ah, al, bh, bl);
-      }
+      uint32_t ah[4], al[4], bh[4], bl[4];
+      ldsm_x4(ah, pa + k0);
+      ldsm_x4(al, pa + lo_a + k0);
+      ldsm_x4(bh, pb + k0);
+      ldsm_x4(bl, pb + lo_b + k0);
+      mma_split2(acc[0], acc[1], ah, al, bh, bl);
     }
   }
   const int g = lane >> 2, t = lane & 3;
@@ -833,13 +902,17 @@ lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int
   AbsorbArgs a{q, dk, mu_k, B, H, d_h, r_k, scale * kLog2e, scale, qp, c0, qsw, hp,
                q_rope, q_rope ? d_r : 0, ws, status_word()};
   const int rq = r_k + a.d_r;
-  if (tc && d_h % 16 == 0 && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
+  // the tensor-core form stages d_h of 64 or 128 with float4 loads of q and
+  // W^K (16-byte aligned, r_k a multiple of 8)
+  if (tc && (d_h == 64 || d_h == 128) && r_k % 8 == 0 &&
+      ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(dk)) & 15) == 0) {
     const size_t smem = absorb_tc_smem(d_h);
-    cudaError_t e = cudaFuncSetAttribute(k_absorb_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = d_h == 128 ? k_absorb_tc<128> : k_absorb_tc<64>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(k_absorb_tc)");
     dim3 grid(H, (rq + kTcCols - 1) / kTcCols, (B + kTcRows - 1) / kTcRows);
-    k_absorb_tc<<<grid, 256, smem, stream>>>(a);
+    kern<<<grid, 256, smem, stream>>>(a);
     return check_cuda(cudaGetLastError(), "launch k_absorb_tc");
   }
   int rows, cols;
