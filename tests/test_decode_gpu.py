@@ -110,9 +110,10 @@ def test_many_units_few_tokens_and_repeat_calls():
 def test_large_batch_absorb_and_combine(d_h, r_k, r_v):
     # From B = 256 with a rank of 192 or more the per-head path forms q' and
     # W^V ubar on the tensor cores with split bf16 operands (the others stay
-    # on the CUDA cores); 300 rows leave a ragged 64-row block, d_h = 40
-    # keeps the CUDA-core absorb with the tensor-core combine, and the
-    # fp32-level bound of run_case holds for the split products.
+    # on the CUDA cores); 300 rows leave a ragged 64-row block, d_h = 16
+    # and 40 keep the CUDA-core absorb (the tensor-core one stages d_h of 64
+    # or 128) with the tensor-core combine, and the fp32-level bound of
+    # run_case holds for the split products.
     B, H = 300, 3
     pick = [(b, h) for b in (0, 1, 63, 64, 255, 256, 299) for h in range(H)]
     run_case(B, H, d_h, 200, r_k, r_v, BF16, units=pick, mu=True, decay=True, seed=d_h + r_k)

@@ -39,6 +39,13 @@ def test_head_counts(H):
     run(2, H, 64, 400, 128, 128, mu=True, seed=H)
 
 
+@pytest.mark.parametrize("d_h", [16, 32, 96, 256])
+def test_head_widths(d_h):
+    # d_h of 64 and 128 form Q' on the tensor cores; the others take the
+    # CUDA-core absorb, which writes the same swizzled operand
+    run(3, 16, d_h, 300, 128, 128, mu=True, seed=d_h)
+
+
 @pytest.mark.parametrize("r_k, r_v", [(64, 128), (128, 256), (192, 128), (256, 128), (256, 256)])
 def test_ranks(r_k, r_v):
     run(2, 16, 128, 333, r_k, r_v, seed=r_k + r_v)
