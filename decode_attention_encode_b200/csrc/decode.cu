@@ -347,14 +347,15 @@ __device__ __forceinline__ void merge_rows(const CombineArgs& a, int h, int b0, 
 
 // merge_sweep: ubar[row] = sum_p exp2(m_p - M) u_p / L over the CTA's
 // (row, 4-column) items, k4 items per row of which the first r4 hold values
-// (the rest are padding and come out 0), eight items per thread at a time
-// so their record loads are in flight together. Rows with no piece come out
-// 0. store(bb, c4, v) places each normalised float4.
+// (the rest are padding and come out 0), four items per thread at a time
+// so their record loads are in flight together (a CTA rarely has more than
+// one or two items per thread: larger blocks take k_combine_tc). Rows with
+// no piece come out 0. store(bb, c4, v) places each normalised float4.
 template <class Store>
 __device__ __forceinline__ void merge_sweep(const CombineArgs& a, int nrows, int k4, int r4,
                                             const int* s_np, const long long* s_off,
                                             const float* s_M, const float* s_inv, Store store) {
-  constexpr int kI = 8;
+  constexpr int kI = 4;
   const long long rstride = a.shared ? (long long)a.H * a.pstride : a.pstride;
   const int nitems = nrows * k4;
   for (int base = threadIdx.x; base < nitems; base += 256 * kI) {
@@ -415,17 +416,18 @@ __device__ __forceinline__ void merge_sweep(const CombineArgs& a, int nrows, int
   }
 }
 
-// One CTA per (head, 32 output channels, 8*ROWS batch rows). The CTA stages
-// its 32 x r_v slice of W^V_up,t (rows padded by 4 floats, so float4 reads
+// One CTA per (head, 32*COLS output channels, 8*ROWS batch rows). The CTA
+// stages its 32*COLS x r_v slice of W^V_up,t (rows padded by 4 floats, so float4 reads
 // of 8 consecutive rows hit distinct bank groups; staged before waiting on
 // the streaming kernel), then merges the partial records of its rows into
 // ubar: one thread per row forms the merged maximum and normaliser, then
 // all threads sweep the (row, 4-column) items with several records in
 // flight each, since this kernel is bound by memory round trips, not
-// bandwidth. Thread (w, l) finally forms out[b][h][i0 + l] for its ROWS
-// rows.
+// bandwidth. Thread (w, l) finally forms out[b][h][i0 + l + 32 j] for its
+// ROWS rows. Three CTAs fit an SM (80 registers), so the 384 CTAs of a
+// 768-sequence batch run in one wave.
 template <int ROWS, int COLS>
-__global__ void __launch_bounds__(256, 2) k_combine(CombineArgs a) {
+__global__ void __launch_bounds__(256, 3) k_combine(CombineArgs a) {
   constexpr int CW = 32 * COLS;  // output channels per CTA
   extern __shared__ __align__(16) float sm_combine[];
   // per row of the CTA: pieces, offset of the first record, merged max,
