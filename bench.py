@@ -57,6 +57,31 @@ def main_kernel(config_name: str):
     return "k_stream", os.path.join(CSRC, "stream.cu")
 
 
+def step_runner(step, eager: bool):
+    """What the device-timed region runs per step: the workload's step
+    replayed from a CUDA graph captured once (the same kernels on the same
+    buffers, launched without per-call host work), or the eager calls.
+    Returns (run, description)."""
+    if eager:
+        return step, "eager library calls"
+    try:
+        stream = torch.cuda.current_stream()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+    except Exception as e:  # a capture the runtime refuses: time the eager calls
+        torch.cuda.synchronize()
+        return step, f"eager library calls (graph capture failed: {type(e).__name__})"
+    return graph.replay, "one step captured as a CUDA graph, replayed"
+
+
 def with_layers(cfg, layers: int):
     """The workload with `layers` layers (0: its own count)."""
     import dataclasses
@@ -74,6 +99,9 @@ def parse_args():
     p.add_argument("--layers", type=int, default=0,
                    help="run the workload with this many layers instead of its own (a smaller "
                         "case for profiler captures; the JSON line names the layer count)")
+    p.add_argument("--eager", action="store_true",
+                   help="time the steps as eager library calls instead of replaying one "
+                        "captured step graph")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -276,10 +304,11 @@ class DecodeWorkload:
             self.enc_split = need > 0
             self.enc_ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
 
-    def step(self, q=None, out=None, lse=None, xk=None, xv=None):
+    def step(self, q=None, out=None, lse=None, xk=None, xv=None, timers=None):
         """One looped decode step: loops outer, layers inner (each loop's
         query depends on the previous loop's output in a real model), then
-        the newest token's latent write."""
+        the newest token's latent write. With `timers` (launch_timers) the
+        main kernel of every decode call is bracketed by its own events."""
         c = self.cfg
         q = self.q if q is None else q
         out = self.out if out is None else out
@@ -287,7 +316,11 @@ class DecodeWorkload:
         self.plan()
         for t in range(c.T):
             for l in range(c.L):
+                if timers is not None:
+                    timers.next()
                 self.call(l, t, q, out, lse)
+        if timers is not None:
+            timers.pause()
         if self.write_latents:
             self.write_newest(self.xk if xk is None else xk, self.xv if xv is None else xv)
 
@@ -382,9 +415,11 @@ class EncodeWorkload:
         self.z = [torch.empty((c.G, c.N, c.r), device=device, dtype=torch.bfloat16)
                   for _ in range(2 * c.L)]
 
-    def step(self, x=None):
+    def step(self, x=None, timers=None):
         x = self.x if x is None else x
         for i in range(2 * self.cfg.L):
+            if timers is not None:
+                timers.next()
             self.lla.lla_encode_with_bias(x[i], self.w_t[i], self.muw[i], z=self.z[i],
                                           z_row_stride=self.cfg.r,
                                           z_group_stride=self.cfg.N * self.cfg.r, split=False)
@@ -401,6 +436,9 @@ def run_encode_bench(args, world, rank, local):
     for _ in range(args.warmup):
         wl.step()
     torch.cuda.synchronize()
+    run_step, execution = step_runner(wl.step, args.eager)
+    run_step()
+    torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -409,20 +447,19 @@ def run_encode_bench(args, world, rank, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        wl.step()
+        run_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     ms_per_step = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
-    kern = []
-    for i in range(2 * cfg.L):
-        with wl.lla.kernel_timer() as kt:
-            wl.lla.lla_encode_with_bias(wl.x[i], wl.w_t[i], wl.muw[i], z=wl.z[i],
-                                        z_row_stride=cfg.r, z_group_stride=cfg.N * cfg.r,
-                                        split=False)
-        kern.append(kt.ms)
-    kern_ms = sum(kern) / len(kern)
+    # every encode kernel of a second pass of the steps, bracketed by its own
+    # pair of CUDA events that the library records on the call's stream
+    timers = wl.lla.launch_timers(args.steps * wl.launches_per_step())
+    with timers:
+        for _ in range(args.steps):
+            wl.step(timers=timers)
+    kern_ms = sum(timers.ms) / len(timers.ms)
     call_bytes = (cfg.T * cfg.N * cfg.G * cfg.d_loop + cfg.G * cfg.N * cfg.r) * 2
     hbm_peak, peak_src = peaks()
     tc_peak, tc_src = tensor_peak()
@@ -439,7 +476,8 @@ def run_encode_bench(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": f"{cfg.name}: lla_encode of N={cfg.N} tokens x G={cfg.G} heads x "
                                f"{cfg.L} layers x 2 axes, stack {cfg.T}x{cfg.d_loop}, r={cfg.r}",
-                   "step": f"{2 * cfg.L} encode calls", "accumulation": "fp32",
+                   "step": f"{2 * cfg.L} encode calls", "execution": execution,
+                   "accumulation": "fp32",
                    "l2": "no flush: each call reads 0.54 GB of fresh input",
                    "parallelism": f"dp{world} (independent sequences per GPU)"},
         "roofline": ({"bound": "tensor", "achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s",
@@ -456,7 +494,11 @@ def run_encode_bench(args, world, rank, local):
         "e2e": None,
     }
     line["roofline"].update({"traffic": profiled_traffic(cfg.name), "kernel": "k_encode",
-                             "kernel_ms_mean": kern_ms, "algorithmic_bytes_per_launch": call_bytes,
+                             "kernel_ms_mean": kern_ms,
+                             "kernel_timing": f"every k_encode launch of a second pass of the "
+                                              f"{args.steps} timed steps, CUDA events on the "
+                                              "call's stream",
+                             "algorithmic_bytes_per_launch": call_bytes,
                              "algorithmic_flops_per_launch": flops})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -750,6 +792,9 @@ def run_lla(args, world, rank, local):
     for _ in range(args.warmup):
         wl.step()
     torch.cuda.synchronize()
+    run_step, execution = step_runner(wl.step, args.eager)
+    run_step()
+    torch.cuda.synchronize()
 
     # device-timed region
     clocks = ClockSampler(local)
@@ -758,25 +803,9 @@ def run_lla(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    call_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(cfg.L)]
     ev[0].record(stream)
-    for k in range(args.steps):
-        if k == args.steps - 1:
-            # time each whole call of the last step's first loop on its own
-            c = cfg
-            wl.plan()
-            for t in range(c.T):
-                for l in range(c.L):
-                    if t == 0:
-                        call_ev[l][0].record(stream)
-                    wl.call(l, t)
-                    if t == 0:
-                        call_ev[l][1].record(stream)
-            if wl.write_latents:
-                wl.write_newest(wl.xk, wl.xv)
-        else:
-            wl.step()
+    for _ in range(args.steps):
+        run_step()
     ev[1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -784,17 +813,34 @@ def run_lla(args, world, rank, local):
     elapsed_ms = ev[0].elapsed_time(ev[1])
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_per_step = elapsed_ms / args.steps
+
+    # each whole call of one eager step's first loop, timed on its own
+    call_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(cfg.L)]
+    wl.plan()
+    for t in range(cfg.T):
+        for l in range(cfg.L):
+            if t == 0:
+                call_ev[l][0].record(stream)
+            wl.call(l, t)
+            if t == 0:
+                call_ev[l][1].record(stream)
+    if wl.write_latents:
+        wl.write_newest(wl.xk, wl.xv)
+    torch.cuda.synchronize()
     call_ms = sorted(a.elapsed_time(b) for a, b in call_ev)
     call_ms_mean = sum(call_ms) / len(call_ms)
 
-    # the main kernel alone, timed with CUDA events that the library records
-    # on the call's stream right around that kernel (one call per layer)
-    kern_ms = []
-    for l in range(cfg.L):
-        with wl.lla.kernel_timer() as kt:
-            wl.call(l, 0)
-        kern_ms.append(kt.ms)
-    kern_ms_mean = sum(kern_ms) / len(kern_ms)
+    # the main kernel alone: a second pass over the same steps in which the
+    # library brackets every main-kernel launch with its own pair of CUDA
+    # events on the call's stream (kept out of the first pass, which gives
+    # value and ms_per_step: an event between two programmatically launched
+    # kernels would order them fully)
+    timers = wl.lla.launch_timers(args.steps * cfg.L * cfg.T)
+    with timers:
+        for _ in range(args.steps):
+            wl.step(timers=timers)
+    kern_ms_mean = sum(timers.ms) / len(timers.ms)
 
     tokens_per_step = cfg.tokens() * cfg.L * cfg.T
     value = aggregate_rate(tokens_per_step, ms_per_step, world)
@@ -889,6 +935,7 @@ def run_lla(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": describe(cfg),
+            "execution": execution,
             "step": (f"one plan kernel, then " if wl.paged else "")
                     + f"{cfg.L * cfg.T} decode calls (T loops x L layers), 3 kernels each"
                     + (f", then {2 * cfg.L} latent writes of the newest token" if wl.write_latents else ""),
@@ -905,6 +952,8 @@ def run_lla(args, world, rank, local):
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": profiled_traffic(cfg.name),
             "kernel": kname, "kernel_ms_mean": kern_ms_mean,
+            "kernel_timing": f"every {kname} launch of a second pass of the {args.steps} timed "
+                             "steps, CUDA events on the call's stream",
             "algorithmic_bytes_per_launch": step_bytes,
             "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs (copy, burst)"
             if peak_src == "measured" else "fallback 6.65 TB/s",

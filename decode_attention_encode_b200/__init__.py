@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     LLAError,
     device_status,
     kernel_timer,
+    launch_timers,
     lib,
     library_path,
     lla2d_decode_attn,

@@ -299,6 +299,43 @@ class kernel_timer:
         return False
 
 
+class launch_timers:
+    """Times the main kernel of each of up to n library calls made inside
+    it, with no synchronisation between the calls: next() before a call
+    points the library's timing hook at a fresh pair of CUDA events. After
+    the block, `ms` lists the elapsed time of every timed kernel."""
+
+    def __init__(self, n):
+        stream = torch.cuda.current_stream()
+        self.pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(n)]
+        for b, e in self.pairs:  # torch creates the CUDA events on first record
+            b.record(stream)
+            e.record(stream)
+        stream.synchronize()
+        self.used = 0
+        self.ms = None
+
+    def next(self):
+        _expect(self.used < len(self.pairs), "launch_timers: more calls than event pairs")
+        b, e = self.pairs[self.used]
+        self.used += 1
+        lib().lla_set_timing_events(ctypes.c_void_p(b.cuda_event), ctypes.c_void_p(e.cuda_event))
+
+    def pause(self):
+        """Calls made until the next next() are not timed."""
+        lib().lla_set_timing_events(None, None)
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        lib().lla_set_timing_events(None, None)
+        torch.cuda.synchronize()
+        self.ms = [b.elapsed_time(e) for b, e in self.pairs[:self.used]]
+        return False
+
+
 def lla_decode_attn_workspace(B, H, N, r_k, r_v) -> int:
     return int(lib().lla_decode_attn_workspace(B, H, N, r_k, r_v))
 

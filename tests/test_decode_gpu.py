@@ -152,6 +152,28 @@ def test_rows_beyond_N_are_never_read(dtype):
     compare(out, lse, units, ref_out, ref_lse, dtype)
 
 
+def test_launch_timers_bracket_each_streaming_kernel_without_syncs():
+    inp = make_decode_inputs(64, 16, 128, 2048, 128, 128, BF16, seed=6)
+    args = (inp["q"], inp["zk"], inp["zv"], inp["dk"], inp["dv"])
+    lla.lla_decode_attn(*args)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with lla.launch_timers(4) as lt:
+        ev[0].record()
+        for _ in range(3):
+            lt.next()
+            lla.lla_decode_attn(*args)
+        lt.pause()
+        lla.lla_decode_attn(*args)  # not timed
+        ev[1].record()
+    assert lt.used == 3 and len(lt.ms) == 3
+    total = ev[0].elapsed_time(ev[1])
+    assert all(m > 0 for m in lt.ms) and sum(lt.ms) < total
+    with pytest.raises(lla.LLAError):
+        with lla.launch_timers(1) as lt:
+            lt.next()
+            lt.next()
+
+
 def test_kernel_timer_brackets_the_streaming_kernel():
     inp = make_decode_inputs(64, 16, 128, 2048, 128, 128, BF16, seed=5)
     args = (inp["q"], inp["zk"], inp["zv"], inp["dk"], inp["dv"])
