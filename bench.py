@@ -874,49 +874,75 @@ def run_lla(args, world, rank, local):
         x_devs = [torch.empty_like(wl.xk), torch.empty_like(wl.xv)] if wl.write_latents else []
         out_host = torch.empty(wl.out.shape, dtype=torch.float32).pin_memory()
         lse_host = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
-        in_ev = [[torch.cuda.Event() for _ in range(c.L)] for _ in range(c.T)]
-        x_ev = torch.cuda.Event()
-        done_ev = [[torch.cuda.Event() for _ in range(c.L)] for _ in range(c.T)]
+        # Each buffer waits only for its own last use: call (l, t)'s query
+        # copy for the next step waits for this step's call (l, t), its
+        # output for this step's read-back of (l, t), so one step's copies
+        # run under the neighbouring steps' calls.
+        ev = lambda: [[torch.cuda.Event() for _ in range(c.L)] for _ in range(c.T)]
+        in_ev, done_ev, back_ev = ev(), ev(), ev()
+        x_ev, wrote_ev, pg_ev, end_ev = (torch.cuda.Event() for _ in range(4))
+        pg_stream = torch.cuda.Stream() if wl.paged else None
+        state = {"first": True}
 
         def e2e_step():
+            first = state["first"]
+            state["first"] = False
+            if wl.paged:  # lengths and table: free once the previous step is done
+                with torch.cuda.stream(pg_stream):
+                    if first:
+                        pg_stream.wait_stream(stream)
+                    else:
+                        pg_stream.wait_event(end_ev)
+                    for d_, h_ in zip(pg_devs, pg_hosts):
+                        d_.copy_(h_, non_blocking=True)
+                    pg_ev.record(pg_stream)
             with torch.cuda.stream(h2d):
-                h2d.wait_stream(stream)  # buffers of the previous step are free
-                for d_, h_ in zip(pg_devs, pg_hosts):
-                    d_.copy_(h_, non_blocking=True)
+                if first:
+                    h2d.wait_stream(stream)
                 for t in range(c.T):
                     for l in range(c.L):
+                        if not first:
+                            h2d.wait_event(done_ev[t][l])  # the previous step's call (l, t)
                         q_dev[l, t].copy_(q_host[l, t], non_blocking=True)
                         if wl.rope:
                             qr_dev[l, t].copy_(qr_host[l, t], non_blocking=True)
                         in_ev[t][l].record(h2d)
+                if not first:
+                    h2d.wait_event(wrote_ev)  # the previous step's latent write
                 for d_, h_ in zip(x_devs, x_hosts):
                     d_.copy_(h_, non_blocking=True)
                 x_ev.record(h2d)
             if wl.paged:  # the step's plan reads the lengths and table just copied
-                stream.wait_event(in_ev[0][0])
+                stream.wait_event(pg_ev)
                 wl.plan()
             for t in range(c.T):
                 for l in range(c.L):
                     stream.wait_event(in_ev[t][l])
+                    if not first:
+                        stream.wait_event(back_ev[t][l])  # out[l, t] has been read back
                     wl.call(l, t, q=q_dev, q_rope=qr_dev)
                     done_ev[t][l].record(stream)
                     with torch.cuda.stream(d2h):
                         d2h.wait_event(done_ev[t][l])
                         out_host[l, t].copy_(wl.out[l, t], non_blocking=True)
                         lse_host[l, t].copy_(wl.lse[l, t], non_blocking=True)
+                        back_ev[t][l].record(d2h)
             if wl.write_latents:
                 stream.wait_event(x_ev)
                 wl.write_newest(*x_devs)
-            stream.wait_stream(d2h)
+            wrote_ev.record(stream)
+            end_ev.record(stream)
 
         for _ in range(2):
             e2e_step()
+        stream.wait_stream(d2h)
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
             e2e_step()
+        stream.wait_stream(d2h)  # the last outputs have landed on the host
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
