@@ -391,28 +391,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     bool ok = true;
     int it = 0;
-    if (!is_k) {
-      for (; ok && it < total; ++it) ok = issue(it);
-    } else if (ntile > 0) {
+    if (!is_k || ntile > 0) {
+      // One loop for both rings, so the load code is laid down once. The
+      // K ring's loads of its first sequence (up to a ring's worth) do not
+      // depend on k_absorb; before anything else it waits for that grid
+      // and stages the sequence's Q', and each later sequence's Q' when
+      // its first tile comes up. The V ring never waits.
       const int b0 = pc.b;
-      // latent loads of the first sequence do not depend on k_absorb
-      while (ok && it < total && it < nring) {
-        tile_of(it / ng);
-        if (pc.b != b0) break;
-        ok = issue(it++);
-      }
-      pdl_wait();
-      if (ok) ok = stage_q(0, b0);
+      bool waited = !is_k;
       int seg = 0, cur_b = b0;
       for (; ok && it < total; ++it) {
         const int lt = it / ng;
         tile_of(lt);
-        if (it - lt * ng == 0 && pc.b != cur_b) {
+        if (!waited && (pc.b != b0 || it >= nring)) {
+          pdl_wait();
+          waited = true;
+          ok = stage_q(0, b0);
+          if (!ok) break;
+        }
+        if (is_k && waited && it - lt * ng == 0 && pc.b != cur_b) {
           cur_b = pc.b;
           ok = stage_q(++seg, cur_b);
           if (!ok) break;
         }
         ok = issue(it);
+      }
+      if (ok && !waited) {  // every tile fitted in the first ring's worth
+        pdl_wait();
+        ok = stage_q(0, b0);
       }
     } else {
       pdl_wait();
