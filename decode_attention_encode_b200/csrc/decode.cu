@@ -983,16 +983,20 @@ lla_status launch_combine(const float* part, int pstride, const float* c0, const
   return check_cuda(cudaLaunchKernelEx(&cfg, fn, a), "launch k_combine");
 }
 
-// Per-head decode takes the tensor-core absorb and combine for bf16
-// latents, large batches and wide ranks only. Both forms are bound by memory
-// round trips at these sizes, and the FFMA work the tensor cores remove
-// grows with B * r. Measured on B200 (whole decode call): B = 64, r = 128
-// and B = 768, r = 24 ran as fast or faster on the CUDA-core forms (327 vs
-// 327 us, 746 vs 751 us), while the LLA-2D shape (B = 256, r = 256) gained
-// 15 us per call on the tensor-core forms.
+// Per-head decode takes the tensor-core combine for bf16 latents, large
+// batches and wide ranks only, and the tensor-core absorb (its second form,
+// staged by lane and warp numbers) for bf16 latents and large batches at any
+// rank. Both forms are bound by memory round trips and instruction issue at
+// these sizes. Measured on B200 (whole decode steps, same box): the first
+// tensor-core forms lost to the CUDA-core ones at B = 64, r = 128 and at
+// B = 768, r = 24; the second absorb wins at B = 768, r = 24 (70.43 ->
+// 70.17 ms per step, three runs each), and the LLA-2D shape (B = 256,
+// r = 256) gains on both.
 bool small_gemm_tc(int esz, int B, int r_k, int r_v) {
   return esz == 2 && B >= 256 && std::max(r_k, r_v) >= 192;
 }
+
+bool absorb_tc(int esz, int B) { return esz == 2 && B >= 256; }
 
 lla_status plan_decode(int B, int H, int N, int r_k, int r_v, int esz, DecodePlan* p) {
   DecodePlan d{};
@@ -1105,7 +1109,7 @@ lla_status run_decode(const float* q, const void* zk, const void* zv, int esz, i
 
   // 1. absorb
   st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, q_rope, d_r,
-                     small_gemm_tc(esz, B, r_k, r_v), span_of(ws, ws_bytes));
+                     absorb_tc(esz, B), span_of(ws, ws_bytes));
   if (st != LLA_OK) return st;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -143,15 +143,17 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
 // zero), r_k + d_r a multiple of 64, at qsw + b * ((r_k + d_r) / 64) * hp *
 // 128. With q_rope non-null the last d_r columns of q' are the rotary query
 // [B*H][d_r] times scale * log2(e) (not absorbed). With tc the contraction
-// runs on the tensor cores (split bf16 operands, fp32 accumulation; d_h a
-// multiple of 16 and q 16-byte aligned, else the CUDA-core form runs);
-// callers pass it for bf16 latents. launch_combine's tc is the same choice.
+// runs on the tensor cores (split bf16 operands, fp32 accumulation; d_h of
+// 64 or 128, r_k a multiple of 8, q and W^K 16-byte aligned, else the
+// CUDA-core form runs); callers pass it for bf16 latents (absorb_tc).
+// launch_combine's tc is chosen by small_gemm_tc.
 lla_status launch_absorb(const float* q, const float* dk, const float* mu_k, int B, int H,
                          int d_h, int r_k, float scale, float* qp, float* c0, cudaStream_t stream,
                          unsigned char* qsw = nullptr, int hp = 0, const float* q_rope = nullptr,
                          int d_r = 0, bool tc = false, Span ws = Span{});
-// whether per-head decode runs launch_absorb / launch_combine with tc
+// whether per-head decode runs launch_combine / launch_absorb with tc
 bool small_gemm_tc(int esz, int B, int r_k, int r_v);
+bool absorb_tc(int esz, int B);
 lla_status launch_combine(const float* part, int pstride, const float* c0, const float* dv,
                           const float* mu_v, int B, int H, int d_h, int r_v, long long N,
                           long long P, int shared, float* out, float* lse, cudaStream_t stream,

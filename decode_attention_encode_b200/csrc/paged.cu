@@ -289,7 +289,7 @@ lla_status run_decode_paged(const float* q, const void* zk, const void* zv, int 
   }
   // 2. absorb (plain launch)
   st = launch_absorb(q, dk, mu_k, B, H, d_h, r_k, scale, qp, c0, stream, nullptr, 0, nullptr, 0,
-                     small_gemm_tc(esz, B, r_k, r_v), span_of(ws, ws_bytes));
+                     absorb_tc(esz, B), span_of(ws, ws_bytes));
   if (st != LLA_OK) return st;
   // 3. stream
   {
