@@ -17,6 +17,14 @@
  *    allocates nothing and keeps no per-call state.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL is the legacy default stream). The library never synchronises.
+ *  - The decode, merge and encode calls may be captured into a CUDA graph
+ *    on a capturing stream once the library has run on that device (its
+ *    first call there allocates the device status word); a replay runs the
+ *    same kernels on the same pointers.
+ *  - Within a decode call the streaming and merge kernels are launched
+ *    programmatically (they may start before the kernel ahead of them ends
+ *    and wait for it before reading its results); every call's first
+ *    kernel is ordered after all earlier work on the stream.
  *  - Arrays are dense, row-major, in the layouts stated per call.
  *  - A call returns LLA_OK once its kernels are queued; an argument problem
  *    found on the host returns an error before anything is launched; a launch
