@@ -751,10 +751,24 @@ lla_status plan_2d(int B, int H, int N, int r_k, int r_v, D2Plan* p) {
   const size_t fixed = 2 * (size_t)d.qbuf_bytes + 2 * (size_t)d.pbuf_bytes + sizeof(Tail2) + 1024;
   // Split the stages between the rings: each ring needs at least one
   // tile's groups (its slots are reused only by later tiles) and gets at
-  // most kMaxStages; K gets the odd one out.
+  // most kMaxStages. A split that uses every stage and gives each ring a
+  // whole number of tiles is taken when there is one (the most even such
+  // split, then the deeper V ring): at r_k = r_v = 256 (two groups per
+  // tile and ring, six stages) 2 K + 4 V and 4 K + 2 V stages both ran the
+  // decode in 312 us against 330 us for 3 + 3. Otherwise V gets half and K
+  // the odd one out.
   const int nst = (int)std::min<size_t>(2 * kMaxStages,
                                         ((size_t)di.smem_optin - fixed) / kStageBytes);
   d.nvs = std::min(kMaxStages, std::max(d.nvg, nst / 2));
+  int best = -1;
+  for (int v = d.nvg; v <= kMaxStages && v < nst; ++v) {
+    const int k = nst - v;
+    if (k > kMaxStages || k < d.nkg || v % d.nvg || k % d.nkg) continue;
+    if (best < 0 || std::abs(k - v) < std::abs((nst - best) - best) ||
+        (std::abs(k - v) == std::abs((nst - best) - best) && v > best))
+      best = v;
+  }
+  if (best > 0) d.nvs = best;
   d.nks = std::min(kMaxStages, nst - d.nvs);
   if (d.nks < d.nkg || d.nvs < d.nvg)
     return fail(LLA_ERR_UNSUPPORTED, "LLA-2D stage rings do not fit in shared memory");
